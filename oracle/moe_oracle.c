@@ -1,0 +1,545 @@
+/*
+ * moe_oracle.c -- plain, slow, obviously-correct CPU oracle for one
+ * Occult-style mixture-of-experts layer.  TEST INFRASTRUCTURE ONLY: the
+ * product library never links, loads or calls this file; only the tests,
+ * the smoke check and the benchmark's CPU-baseline leg do.
+ *
+ * Sources (cited by page title and section/figure):
+ *   [Occult]   "Occult: Optimizing Collaborative Communication across Experts
+ *               for Accelerated Parallel MoE Training and Inference" -- TL;DR,
+ *               Abstract, Figure 2 (three all-to-all strategies), Figure 4
+ *               (ORI/SFD/EPD token states guided by BRIMs), Figure 5 (the two
+ *               BRIMs and their dimensions).
+ *   [Coupling] "Expert Coupling in MoE Pretraining: Reducing All-to-All
+ *               Overhead with Correlated Placement and Token Shuffling" --
+ *               Abstract (top-k routing, once-per-GPU dispatch, correlated
+ *               placement from co-selected expert pairs).
+ *
+ * Arithmetic: every floating-point quantity is computed in double precision
+ * (the pages fix no precision).  Inputs that arrive as float32 or bfloat16
+ * are widened exactly to double before use.  Loops follow the definitions
+ * one term at a time: no blocking, fusion or reordering.
+ *
+ * Readings taken where the pages are silent (each one is listed, with its
+ * reason, in the design notes of the repository):
+ *   R1  BRIM entries are row positions (-1 = not sent); one entry drives both
+ *       the gather into SFD and the scatter back out of it ("bidirectional").
+ *   R2  Rows inside an SFD segment and inside an EPD group are in ascending
+ *       ORI-token order (stable compaction).
+ *   R3  Top-k compares raw logits; equal logits go to the lower expert id;
+ *       output order is descending score.
+ *   R4  Gate weights: softmax over all E logits then gather (renorm = 0), or
+ *       softmax over the k selected logits (renorm = 1).
+ *   R5  The gate weight is applied on the expert side, before the per-rank
+ *       pre-reduce (intra-collaboration), so one return row per (token,rank)
+ *       carries sum_j w_j * FFN_j(x).
+ *   R6  C_T counts every SFD row, including rows whose destination rank is
+ *       the token's own source rank; "remote" rows use the contiguous token
+ *       sharding src(t) = floor(t * R / T).
+ *   R7  Shared experts are not dispatched; they see ORI rows with weight 1
+ *       and are added after the routed combine.
+ *   R8  Placement slot q = slot_of[e]; rank(e) = q / L, loc(e) = q % L;
+ *       EPD groups are laid out in slot order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_DT_F32 0
+#define ORACLE_DT_BF16 1
+#define ORACLE_DT_F64 2
+
+/* Exact widening of one stored element to double.  bfloat16 is the upper
+ * half of an IEEE binary32, so widening is a 16-bit left shift of the bits. */
+static double widen(const void* base, size_t i, int dt) {
+  if (dt == ORACLE_DT_F64) return ((const double*)base)[i];
+  if (dt == ORACLE_DT_F32) return (double)((const float*)base)[i];
+  uint32_t bits = ((uint32_t)((const uint16_t*)base)[i]) << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+static size_t esize(int dt) {
+  return dt == ORACLE_DT_BF16 ? 2 : dt == ORACLE_DT_F32 ? 4 : 8;
+}
+
+int oracle_abi_version(void) { return 1; }
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+/* ------------------------------------------------------------------------
+ * Routing: each token picks k of E experts [Coupling, Abstract: "each token
+ * is routed to k of these experts"]; top-2/4/6/8 appear in [Occult, Fig. 3].
+ * Selection by reading R3, weights by reading R4.
+ *   logits  float32 [T,E]
+ *   idx     int32   [T,k]  (descending score)
+ *   w       double  [T,k]
+ * ---------------------------------------------------------------------- */
+int oracle_route(const float* logits, int T, int E, int k, int renorm,
+                 int32_t* idx, double* w) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + (size_t)t * E;
+    /* k rounds of "best remaining expert": larger logit wins, and on an
+     * equal logit the lower id wins. */
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        int taken = 0;
+        for (int i = 0; i < j; ++i)
+          if (idx[(size_t)t * k + i] == e) taken = 1;
+        if (taken) continue;
+        if (best < 0 || l[e] > l[best]) best = e; /* ties keep the lower id */
+      }
+      idx[(size_t)t * k + j] = best;
+    }
+    /* softmax, stabilised by the row maximum (a no-op in exact arithmetic) */
+    double m = (double)l[0];
+    for (int e = 1; e < E; ++e)
+      if ((double)l[e] > m) m = (double)l[e];
+    double denom = 0.0;
+    if (renorm) {
+      for (int j = 0; j < k; ++j) denom += exp((double)l[idx[(size_t)t * k + j]] - m);
+    } else {
+      for (int e = 0; e < E; ++e) denom += exp((double)l[e] - m);
+    }
+    for (int j = 0; j < k; ++j)
+      w[(size_t)t * k + j] = exp((double)l[idx[(size_t)t * k + j]] - m) / denom;
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * BRIM construction [Occult, Fig. 5; Fig. 4; TL;DR "all-to-all budget C_T"].
+ *   BRIM_0 : int32 [R, T]      rank x ORI token  -> SFD row or -1
+ *   BRIM_1 : int32 [L, cap]    local expert x SFD row -> EPD row or -1
+ *            (cap = T * min(k, R) is the row stride; columns >= C_T unused)
+ *   sfd_token [cap]  : SFD row -> ORI token (inverse of BRIM_0)
+ *   sfd_off  [R+1]   : start of each rank's SFD segment; sfd_off[R] = C_T
+ *   epd_off  [E+1]   : start of each slot's EPD group (slot order, R8)
+ *   epd_sfd  [T*k]   : EPD row -> SFD row (inverse of BRIM_1)
+ *   epd_gate [T*k]   : EPD row -> gate weight of that (token, expert) pair
+ * "Each token is sent once per destination device" [Coupling, Abstract;
+ * Occult, Fig. 2 third strategy].  Ordering by reading R2.
+ * ---------------------------------------------------------------------- */
+int oracle_brim(const int32_t* idx, const double* w, int T, int k,
+                const int32_t* slot_of, int E, int R,
+                int32_t* brim0, int32_t* sfd_token, int32_t* sfd_off,
+                int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                double* epd_gate, int32_t* c_t) {
+  if (R < 1 || E % R != 0 || k < 1 || k > E || T < 0) return -1;
+  const int L = E / R;
+  const int kr = k < R ? k : R;
+  const size_t cap = (size_t)T * kr;
+
+  /* hit(t, r): does token t select at least one expert held by rank r? */
+  char* hit = (char*)calloc((size_t)T * R + 1, 1);
+  if (!hit) return -2;
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) { free(hit); return -3; }
+      hit[(size_t)t * R + slot_of[e] / L] = 1;
+    }
+
+  /* n_r = number of tokens sent to rank r; sfd_off = exclusive prefix. */
+  sfd_off[0] = 0;
+  for (int r = 0; r < R; ++r) {
+    int n = 0;
+    for (int t = 0; t < T; ++t) n += hit[(size_t)t * R + r];
+    sfd_off[r + 1] = sfd_off[r] + n;
+  }
+  *c_t = sfd_off[R];
+
+  /* BRIM_0[r][t] = sfd_off[r] + #{t' < t : hit(t', r)}, else -1. */
+  for (int r = 0; r < R; ++r) {
+    int seen = 0;
+    for (int t = 0; t < T; ++t) {
+      if (hit[(size_t)t * R + r]) {
+        int s = sfd_off[r] + seen;
+        brim0[(size_t)r * T + t] = s;
+        sfd_token[s] = t;
+        ++seen;
+      } else {
+        brim0[(size_t)r * T + t] = -1;
+      }
+    }
+  }
+
+  /* c_q = number of tokens that selected the expert placed at slot q. */
+  int32_t* expert_at_slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+  if (!expert_at_slot) { free(hit); return -2; }
+  for (int e = 0; e < E; ++e) expert_at_slot[slot_of[e]] = e;
+  epd_off[0] = 0;
+  for (int q = 0; q < E; ++q) {
+    int c = 0, e = expert_at_slot[q];
+    for (int t = 0; t < T; ++t)
+      for (int j = 0; j < k; ++j)
+        if (idx[(size_t)t * k + j] == e) ++c;
+    epd_off[q + 1] = epd_off[q] + c;
+  }
+
+  /* every BRIM_1 entry starts as "no expert" */
+  for (size_t i = 0; i < (size_t)L * cap; ++i) brim1[i] = -1;
+
+  /* p = epd_off[slot(e)] + #{t' < t : e in idx[t']};
+   * BRIM_1[loc(e)][BRIM_0[rank(e)][t]] = p. */
+  int32_t* seen_e = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+  if (!seen_e) { free(hit); free(expert_at_slot); return -2; }
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < k; ++j) {
+      int e = idx[(size_t)t * k + j];
+      int q = slot_of[e];
+      int r = q / L, l = q % L;
+      int p = epd_off[q] + seen_e[e];
+      seen_e[e] += 1;
+      int s = brim0[(size_t)r * T + t];
+      brim1[(size_t)l * cap + s] = p;
+      epd_sfd[p] = s;
+      epd_gate[p] = w[(size_t)t * k + j];
+    }
+  }
+  free(seen_e);
+  free(expert_at_slot);
+  free(hit);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Row gathers of the dispatch [Occult, Fig. 4: ORI -> SFD -> EPD].
+ * Rows are copied byte for byte (row_bytes each).
+ * ---------------------------------------------------------------------- */
+void oracle_gather_rows(const void* src, size_t row_bytes, const int32_t* index,
+                        int n_rows, void* dst) {
+  for (int i = 0; i < n_rows; ++i)
+    memcpy((char*)dst + (size_t)i * row_bytes,
+           (const char*)src + (size_t)index[i] * row_bytes, row_bytes);
+}
+
+/* ------------------------------------------------------------------------
+ * One SwiGLU expert applied to one row a[d] (double):
+ *   g_i = sum_c Wg[i][c] a_c,  u_i = sum_c Wu[i][c] a_c  (i < f)
+ *   h_i = silu(g_i) * u_i,     silu(z) = z / (1 + exp(-z))
+ *   o_c = sum_i Wd[c][i] h_i   (c < d)
+ * Wg, Wu are [f, d]; Wd is [d, f]; all in dtype wdt.  h is scratch [f].
+ * The expert's FFN is the "sparse matrix multiplication" stage of the
+ * pipeline [Occult, TL;DR]; SwiGLU is the configured expert kind.
+ * kind 1 = IDENTITY: o = a (a test expert with no weights).
+ * ---------------------------------------------------------------------- */
+static void expert_row(int kind, const double* a, const void* Wg, const void* Wu,
+                       const void* Wd, int wdt, int d, int f, double* h, double* o) {
+  if (kind == 1) {
+    for (int c = 0; c < d; ++c) o[c] = a[c];
+    return;
+  }
+  for (int i = 0; i < f; ++i) {
+    double g = 0.0, u = 0.0;
+    for (int c = 0; c < d; ++c) {
+      g += widen(Wg, (size_t)i * d + c, wdt) * a[c];
+      u += widen(Wu, (size_t)i * d + c, wdt) * a[c];
+    }
+    double silu = g / (1.0 + exp(-g));
+    h[i] = silu * u;
+  }
+  for (int c = 0; c < d; ++c) {
+    double acc = 0.0;
+    for (int i = 0; i < f; ++i) acc += widen(Wd, (size_t)c * f + i, wdt) * h[i];
+    o[c] = acc;
+  }
+}
+
+/* Public single-row expert, used by the oracle's own self-checks. */
+void oracle_expert_row(int kind, const double* a, const void* Wg, const void* Wu,
+                       const void* Wd, int wdt, int d, int f, double* o) {
+  double* h = (double*)malloc(sizeof(double) * (size_t)(f > 0 ? f : 1));
+  expert_row(kind, a, Wg, Wu, Wd, wdt, d, f, h, o);
+  free(h);
+}
+
+/* ------------------------------------------------------------------------
+ * Dense definition of the layer output, with no BRIM anywhere:
+ *   Y[t] = sum_j w[t][j] * FFN_{idx[t][j]}(X[t]) + sum_s FFN_shared_s(X[t])
+ * for the tokens listed in `tokens` (n_tok of them; NULL = all T).
+ *   X    [T, d] dtype xdt
+ *   Wg,Wu [E, f, d], Wd [E, d, f] dtype wdt (expert-id order)
+ *   Sg,Su [S, fs, d], Sd [S, d, fs] (S = 0 allowed)
+ *   Y    [n_tok, d] double
+ * ---------------------------------------------------------------------- */
+int oracle_dense_layer(const void* X, int xdt, int T, int d,
+                       const int32_t* idx, const double* w, int k,
+                       const void* Wg, const void* Wu, const void* Wd, int wdt,
+                       int E, int f, int kind,
+                       const void* Sg, const void* Su, const void* Sd, int S, int fs,
+                       const int32_t* tokens, int n_tok, double* Y) {
+  if (d < 1 || T < 0 || k < 1) return -1;
+  if (tokens == NULL) n_tok = T;
+  const size_t wg_stride = (size_t)f * d, wd_stride = (size_t)d * f;
+  const size_t sg_stride = (size_t)fs * d, sd_stride = (size_t)d * fs;
+  const size_t es = esize(wdt);
+  int bad = 0;
+#pragma omp parallel
+  {
+    int hmax = f > fs ? f : fs;
+    double* a = (double*)malloc(sizeof(double) * (size_t)d);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    double* h = (double*)malloc(sizeof(double) * (size_t)(hmax > 0 ? hmax : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int n = 0; n < n_tok; ++n) {
+      int t = tokens ? tokens[n] : n;
+      double* y = Y + (size_t)n * d;
+      if (t < 0 || t >= T) { bad = 1; continue; }
+      for (int c = 0; c < d; ++c) a[c] = widen(X, (size_t)t * d + c, xdt);
+      for (int c = 0; c < d; ++c) y[c] = 0.0;
+      for (int j = 0; j < k; ++j) {
+        int e = idx[(size_t)t * k + j];
+        if (e < 0 || e >= E) { bad = 1; continue; }
+        expert_row(kind, a, (const char*)Wg + e * wg_stride * es,
+                   (const char*)Wu + e * wg_stride * es,
+                   (const char*)Wd + e * wd_stride * es, wdt, d, f, h, o);
+        for (int c = 0; c < d; ++c) y[c] += w[(size_t)t * k + j] * o[c];
+      }
+      for (int s = 0; s < S; ++s) {
+        expert_row(0, a, (const char*)Sg + s * sg_stride * es, (const char*)Su + s * sg_stride * es,
+                   (const char*)Sd + s * sd_stride * es, wdt, d, fs, h, o);
+        for (int c = 0; c < d; ++c) y[c] += o[c];
+      }
+    }
+    free(a); free(o); free(h);
+  }
+  return bad ? -3 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * The layer the Occult way [Occult, Fig. 4 and Fig. 5; Abstract,
+ * intra-collaboration], one step after another on the BRIMs built by
+ * oracle_brim():
+ *   1. dispatch  X_sfd[s] = X[sfd_token[s]]            (ORI -> SFD)
+ *   2. re-index  X_epd[p] = X_sfd[epd_sfd[p]]          (SFD -> EPD)
+ *   3. experts   O_epd[p] = epd_gate[p] * FFN_{x(p)}(X_epd[p]), where x(p)
+ *                is the expert placed at the slot whose EPD group holds p
+ *   4. pre-reduce (intra-collaboration, one return row per SFD row)
+ *                Y_sfd[s] = sum over l ascending, BRIM_1[l][s] >= 0, of
+ *                           O_epd[BRIM_1[l][s]]
+ *   5. combine   Y[t] = sum over r ascending, BRIM_0[r][t] >= 0, of
+ *                       Y_sfd[BRIM_0[r][t]]
+ *   6. shared    Y[t] += sum over s ascending of FFN_shared_s(X[t])
+ * All in double.  Outputs Y_sfd [C_T, d], Y [T, d] (double).
+ * ---------------------------------------------------------------------- */
+int oracle_occult_layer(const void* X, int xdt, int T, int d,
+                        const int32_t* slot_of, int E, int R, int k,
+                        const int32_t* brim0, const int32_t* sfd_token,
+                        const int32_t* brim1, const int32_t* epd_off,
+                        const int32_t* epd_sfd, const double* epd_gate, int c_t,
+                        const void* Wg, const void* Wu, const void* Wd, int wdt,
+                        int f, int kind,
+                        const void* Sg, const void* Su, const void* Sd, int S, int fs,
+                        double* Y_sfd, double* Y) {
+  if (R < 1 || E % R != 0) return -1;
+  const int L = E / R;
+  const int kr = k < R ? k : R;
+  const size_t cap = (size_t)T * kr;
+  const size_t tk = (size_t)T * k;
+  const size_t es = esize(wdt);
+
+  double* X_sfd = (double*)malloc(sizeof(double) * ((size_t)c_t * d + 1));
+  double* X_epd = (double*)malloc(sizeof(double) * (tk * d + 1));
+  double* O_epd = (double*)malloc(sizeof(double) * (tk * d + 1));
+  int32_t* expert_at_slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+  if (!X_sfd || !X_epd || !O_epd || !expert_at_slot) {
+    free(X_sfd); free(X_epd); free(O_epd); free(expert_at_slot);
+    return -2;
+  }
+  for (int e = 0; e < E; ++e) expert_at_slot[slot_of[e]] = e;
+
+  /* 1. ORI -> SFD */
+  for (int s = 0; s < c_t; ++s)
+    for (int c = 0; c < d; ++c)
+      X_sfd[(size_t)s * d + c] = widen(X, (size_t)sfd_token[s] * d + c, xdt);
+  /* 2. SFD -> EPD */
+  for (size_t p = 0; p < tk; ++p)
+    for (int c = 0; c < d; ++c)
+      X_epd[p * d + c] = X_sfd[(size_t)epd_sfd[p] * d + c];
+  /* 3. expert compute, one EPD group (slot) after another */
+#pragma omp parallel
+  {
+    double* h = (double*)malloc(sizeof(double) * (size_t)(f > 0 ? f : 1));
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 16)
+    for (long long pp = 0; pp < (long long)tk; ++pp) {
+      size_t p = (size_t)pp;
+      int q = 0;
+      while (!(epd_off[q] <= (int)p && (int)p < epd_off[q + 1])) ++q;
+      int e = expert_at_slot[q];
+      expert_row(kind, X_epd + p * d, (const char*)Wg + (size_t)e * f * d * es,
+                 (const char*)Wu + (size_t)e * f * d * es,
+                 (const char*)Wd + (size_t)e * d * f * es, wdt, d, f, h, o);
+      for (int c = 0; c < d; ++c) O_epd[p * d + c] = epd_gate[p] * o[c];
+    }
+    free(h); free(o);
+  }
+  /* 4. intra-collaboration pre-reduce: one return row per SFD row */
+  for (int s = 0; s < c_t; ++s) {
+    for (int c = 0; c < d; ++c) Y_sfd[(size_t)s * d + c] = 0.0;
+    for (int l = 0; l < L; ++l) {
+      int p = brim1[(size_t)l * cap + s];
+      if (p < 0) continue;
+      for (int c = 0; c < d; ++c) Y_sfd[(size_t)s * d + c] += O_epd[(size_t)p * d + c];
+    }
+  }
+  /* 5. combine back into ORI order */
+  for (int t = 0; t < T; ++t) {
+    for (int c = 0; c < d; ++c) Y[(size_t)t * d + c] = 0.0;
+    for (int r = 0; r < R; ++r) {
+      int s = brim0[(size_t)r * T + t];
+      if (s < 0) continue;
+      for (int c = 0; c < d; ++c) Y[(size_t)t * d + c] += Y_sfd[(size_t)s * d + c];
+    }
+  }
+  /* 6. shared experts on ORI rows, weight 1 */
+  if (S > 0) {
+#pragma omp parallel
+    {
+      double* a = (double*)malloc(sizeof(double) * (size_t)d);
+      double* h = (double*)malloc(sizeof(double) * (size_t)(fs > 0 ? fs : 1));
+      double* o = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+      for (int t = 0; t < T; ++t) {
+        for (int c = 0; c < d; ++c) a[c] = widen(X, (size_t)t * d + c, xdt);
+        for (int s = 0; s < S; ++s) {
+          expert_row(0, a, (const char*)Sg + (size_t)s * fs * d * es,
+                     (const char*)Su + (size_t)s * fs * d * es,
+                     (const char*)Sd + (size_t)s * d * fs * es, wdt, d, fs, h, o);
+          for (int c = 0; c < d; ++c) Y[(size_t)t * d + c] += o[c];
+        }
+      }
+      free(a); free(h); free(o);
+    }
+  }
+  free(X_sfd); free(X_epd); free(O_epd); free(expert_at_slot);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Dispatched-row counter for a placement [Coupling, Abstract: a dispatcher
+ * that sends each token to each GPU once; Occult, Fig. 2].
+ *   per_rank[r] = #{t : token t selects an expert held by rank r}
+ *   total       = sum_r per_rank[r]                    (= C_T)
+ *   remote      = #{(t, r) sent : r != floor(t * R / T)}   (reading R6)
+ * ---------------------------------------------------------------------- */
+int oracle_count_dispatched(const int32_t* idx, int T, int k, const int32_t* slot_of,
+                            int E, int R, int32_t* per_rank, int64_t* total,
+                            int64_t* remote) {
+  if (R < 1 || E % R != 0) return -1;
+  const int L = E / R;
+  for (int r = 0; r < R; ++r) per_rank[r] = 0;
+  *total = 0;
+  *remote = 0;
+  for (int t = 0; t < T; ++t) {
+    int src = (int)(((int64_t)t * R) / T);
+    for (int r = 0; r < R; ++r) {
+      int sent = 0;
+      for (int j = 0; j < k; ++j)
+        if (slot_of[idx[(size_t)t * k + j]] / L == r) sent = 1;
+      if (!sent) continue;
+      per_rank[r] += 1;
+      *total += 1;
+      if (r != src) *remote += 1;
+    }
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Expert co-activation pair histogram [Coupling, Abstract: expert pairs
+ * selected together by tokens; Occult, Abstract: "collaborated" experts].
+ *   H[a][b] (a != b) = #{t : a and b both in idx[t]}  (symmetric)
+ *   H[a][a]          = #{t : a in idx[t]}
+ * accumulate = 0 clears H first.
+ * ---------------------------------------------------------------------- */
+void oracle_coact_histogram(const int32_t* idx, int T, int k, int E, uint32_t* H,
+                            int accumulate) {
+  if (!accumulate)
+    for (size_t i = 0; i < (size_t)E * E; ++i) H[i] = 0;
+  for (int t = 0; t < T; ++t)
+    for (int a = 0; a < E; ++a)
+      for (int b = 0; b < E; ++b) {
+        int has_a = 0, has_b = 0;
+        for (int j = 0; j < k; ++j) {
+          if (idx[(size_t)t * k + j] == a) has_a = 1;
+          if (idx[(size_t)t * k + j] == b) has_b = 1;
+        }
+        if (has_a && has_b) H[(size_t)a * E + b] += 1;
+      }
+}
+
+/* ------------------------------------------------------------------------
+ * Correlated placement, greedy [Coupling, Abstract: experts often selected
+ * together go on the same GPU; Occult, TL;DR: expert-placement rescheduling].
+ * The pages name no algorithm; this greedy is the plainest one:
+ *   repeat for rank r = 0 .. R-1:
+ *     seed = unplaced expert with the largest H[a][a] (ties -> lower id)
+ *     while the rank holds fewer than L experts:
+ *       add the unplaced b maximising sum_{a in rank} H[a][b]
+ *       (ties -> larger H[b][b], then lower id)
+ *   slots inside a rank follow insertion order.
+ * H is uint32 [E, E]; slot_of receives the placement.
+ * ---------------------------------------------------------------------- */
+int oracle_place_greedy(const uint32_t* H, int E, int R, int32_t* slot_of) {
+  if (R < 1 || E % R != 0) return -1;
+  const int L = E / R;
+  char* placed = (char*)calloc((size_t)E, 1);
+  int32_t* members = (int32_t*)malloc(sizeof(int32_t) * (size_t)L);
+  if (!placed || !members) { free(placed); free(members); return -2; }
+  for (int r = 0; r < R; ++r) {
+    int n = 0;
+    int seed = -1;
+    for (int a = 0; a < E; ++a) {
+      if (placed[a]) continue;
+      if (seed < 0 || H[(size_t)a * E + a] > H[(size_t)seed * E + seed]) seed = a;
+    }
+    members[n++] = seed;
+    placed[seed] = 1;
+    slot_of[seed] = r * L + 0;
+    while (n < L) {
+      int best = -1;
+      uint64_t best_score = 0;
+      for (int b = 0; b < E; ++b) {
+        if (placed[b]) continue;
+        uint64_t score = 0;
+        for (int i = 0; i < n; ++i) score += H[(size_t)members[i] * E + b];
+        int better = 0;
+        if (best < 0) better = 1;
+        else if (score > best_score) better = 1;
+        else if (score == best_score &&
+                 H[(size_t)b * E + b] > H[(size_t)best * E + best]) better = 1;
+        if (better) { best = b; best_score = score; }
+      }
+      slot_of[best] = r * L + n;
+      members[n++] = best;
+      placed[best] = 1;
+    }
+  }
+  free(placed);
+  free(members);
+  return 0;
+}
