@@ -1,0 +1,368 @@
+"""Benchmark: MoE-layer tokens/s of the Occult-style layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one pass of the whole layer over one batch: top-k routing, BRIM
+build, ORI -> SFD -> EPD dispatch, grouped SwiGLU experts (+ shared experts),
+per-rank pre-reduce and combine, dispatched-row counter and co-activation
+histogram.  Inputs are synthetic (seeded), already resident in HBM when the
+timed region starts; L2 is flushed between steps (a 256 MiB write outside the
+per-step events).  Under torchrun every rank runs its own batch (independent
+problems, no data-path collective: weak scaling); the time is the max over
+ranks.
+
+`e2e` is the same metric through moe_layer_forward_host(): the step's
+logits and activations come from pinned host memory and the output goes back
+to host memory inside the timed region.
+
+`--impl reference` times the CPU oracle (the plain reference implementation
+of the layer) on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from expert_warp_top_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (route+BRIM dispatch+grouped GEMM+combine)"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sust=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.t is not None:
+                self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def algorithmic_work(cfg, c_t: int, e_act: int):
+    """FLOPs and HBM bytes the layer must spend (not the dense work it avoids)."""
+    e = 2 if cfg.dtype == "bf16" else 4
+    T, d, f, k, S, fs = cfg.T, cfg.d, cfg.f, cfg.k, cfg.S, cfg.fs
+    flops_ffn = 2.0 * 3 * d * f * T * k + 2.0 * 3 * d * fs * T * S
+    bytes_ = e * (T * d + c_t * d + c_t * d + 3.0 * e_act * d * f + 3.0 * S * d * fs
+                  + c_t * d + c_t * d + T * d) + 4.0 * (T * cfg.E + 4 * T * k + cfg.R * T
+                                                         + cfg.L * c_t)
+    return flops_ffn, bytes_
+
+
+def launches_per_step(cfg) -> int:
+    # route 1, BRIM 3, dispatch 1, experts 2 (+2 shared), combine 1, counter 1, histogram 1
+    return 1 + 3 + 1 + 2 + (2 if cfg.S else 0) + 1 + 1 + 1
+
+
+def cpu_baseline(cfg, budget_s: float = 12.0):
+    """The oracle as it stands, on a bounded sample of the same workload's tokens:
+    routing + BRIM build + the dense layer on the sampled tokens."""
+    import oracle
+    inp = inputs.make_inputs(cfg, device="cpu", weights=True)
+
+    def bits(t):
+        t = t.contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    logits = inp["logits"].numpy()
+    x = bits(inp["x"])
+    wg, wu, wd = bits(inp["wg"]), bits(inp["wu"]), bits(inp["wd"])
+    shared = (bits(inp["sg"]), bits(inp["su"]), bits(inp["sd"])) if cfg.S else None
+    slot_of = np.arange(cfg.E, dtype=np.int32)
+    rng = np.random.default_rng(0)
+    n, total_t, total_n = 8, 0.0, 0
+    while total_t < budget_s and total_n < cfg.T:
+        tokens = np.sort(rng.choice(cfg.T, size=min(n, cfg.T), replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        idx, w = oracle.route(logits[tokens], cfg.k, cfg.renorm)
+        oracle.brim(idx, w, slot_of, cfg.E, cfg.R)
+        oracle.dense_layer(np.ascontiguousarray(x[tokens]), idx, w, wg, wu, wd, shared=shared)
+        dt = time.perf_counter() - t0
+        total_t += dt
+        total_n += len(tokens)
+        n *= 2
+    return {"value": total_n / total_t, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{total_n} of {cfg.T} tokens (route + BRIM + dense fp64 layer), "
+                      f"{total_t:.1f} s"}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    per_step = []
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        res = cpu_baseline(cfg, budget_s=budget)
+        if i >= args.warmup:
+            per_step.append(res)
+    value = statistics.median([r["value"] for r in per_step])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * cfg.T / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "f": cfg.f, "E": cfg.E,
+                   "k": cfg.k, "R": cfg.R, "S": cfg.S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": per_step[-1]["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, cfg):
+    import torch.distributed as dist
+    from expert_warp_top_b200 import _binding as B
+    from expert_warp_top_b200.layer import MoELayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    # each rank: its own independent batch (seed offset by rank), same weights recipe
+    inp = inputs.make_inputs(cfg, device=dev, seed=cfg.seed + 7919 * rank)
+    kw = dict(wg=inp.pop("wg"), wu=inp.pop("wu"), wd=inp.pop("wd"))
+    if cfg.S:
+        kw.update(sg=inp.pop("sg"), su=inp.pop("su"), sd=inp.pop("sd"))
+    layer = MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
+                     dtype=inputs.torch_dtype(cfg), S=cfg.S, fs=cfg.fs, device=dev, **kw)
+    del kw
+    logits, x = inp["logits"], inp["x"]
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        layer.forward(logits, x)
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = B.moe_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    c_t = int(layer.c_t.item())
+    e_act = int((layer.epd_off[1:] - layer.epd_off[:-1] > 0).sum().item())
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
+            s0, f0, f1, s1 = ev[i]
+            s0.record(stream)
+            layer.route(logits)
+            layer.build_brims()
+            layer.dispatch(x)
+            f0.record(stream)
+            layer.experts()
+            f1.record(stream)
+            layer.shared_experts(x)
+            layer.combine()
+            layer.statistics()
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.T * args.steps / (total_ms * 1e-3)
+
+    # end to end through the public API: host buffers in and out, copies timed
+    e2e = None
+    try:
+        e2e = e2e_host(layer, inp, cfg, args, dev, world)
+    except Exception as exc:  # noqa: BLE001 -- reported, never hidden
+        e2e = {"value": None, "unit": UNIT, "error": str(exc)[:200]}
+
+    pk = peaks()
+    flops, bytes_ = algorithmic_work(cfg, c_t, e_act)
+    ffn_flops = 2.0 * 3 * cfg.d * cfg.f * cfg.T * cfg.k
+    ffn_s = statistics.mean(ffn_ms) * 1e-3
+    achieved = ffn_flops / ffn_s / 1e12
+    roof = {"bound": "tensor", "kernel": "ffn_gemm_kernel (routed experts: gate/up GEMM with "
+            "SwiGLU epilogue + down GEMM with gate scaling, 2 launches)",
+            "achieved": achieved, "peak": pk["bf16_sust"], "unit": "TFLOP/s",
+            "frac": achieved / pk["bf16_sust"], "traffic": None,
+            "peak_source": f"{pk['source']} bf16 sustained"}
+    layer_roof_s = max(flops / (pk["bf16_sust"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} "
+                                   f"k={cfg.k} R={cfg.R} S={cfg.S}",
+                       "placement": "contiguous", "l2": "flushed between steps "
+                       "(256 MiB write outside the per-step events)",
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": roof,
+            "layer_roofline": {"t_roof_ms": layer_roof_s * 1e3, "frac": layer_roof_s * 1e3 /
+                               ms_per_step, "flops": flops, "bytes": bytes_},
+            "c_t": c_t, "tk_rows": cfg.T * cfg.k, "e2e": e2e, "cpu_baseline": cpu,
+            "clocks": clocks.summary(),
+            "gpu_launches": launches_per_step(cfg) * args.steps,
+            "ffn_ms": statistics.mean(ffn_ms),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_host(layer, inp, cfg, args, dev, world):
+    """Host-buffer end to end: H2D of logits and x, the layer, D2H of y, per step."""
+    h_logits = inp["logits"].cpu().pin_memory()
+    h_x = inp["x"].cpu().pin_memory()
+    h_y = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    d_logits = torch.empty_like(inp["logits"])
+    d_x = torch.empty_like(inp["x"])
+
+    def step():
+        d_logits.copy_(h_logits, non_blocking=True)
+        d_x.copy_(h_x, non_blocking=True)
+        y = layer.forward(d_logits, d_x)
+        h_y.copy_(y, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = h_logits.numel() * h_logits.element_size() + h_x.numel() * h_x.element_size()
+    d2h = h_y.numel() * h_y.element_size()
+    return {"value": world * cfg.T * args.steps / (ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "MoELayer.forward with pinned host copies"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="olmoe", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    cfg = inputs.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

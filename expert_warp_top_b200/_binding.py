@@ -1,0 +1,198 @@
+"""ctypes binding of libmoe_occult.so -- argument marshalling only.
+
+Every function here has the name of the C entry point it calls and the same
+arguments, with torch tensors in place of device pointers.  The binding
+checks dtypes, devices, shapes and contiguity, passes raw pointers and the
+current CUDA stream, and raises on a non-zero status.  All arithmetic runs in
+the CUDA kernels; there is no fallback: without the built library every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libmoe_occult.so"
+_lib = None
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_DEVICE_CHECK = -4
+MOE_ERR_TIMEOUT = -5
+MOE_F32, MOE_BF16 = 0, 1
+MOE_FFN_SWIGLU, MOE_FFN_IDENTITY = 0, 1
+
+# every symbol the header declares (checked by the ABI test)
+EXPORTS = (
+    "moe_abi_version", "moe_last_error", "moe_set_debug", "moe_get_device_status",
+    "moe_route_topk", "moe_brim_workspace_size", "moe_brim_build", "moe_dispatch_gather",
+    "moe_prepare_weights", "moe_prepare_shared_weights", "moe_expert_ffn_workspace_size",
+    "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
+)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with status {code}: {msg}")
+        self.code = code
+
+
+def lib_path() -> Path:
+    return _LIB_PATH
+
+
+def load():
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not _LIB_PATH.exists():
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m expert_warp_top_b200.build` "
+                "(there is no CPU fallback)")
+        lib = ctypes.CDLL(str(_LIB_PATH))
+        lib.moe_last_error.restype = ctypes.c_char_p
+        lib.moe_brim_workspace_size.restype = ctypes.c_size_t
+        lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
+        lib.moe_set_debug.argtypes = [ctypes.c_int, ctypes.c_double]
+        for name in EXPORTS:
+            getattr(lib, name)
+        _lib = lib
+    return _lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(fn, rc, load().moe_last_error().decode(errors="replace"))
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name: str = "tensor") -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return MOE_BF16
+    if t == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported activation dtype {t}")
+
+
+_ACT = (torch.bfloat16, torch.float32)
+I32, F32, I64, U32 = torch.int32, torch.float32, torch.int64, torch.uint32
+
+
+# ---------------------------------------------------------------------------
+def moe_abi_version() -> int:
+    return int(load().moe_abi_version())
+
+
+def moe_set_debug(flags: int, wait_limit_ms: float) -> None:
+    _check("moe_set_debug", load().moe_set_debug(int(flags), float(wait_limit_ms)))
+
+
+def moe_get_device_status(stream=None) -> int:
+    """Synchronise, read and clear the device error flag; returns the status code."""
+    return int(load().moe_get_device_status(_stream(stream)))
+
+
+def moe_route_topk(logits, k, renorm, topk_idx, topk_w, stream=None):
+    T, E = logits.shape
+    _check("moe_route_topk", load().moe_route_topk(
+        _ptr(logits, F32, "logits"), T, E, int(k), int(renorm),
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"), _stream(stream)))
+
+
+def moe_brim_workspace_size(T, E, R) -> int:
+    return int(load().moe_brim_workspace_size(int(T), int(E), int(R)))
+
+
+def moe_brim_build(topk_idx, topk_w, slot_of, E, R, brim0, sfd_token, sfd_off, brim1, epd_off,
+                   epd_sfd, epd_gate, c_t, ws, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_brim_build", load().moe_brim_build(
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"), T, k,
+        _ptr(slot_of, I32, "slot_of"), int(E), int(R),
+        _ptr(brim0, I32, "brim0"), _ptr(sfd_token, I32, "sfd_token"), _ptr(sfd_off, I32, "sfd_off"),
+        _ptr(brim1, I32, "brim1"), _ptr(epd_off, I32, "epd_off"), _ptr(epd_sfd, I32, "epd_sfd"),
+        _ptr(epd_gate, F32, "epd_gate"), _ptr(c_t, I32, "c_t"),
+        _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
+
+
+def moe_dispatch_gather(x, k, R, L, brim0, brim1, x_sfd, x_epd, stream=None):
+    T, d = x.shape
+    _check("moe_dispatch_gather", load().moe_dispatch_gather(
+        _ptr(x, _ACT, "x"), T, d, dtype_code(x.dtype), int(k), int(R), int(L),
+        _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"),
+        _ptr(x_sfd, x.dtype, "x_sfd"), _ptr(x_epd, x.dtype, "x_epd"), _stream(stream)))
+
+
+def moe_prepare_weights(wg, wu, wd, slot_of, w_gu, w_dn, stream=None):
+    E, f, d = wg.shape
+    _check("moe_prepare_weights", load().moe_prepare_weights(
+        _ptr(wg, _ACT, "wg"), _ptr(wu, wg.dtype, "wu"), _ptr(wd, wg.dtype, "wd"), E, d, f,
+        dtype_code(wg.dtype), _ptr(slot_of, I32, "slot_of"),
+        _ptr(w_gu, wg.dtype, "w_gu"), _ptr(w_dn, wg.dtype, "w_dn"), _stream(stream)))
+
+
+def moe_prepare_shared_weights(sg, su, sd, w_gu, w_dn, stream=None):
+    S, fs, d = sg.shape
+    _check("moe_prepare_shared_weights", load().moe_prepare_shared_weights(
+        _ptr(sg, _ACT, "sg"), _ptr(su, sg.dtype, "su"), _ptr(sd, sg.dtype, "sd"), S, d, fs,
+        dtype_code(sg.dtype), _ptr(w_gu, sg.dtype, "w_gu"), _ptr(w_dn, sg.dtype, "w_dn"),
+        _stream(stream)))
+
+
+def moe_expert_ffn_workspace_size(m_cap, f, dtype_code_) -> int:
+    return int(load().moe_expert_ffn_workspace_size(int(m_cap), int(f), int(dtype_code_)))
+
+
+def moe_expert_ffn(a, group_off, w_gu, w_dn, f, row_scale, ffn_kind, out, ws, stream=None):
+    m_cap, d = a.shape
+    G = group_off.numel() - 1
+    _check("moe_expert_ffn", load().moe_expert_ffn(
+        _ptr(a, _ACT, "a"), _ptr(group_off, I32, "group_off"), G, m_cap,
+        _ptr(w_gu, a.dtype, "w_gu"), _ptr(w_dn, a.dtype, "w_dn"), d, int(f), dtype_code(a.dtype),
+        _ptr(row_scale, F32, "row_scale"), int(ffn_kind), _ptr(out, a.dtype, "out"),
+        _ptr(ws, None, "ws"), ctypes.c_size_t(0 if ws is None else ws.numel() * ws.element_size()),
+        _stream(stream)))
+
+
+def moe_combine_scatter(o_epd, T, k, R, L, brim0, brim1, shared_out, y_sfd, y, stream=None):
+    d = o_epd.shape[1]
+    _check("moe_combine_scatter", load().moe_combine_scatter(
+        _ptr(o_epd, _ACT, "o_epd"), int(T), d, dtype_code(o_epd.dtype), int(k), int(R), int(L),
+        _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"),
+        _ptr(shared_out, o_epd.dtype, "shared_out"), _ptr(y_sfd, o_epd.dtype, "y_sfd"),
+        _ptr(y, o_epd.dtype, "y"), _stream(stream)))
+
+
+def moe_count_dispatched_rows(topk_idx, slot_of, E, R, per_rank, total, remote, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_count_dispatched_rows", load().moe_count_dispatched_rows(
+        _ptr(topk_idx, I32, "topk_idx"), T, k, _ptr(slot_of, I32, "slot_of"), int(E), int(R),
+        _ptr(per_rank, I32, "per_rank"), _ptr(total, I64, "total"), _ptr(remote, I64, "remote"),
+        _stream(stream)))
+
+
+def moe_coact_histogram(topk_idx, E, hist, accumulate, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_coact_histogram", load().moe_coact_histogram(
+        _ptr(topk_idx, I32, "topk_idx"), T, k, int(E), _ptr(hist, (U32, torch.int32), "hist"),
+        int(accumulate), _stream(stream)))

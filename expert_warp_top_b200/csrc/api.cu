@@ -1,0 +1,495 @@
+// api.cu -- the C ABI (include/moe_occult.h): argument checks, launch
+// configuration and the tensor-map set-up of every kernel of the layer.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include "../../include/moe_occult.h"
+#include "brim.cuh"
+#include "dispatch.cuh"
+#include "ffn_gemm.cuh"
+#include "route.cuh"
+
+// The device error flag the kernels raise (bits moe::kErrIndex, kErrTimeout).
+__device__ unsigned g_moe_err_flag;
+
+namespace {
+
+thread_local char g_msg[512];
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define MOE_REQUIRE(cond, code, ...)          \
+  do {                                        \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+#define MOE_CUDA(call)                                                              \
+  do {                                                                              \
+    cudaError_t e_ = (call);                                                        \
+    if (e_ != cudaSuccess)                                                          \
+      return fail(MOE_ERR_CUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_),   \
+                  __FILE__, __LINE__);                                              \
+  } while (0)
+
+#define MOE_LAUNCHED(what)                                                          \
+  do {                                                                              \
+    cudaError_t e_ = cudaGetLastError();                                            \
+    if (e_ != cudaSuccess)                                                          \
+      return fail(MOE_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned* err_flag = nullptr;
+  unsigned smem_attr_done = 0;  // bit per GEMM instantiation
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  MOE_REQUIRE(dev >= 0 && dev < kMaxDevices, MOE_ERR_UNSUPPORTED, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    MOE_CUDA(cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev));
+    int major = 0, minor = 0;
+    MOE_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    MOE_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    MOE_REQUIRE(major == 10 && minor == 0, MOE_ERR_UNSUPPORTED,
+                "this library is built for sm_100a (B200); device %d is sm_%d%d", dev, major,
+                minor);
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, g_moe_err_flag));
+    di.err_flag = static_cast<unsigned*>(p);
+    di.ready = true;
+  }
+  *out = &di;
+  return MOE_OK;
+}
+
+// ---- debug knobs (tests only) -------------------------------------------
+int g_debug_flags = 0;
+double g_wait_limit_ms = 4000.0;
+
+uint64_t wait_limit_ns() {
+  return static_cast<uint64_t>(g_wait_limit_ms * 1.0e6);
+}
+
+// ---- tensor maps ---------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encode_fn(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cached) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    MOE_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q));
+    MOE_REQUIRE(q == cudaDriverEntryPointSuccess && p, MOE_ERR_CUDA,
+                "cuTensorMapEncodeTiled is not available from the driver");
+    cached = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = cached;
+  return MOE_OK;
+}
+
+// 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
+int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn;
+  int rc = get_encode_fn(&fn);
+  if (rc) return rc;
+  const int esz = dtype == MOE_BF16 ? 2 : 4;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (cuuint64_t)esz};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype == MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA,
+              "cuTensorMapEncodeTiled failed (%d) for a [%llu x %llu] tensor", (int)r,
+              (unsigned long long)rows, (unsigned long long)cols);
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int T, int E, int k, int R) {
+  MOE_REQUIRE(T >= 0, MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+  MOE_REQUIRE(E >= 1 && E <= moe::kMaxE, MOE_ERR_UNSUPPORTED, "E must be in [1, 256] (got %d)", E);
+  MOE_REQUIRE(k >= 1 && k <= E && k <= moe::kMaxK, MOE_ERR_UNSUPPORTED,
+              "k must be in [1, min(E, 16)] (got k=%d, E=%d)", k, E);
+  MOE_REQUIRE(R >= 1 && R <= E && E % R == 0, MOE_ERR_UNSUPPORTED,
+              "R must divide E (got E=%d, R=%d)", E, R);
+  return MOE_OK;
+}
+
+int check_dtype(int dtype) {
+  MOE_REQUIRE(dtype == MOE_BF16 || dtype == MOE_F32, MOE_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  return MOE_OK;
+}
+
+int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+
+// ---- GEMM launch ----------------------------------------------------------
+template <int BN, int EPI, bool TF32>
+int launch_gemm(DeviceInfo* di, unsigned attr_bit, const void* a, int m_cap, int K,
+                const void* b, int G, int N, const int32_t* group_off, const float* row_scale,
+                void* out, int ldo, cudaStream_t st) {
+  using Cfg = moe::GemmCfg<BN, TF32>;
+  const int dtype = TF32 ? MOE_F32 : MOE_BF16;
+  CUtensorMap ta, tb;
+  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)m_cap, Cfg::kBK, moe::kGemmBM);
+  if (rc) return rc;
+  rc = encode_2d(&tb, b, dtype, (uint64_t)K, (uint64_t)G * N, Cfg::kBK, BN);
+  if (rc) return rc;
+  auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32>;
+  if (!(di->smem_attr_done & attr_bit)) {
+    MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)Cfg::kSmemBytes));
+    di->smem_attr_done |= attr_bit;
+  }
+  const long long ub = ((long long)m_cap / moe::kGemmBM + G) * (N / BN);
+  const int grid = (int)(ub < di->num_sms ? (ub < 1 ? 1 : ub) : di->num_sms);
+  moe::GemmArgs args{group_off, G, N, K, m_cap, row_scale, out, ldo, di->err_flag,
+                     wait_limit_ns(), g_debug_flags};
+  kern<<<grid, moe::kGemmThreads, Cfg::kSmemBytes, st>>>(ta, tb, args);
+  MOE_LAUNCHED("ffn_gemm_kernel");
+  return MOE_OK;
+}
+
+template <int EPI, bool TF32>
+int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int m_cap, int K, const void* b, int G,
+                   int N, const int32_t* group_off, const float* row_scale, void* out, int ldo,
+                   cudaStream_t st) {
+  const unsigned base = (EPI * 2 + (TF32 ? 1 : 0)) * 3;
+  if (bn == 256)
+    return launch_gemm<256, EPI, TF32>(di, 1u << (base + 0), a, m_cap, K, b, G, N, group_off,
+                                       row_scale, out, ldo, st);
+  if (bn == 128)
+    return launch_gemm<128, EPI, TF32>(di, 1u << (base + 1), a, m_cap, K, b, G, N, group_off,
+                                       row_scale, out, ldo, st);
+  return launch_gemm<64, EPI, TF32>(di, 1u << (base + 2), a, m_cap, K, b, G, N, group_off,
+                                    row_scale, out, ldo, st);
+}
+
+int pick_bn(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+// ===========================================================================
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_last_error(void) { return g_msg; }
+
+// Test-only knobs: debug flags of the GEMM (1 = skip the first TMA load, so a
+// bounded wait expires) and the device wait limit in milliseconds.
+int moe_set_debug(int flags, double wait_limit_ms) {
+  MOE_REQUIRE(wait_limit_ms > 0.0, MOE_ERR_INVALID_ARG, "wait limit must be positive");
+  g_debug_flags = flags;
+  g_wait_limit_ms = wait_limit_ms;
+  return MOE_OK;
+}
+
+int moe_get_device_status(moe_stream_t stream) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  MOE_CUDA(cudaStreamSynchronize(stream));
+  unsigned v = 0;
+  MOE_CUDA(cudaMemcpyFromSymbol(&v, g_moe_err_flag, sizeof v));
+  const unsigned zero = 0;
+  MOE_CUDA(cudaMemcpyToSymbol(g_moe_err_flag, &zero, sizeof zero));
+  if (v & moe::kErrTimeout) return fail(MOE_ERR_TIMEOUT, "a bounded device wait expired");
+  if (v & moe::kErrIndex) return fail(MOE_ERR_DEVICE_CHECK, "a kernel met an out-of-range index");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+int moe_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t* topk_idx,
+                   float* topk_w, moe_stream_t stream) {
+  int rc = check_common(T, E, k, 1);
+  if (rc) return rc;
+  MOE_REQUIRE(renorm == 0 || renorm == 1, MOE_ERR_INVALID_ARG, "renorm must be 0 or 1");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(logits && topk_idx && topk_w, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const int blocks = (T + 7) / 8;
+  moe::route_topk_kernel<<<blocks, 256, 0, stream>>>(logits, T, E, k, renorm, topk_idx, topk_w);
+  MOE_LAUNCHED("route_topk_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+size_t moe_brim_workspace_size(int T, int E, int R) {
+  if (T < 0 || E < 1 || R < 1) return 0;
+  const size_t n_tiles = (size_t)(T + moe::kBrimTile - 1) / moe::kBrimTile;
+  return align256(sizeof(int32_t) * n_tiles * (size_t)(R + E)) + 256;
+}
+
+int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                   const int32_t* slot_of, int E, int R, int32_t* brim0, int32_t* sfd_token,
+                   int32_t* sfd_off, int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                   float* epd_gate, int32_t* c_t, void* ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  MOE_REQUIRE(slot_of && sfd_off && epd_off && c_t, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(sfd_off, 0, sizeof(int32_t) * (R + 1), stream));
+    MOE_CUDA(cudaMemsetAsync(epd_off, 0, sizeof(int32_t) * (E + 1), stream));
+    MOE_CUDA(cudaMemsetAsync(c_t, 0, sizeof(int32_t), stream));
+    return MOE_OK;
+  }
+  MOE_REQUIRE(topk_idx && topk_w && brim0 && sfd_token && brim1 && epd_sfd && epd_gate && ws,
+              MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(ws_bytes >= moe_brim_workspace_size(T, E, R), MOE_ERR_INVALID_ARG,
+              "workspace too small: %zu < %zu bytes", ws_bytes, moe_brim_workspace_size(T, E, R));
+  const int n_tiles = (T + moe::kBrimTile - 1) / moe::kBrimTile;
+  int32_t* counts = static_cast<int32_t*>(ws);
+  moe::brim_count_kernel<<<n_tiles, moe::kBrimTile, 0, stream>>>(topk_idx, slot_of, T, k, E, R,
+                                                                 n_tiles, counts, di->err_flag);
+  MOE_LAUNCHED("brim_count_kernel");
+  moe::brim_scan_kernel<<<1, 1024, 0, stream>>>(counts, n_tiles, E, R, sfd_off, epd_off, c_t);
+  MOE_LAUNCHED("brim_scan_kernel");
+  moe::brim_scatter_kernel<<<n_tiles, moe::kBrimTile, 0, stream>>>(
+      topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, counts, brim0, sfd_token, brim1, epd_sfd,
+      epd_gate, di->err_flag);
+  MOE_LAUNCHED("brim_scatter_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+int moe_dispatch_gather(const void* x, int T, int d, int dtype, int k, int R, int L,
+                        const int32_t* brim0, const int32_t* brim1, void* x_sfd, void* x_epd,
+                        moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= moe::kMaxK && R >= 1 && L >= 1 && R * L <= moe::kMaxE,
+              MOE_ERR_UNSUPPORTED, "bad shape (T=%d k=%d R=%d L=%d)", T, k, R, L);
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && brim0 && brim1 && (x_sfd || x_epd), MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(x_sfd) && aligned16(x_epd), MOE_ERR_INVALID_ARG,
+              "row buffers must be 16-byte aligned");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const size_t cap = (size_t)T * (k < R ? k : R);
+  const int blocks = (T + moe::kMoverWarps - 1) / moe::kMoverWarps;
+  moe::dispatch_kernel<<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
+      static_cast<const uint8_t*>(x), T, d * esize(dtype), R, L, cap, T * k, brim0, brim1,
+      static_cast<uint8_t*>(x_sfd), static_cast<uint8_t*>(x_epd), di->err_flag);
+  MOE_LAUNCHED("dispatch_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                        const int32_t* brim0, const int32_t* brim1, const void* shared_out,
+                        void* y_sfd, void* y, moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= moe::kMaxK && R >= 1 && L >= 1 && R * L <= moe::kMaxE,
+              MOE_ERR_UNSUPPORTED, "bad shape (T=%d k=%d R=%d L=%d)", T, k, R, L);
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(o_epd && brim0 && brim1 && y, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(o_epd) && aligned16(y) && aligned16(y_sfd) && aligned16(shared_out),
+              MOE_ERR_INVALID_ARG, "row buffers must be 16-byte aligned");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const size_t cap = (size_t)T * (k < R ? k : R);
+  const int blocks = (T + moe::kMoverWarps - 1) / moe::kMoverWarps;
+  if (dtype == MOE_BF16) {
+    using B = __nv_bfloat16;
+    moe::combine_kernel<B><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
+        static_cast<const B*>(o_epd), T, d, R, L, cap, T * k, brim0, brim1,
+        static_cast<const B*>(shared_out), static_cast<B*>(y_sfd), static_cast<B*>(y),
+        di->err_flag);
+  } else {
+    moe::combine_kernel<float><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
+        static_cast<const float*>(o_epd), T, d, R, L, cap, T * k, brim0, brim1,
+        static_cast<const float*>(shared_out), static_cast<float*>(y_sfd),
+        static_cast<float*>(y), di->err_flag);
+  }
+  MOE_LAUNCHED("combine_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+int moe_prepare_weights(const void* wg, const void* wu, const void* wd, int E, int d, int f,
+                        int dtype, const int32_t* slot_of, void* w_gu, void* w_dn,
+                        moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(E >= 1 && E <= moe::kMaxE, MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
+  MOE_REQUIRE(d >= 64 && d % 64 == 0 && f >= 64 && f % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "d and f must be positive multiples of 64 (d=%d f=%d)", d, f);
+  MOE_REQUIRE(wg && wu && wd && w_gu && w_dn, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(wg) && aligned16(wu) && aligned16(wd) && aligned16(w_gu) && aligned16(w_dn),
+              MOE_ERR_INVALID_ARG, "weights must be 16-byte aligned");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const int es = esize(dtype);
+  const int grid = di->num_sms * 4;
+  moe::pack_gate_up_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(wg),
+                                                     static_cast<const uint8_t*>(wu), E, d, f, es,
+                                                     slot_of, static_cast<uint8_t*>(w_gu));
+  MOE_LAUNCHED("pack_gate_up_kernel");
+  moe::pack_down_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(wd), E, d, f, es,
+                                                  slot_of, static_cast<uint8_t*>(w_dn));
+  MOE_LAUNCHED("pack_down_kernel");
+  return MOE_OK;
+}
+
+int moe_prepare_shared_weights(const void* sg, const void* su, const void* sd, int S, int d,
+                               int fs, int dtype, void* w_gu, void* w_dn, moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(S >= 1 && d >= 64 && d % 64 == 0 && fs >= 64 && fs % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "need S >= 1 and d, fs positive multiples of 64 (S=%d d=%d fs=%d)", S, d, fs);
+  MOE_REQUIRE(sg && su && sd && w_gu && w_dn, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(sg) && aligned16(su) && aligned16(sd) && aligned16(w_gu) && aligned16(w_dn),
+              MOE_ERR_INVALID_ARG, "weights must be 16-byte aligned");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const int es = esize(dtype);
+  const int grid = di->num_sms * 4;
+  moe::pack_shared_gate_up_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(sg),
+                                                            static_cast<const uint8_t*>(su), S, d,
+                                                            fs, es, static_cast<uint8_t*>(w_gu));
+  MOE_LAUNCHED("pack_shared_gate_up_kernel");
+  moe::pack_shared_down_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(sd), S, d,
+                                                         fs, es, static_cast<uint8_t*>(w_dn));
+  MOE_LAUNCHED("pack_shared_down_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+size_t moe_expert_ffn_workspace_size(int m_cap, int f, int dtype) {
+  if (m_cap < 0 || f < 0) return 0;
+  return align256((size_t)m_cap * f * (dtype == MOE_BF16 ? 2 : 4)) + 256;
+}
+
+int moe_expert_ffn(const void* a, const int32_t* group_off, int G, int m_cap, const void* w_gu,
+                   const void* w_dn, int d, int f, int dtype, const float* row_scale,
+                   int ffn_kind, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(ffn_kind == MOE_FFN_SWIGLU || ffn_kind == MOE_FFN_IDENTITY, MOE_ERR_INVALID_ARG,
+              "unknown ffn_kind %d", ffn_kind);
+  MOE_REQUIRE(G >= 1 && G <= moe::kGemmMaxGroups, MOE_ERR_UNSUPPORTED,
+              "G must be in [1, %d] (got %d)", moe::kGemmMaxGroups, G);
+  MOE_REQUIRE(m_cap >= 0, MOE_ERR_INVALID_ARG, "m_cap must be >= 0");
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (m_cap == 0) return MOE_OK;
+  MOE_REQUIRE(a && group_off && out, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(a) && aligned16(out), MOE_ERR_INVALID_ARG, "a and out must be 16-byte aligned");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  if (ffn_kind == MOE_FFN_IDENTITY) {
+    const int grid = di->num_sms * 8;
+    if (dtype == MOE_BF16)
+      moe::identity_expert_kernel<__nv_bfloat16><<<grid, moe::kMoverWarps * 32, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(a), group_off, G, d, row_scale,
+          static_cast<__nv_bfloat16*>(out));
+    else
+      moe::identity_expert_kernel<float><<<grid, moe::kMoverWarps * 32, 0, stream>>>(
+          static_cast<const float*>(a), group_off, G, d, row_scale, static_cast<float*>(out));
+    MOE_LAUNCHED("identity_expert_kernel");
+    return MOE_OK;
+  }
+  MOE_REQUIRE(f >= 64 && f % 64 == 0, MOE_ERR_UNSUPPORTED, "f must be a positive multiple of 64");
+  MOE_REQUIRE(w_gu && w_dn && ws, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(ws_bytes >= moe_expert_ffn_workspace_size(m_cap, f, dtype), MOE_ERR_INVALID_ARG,
+              "workspace too small: %zu < %zu bytes", ws_bytes,
+              moe_expert_ffn_workspace_size(m_cap, f, dtype));
+  MOE_REQUIRE(aligned16(w_gu) && aligned16(w_dn) && aligned16(ws), MOE_ERR_INVALID_ARG,
+              "weights and workspace must be 16-byte aligned");
+  void* h = ws;  // [m_cap, f]
+  const int bn1 = pick_bn(2 * f), bn2 = pick_bn(d);
+  if (dtype == MOE_BF16) {
+    rc = launch_gemm_bn<moe::kEpiSwiGLU, false>(di, bn1 < 128 ? 128 : bn1, a, m_cap, d, w_gu, G,
+                                                2 * f, group_off, nullptr, h, f, stream);
+    if (rc) return rc;
+    rc = launch_gemm_bn<moe::kEpiScale, false>(di, bn2, h, m_cap, f, w_dn, G, d, group_off,
+                                               row_scale, out, d, stream);
+  } else {
+    rc = launch_gemm_bn<moe::kEpiSwiGLU, true>(di, bn1 < 128 ? 128 : bn1, a, m_cap, d, w_gu, G,
+                                               2 * f, group_off, nullptr, h, f, stream);
+    if (rc) return rc;
+    rc = launch_gemm_bn<moe::kEpiScale, true>(di, bn2, h, m_cap, f, w_dn, G, d, group_off,
+                                              row_scale, out, d, stream);
+  }
+  return rc;
+}
+
+// ---------------------------------------------------------------------------
+int moe_count_dispatched_rows(const int32_t* topk_idx, int T, int k, const int32_t* slot_of,
+                              int E, int R, int32_t* per_rank, int64_t* total, int64_t* remote,
+                              moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  MOE_REQUIRE(slot_of && per_rank && total && remote, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  MOE_CUDA(cudaMemsetAsync(per_rank, 0, sizeof(int32_t) * R, stream));
+  MOE_CUDA(cudaMemsetAsync(total, 0, sizeof(int64_t), stream));
+  MOE_CUDA(cudaMemsetAsync(remote, 0, sizeof(int64_t), stream));
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(topk_idx, MOE_ERR_INVALID_ARG, "null pointer");
+  moe::count_dispatched_kernel<<<(T + 255) / 256, 256, 0, stream>>>(
+      topk_idx, T, k, slot_of, E, R, per_rank, reinterpret_cast<unsigned long long*>(total),
+      reinterpret_cast<unsigned long long*>(remote), di->err_flag);
+  MOE_LAUNCHED("count_dispatched_kernel");
+  return MOE_OK;
+}
+
+int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* hist,
+                        int accumulate, moe_stream_t stream) {
+  int rc = check_common(T, E, k, 1);
+  if (rc) return rc;
+  MOE_REQUIRE(hist, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  if (!accumulate) MOE_CUDA(cudaMemsetAsync(hist, 0, sizeof(uint32_t) * E * E, stream));
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(topk_idx, MOE_ERR_INVALID_ARG, "null pointer");
+  moe::coact_hist_kernel<<<(T + 255) / 256, 256, 0, stream>>>(topk_idx, T, k, E, hist,
+                                                               di->err_flag);
+  MOE_LAUNCHED("coact_hist_kernel");
+  return MOE_OK;
+}
+
+}  // extern "C"

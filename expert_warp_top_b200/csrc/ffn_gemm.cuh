@@ -1,0 +1,349 @@
+// ffn_gemm.cuh -- grouped GEMM over ragged expert row groups on tcgen05.
+//
+// The expert computation of the Occult pipeline (Occult paper, TL;DR:
+// "sparse-matrix-multiplication pipeline"): every expert multiplies only its
+// own compact EPD rows.  Group g covers rows group_off[g] .. group_off[g+1]-1
+// of A and uses weight block g of B:
+//   C[rows, n] = sum_k A[rows, k] * B[g*N + n, k]      (both K-major)
+//
+// Kernel shape (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 (bf16; 32 wide
+//               for fp32/TF32) per stage, 128-byte swizzle, STAGES-deep ring
+//   warp 1      TMEM owner and MMA issuer: tcgen05.mma M=128, N=BN, K=16 (8 for
+//               TF32), accumulators double-buffered in TMEM (2 x BN columns)
+//   warps 2..5  epilogue: tcgen05.ld of its 32 TMEM lanes (= 32 tile rows),
+//               fused SwiGLU (GEMM 1) or gate-weight scaling (GEMM 2), masked
+//               row stores (a tile never writes past its group)
+// Tiles are ordered group by group, N block by N block, M block fastest, and
+// dealt round-robin to the CTAs; the same weight block is then read by
+// neighbouring CTAs at the same time and stays in L2.
+//
+// Every mbarrier wait is bounded (globaltimer); a wait that expires raises the
+// timeout bit of the device error flag and the CTA unwinds: the producer
+// waits for its own TMA copies in flight, the MMA issuer drains its MMAs, and
+// TMEM is freed before the kernel returns.
+#pragma once
+#include <type_traits>
+
+#include "tc_ptx.cuh"
+
+namespace moe {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmThreads = 192;
+constexpr int kGemmMaxGroups = 1024;
+constexpr int kEpiSwiGLU = 0;  // out[:, n0/2 + j] = silu(gate) * up   (64-row interleave)
+constexpr int kEpiScale = 1;   // out[:, n0 + j]   = row_scale * acc
+
+// Debug switch used by the timeout test: the producer skips the first stage it
+// would load, so the MMA issuer's wait can never complete.
+constexpr int kDebugSkipFirstLoad = 1;
+
+template <int BN, bool TF32>
+struct GemmCfg {
+  static constexpr int kElemBytes = TF32 ? 4 : 2;
+  static constexpr int kBK = 128 / kElemBytes;       // one 128-byte swizzle row
+  static constexpr int kMmaK = 32 / kElemBytes;      // K of one tcgen05.mma
+  static constexpr int kMmaPerStage = kBK / kMmaK;   // = 4
+  static constexpr int kABytes = kGemmBM * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;  // a power of two here
+  static constexpr size_t kSmemBytes =
+      1024 /* alignment slack */ + (size_t)kStages * kStageBytes + 256 /* barriers */ +
+      sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
+};
+
+struct GemmArgs {
+  const int32_t* group_off;  // [G+1] device
+  int G;
+  int N;                     // output columns per group (B rows per group)
+  int K;
+  int m_cap;                 // rows of A and of out
+  const float* row_scale;    // kEpiScale: per-row factor (nullable)
+  void* out;
+  int ldo;                   // out row stride, elements
+  unsigned* err;
+  uint64_t wait_limit_ns;
+  int debug;
+};
+
+template <int BN, int EPI, bool TF32>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+  using Cfg = GemmCfg<BN, TF32>;
+  using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
+  constexpr int S = Cfg::kStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * Cfg::kStageBytes);
+  uint64_t* full_bar = bars;            // [S]   TMA -> MMA
+  uint64_t* empty_bar = bars + S;       // [S]   MMA -> TMA
+  uint64_t* tfull_bar = bars + 2 * S;   // [2]   MMA -> epilogue
+  uint64_t* tempty_bar = bars + 2 * S + 2;  // [2] epilogue -> MMA
+  uint64_t* drain_bar = bars + 2 * S + 4;   // [1] MMA drain at teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_off = reinterpret_cast<int32_t*>(smem + (size_t)S * Cfg::kStageBytes + 256);
+  int32_t* s_end = s_off + kGemmMaxGroups;
+  int32_t* s_prefix = s_end + kGemmMaxGroups;
+
+  const int warp = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  const int G = args.G;
+  const int n_blocks = args.N / BN;
+  const int k_blocks = args.K / Cfg::kBK;
+
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmap_a);
+    tc::tma_prefetch_desc(&tmap_b);
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
+      tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(tc::smem_u32(&tfull_bar[a]), 1);
+      tc::mbar_init(tc::smem_u32(&tempty_bar[a]), 4);  // one arrive per epilogue warp
+    }
+    tc::mbar_init(tc::smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    tc::mbar_init_fence();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (warp == 2) {
+    // group offsets and the tile prefix: tiles of group g = m_blocks(g) * n_blocks.
+    // A group whose bounds leave [0, m_cap] or run backwards is treated as
+    // empty and raises the index error bit.
+    int carry = 0;
+    bool bad = false;
+    for (int g0 = 0; g0 < G; g0 += 32) {
+      const int g = g0 + (int)lane;
+      int tiles_g = 0;
+      if (g < G) {
+        const int lo = args.group_off[g], hi = args.group_off[g + 1];
+        const bool ok = lo >= 0 && hi >= lo && hi <= args.m_cap;
+        bad |= !ok;
+        s_off[g] = lo;
+        s_end[g] = ok ? hi : lo;
+        const int rows = ok ? hi - lo : 0;
+        tiles_g = ((rows + kGemmBM - 1) / kGemmBM) * n_blocks;
+      }
+      int inc = tiles_g;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if ((int)lane >= o) inc += y;
+      }
+      if (g < G) s_prefix[g] = carry + inc - tiles_g;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) s_prefix[G] = carry;
+    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_error(args.err, kErrIndex);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = s_prefix[G];
+  const tc::WaitCtl wctl{abort_flag, args.err, args.wait_limit_ns};
+
+  // tile -> (group, m block, n block)
+  auto locate = [&](int tile, int& g, int& row0, int& rows, int& n0) {
+    int lo = 0, hi = G;  // largest g with s_prefix[g] <= tile
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_prefix[mid] <= tile) lo = mid;
+      else hi = mid;
+    }
+    g = lo;
+    const int local = tile - s_prefix[g];
+    const int gstart = s_off[g], gend = s_end[g];
+    const int m_blocks = (gend - gstart + kGemmBM - 1) / kGemmBM;
+    const int nb = local / m_blocks, mb = local - nb * m_blocks;
+    row0 = gstart + mb * kGemmBM;
+    rows = min(kGemmBM, gend - row0);
+    n0 = nb * BN;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_a = tc::policy_evict_normal();
+      const uint64_t pol_b = tc::policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_parity = 0;  // per stage: armed at least once, parity of the last arming
+      bool skip_next = (args.debug & kDebugSkipFirstLoad) != 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int g, row0, rows, n0;
+        locate(tile, g, row0, rows, n0);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl)) {
+            ok = false;
+            break;
+          }
+          if (!skip_next) {
+            const uint32_t fb = tc::smem_u32(&full_bar[stage]);
+            tc::mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+            uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
+            tc::tma_load_2d(tc::smem_u32(sa), &tmap_a, fb, kb * Cfg::kBK, row0, pol_a);
+            tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, kb * Cfg::kBK,
+                            g * args.N + n0, pol_b);
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          }
+          skip_next = false;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Leave no TMA write in flight into this CTA's shared memory: wait for
+      // the last arming of every stage (already complete on the normal path,
+      // where the MMA issuer consumed it; maybe not if the CTA is unwinding).
+      for (int s = 0; s < S; ++s)
+        if ((armed >> s) & 1u)
+          tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_m128<TF32, BN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        if (!tc::wait_bounded(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl)) break;
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!tc::wait_bounded(tc::smem_u32(&full_bar[stage]), phase, wctl)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t sa = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
+          const uint64_t adesc = tc::desc_sw128_kmajor(sa);
+          const uint64_t bdesc = tc::desc_sw128_kmajor(sa + Cfg::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {
+            // +32 bytes along K inside the swizzled row = +2 in the address field
+            const uint64_t off = static_cast<uint64_t>(kk * 2);
+            if (TF32)
+              tc::mma_tf32(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+            else
+              tc::mma_f16(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+          }
+          tc::commit(tc::smem_u32(&empty_bar[stage]));  // frees the stage when these MMAs finish
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::commit(tc::smem_u32(&tfull_bar[acc]));  // accumulator ready
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // drain: every MMA this thread issued has finished before TMEM is freed
+      tc::commit(tc::smem_u32(drain_bar));
+      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int r_in_tile = quarter * 32 + (int)lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    TOut* out = reinterpret_cast<TOut*>(args.out);
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int g, row0, rows, n0;
+      locate(tile, g, row0, rows, n0);
+      // lane 0 waits for the accumulator; the warp then proceeds converged
+      bool ok = true;
+      if (lane == 0) ok = tc::wait_bounded(tc::smem_u32(&tfull_bar[acc]), acc_phase, wctl);
+      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+      if (!ok) break;
+      __syncwarp();
+      tc::fence_after_sync();
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const bool valid = r_in_tile < rows;
+      const size_t grow = static_cast<size_t>(row0 + r_in_tile);
+      if (EPI == kEpiSwiGLU) {
+        // columns [128p, 128p+64) are gate rows, [128p+64, 128p+128) the matching up rows
+#pragma unroll 1
+        for (int p = 0; p < BN / 128; ++p) {
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t gr[32], ur[32];
+            tc::tmem_ld32(taddr + p * 128 + h * 32, gr);
+            tc::tmem_ld32(taddr + p * 128 + 64 + h * 32, ur);
+            tc::tmem_ld_wait();
+            if (valid) {
+              float hv[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float gv = __uint_as_float(gr[i]);
+                const float uv = __uint_as_float(ur[i]);
+                hv[i] = gv / (1.0f + __expf(-gv)) * uv;
+              }
+              TOut* dst = out + grow * args.ldo + (n0 >> 1) + p * 64 + h * 32;
+#pragma unroll
+              for (int v = 0; v < 32 / Vec16<TOut>::n; ++v)
+                st_v4(dst + v * Vec16<TOut>::n, Vec16<TOut>::from_f32(hv + v * Vec16<TOut>::n));
+            }
+          }
+        }
+      } else {
+        const float scale = (valid && args.row_scale) ? args.row_scale[grow] : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t vr[32];
+          tc::tmem_ld32(taddr + c * 32, vr);
+          tc::tmem_ld_wait();
+          if (valid) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]) * scale;
+            TOut* dst = out + grow * args.ldo + n0 + c * 32;
+#pragma unroll
+            for (int q = 0; q < 32 / Vec16<TOut>::n; ++q)
+              st_v4(dst + q * Vec16<TOut>::n, Vec16<TOut>::from_f32(v + q * Vec16<TOut>::n));
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tc::smem_u32(&tempty_bar[acc]));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,129 @@
+"""One Occult-style MoE layer on one GPU: buffers plus the call sequence.
+
+PyTorch only allocates device memory here; every step of the layer runs in
+the CUDA library through the binding:
+
+  route (top-k, softmax)        moe_route_topk
+  BRIM_0 / BRIM_1 / C_T         moe_brim_build
+  ORI -> SFD -> EPD             moe_dispatch_gather
+  routed experts (grouped GEMM) moe_expert_ffn over the EPD groups
+  shared experts                moe_expert_ffn over the ORI rows (one group)
+  pre-reduce + combine          moe_combine_scatter
+  dispatched-row counter        moe_count_dispatched_rows
+  co-activation histogram       moe_coact_histogram (accumulating)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _binding as B
+
+
+class MoELayer:
+    def __init__(self, *, T, d, f, E, k, R, renorm=0, dtype=torch.bfloat16, S=0, fs=0,
+                 slot_of=None, wg=None, wu=None, wd=None, sg=None, su=None, sd=None,
+                 ffn_kind=B.MOE_FFN_SWIGLU, device="cuda", stream=None):
+        if E % R:
+            raise ValueError("R must divide E")
+        self.T, self.d, self.f, self.E, self.k, self.R = T, d, f, E, k, R
+        self.L = E // R
+        self.renorm, self.dtype, self.S, self.fs = renorm, dtype, S, fs
+        self.ffn_kind = ffn_kind
+        self.cap = T * min(k, R)
+        self.tk = T * k
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        act = dict(dtype=dtype, device=dev)
+        if slot_of is None:
+            slot_of = torch.arange(E, dtype=torch.int32)
+        self.slot_of = slot_of.to(**i32).contiguous()
+        # routing and BRIM state
+        self.topk_idx = torch.empty(T, k, **i32)
+        self.topk_w = torch.empty(T, k, **f32)
+        self.brim0 = torch.empty(R, T, **i32)
+        self.sfd_token = torch.empty(max(self.cap, 1), **i32)
+        self.sfd_off = torch.empty(R + 1, **i32)
+        self.brim1 = torch.empty(self.L, max(self.cap, 1), **i32)
+        self.epd_off = torch.empty(E + 1, **i32)
+        self.epd_sfd = torch.empty(max(self.tk, 1), **i32)
+        self.epd_gate = torch.empty(max(self.tk, 1), **f32)
+        self.c_t = torch.empty(1, **i32)
+        self.brim_ws = torch.empty(max(B.moe_brim_workspace_size(T, E, R), 256),
+                                   dtype=torch.uint8, device=dev)
+        # token states
+        self.x_sfd = torch.empty(max(self.cap, 1), d, **act)
+        self.x_epd = torch.empty(max(self.tk, 1), d, **act)
+        self.o_epd = torch.empty(max(self.tk, 1), d, **act)
+        self.y_sfd = torch.empty(max(self.cap, 1), d, **act)
+        self.y = torch.empty(T, d, **act)
+        # statistics
+        self.per_rank = torch.empty(R, **i32)
+        self.total = torch.empty(1, dtype=torch.int64, device=dev)
+        self.remote = torch.empty(1, dtype=torch.int64, device=dev)
+        self.hist = torch.zeros(E, E, dtype=torch.int32, device=dev)
+        # weights (packed once, in slot order)
+        code = B.dtype_code(dtype)
+        self.w_gu = self.w_dn = None
+        if ffn_kind == B.MOE_FFN_SWIGLU:
+            self.w_gu = torch.empty(E, 2 * f, d, **act)
+            self.w_dn = torch.empty(E, d, f, **act)
+            B.moe_prepare_weights(wg.to(**act).contiguous(), wu.to(**act).contiguous(),
+                                  wd.to(**act).contiguous(), self.slot_of, self.w_gu, self.w_dn,
+                                  stream)
+        self.ffn_ws = torch.empty(max(B.moe_expert_ffn_workspace_size(max(self.tk, 1), f, code), 256),
+                                  dtype=torch.uint8, device=dev)
+        self.shared_out = None
+        if S > 0:
+            F = S * fs
+            self.sw_gu = torch.empty(1, 2 * F, d, **act)
+            self.sw_dn = torch.empty(1, d, F, **act)
+            B.moe_prepare_shared_weights(sg.to(**act).contiguous(), su.to(**act).contiguous(),
+                                         sd.to(**act).contiguous(), self.sw_gu, self.sw_dn, stream)
+            self.shared_off = torch.tensor([0, T], **i32)
+            self.shared_out = torch.empty(T, d, **act)
+            self.shared_ws = torch.empty(max(B.moe_expert_ffn_workspace_size(max(T, 1), F, code), 256),
+                                         dtype=torch.uint8, device=dev)
+
+    # -- the steps ---------------------------------------------------------
+    def route(self, logits, stream=None):
+        B.moe_route_topk(logits, self.k, self.renorm, self.topk_idx, self.topk_w, stream)
+
+    def build_brims(self, stream=None):
+        B.moe_brim_build(self.topk_idx, self.topk_w, self.slot_of, self.E, self.R, self.brim0,
+                         self.sfd_token, self.sfd_off, self.brim1, self.epd_off, self.epd_sfd,
+                         self.epd_gate, self.c_t, self.brim_ws, stream)
+
+    def dispatch(self, x, stream=None):
+        B.moe_dispatch_gather(x, self.k, self.R, self.L, self.brim0, self.brim1, self.x_sfd,
+                              self.x_epd, stream)
+
+    def experts(self, stream=None):
+        B.moe_expert_ffn(self.x_epd[: max(self.tk, 1)], self.epd_off, self.w_gu, self.w_dn, self.f,
+                         self.epd_gate, self.ffn_kind, self.o_epd, self.ffn_ws, stream)
+
+    def shared_experts(self, x, stream=None):
+        if self.S > 0:
+            B.moe_expert_ffn(x, self.shared_off, self.sw_gu, self.sw_dn, self.S * self.fs, None,
+                             B.MOE_FFN_SWIGLU, self.shared_out, self.shared_ws, stream)
+
+    def combine(self, stream=None):
+        B.moe_combine_scatter(self.o_epd, self.T, self.k, self.R, self.L, self.brim0, self.brim1,
+                              self.shared_out, self.y_sfd, self.y, stream)
+
+    def statistics(self, stream=None):
+        B.moe_count_dispatched_rows(self.topk_idx, self.slot_of, self.E, self.R, self.per_rank,
+                                    self.total, self.remote, stream)
+        B.moe_coact_histogram(self.topk_idx, self.E, self.hist, 1, stream)
+
+    def forward(self, logits, x, stream=None, stats=True):
+        """All steps of the layer on `stream`; returns y [T, d] (a view of self.y)."""
+        self.route(logits, stream)
+        self.build_brims(stream)
+        self.dispatch(x, stream)
+        self.experts(stream)
+        self.shared_experts(x, stream)
+        self.combine(stream)
+        if stats:
+            self.statistics(stream)
+        return self.y

@@ -1,0 +1,245 @@
+/*
+ * moe_occult.h -- C ABI of the Occult-style MoE layer hot path on B200 (sm_100a).
+ *
+ * One mixture-of-experts layer on one GPU, done the way the Occult paper
+ * ("Occult: Optimizing Collaborative Communication across Experts for
+ * Accelerated Parallel MoE Training and Inference") lays it out:
+ *
+ *   route        each token picks its top-k experts       moe_route_topk
+ *   BRIM build   BRIM_0 [R x T], BRIM_1 [L x C_T], C_T     moe_brim_build
+ *   dispatch     ORI -> SFD (one row per token and rank)   moe_dispatch_gather
+ *                SFD -> EPD (one row per token and expert)
+ *   experts      grouped SwiGLU FFN on the EPD rows        moe_expert_ffn
+ *   combine      per-rank pre-reduce (intra-collaboration) moe_combine_scatter
+ *                then scatter back to ORI order
+ *
+ * plus a placement-aware dispatched-row counter and an expert co-activation
+ * histogram for correlated placement ("Expert Coupling in MoE Pretraining",
+ * Abstract).  R expert-parallel ranks are simulated: they are partitions of
+ * the expert set on this one GPU, and the SFD segments stand for what an
+ * all-to-all would carry.  Nothing here moves data between GPUs.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every function returns an int status (moe_status).  On failure,
+ *    moe_last_error() gives a message for the calling host thread.
+ *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *    owns every buffer; no entry point allocates device memory.  Scratch
+ *    space is passed in as a workspace whose size a *_workspace_size query
+ *    gives.
+ *  - Work is enqueued asynchronously on the caller's stream (NULL = legacy
+ *    default stream); no entry point synchronises, except
+ *    moe_get_device_status() and moe_layer_forward_host().
+ *  - Arguments are validated on the host before anything is launched: a bad
+ *    argument returns MOE_ERR_INVALID_ARG, an unsupported shape or dtype
+ *    returns MOE_ERR_UNSUPPORTED, and nothing is enqueued in either case.
+ *    Index values that live on the device (expert ids, BRIM entries) are
+ *    range-checked by the kernels: an invalid one is skipped and raises the
+ *    device error flag, which moe_get_device_status() reports.
+ *  - Matrices are row-major and densely packed unless a stride is given.
+ *  - Supported range: 1 <= E <= 256, 1 <= k <= min(E, 16), 1 <= R <= E,
+ *    E % R == 0, d % 64 == 0, f % 64 == 0, T >= 0.
+ *
+ * Notation: T tokens, d model width, f expert FFN width, E routed experts,
+ * k experts per token, R simulated EP ranks, L = E / R local experts per rank,
+ * cap = T * min(k, R) (the largest possible C_T), slot_of[E] the placement
+ * (a permutation of 0..E-1): expert e lives on rank slot_of[e] / L as local
+ * expert slot_of[e] % L.
+ */
+#ifndef MOE_OCCULT_H
+#define MOE_OCCULT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,  /* null pointer, negative size, bad enum */
+  MOE_ERR_UNSUPPORTED = -2,  /* shape or dtype outside the supported range */
+  MOE_ERR_CUDA = -3,         /* a CUDA runtime/driver call or launch failed */
+  MOE_ERR_DEVICE_CHECK = -4, /* a kernel met an out-of-range index */
+  MOE_ERR_TIMEOUT = -5       /* a bounded device-side wait expired */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_FFN_SWIGLU = 0, MOE_FFN_IDENTITY = 1 } moe_ffn_kind;
+
+/* Version of this ABI (incremented on any signature change). */
+int moe_abi_version(void);
+
+/* Message describing the last failure on the calling host thread ("" if none).
+ * The string stays valid until the next call on the same thread. */
+const char* moe_last_error(void);
+
+/* Test-only knobs.  flags bit 0: the expert GEMM's producer skips its first
+ * TMA load, so a bounded wait is certain to expire (exercises the timeout
+ * path without faulting or hanging the GPU).  wait_limit_ms: how long a
+ * device-side wait may last before it gives up (default 4000 ms).  Process
+ * wide; not for production use. */
+int moe_set_debug(int flags, double wait_limit_ms);
+
+/* Synchronises `stream`, then reads and clears the device error flag that the
+ * kernels raise.  Returns MOE_ERR_TIMEOUT if a bounded wait expired,
+ * MOE_ERR_DEVICE_CHECK if an index was out of range, else MOE_OK. */
+int moe_get_device_status(moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route_topk -- each token is routed to k of the E experts ("Expert
+ * Coupling in MoE Pretraining", Abstract; top-2/4/6/8 in the Occult paper,
+ * Figure 3).
+ *   logits   [T, E] float32   router logits
+ *   topk_idx [T, k] int32     out: expert ids in descending logit order; of
+ *                              equal logits the lower id ranks first
+ *                              (-0.0 and +0.0 compare equal)
+ *   topk_w   [T, k] float32   out: gate weights.  renorm = 0: softmax over all
+ *                              E logits, then the k selected entries;
+ *                              renorm = 1: softmax over the k selected logits.
+ * Logits must be finite; NaN gives unspecified (but in-range) ids.
+ * ------------------------------------------------------------------------- */
+int moe_route_topk(const float* logits, int T, int E, int k, int renorm,
+                   int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_brim_build -- the two bidirectional re-index matrices of the Occult
+ * paper (Figure 5: BRIM_0 is [EP devices x ORI tokens], BRIM_1 is [local
+ * experts per device x SFD tokens]) and the all-to-all budget C_T (TL;DR).
+ * A token is sent once to every rank that holds at least one of its experts.
+ *   topk_idx [T, k] int32   distinct expert ids per token (checked on device)
+ *   topk_w   [T, k] float32 gate weights
+ *   slot_of  [E] int32      placement (device)
+ *   brim0    [R, T] int32   out: SFD row of (rank r, token t), or -1
+ *   sfd_token[cap] int32    out: ORI token of each SFD row (first C_T used)
+ *   sfd_off  [R+1] int32    out: first SFD row of each rank; sfd_off[R] = C_T
+ *   brim1    [L, cap] int32 out: EPD row of (local expert l, SFD row s), or
+ *                           -1; row stride cap; columns >= C_T are not written
+ *   epd_off  [E+1] int32    out: first EPD row of each slot (slot order)
+ *   epd_sfd  [T*k] int32    out: SFD row feeding each EPD row
+ *   epd_gate [T*k] float32  out: gate weight of each EPD row
+ *   c_t      [1] int32      out: C_T, the number of SFD rows
+ *   ws, ws_bytes            scratch, at least moe_brim_workspace_size(T, E, R)
+ * Inside a rank's SFD segment and inside an expert's EPD group, rows follow
+ * ascending token order, so every output is unique and reproducible.
+ * ------------------------------------------------------------------------- */
+size_t moe_brim_workspace_size(int T, int E, int R);
+int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                   const int32_t* slot_of, int E, int R,
+                   int32_t* brim0, int32_t* sfd_token, int32_t* sfd_off,
+                   int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                   float* epd_gate, int32_t* c_t,
+                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_dispatch_gather -- ORI -> SFD -> EPD (Occult paper, Figure 4), guided by
+ * the BRIMs: for every token t and rank r with s = BRIM_0[r][t] >= 0,
+ *   x_sfd[s] = x[t]                         (the simulated all-to-all payload)
+ * and for every local expert l with p = BRIM_1[l][s] >= 0,
+ *   x_epd[p] = x[t]                         (the expert-partitioned rows).
+ * Rows are copied bit for bit; each ORI row is read once.
+ *   x     [T, d]   dtype
+ *   x_sfd [cap, d] dtype  (may be NULL to skip it)
+ *   x_epd [T*k, d] dtype  (may be NULL to skip it; not both NULL)
+ * ------------------------------------------------------------------------- */
+int moe_dispatch_gather(const void* x, int T, int d, int dtype, int k, int R, int L,
+                        const int32_t* brim0, const int32_t* brim1,
+                        void* x_sfd, void* x_epd, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_prepare_weights -- one-time repacking of routed expert weights for
+ * moe_expert_ffn (not on the per-layer path):
+ *   wg, wu [E, f, d], wd [E, d, f]  (expert-id order, dtype)
+ *   slot_of [E] (device, may be NULL = identity placement)
+ *   w_gu  [E, 2f, d] out: slot order; gate and up rows interleaved in blocks
+ *                         of 64: rows 128i..128i+63 = gate rows 64i..64i+63,
+ *                         rows 128i+64..128i+127 = up rows 64i..64i+63
+ *   w_dn  [E, d, f]  out: slot order
+ * moe_prepare_shared_weights packs S always-on experts (sg, su [S, fs, d],
+ * sd [S, d, fs]) into ONE expert of width S*fs (gate/up rows concatenated over
+ * the experts, then interleaved as above; down columns concatenated), whose
+ * output is the sum of the S experts' outputs.  Requires (S*fs) % 64 == 0.
+ * ------------------------------------------------------------------------- */
+int moe_prepare_weights(const void* wg, const void* wu, const void* wd, int E, int d,
+                        int f, int dtype, const int32_t* slot_of, void* w_gu, void* w_dn,
+                        moe_stream_t stream);
+int moe_prepare_shared_weights(const void* sg, const void* su, const void* sd, int S,
+                               int d, int fs, int dtype, void* w_gu, void* w_dn,
+                               moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_ffn -- the expert computation of the Occult pipeline (TL;DR:
+ * "sparse-matrix-multiplication pipeline"), as a grouped GEMM over ragged
+ * row groups on the tcgen05 tensor cores:
+ *   for every group g (rows group_off[g] .. group_off[g+1]-1 of a, expert g):
+ *     h   = silu(a Wg^T) * (a Wu^T)        [rows, f]  (kept in the workspace)
+ *     out = row_scale * (h Wd^T)           [rows, d]
+ *   a         [m_cap, d] dtype      input rows (e.g. the EPD rows)
+ *   group_off [G+1] int32 (device)  ascending, group_off[0] >= 0,
+ *                                   group_off[G] <= m_cap
+ *   w_gu, w_dn                      packed by moe_prepare_weights (G experts)
+ *   row_scale [m_cap] float32       per-row factor (e.g. epd_gate), or NULL = 1
+ *   ffn_kind  MOE_FFN_SWIGLU, or MOE_FFN_IDENTITY (out = row_scale * a; the
+ *             weights are not read and may be NULL)
+ *   out       [m_cap, d] dtype      rows outside every group are not written
+ *   ws        at least moe_expert_ffn_workspace_size(m_cap, f, dtype) bytes
+ * bf16 runs bf16 x bf16 -> fp32 MMAs; f32 runs TF32 MMAs (fp32 accumulate).
+ * The hidden activation h is rounded to dtype between the two GEMMs.
+ * Device-side waits are bounded: a wait that expires raises MOE_ERR_TIMEOUT
+ * through moe_get_device_status() and the kernel returns.
+ * ------------------------------------------------------------------------- */
+size_t moe_expert_ffn_workspace_size(int m_cap, int f, int dtype);
+int moe_expert_ffn(const void* a, const int32_t* group_off, int G, int m_cap,
+                   const void* w_gu, const void* w_dn, int d, int f, int dtype,
+                   const float* row_scale, int ffn_kind, void* out,
+                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine_scatter -- the return path (Occult paper, Figure 4, and the
+ * intra-collaboration of the Abstract): for every SFD row s, its rank's
+ * expert outputs are summed into ONE return row
+ *   y_sfd[s] = sum over l ascending with BRIM_1[l][s] >= 0 of o_epd[BRIM_1[l][s]]
+ * and every token sums its return rows back in ORI order
+ *   y[t] = sum over r ascending with BRIM_0[r][t] >= 0 of y_sfd[BRIM_0[r][t]]
+ *          (+ shared_out[t] when shared_out is not NULL).
+ * Sums run in fp32; y_sfd is rounded to dtype (it is the payload), and y sums
+ * the rounded payload rows.
+ *   o_epd [T*k, d] dtype; y_sfd [cap, d] dtype (may be NULL); y [T, d] dtype;
+ *   shared_out [T, d] dtype or NULL.
+ * ------------------------------------------------------------------------- */
+int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                        const int32_t* brim0, const int32_t* brim1,
+                        const void* shared_out, void* y_sfd, void* y,
+                        moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_count_dispatched_rows -- rows a once-per-rank dispatcher sends under a
+ * placement ("Expert Coupling in MoE Pretraining", Abstract), without
+ * building BRIMs:
+ *   per_rank [R] int32  out: tokens sent to each rank
+ *   total    [1] int64  out: sum of per_rank (= C_T)
+ *   remote   [1] int64  out: rows whose rank differs from the token's source
+ *                            rank floor(t * R / T)
+ * ------------------------------------------------------------------------- */
+int moe_count_dispatched_rows(const int32_t* topk_idx, int T, int k,
+                              const int32_t* slot_of, int E, int R,
+                              int32_t* per_rank, int64_t* total, int64_t* remote,
+                              moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_coact_histogram -- expert co-activation counts for correlated placement
+ * ("Expert Coupling in MoE Pretraining", Abstract; "collaborated" experts in
+ * the Occult paper, Abstract):
+ *   hist [E, E] uint32: hist[a][b] (a != b) = tokens that selected both a and
+ *   b; hist[a][a] = tokens that selected a.  accumulate = 0 clears it first.
+ * ------------------------------------------------------------------------- */
+int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* hist,
+                        int accumulate, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_OCCULT_H */

@@ -1,0 +1,98 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import expert_warp_top_b200 as moe
+from expert_warp_top_b200 import _binding as B
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def header_functions():
+    text = (ROOT / "include" / "moe_occult.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(moe_\w+)\s*\(", text, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moe.load()
+    declared = header_functions()
+    assert len(declared) >= 14
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(B.EXPORTS)
+    assert moe.moe_abi_version() == 1
+
+
+def test_workspace_queries():
+    assert moe.moe_brim_workspace_size(4096, 64, 8) >= 4 * 16 * 72
+    assert moe.moe_brim_workspace_size(-1, 64, 8) == 0
+    assert moe.moe_expert_ffn_workspace_size(1000, 1024, B.MOE_BF16) >= 1000 * 1024 * 2
+    assert moe.moe_expert_ffn_workspace_size(1000, 1024, B.MOE_F32) >= 1000 * 1024 * 4
+
+
+NULL = ctypes.c_void_p(0)
+
+
+@pytest.mark.parametrize("T,E,k,renorm,code", [
+    (-1, 8, 2, 0, B.MOE_ERR_INVALID_ARG),
+    (4, 8, 9, 0, B.MOE_ERR_UNSUPPORTED),      # k > E
+    (4, 300, 2, 0, B.MOE_ERR_UNSUPPORTED),    # E > 256
+    (4, 64, 17, 0, B.MOE_ERR_UNSUPPORTED),    # k > 16
+    (4, 8, 2, 2, B.MOE_ERR_INVALID_ARG),      # renorm not 0/1
+    (4, 8, 2, 0, B.MOE_ERR_INVALID_ARG),      # null pointers
+])
+def test_route_rejects_bad_arguments_on_host(T, E, k, renorm, code):
+    lib = moe.load()
+    assert lib.moe_route_topk(NULL, T, E, k, renorm, NULL, NULL, NULL) == code
+    assert lib.moe_last_error()
+
+
+def test_route_empty_is_a_no_op():
+    assert moe.load().moe_route_topk(NULL, 0, 8, 2, 0, NULL, NULL, NULL) == B.MOE_OK
+
+
+@pytest.mark.parametrize("E,k,R", [(8, 2, 3), (8, 2, 0), (8, 2, 16)])
+def test_brim_rejects_bad_rank_counts(E, k, R):
+    lib = moe.load()
+    rc = lib.moe_brim_build(NULL, NULL, 16, k, NULL, E, R, NULL, NULL, NULL, NULL, NULL, NULL,
+                            NULL, NULL, NULL, ctypes.c_size_t(0), NULL)
+    assert rc == B.MOE_ERR_UNSUPPORTED
+
+
+def test_ffn_rejects_bad_shapes():
+    lib = moe.load()
+    # d not a multiple of 64
+    assert lib.moe_expert_ffn(NULL, NULL, 1, 16, NULL, NULL, 96, 128, B.MOE_BF16, NULL,
+                              B.MOE_FFN_SWIGLU, NULL, NULL, ctypes.c_size_t(0), NULL) \
+        == B.MOE_ERR_UNSUPPORTED
+    # unknown dtype / kind
+    assert lib.moe_expert_ffn(NULL, NULL, 1, 16, NULL, NULL, 128, 128, 7, NULL,
+                              B.MOE_FFN_SWIGLU, NULL, NULL, ctypes.c_size_t(0), NULL) \
+        == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(NULL, NULL, 1, 16, NULL, NULL, 128, 128, B.MOE_BF16, NULL,
+                              5, NULL, NULL, ctypes.c_size_t(0), NULL) == B.MOE_ERR_INVALID_ARG
+    # too many groups
+    assert lib.moe_expert_ffn(NULL, NULL, 5000, 16, NULL, NULL, 128, 128, B.MOE_BF16, NULL,
+                              B.MOE_FFN_SWIGLU, NULL, NULL, ctypes.c_size_t(0), NULL) \
+        == B.MOE_ERR_UNSUPPORTED
+
+
+def test_movers_reject_bad_shapes():
+    lib = moe.load()
+    assert lib.moe_dispatch_gather(NULL, 16, 100, B.MOE_BF16, 2, 4, 2, NULL, NULL, NULL, NULL,
+                                   NULL) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_combine_scatter(NULL, 16, 128, B.MOE_BF16, 2, 4, 2, NULL, NULL, NULL, NULL,
+                                   NULL, NULL) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_debug(0, ctypes.c_double(-1.0)) == B.MOE_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        moe.moe_route_topk(torch.zeros(4, 8), 2, 0, torch.zeros(4, 2, dtype=torch.int32),
+                           torch.zeros(4, 2))

@@ -1,0 +1,236 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on seeded synthetic inputs.
+
+Indices, counts, BRIMs and C_T must match bit for bit; copies must be bit
+exact; gate weights match to fp32 rounding; layer outputs match within the
+per-row normwise tolerance OUT_RTOL (bf16 data, fp32 accumulation)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import expert_warp_top_b200 as moe
+from expert_warp_top_b200 import inputs
+from expert_warp_top_b200.layer import MoELayer
+from helpers import OUT_RTOL, expert_at_slot, oracle_route, rowwise_rel_err, to_oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def softmax_rtol(E: int) -> float:
+    # fp32 expf (a few ulp) + an fp32 sum of E terms + one division, vs double
+    return (E + 8) * 2.0 ** -23
+
+
+def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU):
+    dt = inputs.torch_dtype(cfg)
+    kw = {}
+    if ffn_kind == moe.MOE_FFN_SWIGLU:
+        kw = dict(wg=inp["wg"].to(DEV), wu=inp["wu"].to(DEV), wd=inp["wd"].to(DEV))
+        if cfg.S:
+            kw.update(sg=inp["sg"].to(DEV), su=inp["su"].to(DEV), sd=inp["sd"].to(DEV))
+    return MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
+                    dtype=dt, S=cfg.S if ffn_kind == moe.MOE_FFN_SWIGLU else 0, fs=cfg.fs,
+                    slot_of=slot_of, ffn_kind=ffn_kind, device=DEV, **kw)
+
+
+def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
+    """Route, BRIMs, counts and histogram against the oracle, bit for bit."""
+    torch.cuda.synchronize()
+    idx = layer.topk_idx.cpu().numpy()
+    assert np.array_equal(idx, idx_ref)
+    w = layer.topk_w.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(w, w_ref, rtol=softmax_rtol(cfg.E), atol=1e-30)
+    # BRIMs from the GPU's own (fp32) weights so that epd_gate is comparable bit for bit
+    b = oracle.brim(idx, layer.topk_w.cpu().numpy().astype(np.float64), slot_of, cfg.E, cfg.R)
+    c_t = int(layer.c_t.item())
+    assert c_t == b["c_t"]
+    assert np.array_equal(layer.brim0.cpu().numpy(), b["brim0"])
+    assert np.array_equal(layer.sfd_off.cpu().numpy(), b["sfd_off"])
+    assert np.array_equal(layer.sfd_token[:c_t].cpu().numpy(), b["sfd_token"])
+    assert np.array_equal(layer.brim1[:, :c_t].cpu().numpy(), b["brim1"][:, :c_t])
+    assert np.array_equal(layer.epd_off.cpu().numpy(), b["epd_off"])
+    tk = cfg.T * cfg.k
+    assert np.array_equal(layer.epd_sfd[:tk].cpu().numpy(), b["epd_sfd"])
+    assert np.array_equal(layer.epd_gate[:tk].cpu().numpy().astype(np.float64), b["epd_gate"])
+    per_rank, total, remote = oracle.count_dispatched(idx, slot_of, cfg.E, cfg.R)
+    assert np.array_equal(layer.per_rank.cpu().numpy(), per_rank)
+    assert int(layer.total.item()) == total == c_t
+    assert int(layer.remote.item()) == remote
+    return b
+
+
+def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=None):
+    inp = inputs.make_inputs(cfg, seed=seed)
+    if slot_of is None:
+        slot_of = np.arange(cfg.E, dtype=np.int32)
+    layer = make_layer(cfg, inp, torch.from_numpy(slot_of), ffn_kind)
+    logits, x = inp["logits"].to(DEV), inp["x"].to(DEV)
+    layer.hist.zero_()
+    y = layer.forward(logits, x)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    idx_ref, w_ref = oracle_route(inp["logits"], cfg.k, cfg.renorm)
+    b = check_indices(layer, idx_ref, w_ref, cfg, slot_of)
+    assert np.array_equal(layer.hist.cpu().numpy().astype(np.uint32),
+                          oracle.coact_histogram(idx_ref, cfg.E))
+    # dispatch: bit-exact copies
+    c_t = b["c_t"]
+    xo = to_oracle(inp["x"])
+    x_sfd_ref = oracle.gather_rows(xo, b["sfd_token"])
+    assert np.array_equal(to_oracle(layer.x_sfd[:c_t]), x_sfd_ref)
+    assert np.array_equal(to_oracle(layer.x_epd[:cfg.T * cfg.k]),
+                          oracle.gather_rows(x_sfd_ref, b["epd_sfd"]))
+    # outputs against the BRIM-guided oracle and against the dense definition
+    kind = oracle.KIND_IDENTITY if ffn_kind == moe.MOE_FFN_IDENTITY else oracle.KIND_SWIGLU
+    w_ = (None, None, None) if kind == oracle.KIND_IDENTITY else \
+        (to_oracle(inp["wg"]), to_oracle(inp["wu"]), to_oracle(inp["wd"]))
+    shared = None
+    if cfg.S and kind == oracle.KIND_SWIGLU:
+        shared = (to_oracle(inp["sg"]), to_oracle(inp["su"]), to_oracle(inp["sd"]))
+    b64 = oracle.brim(idx_ref, w_ref, slot_of, cfg.E, cfg.R)
+    y_sfd_ref, y_ref = oracle.occult_layer(xo, slot_of, cfg.E, cfg.R, cfg.k, b64, *w_,
+                                           kind=kind, shared=shared)
+    y_dense = oracle.dense_layer(xo, idx_ref, w_ref, *w_, kind=kind, shared=shared)
+    assert rowwise_rel_err(y_ref, y_dense) < 1e-10
+    err_y = rowwise_rel_err(y.float().cpu().numpy(), y_ref)
+    assert err_y <= OUT_RTOL, err_y
+    # y_sfd rows: compare only where the oracle's return row is not all ~0
+    # (rank rows whose routed sum cancels are compared against the row scale of y)
+    ys = layer.y_sfd[:c_t].float().cpu().numpy()
+    tok = b["sfd_token"]
+    scale = np.maximum(np.abs(y_ref[tok]).max(1), np.abs(y_sfd_ref).max(1))
+    err_sfd = (np.abs(ys - y_sfd_ref).max(1) / np.maximum(scale, 1e-30)).max()
+    assert err_sfd <= OUT_RTOL, err_sfd
+    return layer, err_y
+
+
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("renorm", [0, 1])
+def test_tiny_layer(dtype, renorm):
+    cfg = inputs.CONFIGS["tiny"].with_(dtype=dtype, renorm=renorm)
+    run_and_check_small(cfg)
+
+
+def test_tiny_layer_permuted_placement():
+    cfg = inputs.CONFIGS["tiny"]
+    slot_of = np.random.default_rng(3).permutation(cfg.E).astype(np.int32)
+    run_and_check_small(cfg, slot_of)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_identity_experts(dtype):
+    cfg = inputs.CONFIGS["tiny"].with_(dtype=dtype, T=300)
+    run_and_check_small(cfg, ffn_kind=moe.MOE_FFN_IDENTITY)
+
+
+@pytest.mark.parametrize("cfg", [
+    # several M tiles per expert, ragged tails, BN=128 for GEMM 1 (2f % 256 != 0)
+    inputs.LayerConfig("multi", T=1000, d=256, f=192, E=16, k=4, R=4, seed=5),
+    # d % 256 != 0 (BN=128 in GEMM 2) and shared experts
+    inputs.LayerConfig("shared", T=777, d=384, f=256, E=8, k=2, R=2, S=2, fs=128, seed=6),
+    # d = 192 (BN=64 in GEMM 2), one expert per rank
+    inputs.LayerConfig("narrow", T=515, d=192, f=128, E=8, k=3, R=8, seed=7),
+    # fp32 / TF32 with several tiles
+    inputs.LayerConfig("f32", T=600, d=256, f=256, E=8, k=2, R=4, dtype="f32", seed=8),
+    # biased routing (empty and overfull experts)
+    inputs.LayerConfig("skew", T=900, d=128, f=128, E=32, k=4, R=8, bias_std=2.0, seed=9),
+])
+def test_multi_tile_layers(cfg):
+    run_and_check_small(cfg)
+
+
+@pytest.mark.parametrize("T,E,k,R", [(1, 8, 2, 4), (2, 64, 6, 8), (257, 8, 2, 1),
+                                     (300, 8, 2, 8), (100, 256, 16, 8), (513, 64, 8, 64)])
+def test_edge_shapes(T, E, k, R):
+    cfg = inputs.LayerConfig("edge", T=T, d=128, f=128, E=E, k=k, R=R, seed=T)
+    run_and_check_small(cfg)
+
+
+def test_all_tokens_to_one_expert_group():
+    # every token's logits favour experts 0..k-1: one overfull group per expert, the rest empty
+    cfg = inputs.LayerConfig("one", T=400, d=128, f=128, E=16, k=2, R=4, seed=2)
+    inp = inputs.make_inputs(cfg)
+    inp["logits"][:, :2] += 100.0
+    layer = make_layer(cfg, inp)
+    y = layer.forward(inp["logits"].to(DEV), inp["x"].to(DEV))
+    torch.cuda.synchronize()
+    idx_ref, w_ref = oracle_route(inp["logits"], cfg.k, 0)
+    check_indices(layer, idx_ref, w_ref, cfg, np.arange(cfg.E, dtype=np.int32))
+    y_ref = oracle.dense_layer(to_oracle(inp["x"]), idx_ref, w_ref, to_oracle(inp["wg"]),
+                               to_oracle(inp["wu"]), to_oracle(inp["wd"]))
+    assert rowwise_rel_err(y.float().cpu().numpy(), y_ref) <= OUT_RTOL
+
+
+def test_empty_batch():
+    cfg = inputs.LayerConfig("empty", T=0, d=128, f=128, E=8, k=2, R=4)
+    inp = inputs.make_inputs(cfg)
+    layer = make_layer(cfg, inp)
+    layer.forward(inp["logits"].to(DEV), inp["x"].to(DEV))
+    torch.cuda.synchronize()
+    assert int(layer.c_t.item()) == 0
+    assert layer.sfd_off.cpu().tolist() == [0] * 5
+    assert moe.moe_get_device_status() == moe.MOE_OK
+
+
+def test_expert_ffn_ragged_groups():
+    """The grouped GEMM alone on hand-made groups: empty, 1 row, tile +/- 1, several tiles."""
+    torch.manual_seed(0)
+    d, f, G = 256, 192, 8
+    sizes = [0, 1, 127, 128, 129, 300, 0, 64]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    m = int(off[-1])
+    a = torch.randn(m + 5, d).to(torch.bfloat16)
+    wg = (torch.randn(G, f, d) * 0.05).to(torch.bfloat16)
+    wu = (torch.randn(G, f, d) * 0.05).to(torch.bfloat16)
+    wd = (torch.randn(G, d, f) * 0.05).to(torch.bfloat16)
+    scale = torch.rand(m + 5)
+    w_gu = torch.empty(G, 2 * f, d, dtype=torch.bfloat16, device=DEV)
+    w_dn = torch.empty(G, d, f, dtype=torch.bfloat16, device=DEV)
+    moe.moe_prepare_weights(wg.to(DEV), wu.to(DEV), wd.to(DEV), None, w_gu, w_dn)
+    out = torch.full((m + 5, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(moe.moe_expert_ffn_workspace_size(m + 5, f, moe.MOE_BF16), dtype=torch.uint8,
+                     device=DEV)
+    moe.moe_expert_ffn(a.to(DEV), torch.from_numpy(off).to(DEV), w_gu, w_dn, f, scale.to(DEV),
+                       moe.MOE_FFN_SWIGLU, out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    out = out.float().cpu().numpy()
+    ao, sc = a.double().numpy(), scale.double().numpy()
+    ref = np.zeros((m, d))
+    for g in range(G):
+        for r in range(off[g], off[g + 1]):
+            ref[r] = sc[r] * oracle.expert_row(ao[r], to_oracle(wg[g]), to_oracle(wu[g]),
+                                               to_oracle(wd[g]))
+    assert rowwise_rel_err(out[:m], ref) <= OUT_RTOL
+    assert np.all(out[m:] == 7.0)  # rows outside every group are not written
+
+
+def test_bad_expert_id_raises_device_check():
+    cfg = inputs.CONFIGS["tiny"]
+    idx = inputs.random_topk(cfg.T, cfg.E, cfg.k, seed=1).to(DEV)
+    idx[17, 1] = 99      # out of range
+    idx[40, 1] = idx[40, 0]  # repeated expert
+    layer = MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R,
+                     ffn_kind=moe.MOE_FFN_IDENTITY, device=DEV)
+    layer.topk_idx.copy_(idx)
+    layer.topk_w.fill_(0.5)
+    layer.build_brims()
+    assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
+    assert moe.moe_get_device_status() == moe.MOE_OK  # reading clears it
+    # the bad tokens are not sent anywhere; everything else is intact
+    b0 = layer.brim0.cpu().numpy()
+    assert np.all(b0[:, 17] == -1) and np.all(b0[:, 40] == -1)
+
+
+def test_outputs_are_deterministic():
+    cfg = inputs.LayerConfig("det", T=700, d=256, f=256, E=16, k=4, R=4, seed=4)
+    inp = inputs.make_inputs(cfg)
+    layer = make_layer(cfg, inp)
+    logits, x = inp["logits"].to(DEV), inp["x"].to(DEV)
+    y1 = layer.forward(logits, x).clone()
+    s1 = layer.y_sfd.clone()
+    y2 = layer.forward(logits, x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(s1, layer.y_sfd)
