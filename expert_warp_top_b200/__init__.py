@@ -7,7 +7,7 @@ The CUDA library is loaded on first use; without it every call raises.
 from ._binding import (  # noqa: F401
     EXPORTS, MOE_BF16, MOE_F32, MOE_FFN_IDENTITY, MOE_FFN_SWIGLU, MOE_OK, MOE_ERR_CUDA,
     MOE_ERR_DEVICE_CHECK, MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MoeError,
-    dtype_code, lib_path, load, moe_abi_version, moe_brim_build, moe_brim_workspace_size,
+    dtype_code, lib_path, load, moe_abi_version, moe_brim_build, moe_brim_build_noalloc, moe_brim_workspace_size,
     moe_coact_histogram, moe_combine_scatter, moe_count_dispatched_rows, moe_dispatch_gather,
     moe_expert_ffn, moe_expert_ffn_workspace_size, moe_get_device_status,
     moe_prepare_shared_weights, moe_prepare_weights, moe_route_topk, moe_set_debug,

@@ -29,7 +29,8 @@ MOE_FFN_SWIGLU, MOE_FFN_IDENTITY = 0, 1
 # every symbol the header declares (checked by the ABI test)
 EXPORTS = (
     "moe_abi_version", "moe_last_error", "moe_set_debug", "moe_get_device_status",
-    "moe_route_topk", "moe_brim_workspace_size", "moe_brim_build", "moe_dispatch_gather",
+    "moe_route_topk", "moe_brim_workspace_size", "moe_brim_build", "moe_brim_build_noalloc",
+    "moe_dispatch_gather",
     "moe_prepare_weights", "moe_prepare_shared_weights", "moe_expert_ffn_workspace_size",
     "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
 )
@@ -133,6 +134,17 @@ def moe_brim_build(topk_idx, topk_w, slot_of, E, R, brim0, sfd_token, sfd_off, b
         _ptr(brim1, I32, "brim1"), _ptr(epd_off, I32, "epd_off"), _ptr(epd_sfd, I32, "epd_sfd"),
         _ptr(epd_gate, F32, "epd_gate"), _ptr(c_t, I32, "c_t"),
         _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
+
+
+def moe_brim_build_noalloc(topk_idx, topk_w, slot_of, E, R, brim0, sfd_token, sfd_off, brim1,
+                           epd_off, epd_sfd, epd_gate, c_t, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_brim_build_noalloc", load().moe_brim_build_noalloc(
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"), T, k,
+        _ptr(slot_of, I32, "slot_of"), int(E), int(R),
+        _ptr(brim0, I32, "brim0"), _ptr(sfd_token, I32, "sfd_token"), _ptr(sfd_off, I32, "sfd_off"),
+        _ptr(brim1, I32, "brim1"), _ptr(epd_off, I32, "epd_off"), _ptr(epd_sfd, I32, "epd_sfd"),
+        _ptr(epd_gate, F32, "epd_gate"), _ptr(c_t, I32, "c_t"), _stream(stream)))
 
 
 def moe_dispatch_gather(x, k, R, L, brim0, brim1, x_sfd, x_epd, stream=None):

@@ -19,6 +19,11 @@
 // The device error flag the kernels raise (bits moe::kErrIndex, kErrTimeout).
 __device__ unsigned g_moe_err_flag;
 
+// Fixed scratch of moe_brim_build_noalloc (1 MiB, held by every GPU that loads
+// this library until the process exits).
+constexpr size_t kNoAllocScratchInts = size_t(1) << 18;
+static __device__ __align__(256) int32_t g_brim_noalloc_scratch[kNoAllocScratchInts];
+
 namespace {
 
 thread_local char g_msg[512];
@@ -82,6 +87,28 @@ int device_info(DeviceInfo** out) {
     di.ready = true;
   }
   *out = &di;
+  return MOE_OK;
+}
+
+// Device address of g_brim_noalloc_scratch on the current device.  The
+// array's name in host code is only a host-side stand-in, so the address is
+// looked up with cudaGetSymbolAddress, once per device, with that device
+// current, and cached.
+int32_t* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  MOE_REQUIRE(dev >= 0 && dev < kMaxDevices, MOE_ERR_UNSUPPORTED, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, g_brim_noalloc_scratch));
+    MOE_REQUIRE(p != nullptr, MOE_ERR_CUDA, "no device address for the fixed scratch array");
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
   return MOE_OK;
 }
 
@@ -285,6 +312,50 @@ int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
   MOE_LAUNCHED("brim_scan_kernel");
   moe::brim_scatter_kernel<<<n_tiles, moe::kBrimTile, 0, stream>>>(
       topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, counts, brim0, sfd_token, brim1, epd_sfd,
+      epd_gate, di->err_flag);
+  MOE_LAUNCHED("brim_scatter_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// moe_brim_build_noalloc: the BRIM build for callers that cannot allocate
+// device memory or lend a workspace (see the header).  Its scratch is a fixed
+// file-scope device array; host code only ever uses the device address that
+// cudaGetSymbolAddress returns for it, looked up once per device.
+int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                           const int32_t* slot_of, int E, int R, int32_t* brim0,
+                           int32_t* sfd_token, int32_t* sfd_off, int32_t* brim1,
+                           int32_t* epd_off, int32_t* epd_sfd, float* epd_gate, int32_t* c_t,
+                           moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  MOE_REQUIRE(slot_of && sfd_off && epd_off && c_t, MOE_ERR_INVALID_ARG, "null pointer");
+  const size_t n_tiles = ((size_t)T + moe::kBrimTile - 1) / moe::kBrimTile;
+  const size_t need = n_tiles * (size_t)(R + E);
+  MOE_REQUIRE(need <= kNoAllocScratchInts, MOE_ERR_UNSUPPORTED,
+              "moe_brim_build_noalloc: T=%d, R=%d, E=%d needs %zu scratch entries, more than "
+              "its fixed %zu (1 MiB); use moe_brim_build with a workspace",
+              T, R, E, need, kNoAllocScratchInts);
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  int32_t* counts = nullptr;
+  if ((rc = noalloc_scratch(&counts))) return rc;
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(sfd_off, 0, sizeof(int32_t) * (R + 1), stream));
+    MOE_CUDA(cudaMemsetAsync(epd_off, 0, sizeof(int32_t) * (E + 1), stream));
+    MOE_CUDA(cudaMemsetAsync(c_t, 0, sizeof(int32_t), stream));
+    return MOE_OK;
+  }
+  MOE_REQUIRE(topk_idx && topk_w && brim0 && sfd_token && brim1 && epd_sfd && epd_gate,
+              MOE_ERR_INVALID_ARG, "null pointer");
+  const int nt = (int)n_tiles;
+  moe::brim_count_kernel<<<nt, moe::kBrimTile, 0, stream>>>(topk_idx, slot_of, T, k, E, R, nt,
+                                                            counts, di->err_flag);
+  MOE_LAUNCHED("brim_count_kernel");
+  moe::brim_scan_kernel<<<1, 1024, 0, stream>>>(counts, nt, E, R, sfd_off, epd_off, c_t);
+  MOE_LAUNCHED("brim_scan_kernel");
+  moe::brim_scatter_kernel<<<nt, moe::kBrimTile, 0, stream>>>(
+      topk_idx, topk_w, slot_of, T, k, E, R, nt, counts, brim0, sfd_token, brim1, epd_sfd,
       epd_gate, di->err_flag);
   MOE_LAUNCHED("brim_scatter_kernel");
   return MOE_OK;

@@ -135,6 +135,35 @@ int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
                    void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_brim_build_noalloc -- the same BRIM build as moe_brim_build, for callers
+ * that must not allocate device memory at all.  It has no counterpart in the
+ * paper; it exists for the host side of this library.
+ * Who needs it: code embedded in a host framework that owns every byte of
+ * device memory through its own pool (a raw cudaMalloc would bypass that
+ * pool's accounting and limits), and code on a latency-critical path where
+ * cudaMalloc / cudaFree are off limits because they can synchronise the
+ * device and stall unrelated streams.  Such callers may also have no
+ * workspace to lend, so this entry point takes none.
+ * Scratch: a fixed array of 1 MiB (262144 int32) in this library's device
+ * memory, reserved on every GPU that loads the library until the process
+ * exits.  A call needs ceil(T / 256) * (R + E) entries of it; a larger call
+ * returns MOE_ERR_UNSUPPORTED and enqueues nothing.  The passes overwrite
+ * every scratch entry they read, so nothing has to be cleared between calls.
+ * All calls on a device share the one array: calls that may run on the GPU at
+ * the same time (e.g. on two streams without ordering) race on it and must be
+ * serialised by the caller.
+ * Set-up: the first call on each device looks up the array's device address
+ * with that device current; make that first call before any stream capture.
+ * The call allocates nothing: no cudaMalloc, no cudaFree.
+ * Arguments and outputs are those of moe_brim_build, without ws / ws_bytes.
+ * ------------------------------------------------------------------------- */
+int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                           const int32_t* slot_of, int E, int R,
+                           int32_t* brim0, int32_t* sfd_token, int32_t* sfd_off,
+                           int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                           float* epd_gate, int32_t* c_t, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_dispatch_gather -- ORI -> SFD -> EPD (Occult paper, Figure 4), guided by
  * the BRIMs: for every token t and rank r with s = BRIM_0[r][t] >= 0,
  *   x_sfd[s] = x[t]                         (the simulated all-to-all payload)
