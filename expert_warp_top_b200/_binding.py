@@ -175,11 +175,17 @@ def moe_expert_ffn_workspace_size(m_cap, f, dtype_code_) -> int:
     return int(load().moe_expert_ffn_workspace_size(int(m_cap), int(f), int(dtype_code_)))
 
 
-def moe_expert_ffn(a, group_off, w_gu, w_dn, f, row_scale, ffn_kind, out, ws, stream=None):
-    m_cap, d = a.shape
+def moe_expert_ffn(a, group_off, w_gu, w_dn, f, row_scale, ffn_kind, out, ws, stream=None,
+                   a_row_index=None, m_cap=None):
+    """out = row_scale * FFN_g(rows) per group; rows are a[a_row_index[p]] when a
+    row index is given (m_cap = its length), else a[p] (m_cap = rows of a)."""
+    a_rows, d = a.shape
+    if m_cap is None:
+        m_cap = a_row_index.numel() if a_row_index is not None else a_rows
     G = group_off.numel() - 1
     _check("moe_expert_ffn", load().moe_expert_ffn(
-        _ptr(a, _ACT, "a"), _ptr(group_off, I32, "group_off"), G, m_cap,
+        _ptr(a, _ACT, "a"), int(a_rows), _ptr(a_row_index, I32, "a_row_index"),
+        _ptr(group_off, I32, "group_off"), G, int(m_cap),
         _ptr(w_gu, a.dtype, "w_gu"), _ptr(w_dn, a.dtype, "w_dn"), d, int(f), dtype_code(a.dtype),
         _ptr(row_scale, F32, "row_scale"), int(ffn_kind), _ptr(out, a.dtype, "out"),
         _ptr(ws, None, "ws"), ctypes.c_size_t(0 if ws is None else ws.numel() * ws.element_size()),

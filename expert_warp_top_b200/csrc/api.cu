@@ -183,18 +183,22 @@ int check_dtype(int dtype) {
 int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
 
 // ---- GEMM launch ----------------------------------------------------------
-template <int BN, int EPI, bool TF32>
-int launch_gemm(DeviceInfo* di, unsigned attr_bit, const void* a, int m_cap, int K,
-                const void* b, int G, int N, const int32_t* group_off, const float* row_scale,
-                void* out, int ldo, cudaStream_t st) {
+// A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
+// gathered from it (row p = a[a_row_index[p]]), else they are a's first m_cap.
+template <int BN, int EPI, bool TF32, bool GATHER>
+int launch_gemm(DeviceInfo* di, unsigned attr_bit, const void* a, int a_rows,
+                const int32_t* a_row_index, int m_cap, int K, const void* b, int G, int N,
+                const int32_t* group_off, const float* row_scale, void* out, int ldo,
+                cudaStream_t st) {
   using Cfg = moe::GemmCfg<BN, TF32>;
   const int dtype = TF32 ? MOE_F32 : MOE_BF16;
   CUtensorMap ta, tb;
-  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)m_cap, Cfg::kBK, moe::kGemmBM);
+  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK,
+                     GATHER ? 1u : (uint32_t)moe::kGemmBM);
   if (rc) return rc;
   rc = encode_2d(&tb, b, dtype, (uint64_t)K, (uint64_t)G * N, Cfg::kBK, BN);
   if (rc) return rc;
-  auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32>;
+  auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32, GATHER>;
   if (!(di->smem_attr_done & attr_bit)) {
     MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)Cfg::kSmemBytes));
@@ -202,31 +206,85 @@ int launch_gemm(DeviceInfo* di, unsigned attr_bit, const void* a, int m_cap, int
   }
   const long long ub = ((long long)m_cap / moe::kGemmBM + G) * (N / BN);
   const int grid = (int)(ub < di->num_sms ? (ub < 1 ? 1 : ub) : di->num_sms);
-  moe::GemmArgs args{group_off, G, N, K, m_cap, row_scale, out, ldo, di->err_flag,
-                     wait_limit_ns(), g_debug_flags};
+  moe::GemmArgs args{group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo,
+                     di->err_flag, wait_limit_ns(), g_debug_flags};
   kern<<<grid, moe::kGemmThreads, Cfg::kSmemBytes, st>>>(ta, tb, args);
   MOE_LAUNCHED("ffn_gemm_kernel");
   return MOE_OK;
 }
 
-template <int EPI, bool TF32>
-int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int m_cap, int K, const void* b, int G,
-                   int N, const int32_t* group_off, const float* row_scale, void* out, int ldo,
-                   cudaStream_t st) {
-  const unsigned base = (EPI * 2 + (TF32 ? 1 : 0)) * 3;
+template <int EPI, bool TF32, bool GATHER>
+int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int a_rows, const int32_t* a_row_index,
+                   int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
+                   const float* row_scale, void* out, int ldo, cudaStream_t st) {
+  const unsigned base = ((EPI * 2 + (TF32 ? 1 : 0)) * 2 + (GATHER ? 1 : 0)) * 3;
   if (bn == 256)
-    return launch_gemm<256, EPI, TF32>(di, 1u << (base + 0), a, m_cap, K, b, G, N, group_off,
-                                       row_scale, out, ldo, st);
+    return launch_gemm<256, EPI, TF32, GATHER>(di, 1u << (base + 0), a, a_rows, a_row_index,
+                                               m_cap, K, b, G, N, group_off, row_scale, out, ldo,
+                                               st);
   if (bn == 128)
-    return launch_gemm<128, EPI, TF32>(di, 1u << (base + 1), a, m_cap, K, b, G, N, group_off,
-                                       row_scale, out, ldo, st);
-  return launch_gemm<64, EPI, TF32>(di, 1u << (base + 2), a, m_cap, K, b, G, N, group_off,
-                                    row_scale, out, ldo, st);
+    return launch_gemm<128, EPI, TF32, GATHER>(di, 1u << (base + 1), a, a_rows, a_row_index,
+                                               m_cap, K, b, G, N, group_off, row_scale, out, ldo,
+                                               st);
+  return launch_gemm<64, EPI, TF32, GATHER>(di, 1u << (base + 2), a, a_rows, a_row_index, m_cap,
+                                            K, b, G, N, group_off, row_scale, out, ldo, st);
+}
+
+// How many warps share one token row in the movers: one warp per token when
+// the batch fills the GPU (>= 32 warps per SM), more for small batches.
+int mover_parts(const DeviceInfo* di, int T, int max_parts) {
+  const long long want = (long long)di->num_sms * 32;
+  int P = (int)((want + T - 1) / (T > 0 ? T : 1));
+  if (P > max_parts) P = max_parts;
+  return P < 1 ? 1 : P;
 }
 
 int pick_bn(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The BRIM passes, compiled for a bound KMAX >= k so per-token state stays in
+// registers.
+template <int KMAX>
+int launch_brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                       const int32_t* slot_of, int E, int R, int32_t* brim0, int32_t* sfd_token,
+                       int32_t* sfd_off, int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                       float* epd_gate, int32_t* c_t, uint32_t* scratch, unsigned* err,
+                       cudaStream_t stream) {
+  const int n_tiles = (T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
+  const int blocks = (n_tiles + 3) / 4;
+  moe::brim_mask_kernel<KMAX><<<blocks, 128, 0, stream>>>(topk_idx, slot_of, T, k, E, R, n_tiles,
+                                                          scratch, err);
+  MOE_LAUNCHED("brim_mask_kernel");
+  moe::brim_scan_kernel<<<1, 1024, 0, stream>>>(scratch, n_tiles, E, R, sfd_off, epd_off, c_t);
+  MOE_LAUNCHED("brim_scan_kernel");
+  moe::brim_scatter_kernel<KMAX><<<blocks, 128, 0, stream>>>(
+      topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, reinterpret_cast<const int32_t*>(scratch),
+      brim0, sfd_token, brim1, epd_sfd, epd_gate);
+  MOE_LAUNCHED("brim_scatter_kernel");
+  return MOE_OK;
+}
+
+int brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int k, const int32_t* slot_of,
+                int E, int R, int32_t* brim0, int32_t* sfd_token, int32_t* sfd_off, int32_t* brim1,
+                int32_t* epd_off, int32_t* epd_sfd, float* epd_gate, int32_t* c_t,
+                uint32_t* scratch, unsigned* err, cudaStream_t stream) {
+#define MOE_BRIM_K(KM)                                                                        \
+  return launch_brim_passes<KM>(topk_idx, topk_w, T, k, slot_of, E, R, brim0, sfd_token,      \
+                                sfd_off, brim1, epd_off, epd_sfd, epd_gate, c_t, scratch, err, \
+                                stream)
+  if (k <= 2) MOE_BRIM_K(2);
+  if (k <= 4) MOE_BRIM_K(4);
+  if (k <= 8) MOE_BRIM_K(8);
+  MOE_BRIM_K(16);
+#undef MOE_BRIM_K
+}
+
+// Scratch entries (one 32-bit word per column per 32-token tile) of a BRIM build.
+size_t brim_scratch_entries(int T, int E, int R) {
+  const size_t n_tiles = ((size_t)T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
+  return n_tiles * (size_t)(R + E);
+}
 
 }  // namespace
 
@@ -279,8 +337,7 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t
 // ---------------------------------------------------------------------------
 size_t moe_brim_workspace_size(int T, int E, int R) {
   if (T < 0 || E < 1 || R < 1) return 0;
-  const size_t n_tiles = (size_t)(T + moe::kBrimTile - 1) / moe::kBrimTile;
-  return align256(sizeof(int32_t) * n_tiles * (size_t)(R + E)) + 256;
+  return align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)) + 256;
 }
 
 int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
@@ -303,17 +360,9 @@ int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
               MOE_ERR_INVALID_ARG, "null pointer");
   MOE_REQUIRE(ws_bytes >= moe_brim_workspace_size(T, E, R), MOE_ERR_INVALID_ARG,
               "workspace too small: %zu < %zu bytes", ws_bytes, moe_brim_workspace_size(T, E, R));
-  const int n_tiles = (T + moe::kBrimTile - 1) / moe::kBrimTile;
-  int32_t* counts = static_cast<int32_t*>(ws);
-  moe::brim_count_kernel<<<n_tiles, moe::kBrimTile, 0, stream>>>(topk_idx, slot_of, T, k, E, R,
-                                                                 n_tiles, counts, di->err_flag);
-  MOE_LAUNCHED("brim_count_kernel");
-  moe::brim_scan_kernel<<<1, 1024, 0, stream>>>(counts, n_tiles, E, R, sfd_off, epd_off, c_t);
-  MOE_LAUNCHED("brim_scan_kernel");
-  moe::brim_scatter_kernel<<<n_tiles, moe::kBrimTile, 0, stream>>>(
-      topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, counts, brim0, sfd_token, brim1, epd_sfd,
-      epd_gate, di->err_flag);
-  MOE_LAUNCHED("brim_scatter_kernel");
+  return brim_passes(topk_idx, topk_w, T, k, slot_of, E, R, brim0, sfd_token, sfd_off, brim1,
+                     epd_off, epd_sfd, epd_gate, c_t, static_cast<uint32_t*>(ws), di->err_flag,
+                     stream);
   return MOE_OK;
 }
 
@@ -330,8 +379,7 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
   int rc = check_common(T, E, k, R);
   if (rc) return rc;
   MOE_REQUIRE(slot_of && sfd_off && epd_off && c_t, MOE_ERR_INVALID_ARG, "null pointer");
-  const size_t n_tiles = ((size_t)T + moe::kBrimTile - 1) / moe::kBrimTile;
-  const size_t need = n_tiles * (size_t)(R + E);
+  const size_t need = brim_scratch_entries(T, E, R);
   MOE_REQUIRE(need <= kNoAllocScratchInts, MOE_ERR_UNSUPPORTED,
               "moe_brim_build_noalloc: T=%d, R=%d, E=%d needs %zu scratch entries, more than "
               "its fixed %zu (1 MiB); use moe_brim_build with a workspace",
@@ -348,16 +396,9 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
   }
   MOE_REQUIRE(topk_idx && topk_w && brim0 && sfd_token && brim1 && epd_sfd && epd_gate,
               MOE_ERR_INVALID_ARG, "null pointer");
-  const int nt = (int)n_tiles;
-  moe::brim_count_kernel<<<nt, moe::kBrimTile, 0, stream>>>(topk_idx, slot_of, T, k, E, R, nt,
-                                                            counts, di->err_flag);
-  MOE_LAUNCHED("brim_count_kernel");
-  moe::brim_scan_kernel<<<1, 1024, 0, stream>>>(counts, nt, E, R, sfd_off, epd_off, c_t);
-  MOE_LAUNCHED("brim_scan_kernel");
-  moe::brim_scatter_kernel<<<nt, moe::kBrimTile, 0, stream>>>(
-      topk_idx, topk_w, slot_of, T, k, E, R, nt, counts, brim0, sfd_token, brim1, epd_sfd,
-      epd_gate, di->err_flag);
-  MOE_LAUNCHED("brim_scatter_kernel");
+  return brim_passes(topk_idx, topk_w, T, k, slot_of, E, R, brim0, sfd_token, sfd_off, brim1,
+                     epd_off, epd_sfd, epd_gate, c_t, reinterpret_cast<uint32_t*>(counts),
+                     di->err_flag, stream);
   return MOE_OK;
 }
 
@@ -377,9 +418,13 @@ int moe_dispatch_gather(const void* x, int T, int d, int dtype, int k, int R, in
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
   const size_t cap = (size_t)T * (k < R ? k : R);
-  const int blocks = (T + moe::kMoverWarps - 1) / moe::kMoverWarps;
-  moe::dispatch_kernel<<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
-      static_cast<const uint8_t*>(x), T, d * esize(dtype), R, L, cap, T * k, brim0, brim1,
+  constexpr int CH = 4;  // 512-byte chunks in flight per warp
+  const int row_bytes = d * esize(dtype);
+  const int P = mover_parts(di, T, (row_bytes + CH * 512 - 1) / (CH * 512));
+  const long long warps = (long long)T * P;
+  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
+  moe::dispatch_kernel<CH><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
+      static_cast<const uint8_t*>(x), T, row_bytes, P, R, L, cap, T * k, brim0, brim1,
       static_cast<uint8_t*>(x_sfd), static_cast<uint8_t*>(x_epd), di->err_flag);
   MOE_LAUNCHED("dispatch_kernel");
   return MOE_OK;
@@ -401,19 +446,27 @@ int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
   const size_t cap = (size_t)T * (k < R ? k : R);
-  const int blocks = (T + moe::kMoverWarps - 1) / moe::kMoverWarps;
+  const int P = mover_parts(di, T, (d * esize(dtype) + 511) / 512);
+  const long long warps = (long long)T * P;
+  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
+#define MOE_COMBINE(TA, KM)                                                                    \
+  moe::combine_kernel<TA, KM><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(                   \
+      static_cast<const TA*>(o_epd), T, d, P, R, L, cap, T * k, brim0, brim1,                  \
+      static_cast<const TA*>(shared_out), static_cast<TA*>(y_sfd), static_cast<TA*>(y),        \
+      di->err_flag)
   if (dtype == MOE_BF16) {
     using B = __nv_bfloat16;
-    moe::combine_kernel<B><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
-        static_cast<const B*>(o_epd), T, d, R, L, cap, T * k, brim0, brim1,
-        static_cast<const B*>(shared_out), static_cast<B*>(y_sfd), static_cast<B*>(y),
-        di->err_flag);
+    if (k <= 2) MOE_COMBINE(B, 2);
+    else if (k <= 4) MOE_COMBINE(B, 4);
+    else if (k <= 8) MOE_COMBINE(B, 8);
+    else MOE_COMBINE(B, 16);
   } else {
-    moe::combine_kernel<float><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
-        static_cast<const float*>(o_epd), T, d, R, L, cap, T * k, brim0, brim1,
-        static_cast<const float*>(shared_out), static_cast<float*>(y_sfd),
-        static_cast<float*>(y), di->err_flag);
+    if (k <= 2) MOE_COMBINE(float, 2);
+    else if (k <= 4) MOE_COMBINE(float, 4);
+    else if (k <= 8) MOE_COMBINE(float, 8);
+    else MOE_COMBINE(float, 16);
   }
+#undef MOE_COMBINE
   MOE_LAUNCHED("combine_kernel");
   return MOE_OK;
 }
@@ -473,7 +526,8 @@ size_t moe_expert_ffn_workspace_size(int m_cap, int f, int dtype) {
   return align256((size_t)m_cap * f * (dtype == MOE_BF16 ? 2 : 4)) + 256;
 }
 
-int moe_expert_ffn(const void* a, const int32_t* group_off, int G, int m_cap, const void* w_gu,
+int moe_expert_ffn(const void* a, int a_rows, const int32_t* a_row_index,
+                   const int32_t* group_off, int G, int m_cap, const void* w_gu,
                    const void* w_dn, int d, int f, int dtype, const float* row_scale,
                    int ffn_kind, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
   int rc = check_dtype(dtype);
@@ -482,14 +536,19 @@ int moe_expert_ffn(const void* a, const int32_t* group_off, int G, int m_cap, co
               "unknown ffn_kind %d", ffn_kind);
   MOE_REQUIRE(G >= 1 && G <= moe::kGemmMaxGroups, MOE_ERR_UNSUPPORTED,
               "G must be in [1, %d] (got %d)", moe::kGemmMaxGroups, G);
-  MOE_REQUIRE(m_cap >= 0, MOE_ERR_INVALID_ARG, "m_cap must be >= 0");
+  MOE_REQUIRE(m_cap >= 0 && a_rows >= 0, MOE_ERR_INVALID_ARG, "m_cap and a_rows must be >= 0");
+  MOE_REQUIRE(a_row_index || a_rows >= m_cap, MOE_ERR_INVALID_ARG,
+              "without a row index, a needs at least m_cap rows (a_rows=%d m_cap=%d)", a_rows,
+              m_cap);
   MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
   if (m_cap == 0) return MOE_OK;
-  MOE_REQUIRE(a && group_off && out, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(a && group_off && out && a_rows > 0, MOE_ERR_INVALID_ARG, "null pointer or empty a");
   MOE_REQUIRE(aligned16(a) && aligned16(out), MOE_ERR_INVALID_ARG, "a and out must be 16-byte aligned");
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
   if (ffn_kind == MOE_FFN_IDENTITY) {
+    MOE_REQUIRE(a_row_index == nullptr, MOE_ERR_UNSUPPORTED,
+                "the identity expert takes its rows in place (no row index)");
     const int grid = di->num_sms * 8;
     if (dtype == MOE_BF16)
       moe::identity_expert_kernel<__nv_bfloat16><<<grid, moe::kMoverWarps * 32, 0, stream>>>(
@@ -511,17 +570,27 @@ int moe_expert_ffn(const void* a, const int32_t* group_off, int G, int m_cap, co
   void* h = ws;  // [m_cap, f]
   const int bn1 = pick_bn(2 * f), bn2 = pick_bn(d);
   if (dtype == MOE_BF16) {
-    rc = launch_gemm_bn<moe::kEpiSwiGLU, false>(di, bn1 < 128 ? 128 : bn1, a, m_cap, d, w_gu, G,
-                                                2 * f, group_off, nullptr, h, f, stream);
+    rc = a_row_index
+             ? launch_gemm_bn<moe::kEpiSwiGLU, false, true>(di, bn1, a, a_rows, a_row_index,
+                                                            m_cap, d, w_gu, G, 2 * f, group_off,
+                                                            nullptr, h, f, stream)
+             : launch_gemm_bn<moe::kEpiSwiGLU, false, false>(di, bn1, a, a_rows, nullptr, m_cap,
+                                                             d, w_gu, G, 2 * f, group_off,
+                                                             nullptr, h, f, stream);
     if (rc) return rc;
-    rc = launch_gemm_bn<moe::kEpiScale, false>(di, bn2, h, m_cap, f, w_dn, G, d, group_off,
-                                               row_scale, out, d, stream);
+    rc = launch_gemm_bn<moe::kEpiScale, false, false>(di, bn2, h, m_cap, nullptr, m_cap, f, w_dn,
+                                                      G, d, group_off, row_scale, out, d, stream);
   } else {
-    rc = launch_gemm_bn<moe::kEpiSwiGLU, true>(di, bn1 < 128 ? 128 : bn1, a, m_cap, d, w_gu, G,
-                                               2 * f, group_off, nullptr, h, f, stream);
+    rc = a_row_index
+             ? launch_gemm_bn<moe::kEpiSwiGLU, true, true>(di, bn1, a, a_rows, a_row_index,
+                                                           m_cap, d, w_gu, G, 2 * f, group_off,
+                                                           nullptr, h, f, stream)
+             : launch_gemm_bn<moe::kEpiSwiGLU, true, false>(di, bn1, a, a_rows, nullptr, m_cap,
+                                                            d, w_gu, G, 2 * f, group_off,
+                                                            nullptr, h, f, stream);
     if (rc) return rc;
-    rc = launch_gemm_bn<moe::kEpiScale, true>(di, bn2, h, m_cap, f, w_dn, G, d, group_off,
-                                              row_scale, out, d, stream);
+    rc = launch_gemm_bn<moe::kEpiScale, true, false>(di, bn2, h, m_cap, nullptr, m_cap, f, w_dn,
+                                                     G, d, group_off, row_scale, out, d, stream);
   }
   return rc;
 }
@@ -540,9 +609,23 @@ int moe_count_dispatched_rows(const int32_t* topk_idx, int T, int k, const int32
   MOE_CUDA(cudaMemsetAsync(remote, 0, sizeof(int64_t), stream));
   if (T == 0) return MOE_OK;
   MOE_REQUIRE(topk_idx, MOE_ERR_INVALID_ARG, "null pointer");
-  moe::count_dispatched_kernel<<<(T + 255) / 256, 256, 0, stream>>>(
-      topk_idx, T, k, slot_of, E, R, per_rank, reinterpret_cast<unsigned long long*>(total),
-      reinterpret_cast<unsigned long long*>(remote), di->err_flag);
+  {
+    auto* tot = reinterpret_cast<unsigned long long*>(total);
+    auto* rem = reinterpret_cast<unsigned long long*>(remote);
+    const int blocks = (T + 255) / 256;
+    if (k <= 2)
+      moe::count_dispatched_kernel<2><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
+                                                                  per_rank, tot, rem, di->err_flag);
+    else if (k <= 4)
+      moe::count_dispatched_kernel<4><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
+                                                                  per_rank, tot, rem, di->err_flag);
+    else if (k <= 8)
+      moe::count_dispatched_kernel<8><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
+                                                                  per_rank, tot, rem, di->err_flag);
+    else
+      moe::count_dispatched_kernel<16><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
+                                                                   per_rank, tot, rem, di->err_flag);
+  }
   MOE_LAUNCHED("count_dispatched_kernel");
   return MOE_OK;
 }
@@ -557,8 +640,17 @@ int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* 
   if (!accumulate) MOE_CUDA(cudaMemsetAsync(hist, 0, sizeof(uint32_t) * E * E, stream));
   if (T == 0) return MOE_OK;
   MOE_REQUIRE(topk_idx, MOE_ERR_INVALID_ARG, "null pointer");
-  moe::coact_hist_kernel<<<(T + 255) / 256, 256, 0, stream>>>(topk_idx, T, k, E, hist,
-                                                               di->err_flag);
+  {
+    const int blocks = (T + 255) / 256;
+    if (k <= 2)
+      moe::coact_hist_kernel<2><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+    else if (k <= 4)
+      moe::coact_hist_kernel<4><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+    else if (k <= 8)
+      moe::coact_hist_kernel<8><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+    else
+      moe::coact_hist_kernel<16><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+  }
   MOE_LAUNCHED("coact_hist_kernel");
   return MOE_OK;
 }

@@ -9,82 +9,111 @@
 // row count C_T is the all-to-all budget (Occult paper, TL;DR).
 //
 // Positions are stable (ascending token order inside every rank segment and
-// every expert group), which makes them unique.  They come from a three-pass
-// deterministic scan over tiles of 256 tokens:
-//   1. count   : per tile, how many tokens hit each rank and each slot
-//   2. scan    : exclusive scan of the tile counts per column, column totals
-//                -> sfd_off, epd_off, C_T, and each tile's global base
-//   3. scatter : inside a tile, a token's rank among the tile's tokens that hit
-//                the same column is the popcount of a per-warp lane mask plus
-//                the counts of the earlier warps; add the tile base, write.
+// every expert group), which makes them unique.  Tokens are taken in tiles of
+// 32, one warp per tile and one lane per token.  A "column" is a rank (c < R)
+// or an expert slot (c = R + q).
+//   1. mask    : per tile and column, the 32-bit mask of lanes that hit it
+//   2. scan    : per column, exclusive scan of popcount(mask) over the tiles;
+//                column totals give sfd_off, epd_off and C_T; the masks are
+//                replaced in place by each tile's first global row
+//   3. scatter : each lane rebuilds its tile's masks and finds its row in
+//                column c as base[c][tile] + popcount(mask_c & lanes below it)
+// No pass depends on the order in which atomics land.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kBrimTile = 256;     // tokens per tile (one per thread)
-constexpr int kBrimWarps = kBrimTile / 32;
+constexpr int kBrimTileTokens = 32;  // one warp
 constexpr int kMaxK = 16;
 constexpr int kMaxE = 256;
+constexpr int kMaxCols = 2 * kMaxE;
 
-// Gather one token's experts, slots and distinct ranks.  Returns false (and
-// raises the error flag) when an expert id is out of range or repeated.
+// One token's experts, as slots, with their ranks; `first[j]` marks the first
+// expert of each distinct rank.  KMAX is a compile-time bound on k so that
+// every array lives in registers.
+template <int KMAX>
 struct TokenRoute {
-  int n_rank;               // distinct ranks hit
-  int rank[kMaxK];          // the ranks, in order of first appearance
-  int slot[kMaxK];          // slot of each selected expert
+  int slot[KMAX];
+  int rank[KMAX];
+  bool first[KMAX];
 };
 
+// Loads token t's route.  Returns false (and raises the error flag) when an
+// expert id is out of range or repeated; such a token is sent nowhere.
+template <int KMAX>
 __device__ __forceinline__ bool load_token_route(const int32_t* __restrict__ topk_idx,
                                                  const int32_t* __restrict__ slot_of, int t,
-                                                 int k, int E, int L, TokenRoute& tr,
+                                                 int k, int E, int L, TokenRoute<KMAX>& tr,
                                                  unsigned* err) {
-  tr.n_rank = 0;
   bool ok = true;
-  for (int j = 0; j < k; ++j) {
-    int e = topk_idx[(size_t)t * k + j];
-    int q = -1;
-    if (e >= 0 && e < E) q = slot_of[e];
-    if (q < 0 || q >= E) {
-      ok = false;
-      tr.slot[j] = -1;
-      continue;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    tr.slot[j] = -1;
+    tr.rank[j] = -1;
+    if (j < k) {
+      const int e = __ldg(topk_idx + (size_t)t * k + j);
+      const int q = (e >= 0 && e < E) ? __ldg(slot_of + e) : -1;
+      if (q < 0 || q >= E) ok = false;
+      tr.slot[j] = q;
+      tr.rank[j] = q >= 0 ? q / L : -1;
     }
-    for (int i = 0; i < j; ++i)
-      if (tr.slot[i] == q) ok = false;  // the same expert twice
-    tr.slot[j] = q;
-    const int r = q / L;
-    bool seen = false;
-    for (int i = 0; i < tr.n_rank; ++i) seen |= (tr.rank[i] == r);
-    if (!seen) tr.rank[tr.n_rank++] = r;
   }
-  if (!ok) raise_error(err, kErrIndex);
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    bool first = j < k;
+#pragma unroll
+    for (int i = 0; i < j; ++i) {
+      if (j < k) {  // entries past k are padding and compare with nothing
+        if (tr.slot[i] == tr.slot[j]) ok = false;  // the same expert twice
+        if (tr.rank[i] == tr.rank[j]) first = false;
+      }
+    }
+    tr.first[j] = first;
+  }
+  if (!ok && err) raise_error(err, kErrIndex);
   return ok;
 }
 
-// ---- pass 1 ---------------------------------------------------------------
-// counts[c][tile] (column-major, so a column's tiles are contiguous):
-//   c < R      : tokens of the tile that hit rank c
-//   c = R + q  : tokens of the tile that selected the expert at slot q
-__global__ void __launch_bounds__(kBrimTile) brim_count_kernel(
-    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ slot_of, int T, int k,
-    int E, int R, int n_tiles, int32_t* __restrict__ counts, unsigned* err) {
-  __shared__ int32_t sc[kMaxE * 2];
-  const int ncol = R + E;
-  const int L = E / R;
-  for (int c = threadIdx.x; c < ncol; c += blockDim.x) sc[c] = 0;
-  __syncthreads();
-  const int t = blockIdx.x * kBrimTile + threadIdx.x;
-  if (t < T) {
-    TokenRoute tr;
-    if (load_token_route(topk_idx, slot_of, t, k, E, L, tr, err)) {
-      for (int i = 0; i < tr.n_rank; ++i) atomicAdd(&sc[tr.rank[i]], 1);
-      for (int j = 0; j < k; ++j) atomicAdd(&sc[R + tr.slot[j]], 1);
+// Build this warp's tile masks in shared memory (mask[c], ncol entries).
+template <int KMAX>
+__device__ __forceinline__ void tile_masks(uint32_t* mask, int ncol, int R, bool active, int k,
+                                           const TokenRoute<KMAX>& tr) {
+  const unsigned lane = lane_id();
+  for (int c = lane; c < ncol; c += 32) mask[c] = 0u;
+  __syncwarp();
+  if (active) {
+    const uint32_t bit = 1u << lane;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        atomicOr(&mask[R + tr.slot[j]], bit);
+        if (tr.first[j]) atomicOr(&mask[tr.rank[j]], bit);
+      }
     }
   }
-  __syncthreads();
-  for (int c = threadIdx.x; c < ncol; c += blockDim.x)
-    counts[(size_t)c * n_tiles + blockIdx.x] = sc[c];
+  __syncwarp();
+}
+
+// ---- pass 1 ---------------------------------------------------------------
+// masks[c * n_tiles + tile]
+template <int KMAX>
+__global__ void __launch_bounds__(128) brim_mask_kernel(const int32_t* __restrict__ topk_idx,
+                                                        const int32_t* __restrict__ slot_of,
+                                                        int T, int k, int E, int R, int n_tiles,
+                                                        uint32_t* __restrict__ masks,
+                                                        unsigned* err) {
+  __shared__ uint32_t sm[4][kMaxCols];
+  const int w = threadIdx.x >> 5;
+  const int tile = blockIdx.x * 4 + w;
+  if (tile >= n_tiles) return;
+  const int ncol = R + E, L = E / R;
+  const unsigned lane = lane_id();
+  const int t = tile * kBrimTileTokens + (int)lane;
+  TokenRoute<KMAX> tr;
+  const bool active = t < T && load_token_route<KMAX>(topk_idx, slot_of, t, k, E, L, tr, err);
+  tile_masks<KMAX>(sm[w], ncol, R, active, k, tr);
+  for (int c = lane; c < ncol; c += 32) masks[(size_t)c * n_tiles + tile] = sm[w][c];
 }
 
 // Inclusive scan of one value per lane across the warp.
@@ -98,7 +127,7 @@ __device__ __forceinline__ int warp_inclusive_scan(int x) {
   return x;
 }
 
-// Exclusive scan of n values (smem) by one warp, chunk by chunk; returns the total.
+// Exclusive scan of n values (smem) by one warp; returns the total.
 __device__ __forceinline__ int warp_exclusive_scan_smem(const int32_t* in, int32_t* out, int n) {
   const unsigned lane = lane_id();
   int carry = 0;
@@ -113,30 +142,35 @@ __device__ __forceinline__ int warp_exclusive_scan_smem(const int32_t* in, int32
 }
 
 // ---- pass 2 ---------------------------------------------------------------
-// One block of 32 warps.  counts[c][tile] becomes the global first row of
-// `tile` in column c; sfd_off / epd_off / C_T are written.
-__global__ void __launch_bounds__(1024) brim_scan_kernel(int32_t* __restrict__ counts,
+// One block of 32 warps.  Each warp scans whole columns: lane i sums a
+// contiguous run of tiles, a warp scan orders the runs, each lane writes its
+// run's bases.  The mask words are replaced by the tile's first global row.
+__global__ void __launch_bounds__(1024) brim_scan_kernel(uint32_t* __restrict__ masks,
                                                         int n_tiles, int E, int R,
                                                         int32_t* __restrict__ sfd_off,
                                                         int32_t* __restrict__ epd_off,
                                                         int32_t* __restrict__ c_t) {
-  __shared__ int32_t total[kMaxE * 2];
-  __shared__ int32_t colbase[kMaxE * 2];
+  __shared__ int32_t total[kMaxCols];
+  __shared__ int32_t colbase[kMaxCols];
   const int ncol = R + E;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const unsigned lane = lane_id();
-  // per column: exclusive scan over its tiles (tile order = token order)
+  const int run = (n_tiles + 31) / 32;  // tiles per lane
   for (int c = warp; c < ncol; c += nwarps) {
-    int32_t* col = counts + (size_t)c * n_tiles;
-    int carry = 0;
-    for (int b0 = 0; b0 < n_tiles; b0 += 32) {
-      const int b = b0 + (int)lane;
-      const int n = b < n_tiles ? col[b] : 0;
-      const int inc = warp_inclusive_scan(n);
-      if (b < n_tiles) col[b] = carry + inc - n;
-      carry += __shfl_sync(0xffffffffu, inc, 31);
+    uint32_t* col = masks + (size_t)c * n_tiles;
+    const int b0 = (int)lane * run;
+    const int b1 = min(b0 + run, n_tiles);
+    int sum = 0;
+#pragma unroll 8
+    for (int b = b0; b < b1; ++b) sum += __popc(col[b]);
+    const int inc = warp_inclusive_scan(sum);
+    int base = inc - sum;
+    for (int b = b0; b < b1; ++b) {
+      const int n = __popc(col[b]);
+      col[b] = (uint32_t)base;
+      base += n;
     }
-    if (lane == 0) total[c] = carry;
+    if (lane == 31) total[c] = inc;
   }
   __syncthreads();
   // where each rank's SFD segment and each slot's EPD group starts
@@ -154,109 +188,114 @@ __global__ void __launch_bounds__(1024) brim_scan_kernel(int32_t* __restrict__ c
   }
   __syncthreads();
   const int n_all = ncol * n_tiles;
-  for (int i = threadIdx.x; i < n_all; i += blockDim.x) counts[i] += colbase[i / n_tiles];
+  for (int i = threadIdx.x; i < n_all; i += blockDim.x)
+    masks[i] = (uint32_t)((int32_t)masks[i] + colbase[i / n_tiles]);
 }
 
 // ---- pass 3 ---------------------------------------------------------------
-__global__ void __launch_bounds__(kBrimTile) brim_scatter_kernel(
+template <int KMAX>
+__global__ void __launch_bounds__(128) brim_scatter_kernel(
     const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
     const int32_t* __restrict__ slot_of, int T, int k, int E, int R, int n_tiles,
     const int32_t* __restrict__ tile_base, int32_t* __restrict__ brim0,
     int32_t* __restrict__ sfd_token, int32_t* __restrict__ brim1,
-    int32_t* __restrict__ epd_sfd, float* __restrict__ epd_gate, unsigned* err) {
-  __shared__ uint32_t mask[kBrimWarps][kMaxE * 2];  // lanes of warp w that hit column c
-  __shared__ int32_t before[kBrimWarps][kMaxE * 2]; // hits in warps < w, plus the tile base
-  const int ncol = R + E;
-  const int L = E / R;
+    int32_t* __restrict__ epd_sfd, float* __restrict__ epd_gate) {
+  __shared__ uint32_t sm[4][kMaxCols];
+  const int w = threadIdx.x >> 5;
+  const int tile = blockIdx.x * 4 + w;
+  if (tile >= n_tiles) return;
+  const int ncol = R + E, L = E / R;
   const size_t cap = (size_t)T * (k < R ? k : R);
-  const int warp = threadIdx.x >> 5;
   const unsigned lane = lane_id();
-  for (int i = threadIdx.x; i < kBrimWarps * ncol; i += blockDim.x)
-    mask[i / ncol][i % ncol] = 0u;
-  __syncthreads();
-
-  const int t = blockIdx.x * kBrimTile + threadIdx.x;
-  TokenRoute tr;
-  bool ok = false;
-  if (t < T) {
-    ok = load_token_route(topk_idx, slot_of, t, k, E, L, tr, err);
-    if (ok) {
-      for (int i = 0; i < tr.n_rank; ++i) atomicOr(&mask[warp][tr.rank[i]], 1u << lane);
-      for (int j = 0; j < k; ++j) atomicOr(&mask[warp][R + tr.slot[j]], 1u << lane);
-    }
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < ncol; c += blockDim.x) {
-    int run = tile_base[(size_t)c * n_tiles + blockIdx.x];
-    for (int w = 0; w < kBrimWarps; ++w) {
-      before[w][c] = run;
-      run += __popc(mask[w][c]);
-    }
-  }
-  __syncthreads();
+  const int t = tile * kBrimTileTokens + (int)lane;
+  TokenRoute<KMAX> tr;
+  // the error flag was raised by pass 1 already
+  const bool active = t < T && load_token_route<KMAX>(topk_idx, slot_of, t, k, E, L, tr, nullptr);
+  tile_masks<KMAX>(sm[w], ncol, R, active, k, tr);
   if (t >= T) return;
-
-  const uint32_t lt = (1u << lane) - 1u;
-  // BRIM_0 column of this token (every rank: a row or -1) and sfd_token
-  int s_of_rank[kMaxK];
   for (int r = 0; r < R; ++r) brim0[(size_t)r * T + t] = -1;
-  if (!ok) return;
-  for (int i = 0; i < tr.n_rank; ++i) {
-    const int r = tr.rank[i];
-    const int s = before[warp][r] + __popc(mask[warp][r] & lt);
-    s_of_rank[i] = s;
-    brim0[(size_t)r * T + t] = s;
-    sfd_token[s] = t;
-    // every local expert of this rank starts as "not selected" for row s
-    for (int l = 0; l < L; ++l) brim1[(size_t)l * cap + s] = -1;
+  if (!active) return;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int32_t* base = tile_base + tile;  // base[c] at base[c * n_tiles]
+  int s_of[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    s_of[j] = -1;
+    if (j < k && tr.first[j]) {
+      const int r = tr.rank[j];
+      s_of[j] = __ldg(base + (size_t)r * n_tiles) + __popc(sm[w][r] & lt);
+    }
   }
-  for (int j = 0; j < k; ++j) {
-    const int q = tr.slot[j];
-    const int r = q / L, l = q - r * L;
-    int s = -1;
-    for (int i = 0; i < tr.n_rank; ++i)
-      if (tr.rank[i] == r) s = s_of_rank[i];
-    const int p = before[warp][R + q] + __popc(mask[warp][R + q] & lt);
-    brim1[(size_t)l * cap + s] = p;
-    epd_sfd[p] = s;
-    epd_gate[p] = topk_w[(size_t)t * k + j];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k && tr.first[j]) {
+      const int s = s_of[j];
+      brim0[(size_t)tr.rank[j] * T + t] = s;
+      sfd_token[s] = t;
+      // every local expert of this rank starts as "not selected" for row s
+      for (int l = 0; l < L; ++l) brim1[(size_t)l * cap + s] = -1;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k) {
+      const int q = tr.slot[j];
+      int s = -1;
+#pragma unroll
+      for (int i = 0; i <= j; ++i)
+        if (tr.first[i] && tr.rank[i] == tr.rank[j]) s = s_of[i];
+      const int p = __ldg(base + (size_t)(R + q) * n_tiles) + __popc(sm[w][R + q] & lt);
+      brim1[(size_t)(q - tr.rank[j] * L) * cap + s] = p;
+      epd_sfd[p] = s;
+      epd_gate[p] = __ldg(topk_w + (size_t)t * k + j);
+    }
   }
 }
 
 // ---- placement-aware dispatched-row counter ------------------------------
+// Warp-aggregated: lanes holding the same rank are merged with match.any
+// before one shared atomic; totals are warp-reduced before one global atomic.
+template <int KMAX>
 __global__ void __launch_bounds__(256) count_dispatched_kernel(
     const int32_t* __restrict__ topk_idx, int T, int k, const int32_t* __restrict__ slot_of,
     int E, int R, int32_t* __restrict__ per_rank, unsigned long long* __restrict__ total,
     unsigned long long* __restrict__ remote, unsigned* err) {
   __shared__ int32_t sc[kMaxE];
-  __shared__ unsigned long long s_total, s_remote;
+  __shared__ unsigned s_total, s_remote;
   const int L = E / R;
   for (int r = threadIdx.x; r < R; r += blockDim.x) sc[r] = 0;
   if (threadIdx.x == 0) {
-    s_total = 0ull;
-    s_remote = 0ull;
+    s_total = 0u;
+    s_remote = 0u;
   }
   __syncthreads();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < T) {
-    TokenRoute tr;
-    if (load_token_route(topk_idx, slot_of, t, k, E, L, tr, err)) {
-      const int src = (int)(((long long)t * R) / T);
-      int n_remote = 0;
-      for (int i = 0; i < tr.n_rank; ++i) {
-        atomicAdd(&sc[tr.rank[i]], 1);
-        n_remote += (tr.rank[i] != src);
-      }
-      atomicAdd(&s_total, (unsigned long long)tr.n_rank);
-      if (n_remote) atomicAdd(&s_remote, (unsigned long long)n_remote);
+  TokenRoute<KMAX> tr;
+  const bool active = t < T && load_token_route<KMAX>(topk_idx, slot_of, t, k, E, L, tr, err);
+  const int src = (int)(((long long)t * R) / (T > 0 ? T : 1));
+  unsigned n_rank = 0, n_remote = 0;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const int r = (active && j < k && tr.first[j]) ? tr.rank[j] : -1;
+    if (r >= 0) {
+      ++n_rank;
+      n_remote += (r != src);
     }
+    const unsigned same = __match_any_sync(0xffffffffu, r);
+    if (r >= 0 && (int)lane_id() == __ffs(same) - 1) atomicAdd(&sc[r], __popc(same));
+  }
+  n_rank = __reduce_add_sync(0xffffffffu, n_rank);
+  n_remote = __reduce_add_sync(0xffffffffu, n_remote);
+  if (lane_id() == 0) {
+    atomicAdd(&s_total, n_rank);
+    atomicAdd(&s_remote, n_remote);
   }
   __syncthreads();
   for (int r = threadIdx.x; r < R; r += blockDim.x)
     if (sc[r]) atomicAdd(&per_rank[r], sc[r]);
   if (threadIdx.x == 0) {
-    if (s_total) atomicAdd(total, s_total);
-    if (s_remote) atomicAdd(remote, s_remote);
+    if (s_total) atomicAdd(total, (unsigned long long)s_total);
+    if (s_remote) atomicAdd(remote, (unsigned long long)s_remote);
   }
 }
 
@@ -264,6 +303,7 @@ __global__ void __launch_bounds__(256) count_dispatched_kernel(
 // Integer atomics, so the result does not depend on the order they land in.
 // Small E: a per-block histogram in shared memory flushed once per block.
 constexpr int kHistSmemE = 64;
+template <int KMAX>
 __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restrict__ topk_idx,
                                                          int T, int k, int E,
                                                          uint32_t* __restrict__ hist,
@@ -276,22 +316,30 @@ __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restri
   }
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t < T) {
-    int ids[kMaxK];
+    int ids[KMAX];
     bool ok = true;
-    for (int j = 0; j < k; ++j) {
-      ids[j] = topk_idx[(size_t)t * k + j];
-      if (ids[j] < 0 || ids[j] >= E) ok = false;
-      for (int i = 0; i < j; ++i) ok &= ids[i] != ids[j];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ids[j] = 0;
+      if (j < k) {
+        ids[j] = __ldg(topk_idx + (size_t)t * k + j);
+        if (ids[j] < 0 || ids[j] >= E) ok = false;
+#pragma unroll
+        for (int i = 0; i < j; ++i) ok &= ids[i] != ids[j];
+      }
     }
     if (!ok) {
       raise_error(err, kErrIndex);
     } else {
-      for (int a = 0; a < k; ++a)
-        for (int b = 0; b < k; ++b) {
-          const int cell = ids[a] * E + ids[b];
-          if (use_smem) atomicAdd(&sh[cell], 1u);
-          else atomicAdd(&hist[cell], 1u);
-        }
+#pragma unroll
+      for (int a = 0; a < KMAX; ++a)
+#pragma unroll
+        for (int b = 0; b < KMAX; ++b)
+          if (a < k && b < k) {
+            const int cell = ids[a] * E + ids[b];
+            if (use_smem) atomicAdd(&sh[cell], 1u);
+            else atomicAdd(&hist[cell], 1u);
+          }
     }
   }
   if (use_smem) {

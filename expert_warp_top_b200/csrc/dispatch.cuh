@@ -9,176 +9,212 @@
 // device that a token co-activates ("intra-collaboration") are summed before
 // the single return row leaves the device.
 //
-// All movers work one warp per token and move 16 bytes per lane per access
-// (128-bit, fully coalesced 512-byte warp accesses).  A warp first reads the
-// token's BRIM entries into a short destination list, then streams the row.
+// The movers split every token row into 512-byte slices (16 bytes per lane,
+// fully coalesced 128-bit accesses) and give each warp one slice (or a few), so
+// a batch of a few thousand tokens still fills every SM.  A warp first reads
+// its token's BRIM entries into a short destination list in shared memory,
+// then moves its slice.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int kMoverWarps = 8;     // warps per block
-constexpr int kMaxDst = 32;        // >= min(k,R) + k for k <= 16
+constexpr int kMaxDst = 16;        // >= k (and >= min(k, R))
 
-// Collect, for token t, the SFD rows (ascending rank) and for each of them
-// its EPD rows (ascending local expert).  n_sfd <= min(k, R); p_start has
-// n_sfd + 1 entries into p_list.  Out-of-range entries raise the error flag
-// and are dropped.
-struct DstList {
+// Destinations of one token, per warp, in shared memory:
+//   sfd[i]   SFD rows of the ranks the token is sent to (ascending rank)
+//   p[j]     EPD rows of its experts, ascending (rank, local expert), and
+//   p_sfd[j] the SFD row each of them hangs off
+struct WarpDst {
   int n_sfd;
-  int sfd[16];
-  int p_start[17];
-  int p_list[16];
+  int n_p;
+  int sfd[kMaxDst];
+  int p[kMaxDst];
+  int p_sfd[kMaxDst];
 };
 
+// Reads token t's BRIM_0 column and, for every (rank, local expert) slot, its
+// BRIM_1 entry; ballots keep ascending order.  Out-of-range entries raise the
+// error flag and are dropped.
 __device__ __forceinline__ void collect_dst(const int32_t* __restrict__ brim0,
                                             const int32_t* __restrict__ brim1, int t, int T,
-                                            int R, int L, size_t cap, int tk, DstList& dl,
+                                            int R, int L, size_t cap, int tk, WarpDst& w,
                                             unsigned* err) {
   const unsigned lane = lane_id();
-  dl.n_sfd = 0;
-  int np = 0;
+  const uint32_t lt = (1u << lane) - 1u;
   bool bad = false;
+  int n = 0;
   for (int r0 = 0; r0 < R; r0 += 32) {
     const int r = r0 + (int)lane;
-    int s = (r < R) ? brim0[(size_t)r * T + t] : -1;
+    int s = (r < R) ? __ldg(brim0 + (size_t)r * T + t) : -1;
     if (s >= (int)cap) {
       bad = true;
       s = -1;
     }
-    unsigned hit = __ballot_sync(0xffffffffu, s >= 0);
-    while (hit) {
-      const int src = __ffs(hit) - 1;
-      hit &= hit - 1;
-      const int sv = __shfl_sync(0xffffffffu, s, src);
-      if (dl.n_sfd < 16) {
-        dl.sfd[dl.n_sfd] = sv;
-        dl.p_start[dl.n_sfd] = np;
-        // this SFD row's local experts
-        for (int l0 = 0; l0 < L; l0 += 32) {
-          const int l = l0 + (int)lane;
-          int p = (l < L) ? brim1[(size_t)l * cap + sv] : -1;
-          if (p >= tk) {
-            bad = true;
-            p = -1;
-          }
-          unsigned ph = __ballot_sync(0xffffffffu, p >= 0);
-          while (ph) {
-            const int ps = __ffs(ph) - 1;
-            ph &= ph - 1;
-            const int pv = __shfl_sync(0xffffffffu, p, ps);
-            if (np < 16) dl.p_list[np++] = pv;
-            else bad = true;
-          }
-        }
-        dl.n_sfd++;
-      } else {
+    const unsigned hit = __ballot_sync(0xffffffffu, s >= 0);
+    const int pos = n + __popc(hit & lt);
+    if (s >= 0 && pos < kMaxDst) w.sfd[pos] = s;
+    n += __popc(hit);
+  }
+  if (n > kMaxDst) bad = true;
+  const int n_sfd = min(n, kMaxDst);
+  n = 0;
+  const int E = R * L;
+  for (int q0 = 0; q0 < E; q0 += 32) {
+    const int q = q0 + (int)lane;
+    int s = -1, p = -1;
+    if (q < E) {
+      const int r = q / L, l = q - r * L;
+      s = __ldg(brim0 + (size_t)r * T + t);
+      if (s >= 0 && s < (int)cap) p = __ldg(brim1 + (size_t)l * cap + s);
+      if (p >= tk) {
         bad = true;
+        p = -1;
       }
     }
+    const unsigned hit = __ballot_sync(0xffffffffu, p >= 0);
+    const int pos = n + __popc(hit & lt);
+    if (p >= 0 && pos < kMaxDst) {
+      w.p[pos] = p;
+      w.p_sfd[pos] = s;
+    }
+    n += __popc(hit);
   }
-  dl.p_start[dl.n_sfd] = np;
+  if (n > kMaxDst) bad = true;
+  if (lane == 0) {
+    w.n_sfd = n_sfd;
+    w.n_p = min(n, kMaxDst);
+  }
   if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(err, kErrIndex);
+  __syncwarp();
 }
 
 // x_sfd[s] = x[t] and x_epd[p] = x[t] for every destination of token t.
+// One warp per token (P > 1: per 1/P of its row, for small batches); the row
+// is read CH x 512 bytes at a time, all CH loads in flight before the stores.
+template <int CH>
 __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
-    const uint8_t* __restrict__ x, int T, int row_bytes, int R, int L, size_t cap, int tk,
+    const uint8_t* __restrict__ x, int T, int row_bytes, int P, int R, int L, size_t cap, int tk,
     const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
     uint8_t* __restrict__ x_sfd, uint8_t* __restrict__ x_epd, unsigned* err) {
-  const int t = blockIdx.x * kMoverWarps + (threadIdx.x >> 5);
+  __shared__ WarpDst sdst[kMoverWarps];
+  const int wib = threadIdx.x >> 5;
+  const long long wg = (long long)blockIdx.x * kMoverWarps + wib;
+  const int t = (int)(wg / P);
   if (t >= T) return;
+  const int part = (int)(wg - (long long)t * P);
   const unsigned lane = lane_id();
-  DstList dl;
-  collect_dst(brim0, brim1, t, T, R, L, cap, tk, dl, err);
+  WarpDst& w = sdst[wib];
+  collect_dst(brim0, brim1, t, T, R, L, cap, tk, w, err);
+  const int span = (row_bytes + P - 1) / P;
+  const int lo = part * span, hi = min(row_bytes, lo + span);
   const uint8_t* src = x + (size_t)t * row_bytes;
-  const int n_p = dl.p_start[dl.n_sfd];
-  // 4 x 512 bytes in flight per warp per step
-  for (int off0 = 0; off0 < row_bytes; off0 += 4 * 512) {
-    uint4 v[4];
+  const int n_sfd = x_sfd ? w.n_sfd : 0, n_p = x_epd ? w.n_p : 0;
+  for (int off0 = lo; off0 < hi; off0 += CH * 512) {
+    uint4 v[CH];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < CH; ++u) {
       const int off = off0 + u * 512 + (int)lane * 16;
-      if (off < row_bytes) v[u] = ld_nc_v4(src + off);
+      if (off < hi) v[u] = ld_nc_v4(src + off);
     }
+    for (int i = 0; i < n_sfd; ++i) {
+      uint8_t* dst = x_sfd + (size_t)w.sfd[i] * row_bytes;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int off = off0 + u * 512 + (int)lane * 16;
-      if (off >= row_bytes) continue;
-      if (x_sfd)
-        for (int i = 0; i < dl.n_sfd; ++i) st_v4(x_sfd + (size_t)dl.sfd[i] * row_bytes + off, v[u]);
-      if (x_epd)
-        for (int i = 0; i < n_p; ++i) st_v4(x_epd + (size_t)dl.p_list[i] * row_bytes + off, v[u]);
+      for (int u = 0; u < CH; ++u) {
+        const int off = off0 + u * 512 + (int)lane * 16;
+        if (off < hi) st_v4(dst + off, v[u]);
+      }
+    }
+    for (int i = 0; i < n_p; ++i) {
+      uint8_t* dst = x_epd + (size_t)w.p[i] * row_bytes;
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int off = off0 + u * 512 + (int)lane * 16;
+        if (off < hi) st_v4(dst + off, v[u]);
+      }
     }
   }
 }
 
-// y_sfd[s] = sum_l o_epd[BRIM_1[l][s]] (fp32, rounded to T); y[t] = sum_r y_sfd[..]
+// y_sfd[s] = sum_l o_epd[BRIM_1[l][s]] (fp32, rounded to TA); y[t] = sum_r y_sfd[..]
 // (+ shared[t]).  y sums the rounded payload rows, exactly as if it had read
-// them back.
-template <typename TA>
+// them back.  One warp per token (or 1/P of its row); the k expert rows of the
+// next 512-byte slice are loaded while the current slice is summed, so up to
+// 2k loads are in flight per warp.  KMAX >= k bounds the register arrays.
+template <typename TA, int KMAX>
 __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
-    const TA* __restrict__ o_epd, int T, int d, int R, int L, size_t cap, int tk,
+    const TA* __restrict__ o_epd, int T, int d, int P, int R, int L, size_t cap, int tk,
     const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
     const TA* __restrict__ shared_out, TA* __restrict__ y_sfd, TA* __restrict__ y,
     unsigned* err) {
   constexpr int VN = Vec16<TA>::n;  // elements per 16 bytes
-  const int t = blockIdx.x * kMoverWarps + (threadIdx.x >> 5);
+  constexpr int SL = 32 * VN;       // elements per 512-byte slice
+  __shared__ WarpDst sdst[kMoverWarps];
+  const int wib = threadIdx.x >> 5;
+  const long long wg = (long long)blockIdx.x * kMoverWarps + wib;
+  const int t = (int)(wg / P);
   if (t >= T) return;
+  const int part = (int)(wg - (long long)t * P);
   const unsigned lane = lane_id();
-  DstList dl;
-  collect_dst(brim0, brim1, t, T, R, L, cap, tk, dl, err);
-  for (int c0 = 0; c0 < d; c0 += 2 * 32 * VN) {
-    float ya[2][VN];
+  WarpDst& w = sdst[wib];
+  collect_dst(brim0, brim1, t, T, R, L, cap, tk, w, err);
+  const int n_slices = (d + SL - 1) / SL;
+  const int per = (n_slices + P - 1) / P;
+  const int s_lo = part * per, s_hi = min(n_slices, s_lo + per);
+  const int n_p = min(w.n_p, KMAX);
+  int prow[KMAX], psfd[KMAX];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+  for (int j = 0; j < KMAX; ++j) {
+    prow[j] = j < n_p ? w.p[j] : 0;
+    psfd[j] = j < n_p ? w.p_sfd[j] : -1;
+  }
+  uint4 cur[KMAX], nxt[KMAX];
+  auto load_slice = [&](int sl, uint4 (&v)[KMAX]) {
+    const int c = sl * SL + (int)lane * VN;
 #pragma unroll
-      for (int i = 0; i < VN; ++i) ya[u][i] = 0.f;
-    for (int i = 0; i < dl.n_sfd; ++i) {
-      float acc[2][VN];
+    for (int j = 0; j < KMAX; ++j)
+      if (j < n_p && c < d) v[j] = ld_nc_v4(o_epd + (size_t)prow[j] * d + c);
+  };
+  if (s_lo < s_hi) load_slice(s_lo, cur);
+  for (int sl = s_lo; sl < s_hi; ++sl) {
+    if (sl + 1 < s_hi) load_slice(sl + 1, nxt);
+    const int c = sl * SL + (int)lane * VN;
+    if (c < d) {
+      float acc[VN], ya[VN];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int e = 0; e < VN; ++e) ya[e] = acc[e] = 0.f;
 #pragma unroll
-        for (int e = 0; e < VN; ++e) acc[u][e] = 0.f;
-      for (int j = dl.p_start[i]; j < dl.p_start[i + 1]; ++j) {
-        const TA* row = o_epd + (size_t)dl.p_list[j] * d;
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < n_p) {
+          float f[VN];
+          Vec16<TA>::to_f32(cur[j], f);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = c0 + u * 32 * VN + (int)lane * VN;
-          if (c < d) {
-            float f[VN];
-            Vec16<TA>::to_f32(ld_nc_v4(row + c), f);
+          for (int e = 0; e < VN; ++e) acc[e] += f[e];
+          // the last expert of this rank: emit the rank's return row
+          if (j + 1 == n_p || psfd[j + 1 < KMAX ? j + 1 : j] != psfd[j]) {
+            const uint4 packed = Vec16<TA>::from_f32(acc);
+            if (y_sfd) st_v4(y_sfd + (size_t)psfd[j] * d + c, packed);
+            float rounded[VN];
+            Vec16<TA>::to_f32(packed, rounded);
 #pragma unroll
-            for (int e = 0; e < VN; ++e) acc[u][e] += f[e];
+            for (int e = 0; e < VN; ++e) {
+              ya[e] += rounded[e];
+              acc[e] = 0.f;
+            }
           }
         }
       }
+      if (shared_out) {
+        float f[VN];
+        Vec16<TA>::to_f32(ld_nc_v4(shared_out + (size_t)t * d + c), f);
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = c0 + u * 32 * VN + (int)lane * VN;
-        if (c < d) {
-          const uint4 packed = Vec16<TA>::from_f32(acc[u]);
-          if (y_sfd) st_v4(y_sfd + (size_t)dl.sfd[i] * d + c, packed);
-          float rounded[VN];
-          Vec16<TA>::to_f32(packed, rounded);
-#pragma unroll
-          for (int e = 0; e < VN; ++e) ya[u][e] += rounded[e];
-        }
+        for (int e = 0; e < VN; ++e) ya[e] += f[e];
       }
+      st_v4(y + (size_t)t * d + c, Vec16<TA>::from_f32(ya));
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = c0 + u * 32 * VN + (int)lane * VN;
-      if (c < d) {
-        if (shared_out) {
-          float f[VN];
-          Vec16<TA>::to_f32(ld_nc_v4(shared_out + (size_t)t * d + c), f);
-#pragma unroll
-          for (int e = 0; e < VN; ++e) ya[u][e] += f[e];
-        }
-        st_v4(y + (size_t)t * d + c, Vec16<TA>::from_f32(ya[u]));
-      }
-    }
+    for (int j = 0; j < KMAX; ++j) cur[j] = nxt[j];
   }
 }
 

@@ -8,7 +8,10 @@
 //
 // Kernel shape (one persistent CTA per SM, 192 threads):
 //   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 (bf16; 32 wide
-//               for fp32/TF32) per stage, 128-byte swizzle, STAGES-deep ring
+//               for fp32/TF32) per stage, 128-byte swizzle, STAGES-deep ring.
+//               With a row index (GATHER), the A tile's rows are gathered:
+//               each of the 32 lanes issues one tile::gather4 of 4 rows, so the
+//               compact EPD rows are read straight out of the SFD payload.
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma M=128, N=BN, K=16 (8 for
 //               TF32), accumulators double-buffered in TMEM (2 x BN columns)
 //   warps 2..5  epilogue: tcgen05.ld of its 32 TMEM lanes (= 32 tile rows),
@@ -57,6 +60,8 @@ struct GemmCfg {
 
 struct GemmArgs {
   const int32_t* group_off;  // [G+1] device
+  const int32_t* a_row_index;  // GATHER: row of A feeding each of the m_cap rows
+  int a_rows;                // GATHER: rows of A
   int G;
   int N;                     // output columns per group (B rows per group)
   int K;
@@ -69,7 +74,7 @@ struct GemmArgs {
   int debug;
 };
 
-template <int BN, int EPI, bool TF32>
+template <int BN, int EPI, bool TF32, bool GATHER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
@@ -175,7 +180,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop: lane 0 waits, arms the stage and loads B;
+    // in GATHER mode every lane then gathers 4 of the tile's 128 A rows.
+    if (GATHER || lane == 0) {
       const uint64_t pol_a = tc::policy_evict_normal();
       const uint64_t pol_b = tc::policy_evict_last();
       int stage = 0;
@@ -183,21 +190,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t armed = 0, armed_parity = 0;  // per stage: armed at least once, parity of the last arming
       bool skip_next = (args.debug & kDebugSkipFirstLoad) != 0;
       bool ok = true;
+      bool bad_row = false;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         int g, row0, rows, n0;
         locate(tile, g, row0, rows, n0);
+        int ri[4] = {0, 0, 0, 0};
+        if (GATHER) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int i = (int)lane * 4 + r;
+            if (i < rows) {
+              const int v = __ldg(args.a_row_index + row0 + i);
+              if (v >= 0 && v < args.a_rows) ri[r] = v;
+              else bad_row = true;
+            }
+          }
+        }
         for (int kb = 0; kb < k_blocks; ++kb) {
-          if (!tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl)) {
+          bool go = true;
+          if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl);
+          if (GATHER) go = __shfl_sync(0xffffffffu, go, 0) != 0;
+          if (!go) {
             ok = false;
             break;
           }
           if (!skip_next) {
             const uint32_t fb = tc::smem_u32(&full_bar[stage]);
-            tc::mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
             uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
-            tc::tma_load_2d(tc::smem_u32(sa), &tmap_a, fb, kb * Cfg::kBK, row0, pol_a);
-            tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, kb * Cfg::kBK,
-                            g * args.N + n0, pol_b);
+            if (lane == 0) {
+              tc::mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+              if (!GATHER)
+                tc::tma_load_2d(tc::smem_u32(sa), &tmap_a, fb, kb * Cfg::kBK, row0, pol_a);
+              tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, kb * Cfg::kBK,
+                              g * args.N + n0, pol_b);
+            }
+            if (GATHER) {
+              __syncwarp();
+              tc::tma_gather4(tc::smem_u32(sa + lane * 512), &tmap_a, fb, kb * Cfg::kBK, ri[0],
+                              ri[1], ri[2], ri[3], pol_a);
+            }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
@@ -208,12 +239,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      if (GATHER && __any_sync(0xffffffffu, bad_row) && lane == 0) raise_error(args.err, kErrIndex);
       // Leave no TMA write in flight into this CTA's shared memory: wait for
       // the last arming of every stage (already complete on the normal path,
       // where the MMA issuer consumed it; maybe not if the CTA is unwinding).
-      for (int s = 0; s < S; ++s)
-        if ((armed >> s) & 1u)
-          tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
+      if (lane == 0)
+        for (int s = 0; s < S; ++s)
+          if ((armed >> s) & 1u)
+            tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

@@ -86,6 +86,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint3
       : "memory");
 }
 
+// Four rows (r0..r3, any order) of a 2-D tensor whose map has a one-row box:
+// 4 x box-width elements land as four consecutive rows at dst.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* map, uint32_t bar, int c0,
+                                            int r0, int r1, int r2, int r3, uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "l"(cache_hint)
+      : "memory");
+}
+
 // L2 cache-policy operands (createpolicy.fractional with fraction 1.0).
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;

@@ -5,8 +5,17 @@ the CUDA library through the binding:
 
   route (top-k, softmax)        moe_route_topk
   BRIM_0 / BRIM_1 / C_T         moe_brim_build
-  ORI -> SFD -> EPD             moe_dispatch_gather
+  ORI -> SFD (-> EPD)           moe_dispatch_gather
   routed experts (grouped GEMM) moe_expert_ffn over the EPD groups
+
+How the experts reach their EPD rows (epd_mode):
+  "stored"  the dispatch writes the EPD rows; the GEMM reads them as tiles
+  "direct"  one local expert per rank (L = 1): the EPD state is the SFD state
+            row for row (same order, same groups), so the GEMM reads the SFD
+            payload as it is and no EPD copy exists
+  "gather"  the GEMM gathers each EPD row out of the SFD payload (TMA gather4
+            by epd_sfd); measured slower on B200 than "stored", kept as an option
+  "auto"    "direct" when L = 1, else "stored"
   shared experts                moe_expert_ffn over the ORI rows (one group)
   pre-reduce + combine          moe_combine_scatter
   dispatched-row counter        moe_count_dispatched_rows
@@ -22,13 +31,22 @@ from . import _binding as B
 class MoELayer:
     def __init__(self, *, T, d, f, E, k, R, renorm=0, dtype=torch.bfloat16, S=0, fs=0,
                  slot_of=None, wg=None, wu=None, wd=None, sg=None, su=None, sd=None,
-                 ffn_kind=B.MOE_FFN_SWIGLU, device="cuda", stream=None):
+                 ffn_kind=B.MOE_FFN_SWIGLU, device="cuda", stream=None, epd_mode="auto"):
         if E % R:
             raise ValueError("R must divide E")
         self.T, self.d, self.f, self.E, self.k, self.R = T, d, f, E, k, R
         self.L = E // R
         self.renorm, self.dtype, self.S, self.fs = renorm, dtype, S, fs
         self.ffn_kind = ffn_kind
+        if epd_mode == "auto":
+            epd_mode = "direct" if E // R == 1 else "stored"
+        if epd_mode not in ("stored", "direct", "gather"):
+            raise ValueError(f"unknown epd_mode {epd_mode!r}")
+        if epd_mode == "direct" and E // R != 1:
+            raise ValueError("epd_mode='direct' needs one expert per rank (L = 1)")
+        if ffn_kind == B.MOE_FFN_IDENTITY and epd_mode == "gather":
+            epd_mode = "stored"  # the identity expert works on rows in place
+        self.epd_mode = epd_mode
         self.cap = T * min(k, R)
         self.tk = T * k
         dev = torch.device(device)
@@ -53,7 +71,7 @@ class MoELayer:
                                    dtype=torch.uint8, device=dev)
         # token states
         self.x_sfd = torch.empty(max(self.cap, 1), d, **act)
-        self.x_epd = torch.empty(max(self.tk, 1), d, **act)
+        self.x_epd = torch.empty(max(self.tk, 1), d, **act) if epd_mode == "stored" else None
         self.o_epd = torch.empty(max(self.tk, 1), d, **act)
         self.y_sfd = torch.empty(max(self.cap, 1), d, **act)
         self.y = torch.empty(T, d, **act)
@@ -99,8 +117,18 @@ class MoELayer:
                               self.x_epd, stream)
 
     def experts(self, stream=None):
-        B.moe_expert_ffn(self.x_epd[: max(self.tk, 1)], self.epd_off, self.w_gu, self.w_dn, self.f,
-                         self.epd_gate, self.ffn_kind, self.o_epd, self.ffn_ws, stream)
+        m_cap = max(self.tk, 1)
+        if self.epd_mode == "stored":
+            B.moe_expert_ffn(self.x_epd, self.epd_off, self.w_gu, self.w_dn, self.f,
+                             self.epd_gate, self.ffn_kind, self.o_epd, self.ffn_ws, stream)
+        elif self.epd_mode == "direct":
+            B.moe_expert_ffn(self.x_sfd, self.epd_off, self.w_gu, self.w_dn, self.f,
+                             self.epd_gate, self.ffn_kind, self.o_epd, self.ffn_ws, stream,
+                             m_cap=m_cap)
+        else:
+            B.moe_expert_ffn(self.x_sfd, self.epd_off, self.w_gu, self.w_dn, self.f,
+                             self.epd_gate, self.ffn_kind, self.o_epd, self.ffn_ws, stream,
+                             a_row_index=self.epd_sfd, m_cap=m_cap)
 
     def shared_experts(self, x, stream=None):
         if self.S > 0:

@@ -146,8 +146,9 @@ int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
  * workspace to lend, so this entry point takes none.
  * Scratch: a fixed array of 1 MiB (262144 int32) in this library's device
  * memory, reserved on every GPU that loads the library until the process
- * exits.  A call needs ceil(T / 256) * (R + E) entries of it; a larger call
- * returns MOE_ERR_UNSUPPORTED and enqueues nothing.  The passes overwrite
+ * exits.  A call needs ceil(T / 32) * (R + E) entries of it (T <= 116k tokens
+ * at E = 64, R = 8); a larger call returns MOE_ERR_UNSUPPORTED and enqueues
+ * nothing.  The passes overwrite
  * every scratch entry they read, so nothing has to be cleared between calls.
  * All calls on a device share the one array: calls that may run on the GPU at
  * the same time (e.g. on two streams without ordering) race on it and must be
@@ -203,25 +204,33 @@ int moe_prepare_shared_weights(const void* sg, const void* su, const void* sd, i
  * moe_expert_ffn -- the expert computation of the Occult pipeline (TL;DR:
  * "sparse-matrix-multiplication pipeline"), as a grouped GEMM over ragged
  * row groups on the tcgen05 tensor cores:
- *   for every group g (rows group_off[g] .. group_off[g+1]-1 of a, expert g):
- *     h   = silu(a Wg^T) * (a Wu^T)        [rows, f]  (kept in the workspace)
+ *   for every group g (rows group_off[g] .. group_off[g+1]-1, expert g):
+ *     h   = silu(A Wg^T) * (A Wu^T)        [rows, f]  (kept in the workspace)
  *     out = row_scale * (h Wd^T)           [rows, d]
- *   a         [m_cap, d] dtype      input rows (e.g. the EPD rows)
- *   group_off [G+1] int32 (device)  ascending, group_off[0] >= 0,
- *                                   group_off[G] <= m_cap
- *   w_gu, w_dn                      packed by moe_prepare_weights (G experts)
- *   row_scale [m_cap] float32       per-row factor (e.g. epd_gate), or NULL = 1
- *   ffn_kind  MOE_FFN_SWIGLU, or MOE_FFN_IDENTITY (out = row_scale * a; the
- *             weights are not read and may be NULL)
- *   out       [m_cap, d] dtype      rows outside every group are not written
- *   ws        at least moe_expert_ffn_workspace_size(m_cap, f, dtype) bytes
+ *   a           [a_rows, d] dtype      the source rows
+ *   a_row_index [m_cap] int32 or NULL  with it, GEMM row p reads a[a_row_index[p]]
+ *                                      (e.g. the SFD payload with epd_sfd: the
+ *                                      EPD rows are gathered on the fly by TMA and
+ *                                      never stored); without it, row p is a[p]
+ *                                      and a_rows must be >= m_cap
+ *   group_off   [G+1] int32 (device)   ascending, group_off[0] >= 0,
+ *                                      group_off[G] <= m_cap (violations are
+ *                                      treated as empty groups and raise the
+ *                                      device error flag)
+ *   w_gu, w_dn                         packed by moe_prepare_weights (G experts)
+ *   row_scale   [m_cap] float32        per-row factor (e.g. epd_gate), or NULL = 1
+ *   ffn_kind    MOE_FFN_SWIGLU, or MOE_FFN_IDENTITY (out = row_scale * a; needs
+ *               a_row_index == NULL; the weights are not read and may be NULL)
+ *   out         [m_cap, d] dtype       rows outside every group are not written
+ *   ws          at least moe_expert_ffn_workspace_size(m_cap, f, dtype) bytes
  * bf16 runs bf16 x bf16 -> fp32 MMAs; f32 runs TF32 MMAs (fp32 accumulate).
  * The hidden activation h is rounded to dtype between the two GEMMs.
  * Device-side waits are bounded: a wait that expires raises MOE_ERR_TIMEOUT
  * through moe_get_device_status() and the kernel returns.
  * ------------------------------------------------------------------------- */
 size_t moe_expert_ffn_workspace_size(int m_cap, int f, int dtype);
-int moe_expert_ffn(const void* a, const int32_t* group_off, int G, int m_cap,
+int moe_expert_ffn(const void* a, int a_rows, const int32_t* a_row_index,
+                   const int32_t* group_off, int G, int m_cap,
                    const void* w_gu, const void* w_dn, int d, int f, int dtype,
                    const float* row_scale, int ffn_kind, void* out,
                    void* ws, size_t ws_bytes, moe_stream_t stream);

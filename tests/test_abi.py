@@ -66,20 +66,19 @@ def test_brim_rejects_bad_rank_counts(E, k, R):
 
 def test_ffn_rejects_bad_shapes():
     lib = moe.load()
-    # d not a multiple of 64
-    assert lib.moe_expert_ffn(NULL, NULL, 1, 16, NULL, NULL, 96, 128, B.MOE_BF16, NULL,
-                              B.MOE_FFN_SWIGLU, NULL, NULL, ctypes.c_size_t(0), NULL) \
-        == B.MOE_ERR_UNSUPPORTED
-    # unknown dtype / kind
-    assert lib.moe_expert_ffn(NULL, NULL, 1, 16, NULL, NULL, 128, 128, 7, NULL,
-                              B.MOE_FFN_SWIGLU, NULL, NULL, ctypes.c_size_t(0), NULL) \
-        == B.MOE_ERR_INVALID_ARG
-    assert lib.moe_expert_ffn(NULL, NULL, 1, 16, NULL, NULL, 128, 128, B.MOE_BF16, NULL,
-                              5, NULL, NULL, ctypes.c_size_t(0), NULL) == B.MOE_ERR_INVALID_ARG
-    # too many groups
-    assert lib.moe_expert_ffn(NULL, NULL, 5000, 16, NULL, NULL, 128, 128, B.MOE_BF16, NULL,
-                              B.MOE_FFN_SWIGLU, NULL, NULL, ctypes.c_size_t(0), NULL) \
-        == B.MOE_ERR_UNSUPPORTED
+
+    def ffn(G=1, a_rows=16, ridx=NULL, m_cap=16, d=128, f=128, dtype=B.MOE_BF16,
+            kind=B.MOE_FFN_SWIGLU):
+        return lib.moe_expert_ffn(NULL, a_rows, ridx, NULL, G, m_cap, NULL, NULL, d, f, dtype,
+                                  NULL, kind, NULL, NULL, ctypes.c_size_t(0), NULL)
+
+    assert ffn(d=96) == B.MOE_ERR_UNSUPPORTED            # d not a multiple of 64
+    assert ffn(dtype=7) == B.MOE_ERR_INVALID_ARG          # unknown dtype
+    assert ffn(kind=5) == B.MOE_ERR_INVALID_ARG           # unknown kind
+    assert ffn(G=5000) == B.MOE_ERR_UNSUPPORTED           # too many groups
+    assert ffn(a_rows=8, m_cap=16) == B.MOE_ERR_INVALID_ARG  # a too short without a row index
+    assert ffn(m_cap=-1) == B.MOE_ERR_INVALID_ARG
+    assert ffn() == B.MOE_ERR_INVALID_ARG                 # null pointers
 
 
 def test_movers_reject_bad_shapes():

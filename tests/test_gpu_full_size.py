@@ -42,6 +42,7 @@ def correlated_placement(cfg):
     ("corr_prefill", "contiguous"), ("corr_prefill", "histogram"),
 ])
 def test_full_size_layer(name, placement):
+    """The layer as the benchmark runs it (epd_mode auto)."""
     cfg = inputs.CONFIGS[name]
     inp = inputs.make_inputs(cfg, device=DEV)
     slot_of = (np.arange(cfg.E, dtype=np.int32) if placement == "contiguous"

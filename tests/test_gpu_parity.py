@@ -22,7 +22,7 @@ def softmax_rtol(E: int) -> float:
     return (E + 8) * 2.0 ** -23
 
 
-def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU):
+def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, epd_mode="auto"):
     dt = inputs.torch_dtype(cfg)
     kw = {}
     if ffn_kind == moe.MOE_FFN_SWIGLU:
@@ -31,7 +31,7 @@ def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU):
             kw.update(sg=inp["sg"].to(DEV), su=inp["su"].to(DEV), sd=inp["sd"].to(DEV))
     return MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
                     dtype=dt, S=cfg.S if ffn_kind == moe.MOE_FFN_SWIGLU else 0, fs=cfg.fs,
-                    slot_of=slot_of, ffn_kind=ffn_kind, device=DEV, **kw)
+                    slot_of=slot_of, ffn_kind=ffn_kind, device=DEV, epd_mode=epd_mode, **kw)
 
 
 def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
@@ -60,11 +60,12 @@ def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
     return b
 
 
-def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=None):
+def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=None,
+                        epd_mode="auto"):
     inp = inputs.make_inputs(cfg, seed=seed)
     if slot_of is None:
         slot_of = np.arange(cfg.E, dtype=np.int32)
-    layer = make_layer(cfg, inp, torch.from_numpy(slot_of), ffn_kind)
+    layer = make_layer(cfg, inp, torch.from_numpy(slot_of), ffn_kind, epd_mode)
     logits, x = inp["logits"].to(DEV), inp["x"].to(DEV)
     layer.hist.zero_()
     y = layer.forward(logits, x)
@@ -79,8 +80,9 @@ def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=Non
     xo = to_oracle(inp["x"])
     x_sfd_ref = oracle.gather_rows(xo, b["sfd_token"])
     assert np.array_equal(to_oracle(layer.x_sfd[:c_t]), x_sfd_ref)
-    assert np.array_equal(to_oracle(layer.x_epd[:cfg.T * cfg.k]),
-                          oracle.gather_rows(x_sfd_ref, b["epd_sfd"]))
+    if layer.x_epd is not None:
+        assert np.array_equal(to_oracle(layer.x_epd[:cfg.T * cfg.k]),
+                              oracle.gather_rows(x_sfd_ref, b["epd_sfd"]))
     # outputs against the BRIM-guided oracle and against the dense definition
     kind = oracle.KIND_IDENTITY if ffn_kind == moe.MOE_FFN_IDENTITY else oracle.KIND_SWIGLU
     w_ = (None, None, None) if kind == oracle.KIND_IDENTITY else \
@@ -113,10 +115,29 @@ def test_tiny_layer(dtype, renorm):
     run_and_check_small(cfg)
 
 
-def test_tiny_layer_permuted_placement():
+@pytest.mark.parametrize("epd_mode", ["stored", "gather"])
+def test_tiny_layer_permuted_placement(epd_mode):
     cfg = inputs.CONFIGS["tiny"]
     slot_of = np.random.default_rng(3).permutation(cfg.E).astype(np.int32)
-    run_and_check_small(cfg, slot_of)
+    run_and_check_small(cfg, slot_of, epd_mode=epd_mode)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_gathered_epd_rows(dtype):
+    """The GEMM gathering its EPD rows out of the SFD payload (TMA gather4)."""
+    cfg = inputs.LayerConfig("gather", T=900, d=256, f=128, E=16, k=4, R=4, dtype=dtype, seed=13)
+    run_and_check_small(cfg, epd_mode="gather")
+
+
+@pytest.mark.parametrize("epd_mode", ["direct", "stored"])
+def test_one_expert_per_rank(epd_mode):
+    """L = 1: the EPD state equals the SFD state; "direct" runs the GEMM on the payload."""
+    cfg = inputs.LayerConfig("l1", T=700, d=256, f=256, E=8, k=2, R=8, renorm=1, seed=14)
+    layer, _ = run_and_check_small(cfg, epd_mode=epd_mode)
+    c_t = int(layer.c_t.item())
+    assert c_t == cfg.T * cfg.k
+    assert torch.equal(layer.epd_sfd[:c_t].cpu(), torch.arange(c_t, dtype=torch.int32))
+    assert torch.equal(layer.epd_off.cpu(), layer.sfd_off.cpu())
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -205,6 +226,39 @@ def test_expert_ffn_ragged_groups():
                                                to_oracle(wd[g]))
     assert rowwise_rel_err(out[:m], ref) <= OUT_RTOL
     assert np.all(out[m:] == 7.0)  # rows outside every group are not written
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_expert_ffn_gathered_rows(dtype):
+    """The grouped GEMM reading its rows through a row index (TMA gather4)."""
+    g = torch.Generator().manual_seed(1)
+    d, f, G, a_rows = 128, 256, 4, 1000
+    sizes = [129, 0, 3, 300]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    m = int(off[-1])
+    a = torch.randn(a_rows, d, generator=g).to(dtype)
+    ridx = torch.randint(0, a_rows, (m,), generator=g, dtype=torch.int32)
+    wg = (torch.randn(G, f, d, generator=g) * 0.05).to(dtype)
+    wu = (torch.randn(G, f, d, generator=g) * 0.05).to(dtype)
+    wd = (torch.randn(G, d, f, generator=g) * 0.05).to(dtype)
+    w_gu = torch.empty(G, 2 * f, d, dtype=dtype, device=DEV)
+    w_dn = torch.empty(G, d, f, dtype=dtype, device=DEV)
+    moe.moe_prepare_weights(wg.to(DEV), wu.to(DEV), wd.to(DEV), None, w_gu, w_dn)
+    out = torch.zeros(m, d, dtype=dtype, device=DEV)
+    ws = torch.empty(moe.moe_expert_ffn_workspace_size(m, f, moe.dtype_code(dtype)),
+                     dtype=torch.uint8, device=DEV)
+    moe.moe_expert_ffn(a.to(DEV), torch.from_numpy(off).to(DEV), w_gu, w_dn, f, None,
+                       moe.MOE_FFN_SWIGLU, out, ws, a_row_index=ridx.to(DEV))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    out = out.float().cpu().numpy()
+    ao = a.double().numpy()
+    ref = np.zeros((m, d))
+    for gi in range(G):
+        for r in range(off[gi], off[gi + 1]):
+            ref[r] = oracle.expert_row(ao[int(ridx[r])], to_oracle(wg[gi]), to_oracle(wu[gi]),
+                                       to_oracle(wd[gi]))
+    assert rowwise_rel_err(out, ref) <= OUT_RTOL
 
 
 def test_bad_expert_id_raises_device_check():
