@@ -14,6 +14,7 @@
 #include "brim.cuh"
 #include "dispatch.cuh"
 #include "ffn_gemm.cuh"
+#include "ffn_gemm_pair.cuh"
 #include "route.cuh"
 
 // The device error flag the kernels raise (bits moe::kErrIndex, kErrTimeout).
@@ -63,6 +64,8 @@ struct DeviceInfo {
   int num_sms = 0;
   unsigned* err_flag = nullptr;
   unsigned smem_attr_done = 0;  // bit per GEMM instantiation
+  unsigned pair_attr_done = 0;  // bit per CTA-pair GEMM instantiation
+  int pair_max_clusters[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -182,6 +185,12 @@ int check_dtype(int dtype) {
 
 int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
 
+int pick_bn(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
+
+// host-side debug bits (test only): force the single-CTA or the CTA-pair GEMM
+constexpr int kDebugForceSingle = 2;
+constexpr int kDebugForcePair = 4;
+
 // ---- GEMM launch ----------------------------------------------------------
 // A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
 // gathered from it (row p = a[a_row_index[p]]), else they are a's first m_cap.
@@ -230,6 +239,76 @@ int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int a_rows, const int3
                                             K, b, G, N, group_off, row_scale, out, ldo, st);
 }
 
+// The same GEMM on CTA pairs (cluster of 2, M = 256 tiles).  Needs BN/2 >= 64.
+template <int BN, int EPI, bool TF32>
+int launch_gemm_pair(DeviceInfo* di, int slot, const void* a, int a_rows, int m_cap, int K,
+                     const void* b, int G, int N, const int32_t* group_off,
+                     const float* row_scale, void* out, int ldo, cudaStream_t st) {
+  using Cfg = moe::PairCfg<BN, TF32>;
+  const int dtype = TF32 ? MOE_F32 : MOE_BF16;
+  CUtensorMap ta, tb;
+  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
+  if (rc) return rc;
+  rc = encode_2d(&tb, b, dtype, (uint64_t)K, (uint64_t)G * N, Cfg::kBK, BN / 2);
+  if (rc) return rc;
+  auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!(di->pair_attr_done & (1u << slot))) {
+    MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)Cfg::kSmemBytes));
+    cfg.gridDim = dim3(2 * (di->num_sms / 2), 1, 1);
+    int clusters = 0;
+    MOE_CUDA(cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg));
+    MOE_REQUIRE(clusters >= 1, MOE_ERR_UNSUPPORTED, "no CTA pair fits on this device");
+    di->pair_max_clusters[slot] = clusters;
+    di->pair_attr_done |= 1u << slot;
+  }
+  const long long ub = ((long long)m_cap / moe::kPairBM + G) * (N / BN);
+  const long long pairs = ub < di->pair_max_clusters[slot] ? (ub < 1 ? 1 : ub)
+                                                            : di->pair_max_clusters[slot];
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  moe::GemmArgs args{group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo,
+                     di->err_flag, wait_limit_ns(), g_debug_flags};
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
+  return MOE_OK;
+}
+
+// GEMM over the groups, on CTA pairs when the groups are tall enough to fill
+// 256-row tiles (and the rows are read in place), else on single CTAs.
+template <int EPI, bool TF32>
+int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_index,
+                     int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
+                     const float* row_scale, void* out, int ldo, cudaStream_t st) {
+  const bool tall = (long long)m_cap >= 192LL * G;
+  bool pair = !a_row_index && N % 128 == 0 && tall;
+  if (g_debug_flags & kDebugForceSingle) pair = false;
+  if ((g_debug_flags & kDebugForcePair) && !a_row_index && N % 128 == 0) pair = true;
+  if (pair) {
+    const int slot = (EPI * 2 + (TF32 ? 1 : 0)) * 2;
+    if (N % 256 == 0)
+      return launch_gemm_pair<256, EPI, TF32>(di, slot, a, a_rows, m_cap, K, b, G, N, group_off,
+                                              row_scale, out, ldo, st);
+    return launch_gemm_pair<128, EPI, TF32>(di, slot + 1, a, a_rows, m_cap, K, b, G, N,
+                                            group_off, row_scale, out, ldo, st);
+  }
+  const int bn = pick_bn(N);
+  if (a_row_index)
+    return launch_gemm_bn<EPI, TF32, true>(di, bn, a, a_rows, a_row_index, m_cap, K, b, G, N,
+                                           group_off, row_scale, out, ldo, st);
+  return launch_gemm_bn<EPI, TF32, false>(di, bn, a, a_rows, nullptr, m_cap, K, b, G, N,
+                                          group_off, row_scale, out, ldo, st);
+}
+
 // How many warps share one token row in the movers: one warp per token when
 // the batch fills the GPU (>= 32 warps per SM), more for small batches.
 int mover_parts(const DeviceInfo* di, int T, int max_parts) {
@@ -239,7 +318,7 @@ int mover_parts(const DeviceInfo* di, int T, int max_parts) {
   return P < 1 ? 1 : P;
 }
 
-int pick_bn(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
+
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -568,29 +647,18 @@ int moe_expert_ffn(const void* a, int a_rows, const int32_t* a_row_index,
   MOE_REQUIRE(aligned16(w_gu) && aligned16(w_dn) && aligned16(ws), MOE_ERR_INVALID_ARG,
               "weights and workspace must be 16-byte aligned");
   void* h = ws;  // [m_cap, f]
-  const int bn1 = pick_bn(2 * f), bn2 = pick_bn(d);
   if (dtype == MOE_BF16) {
-    rc = a_row_index
-             ? launch_gemm_bn<moe::kEpiSwiGLU, false, true>(di, bn1, a, a_rows, a_row_index,
-                                                            m_cap, d, w_gu, G, 2 * f, group_off,
-                                                            nullptr, h, f, stream)
-             : launch_gemm_bn<moe::kEpiSwiGLU, false, false>(di, bn1, a, a_rows, nullptr, m_cap,
-                                                             d, w_gu, G, 2 * f, group_off,
-                                                             nullptr, h, f, stream);
+    rc = launch_gemm_auto<moe::kEpiSwiGLU, false>(di, a, a_rows, a_row_index, m_cap, d, w_gu, G,
+                                                  2 * f, group_off, nullptr, h, f, stream);
     if (rc) return rc;
-    rc = launch_gemm_bn<moe::kEpiScale, false, false>(di, bn2, h, m_cap, nullptr, m_cap, f, w_dn,
-                                                      G, d, group_off, row_scale, out, d, stream);
+    rc = launch_gemm_auto<moe::kEpiScale, false>(di, h, m_cap, nullptr, m_cap, f, w_dn, G, d,
+                                                 group_off, row_scale, out, d, stream);
   } else {
-    rc = a_row_index
-             ? launch_gemm_bn<moe::kEpiSwiGLU, true, true>(di, bn1, a, a_rows, a_row_index,
-                                                           m_cap, d, w_gu, G, 2 * f, group_off,
-                                                           nullptr, h, f, stream)
-             : launch_gemm_bn<moe::kEpiSwiGLU, true, false>(di, bn1, a, a_rows, nullptr, m_cap,
-                                                            d, w_gu, G, 2 * f, group_off,
-                                                            nullptr, h, f, stream);
+    rc = launch_gemm_auto<moe::kEpiSwiGLU, true>(di, a, a_rows, a_row_index, m_cap, d, w_gu, G,
+                                                 2 * f, group_off, nullptr, h, f, stream);
     if (rc) return rc;
-    rc = launch_gemm_bn<moe::kEpiScale, true, false>(di, bn2, h, m_cap, nullptr, m_cap, f, w_dn,
-                                                     G, d, group_off, row_scale, out, d, stream);
+    rc = launch_gemm_auto<moe::kEpiScale, true>(di, h, m_cap, nullptr, m_cap, f, w_dn, G, d,
+                                                group_off, row_scale, out, d, stream);
   }
   return rc;
 }

@@ -74,6 +74,94 @@ struct GemmArgs {
   int debug;
 };
 
+// Epilogue of one accumulator tile for this thread's TMEM lane (= one tile
+// row): tcgen05.ld 32 columns at a time, fused SwiGLU or row scaling, and a
+// masked store of the row.  Every lane of the warp must call it (tcgen05.ld is
+// warp-collective); `valid` masks the stores.
+template <int BN, int EPI, typename TOut>
+__device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t grow, int n0,
+                                              const float* row_scale, TOut* out, int ldo) {
+  if (EPI == kEpiSwiGLU) {
+    // columns [128p, 128p+64) are gate rows, [128p+64, 128p+128) the matching up rows
+#pragma unroll 1
+    for (int p = 0; p < BN / 128; ++p) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t gr[32], ur[32];
+        tc::tmem_ld32(taddr + p * 128 + h * 32, gr);
+        tc::tmem_ld32(taddr + p * 128 + 64 + h * 32, ur);
+        tc::tmem_ld_wait();
+        if (valid) {
+          float hv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gv = __uint_as_float(gr[i]);
+            const float uv = __uint_as_float(ur[i]);
+            hv[i] = gv / (1.0f + __expf(-gv)) * uv;
+          }
+          TOut* dst = out + grow * ldo + (n0 >> 1) + p * 64 + h * 32;
+#pragma unroll
+          for (int v = 0; v < 32 / Vec16<TOut>::n; ++v)
+            st_v4(dst + v * Vec16<TOut>::n, Vec16<TOut>::from_f32(hv + v * Vec16<TOut>::n));
+        }
+      }
+    }
+  } else {
+    const float scale = (valid && row_scale) ? row_scale[grow] : 1.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t vr[32];
+      tc::tmem_ld32(taddr + c * 32, vr);
+      tc::tmem_ld_wait();
+      if (valid) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]) * scale;
+        TOut* dst = out + grow * ldo + n0 + c * 32;
+#pragma unroll
+        for (int q = 0; q < 32 / Vec16<TOut>::n; ++q)
+          st_v4(dst + q * Vec16<TOut>::n, Vec16<TOut>::from_f32(v + q * Vec16<TOut>::n));
+      }
+    }
+  }
+}
+
+// Tile prefix of the groups (one warp): s_off/s_end hold each group's rows
+// (a group whose bounds leave [0, m_cap] or run backwards is treated as empty
+// and raises the index error bit); s_prefix[g] = first tile of group g, where
+// group g has ceil(rows / bm) * n_blocks tiles; s_prefix[G] = all tiles.
+__device__ __forceinline__ void group_tile_prefix(const int32_t* group_off, int G, int m_cap,
+                                                  int bm, int n_blocks, int32_t* s_off,
+                                                  int32_t* s_end, int32_t* s_prefix,
+                                                  unsigned* err) {
+  const unsigned lane = lane_id();
+  int carry = 0;
+  bool bad = false;
+  for (int g0 = 0; g0 < G; g0 += 32) {
+    const int g = g0 + (int)lane;
+    int tiles_g = 0;
+    if (g < G) {
+      const int lo = group_off[g], hi = group_off[g + 1];
+      const bool ok = lo >= 0 && hi >= lo && hi <= m_cap;
+      bad |= !ok;
+      s_off[g] = lo;
+      s_end[g] = ok ? hi : lo;
+      const int rows = ok ? hi - lo : 0;
+      tiles_g = ((rows + bm - 1) / bm) * n_blocks;
+    }
+    int inc = tiles_g;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if ((int)lane >= o) inc += y;
+    }
+    if (g < G) s_prefix[g] = carry + inc - tiles_g;
+    carry += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  if (lane == 0) s_prefix[G] = carry;
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_error(err, kErrIndex);
+}
+
 template <int BN, int EPI, bool TF32, bool GATHER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -317,49 +405,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool valid = r_in_tile < rows;
       const size_t grow = static_cast<size_t>(row0 + r_in_tile);
-      if (EPI == kEpiSwiGLU) {
-        // columns [128p, 128p+64) are gate rows, [128p+64, 128p+128) the matching up rows
-#pragma unroll 1
-        for (int p = 0; p < BN / 128; ++p) {
-#pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            uint32_t gr[32], ur[32];
-            tc::tmem_ld32(taddr + p * 128 + h * 32, gr);
-            tc::tmem_ld32(taddr + p * 128 + 64 + h * 32, ur);
-            tc::tmem_ld_wait();
-            if (valid) {
-              float hv[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float gv = __uint_as_float(gr[i]);
-                const float uv = __uint_as_float(ur[i]);
-                hv[i] = gv / (1.0f + __expf(-gv)) * uv;
-              }
-              TOut* dst = out + grow * args.ldo + (n0 >> 1) + p * 64 + h * 32;
-#pragma unroll
-              for (int v = 0; v < 32 / Vec16<TOut>::n; ++v)
-                st_v4(dst + v * Vec16<TOut>::n, Vec16<TOut>::from_f32(hv + v * Vec16<TOut>::n));
-            }
-          }
-        }
-      } else {
-        const float scale = (valid && args.row_scale) ? args.row_scale[grow] : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t vr[32];
-          tc::tmem_ld32(taddr + c * 32, vr);
-          tc::tmem_ld_wait();
-          if (valid) {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]) * scale;
-            TOut* dst = out + grow * args.ldo + n0 + c * 32;
-#pragma unroll
-            for (int q = 0; q < 32 / Vec16<TOut>::n; ++q)
-              st_v4(dst + q * Vec16<TOut>::n, Vec16<TOut>::from_f32(v + q * Vec16<TOut>::n));
-          }
-        }
-      }
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args.row_scale, out, args.ldo);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tc::smem_u32(&tempty_bar[acc]));

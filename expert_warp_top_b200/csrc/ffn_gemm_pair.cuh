@@ -1,0 +1,262 @@
+// ffn_gemm_pair.cuh -- the grouped expert GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same computation as ffn_gemm.cuh (one expert group per tile, SwiGLU or
+// gate-scaled epilogue), but a cluster of two CTAs works on a 256-row tile:
+// each CTA holds its own 128 rows of A and one half (BN/2 rows) of the weight
+// tile B, and one tcgen05.mma with M = 256 multiplies the pair's A by the whole
+// B.  Per SM this halves the B bytes that TMA has to bring in (32 KB per
+// k-block instead of 48 KB at BN = 256), which leaves room for a 6-deep
+// shared-memory ring and lets the tensor pipe run closer to its peak.
+//
+// Roles, in both CTAs unless noted:
+//   warp 0      TMA producer for this CTA's A rows and B half, into its own
+//               shared memory (no multicast); both CTAs' loads count their
+//               bytes on CTA 0's full barrier, which CTA 0 arms for the pair
+//   warp 1      CTA 0 only: MMA issuer for the pair
+//   warps 2..5  epilogue of this CTA's 128 accumulator rows (its own TMEM)
+// Hand-offs across the pair: the MMA issuer's commits arrive on the empty and
+// tfull barriers of both CTAs (multicast commit); CTA 1's epilogue warps
+// arrive remotely on CTA 0's tempty barrier.  Every wait is bounded; a pair
+// that gives up unwinds, drains its MMAs, meets at a cluster barrier and
+// frees TMEM.
+#pragma once
+#include "ffn_gemm.cuh"
+
+namespace moe {
+
+constexpr int kPairBM = 256;  // rows per pair tile, 128 per CTA
+
+template <int BN, bool TF32>
+struct PairCfg {
+  static constexpr int kElemBytes = TF32 ? 4 : 2;
+  static constexpr int kBK = 128 / kElemBytes;
+  static constexpr int kMmaK = 32 / kElemBytes;
+  static constexpr int kMmaPerStage = kBK / kMmaK;
+  static constexpr int kABytes = 128 * 128;          // this CTA's 128 rows of A
+  static constexpr int kBBytes = (BN / 2) * 128;     // this CTA's half of B
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 512 +
+                                       sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
+};
+
+template <int BN, int EPI, bool TF32>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                         const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+  static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
+  using Cfg = PairCfg<BN, TF32>;
+  using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
+  constexpr int S = Cfg::kStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * Cfg::kStageBytes);
+  uint64_t* full_bar = bars;                 // [S] CTA 0: both CTAs' TMA -> MMA
+  uint64_t* empty_bar = bars + S;            // [S] MMA (multicast) -> producers
+  uint64_t* tfull_bar = bars + 2 * S;        // [2] MMA (multicast) -> epilogues
+  uint64_t* tempty_bar = bars + 2 * S + 2;   // [2] CTA 0 only: 8 epilogue warps -> MMA
+  uint64_t* drain_bar = bars + 2 * S + 4;    // [1] MMA drain at teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_off = reinterpret_cast<int32_t*>(smem + (size_t)S * Cfg::kStageBytes + 512);
+  int32_t* s_end = s_off + kGemmMaxGroups;
+  int32_t* s_prefix = s_end + kGemmMaxGroups;
+
+  const int warp = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  const uint32_t rank = tc::cluster_ctarank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int G = args.G;
+  const int n_blocks = args.N / BN;
+  const int k_blocks = args.K / Cfg::kBK;
+
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmap_a);
+    tc::tma_prefetch_desc(&tmap_b);
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
+      tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(tc::smem_u32(&tfull_bar[a]), 1);
+      tc::mbar_init(tc::smem_u32(&tempty_bar[a]), 8);  // 4 epilogue warps x 2 CTAs
+    }
+    tc::mbar_init(tc::smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    tc::mbar_init_fence();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc_pair(tc::smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc::tmem_relinquish_pair();
+  }
+  if (warp == 2)
+    group_tile_prefix(args.group_off, G, args.m_cap, kPairBM, n_blocks, s_off, s_end, s_prefix,
+                      args.err);
+  tc::fence_before_sync();
+  __syncwarp();
+  tc::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = s_prefix[G];
+  const tc::WaitCtl wctl{abort_flag, args.err, args.wait_limit_ns};
+
+  auto locate = [&](int tile, int& g, int& row0, int& gend, int& n0) {
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_prefix[mid] <= tile) lo = mid;
+      else hi = mid;
+    }
+    g = lo;
+    const int local = tile - s_prefix[g];
+    const int gstart = s_off[g];
+    gend = s_end[g];
+    const int m_blocks = (gend - gstart + kPairBM - 1) / kPairBM;
+    const int nb = local / m_blocks, mb = local - nb * m_blocks;
+    row0 = gstart + mb * kPairBM;
+    n0 = nb * BN;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_a = tc::policy_evict_normal();
+      const uint64_t pol_b = tc::policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_parity = 0;
+      bool skip_next = (args.debug & kDebugSkipFirstLoad) != 0 && rank == 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        int g, row0, gend, n0;
+        locate(tile, g, row0, gend, n0);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl)) {
+            ok = false;
+            break;
+          }
+          if (!skip_next) {
+            const uint32_t fb = tc::smem_u32(&full_bar[stage]);
+            const uint32_t fb_pair = tc::mapa_shared(fb, 0);  // the barrier in CTA 0
+            uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
+            if (rank == 0) tc::mbar_arrive_expect_tx(fb, 2 * Cfg::kStageBytes);
+            tc::tma_load_2d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, kb * Cfg::kBK,
+                                 row0 + (int)rank * 128, pol_a);
+            tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
+                                 kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          }
+          skip_next = false;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // CTA 0 waits for the last arming of every stage (its bytes include CTA 1's)
+      if (rank == 0)
+        for (int s = 0; s < S; ++s)
+          if ((armed >> s) & 1u)
+            tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = tc::idesc_f32acc<TF32, 256, BN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        if (!tc::wait_bounded_cluster(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl)) break;
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!tc::wait_bounded_cluster(tc::smem_u32(&full_bar[stage]), phase, wctl)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t sa = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
+          const uint64_t adesc = tc::desc_sw128_kmajor(sa);
+          const uint64_t bdesc = tc::desc_sw128_kmajor(sa + Cfg::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(kk * 2);
+            if (TF32)
+              tc::mma_tf32_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+            else
+              tc::mma_f16_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+          }
+          // frees this stage in both CTAs once these MMAs have read it
+          tc::commit_pair_multicast(tc::smem_u32(&empty_bar[stage]), 0x3);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::commit_pair_multicast(tc::smem_u32(&tfull_bar[acc]), 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc::commit_pair_multicast(tc::smem_u32(drain_bar), 0x1);
+      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int r_in_half = quarter * 32 + (int)lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    TOut* out = reinterpret_cast<TOut*>(args.out);
+    const uint32_t tempty_local = tc::smem_u32(&tempty_bar[0]);
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      int g, row0, gend, n0;
+      locate(tile, g, row0, gend, n0);
+      bool ok = true;
+      if (lane == 0) ok = tc::wait_bounded(tc::smem_u32(&tfull_bar[acc]), acc_phase, wctl);
+      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+      if (!ok) break;
+      __syncwarp();
+      tc::fence_after_sync();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      const int grow_i = row0 + (int)rank * 128 + r_in_half;
+      const bool valid = grow_i < gend;
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, static_cast<size_t>(grow_i), n0, args.row_scale,
+                                   out, args.ldo);
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t bar = tempty_local + static_cast<uint32_t>(acc * sizeof(uint64_t));
+        if (rank == 0) tc::mbar_arrive(bar);
+        else tc::mbar_arrive_remote(tc::mapa_shared(bar, 0));
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  // Both CTAs meet here only after their own work is done and the MMA issuer
+  // has drained, so no MMA still reads the peer's shared memory or TMEM.
+  tc::fence_before_sync();
+  __syncwarp();
+  tc::cluster_sync();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -162,6 +162,33 @@ def test_multi_tile_layers(cfg):
     run_and_check_small(cfg)
 
 
+# test-only switches of the library: force the single-CTA or the CTA-pair GEMM
+FORCE_SINGLE, FORCE_PAIR = 2, 4
+
+
+@pytest.fixture
+def gemm_variant(request):
+    moe.moe_set_debug(request.param, 4000.0)
+    yield request.param
+    moe.moe_set_debug(0, 4000.0)
+
+
+@pytest.mark.parametrize("gemm_variant", [FORCE_SINGLE, FORCE_PAIR], indirect=True)
+@pytest.mark.parametrize("cfg", [
+    # 256-row pair tiles over ragged groups, BN = 256 / 256
+    inputs.LayerConfig("pair", T=1500, d=256, f=256, E=8, k=2, R=4, seed=21),
+    # BN = 128 in both GEMMs (2f = 384, d = 384), skewed groups, shared experts
+    inputs.LayerConfig("pair128", T=1100, d=384, f=192, E=16, k=4, R=4, bias_std=1.5,
+                       S=1, fs=128, seed=22),
+    # TF32 on pairs
+    inputs.LayerConfig("pairf32", T=800, d=256, f=128, E=4, k=2, R=2, dtype="f32", seed=23),
+    # tiny groups: most pair tiles are mostly empty
+    inputs.LayerConfig("pairsmall", T=40, d=128, f=128, E=16, k=4, R=4, seed=24),
+], ids=["pair", "pair128", "pairf32", "pairsmall"])
+def test_gemm_variants(cfg, gemm_variant):
+    run_and_check_small(cfg)
+
+
 @pytest.mark.parametrize("T,E,k,R", [(1, 8, 2, 4), (2, 64, 6, 8), (257, 8, 2, 1),
                                      (300, 8, 2, 8), (100, 256, 16, 8), (513, 64, 8, 64)])
 def test_edge_shapes(T, E, k, R):
