@@ -134,11 +134,12 @@ def launches_per_step(cfg) -> int:
     return 1 + 3 + 1 + 2 + (2 if cfg.S else 0) + 1 + 1 + 1
 
 
-def cpu_baseline(cfg, budget_s: float = 12.0):
+def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
     """The oracle as it stands, on a bounded sample of the same workload's tokens:
     routing + BRIM build + the dense layer on the sampled tokens."""
     import oracle
-    inp = inputs.make_inputs(cfg, device="cpu", weights=True)
+    if inp is None:
+        inp = inputs.make_inputs(cfg, device="cpu", weights=True)
 
     def bits(t):
         t = t.contiguous()
@@ -174,8 +175,9 @@ def run_reference(args, cfg):
     import oracle
     per_step = []
     budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    inp = inputs.make_inputs(cfg, device="cpu", weights=True)
     for i in range(args.warmup + args.steps):
-        res = cpu_baseline(cfg, budget_s=budget)
+        res = cpu_baseline(cfg, budget_s=budget, inp=inp)
         if i >= args.warmup:
             per_step.append(res)
     value = statistics.median([r["value"] for r in per_step])
@@ -355,32 +357,23 @@ def run_ours(args, cfg):
 
 
 def e2e_host(layer, inp, cfg, args, dev, world):
-    """Host-buffer end to end: H2D of logits and x, the layer, D2H of y, per step."""
+    """End to end through moe_layer_forward_host: each step copies that step's
+    logits and activations from pinned host memory, runs the whole layer and
+    copies y back to pinned host memory, then synchronises (host wall clock)."""
     h_logits = inp["logits"].cpu().pin_memory()
     h_x = inp["x"].cpu().pin_memory()
     h_y = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
-    stream = torch.cuda.current_stream(dev)
-    d_logits = torch.empty_like(inp["logits"])
-    d_x = torch.empty_like(inp["x"])
-
-    def step():
-        d_logits.copy_(h_logits, non_blocking=True)
-        d_x.copy_(h_x, non_blocking=True)
-        y = layer.forward(d_logits, d_x)
-        h_y.copy_(y, non_blocking=True)
-
-    for _ in range(max(1, args.warmup)):
-        step()
+    for _ in range(args.warmup):
+        layer.forward_host(h_logits, h_x, h_y)
     torch.cuda.synchronize(dev)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(args.steps):
-        step()
-    e.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = s.elapsed_time(e)
     if world > 1:
         import torch.distributed as dist
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        layer.forward_host(h_logits, h_x, h_y)
+    ms = (time.perf_counter() - t0) * 1e3
+    if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
@@ -388,7 +381,7 @@ def e2e_host(layer, inp, cfg, args, dev, world):
     d2h = h_y.numel() * h_y.element_size()
     return {"value": world * cfg.T * args.steps / (ms * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "api": "MoELayer.forward with pinned host copies"}
+            "api": "moe_layer_forward_host (C ABI, pinned host buffers, wall clock)"}
 
 
 def main():

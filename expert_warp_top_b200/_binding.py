@@ -33,6 +33,7 @@ EXPORTS = (
     "moe_dispatch_gather",
     "moe_prepare_weights", "moe_prepare_shared_weights", "moe_expert_ffn_workspace_size",
     "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
+    "moe_layer_workspace_size", "moe_layer_forward", "moe_layer_forward_host",
 )
 
 
@@ -58,6 +59,7 @@ def load():
         lib.moe_last_error.restype = ctypes.c_char_p
         lib.moe_brim_workspace_size.restype = ctypes.c_size_t
         lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
+        lib.moe_layer_workspace_size.restype = ctypes.c_size_t
         lib.moe_set_debug.argtypes = [ctypes.c_int, ctypes.c_double]
         for name in EXPORTS:
             getattr(lib, name)
@@ -214,3 +216,48 @@ def moe_coact_histogram(topk_idx, E, hist, accumulate, stream=None):
     _check("moe_coact_histogram", load().moe_coact_histogram(
         _ptr(topk_idx, I32, "topk_idx"), T, k, int(E), _ptr(hist, (U32, torch.int32), "hist"),
         int(accumulate), _stream(stream)))
+
+
+def _host_ptr(t: torch.Tensor, dtype, name: str) -> ctypes.c_void_p:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def moe_layer_workspace_size(T, d, f, E, k, R, S, fs, dtype_code_, host_staging) -> int:
+    return int(load().moe_layer_workspace_size(int(T), int(d), int(f), int(E), int(k), int(R),
+                                               int(S), int(fs), int(dtype_code_),
+                                               int(host_staging)))
+
+
+def moe_layer_forward(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, y, ws, sw_gu=None,
+                      sw_dn=None, S=0, fs=0, c_t=None, per_rank=None, total=None, remote=None,
+                      hist=None, stream=None):
+    T, E = logits.shape
+    d = x.shape[1]
+    _check("moe_layer_forward", load().moe_layer_forward(
+        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(S), int(fs),
+        dtype_code(x.dtype), _ptr(logits, F32, "logits"), _ptr(x, _ACT, "x"),
+        _ptr(slot_of, I32, "slot_of"), _ptr(w_gu, x.dtype, "w_gu"), _ptr(w_dn, x.dtype, "w_dn"),
+        _ptr(sw_gu, x.dtype, "sw_gu"), _ptr(sw_dn, x.dtype, "sw_dn"), _ptr(y, x.dtype, "y"),
+        _ptr(c_t, I32, "c_t"), _ptr(per_rank, I32, "per_rank"), _ptr(total, I64, "total"),
+        _ptr(remote, I64, "remote"), _ptr(hist, (U32, torch.int32), "hist"),
+        _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
+
+
+def moe_layer_forward_host(h_logits, h_x, k, R, renorm, slot_of, w_gu, w_dn, f, h_y, ws,
+                           sw_gu=None, sw_dn=None, S=0, fs=0, stream=None):
+    """The layer on host buffers: H2D copies, every step, D2H copy, then synchronise."""
+    T, E = h_logits.shape
+    d = h_x.shape[1]
+    _check("moe_layer_forward_host", load().moe_layer_forward_host(
+        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(S), int(fs),
+        dtype_code(h_x.dtype), _host_ptr(h_logits, F32, "h_logits"), _host_ptr(h_x, _ACT, "h_x"),
+        _ptr(slot_of, I32, "slot_of"), _ptr(w_gu, h_x.dtype, "w_gu"),
+        _ptr(w_dn, h_x.dtype, "w_dn"), _ptr(sw_gu, h_x.dtype, "sw_gu"),
+        _ptr(sw_dn, h_x.dtype, "sw_dn"), _host_ptr(h_y, h_x.dtype, "h_y"),
+        _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))

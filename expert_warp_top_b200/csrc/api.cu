@@ -724,3 +724,207 @@ int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// The whole layer.  The workspace is carved into the layer's intermediate
+// state, every region 256-byte aligned.
+__global__ void set_pair_kernel(int32_t* p, int a, int b) {
+  p[0] = a;
+  p[1] = b;
+}
+
+namespace {
+
+struct LayerCarve {
+  size_t off = 0;
+  char* base = nullptr;
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align256(sizeof(T) * (count ? count : 1));
+    return p;
+  }
+};
+
+struct LayerState {
+  float* logits; void* x; void* y;   // host staging (host variant only)
+  int32_t* topk_idx; float* topk_w;
+  int32_t *brim0, *sfd_token, *sfd_off, *brim1, *epd_off, *epd_sfd; float* epd_gate;
+  int32_t* c_t; void* brim_ws; size_t brim_ws_bytes;
+  void *x_sfd, *x_epd, *o_epd, *y_sfd, *shared_out;
+  void* ffn_ws; size_t ffn_ws_bytes; void* sffn_ws; size_t sffn_ws_bytes;
+  int32_t* shared_off;
+  int32_t* per_rank; int64_t* total; int64_t* remote; uint32_t* hist;
+};
+
+size_t carve_layer(char* base, int T, int d, int f, int E, int k, int R, int S, int fs,
+                   int dtype, bool host, LayerState* st) {
+  LayerCarve c;
+  c.base = base;
+  LayerState s{};
+  const int es = esize(dtype);
+  const size_t cap = (size_t)T * (k < R ? k : R), tk = (size_t)T * k;
+  const int L = E / R;
+  if (host) {
+    s.logits = c.take<float>((size_t)T * E);
+    s.x = c.take<char>((size_t)T * d * es);
+    s.y = c.take<char>((size_t)T * d * es);
+  }
+  s.topk_idx = c.take<int32_t>(tk);
+  s.topk_w = c.take<float>(tk);
+  s.brim0 = c.take<int32_t>((size_t)R * T);
+  s.sfd_token = c.take<int32_t>(cap);
+  s.sfd_off = c.take<int32_t>(R + 1);
+  s.brim1 = c.take<int32_t>((size_t)L * cap);
+  s.epd_off = c.take<int32_t>(E + 1);
+  s.epd_sfd = c.take<int32_t>(tk);
+  s.epd_gate = c.take<float>(tk);
+  s.c_t = c.take<int32_t>(1);
+  s.brim_ws_bytes = moe_brim_workspace_size(T, E, R);
+  s.brim_ws = c.take<char>(s.brim_ws_bytes);
+  s.x_sfd = c.take<char>(cap * d * es);
+  s.x_epd = L > 1 ? c.take<char>(tk * d * es) : nullptr;
+  s.o_epd = c.take<char>(tk * d * es);
+  s.y_sfd = c.take<char>(cap * d * es);
+  s.ffn_ws_bytes = moe_expert_ffn_workspace_size((int)(tk ? tk : 1), f, dtype);
+  s.ffn_ws = c.take<char>(s.ffn_ws_bytes);
+  if (S > 0) {
+    s.shared_out = c.take<char>((size_t)T * d * es);
+    s.sffn_ws_bytes = moe_expert_ffn_workspace_size(T ? T : 1, S * fs, dtype);
+    s.sffn_ws = c.take<char>(s.sffn_ws_bytes);
+    s.shared_off = c.take<int32_t>(2);
+  }
+  s.per_rank = c.take<int32_t>(R);
+  s.total = c.take<int64_t>(1);
+  s.remote = c.take<int64_t>(1);
+  s.hist = c.take<uint32_t>((size_t)E * E);
+  if (!host) {
+    s.logits = nullptr;
+    s.x = s.y = nullptr;
+  }
+  if (st) *st = s;
+  return c.off + 256;
+}
+
+int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs, int dtype,
+                const float* logits, const void* x, const int32_t* slot_of, const void* w_gu,
+                const void* w_dn, const void* sw_gu, const void* sw_dn, void* y, int32_t* c_t_out,
+                int32_t* per_rank, int64_t* total, int64_t* remote, uint32_t* hist,
+                const LayerState& st, cudaStream_t stream) {
+  const int L = E / R;
+  const size_t tk = (size_t)T * k;
+  const size_t cap = (size_t)T * (k < R ? k : R);
+  int rc;
+  if ((rc = moe_route_topk(logits, T, E, k, renorm, st.topk_idx, st.topk_w, stream))) return rc;
+  if ((rc = moe_brim_build(st.topk_idx, st.topk_w, T, k, slot_of, E, R, st.brim0, st.sfd_token,
+                           st.sfd_off, st.brim1, st.epd_off, st.epd_sfd, st.epd_gate, st.c_t,
+                           st.brim_ws, st.brim_ws_bytes, stream)))
+    return rc;
+  if ((rc = moe_dispatch_gather(x, T, d, dtype, k, R, L, st.brim0, st.brim1, st.x_sfd, st.x_epd,
+                                stream)))
+    return rc;
+  // with L = 1 the EPD state is the SFD state row for row: run on the payload
+  const void* a = L > 1 ? st.x_epd : st.x_sfd;
+  const int a_rows = (int)(L > 1 ? (tk ? tk : 1) : (cap ? cap : 1));
+  if ((rc = moe_expert_ffn(a, a_rows, nullptr, st.epd_off, E, (int)(tk ? tk : 1), w_gu, w_dn, d,
+                           f, dtype, st.epd_gate, MOE_FFN_SWIGLU, st.o_epd, st.ffn_ws,
+                           st.ffn_ws_bytes, stream)))
+    return rc;
+  if (S > 0) {
+    set_pair_kernel<<<1, 1, 0, stream>>>(st.shared_off, 0, T);  // the one shared group: [0, T)
+    MOE_LAUNCHED("set_pair_kernel");
+    if ((rc = moe_expert_ffn(x, T, nullptr, st.shared_off, 1, T, sw_gu, sw_dn, d, S * fs, dtype,
+                             nullptr, MOE_FFN_SWIGLU, st.shared_out, st.sffn_ws,
+                             st.sffn_ws_bytes, stream)))
+      return rc;
+  }
+  if ((rc = moe_combine_scatter(st.o_epd, T, d, dtype, k, R, L, st.brim0, st.brim1,
+                                S > 0 ? st.shared_out : nullptr, st.y_sfd, y, stream)))
+    return rc;
+  if ((rc = moe_count_dispatched_rows(st.topk_idx, T, k, slot_of, E, R,
+                                      per_rank ? per_rank : st.per_rank, total ? total : st.total,
+                                      remote ? remote : st.remote, stream)))
+    return rc;
+  if ((rc = moe_coact_histogram(st.topk_idx, T, k, E, hist ? hist : st.hist, hist ? 1 : 0,
+                                stream)))
+    return rc;
+  if (c_t_out) MOE_CUDA(cudaMemcpyAsync(c_t_out, st.c_t, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                                        stream));
+  return MOE_OK;
+}
+
+int check_layer_args(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                     int dtype) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  if ((rc = check_dtype(dtype))) return rc;
+  MOE_REQUIRE(renorm == 0 || renorm == 1, MOE_ERR_INVALID_ARG, "renorm must be 0 or 1");
+  MOE_REQUIRE(d >= 64 && d % 64 == 0 && f >= 64 && f % 64 == 0, MOE_ERR_UNSUPPORTED,
+              "d and f must be positive multiples of 64 (d=%d f=%d)", d, f);
+  MOE_REQUIRE(S >= 0 && (S == 0 || (fs >= 64 && fs % 64 == 0)), MOE_ERR_UNSUPPORTED,
+              "shared experts need fs a positive multiple of 64 (S=%d fs=%d)", S, fs);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_layer_workspace_size(int T, int d, int f, int E, int k, int R, int S, int fs,
+                                int dtype, int host_staging) {
+  if (check_layer_args(T, d, f, E, k, R, 0, S, fs, dtype)) return 0;
+  return carve_layer(nullptr, T, d, f, E, k, R, S, fs, dtype, host_staging != 0, nullptr);
+}
+
+int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                      int dtype, const float* logits, const void* x, const int32_t* slot_of,
+                      const void* w_gu, const void* w_dn, const void* sw_gu, const void* sw_dn,
+                      void* y, int32_t* c_t, int32_t* per_rank, int64_t* total, int64_t* remote,
+                      uint32_t* hist, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_layer_args(T, d, f, E, k, R, renorm, S, fs, dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(ws && aligned16(ws), MOE_ERR_INVALID_ARG, "workspace missing or misaligned");
+  const size_t need = carve_layer(nullptr, T, d, f, E, k, R, S, fs, dtype, false, nullptr);
+  MOE_REQUIRE(ws_bytes >= need, MOE_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes",
+              ws_bytes, need);
+  MOE_REQUIRE(S == 0 || (sw_gu && sw_dn), MOE_ERR_INVALID_ARG, "shared weights missing");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(logits && x && y && slot_of && w_gu && w_dn, MOE_ERR_INVALID_ARG, "null pointer");
+  char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  LayerState st;
+  carve_layer(base, T, d, f, E, k, R, S, fs, dtype, false, &st);
+  return layer_steps(T, d, f, E, k, R, renorm, S, fs, dtype, logits, x, slot_of, w_gu, w_dn,
+                     sw_gu, sw_dn, y, c_t, per_rank, total, remote, hist, st, stream);
+}
+
+int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                           int dtype, const float* h_logits, const void* h_x,
+                           const int32_t* slot_of, const void* w_gu, const void* w_dn,
+                           const void* sw_gu, const void* sw_dn, void* h_y, void* ws,
+                           size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_layer_args(T, d, f, E, k, R, renorm, S, fs, dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(ws && aligned16(ws), MOE_ERR_INVALID_ARG, "workspace missing or misaligned");
+  const size_t need = carve_layer(nullptr, T, d, f, E, k, R, S, fs, dtype, true, nullptr);
+  MOE_REQUIRE(ws_bytes >= need, MOE_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes",
+              ws_bytes, need);
+  MOE_REQUIRE(S == 0 || (sw_gu && sw_dn), MOE_ERR_INVALID_ARG, "shared weights missing");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(h_logits && h_x && h_y && slot_of && w_gu && w_dn, MOE_ERR_INVALID_ARG,
+              "null pointer");
+  char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  LayerState st;
+  carve_layer(base, T, d, f, E, k, R, S, fs, dtype, true, &st);
+  const size_t xb = (size_t)T * d * esize(dtype);
+  MOE_CUDA(cudaMemcpyAsync(st.logits, h_logits, sizeof(float) * (size_t)T * E,
+                           cudaMemcpyHostToDevice, stream));
+  MOE_CUDA(cudaMemcpyAsync(st.x, h_x, xb, cudaMemcpyHostToDevice, stream));
+  rc = layer_steps(T, d, f, E, k, R, renorm, S, fs, dtype, st.logits, st.x, slot_of, w_gu, w_dn,
+                   sw_gu, sw_dn, st.y, nullptr, nullptr, nullptr, nullptr, nullptr, st, stream);
+  if (rc) return rc;
+  MOE_CUDA(cudaMemcpyAsync(h_y, st.y, xb, cudaMemcpyDeviceToHost, stream));
+  MOE_CUDA(cudaStreamSynchronize(stream));
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -155,3 +155,33 @@ class MoELayer:
         if stats:
             self.statistics(stream)
         return self.y
+
+    # -- the whole layer through one C call ---------------------------------
+    def _layer_ws(self, host: bool):
+        key = "_ws_host" if host else "_ws_dev"
+        ws = getattr(self, key, None)
+        if ws is None:
+            n = B.moe_layer_workspace_size(self.T, self.d, self.f, self.E, self.k, self.R, self.S,
+                                           self.fs, B.dtype_code(self.dtype), int(host))
+            ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.y.device)
+            setattr(self, key, ws)
+        return ws
+
+    def forward_fused(self, logits, x, y=None, stream=None):
+        """All steps in one moe_layer_forward call (state in a layer workspace)."""
+        y = self.y if y is None else y
+        B.moe_layer_forward(logits, x, self.k, self.R, self.renorm, self.slot_of, self.w_gu,
+                            self.w_dn, self.f, y, self._layer_ws(False),
+                            sw_gu=getattr(self, "sw_gu", None), sw_dn=getattr(self, "sw_dn", None),
+                            S=self.S, fs=self.fs, c_t=self.c_t, per_rank=self.per_rank,
+                            total=self.total, remote=self.remote, hist=self.hist, stream=stream)
+        return y
+
+    def forward_host(self, h_logits, h_x, h_y, stream=None):
+        """Host buffers in and out through moe_layer_forward_host (synchronises)."""
+        B.moe_layer_forward_host(h_logits, h_x, self.k, self.R, self.renorm, self.slot_of,
+                                 self.w_gu, self.w_dn, self.f, h_y, self._layer_ws(True),
+                                 sw_gu=getattr(self, "sw_gu", None),
+                                 sw_dn=getattr(self, "sw_dn", None), S=self.S, fs=self.fs,
+                                 stream=stream)
+        return h_y

@@ -277,6 +277,47 @@ int moe_count_dispatched_rows(const int32_t* topk_idx, int T, int k,
 int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* hist,
                         int accumulate, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_layer_forward -- the whole layer in one call, every step of the hot
+ * path in order on `stream`: moe_route_topk, moe_brim_build,
+ * moe_dispatch_gather, moe_expert_ffn (routed experts over the EPD groups,
+ * then the S shared experts over the ORI rows), moe_combine_scatter,
+ * moe_count_dispatched_rows and moe_coact_histogram.
+ *   logits [T, E] f32, x [T, d] dtype, y [T, d] dtype  (device)
+ *   slot_of [E] int32 (device) placement used to pack w_gu / w_dn
+ *   w_gu, w_dn   routed weights packed by moe_prepare_weights with slot_of
+ *   sw_gu, sw_dn shared weights packed by moe_prepare_shared_weights
+ *                (S shared experts of width fs; NULL when S = 0)
+ *   stats        optional device outputs, each may be NULL:
+ *                c_t [1] int32; per_rank [R] int32, total [1] int64,
+ *                remote [1] int64 (the dispatched-row counter);
+ *                hist [E, E] uint32 (the co-activation histogram is ADDED
+ *                to it).  Outputs left NULL are still computed, into the
+ *                workspace.
+ *   ws           at least moe_layer_workspace_size(...) bytes, 256-byte aligned;
+ *                it holds every intermediate state (top-k, BRIMs, SFD / EPD
+ *                rows, return rows) for the duration of the call
+ * With one expert per rank (E == R) the GEMM reads the SFD payload in place
+ * (the EPD state equals it row for row); otherwise the dispatch stores the
+ * EPD rows.
+ * moe_layer_forward_host -- the same, with logits, x and y in HOST memory
+ * (pinned memory makes the copies asynchronous DMA): copies logits and x to
+ * device staging in the workspace, runs the layer, copies y back and
+ * synchronises `stream` before returning (one cudaMemcpyAsync per buffer).
+ * ------------------------------------------------------------------------- */
+size_t moe_layer_workspace_size(int T, int d, int f, int E, int k, int R, int S, int fs,
+                                int dtype, int host_staging);
+int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                      int dtype, const float* logits, const void* x, const int32_t* slot_of,
+                      const void* w_gu, const void* w_dn, const void* sw_gu, const void* sw_dn,
+                      void* y, int32_t* c_t, int32_t* per_rank, int64_t* total, int64_t* remote,
+                      uint32_t* hist, void* ws, size_t ws_bytes, moe_stream_t stream);
+int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                           int dtype, const float* h_logits, const void* h_x,
+                           const int32_t* slot_of, const void* w_gu, const void* w_dn,
+                           const void* sw_gu, const void* sw_dn, void* h_y,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
