@@ -38,6 +38,25 @@ import torch  # noqa: E402
 from expert_warp_top_b200 import inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (route+BRIM dispatch+grouped GEMM+combine)"
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
+# GEMM launches of one layer step, from one ncu capture (profiles/ffn_gemm_pair_olmoe.md),
+# valid only while the GEMM sources hash to `src`; otherwise reported as null.
+GEMM_TRAFFIC = {"olmoe": {"bytes": 1178.5e6, "src": "b458d748954b8030"}}
+
+
+def gemm_src_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("ffn_gemm.cuh", "ffn_gemm_pair.cuh", "tc_ptx.cuh"):
+        with open(os.path.join(ROOT, "expert_warp_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def gemm_traffic(cfg):
+    rec = GEMM_TRAFFIC.get(cfg.name)
+    return rec["bytes"] if rec and rec["src"] == gemm_src_hash() else None
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -212,11 +231,13 @@ def run_ours(args, cfg):
                                 device_id=dev)
     # each rank: its own independent batch (seed offset by rank), same weights recipe
     inp = inputs.make_inputs(cfg, device=dev, seed=cfg.seed + 7919 * rank)
+    slot_of, placement_info = placement(cfg, args.placement, dev, inp["logits"])
     kw = dict(wg=inp.pop("wg"), wu=inp.pop("wu"), wd=inp.pop("wd"))
     if cfg.S:
         kw.update(sg=inp.pop("sg"), su=inp.pop("su"), sd=inp.pop("sd"))
     layer = MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
-                     dtype=inputs.torch_dtype(cfg), S=cfg.S, fs=cfg.fs, device=dev, **kw)
+                     dtype=inputs.torch_dtype(cfg), S=cfg.S, fs=cfg.fs, slot_of=slot_of,
+                     device=dev, **kw)
     del kw
     logits, x = inp["logits"], inp["x"]
     stream = torch.cuda.current_stream(dev)
@@ -325,7 +346,7 @@ def run_ours(args, cfg):
     roof = {"bound": "tensor", "kernel": "ffn_gemm_kernel (routed experts: gate/up GEMM with "
             "SwiGLU epilogue + down GEMM with gate scaling, 2 launches)",
             "achieved": achieved, "peak": pk["bf16_sust"], "unit": "TFLOP/s",
-            "frac": achieved / pk["bf16_sust"], "traffic": None,
+            "frac": achieved / pk["bf16_sust"], "traffic": gemm_traffic(cfg),
             "peak_source": f"{pk['source']} bf16 sustained"}
     layer_roof_s = max(flops / (pk["bf16_sust"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
     cpu = None
@@ -339,7 +360,7 @@ def run_ours(args, cfg):
             "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} "
                                    f"k={cfg.k} R={cfg.R} S={cfg.S}",
-                       "placement": "contiguous", "l2": "flushed between steps "
+                       "placement": placement_info, "l2": "flushed between steps "
                        "(256 MiB write outside the per-step events)",
                        "parallelism": f"{world} independent replicas"},
             "roofline": roof,
@@ -354,6 +375,42 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def placement(cfg, how, dev, logits):
+    """slot_of for the run.  "histogram": correlated placement from the expert
+    co-activation histogram of a separate calibration batch (T = 32768, seed 1),
+    routed and counted on the GPU, placed by moe_place_greedy; reports the C_T
+    of the evaluation batch under contiguous and under this placement."""
+    from expert_warp_top_b200 import _binding as B
+    ident = torch.arange(cfg.E, dtype=torch.int32)
+    if how == "contiguous":
+        return ident, "contiguous"
+    calib = cfg.with_(T=32768, seed=1)
+    c_logits = inputs.make_logits(calib, device=dev)
+    idx = torch.empty(calib.T, calib.k, dtype=torch.int32, device=dev)
+    w = torch.empty(calib.T, calib.k, dtype=torch.float32, device=dev)
+    B.moe_route_topk(c_logits, calib.k, 0, idx, w)
+    hist = torch.zeros(cfg.E, cfg.E, dtype=torch.int32, device=dev)
+    B.moe_coact_histogram(idx, cfg.E, hist, 0)
+    slot_of = B.moe_place_greedy(hist, cfg.R)
+    # C_T of the evaluation batch under both placements (the counter kernel)
+    e_idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    e_w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
+    B.moe_route_topk(logits, cfg.k, cfg.renorm, e_idx, e_w)
+    per = torch.empty(cfg.R, dtype=torch.int32, device=dev)
+    tot = torch.empty(1, dtype=torch.int64, device=dev)
+    rem = torch.empty(1, dtype=torch.int64, device=dev)
+    out = {}
+    for name, s in (("contiguous", ident), ("histogram", slot_of)):
+        B.moe_count_dispatched_rows(e_idx, s.to(dev), cfg.E, cfg.R, per, tot, rem)
+        out[name] = int(tot.item())
+    tk = cfg.T * cfg.k
+    return slot_of, {"placement": "histogram (calibration batch T=32768, seed 1)",
+                     "c_t_contiguous": out["contiguous"], "c_t_histogram": out["histogram"],
+                     "tk_rows": tk,
+                     "row_reduction_vs_per_expert": 1 - out["histogram"] / tk,
+                     "row_reduction_vs_contiguous": 1 - out["histogram"] / out["contiguous"]}
 
 
 def e2e_host(layer, inp, cfg, args, dev, world):
@@ -392,6 +449,7 @@ def main():
     ap.add_argument("--config", default="olmoe", choices=sorted(inputs.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--placement", default="contiguous", choices=["contiguous", "histogram"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     cfg = inputs.CONFIGS[args.config]

@@ -34,6 +34,7 @@ EXPORTS = (
     "moe_prepare_weights", "moe_prepare_shared_weights", "moe_expert_ffn_workspace_size",
     "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
     "moe_layer_workspace_size", "moe_layer_forward", "moe_layer_forward_host",
+    "moe_place_greedy",
 )
 
 
@@ -261,3 +262,18 @@ def moe_layer_forward_host(h_logits, h_x, k, R, renorm, slot_of, w_gu, w_dn, f, 
         _ptr(w_dn, h_x.dtype, "w_dn"), _ptr(sw_gu, h_x.dtype, "sw_gu"),
         _ptr(sw_dn, h_x.dtype, "sw_dn"), _host_ptr(h_y, h_x.dtype, "h_y"),
         _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
+
+
+def moe_place_greedy(hist, R) -> torch.Tensor:
+    """Correlated placement (host): hist [E, E] (any integer tensor) -> slot_of int32 [E]."""
+    h = hist.detach().to("cpu").to(torch.int64)
+    if (h < 0).any() or (h > 0xFFFFFFFF).any():
+        raise ValueError("histogram counts must fit in uint32")
+    h32 = h.to(torch.int32).contiguous()  # same bits as uint32 for counts < 2^31
+    if (h >= 2 ** 31).any():
+        raise ValueError("histogram counts must be < 2^31")
+    E = h.shape[0]
+    slot_of = torch.empty(E, dtype=torch.int32)
+    _check("moe_place_greedy", load().moe_place_greedy(
+        ctypes.c_void_p(h32.data_ptr()), int(E), int(R), ctypes.c_void_p(slot_of.data_ptr())))
+    return slot_of

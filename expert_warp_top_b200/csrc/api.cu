@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "../../include/moe_occult.h"
 #include "brim.cuh"
@@ -928,3 +929,40 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Correlated placement (host).
+extern "C" int moe_place_greedy(const uint32_t* hist, int E, int R, int32_t* slot_of) {
+  MOE_REQUIRE(hist && slot_of, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(E >= 1 && E <= moe::kMaxE && R >= 1 && E % R == 0, MOE_ERR_UNSUPPORTED,
+              "need 1 <= E <= 256 and R dividing E (E=%d R=%d)", E, R);
+  const int L = E / R;
+  std::vector<char> free_(E, 1);
+  // affinity[b] = sum over the current rank's members a of hist[a][b]
+  std::vector<uint64_t> affinity(E);
+  auto self = [&](int e) { return hist[(size_t)e * E + e]; };
+  for (int r = 0; r < R; ++r) {
+    std::fill(affinity.begin(), affinity.end(), 0);
+    for (int n = 0; n < L; ++n) {
+      int pick = -1;
+      for (int b = 0; b < E; ++b) {
+        if (!free_[b]) continue;
+        if (pick < 0) {
+          pick = b;
+          continue;
+        }
+        // first member: most-selected expert; then: strongest co-activation,
+        // ties by self count, then by lower id (b ascends, so `>` keeps it)
+        const bool better =
+            n == 0 ? self(b) > self(pick)
+                   : (affinity[b] > affinity[pick] ||
+                      (affinity[b] == affinity[pick] && self(b) > self(pick)));
+        if (better) pick = b;
+      }
+      free_[pick] = 0;
+      slot_of[pick] = r * L + n;
+      for (int b = 0; b < E; ++b) affinity[b] += hist[(size_t)pick * E + b];
+    }
+  }
+  return MOE_OK;
+}

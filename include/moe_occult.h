@@ -278,6 +278,22 @@ int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* 
                         int accumulate, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_place_greedy -- correlated expert placement from a co-activation
+ * histogram ("Expert Coupling in MoE Pretraining", Abstract: experts that are
+ * often selected together go on the same GPU; Occult paper, TL;DR:
+ * expert-placement rescheduling).  HOST function (no GPU work):
+ *   hist    [E, E] uint32, HOST memory (e.g. moe_coact_histogram of a
+ *           calibration batch, copied back)
+ *   slot_of [E] int32, HOST memory, out: the placement
+ * Ranks are filled one after another: a rank is seeded with the unplaced
+ * expert selected by the most tokens (hist[a][a]; ties -> lower id), then
+ * grows by the unplaced expert with the largest co-activation count with the
+ * rank's members (ties -> larger hist[b][b], then lower id) until it holds L
+ * experts; slots inside a rank follow that order.
+ * ------------------------------------------------------------------------- */
+int moe_place_greedy(const uint32_t* hist, int E, int R, int32_t* slot_of);
+
+/* ---------------------------------------------------------------------------
  * moe_layer_forward -- the whole layer in one call, every step of the hot
  * path in order on `stream`: moe_route_topk, moe_brim_build,
  * moe_dispatch_gather, moe_expert_ffn (routed experts over the EPD groups,

@@ -95,3 +95,27 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         moe.moe_route_topk(torch.zeros(4, 8), 2, 0, torch.zeros(4, 2, dtype=torch.int32),
                            torch.zeros(4, 2))
+
+
+def test_place_greedy_matches_oracle():
+    """The library's host-side placement against the oracle's, bit for bit."""
+    import numpy as np
+    import torch
+    import oracle
+    from expert_warp_top_b200 import inputs
+    rng = np.random.default_rng(0)
+    for E, R in [(8, 2), (64, 8), (16, 16), (32, 1), (256, 8)]:
+        h = rng.integers(0, 50, size=(E, E)).astype(np.uint32)
+        h = (h + h.T).astype(np.uint32)
+        got = moe.moe_place_greedy(torch.from_numpy(h.astype(np.int64)), R).numpy()
+        assert np.array_equal(got, oracle.place_greedy(h, R)), (E, R)
+    # ties everywhere: a constant histogram
+    h = np.full((16, 16), 7, np.uint32)
+    assert np.array_equal(moe.moe_place_greedy(torch.from_numpy(h.astype(np.int64)), 4).numpy(),
+                          oracle.place_greedy(h, 4))
+    # the planted-group workload
+    cfg = inputs.CONFIGS["corr_prefill"].with_(T=4096, seed=1)
+    idx, _ = oracle.route(inputs.make_logits(cfg).numpy(), cfg.k, 0)
+    h = oracle.coact_histogram(idx, cfg.E)
+    assert np.array_equal(moe.moe_place_greedy(torch.from_numpy(h.astype(np.int64)), cfg.R).numpy(),
+                          oracle.place_greedy(h, cfg.R))
