@@ -5,9 +5,9 @@
 One step = one pass of the whole layer over one batch: top-k routing, BRIM
 build, ORI -> SFD -> EPD dispatch, grouped SwiGLU experts (+ shared experts),
 per-rank pre-reduce and combine, dispatched-row counter and co-activation
-histogram.  Inputs are synthetic (seeded), already resident in HBM when the
-timed region starts; L2 is flushed between steps (a 256 MiB write outside the
-per-step events).  Under torchrun every rank runs its own batch (independent
+histogram, replayed from one CUDA graph.  Inputs are synthetic (seeded),
+already resident in HBM when the timed region starts; L2 is flushed between
+steps (a 256 MiB write outside the per-step events).  Under torchrun every rank runs its own batch (independent
 problems, no data-path collective: weak scaling); the time is the max over
 ranks.
 
@@ -149,8 +149,9 @@ def algorithmic_work(cfg, c_t: int, e_act: int):
 
 
 def launches_per_step(cfg) -> int:
-    # route 1, BRIM 3, dispatch 1, experts 2 (+2 shared), combine 1, counter 1, histogram 1
-    return 1 + 3 + 1 + 2 + (2 if cfg.S else 0) + 1 + 1 + 1
+    # routing + BRIM masks + counter + histogram (one kernel), BRIM scatter 1, dispatch 1,
+    # experts 2 (+2 shared), combine 1
+    return 1 + 1 + 1 + 2 + (2 if cfg.S else 0) + 1
 
 
 def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
@@ -244,13 +245,11 @@ def run_ours(args, cfg):
     torch.cuda.synchronize(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    # The step is replayed from three CUDA graphs so that host launch overhead
-    # does not enter the timing: [route, BRIM, dispatch], [routed experts],
-    # [shared experts, combine, counter, histogram].  Events between the
-    # replays time the routed-expert GEMMs on their own.
+    # The step is replayed from one CUDA graph, so host launch overhead does not
+    # enter the timing.  Two external event-record nodes inside the graph time
+    # the routed-expert GEMMs on their own within every timed step.
     def part_a():
-        layer.route(logits)
-        layer.build_brims()
+        layer.route_brim(logits)  # routing, BRIMs, counter, histogram
         layer.dispatch(x)
 
     def part_b():
@@ -259,7 +258,6 @@ def run_ours(args, cfg):
     def part_c():
         layer.shared_experts(x)
         layer.combine()
-        layer.statistics()
 
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
@@ -271,43 +269,40 @@ def run_ours(args, cfg):
     status = B.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
-    graphs = []
-    for part in (part_a, part_b, part_c):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=side):
-            part()
-        graphs.append(g)
+    f0 = torch.cuda.Event(enable_timing=True, external=True)
+    f1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        part_a()
+        f0.record(side)
+        part_b()
+        f1.record(side)
+        part_c()
     torch.cuda.synchronize(dev)
     c_t = int(layer.c_t.item())
     e_act = int((layer.epd_off[1:] - layer.epd_off[:-1] > 0).sum().item())
 
-    def replay_step():
-        for g in graphs:
-            g.replay()
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    step_ms, ffn_ms = [], []
     with ClockSampler(local_rank) as clocks:
         # keep the GPU busy until the sampler reports, so its samples see the load
         t_end = time.time() + 5.0
         while clocks.n_samples() < 2 and time.time() < t_end:
             for _ in range(20):
-                replay_step()
+                graph.replay()
             torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
             flush.fill_(i & 0xFF)  # evict the previous step's working set from L2
-            s0, f0, f1, s1 = ev[i]
             s0.record(stream)
-            graphs[0].replay()
-            f0.record(stream)
-            graphs[1].replay()
-            f1.record(stream)
-            graphs[2].replay()
+            graph.replay()
             s1.record(stream)
+            s1.synchronize()
+            step_ms.append(s0.elapsed_time(s1))
+            ffn_ms.append(f0.elapsed_time(f1))
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
@@ -316,13 +311,11 @@ def run_ours(args, cfg):
         n0 = clocks.n_samples()
         while clocks.n_samples() < n0 + 2 and time.time() < t_end:
             for _ in range(20):
-                replay_step()
+                graph.replay()
             torch.cuda.synchronize(dev)
     status = B.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
-    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)]
-    ffn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], device=dev)

@@ -34,7 +34,7 @@ EXPORTS = (
     "moe_prepare_weights", "moe_prepare_shared_weights", "moe_expert_ffn_workspace_size",
     "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
     "moe_layer_workspace_size", "moe_layer_forward", "moe_layer_forward_host",
-    "moe_place_greedy",
+    "moe_place_greedy", "moe_route_brim_workspace_size", "moe_route_brim",
 )
 
 
@@ -61,6 +61,7 @@ def load():
         lib.moe_brim_workspace_size.restype = ctypes.c_size_t
         lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
         lib.moe_layer_workspace_size.restype = ctypes.c_size_t
+        lib.moe_route_brim_workspace_size.restype = ctypes.c_size_t
         lib.moe_set_debug.argtypes = [ctypes.c_int, ctypes.c_double]
         for name in EXPORTS:
             getattr(lib, name)
@@ -148,6 +149,25 @@ def moe_brim_build_noalloc(topk_idx, topk_w, slot_of, E, R, brim0, sfd_token, sf
         _ptr(brim0, I32, "brim0"), _ptr(sfd_token, I32, "sfd_token"), _ptr(sfd_off, I32, "sfd_off"),
         _ptr(brim1, I32, "brim1"), _ptr(epd_off, I32, "epd_off"), _ptr(epd_sfd, I32, "epd_sfd"),
         _ptr(epd_gate, F32, "epd_gate"), _ptr(c_t, I32, "c_t"), _stream(stream)))
+
+
+def moe_route_brim_workspace_size(T, E, R) -> int:
+    return int(load().moe_route_brim_workspace_size(int(T), int(E), int(R)))
+
+
+def moe_route_brim(logits, k, renorm, slot_of, R, topk_idx, topk_w, brim0, sfd_token, sfd_off,
+                   brim1, epd_off, epd_sfd, epd_gate, c_t, ws, per_rank=None, total=None,
+                   remote=None, hist=None, hist_accumulate=0, stream=None):
+    T, E = logits.shape
+    _check("moe_route_brim", load().moe_route_brim(
+        _ptr(logits, F32, "logits"), T, E, int(k), int(renorm), _ptr(slot_of, I32, "slot_of"),
+        int(R), _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"),
+        _ptr(brim0, I32, "brim0"), _ptr(sfd_token, I32, "sfd_token"), _ptr(sfd_off, I32, "sfd_off"),
+        _ptr(brim1, I32, "brim1"), _ptr(epd_off, I32, "epd_off"), _ptr(epd_sfd, I32, "epd_sfd"),
+        _ptr(epd_gate, F32, "epd_gate"), _ptr(c_t, I32, "c_t"),
+        _ptr(per_rank, I32, "per_rank"), _ptr(total, I64, "total"), _ptr(remote, I64, "remote"),
+        _ptr(hist, (U32, torch.int32), "hist"), int(hist_accumulate),
+        _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
 
 
 def moe_dispatch_gather(x, k, R, L, brim0, brim1, x_sfd, x_epd, stream=None):

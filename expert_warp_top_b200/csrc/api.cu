@@ -17,6 +17,7 @@
 #include "ffn_gemm.cuh"
 #include "ffn_gemm_pair.cuh"
 #include "route.cuh"
+#include "route_brim.cuh"
 
 // The device error flag the kernels raise (bits moe::kErrIndex, kErrTimeout).
 __device__ unsigned g_moe_err_flag;
@@ -114,6 +115,25 @@ int noalloc_scratch(int32_t** out) {
   }
   *out = g_noalloc_ptr[dev];
   return MOE_OK;
+}
+
+// Every kernel is launched with programmatic stream serialization, so the next
+// kernel on the stream can be scheduled while this one finishes; each kernel
+// starts with griddepcontrol.wait (moe::pdl_enter) before it touches memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ---- debug knobs (tests only) -------------------------------------------
@@ -218,7 +238,7 @@ int launch_gemm(DeviceInfo* di, unsigned attr_bit, const void* a, int a_rows,
   const int grid = (int)(ub < di->num_sms ? (ub < 1 ? 1 : ub) : di->num_sms);
   moe::GemmArgs args{group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo,
                      di->err_flag, wait_limit_ns(), g_debug_flags};
-  kern<<<grid, moe::kGemmThreads, Cfg::kSmemBytes, st>>>(ta, tb, args);
+  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, args));
   MOE_LAUNCHED("ffn_gemm_kernel");
   return MOE_OK;
 }
@@ -254,16 +274,18 @@ int launch_gemm_pair(DeviceInfo* di, int slot, const void* a, int a_rows, int m_
   if (rc) return rc;
   auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32>;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
   if (!(di->pair_attr_done & (1u << slot))) {
     MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)Cfg::kSmemBytes));
@@ -278,6 +300,7 @@ int launch_gemm_pair(DeviceInfo* di, int slot, const void* a, int a_rows, int m_
   const long long pairs = ub < di->pair_max_clusters[slot] ? (ub < 1 ? 1 : ub)
                                                             : di->pair_max_clusters[slot];
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.numAttrs = 2;
   moe::GemmArgs args{group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo,
                      di->err_flag, wait_limit_ns(), g_debug_flags};
   MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
@@ -290,7 +313,10 @@ template <int EPI, bool TF32>
 int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_index,
                      int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
                      const float* row_scale, void* out, int ldo, cudaStream_t st) {
-  const bool tall = (long long)m_cap >= 192LL * G;
+#ifndef MOE_PAIR_MIN_ROWS
+#define MOE_PAIR_MIN_ROWS 192
+#endif
+  const bool tall = (long long)m_cap >= (long long)MOE_PAIR_MIN_ROWS * G;
   bool pair = !a_row_index && N % 128 == 0 && tall;
   if (g_debug_flags & kDebugForceSingle) pair = false;
   if ((g_debug_flags & kDebugForcePair) && !a_row_index && N % 128 == 0) pair = true;
@@ -333,14 +359,14 @@ int launch_brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int 
                        cudaStream_t stream) {
   const int n_tiles = (T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
   const int blocks = (n_tiles + 3) / 4;
-  moe::brim_mask_kernel<KMAX><<<blocks, 128, 0, stream>>>(topk_idx, slot_of, T, k, E, R, n_tiles,
-                                                          scratch, err);
+  MOE_CUDA(launch_k(moe::brim_mask_kernel<KMAX>, blocks, 128, 0, stream, topk_idx, slot_of, T, k, E, R, n_tiles,
+                                                          scratch, err));
   MOE_LAUNCHED("brim_mask_kernel");
-  moe::brim_scan_kernel<<<1, 1024, 0, stream>>>(scratch, n_tiles, E, R, sfd_off, epd_off, c_t);
+  MOE_CUDA(launch_k(moe::brim_scan_kernel, 1, 1024, 0, stream, scratch, n_tiles, E, R, sfd_off, epd_off, c_t));
   MOE_LAUNCHED("brim_scan_kernel");
-  moe::brim_scatter_kernel<KMAX><<<blocks, 128, 0, stream>>>(
+  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KMAX>, blocks, 128, 0, stream, 
       topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, reinterpret_cast<const int32_t*>(scratch),
-      brim0, sfd_token, brim1, epd_sfd, epd_gate);
+      brim0, sfd_token, brim1, epd_sfd, epd_gate));
   MOE_LAUNCHED("brim_scatter_kernel");
   return MOE_OK;
 }
@@ -409,7 +435,7 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
   const int blocks = (T + 7) / 8;
-  moe::route_topk_kernel<<<blocks, 256, 0, stream>>>(logits, T, E, k, renorm, topk_idx, topk_w);
+  MOE_CUDA(launch_k(moe::route_topk_kernel, blocks, 256, 0, stream, logits, T, E, k, renorm, topk_idx, topk_w));
   MOE_LAUNCHED("route_topk_kernel");
   return MOE_OK;
 }
@@ -483,6 +509,75 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
 }
 
 // ---------------------------------------------------------------------------
+size_t moe_route_brim_workspace_size(int T, int E, int R) {
+  if (T < 0 || E < 1 || R < 1) return 0;
+  return align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)) + 512;
+}
+
+int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const int32_t* slot_of,
+                   int R, int32_t* topk_idx, float* topk_w, int32_t* brim0, int32_t* sfd_token,
+                   int32_t* sfd_off, int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                   float* epd_gate, int32_t* c_t, int32_t* per_rank, int64_t* total,
+                   int64_t* remote, uint32_t* hist, int hist_accumulate, void* ws,
+                   size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  MOE_REQUIRE(renorm == 0 || renorm == 1, MOE_ERR_INVALID_ARG, "renorm must be 0 or 1");
+  MOE_REQUIRE(slot_of && sfd_off && epd_off && c_t, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE((per_rank == nullptr) == (total == nullptr) && (total == nullptr) == (remote == nullptr),
+              MOE_ERR_INVALID_ARG, "per_rank, total and remote are given together or not at all");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  if (per_rank) {
+    MOE_CUDA(cudaMemsetAsync(per_rank, 0, sizeof(int32_t) * R, stream));
+    MOE_CUDA(cudaMemsetAsync(total, 0, sizeof(int64_t), stream));
+    MOE_CUDA(cudaMemsetAsync(remote, 0, sizeof(int64_t), stream));
+  }
+  if (hist && !hist_accumulate)
+    MOE_CUDA(cudaMemsetAsync(hist, 0, sizeof(uint32_t) * E * E, stream));
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(sfd_off, 0, sizeof(int32_t) * (R + 1), stream));
+    MOE_CUDA(cudaMemsetAsync(epd_off, 0, sizeof(int32_t) * (E + 1), stream));
+    MOE_CUDA(cudaMemsetAsync(c_t, 0, sizeof(int32_t), stream));
+    return MOE_OK;
+  }
+  MOE_REQUIRE(logits && topk_idx && topk_w && brim0 && sfd_token && brim1 && epd_sfd && epd_gate &&
+                  ws,
+              MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(ws_bytes >= moe_route_brim_workspace_size(T, E, R), MOE_ERR_INVALID_ARG,
+              "workspace too small: %zu < %zu bytes", ws_bytes,
+              moe_route_brim_workspace_size(T, E, R));
+  MOE_REQUIRE(aligned16(ws), MOE_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  uint32_t* masks = static_cast<uint32_t*>(ws);
+  unsigned* ticket = reinterpret_cast<unsigned*>(
+      static_cast<char*>(ws) + align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)));
+  MOE_CUDA(cudaMemsetAsync(ticket, 0, sizeof(unsigned), stream));
+  const int n_tiles = (T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
+  auto* tot = reinterpret_cast<unsigned long long*>(total);
+  auto* rem = reinterpret_cast<unsigned long long*>(remote);
+#define MOE_ROUTE_BRIM(KM)                                                                    \
+  MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM>, dim3(n_tiles), dim3(1024), 0, stream,    \
+                    logits, T, E, k, renorm, slot_of, R, n_tiles, topk_idx, topk_w, masks,      \
+                    sfd_off, epd_off, c_t, per_rank, tot, rem, hist, ticket, di->err_flag));    \
+  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3((n_tiles + 3) / 4), dim3(128), 0,      \
+                    stream, topk_idx, topk_w, slot_of, T, k, E, R, n_tiles,                     \
+                    reinterpret_cast<const int32_t*>(masks), brim0, sfd_token, brim1, epd_sfd,  \
+                    epd_gate))
+  if (k <= 2) {
+    MOE_ROUTE_BRIM(2);
+  } else if (k <= 4) {
+    MOE_ROUTE_BRIM(4);
+  } else if (k <= 8) {
+    MOE_ROUTE_BRIM(8);
+  } else {
+    MOE_ROUTE_BRIM(16);
+  }
+#undef MOE_ROUTE_BRIM
+  MOE_LAUNCHED("route_brim_tile_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
 int moe_dispatch_gather(const void* x, int T, int d, int dtype, int k, int R, int L,
                         const int32_t* brim0, const int32_t* brim1, void* x_sfd, void* x_epd,
                         moe_stream_t stream) {
@@ -503,9 +598,9 @@ int moe_dispatch_gather(const void* x, int T, int d, int dtype, int k, int R, in
   const int P = mover_parts(di, T, (row_bytes + CH * 512 - 1) / (CH * 512));
   const long long warps = (long long)T * P;
   const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
-  moe::dispatch_kernel<CH><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(
+  MOE_CUDA(launch_k(moe::dispatch_kernel<CH>, blocks, moe::kMoverWarps * 32, 0, stream, 
       static_cast<const uint8_t*>(x), T, row_bytes, P, R, L, cap, T * k, brim0, brim1,
-      static_cast<uint8_t*>(x_sfd), static_cast<uint8_t*>(x_epd), di->err_flag);
+      static_cast<uint8_t*>(x_sfd), static_cast<uint8_t*>(x_epd), di->err_flag));
   MOE_LAUNCHED("dispatch_kernel");
   return MOE_OK;
 }
@@ -530,10 +625,10 @@ int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R
   const long long warps = (long long)T * P;
   const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
 #define MOE_COMBINE(TA, KM)                                                                    \
-  moe::combine_kernel<TA, KM><<<blocks, moe::kMoverWarps * 32, 0, stream>>>(                   \
+  MOE_CUDA(launch_k(moe::combine_kernel<TA, KM>, blocks, moe::kMoverWarps * 32, 0, stream,                    \
       static_cast<const TA*>(o_epd), T, d, P, R, L, cap, T * k, brim0, brim1,                  \
       static_cast<const TA*>(shared_out), static_cast<TA*>(y_sfd), static_cast<TA*>(y),        \
-      di->err_flag)
+      di->err_flag))
   if (dtype == MOE_BF16) {
     using B = __nv_bfloat16;
     if (k <= 2) MOE_COMBINE(B, 2);
@@ -567,12 +662,12 @@ int moe_prepare_weights(const void* wg, const void* wu, const void* wd, int E, i
   if ((rc = device_info(&di))) return rc;
   const int es = esize(dtype);
   const int grid = di->num_sms * 4;
-  moe::pack_gate_up_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(wg),
+  MOE_CUDA(launch_k(moe::pack_gate_up_kernel, grid, 256, 0, stream, static_cast<const uint8_t*>(wg),
                                                      static_cast<const uint8_t*>(wu), E, d, f, es,
-                                                     slot_of, static_cast<uint8_t*>(w_gu));
+                                                     slot_of, static_cast<uint8_t*>(w_gu)));
   MOE_LAUNCHED("pack_gate_up_kernel");
-  moe::pack_down_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(wd), E, d, f, es,
-                                                  slot_of, static_cast<uint8_t*>(w_dn));
+  MOE_CUDA(launch_k(moe::pack_down_kernel, grid, 256, 0, stream, static_cast<const uint8_t*>(wd), E, d, f, es,
+                                                  slot_of, static_cast<uint8_t*>(w_dn)));
   MOE_LAUNCHED("pack_down_kernel");
   return MOE_OK;
 }
@@ -590,12 +685,12 @@ int moe_prepare_shared_weights(const void* sg, const void* su, const void* sd, i
   if ((rc = device_info(&di))) return rc;
   const int es = esize(dtype);
   const int grid = di->num_sms * 4;
-  moe::pack_shared_gate_up_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(sg),
+  MOE_CUDA(launch_k(moe::pack_shared_gate_up_kernel, grid, 256, 0, stream, static_cast<const uint8_t*>(sg),
                                                             static_cast<const uint8_t*>(su), S, d,
-                                                            fs, es, static_cast<uint8_t*>(w_gu));
+                                                            fs, es, static_cast<uint8_t*>(w_gu)));
   MOE_LAUNCHED("pack_shared_gate_up_kernel");
-  moe::pack_shared_down_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(sd), S, d,
-                                                         fs, es, static_cast<uint8_t*>(w_dn));
+  MOE_CUDA(launch_k(moe::pack_shared_down_kernel, grid, 256, 0, stream, static_cast<const uint8_t*>(sd), S, d,
+                                                         fs, es, static_cast<uint8_t*>(w_dn)));
   MOE_LAUNCHED("pack_shared_down_kernel");
   return MOE_OK;
 }
@@ -631,12 +726,12 @@ int moe_expert_ffn(const void* a, int a_rows, const int32_t* a_row_index,
                 "the identity expert takes its rows in place (no row index)");
     const int grid = di->num_sms * 8;
     if (dtype == MOE_BF16)
-      moe::identity_expert_kernel<__nv_bfloat16><<<grid, moe::kMoverWarps * 32, 0, stream>>>(
+      MOE_CUDA(launch_k(moe::identity_expert_kernel<__nv_bfloat16>, grid, moe::kMoverWarps * 32, 0, stream, 
           static_cast<const __nv_bfloat16*>(a), group_off, G, d, row_scale,
-          static_cast<__nv_bfloat16*>(out));
+          static_cast<__nv_bfloat16*>(out)));
     else
-      moe::identity_expert_kernel<float><<<grid, moe::kMoverWarps * 32, 0, stream>>>(
-          static_cast<const float*>(a), group_off, G, d, row_scale, static_cast<float*>(out));
+      MOE_CUDA(launch_k(moe::identity_expert_kernel<float>, grid, moe::kMoverWarps * 32, 0, stream, 
+          static_cast<const float*>(a), group_off, G, d, row_scale, static_cast<float*>(out)));
     MOE_LAUNCHED("identity_expert_kernel");
     return MOE_OK;
   }
@@ -683,17 +778,17 @@ int moe_count_dispatched_rows(const int32_t* topk_idx, int T, int k, const int32
     auto* rem = reinterpret_cast<unsigned long long*>(remote);
     const int blocks = (T + 255) / 256;
     if (k <= 2)
-      moe::count_dispatched_kernel<2><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
-                                                                  per_rank, tot, rem, di->err_flag);
+      MOE_CUDA(launch_k(moe::count_dispatched_kernel<2>, blocks, 256, 0, stream, topk_idx, T, k, slot_of, E, R,
+                                                                  per_rank, tot, rem, di->err_flag));
     else if (k <= 4)
-      moe::count_dispatched_kernel<4><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
-                                                                  per_rank, tot, rem, di->err_flag);
+      MOE_CUDA(launch_k(moe::count_dispatched_kernel<4>, blocks, 256, 0, stream, topk_idx, T, k, slot_of, E, R,
+                                                                  per_rank, tot, rem, di->err_flag));
     else if (k <= 8)
-      moe::count_dispatched_kernel<8><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
-                                                                  per_rank, tot, rem, di->err_flag);
+      MOE_CUDA(launch_k(moe::count_dispatched_kernel<8>, blocks, 256, 0, stream, topk_idx, T, k, slot_of, E, R,
+                                                                  per_rank, tot, rem, di->err_flag));
     else
-      moe::count_dispatched_kernel<16><<<blocks, 256, 0, stream>>>(topk_idx, T, k, slot_of, E, R,
-                                                                   per_rank, tot, rem, di->err_flag);
+      MOE_CUDA(launch_k(moe::count_dispatched_kernel<16>, blocks, 256, 0, stream, topk_idx, T, k, slot_of, E, R,
+                                                                   per_rank, tot, rem, di->err_flag));
   }
   MOE_LAUNCHED("count_dispatched_kernel");
   return MOE_OK;
@@ -712,13 +807,13 @@ int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* 
   {
     const int blocks = (T + 255) / 256;
     if (k <= 2)
-      moe::coact_hist_kernel<2><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+      MOE_CUDA(launch_k(moe::coact_hist_kernel<2>, blocks, 256, 0, stream, topk_idx, T, k, E, hist, di->err_flag));
     else if (k <= 4)
-      moe::coact_hist_kernel<4><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+      MOE_CUDA(launch_k(moe::coact_hist_kernel<4>, blocks, 256, 0, stream, topk_idx, T, k, E, hist, di->err_flag));
     else if (k <= 8)
-      moe::coact_hist_kernel<8><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+      MOE_CUDA(launch_k(moe::coact_hist_kernel<8>, blocks, 256, 0, stream, topk_idx, T, k, E, hist, di->err_flag));
     else
-      moe::coact_hist_kernel<16><<<blocks, 256, 0, stream>>>(topk_idx, T, k, E, hist, di->err_flag);
+      MOE_CUDA(launch_k(moe::coact_hist_kernel<16>, blocks, 256, 0, stream, topk_idx, T, k, E, hist, di->err_flag));
   }
   MOE_LAUNCHED("coact_hist_kernel");
   return MOE_OK;
@@ -730,6 +825,7 @@ int moe_coact_histogram(const int32_t* topk_idx, int T, int k, int E, uint32_t* 
 // The whole layer.  The workspace is carved into the layer's intermediate
 // state, every region 256-byte aligned.
 __global__ void set_pair_kernel(int32_t* p, int a, int b) {
+  moe::pdl_enter();
   p[0] = a;
   p[1] = b;
 }
@@ -781,7 +877,7 @@ size_t carve_layer(char* base, int T, int d, int f, int E, int k, int R, int S, 
   s.epd_sfd = c.take<int32_t>(tk);
   s.epd_gate = c.take<float>(tk);
   s.c_t = c.take<int32_t>(1);
-  s.brim_ws_bytes = moe_brim_workspace_size(T, E, R);
+  s.brim_ws_bytes = moe_route_brim_workspace_size(T, E, R);
   s.brim_ws = c.take<char>(s.brim_ws_bytes);
   s.x_sfd = c.take<char>(cap * d * es);
   s.x_epd = L > 1 ? c.take<char>(tk * d * es) : nullptr;
@@ -816,9 +912,11 @@ int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int S, int
   const size_t tk = (size_t)T * k;
   const size_t cap = (size_t)T * (k < R ? k : R);
   int rc;
-  if ((rc = moe_route_topk(logits, T, E, k, renorm, st.topk_idx, st.topk_w, stream))) return rc;
-  if ((rc = moe_brim_build(st.topk_idx, st.topk_w, T, k, slot_of, E, R, st.brim0, st.sfd_token,
-                           st.sfd_off, st.brim1, st.epd_off, st.epd_sfd, st.epd_gate, st.c_t,
+  if ((rc = moe_route_brim(logits, T, E, k, renorm, slot_of, R, st.topk_idx, st.topk_w, st.brim0,
+                           st.sfd_token, st.sfd_off, st.brim1, st.epd_off, st.epd_sfd,
+                           st.epd_gate, c_t_out ? c_t_out : st.c_t,
+                           per_rank ? per_rank : st.per_rank, total ? total : st.total,
+                           remote ? remote : st.remote, hist ? hist : st.hist, hist ? 1 : 0,
                            st.brim_ws, st.brim_ws_bytes, stream)))
     return rc;
   if ((rc = moe_dispatch_gather(x, T, d, dtype, k, R, L, st.brim0, st.brim1, st.x_sfd, st.x_epd,
@@ -832,7 +930,7 @@ int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int S, int
                            st.ffn_ws_bytes, stream)))
     return rc;
   if (S > 0) {
-    set_pair_kernel<<<1, 1, 0, stream>>>(st.shared_off, 0, T);  // the one shared group: [0, T)
+    MOE_CUDA(launch_k(set_pair_kernel, 1, 1, 0, stream, st.shared_off, 0, T));  // the one shared group: [0, T)
     MOE_LAUNCHED("set_pair_kernel");
     if ((rc = moe_expert_ffn(x, T, nullptr, st.shared_off, 1, T, sw_gu, sw_dn, d, S * fs, dtype,
                              nullptr, MOE_FFN_SWIGLU, st.shared_out, st.sffn_ws,
@@ -842,15 +940,6 @@ int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int S, int
   if ((rc = moe_combine_scatter(st.o_epd, T, d, dtype, k, R, L, st.brim0, st.brim1,
                                 S > 0 ? st.shared_out : nullptr, st.y_sfd, y, stream)))
     return rc;
-  if ((rc = moe_count_dispatched_rows(st.topk_idx, T, k, slot_of, E, R,
-                                      per_rank ? per_rank : st.per_rank, total ? total : st.total,
-                                      remote ? remote : st.remote, stream)))
-    return rc;
-  if ((rc = moe_coact_histogram(st.topk_idx, T, k, E, hist ? hist : st.hist, hist ? 1 : 0,
-                                stream)))
-    return rc;
-  if (c_t_out) MOE_CUDA(cudaMemcpyAsync(c_t_out, st.c_t, sizeof(int32_t), cudaMemcpyDeviceToDevice,
-                                        stream));
   return MOE_OK;
 }
 

@@ -39,12 +39,13 @@ struct TokenRoute {
   bool first[KMAX];
 };
 
-// Loads token t's route.  Returns false (and raises the error flag) when an
-// expert id is out of range or repeated; such a token is sent nowhere.
+// Builds a token's route from its k expert ids.  Returns false (and raises
+// the error flag) when an expert id is out of range or repeated; such a token
+// is sent nowhere.
 template <int KMAX>
-__device__ __forceinline__ bool load_token_route(const int32_t* __restrict__ topk_idx,
-                                                 const int32_t* __restrict__ slot_of, int t,
-                                                 int k, int E, int L, TokenRoute<KMAX>& tr,
+__device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
+                                                 const int32_t* __restrict__ slot_of, int k,
+                                                 int E, int L, TokenRoute<KMAX>& tr,
                                                  unsigned* err) {
   bool ok = true;
 #pragma unroll
@@ -52,7 +53,7 @@ __device__ __forceinline__ bool load_token_route(const int32_t* __restrict__ top
     tr.slot[j] = -1;
     tr.rank[j] = -1;
     if (j < k) {
-      const int e = __ldg(topk_idx + (size_t)t * k + j);
+      const int e = ids[j];
       const int q = (e >= 0 && e < E) ? __ldg(slot_of + e) : -1;
       if (q < 0 || q >= E) ok = false;
       tr.slot[j] = q;
@@ -73,6 +74,18 @@ __device__ __forceinline__ bool load_token_route(const int32_t* __restrict__ top
   }
   if (!ok && err) raise_error(err, kErrIndex);
   return ok;
+}
+
+// Loads token t's k expert ids from topk_idx and builds its route.
+template <int KMAX>
+__device__ __forceinline__ bool load_token_route(const int32_t* __restrict__ topk_idx,
+                                                 const int32_t* __restrict__ slot_of, int t,
+                                                 int k, int E, int L, TokenRoute<KMAX>& tr,
+                                                 unsigned* err) {
+  int ids[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) ids[j] = j < k ? __ldg(topk_idx + (size_t)t * k + j) : -1;
+  return make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
 }
 
 // Build this warp's tile masks in shared memory (mask[c], ncol entries).
@@ -103,6 +116,7 @@ __global__ void __launch_bounds__(128) brim_mask_kernel(const int32_t* __restric
                                                         int T, int k, int E, int R, int n_tiles,
                                                         uint32_t* __restrict__ masks,
                                                         unsigned* err) {
+  pdl_enter();
   __shared__ uint32_t sm[4][kMaxCols];
   const int w = threadIdx.x >> 5;
   const int tile = blockIdx.x * 4 + w;
@@ -145,13 +159,13 @@ __device__ __forceinline__ int warp_exclusive_scan_smem(const int32_t* in, int32
 // One block of 32 warps.  Each warp scans whole columns: lane i sums a
 // contiguous run of tiles, a warp scan orders the runs, each lane writes its
 // run's bases.  The mask words are replaced by the tile's first global row.
-__global__ void __launch_bounds__(1024) brim_scan_kernel(uint32_t* __restrict__ masks,
-                                                        int n_tiles, int E, int R,
-                                                        int32_t* __restrict__ sfd_off,
-                                                        int32_t* __restrict__ epd_off,
-                                                        int32_t* __restrict__ c_t) {
-  __shared__ int32_t total[kMaxCols];
-  __shared__ int32_t colbase[kMaxCols];
+// Reads go to L2 (ld.cg): the masks may have been written by other blocks of
+// the same grid.
+__device__ __forceinline__ void scan_columns(uint32_t* __restrict__ masks, int n_tiles, int E,
+                                             int R, int32_t* __restrict__ sfd_off,
+                                             int32_t* __restrict__ epd_off,
+                                             int32_t* __restrict__ c_t, int32_t* total,
+                                             int32_t* colbase) {
   const int ncol = R + E;
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const unsigned lane = lane_id();
@@ -162,11 +176,11 @@ __global__ void __launch_bounds__(1024) brim_scan_kernel(uint32_t* __restrict__ 
     const int b1 = min(b0 + run, n_tiles);
     int sum = 0;
 #pragma unroll 8
-    for (int b = b0; b < b1; ++b) sum += __popc(col[b]);
+    for (int b = b0; b < b1; ++b) sum += __popc(__ldcg(col + b));
     const int inc = warp_inclusive_scan(sum);
     int base = inc - sum;
     for (int b = b0; b < b1; ++b) {
-      const int n = __popc(col[b]);
+      const int n = __popc(__ldcg(col + b));
       col[b] = (uint32_t)base;
       base += n;
     }
@@ -192,6 +206,17 @@ __global__ void __launch_bounds__(1024) brim_scan_kernel(uint32_t* __restrict__ 
     masks[i] = (uint32_t)((int32_t)masks[i] + colbase[i / n_tiles]);
 }
 
+__global__ void __launch_bounds__(1024) brim_scan_kernel(uint32_t* __restrict__ masks,
+                                                        int n_tiles, int E, int R,
+                                                        int32_t* __restrict__ sfd_off,
+                                                        int32_t* __restrict__ epd_off,
+                                                        int32_t* __restrict__ c_t) {
+  pdl_enter();
+  __shared__ int32_t total[kMaxCols];
+  __shared__ int32_t colbase[kMaxCols];
+  scan_columns(masks, n_tiles, E, R, sfd_off, epd_off, c_t, total, colbase);
+}
+
 // ---- pass 3 ---------------------------------------------------------------
 template <int KMAX>
 __global__ void __launch_bounds__(128) brim_scatter_kernel(
@@ -200,6 +225,7 @@ __global__ void __launch_bounds__(128) brim_scatter_kernel(
     const int32_t* __restrict__ tile_base, int32_t* __restrict__ brim0,
     int32_t* __restrict__ sfd_token, int32_t* __restrict__ brim1,
     int32_t* __restrict__ epd_sfd, float* __restrict__ epd_gate) {
+  pdl_enter();
   __shared__ uint32_t sm[4][kMaxCols];
   const int w = threadIdx.x >> 5;
   const int tile = blockIdx.x * 4 + w;
@@ -260,6 +286,7 @@ __global__ void __launch_bounds__(256) count_dispatched_kernel(
     const int32_t* __restrict__ topk_idx, int T, int k, const int32_t* __restrict__ slot_of,
     int E, int R, int32_t* __restrict__ per_rank, unsigned long long* __restrict__ total,
     unsigned long long* __restrict__ remote, unsigned* err) {
+  pdl_enter();
   __shared__ int32_t sc[kMaxE];
   __shared__ unsigned s_total, s_remote;
   const int L = E / R;
@@ -308,6 +335,7 @@ __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restri
                                                          int T, int k, int E,
                                                          uint32_t* __restrict__ hist,
                                                          unsigned* err) {
+  pdl_enter();
   __shared__ uint32_t sh[kHistSmemE * kHistSmemE];
   const bool use_smem = E <= kHistSmemE;
   if (use_smem) {

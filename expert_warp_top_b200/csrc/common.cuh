@@ -96,4 +96,21 @@ __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
 
 __device__ __forceinline__ unsigned lane_id() { return threadIdx.x & 31u; }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so
+// that the next kernel on the stream may be scheduled before this one ends;
+// each kernel therefore waits for its predecessors (and for their memory
+// operations to be visible) before it touches global memory, and then lets
+// its own dependents be scheduled.  Both are no-ops without the launch
+// attribute.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
 }  // namespace moe

@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
     const uint8_t* __restrict__ x, int T, int row_bytes, int P, int R, int L, size_t cap, int tk,
     const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
     uint8_t* __restrict__ x_sfd, uint8_t* __restrict__ x_epd, unsigned* err) {
+  pdl_enter();
   __shared__ WarpDst sdst[kMoverWarps];
   const int wib = threadIdx.x >> 5;
   const long long wg = (long long)blockIdx.x * kMoverWarps + wib;
@@ -148,6 +149,7 @@ __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
     const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
     const TA* __restrict__ shared_out, TA* __restrict__ y_sfd, TA* __restrict__ y,
     unsigned* err) {
+  pdl_enter();
   constexpr int VN = Vec16<TA>::n;  // elements per 16 bytes
   constexpr int SL = 32 * VN;       // elements per 512-byte slice
   __shared__ WarpDst sdst[kMoverWarps];
@@ -223,6 +225,7 @@ template <typename TA>
 __global__ void __launch_bounds__(kMoverWarps * 32) identity_expert_kernel(
     const TA* __restrict__ a, const int32_t* __restrict__ group_off, int G, int d,
     const float* __restrict__ row_scale, TA* __restrict__ out) {
+  pdl_enter();
   constexpr int VN = Vec16<TA>::n;
   const int lo = group_off[0], hi = group_off[G];
   const int lane = (int)lane_id();
@@ -250,6 +253,7 @@ __global__ void pack_gate_up_kernel(const uint8_t* __restrict__ wg, const uint8_
                                     int E, int d, int f, int esz,
                                     const int32_t* __restrict__ slot_of,
                                     uint8_t* __restrict__ w_gu) {
+  pdl_enter();
   const long long n_rows = (long long)E * 2 * f;
   const int row_bytes = d * esz;
   for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < n_rows;
@@ -266,6 +270,7 @@ __global__ void pack_gate_up_kernel(const uint8_t* __restrict__ wg, const uint8_
 // w_dn[slot(e)] = wd[e]
 __global__ void pack_down_kernel(const uint8_t* __restrict__ wd, int E, int d, int f, int esz,
                                  const int32_t* __restrict__ slot_of, uint8_t* __restrict__ w_dn) {
+  pdl_enter();
   const long long n_rows = (long long)E * d;
   const int row_bytes = f * esz;
   for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < n_rows;
@@ -282,6 +287,7 @@ __global__ void pack_down_kernel(const uint8_t* __restrict__ wd, int E, int d, i
 __global__ void pack_shared_gate_up_kernel(const uint8_t* __restrict__ sg,
                                            const uint8_t* __restrict__ su, int S, int d, int fs,
                                            int esz, uint8_t* __restrict__ w_gu) {
+  pdl_enter();
   const int F = S * fs;
   const int row_bytes = d * esz;
   for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < 2LL * F;
@@ -298,6 +304,7 @@ __global__ void pack_shared_gate_up_kernel(const uint8_t* __restrict__ sg,
 // down'[c][s*fs + i] = sd[s][c][i]
 __global__ void pack_shared_down_kernel(const uint8_t* __restrict__ sd, int S, int d, int fs,
                                         int esz, uint8_t* __restrict__ w_dn) {
+  pdl_enter();
   const int seg_bytes = fs * esz;
   for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
        w < (long long)S * d; w += (long long)gridDim.x * (blockDim.x >> 5)) {

@@ -42,6 +42,18 @@ constexpr int kEpiScale = 1;   // out[:, n0 + j]   = row_scale * acc
 // would load, so the MMA issuer's wait can never complete.
 constexpr int kDebugSkipFirstLoad = 1;
 
+// Tile order inside a group: M blocks fastest (default; concurrently running
+// CTAs share one weight block in L2) or N blocks fastest (they share A rows).
+#ifndef MOE_RASTER_N_FASTEST
+#define MOE_RASTER_N_FASTEST 0
+#endif
+constexpr bool kRasterNFastest = MOE_RASTER_N_FASTEST != 0;
+// L2 policy of the weight tiles: keep them (evict_last, default) or not.
+#ifndef MOE_WEIGHTS_EVICT_LAST
+#define MOE_WEIGHTS_EVICT_LAST 1
+#endif
+constexpr bool kWeightsEvictLast = MOE_WEIGHTS_EVICT_LAST != 0;
+
 template <int BN, bool TF32>
 struct GemmCfg {
   static constexpr int kElemBytes = TF32 ? 4 : 2;
@@ -211,6 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tmem_alloc(tc::smem_u32(tmem_slot), Cfg::kTmemCols);
     tc::tmem_relinquish();
   }
+  pdl_enter();  // predecessors' outputs (group offsets, A rows) are visible from here
   if (warp == 2) {
     // group offsets and the tile prefix: tiles of group g = m_blocks(g) * n_blocks.
     // A group whose bounds leave [0, m_cap] or run backwards is treated as
@@ -260,7 +273,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int local = tile - s_prefix[g];
     const int gstart = s_off[g], gend = s_end[g];
     const int m_blocks = (gend - gstart + kGemmBM - 1) / kGemmBM;
-    const int nb = local / m_blocks, mb = local - nb * m_blocks;
+    int nb, mb;
+    if (kRasterNFastest) {
+      mb = local / n_blocks;
+      nb = local - mb * n_blocks;
+    } else {
+      nb = local / m_blocks;
+      mb = local - nb * m_blocks;
+    }
     row0 = gstart + mb * kGemmBM;
     rows = min(kGemmBM, gend - row0);
     n0 = nb * BN;
@@ -272,7 +292,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // in GATHER mode every lane then gathers 4 of the tile's 128 A rows.
     if (GATHER || lane == 0) {
       const uint64_t pol_a = tc::policy_evict_normal();
-      const uint64_t pol_b = tc::policy_evict_last();
+      const uint64_t pol_b = kWeightsEvictLast ? tc::policy_evict_last() : tc::policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per stage: armed at least once, parity of the last arming

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tmem_alloc_pair(tc::smem_u32(tmem_slot), Cfg::kTmemCols);
     tc::tmem_relinquish_pair();
   }
+  pdl_enter();  // predecessors' outputs (group offsets, A rows) are visible from here
   if (warp == 2)
     group_tile_prefix(args.group_off, G, args.m_cap, kPairBM, n_blocks, s_off, s_end, s_prefix,
                       args.err);
@@ -116,7 +117,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int gstart = s_off[g];
     gend = s_end[g];
     const int m_blocks = (gend - gstart + kPairBM - 1) / kPairBM;
-    const int nb = local / m_blocks, mb = local - nb * m_blocks;
+    int nb, mb;
+    if (kRasterNFastest) {
+      mb = local / n_blocks;
+      nb = local - mb * n_blocks;
+    } else {
+      nb = local / m_blocks;
+      mb = local - nb * m_blocks;
+    }
     row0 = gstart + mb * kPairBM;
     n0 = nb * BN;
   };
@@ -125,7 +133,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_a = tc::policy_evict_normal();
-      const uint64_t pol_b = tc::policy_evict_last();
+      const uint64_t pol_b = kWeightsEvictLast ? tc::policy_evict_last() : tc::policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;

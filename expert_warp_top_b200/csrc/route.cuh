@@ -25,15 +25,12 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
-                                                         int T, int E, int k, int renorm,
-                                                         int32_t* __restrict__ topk_idx,
-                                                         float* __restrict__ topk_w) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// Routes one token with the whole warp.  On return lane j < k holds the j-th
+// selected expert id in *sel_id and its gate weight in *gate (other lanes:
+// unspecified).  All lanes must call it.
+__device__ __forceinline__ void route_token_warp(const float* __restrict__ row, int E, int k,
+                                                 int renorm, int* sel_id_out, float* gate_out) {
   const unsigned lane = lane_id();
-  if (warp >= T) return;
-  const float* row = logits + (size_t)warp * E;
-
   float v[kRouteMaxPerLane];
   uint32_t key[kRouteMaxPerLane];
   const int per_lane = (E + 31) >> 5;
@@ -100,9 +97,24 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     denom = part;
   }
+  *sel_id_out = sel_id;
+  *gate_out = expf(sel_logit - m) / denom;
+}
+
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
+                                                         int T, int E, int k, int renorm,
+                                                         int32_t* __restrict__ topk_idx,
+                                                         float* __restrict__ topk_w) {
+  pdl_enter();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const unsigned lane = lane_id();
+  if (warp >= T) return;
+  int id;
+  float gate;
+  route_token_warp(logits + (size_t)warp * E, E, k, renorm, &id, &gate);
   if ((int)lane < k) {
-    topk_idx[(size_t)warp * k + lane] = sel_id;
-    topk_w[(size_t)warp * k + lane] = expf(sel_logit - m) / denom;
+    topk_idx[(size_t)warp * k + lane] = id;
+    topk_w[(size_t)warp * k + lane] = gate;
   }
 }
 

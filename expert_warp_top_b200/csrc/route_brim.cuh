@@ -1,0 +1,107 @@
+// route_brim.cuh -- routing, the BRIM passes 1-2, the dispatched-row counter
+// and the co-activation histogram in one kernel.
+//
+// The same computation as moe_route_topk + brim passes 1-2 (brim.cuh) +
+// moe_count_dispatched_rows + moe_coact_histogram, in one launch instead of
+// five: one block of 32 warps per 32-token tile.  Each warp routes one token
+// (route_token_warp, the very code of moe_route_topk); warp 0 then takes the
+// tile lane-per-token, builds its column masks, and adds the tile's
+// contributions to the counter and the histogram.  The last block to finish
+// (a ticket taken after a memory fence) runs the column scan, so pass 3 of the
+// BRIM build can follow directly.
+#pragma once
+#include "brim.cuh"
+#include "route.cuh"
+
+namespace moe {
+
+template <int KMAX>
+__global__ void __launch_bounds__(1024) route_brim_tile_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int renorm,
+    const int32_t* __restrict__ slot_of, int R, int n_tiles, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, uint32_t* __restrict__ masks, int32_t* __restrict__ sfd_off,
+    int32_t* __restrict__ epd_off, int32_t* __restrict__ c_t, int32_t* __restrict__ per_rank,
+    unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
+    uint32_t* __restrict__ hist, unsigned* __restrict__ ticket, unsigned* err) {
+  pdl_enter();
+  __shared__ int s_ids[32][KMAX];
+  __shared__ uint32_t s_mask[kMaxCols];
+  __shared__ int32_t s_scan_a[kMaxCols], s_scan_b[kMaxCols];
+  __shared__ bool s_last;
+  const int warp = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  const int tile = blockIdx.x;
+  const int L = E / R, ncol = R + E;
+
+  // 1. each warp routes one token of the tile
+  {
+    const int t = tile * kBrimTileTokens + warp;
+    int id = -1;
+    float gate = 0.f;
+    if (t < T) {
+      route_token_warp(logits + (size_t)t * E, E, k, renorm, &id, &gate);
+      if ((int)lane < k) {
+        topk_idx[(size_t)t * k + lane] = id;
+        topk_w[(size_t)t * k + lane] = gate;
+      }
+    }
+    if ((int)lane < KMAX) s_ids[warp][lane] = (t < T && (int)lane < k) ? id : -1;
+  }
+  __syncthreads();
+
+  // 2. warp 0, one lane per token: masks, counter, histogram
+  if (warp == 0) {
+    const int t = tile * kBrimTileTokens + (int)lane;
+    int ids[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) ids[j] = s_ids[lane][j];
+    TokenRoute<KMAX> tr;
+    const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
+    tile_masks<KMAX>(s_mask, ncol, R, active, k, tr);
+    for (int c = lane; c < ncol; c += 32) masks[(size_t)c * n_tiles + tile] = s_mask[c];
+    if (per_rank) {
+      // tokens per rank: popcount of the rank columns; remote: ranks other than
+      // the token's source rank floor(t * R / T)
+      for (int r = lane; r < R; r += 32) {
+        const int n = __popc(s_mask[r]);
+        if (n) atomicAdd(&per_rank[r], n);
+      }
+      const int src = (int)(((long long)t * R) / (T > 0 ? T : 1));
+      unsigned n_rank = 0, n_remote = 0;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (active && j < k && tr.first[j]) {
+          ++n_rank;
+          n_remote += tr.rank[j] != src;
+        }
+      n_rank = __reduce_add_sync(0xffffffffu, n_rank);
+      n_remote = __reduce_add_sync(0xffffffffu, n_remote);
+      if (lane == 0) {
+        if (n_rank) atomicAdd(total, (unsigned long long)n_rank);
+        if (n_remote) atomicAdd(remote, (unsigned long long)n_remote);
+      }
+    }
+    if (hist && active) {
+#pragma unroll
+      for (int a = 0; a < KMAX; ++a)
+#pragma unroll
+        for (int b = 0; b < KMAX; ++b)
+          if (a < k && b < k) atomicAdd(&hist[ids[a] * E + ids[b]], 1u);
+    }
+  }
+
+  // 3. the last tile to finish scans the columns
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    scan_columns(masks, n_tiles, E, R, sfd_off, epd_off, c_t, s_scan_a, s_scan_b);
+    if (threadIdx.x == 0) *ticket = 0u;
+  }
+}
+
+}  // namespace moe

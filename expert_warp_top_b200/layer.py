@@ -67,7 +67,8 @@ class MoELayer:
         self.epd_sfd = torch.empty(max(self.tk, 1), **i32)
         self.epd_gate = torch.empty(max(self.tk, 1), **f32)
         self.c_t = torch.empty(1, **i32)
-        self.brim_ws = torch.empty(max(B.moe_brim_workspace_size(T, E, R), 256),
+        self.brim_ws = torch.empty(max(B.moe_brim_workspace_size(T, E, R),
+                                       B.moe_route_brim_workspace_size(T, E, R), 256),
                                    dtype=torch.uint8, device=dev)
         # token states
         self.x_sfd = torch.empty(max(self.cap, 1), d, **act)
@@ -112,6 +113,14 @@ class MoELayer:
                          self.sfd_token, self.sfd_off, self.brim1, self.epd_off, self.epd_sfd,
                          self.epd_gate, self.c_t, self.brim_ws, stream)
 
+    def route_brim(self, logits, stream=None):
+        """Routing, BRIMs, counter and histogram in two launches (moe_route_brim)."""
+        B.moe_route_brim(logits, self.k, self.renorm, self.slot_of, self.R, self.topk_idx,
+                         self.topk_w, self.brim0, self.sfd_token, self.sfd_off, self.brim1,
+                         self.epd_off, self.epd_sfd, self.epd_gate, self.c_t, self.brim_ws,
+                         per_rank=self.per_rank, total=self.total, remote=self.remote,
+                         hist=self.hist, hist_accumulate=1, stream=stream)
+
     def dispatch(self, x, stream=None):
         B.moe_dispatch_gather(x, self.k, self.R, self.L, self.brim0, self.brim1, self.x_sfd,
                               self.x_epd, stream)
@@ -144,15 +153,21 @@ class MoELayer:
                                     self.total, self.remote, stream)
         B.moe_coact_histogram(self.topk_idx, self.E, self.hist, 1, stream)
 
-    def forward(self, logits, x, stream=None, stats=True):
-        """All steps of the layer on `stream`; returns y [T, d] (a view of self.y)."""
-        self.route(logits, stream)
-        self.build_brims(stream)
+    def forward(self, logits, x, stream=None, fused_index=True):
+        """All steps of the layer on `stream`; returns y [T, d] (a view of self.y).
+
+        fused_index: routing, BRIMs, counter and histogram through moe_route_brim
+        (two launches); otherwise through the four separate entry points."""
+        if fused_index:
+            self.route_brim(logits, stream)
+        else:
+            self.route(logits, stream)
+            self.build_brims(stream)
         self.dispatch(x, stream)
         self.experts(stream)
         self.shared_experts(x, stream)
         self.combine(stream)
-        if stats:
+        if not fused_index:
             self.statistics(stream)
         return self.y
 

@@ -165,6 +165,27 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
                            float* epd_gate, int32_t* c_t, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_route_brim -- moe_route_topk, moe_brim_build, moe_count_dispatched_rows
+ * and moe_coact_histogram in two kernel launches instead of six: one block per
+ * 32-token tile routes its tokens (warp per token, the code of
+ * moe_route_topk), builds the tile's BRIM column masks and adds to the counter
+ * and the histogram; the last tile to finish scans the columns; a second kernel
+ * scatters BRIM_0 / BRIM_1 and their inverses.  Every output is bit for bit
+ * the one the separate entry points produce.
+ *   arguments as in those entry points; per_rank / total / remote are given
+ *   together or all NULL (counter skipped); hist may be NULL (histogram
+ *   skipped), else it is cleared first unless hist_accumulate != 0.
+ *   ws  at least moe_route_brim_workspace_size(T, E, R) bytes, 16-byte aligned
+ * ------------------------------------------------------------------------- */
+size_t moe_route_brim_workspace_size(int T, int E, int R);
+int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const int32_t* slot_of,
+                   int R, int32_t* topk_idx, float* topk_w, int32_t* brim0, int32_t* sfd_token,
+                   int32_t* sfd_off, int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
+                   float* epd_gate, int32_t* c_t, int32_t* per_rank, int64_t* total,
+                   int64_t* remote, uint32_t* hist, int hist_accumulate, void* ws,
+                   size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_dispatch_gather -- ORI -> SFD -> EPD (Occult paper, Figure 4), guided by
  * the BRIMs: for every token t and rank r with s = BRIM_0[r][t] >= 0,
  *   x_sfd[s] = x[t]                         (the simulated all-to-all payload)

@@ -61,14 +61,14 @@ def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
 
 
 def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=None,
-                        epd_mode="auto"):
+                        epd_mode="auto", fused_index=True):
     inp = inputs.make_inputs(cfg, seed=seed)
     if slot_of is None:
         slot_of = np.arange(cfg.E, dtype=np.int32)
     layer = make_layer(cfg, inp, torch.from_numpy(slot_of), ffn_kind, epd_mode)
     logits, x = inp["logits"].to(DEV), inp["x"].to(DEV)
     layer.hist.zero_()
-    y = layer.forward(logits, x)
+    y = layer.forward(logits, x, fused_index=fused_index)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status() == moe.MOE_OK
     idx_ref, w_ref = oracle_route(inp["logits"], cfg.k, cfg.renorm)
@@ -113,6 +113,37 @@ def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=Non
 def test_tiny_layer(dtype, renorm):
     cfg = inputs.CONFIGS["tiny"].with_(dtype=dtype, renorm=renorm)
     run_and_check_small(cfg)
+
+
+@pytest.mark.parametrize("cfg", [
+    inputs.CONFIGS["tiny"],
+    inputs.LayerConfig("sep", T=1000, d=256, f=192, E=16, k=4, R=4, seed=5),
+    inputs.LayerConfig("sep16", T=300, d=128, f=128, E=256, k=16, R=8, seed=3),
+], ids=["tiny", "sep", "sep16"])
+def test_separate_index_entry_points(cfg):
+    """moe_route_topk + moe_brim_build + counter + histogram called one by one."""
+    run_and_check_small(cfg, fused_index=False)
+
+
+def test_fused_index_equals_separate():
+    cfg = inputs.LayerConfig("fz", T=3000, d=128, f=128, E=64, k=6, R=8, bias_std=1.0, seed=17)
+    inp = inputs.make_inputs(cfg)
+    a = make_layer(cfg, inp)
+    b = make_layer(cfg, inp)
+    logits, x = inp["logits"].to(DEV), inp["x"].to(DEV)
+    a.hist.zero_(); b.hist.zero_()
+    ya = a.forward(logits, x, fused_index=True)
+    yb = b.forward(logits, x, fused_index=False)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    c_t = int(a.c_t.item())
+    assert c_t == int(b.c_t.item())
+    for name in ("topk_idx", "topk_w", "brim0", "sfd_off", "epd_off", "epd_sfd", "epd_gate",
+                 "per_rank", "total", "remote", "hist"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    assert torch.equal(a.sfd_token[:c_t], b.sfd_token[:c_t])
+    assert torch.equal(a.brim1[:, :c_t], b.brim1[:, :c_t])
+    assert torch.equal(ya, yb)
 
 
 @pytest.mark.parametrize("epd_mode", ["stored", "gather"])
