@@ -223,6 +223,18 @@ def occult_layer(x, slot_of, E, R, k, b, wg, wu, wd, kind=KIND_SWIGLU, shared=No
     return y_sfd[:c_t], y
 
 
+def prune(idx, w, slot_of, E, R, m):
+    """Routing-score-based collaboration pruning (returns pruned copies)."""
+    idx = np.array(idx, dtype=np.int32, order="C", copy=True)
+    w = np.array(w, dtype=np.float64, order="C", copy=True)
+    slot_of = np.ascontiguousarray(slot_of, dtype=np.int32)
+    T, k = idx.shape
+    rc = lib().oracle_prune(_p(idx), _p(w), T, k, _p(slot_of), E, R, int(m))
+    if rc != 0:
+        raise ValueError(f"oracle_prune failed ({rc})")
+    return idx, w
+
+
 def count_dispatched(idx, slot_of, E, R):
     """(per_rank int32 [R], total, remote) for one placement."""
     idx = np.ascontiguousarray(idx, dtype=np.int32)

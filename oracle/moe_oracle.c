@@ -40,6 +40,14 @@
  *       and are added after the routed combine.
  *   R8  Placement slot q = slot_of[e]; rank(e) = q / L, loc(e) = q % L;
  *       EPD groups are laid out in slot order.
+ *   R9  Routing-score-based collaboration pruning keeps, per token, the first
+ *       m distinct ranks met along its descending-score expert list (so the
+ *       ranks of its highest-scoring experts), drops every assignment on any
+ *       other rank (expert id -1 = empty slot), and rescales the kept gate
+ *       weights so that their sum equals the sum before pruning.
+ *   R10 An expert id of -1 in a top-k list is an empty slot: it is sent
+ *       nowhere and contributes nothing.  Any other id outside [0, E) is an
+ *       error.
  */
 #include <math.h>
 #include <stdint.h>
@@ -158,6 +166,7 @@ int oracle_brim(const int32_t* idx, const double* w, int T, int k,
   for (int t = 0; t < T; ++t)
     for (int j = 0; j < k; ++j) {
       int e = idx[(size_t)t * k + j];
+      if (e == -1) continue; /* empty slot (R10) */
       if (e < 0 || e >= E) { free(hit); return -3; }
       hit[(size_t)t * R + slot_of[e] / L] = 1;
     }
@@ -209,6 +218,7 @@ int oracle_brim(const int32_t* idx, const double* w, int T, int k,
   for (int t = 0; t < T; ++t) {
     for (int j = 0; j < k; ++j) {
       int e = idx[(size_t)t * k + j];
+      if (e == -1) continue;
       int q = slot_of[e];
       int r = q / L, l = q % L;
       int p = epd_off[q] + seen_e[e];
@@ -312,6 +322,7 @@ int oracle_dense_layer(const void* X, int xdt, int T, int d,
       for (int c = 0; c < d; ++c) y[c] = 0.0;
       for (int j = 0; j < k; ++j) {
         int e = idx[(size_t)t * k + j];
+        if (e == -1) continue; /* empty slot (R10) */
         if (e < 0 || e >= E) { bad = 1; continue; }
         expert_row(kind, a, (const char*)Wg + e * wg_stride * es,
                    (const char*)Wu + e * wg_stride * es,
@@ -376,16 +387,18 @@ int oracle_occult_layer(const void* X, int xdt, int T, int d,
     for (int c = 0; c < d; ++c)
       X_sfd[(size_t)s * d + c] = widen(X, (size_t)sfd_token[s] * d + c, xdt);
   /* 2. SFD -> EPD */
-  for (size_t p = 0; p < tk; ++p)
+  for (size_t p = 0; p < (size_t)epd_off[E]; ++p)
     for (int c = 0; c < d; ++c)
       X_epd[p * d + c] = X_sfd[(size_t)epd_sfd[p] * d + c];
-  /* 3. expert compute, one EPD group (slot) after another */
+  /* 3. expert compute, one EPD group (slot) after another; with empty slots
+   *    (R10) only the first epd_off[E] EPD rows exist */
+  const size_t n_epd = (size_t)epd_off[E];
 #pragma omp parallel
   {
     double* h = (double*)malloc(sizeof(double) * (size_t)(f > 0 ? f : 1));
     double* o = (double*)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(dynamic, 16)
-    for (long long pp = 0; pp < (long long)tk; ++pp) {
+    for (long long pp = 0; pp < (long long)n_epd; ++pp) {
       size_t p = (size_t)pp;
       int q = 0;
       while (!(epd_off[q] <= (int)p && (int)p < epd_off[q + 1])) ++q;
@@ -440,6 +453,56 @@ int oracle_occult_layer(const void* X, int xdt, int T, int d,
 }
 
 /* ------------------------------------------------------------------------
+ * Routing-score-based collaboration pruning [Occult, TL;DR: two pruning
+ * schemes, routing-score-based and similarity-based, minimise the all-to-all
+ * budget C_T; Abstract: collaboration pruning controllably minimises the
+ * cost], by reading R9.  In place on idx [T,k] (descending score) and
+ * w [T,k]:
+ *   keep = the first m distinct ranks met walking j = 0 .. k-1
+ *   for j with rank(idx[t][j]) not in keep: idx = -1, w = 0
+ *   kept w_j *= (sum_j w_j before) / (sum of kept w_j)
+ * m >= the number of distinct ranks leaves the token unchanged.
+ * ---------------------------------------------------------------------- */
+int oracle_prune(int32_t* idx, double* w, int T, int k, const int32_t* slot_of, int E, int R,
+                 int m) {
+  if (R < 1 || E % R != 0 || m < 1) return -1;
+  const int L = E / R;
+  int32_t* keep = (int32_t*)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+  if (!keep) return -2;
+  for (int t = 0; t < T; ++t) {
+    int32_t* id = idx + (size_t)t * k;
+    double* wt = w + (size_t)t * k;
+    int n_keep = 0;
+    for (int j = 0; j < k; ++j) {
+      if (id[j] == -1) continue;
+      int r = slot_of[id[j]] / L, known = 0;
+      for (int i = 0; i < n_keep; ++i)
+        if (keep[i] == r) known = 1;
+      if (!known && n_keep < m) keep[n_keep++] = r;
+    }
+    double before = 0.0, kept = 0.0;
+    for (int j = 0; j < k; ++j) before += wt[j];
+    for (int j = 0; j < k; ++j) {
+      if (id[j] == -1) continue;
+      int r = slot_of[id[j]] / L, in = 0;
+      for (int i = 0; i < n_keep; ++i)
+        if (keep[i] == r) in = 1;
+      if (in) {
+        kept += wt[j];
+      } else {
+        id[j] = -1;
+        wt[j] = 0.0;
+      }
+    }
+    if (kept > 0.0)
+      for (int j = 0; j < k; ++j)
+        if (id[j] != -1) wt[j] = wt[j] * before / kept;
+  }
+  free(keep);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
  * Dispatched-row counter for a placement [Coupling, Abstract: a dispatcher
  * that sends each token to each GPU once; Occult, Fig. 2].
  *   per_rank[r] = #{t : token t selects an expert held by rank r}
@@ -458,8 +521,10 @@ int oracle_count_dispatched(const int32_t* idx, int T, int k, const int32_t* slo
     int src = (int)(((int64_t)t * R) / T);
     for (int r = 0; r < R; ++r) {
       int sent = 0;
-      for (int j = 0; j < k; ++j)
-        if (slot_of[idx[(size_t)t * k + j]] / L == r) sent = 1;
+      for (int j = 0; j < k; ++j) {
+        int e = idx[(size_t)t * k + j];
+        if (e != -1 && slot_of[e] / L == r) sent = 1;
+      }
       if (!sent) continue;
       per_rank[r] += 1;
       *total += 1;

@@ -401,3 +401,84 @@ def test_greedy_placement_recovers_planted_groups():
     L = cfg.L
     uniform = cfg.R * (1 - math.comb(cfg.E - L, cfg.k) / math.comb(cfg.E, cfg.k))
     assert abs(c_corr / cfg.T - (0.8 + 0.2 * uniform)) < 0.05
+
+
+# --------------------------------------------------------------------------
+# routing-score-based collaboration pruning
+# --------------------------------------------------------------------------
+def test_prune_hand_worked():
+    with open(os.path.join(GOLDEN, "prune_small.json")) as fh:
+        g = json.load(fh)
+    idx = np.array(g["topk_idx"], np.int32)
+    w = np.array(g["topk_w"], np.float64)
+    ident = np.arange(g["E"], dtype=np.int32)
+    assert oracle.brim(idx, w, ident, g["E"], g["R"])["c_t"] == g["c_t_before"]
+    pi, pw = oracle.prune(idx, w, ident, g["E"], g["R"], g["m"])
+    assert pi.tolist() == g["pruned_idx"]
+    np.testing.assert_allclose(pw, np.array(g["pruned_w"]), rtol=1e-15)
+    assert oracle.brim(pi, pw, ident, g["E"], g["R"])["c_t"] == g["c_t_after"]
+    # m = R keeps everything
+    pi2, pw2 = oracle.prune(idx, w, ident, g["E"], g["R"], g["R"])
+    assert np.array_equal(pi2, idx) and np.array_equal(pw2, w)
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 8])
+def test_prune_properties(m):
+    cfg = inputs.CONFIGS["olmoe"].with_(T=600)
+    idx, w = oracle.route(inputs.make_logits(cfg).numpy(), cfg.k, 0)
+    slot_of = np.random.default_rng(6).permutation(cfg.E).astype(np.int32)
+    pi, pw = oracle.prune(idx, w, slot_of, cfg.E, cfg.R, m)
+    L = cfg.L
+    # gate sums are preserved; dropped entries carry no weight
+    np.testing.assert_allclose(pw.sum(1), w.sum(1), rtol=1e-13)
+    assert np.all(pw[pi == -1] == 0)
+    # kept entries are unchanged ids in their places; at most m ranks per token;
+    # the top-1 expert is always kept
+    keep = pi != -1
+    assert np.array_equal(pi[keep], idx[keep])
+    assert np.all(pi[:, 0] == idx[:, 0])
+    for t in range(cfg.T):
+        ranks = {slot_of[e] // L for e in pi[t] if e != -1}
+        assert len(ranks) <= m
+        # a kept rank is one of the first m distinct ranks of the original order
+        first = []
+        for e in idx[t]:
+            r = slot_of[e] // L
+            if r not in first:
+                first.append(r)
+        assert ranks == set(first[:m])
+    # BRIMs and counter with empty slots: one EPD row per kept assignment
+    b = oracle.brim(pi, pw, slot_of, cfg.E, cfg.R)
+    _check_brim_invariants_with_empty(pi, b, cfg.E, cfg.R)
+    _, total, _ = oracle.count_dispatched(pi, slot_of, cfg.E, cfg.R)
+    assert total == b["c_t"] <= cfg.T * m
+    if m == 1:
+        assert b["c_t"] == cfg.T
+
+
+def _check_brim_invariants_with_empty(idx, b, E, R):
+    n_valid = int((idx != -1).sum())
+    assert b["epd_off"][E] == n_valid
+    valid = b["brim1"][:, :b["c_t"]]
+    assert sorted(valid[valid >= 0].tolist()) == list(range(n_valid))
+    assert sorted(b["brim0"][b["brim0"] >= 0].tolist()) == list(range(b["c_t"]))
+
+
+def test_pruned_layer_emulation_equals_dense():
+    cfg = inputs.CONFIGS["tiny"].with_(T=64, E=8, k=4, R=4)
+    inp = inputs.make_inputs(cfg)
+    x = bf16_bits(inp["x"])
+    wg, wu, wd = bf16_bits(inp["wg"]), bf16_bits(inp["wu"]), bf16_bits(inp["wd"])
+    idx, w = oracle.route(inp["logits"].numpy(), cfg.k, 0)
+    slot_of = np.arange(cfg.E, dtype=np.int32)
+    pi, pw = oracle.prune(idx, w, slot_of, cfg.E, cfg.R, 1)
+    b = oracle.brim(pi, pw, slot_of, cfg.E, cfg.R)
+    _, y = oracle.occult_layer(x, slot_of, cfg.E, cfg.R, cfg.k, b, wg, wu, wd)
+    y_dense = oracle.dense_layer(x, pi, pw, wg, wu, wd)
+    scale = np.abs(y_dense).max(1, keepdims=True)
+    assert np.all(np.abs(y - y_dense) <= 1e-12 * scale)
+    # identity experts: a pruned token returns its (preserved) gate sum times x
+    _, yi = oracle.occult_layer(inp["x"].float().numpy(), slot_of, cfg.E, cfg.R, cfg.k, b,
+                                None, None, None, kind=oracle.KIND_IDENTITY)
+    np.testing.assert_allclose(yi, w.sum(1, keepdims=True) * inp["x"].double().numpy(),
+                               rtol=1e-12)
