@@ -238,7 +238,21 @@ def run_ours(args, cfg):
         kw.update(sg=inp.pop("sg"), su=inp.pop("su"), sd=inp.pop("sd"))
     layer = MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
                      dtype=inputs.torch_dtype(cfg), S=cfg.S, fs=cfg.fs, slot_of=slot_of,
-                     device=dev, **kw)
+                     device=dev, prune_m=args.prune, **kw)
+    prune_info = None
+    if args.prune > 0:
+        # the same layer without pruning, once, for C_T and the output deviation
+        layer.prune_m = 0
+        y_full = layer.forward(inp["logits"], inp["x"]).clone()
+        c_t_full = int(layer.c_t.item())
+        layer.prune_m = args.prune
+        y_pruned = layer.forward(inp["logits"], inp["x"]).float()
+        dev_rows = (y_pruned - y_full.float()).abs().amax(1) / y_full.float().abs().amax(1).clamp_min(1e-30)
+        prune_info = {"m": args.prune, "c_t_unpruned": c_t_full, "c_t_pruned": int(layer.c_t.item()),
+                      "c_t_reduction": 1 - int(layer.c_t.item()) / max(c_t_full, 1),
+                      "output_max_row_rel_dev": float(dev_rows.max()),
+                      "output_mean_row_rel_dev": float(dev_rows.mean())}
+        torch.cuda.synchronize(dev)
     del kw
     logits, x = inp["logits"], inp["x"]
     stream = torch.cuda.current_stream(dev)
@@ -373,6 +387,7 @@ def run_ours(args, cfg):
             "layer_roofline": {"t_roof_ms": layer_roof_s * 1e3, "frac": layer_roof_s * 1e3 /
                                ms_per_step, "flops": flops, "bytes": bytes_},
             "c_t": c_t, "tk_rows": cfg.T * cfg.k, "e2e": e2e, "cpu_baseline": cpu,
+            "prune": prune_info,
             "clocks": clocks.summary(),
             "gpu_launches": launches_per_step(cfg) * args.steps,
             "ffn_ms": statistics.mean(ffn_ms),
@@ -456,6 +471,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--placement", default="contiguous", choices=["contiguous", "histogram"])
+    ap.add_argument("--prune", type=int, default=0,
+                    help="routing-score-based collaboration pruning: keep each token's first "
+                         "PRUNE ranks (0 = off)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     cfg = inputs.CONFIGS[args.config]

@@ -12,6 +12,6 @@ from ._binding import (  # noqa: F401
     moe_expert_ffn, moe_expert_ffn_workspace_size, moe_get_device_status,
     moe_prepare_shared_weights, moe_prepare_weights, moe_route_topk, moe_set_debug,
     moe_layer_workspace_size, moe_layer_forward, moe_layer_forward_host, moe_place_greedy,
-    moe_route_brim, moe_route_brim_workspace_size,
+    moe_route_brim, moe_route_brim_workspace_size, moe_prune_topk,
 )
 from .layer import MoELayer  # noqa: F401

@@ -34,7 +34,7 @@ EXPORTS = (
     "moe_prepare_weights", "moe_prepare_shared_weights", "moe_expert_ffn_workspace_size",
     "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
     "moe_layer_workspace_size", "moe_layer_forward", "moe_layer_forward_host",
-    "moe_place_greedy", "moe_route_brim_workspace_size", "moe_route_brim",
+    "moe_place_greedy", "moe_route_brim_workspace_size", "moe_route_brim", "moe_prune_topk",
 )
 
 
@@ -155,13 +155,20 @@ def moe_route_brim_workspace_size(T, E, R) -> int:
     return int(load().moe_route_brim_workspace_size(int(T), int(E), int(R)))
 
 
+def moe_prune_topk(topk_idx, topk_w, slot_of, E, R, m, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_prune_topk", load().moe_prune_topk(
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"), T, k,
+        _ptr(slot_of, I32, "slot_of"), int(E), int(R), int(m), _stream(stream)))
+
+
 def moe_route_brim(logits, k, renorm, slot_of, R, topk_idx, topk_w, brim0, sfd_token, sfd_off,
                    brim1, epd_off, epd_sfd, epd_gate, c_t, ws, per_rank=None, total=None,
-                   remote=None, hist=None, hist_accumulate=0, stream=None):
+                   remote=None, hist=None, hist_accumulate=0, prune_m=0, stream=None):
     T, E = logits.shape
     _check("moe_route_brim", load().moe_route_brim(
         _ptr(logits, F32, "logits"), T, E, int(k), int(renorm), _ptr(slot_of, I32, "slot_of"),
-        int(R), _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"),
+        int(R), int(prune_m), _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"),
         _ptr(brim0, I32, "brim0"), _ptr(sfd_token, I32, "sfd_token"), _ptr(sfd_off, I32, "sfd_off"),
         _ptr(brim1, I32, "brim1"), _ptr(epd_off, I32, "epd_off"), _ptr(epd_sfd, I32, "epd_sfd"),
         _ptr(epd_gate, F32, "epd_gate"), _ptr(c_t, I32, "c_t"),
@@ -257,11 +264,11 @@ def moe_layer_workspace_size(T, d, f, E, k, R, S, fs, dtype_code_, host_staging)
 
 def moe_layer_forward(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, y, ws, sw_gu=None,
                       sw_dn=None, S=0, fs=0, c_t=None, per_rank=None, total=None, remote=None,
-                      hist=None, stream=None):
+                      hist=None, prune_m=0, stream=None):
     T, E = logits.shape
     d = x.shape[1]
     _check("moe_layer_forward", load().moe_layer_forward(
-        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(S), int(fs),
+        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(prune_m), int(S), int(fs),
         dtype_code(x.dtype), _ptr(logits, F32, "logits"), _ptr(x, _ACT, "x"),
         _ptr(slot_of, I32, "slot_of"), _ptr(w_gu, x.dtype, "w_gu"), _ptr(w_dn, x.dtype, "w_dn"),
         _ptr(sw_gu, x.dtype, "sw_gu"), _ptr(sw_dn, x.dtype, "sw_dn"), _ptr(y, x.dtype, "y"),
@@ -271,12 +278,12 @@ def moe_layer_forward(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, y, ws, sw
 
 
 def moe_layer_forward_host(h_logits, h_x, k, R, renorm, slot_of, w_gu, w_dn, f, h_y, ws,
-                           sw_gu=None, sw_dn=None, S=0, fs=0, stream=None):
+                           sw_gu=None, sw_dn=None, S=0, fs=0, prune_m=0, stream=None):
     """The layer on host buffers: H2D copies, every step, D2H copy, then synchronise."""
     T, E = h_logits.shape
     d = h_x.shape[1]
     _check("moe_layer_forward_host", load().moe_layer_forward_host(
-        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(S), int(fs),
+        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(prune_m), int(S), int(fs),
         dtype_code(h_x.dtype), _host_ptr(h_logits, F32, "h_logits"), _host_ptr(h_x, _ACT, "h_x"),
         _ptr(slot_of, I32, "slot_of"), _ptr(w_gu, h_x.dtype, "w_gu"),
         _ptr(w_dn, h_x.dtype, "w_dn"), _ptr(sw_gu, h_x.dtype, "sw_gu"),

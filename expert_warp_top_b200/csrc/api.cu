@@ -509,13 +509,40 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
 }
 
 // ---------------------------------------------------------------------------
+int moe_prune_topk(int32_t* topk_idx, float* topk_w, int T, int k, const int32_t* slot_of, int E,
+                   int R, int m, moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  MOE_REQUIRE(m >= 1, MOE_ERR_INVALID_ARG, "m must be >= 1 (got %d)", m);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(topk_idx && topk_w && slot_of, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const dim3 grid((T + 255) / 256), block(256);
+#define MOE_PRUNE(KM) \
+  MOE_CUDA(launch_k(moe::prune_kernel<KM>, grid, block, 0, stream, topk_idx, topk_w, T, k, slot_of, E, R, m))
+  if (k <= 2) {
+    MOE_PRUNE(2);
+  } else if (k <= 4) {
+    MOE_PRUNE(4);
+  } else if (k <= 8) {
+    MOE_PRUNE(8);
+  } else {
+    MOE_PRUNE(16);
+  }
+#undef MOE_PRUNE
+  MOE_LAUNCHED("prune_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
 size_t moe_route_brim_workspace_size(int T, int E, int R) {
   if (T < 0 || E < 1 || R < 1) return 0;
   return align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)) + 512;
 }
 
 int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const int32_t* slot_of,
-                   int R, int32_t* topk_idx, float* topk_w, int32_t* brim0, int32_t* sfd_token,
+                   int R, int prune_m, int32_t* topk_idx, float* topk_w, int32_t* brim0, int32_t* sfd_token,
                    int32_t* sfd_off, int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
                    float* epd_gate, int32_t* c_t, int32_t* per_rank, int64_t* total,
                    int64_t* remote, uint32_t* hist, int hist_accumulate, void* ws,
@@ -523,6 +550,7 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   int rc = check_common(T, E, k, R);
   if (rc) return rc;
   MOE_REQUIRE(renorm == 0 || renorm == 1, MOE_ERR_INVALID_ARG, "renorm must be 0 or 1");
+  MOE_REQUIRE(prune_m >= 0, MOE_ERR_INVALID_ARG, "prune_m must be >= 0 (0 = no pruning)");
   MOE_REQUIRE(slot_of && sfd_off && epd_off && c_t, MOE_ERR_INVALID_ARG, "null pointer");
   MOE_REQUIRE((per_rank == nullptr) == (total == nullptr) && (total == nullptr) == (remote == nullptr),
               MOE_ERR_INVALID_ARG, "per_rank, total and remote are given together or not at all");
@@ -557,7 +585,8 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   auto* rem = reinterpret_cast<unsigned long long*>(remote);
 #define MOE_ROUTE_BRIM(KM)                                                                    \
   MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM>, dim3(n_tiles), dim3(1024), 0, stream,    \
-                    logits, T, E, k, renorm, slot_of, R, n_tiles, topk_idx, topk_w, masks,      \
+                    logits, T, E, k, renorm, slot_of, R, prune_m, n_tiles, topk_idx, topk_w,    \
+                    masks,                                                                      \
                     sfd_off, epd_off, c_t, per_rank, tot, rem, hist, ticket, di->err_flag));    \
   MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3((n_tiles + 3) / 4), dim3(128), 0,      \
                     stream, topk_idx, topk_w, slot_of, T, k, E, R, n_tiles,                     \
@@ -903,7 +932,8 @@ size_t carve_layer(char* base, int T, int d, int f, int E, int k, int R, int S, 
   return c.off + 256;
 }
 
-int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs, int dtype,
+int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int prune_m, int S, int fs,
+                int dtype,
                 const float* logits, const void* x, const int32_t* slot_of, const void* w_gu,
                 const void* w_dn, const void* sw_gu, const void* sw_dn, void* y, int32_t* c_t_out,
                 int32_t* per_rank, int64_t* total, int64_t* remote, uint32_t* hist,
@@ -912,7 +942,8 @@ int layer_steps(int T, int d, int f, int E, int k, int R, int renorm, int S, int
   const size_t tk = (size_t)T * k;
   const size_t cap = (size_t)T * (k < R ? k : R);
   int rc;
-  if ((rc = moe_route_brim(logits, T, E, k, renorm, slot_of, R, st.topk_idx, st.topk_w, st.brim0,
+  if ((rc = moe_route_brim(logits, T, E, k, renorm, slot_of, R, prune_m, st.topk_idx, st.topk_w,
+                           st.brim0,
                            st.sfd_token, st.sfd_off, st.brim1, st.epd_off, st.epd_sfd,
                            st.epd_gate, c_t_out ? c_t_out : st.c_t,
                            per_rank ? per_rank : st.per_rank, total ? total : st.total,
@@ -966,8 +997,8 @@ size_t moe_layer_workspace_size(int T, int d, int f, int E, int k, int R, int S,
   return carve_layer(nullptr, T, d, f, E, k, R, S, fs, dtype, host_staging != 0, nullptr);
 }
 
-int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
-                      int dtype, const float* logits, const void* x, const int32_t* slot_of,
+int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int prune_m, int S,
+                      int fs, int dtype, const float* logits, const void* x, const int32_t* slot_of,
                       const void* w_gu, const void* w_dn, const void* sw_gu, const void* sw_dn,
                       void* y, int32_t* c_t, int32_t* per_rank, int64_t* total, int64_t* remote,
                       uint32_t* hist, void* ws, size_t ws_bytes, moe_stream_t stream) {
@@ -983,12 +1014,14 @@ int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int 
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   LayerState st;
   carve_layer(base, T, d, f, E, k, R, S, fs, dtype, false, &st);
-  return layer_steps(T, d, f, E, k, R, renorm, S, fs, dtype, logits, x, slot_of, w_gu, w_dn,
+  MOE_REQUIRE(prune_m >= 0, MOE_ERR_INVALID_ARG, "prune_m must be >= 0 (0 = no pruning)");
+  return layer_steps(T, d, f, E, k, R, renorm, prune_m, S, fs, dtype, logits, x, slot_of, w_gu,
+                     w_dn,
                      sw_gu, sw_dn, y, c_t, per_rank, total, remote, hist, st, stream);
 }
 
-int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
-                           int dtype, const float* h_logits, const void* h_x,
+int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int prune_m,
+                           int S, int fs, int dtype, const float* h_logits, const void* h_x,
                            const int32_t* slot_of, const void* w_gu, const void* w_dn,
                            const void* sw_gu, const void* sw_dn, void* h_y, void* ws,
                            size_t ws_bytes, moe_stream_t stream) {
@@ -1009,7 +1042,9 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
   MOE_CUDA(cudaMemcpyAsync(st.logits, h_logits, sizeof(float) * (size_t)T * E,
                            cudaMemcpyHostToDevice, stream));
   MOE_CUDA(cudaMemcpyAsync(st.x, h_x, xb, cudaMemcpyHostToDevice, stream));
-  rc = layer_steps(T, d, f, E, k, R, renorm, S, fs, dtype, st.logits, st.x, slot_of, w_gu, w_dn,
+  MOE_REQUIRE(prune_m >= 0, MOE_ERR_INVALID_ARG, "prune_m must be >= 0 (0 = no pruning)");
+  rc = layer_steps(T, d, f, E, k, R, renorm, prune_m, S, fs, dtype, st.logits, st.x, slot_of,
+                   w_gu, w_dn,
                    sw_gu, sw_dn, st.y, nullptr, nullptr, nullptr, nullptr, nullptr, st, stream);
   if (rc) return rc;
   MOE_CUDA(cudaMemcpyAsync(h_y, st.y, xb, cudaMemcpyDeviceToHost, stream));

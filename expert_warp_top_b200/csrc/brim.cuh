@@ -39,9 +39,10 @@ struct TokenRoute {
   bool first[KMAX];
 };
 
-// Builds a token's route from its k expert ids.  Returns false (and raises
-// the error flag) when an expert id is out of range or repeated; such a token
-// is sent nowhere.
+// Builds a token's route from its k expert ids.  An id of -1 is an empty slot
+// (a pruned assignment): it is sent nowhere and is not an error.  Returns
+// false (and raises the error flag) when an id is otherwise out of range or
+// repeated; such a token is sent nowhere.
 template <int KMAX>
 __device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
                                                  const int32_t* __restrict__ slot_of, int k,
@@ -52,7 +53,7 @@ __device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
   for (int j = 0; j < KMAX; ++j) {
     tr.slot[j] = -1;
     tr.rank[j] = -1;
-    if (j < k) {
+    if (j < k && ids[j] != -1) {
       const int e = ids[j];
       const int q = (e >= 0 && e < E) ? __ldg(slot_of + e) : -1;
       if (q < 0 || q >= E) ok = false;
@@ -62,11 +63,11 @@ __device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
   }
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
-    bool first = j < k;
+    bool first = j < k && tr.slot[j] >= 0;
 #pragma unroll
     for (int i = 0; i < j; ++i) {
-      if (j < k) {  // entries past k are padding and compare with nothing
-        if (tr.slot[i] == tr.slot[j]) ok = false;  // the same expert twice
+      if (j < k && tr.slot[j] >= 0 && tr.slot[i] >= 0) {  // empty slots compare with nothing
+        if (tr.slot[i] == tr.slot[j]) ok = false;         // the same expert twice
         if (tr.rank[i] == tr.rank[j]) first = false;
       }
     }
@@ -74,6 +75,59 @@ __device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
   }
   if (!ok && err) raise_error(err, kErrIndex);
   return ok;
+}
+
+// Routing-score-based collaboration pruning of one token (in registers): keep
+// the first m distinct ranks met along the descending-score list, empty every
+// slot on another rank, and rescale the kept gates to the original sum.
+template <int KMAX>
+__device__ __forceinline__ void prune_token(int (&ids)[KMAX], float (&gates)[KMAX],
+                                            const int32_t* __restrict__ slot_of, int k, int E,
+                                            int L, int m) {
+  int rank[KMAX];
+  bool keep[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const int e = ids[j];
+    rank[j] = (j < k && e >= 0 && e < E) ? __ldg(slot_of + e) / L : -1;
+  }
+  int n_kept_ranks = 0;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    keep[j] = false;
+    if (rank[j] < 0) continue;
+    bool seen = false, seen_kept = false;
+#pragma unroll
+    for (int i = 0; i < j; ++i)
+      if (rank[i] == rank[j]) {
+        seen = true;
+        seen_kept |= keep[i];
+      }
+    if (!seen && n_kept_ranks < m) {
+      keep[j] = true;
+      ++n_kept_ranks;
+    } else if (seen) {
+      keep[j] = seen_kept;
+    }
+  }
+  float before = 0.f, kept = 0.f;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    if (j < k) {
+      before += gates[j];
+      if (keep[j]) kept += gates[j];
+    }
+  const float scale = kept > 0.f ? before / kept : 0.f;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    if (j < k) {
+      if (keep[j]) {
+        gates[j] *= scale;
+      } else if (rank[j] >= 0) {
+        ids[j] = -1;
+        gates[j] = 0.f;
+      }
+    }
 }
 
 // Loads token t's k expert ids from topk_idx and builds its route.
@@ -99,7 +153,7 @@ __device__ __forceinline__ void tile_masks(uint32_t* mask, int ncol, int R, bool
     const uint32_t bit = 1u << lane;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      if (j < k) {
+      if (j < k && tr.slot[j] >= 0) {
         atomicOr(&mask[R + tr.slot[j]], bit);
         if (tr.first[j]) atomicOr(&mask[tr.rank[j]], bit);
       }
@@ -264,7 +318,7 @@ __global__ void __launch_bounds__(128) brim_scatter_kernel(
   }
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
-    if (j < k) {
+    if (j < k && tr.slot[j] >= 0) {
       const int q = tr.slot[j];
       int s = -1;
 #pragma unroll
@@ -351,9 +405,9 @@ __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restri
       ids[j] = 0;
       if (j < k) {
         ids[j] = __ldg(topk_idx + (size_t)t * k + j);
-        if (ids[j] < 0 || ids[j] >= E) ok = false;
+        if (ids[j] != -1 && (ids[j] < 0 || ids[j] >= E)) ok = false;
 #pragma unroll
-        for (int i = 0; i < j; ++i) ok &= ids[i] != ids[j];
+        for (int i = 0; i < j; ++i) ok &= ids[j] == -1 || ids[i] != ids[j];
       }
     }
     if (!ok) {
@@ -363,7 +417,7 @@ __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restri
       for (int a = 0; a < KMAX; ++a)
 #pragma unroll
         for (int b = 0; b < KMAX; ++b)
-          if (a < k && b < k) {
+          if (a < k && b < k && ids[a] >= 0 && ids[b] >= 0) {
             const int cell = ids[a] * E + ids[b];
             if (use_smem) atomicAdd(&sh[cell], 1u);
             else atomicAdd(&hist[cell], 1u);
@@ -375,6 +429,31 @@ __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restri
     for (int i = threadIdx.x; i < E * E; i += blockDim.x)
       if (sh[i]) atomicAdd(&hist[i], sh[i]);
   }
+}
+
+// ---- collaboration pruning, in place ----------------------------------------
+template <int KMAX>
+__global__ void __launch_bounds__(256) prune_kernel(int32_t* __restrict__ topk_idx,
+                                                    float* __restrict__ topk_w, int T, int k,
+                                                    const int32_t* __restrict__ slot_of, int E,
+                                                    int R, int m) {
+  pdl_enter();
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  int ids[KMAX];
+  float gates[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    ids[j] = j < k ? topk_idx[(size_t)t * k + j] : -1;
+    gates[j] = j < k ? topk_w[(size_t)t * k + j] : 0.f;
+  }
+  prune_token<KMAX>(ids, gates, slot_of, k, E, E / R, m);
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    if (j < k) {
+      topk_idx[(size_t)t * k + j] = ids[j];
+      topk_w[(size_t)t * k + j] = gates[j];
+    }
 }
 
 }  // namespace moe

@@ -18,13 +18,15 @@ namespace moe {
 template <int KMAX>
 __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
-    const int32_t* __restrict__ slot_of, int R, int n_tiles, int32_t* __restrict__ topk_idx,
+    const int32_t* __restrict__ slot_of, int R, int prune_m, int n_tiles,
+    int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_w, uint32_t* __restrict__ masks, int32_t* __restrict__ sfd_off,
     int32_t* __restrict__ epd_off, int32_t* __restrict__ c_t, int32_t* __restrict__ per_rank,
     unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
     uint32_t* __restrict__ hist, unsigned* __restrict__ ticket, unsigned* err) {
   pdl_enter();
   __shared__ int s_ids[32][KMAX];
+  __shared__ float s_gates[32][KMAX];
   __shared__ uint32_t s_mask[kMaxCols];
   __shared__ int32_t s_scan_a[kMaxCols], s_scan_b[kMaxCols];
   __shared__ bool s_last;
@@ -38,14 +40,11 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
     const int t = tile * kBrimTileTokens + warp;
     int id = -1;
     float gate = 0.f;
-    if (t < T) {
-      route_token_warp(logits + (size_t)t * E, E, k, renorm, &id, &gate);
-      if ((int)lane < k) {
-        topk_idx[(size_t)t * k + lane] = id;
-        topk_w[(size_t)t * k + lane] = gate;
-      }
+    if (t < T) route_token_warp(logits + (size_t)t * E, E, k, renorm, &id, &gate);
+    if ((int)lane < KMAX) {
+      s_ids[warp][lane] = (t < T && (int)lane < k) ? id : -1;
+      s_gates[warp][lane] = (t < T && (int)lane < k) ? gate : 0.f;
     }
-    if ((int)lane < KMAX) s_ids[warp][lane] = (t < T && (int)lane < k) ? id : -1;
   }
   __syncthreads();
 
@@ -53,8 +52,20 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
   if (warp == 0) {
     const int t = tile * kBrimTileTokens + (int)lane;
     int ids[KMAX];
+    float gates[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) ids[j] = s_ids[lane][j];
+    for (int j = 0; j < KMAX; ++j) {
+      ids[j] = s_ids[lane][j];
+      gates[j] = s_gates[lane][j];
+    }
+    if (prune_m > 0 && t < T) prune_token<KMAX>(ids, gates, slot_of, k, E, L, prune_m);
+    if (t < T)
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k) {
+          topk_idx[(size_t)t * k + j] = ids[j];
+          topk_w[(size_t)t * k + j] = gates[j];
+        }
     TokenRoute<KMAX> tr;
     const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
     tile_masks<KMAX>(s_mask, ncol, R, active, k, tr);
@@ -86,7 +97,8 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
       for (int a = 0; a < KMAX; ++a)
 #pragma unroll
         for (int b = 0; b < KMAX; ++b)
-          if (a < k && b < k) atomicAdd(&hist[ids[a] * E + ids[b]], 1u);
+          if (a < k && b < k && ids[a] >= 0 && ids[b] >= 0)
+            atomicAdd(&hist[ids[a] * E + ids[b]], 1u);
     }
   }
 

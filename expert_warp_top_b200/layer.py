@@ -31,13 +31,15 @@ from . import _binding as B
 class MoELayer:
     def __init__(self, *, T, d, f, E, k, R, renorm=0, dtype=torch.bfloat16, S=0, fs=0,
                  slot_of=None, wg=None, wu=None, wd=None, sg=None, su=None, sd=None,
-                 ffn_kind=B.MOE_FFN_SWIGLU, device="cuda", stream=None, epd_mode="auto"):
+                 ffn_kind=B.MOE_FFN_SWIGLU, device="cuda", stream=None, epd_mode="auto",
+                 prune_m=0):
         if E % R:
             raise ValueError("R must divide E")
         self.T, self.d, self.f, self.E, self.k, self.R = T, d, f, E, k, R
         self.L = E // R
         self.renorm, self.dtype, self.S, self.fs = renorm, dtype, S, fs
         self.ffn_kind = ffn_kind
+        self.prune_m = prune_m  # > 0: routing-score-based collaboration pruning
         if epd_mode == "auto":
             epd_mode = "direct" if E // R == 1 else "stored"
         if epd_mode not in ("stored", "direct", "gather"):
@@ -119,7 +121,7 @@ class MoELayer:
                          self.topk_w, self.brim0, self.sfd_token, self.sfd_off, self.brim1,
                          self.epd_off, self.epd_sfd, self.epd_gate, self.c_t, self.brim_ws,
                          per_rank=self.per_rank, total=self.total, remote=self.remote,
-                         hist=self.hist, hist_accumulate=1, stream=stream)
+                         hist=self.hist, hist_accumulate=1, prune_m=self.prune_m, stream=stream)
 
     def dispatch(self, x, stream=None):
         B.moe_dispatch_gather(x, self.k, self.R, self.L, self.brim0, self.brim1, self.x_sfd,
@@ -162,6 +164,9 @@ class MoELayer:
             self.route_brim(logits, stream)
         else:
             self.route(logits, stream)
+            if self.prune_m > 0:
+                B.moe_prune_topk(self.topk_idx, self.topk_w, self.slot_of, self.E, self.R,
+                                 self.prune_m, stream)
             self.build_brims(stream)
         self.dispatch(x, stream)
         self.experts(stream)
@@ -189,7 +194,8 @@ class MoELayer:
                             self.w_dn, self.f, y, self._layer_ws(False),
                             sw_gu=getattr(self, "sw_gu", None), sw_dn=getattr(self, "sw_dn", None),
                             S=self.S, fs=self.fs, c_t=self.c_t, per_rank=self.per_rank,
-                            total=self.total, remote=self.remote, hist=self.hist, stream=stream)
+                            total=self.total, remote=self.remote, hist=self.hist,
+                            prune_m=self.prune_m, stream=stream)
         return y
 
     def forward_host(self, h_logits, h_x, h_y, stream=None):
@@ -198,5 +204,5 @@ class MoELayer:
                                  self.w_gu, self.w_dn, self.f, h_y, self._layer_ws(True),
                                  sw_gu=getattr(self, "sw_gu", None),
                                  sw_dn=getattr(self, "sw_dn", None), S=self.S, fs=self.fs,
-                                 stream=stream)
+                                 prune_m=self.prune_m, stream=stream)
         return h_y

@@ -106,11 +106,31 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renorm,
                    int32_t* topk_idx, float* topk_w, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_prune_topk -- routing-score-based collaboration pruning (Occult paper,
+ * TL;DR: two pruning schemes, routing-score-based and similarity-based, that
+ * minimise the all-to-all budget C_T; Abstract: collaboration pruning
+ * controllably minimises the cost).  In place, per token, on a top-k list in
+ * descending score order:
+ *   keep the first m distinct ranks met along the list (the ranks of the
+ *   token's highest-scoring experts); every assignment on another rank becomes
+ *   an empty slot (id -1, weight 0); the kept weights are rescaled so that
+ *   their sum equals the sum before pruning.
+ *   topk_idx [T, k] int32, topk_w [T, k] float32 (device, in place)
+ *   m >= 1; m >= the token's number of distinct ranks leaves it unchanged.
+ * An id of -1 is accepted everywhere downstream as an empty slot: the BRIM
+ * build, the dispatch, the counter and the histogram skip it, and the EPD
+ * state then has epd_off[E] <= T*k rows.
+ * ------------------------------------------------------------------------- */
+int moe_prune_topk(int32_t* topk_idx, float* topk_w, int T, int k, const int32_t* slot_of,
+                   int E, int R, int m, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_brim_build -- the two bidirectional re-index matrices of the Occult
  * paper (Figure 5: BRIM_0 is [EP devices x ORI tokens], BRIM_1 is [local
  * experts per device x SFD tokens]) and the all-to-all budget C_T (TL;DR).
  * A token is sent once to every rank that holds at least one of its experts.
- *   topk_idx [T, k] int32   distinct expert ids per token (checked on device)
+ *   topk_idx [T, k] int32   distinct expert ids per token, or -1 for an empty
+ *                           slot (checked on device)
  *   topk_w   [T, k] float32 gate weights
  *   slot_of  [E] int32      placement (device)
  *   brim0    [R, T] int32   out: SFD row of (rank r, token t), or -1
@@ -172,14 +192,16 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
  * and the histogram; the last tile to finish scans the columns; a second kernel
  * scatters BRIM_0 / BRIM_1 and their inverses.  Every output is bit for bit
  * the one the separate entry points produce.
- *   arguments as in those entry points; per_rank / total / remote are given
+ *   prune_m > 0 applies moe_prune_topk with m = prune_m between routing and
+ *   the BRIMs (0 = no pruning);
+ *   other arguments as in those entry points; per_rank / total / remote are given
  *   together or all NULL (counter skipped); hist may be NULL (histogram
  *   skipped), else it is cleared first unless hist_accumulate != 0.
  *   ws  at least moe_route_brim_workspace_size(T, E, R) bytes, 16-byte aligned
  * ------------------------------------------------------------------------- */
 size_t moe_route_brim_workspace_size(int T, int E, int R);
 int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const int32_t* slot_of,
-                   int R, int32_t* topk_idx, float* topk_w, int32_t* brim0, int32_t* sfd_token,
+                   int R, int prune_m, int32_t* topk_idx, float* topk_w, int32_t* brim0, int32_t* sfd_token,
                    int32_t* sfd_off, int32_t* brim1, int32_t* epd_off, int32_t* epd_sfd,
                    float* epd_gate, int32_t* c_t, int32_t* per_rank, int64_t* total,
                    int64_t* remote, uint32_t* hist, int hist_accumulate, void* ws,
@@ -334,6 +356,8 @@ int moe_place_greedy(const uint32_t* hist, int E, int R, int32_t* slot_of);
  *   ws           at least moe_layer_workspace_size(...) bytes, 256-byte aligned;
  *                it holds every intermediate state (top-k, BRIMs, SFD / EPD
  *                rows, return rows) for the duration of the call
+ * prune_m > 0 prunes each token to its first prune_m ranks (moe_prune_topk)
+ * before the BRIMs are built; 0 keeps every assignment.
  * With one expert per rank (E == R) the GEMM reads the SFD payload in place
  * (the EPD state equals it row for row); otherwise the dispatch stores the
  * EPD rows.
@@ -344,13 +368,13 @@ int moe_place_greedy(const uint32_t* hist, int E, int R, int32_t* slot_of);
  * ------------------------------------------------------------------------- */
 size_t moe_layer_workspace_size(int T, int d, int f, int E, int k, int R, int S, int fs,
                                 int dtype, int host_staging);
-int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
-                      int dtype, const float* logits, const void* x, const int32_t* slot_of,
+int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int prune_m, int S,
+                      int fs, int dtype, const float* logits, const void* x, const int32_t* slot_of,
                       const void* w_gu, const void* w_dn, const void* sw_gu, const void* sw_dn,
                       void* y, int32_t* c_t, int32_t* per_rank, int64_t* total, int64_t* remote,
                       uint32_t* hist, void* ws, size_t ws_bytes, moe_stream_t stream);
-int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
-                           int dtype, const float* h_logits, const void* h_x,
+int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int prune_m,
+                           int S, int fs, int dtype, const float* h_logits, const void* h_x,
                            const int32_t* slot_of, const void* w_gu, const void* w_dn,
                            const void* sw_gu, const void* sw_dn, void* h_y,
                            void* ws, size_t ws_bytes, moe_stream_t stream);

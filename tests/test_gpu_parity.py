@@ -22,7 +22,7 @@ def softmax_rtol(E: int) -> float:
     return (E + 8) * 2.0 ** -23
 
 
-def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, epd_mode="auto"):
+def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, epd_mode="auto", prune_m=0):
     dt = inputs.torch_dtype(cfg)
     kw = {}
     if ffn_kind == moe.MOE_FFN_SWIGLU:
@@ -31,7 +31,8 @@ def make_layer(cfg, inp, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, epd_mode="au
             kw.update(sg=inp["sg"].to(DEV), su=inp["su"].to(DEV), sd=inp["sd"].to(DEV))
     return MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
                     dtype=dt, S=cfg.S if ffn_kind == moe.MOE_FFN_SWIGLU else 0, fs=cfg.fs,
-                    slot_of=slot_of, ffn_kind=ffn_kind, device=DEV, epd_mode=epd_mode, **kw)
+                    slot_of=slot_of, ffn_kind=ffn_kind, device=DEV, epd_mode=epd_mode,
+                    prune_m=prune_m, **kw)
 
 
 def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
@@ -50,9 +51,10 @@ def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
     assert np.array_equal(layer.sfd_token[:c_t].cpu().numpy(), b["sfd_token"])
     assert np.array_equal(layer.brim1[:, :c_t].cpu().numpy(), b["brim1"][:, :c_t])
     assert np.array_equal(layer.epd_off.cpu().numpy(), b["epd_off"])
-    tk = cfg.T * cfg.k
-    assert np.array_equal(layer.epd_sfd[:tk].cpu().numpy(), b["epd_sfd"])
-    assert np.array_equal(layer.epd_gate[:tk].cpu().numpy().astype(np.float64), b["epd_gate"])
+    n_epd = int(b["epd_off"][-1])  # T*k, or fewer with empty (pruned) slots
+    assert np.array_equal(layer.epd_sfd[:n_epd].cpu().numpy(), b["epd_sfd"][:n_epd])
+    assert np.array_equal(layer.epd_gate[:n_epd].cpu().numpy().astype(np.float64),
+                          b["epd_gate"][:n_epd])
     per_rank, total, remote = oracle.count_dispatched(idx, slot_of, cfg.E, cfg.R)
     assert np.array_equal(layer.per_rank.cpu().numpy(), per_rank)
     assert int(layer.total.item()) == total == c_t
@@ -61,17 +63,19 @@ def check_indices(layer, idx_ref, w_ref, cfg, slot_of):
 
 
 def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=None,
-                        epd_mode="auto", fused_index=True):
+                        epd_mode="auto", fused_index=True, prune_m=0):
     inp = inputs.make_inputs(cfg, seed=seed)
     if slot_of is None:
         slot_of = np.arange(cfg.E, dtype=np.int32)
-    layer = make_layer(cfg, inp, torch.from_numpy(slot_of), ffn_kind, epd_mode)
+    layer = make_layer(cfg, inp, torch.from_numpy(slot_of), ffn_kind, epd_mode, prune_m)
     logits, x = inp["logits"].to(DEV), inp["x"].to(DEV)
     layer.hist.zero_()
     y = layer.forward(logits, x, fused_index=fused_index)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status() == moe.MOE_OK
     idx_ref, w_ref = oracle_route(inp["logits"], cfg.k, cfg.renorm)
+    if prune_m:
+        idx_ref, w_ref = oracle.prune(idx_ref, w_ref, slot_of, cfg.E, cfg.R, prune_m)
     b = check_indices(layer, idx_ref, w_ref, cfg, slot_of)
     assert np.array_equal(layer.hist.cpu().numpy().astype(np.uint32),
                           oracle.coact_histogram(idx_ref, cfg.E))
@@ -81,8 +85,9 @@ def run_and_check_small(cfg, slot_of=None, ffn_kind=moe.MOE_FFN_SWIGLU, seed=Non
     x_sfd_ref = oracle.gather_rows(xo, b["sfd_token"])
     assert np.array_equal(to_oracle(layer.x_sfd[:c_t]), x_sfd_ref)
     if layer.x_epd is not None:
-        assert np.array_equal(to_oracle(layer.x_epd[:cfg.T * cfg.k]),
-                              oracle.gather_rows(x_sfd_ref, b["epd_sfd"]))
+        n_epd = int(b["epd_off"][-1])
+        assert np.array_equal(to_oracle(layer.x_epd[:n_epd]),
+                              oracle.gather_rows(x_sfd_ref, b["epd_sfd"][:n_epd]))
     # outputs against the BRIM-guided oracle and against the dense definition
     kind = oracle.KIND_IDENTITY if ffn_kind == moe.MOE_FFN_IDENTITY else oracle.KIND_SWIGLU
     w_ = (None, None, None) if kind == oracle.KIND_IDENTITY else \
@@ -346,3 +351,35 @@ def test_outputs_are_deterministic():
     y2 = layer.forward(logits, x).clone()
     torch.cuda.synchronize()
     assert torch.equal(y1, y2) and torch.equal(s1, layer.y_sfd)
+
+
+
+# ---------------------------------------------------------------------------
+# routing-score-based collaboration pruning
+@pytest.mark.parametrize("m", [1, 2, 3])
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "separate"])
+def test_pruned_layer(m, fused):
+    cfg = inputs.LayerConfig("prune", T=700, d=128, f=128, E=32, k=6, R=8, bias_std=0.5,
+                             seed=40 + m)
+    slot_of = np.random.default_rng(m).permutation(cfg.E).astype(np.int32)
+    layer, _ = run_and_check_small(cfg, slot_of, fused_index=fused, prune_m=m)
+    c_t = int(layer.c_t.item())
+    assert c_t <= cfg.T * m
+    if m == 1:
+        assert c_t == cfg.T
+
+
+def test_prune_kernel_equals_fused_prune():
+    cfg = inputs.LayerConfig("prunek", T=2000, d=128, f=128, E=64, k=8, R=8, seed=44)
+    inp = inputs.make_inputs(cfg, weights=False)
+    a = make_layer(cfg, inp, ffn_kind=moe.MOE_FFN_IDENTITY, prune_m=2)
+    logits = inp["logits"].to(DEV)
+    a.route_brim(logits)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=DEV)
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(logits, cfg.k, 0, idx, w)
+    moe.moe_prune_topk(idx, w, a.slot_of, cfg.E, cfg.R, 2)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    assert torch.equal(idx, a.topk_idx) and torch.equal(w, a.topk_w)
+    assert (idx == -1).any()
