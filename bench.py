@@ -61,6 +61,26 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest value of x over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(cfg, rank: int) -> int:
+    """Each rank runs its own independent batch (weak scaling): a distinct seed."""
+    return cfg.seed + 7919 * rank
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Tokens all ranks processed divided by the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_ms * 1e-3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -231,7 +251,7 @@ def run_ours(args, cfg):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     # each rank: its own independent batch (seed offset by rank), same weights recipe
-    inp = inputs.make_inputs(cfg, device=dev, seed=cfg.seed + 7919 * rank)
+    inp = inputs.make_inputs(cfg, device=dev, seed=rank_seed(cfg, rank))
     slot_of, placement_info = placement(cfg, args.placement, dev, inp["logits"])
     kw = dict(wg=inp.pop("wg"), wu=inp.pop("wu"), wd=inp.pop("wd"))
     if cfg.S:
@@ -330,13 +350,9 @@ def run_ours(args, cfg):
     status = B.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
-    value = world * cfg.T * args.steps / (total_ms * 1e-3)
+    value = whole_job_tokens_per_s(cfg.T, args.steps, world, total_ms)
 
     # end to end through the public API: host buffers in and out, copies timed
     e2e = None
@@ -450,14 +466,10 @@ def e2e_host(layer, inp, cfg, args, dev, world):
     t0 = time.perf_counter()
     for _ in range(args.steps):
         layer.forward_host(h_logits, h_x, h_y)
-    ms = (time.perf_counter() - t0) * 1e3
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks((time.perf_counter() - t0) * 1e3, dev)
     h2d = h_logits.numel() * h_logits.element_size() + h_x.numel() * h_x.element_size()
     d2h = h_y.numel() * h_y.element_size()
-    return {"value": world * cfg.T * args.steps / (ms * 1e-3), "unit": UNIT,
+    return {"value": whole_job_tokens_per_s(cfg.T, args.steps, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "api": "moe_layer_forward_host (C ABI, pinned host buffers, wall clock)"}
 
