@@ -269,3 +269,71 @@ def place_greedy(hist, R):
     if rc != 0:
         raise ValueError(f"oracle_place_greedy failed ({rc})")
     return slot_of
+
+
+def dense_layer_backward(x, idx, w, wg, wu, wd, dy, kind=KIND_SWIGLU, shared=None,
+                         tokens=None, experts=None, shared_grads=False):
+    """Backward of :func:`dense_layer` for the upstream gradient ``dy`` [T,d].
+
+    Returns a dict with ``dx`` [n,d] and ``dw`` [n,k] (n = len(tokens) or T),
+    and, when ``experts`` lists expert ids, ``dwg``/``dwu`` [n_exp,f,d] and
+    ``dwd`` [n_exp,d,f]; with ``shared_grads`` the shared experts' ``dsg``,
+    ``dsu``, ``dsd``.  Everything in double.
+    """
+    x = np.ascontiguousarray(x)
+    T, d = x.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    k = idx.shape[1]
+    if kind == KIND_IDENTITY:
+        E, f, wdt = int(idx.max()) + 1 if idx.size else 1, 0, DT_F64
+        wg = wu = wd = None
+    else:
+        wg = np.ascontiguousarray(wg); wu = np.ascontiguousarray(wu)
+        wd = np.ascontiguousarray(wd)
+        E, f, wdt = wg.shape[0], wg.shape[1], _dt(wg)
+    if shared is not None:
+        sg, su, sd = (np.ascontiguousarray(a) for a in shared)
+        S, fs = sg.shape[0], sg.shape[1]
+        if kind == KIND_IDENTITY:
+            wdt = _dt(sg)
+    else:
+        sg = su = sd = None
+        S, fs = 0, 0
+    if tokens is not None:
+        tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = len(tokens)
+    else:
+        n = T
+    out = dict(dx=np.empty((n, d)), dw=np.empty((n, k)))
+    if experts is not None:
+        experts = np.ascontiguousarray(experts, dtype=np.int32)
+        ne = len(experts)
+        out.update(dwg=np.empty((ne, f, d)), dwu=np.empty((ne, f, d)), dwd=np.empty((ne, d, f)))
+    else:
+        ne = 0
+    if shared_grads and S:
+        out.update(dsg=np.empty((S, fs, d)), dsu=np.empty((S, fs, d)), dsd=np.empty((S, d, fs)))
+    rc = lib().oracle_dense_layer_backward(
+        _p(x), _dt(x), T, d, _p(idx), _p(w), k, _p(wg), _p(wu), _p(wd), wdt, E, f, int(kind),
+        _p(sg), _p(su), _p(sd), S, fs, _p(dy), _p(tokens), n, _p(out["dx"]), _p(out["dw"]),
+        _p(experts), ne, _p(out.get("dwg")), _p(out.get("dwu")), _p(out.get("dwd")),
+        _p(out.get("dsg")), _p(out.get("dsu")), _p(out.get("dsd")))
+    if rc != 0:
+        raise ValueError(f"oracle_dense_layer_backward failed ({rc})")
+    return out
+
+
+def route_backward(logits, idx, dw, renorm: int):
+    """Gradient of the logits [T,E] (double) from the gate-weight gradient dw [T,k]."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    dw = np.ascontiguousarray(dw, dtype=np.float64)
+    k = idx.shape[1]
+    dl = np.empty((T, E))
+    rc = lib().oracle_route_backward(_p(logits), T, E, k, int(renorm), _p(idx), _p(dw), _p(dl))
+    if rc != 0:
+        raise ValueError(f"oracle_route_backward failed ({rc})")
+    return dl

@@ -48,6 +48,13 @@
  *   R10 An expert id of -1 in a top-k list is an empty slot: it is sent
  *       nowhere and contributes nothing.  Any other id outside [0, E) is an
  *       error.
+ *   R11 The backward pass is the exact derivative of the layer output for
+ *       fixed expert choices: the top-k selection is piecewise constant and
+ *       passes no gradient; the gate weights pass theirs through the softmax
+ *       variant of R4.  It is defined for unpruned routing.
+ *   R12 A weight gradient sums, over every (token, slot) routed to that
+ *       expert in ascending token order, the outer products of that row;
+ *       shared experts take every token with weight 1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -606,5 +613,233 @@ int oracle_place_greedy(const uint32_t* H, int E, int R, int32_t* slot_of) {
   }
   free(placed);
   free(members);
+  return 0;
+}
+
+
+/* ------------------------------------------------------------------------
+ * Backward pass (readings R11, R12).  The forward of one (token, expert)
+ * row is, with a = X[t] and gate weight w:
+ *     g = Wg a,  u = Wu a,  h_i = silu(g_i) u_i,  o = Wd h,  out = w o
+ * so for an upstream gradient dy = dL/d(out):
+ *     dL/dw     = <dy, o>
+ *     dh        = w Wd^T dy
+ *     dg_i      = dh_i u_i silu'(g_i),  silu'(z) = s (1 + z (1 - s)), s = 1/(1+e^-z)
+ *     du_i      = dh_i silu(g_i)
+ *     dL/da     = Wg^T dg + Wu^T du
+ *     dL/dWd    = w dy h^T,  dL/dWg = dg a^T,  dL/dWu = du a^T
+ * The identity expert (kind 1) has o = a: dL/dw = <dy, a>, dL/da = w dy.
+ *
+ * row_backward() fills h, dg, du (each [f]) and returns dL/dw; da (if not
+ * NULL) receives dL/da.  Weights are one expert's Wg,Wu [f,d], Wd [d,f].
+ * ---------------------------------------------------------------------- */
+static double row_backward(int kind, const double* a, const double* dy, double w,
+                           const void* Wg, const void* Wu, const void* Wd, int wdt,
+                           int d, int f, double* h, double* dg, double* du, double* da) {
+  if (kind == 1) {
+    double dw = 0.0;
+    for (int c = 0; c < d; ++c) dw += dy[c] * a[c];
+    if (da)
+      for (int c = 0; c < d; ++c) da[c] = w * dy[c];
+    return dw;
+  }
+  double dw = 0.0;
+  for (int i = 0; i < f; ++i) {
+    double g = 0.0, u = 0.0;
+    for (int c = 0; c < d; ++c) {
+      g += widen(Wg, (size_t)i * d + c, wdt) * a[c];
+      u += widen(Wu, (size_t)i * d + c, wdt) * a[c];
+    }
+    double s = 1.0 / (1.0 + exp(-g));
+    double silu = g * s;
+    h[i] = silu * u;
+    double wd_dy = 0.0; /* (Wd^T dy)_i */
+    for (int c = 0; c < d; ++c) wd_dy += widen(Wd, (size_t)c * f + i, wdt) * dy[c];
+    dw += wd_dy * h[i]; /* <dy, Wd h> summed by i */
+    double dh = w * wd_dy;
+    dg[i] = dh * u * s * (1.0 + g * (1.0 - s));
+    du[i] = dh * silu;
+  }
+  if (da)
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < f; ++i)
+        acc += widen(Wg, (size_t)i * d + c, wdt) * dg[i] + widen(Wu, (size_t)i * d + c, wdt) * du[i];
+      da[c] = acc;
+    }
+  return dw;
+}
+
+/* ------------------------------------------------------------------------
+ * Dense backward of the layer (no BRIM anywhere), the derivative of
+ * oracle_dense_layer() for an upstream gradient dY [T, d] (double):
+ *   dX[t]    = sum_j dL/da of row (t, j) + sum_s dL/da of shared row (t, s)
+ *   dW[t][j] = dL/dw of row (t, j)                     (0 for an empty slot)
+ * for the tokens in `tokens` (NULL = all T; outputs [n_tok, d], [n_tok, k];
+ * either output may be NULL).
+ * Weight gradients, each optional (NULL = not computed), over ALL T tokens:
+ *   dWg, dWu [n_exp, f, d], dWd [n_exp, d, f] for the experts listed in
+ *   `experts` (n_exp of them), and dSg, dSu [S, fs, d], dSd [S, d, fs].
+ * ---------------------------------------------------------------------- */
+int oracle_dense_layer_backward(const void* X, int xdt, int T, int d,
+                                const int32_t* idx, const double* w, int k,
+                                const void* Wg, const void* Wu, const void* Wd, int wdt,
+                                int E, int f, int kind,
+                                const void* Sg, const void* Su, const void* Sd, int S, int fs,
+                                const double* dY, const int32_t* tokens, int n_tok,
+                                double* dX, double* dW,
+                                const int32_t* experts, int n_exp,
+                                double* dWg, double* dWu, double* dWd,
+                                double* dSg, double* dSu, double* dSd) {
+  if (d < 1 || T < 0 || k < 1) return -1;
+  if (tokens == NULL) n_tok = T;
+  const size_t wg_stride = (size_t)f * d, wd_stride = (size_t)d * f;
+  const size_t sg_stride = (size_t)fs * d, sd_stride = (size_t)d * fs;
+  const size_t es = esize(wdt);
+  const int hmax = (f > fs ? f : fs) > 0 ? (f > fs ? f : fs) : 1;
+  int bad = 0;
+
+  /* 1. per-token input gradient and gate-weight gradient */
+  if (dX || dW) {
+#pragma omp parallel
+    {
+      double* a = (double*)malloc(sizeof(double) * (size_t)d);
+      double* da = (double*)malloc(sizeof(double) * (size_t)d);
+      double* h = (double*)malloc(sizeof(double) * (size_t)hmax);
+      double* dg = (double*)malloc(sizeof(double) * (size_t)hmax);
+      double* du = (double*)malloc(sizeof(double) * (size_t)hmax);
+#pragma omp for schedule(dynamic, 1)
+      for (int n = 0; n < n_tok; ++n) {
+        int t = tokens ? tokens[n] : n;
+        if (t < 0 || t >= T) { bad = 1; continue; }
+        const double* dy = dY + (size_t)t * d;
+        for (int c = 0; c < d; ++c) a[c] = widen(X, (size_t)t * d + c, xdt);
+        if (dX)
+          for (int c = 0; c < d; ++c) dX[(size_t)n * d + c] = 0.0;
+        for (int j = 0; j < k; ++j) {
+          int e = idx[(size_t)t * k + j];
+          if (dW) dW[(size_t)n * k + j] = 0.0;
+          if (e == -1) continue;
+          if (e < 0 || e >= E) { bad = 1; continue; }
+          double g = row_backward(kind, a, dy, w[(size_t)t * k + j],
+                                  (const char*)Wg + e * wg_stride * es,
+                                  (const char*)Wu + e * wg_stride * es,
+                                  (const char*)Wd + e * wd_stride * es, wdt, d, f, h, dg, du,
+                                  dX ? da : NULL);
+          if (dW) dW[(size_t)n * k + j] = g;
+          if (dX)
+            for (int c = 0; c < d; ++c) dX[(size_t)n * d + c] += da[c];
+        }
+        if (dX)
+          for (int s = 0; s < S; ++s) {
+            row_backward(0, a, dy, 1.0, (const char*)Sg + s * sg_stride * es,
+                         (const char*)Su + s * sg_stride * es, (const char*)Sd + s * sd_stride * es,
+                         wdt, d, fs, h, dg, du, da);
+            for (int c = 0; c < d; ++c) dX[(size_t)n * d + c] += da[c];
+          }
+      }
+      free(a); free(da); free(h); free(dg); free(du);
+    }
+  }
+
+  /* 2. weight gradients: for each listed expert (then each shared expert),
+   *    gather its rows (t ascending, then slot j), compute each row's h, dg,
+   *    du, then sum the outer products entry by entry in row order. */
+  int n_w = (dWg || dWu || dWd) && kind == 0 ? n_exp : 0;
+  int n_s = (dSg || dSu || dSd) ? S : 0;
+  for (int q = 0; q < n_w + n_s; ++q) {
+    int shared = q >= n_w;
+    int e = shared ? q - n_w : experts[q];
+    int ff = shared ? fs : f;
+    if (!shared && (e < 0 || e >= E)) { bad = 1; continue; }
+    const char* g_w = shared ? (const char*)Sg + e * sg_stride * es : (const char*)Wg + e * wg_stride * es;
+    const char* u_w = shared ? (const char*)Su + e * sg_stride * es : (const char*)Wu + e * wg_stride * es;
+    const char* d_w = shared ? (const char*)Sd + e * sd_stride * es : (const char*)Wd + e * wd_stride * es;
+    double* og = shared ? (dSg ? dSg + (size_t)e * sg_stride : NULL) : (dWg ? dWg + (size_t)q * wg_stride : NULL);
+    double* ou = shared ? (dSu ? dSu + (size_t)e * sg_stride : NULL) : (dWu ? dWu + (size_t)q * wg_stride : NULL);
+    double* od = shared ? (dSd ? dSd + (size_t)e * sd_stride : NULL) : (dWd ? dWd + (size_t)q * wd_stride : NULL);
+    /* the rows of this expert */
+    int n_rows = 0;
+    int32_t* row_t = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T * (shared ? 1 : k) : 1));
+    double* row_w = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T * (shared ? 1 : k) : 1));
+    for (int t = 0; t < T; ++t) {
+      if (shared) { row_t[n_rows] = t; row_w[n_rows++] = 1.0; continue; }
+      for (int j = 0; j < k; ++j)
+        if (idx[(size_t)t * k + j] == e) { row_t[n_rows] = t; row_w[n_rows++] = w[(size_t)t * k + j]; }
+    }
+    size_t nr = (size_t)(n_rows > 0 ? n_rows : 1);
+    double* A = (double*)malloc(sizeof(double) * nr * d);
+    double* H = (double*)malloc(sizeof(double) * nr * ff);
+    double* DG = (double*)malloc(sizeof(double) * nr * ff);
+    double* DU = (double*)malloc(sizeof(double) * nr * ff);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n_rows; ++r) {
+      double* a = A + (size_t)r * d;
+      for (int c = 0; c < d; ++c) a[c] = widen(X, (size_t)row_t[r] * d + c, xdt);
+      row_backward(0, a, dY + (size_t)row_t[r] * d, row_w[r], g_w, u_w, d_w, wdt, d, ff,
+                   H + (size_t)r * ff, DG + (size_t)r * ff, DU + (size_t)r * ff, NULL);
+    }
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < ff; ++i)
+      for (int c = 0; c < d; ++c) {
+        double sg = 0.0, su = 0.0, sd = 0.0;
+        for (int r = 0; r < n_rows; ++r) {
+          double ac = A[(size_t)r * d + c];
+          sg += DG[(size_t)r * ff + i] * ac;
+          su += DU[(size_t)r * ff + i] * ac;
+          sd += row_w[r] * dY[(size_t)row_t[r] * d + c] * H[(size_t)r * ff + i];
+        }
+        if (og) og[(size_t)i * d + c] = sg;
+        if (ou) ou[(size_t)i * d + c] = su;
+        if (od) od[(size_t)c * ff + i] = sd;
+      }
+    free(row_t); free(row_w); free(A); free(H); free(DG); free(DU);
+  }
+  return bad ? -3 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Routing backward (reading R11): the gradient of the logits from the
+ * gradient of the k gate weights, the selection held fixed.  With q the
+ * normalised probabilities of R4 -- over all E logits (renorm = 0) or over
+ * the k selected ones (renorm = 1, q_e = 0 for the others) -- each gate is
+ * w_j = q_{idx_j}, and
+ *     dw_j / dl_e = w_j (delta(e, idx_j) - q_e)   for e in the softmax set,
+ *                   0                              otherwise,
+ *     dL/dl_e     = sum_j dL/dw_j * dw_j / dl_e.
+ * The gates are recomputed from the logits (double).  Empty slots (-1)
+ * carry no gradient.  dlogits [T, E] double.
+ * ---------------------------------------------------------------------- */
+int oracle_route_backward(const float* logits, int T, int E, int k, int renorm,
+                          const int32_t* idx, const double* dw, double* dlogits) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+  double* q = (double*)malloc(sizeof(double) * (size_t)E);
+  for (int t = 0; t < T; ++t) {
+    const float* l = logits + (size_t)t * E;
+    const int32_t* id = idx + (size_t)t * k;
+    double m = (double)l[0];
+    for (int e = 1; e < E; ++e)
+      if ((double)l[e] > m) m = (double)l[e];
+    for (int e = 0; e < E; ++e) {
+      int in_set = !renorm;
+      for (int j = 0; j < k; ++j)
+        if (id[j] == e) in_set = 1;
+      q[e] = in_set ? exp((double)l[e] - m) : 0.0;
+    }
+    double z = 0.0;
+    for (int e = 0; e < E; ++e) z += q[e];
+    for (int e = 0; e < E; ++e) q[e] /= z;
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int j = 0; j < k; ++j) {
+        if (id[j] < 0) continue;
+        double wj = q[id[j]];
+        double jac = wj * ((id[j] == e ? 1.0 : 0.0) - q[e]); /* q_e = 0 off the set */
+        acc += dw[(size_t)t * k + j] * jac;
+      }
+      dlogits[(size_t)t * E + e] = acc;
+    }
+  }
+  free(q);
   return 0;
 }
