@@ -42,7 +42,7 @@ METRIC = "MoE-layer tokens/s (route+BRIM dispatch+grouped GEMM+combine)"
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
 # GEMM launches of one layer step, from one ncu capture (profiles/ffn_gemm_pair_olmoe.md),
 # valid only while the GEMM sources hash to `src`; otherwise reported as null.
-GEMM_TRAFFIC = {"olmoe": {"bytes": 1178.5e6, "src": "b458d748954b8030"}}
+GEMM_TRAFFIC = {"olmoe": {"bytes": 1179.2e6, "src": "99a471e2b083403a"}}
 
 
 def gemm_src_hash() -> str:
