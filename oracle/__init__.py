@@ -275,7 +275,8 @@ def dense_layer_backward(x, idx, w, wg, wu, wd, dy, kind=KIND_SWIGLU, shared=Non
                          tokens=None, experts=None, shared_grads=False):
     """Backward of :func:`dense_layer` for the upstream gradient ``dy`` [T,d].
 
-    Returns a dict with ``dx`` [n,d] and ``dw`` [n,k] (n = len(tokens) or T),
+    Returns a dict with ``dx`` [n,d], ``dw`` [n,k] (n = len(tokens) or T) and
+    ``dw_abs`` [n,k] (the sum of |terms| of each dw: its condition magnitude),
     and, when ``experts`` lists expert ids, ``dwg``/``dwu`` [n_exp,f,d] and
     ``dwd`` [n_exp,d,f]; with ``shared_grads`` the shared experts' ``dsg``,
     ``dsu``, ``dsd``.  Everything in double.
@@ -306,7 +307,7 @@ def dense_layer_backward(x, idx, w, wg, wu, wd, dy, kind=KIND_SWIGLU, shared=Non
         n = len(tokens)
     else:
         n = T
-    out = dict(dx=np.empty((n, d)), dw=np.empty((n, k)))
+    out = dict(dx=np.empty((n, d)), dw=np.empty((n, k)), dw_abs=np.empty((n, k)))
     if experts is not None:
         experts = np.ascontiguousarray(experts, dtype=np.int32)
         ne = len(experts)
@@ -318,7 +319,7 @@ def dense_layer_backward(x, idx, w, wg, wu, wd, dy, kind=KIND_SWIGLU, shared=Non
     rc = lib().oracle_dense_layer_backward(
         _p(x), _dt(x), T, d, _p(idx), _p(w), k, _p(wg), _p(wu), _p(wd), wdt, E, f, int(kind),
         _p(sg), _p(su), _p(sd), S, fs, _p(dy), _p(tokens), n, _p(out["dx"]), _p(out["dw"]),
-        _p(experts), ne, _p(out.get("dwg")), _p(out.get("dwu")), _p(out.get("dwd")),
+        _p(out["dw_abs"]), _p(experts), ne, _p(out.get("dwg")), _p(out.get("dwu")), _p(out.get("dwd")),
         _p(out.get("dsg")), _p(out.get("dsu")), _p(out.get("dsd")))
     if rc != 0:
         raise ValueError(f"oracle_dense_layer_backward failed ({rc})")

@@ -631,16 +631,24 @@ int oracle_place_greedy(const uint32_t* H, int E, int R, int32_t* slot_of) {
  * The identity expert (kind 1) has o = a: dL/dw = <dy, a>, dL/da = w dy.
  *
  * row_backward() fills h, dg, du (each [f]) and returns dL/dw; da (if not
- * NULL) receives dL/da.  Weights are one expert's Wg,Wu [f,d], Wd [d,f].
+ * NULL) receives dL/da, and dw_abs (if not NULL) the sum of the absolute
+ * values of the terms of dL/dw (sum_i |(Wd^T dy)_i h_i|), the magnitude its
+ * rounding error scales with.  Weights are one expert's Wg,Wu [f,d], Wd [d,f].
  * ---------------------------------------------------------------------- */
 static double row_backward(int kind, const double* a, const double* dy, double w,
                            const void* Wg, const void* Wu, const void* Wd, int wdt,
-                           int d, int f, double* h, double* dg, double* du, double* da) {
+                           int d, int f, double* h, double* dg, double* du, double* da,
+                           double* dw_abs) {
+  double abs_sum = 0.0; /* sum of |terms| of dL/dw: its condition magnitude */
   if (kind == 1) {
     double dw = 0.0;
-    for (int c = 0; c < d; ++c) dw += dy[c] * a[c];
+    for (int c = 0; c < d; ++c) {
+      dw += dy[c] * a[c];
+      abs_sum += fabs(dy[c] * a[c]);
+    }
     if (da)
       for (int c = 0; c < d; ++c) da[c] = w * dy[c];
+    if (dw_abs) *dw_abs = abs_sum;
     return dw;
   }
   double dw = 0.0;
@@ -656,6 +664,7 @@ static double row_backward(int kind, const double* a, const double* dy, double w
     double wd_dy = 0.0; /* (Wd^T dy)_i */
     for (int c = 0; c < d; ++c) wd_dy += widen(Wd, (size_t)c * f + i, wdt) * dy[c];
     dw += wd_dy * h[i]; /* <dy, Wd h> summed by i */
+    abs_sum += fabs(wd_dy * h[i]);
     double dh = w * wd_dy;
     dg[i] = dh * u * s * (1.0 + g * (1.0 - s));
     du[i] = dh * silu;
@@ -667,6 +676,7 @@ static double row_backward(int kind, const double* a, const double* dy, double w
         acc += widen(Wg, (size_t)i * d + c, wdt) * dg[i] + widen(Wu, (size_t)i * d + c, wdt) * du[i];
       da[c] = acc;
     }
+  if (dw_abs) *dw_abs = abs_sum;
   return dw;
 }
 
@@ -675,8 +685,9 @@ static double row_backward(int kind, const double* a, const double* dy, double w
  * oracle_dense_layer() for an upstream gradient dY [T, d] (double):
  *   dX[t]    = sum_j dL/da of row (t, j) + sum_s dL/da of shared row (t, s)
  *   dW[t][j] = dL/dw of row (t, j)                     (0 for an empty slot)
- * for the tokens in `tokens` (NULL = all T; outputs [n_tok, d], [n_tok, k];
- * either output may be NULL).
+ *   dW_abs[t][j] = the sum of |terms| of dW[t][j]        (its condition magnitude)
+ * for the tokens in `tokens` (NULL = all T; outputs [n_tok, d], [n_tok, k],
+ * [n_tok, k]; any of them may be NULL).
  * Weight gradients, each optional (NULL = not computed), over ALL T tokens:
  *   dWg, dWu [n_exp, f, d], dWd [n_exp, d, f] for the experts listed in
  *   `experts` (n_exp of them), and dSg, dSu [S, fs, d], dSd [S, d, fs].
@@ -687,7 +698,7 @@ int oracle_dense_layer_backward(const void* X, int xdt, int T, int d,
                                 int E, int f, int kind,
                                 const void* Sg, const void* Su, const void* Sd, int S, int fs,
                                 const double* dY, const int32_t* tokens, int n_tok,
-                                double* dX, double* dW,
+                                double* dX, double* dW, double* dW_abs,
                                 const int32_t* experts, int n_exp,
                                 double* dWg, double* dWu, double* dWd,
                                 double* dSg, double* dSu, double* dSd) {
@@ -700,7 +711,7 @@ int oracle_dense_layer_backward(const void* X, int xdt, int T, int d,
   int bad = 0;
 
   /* 1. per-token input gradient and gate-weight gradient */
-  if (dX || dW) {
+  if (dX || dW || dW_abs) {
 #pragma omp parallel
     {
       double* a = (double*)malloc(sizeof(double) * (size_t)d);
@@ -719,14 +730,17 @@ int oracle_dense_layer_backward(const void* X, int xdt, int T, int d,
         for (int j = 0; j < k; ++j) {
           int e = idx[(size_t)t * k + j];
           if (dW) dW[(size_t)n * k + j] = 0.0;
+          if (dW_abs) dW_abs[(size_t)n * k + j] = 0.0;
           if (e == -1) continue;
           if (e < 0 || e >= E) { bad = 1; continue; }
+          double g_abs = 0.0;
           double g = row_backward(kind, a, dy, w[(size_t)t * k + j],
                                   (const char*)Wg + e * wg_stride * es,
                                   (const char*)Wu + e * wg_stride * es,
                                   (const char*)Wd + e * wd_stride * es, wdt, d, f, h, dg, du,
-                                  dX ? da : NULL);
+                                  dX ? da : NULL, &g_abs);
           if (dW) dW[(size_t)n * k + j] = g;
+          if (dW_abs) dW_abs[(size_t)n * k + j] = g_abs;
           if (dX)
             for (int c = 0; c < d; ++c) dX[(size_t)n * d + c] += da[c];
         }
@@ -734,7 +748,7 @@ int oracle_dense_layer_backward(const void* X, int xdt, int T, int d,
           for (int s = 0; s < S; ++s) {
             row_backward(0, a, dy, 1.0, (const char*)Sg + s * sg_stride * es,
                          (const char*)Su + s * sg_stride * es, (const char*)Sd + s * sd_stride * es,
-                         wdt, d, fs, h, dg, du, da);
+                         wdt, d, fs, h, dg, du, da, NULL);
             for (int c = 0; c < d; ++c) dX[(size_t)n * d + c] += da[c];
           }
       }
@@ -777,7 +791,7 @@ int oracle_dense_layer_backward(const void* X, int xdt, int T, int d,
       double* a = A + (size_t)r * d;
       for (int c = 0; c < d; ++c) a[c] = widen(X, (size_t)row_t[r] * d + c, xdt);
       row_backward(0, a, dY + (size_t)row_t[r] * d, row_w[r], g_w, u_w, d_w, wdt, d, ff,
-                   H + (size_t)r * ff, DG + (size_t)r * ff, DU + (size_t)r * ff, NULL);
+                   H + (size_t)r * ff, DG + (size_t)r * ff, DU + (size_t)r * ff, NULL, NULL);
     }
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < ff; ++i)

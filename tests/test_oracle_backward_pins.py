@@ -61,6 +61,8 @@ def test_layer_backward_equals_finite_differences(seed):
     fun = lambda: _loss(x, idx, w, wg, wu, wd, shared, dy)  # noqa: E731
     _close(got["dx"], _fd(fun, x))
     _close(got["dw"], _fd(fun, w))
+    assert (got["dw_abs"] >= np.abs(got["dw"]) * (1 - 1e-12)).all()
+    assert (got["dw_abs"] > np.abs(got["dw"]) * 1.01).any()  # some terms cancel
     _close(got["dwg"], _fd(fun, wg))
     _close(got["dwu"], _fd(fun, wu))
     _close(got["dwd"], _fd(fun, wd))
@@ -101,6 +103,9 @@ def test_identity_expert_closed_form():
     np.testing.assert_allclose(got["dx"], w.sum(1, keepdims=True) * dy, rtol=1e-14)
     np.testing.assert_allclose(got["dw"], np.repeat((dy * x).sum(1, keepdims=True), 2, 1),
                                rtol=1e-13)
+    # the condition magnitude of dw_j: sum over c of |dY_c X_c|
+    np.testing.assert_allclose(got["dw_abs"],
+                               np.repeat(np.abs(dy * x).sum(1, keepdims=True), 2, 1), rtol=1e-13)
 
 
 def _route_problem(seed, T=6, E=7):
