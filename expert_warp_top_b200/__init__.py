@@ -1,6 +1,8 @@
 """expert_warp_top_b200: the hot path of an Occult-style mixture-of-experts
 layer (top-k routing, BRIM-guided dispatch, grouped SwiGLU experts on tcgen05,
-per-rank pre-reduce and combine) as hand-written CUDA for B200 (sm_100a).
+per-rank pre-reduce and combine) as hand-written CUDA for B200 (sm_100a),
+with its training backward (input- and weight-gradient GEMMs on tcgen05,
+routing backward) through the same BRIMs.
 
 The CUDA library is loaded on first use; without it every call raises.
 """
@@ -13,5 +15,8 @@ from ._binding import (  # noqa: F401
     moe_prepare_shared_weights, moe_prepare_weights, moe_route_topk, moe_set_debug,
     moe_layer_workspace_size, moe_layer_forward, moe_layer_forward_host, moe_place_greedy,
     moe_route_brim, moe_route_brim_workspace_size, moe_prune_topk,
+    moe_expert_ffn_train, moe_expert_ffn_backward, moe_expert_ffn_backward_workspace_size,
+    moe_route_backward, moe_layer_train_workspace_size, moe_layer_forward_train,
+    moe_layer_backward,
 )
-from .layer import MoELayer  # noqa: F401
+from .layer import MoELayer, unpack_gate_up  # noqa: F401

@@ -35,6 +35,9 @@ EXPORTS = (
     "moe_expert_ffn", "moe_combine_scatter", "moe_count_dispatched_rows", "moe_coact_histogram",
     "moe_layer_workspace_size", "moe_layer_forward", "moe_layer_forward_host",
     "moe_place_greedy", "moe_route_brim_workspace_size", "moe_route_brim", "moe_prune_topk",
+    "moe_expert_ffn_train", "moe_expert_ffn_backward_workspace_size", "moe_expert_ffn_backward",
+    "moe_route_backward", "moe_layer_train_workspace_size", "moe_layer_forward_train",
+    "moe_layer_backward",
 )
 
 
@@ -62,6 +65,8 @@ def load():
         lib.moe_expert_ffn_workspace_size.restype = ctypes.c_size_t
         lib.moe_layer_workspace_size.restype = ctypes.c_size_t
         lib.moe_route_brim_workspace_size.restype = ctypes.c_size_t
+        lib.moe_expert_ffn_backward_workspace_size.restype = ctypes.c_size_t
+        lib.moe_layer_train_workspace_size.restype = ctypes.c_size_t
         lib.moe_set_debug.argtypes = [ctypes.c_int, ctypes.c_double]
         for name in EXPORTS:
             getattr(lib, name)
@@ -289,6 +294,94 @@ def moe_layer_forward_host(h_logits, h_x, k, R, renorm, slot_of, w_gu, w_dn, f, 
         _ptr(w_dn, h_x.dtype, "w_dn"), _ptr(sw_gu, h_x.dtype, "sw_gu"),
         _ptr(sw_dn, h_x.dtype, "sw_dn"), _host_ptr(h_y, h_x.dtype, "h_y"),
         _ptr(ws, None, "ws"), ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# training
+BF16 = torch.bfloat16
+
+
+def _nbytes(t) -> ctypes.c_size_t:
+    return ctypes.c_size_t(0 if t is None else t.numel() * t.element_size())
+
+
+def moe_expert_ffn_train(a, group_off, w_gu, w_dn, f, row_scale, z, h, out, m_cap=None,
+                         stream=None):
+    """out = row_scale * FFN_g(a rows); also keeps z (pre-activations) and h."""
+    a_rows, d = a.shape
+    m_cap = a_rows if m_cap is None else m_cap
+    _check("moe_expert_ffn_train", load().moe_expert_ffn_train(
+        _ptr(a, BF16, "a"), int(a_rows), _ptr(group_off, I32, "group_off"),
+        group_off.numel() - 1, int(m_cap), _ptr(w_gu, BF16, "w_gu"), _ptr(w_dn, BF16, "w_dn"),
+        int(d), int(f), _ptr(row_scale, F32, "row_scale"), _ptr(z, BF16, "z"), _ptr(h, BF16, "h"),
+        _ptr(out, BF16, "out"), _stream(stream)))
+
+
+def moe_expert_ffn_backward_workspace_size(m_cap: int, f: int) -> int:
+    return int(load().moe_expert_ffn_backward_workspace_size(int(m_cap), int(f)))
+
+
+def moe_expert_ffn_backward(dout, a, z, group_off, w_gu, w_dn, f, row_scale, dx, d_row_scale,
+                            dw_gu, dw_dn, ws, accumulate=0, m_cap=None, stream=None):
+    """Gradients of moe_expert_ffn_train: dx, d_row_scale, dw_gu, dw_dn (any may be None
+    except dx); the weight gradients' dtype (float32 or bfloat16) is taken from them."""
+    a_rows, d = a.shape
+    m_cap = a_rows if m_cap is None else m_cap
+    dw = dw_gu if dw_gu is not None else dw_dn
+    dw_dtype = dtype_code(dw.dtype) if dw is not None else MOE_F32
+    _check("moe_expert_ffn_backward", load().moe_expert_ffn_backward(
+        _ptr(dout, BF16, "dout"), _ptr(a, BF16, "a"), int(a_rows), _ptr(z, BF16, "z"),
+        _ptr(group_off, I32, "group_off"), group_off.numel() - 1, int(m_cap),
+        _ptr(w_gu, BF16, "w_gu"), _ptr(w_dn, BF16, "w_dn"), int(d), int(f),
+        _ptr(row_scale, F32, "row_scale"), _ptr(dx, BF16, "dx"),
+        _ptr(d_row_scale, F32, "d_row_scale"), _ptr(dw_gu, _ACT, "dw_gu"),
+        _ptr(dw_dn, _ACT, "dw_dn"), int(dw_dtype), int(accumulate), _ptr(ws, None, "ws"),
+        _nbytes(ws), _stream(stream)))
+
+
+def moe_route_backward(logits, k, renorm, topk_idx, slot_of, R, brim0, brim1, d_gate_epd,
+                       d_logits, d_topk_w=None, stream=None):
+    T, E = logits.shape
+    _check("moe_route_backward", load().moe_route_backward(
+        _ptr(logits, F32, "logits"), int(T), int(E), int(k), int(renorm),
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(slot_of, I32, "slot_of"), int(R),
+        _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"), _ptr(d_gate_epd, F32, "d_gate_epd"),
+        _ptr(d_logits, F32, "d_logits"), _ptr(d_topk_w, F32, "d_topk_w"), _stream(stream)))
+
+
+def moe_layer_train_workspace_size(T, d, f, E, k, R, S=0, fs=0) -> int:
+    return int(load().moe_layer_train_workspace_size(int(T), int(d), int(f), int(E), int(k),
+                                                     int(R), int(S), int(fs)))
+
+
+def moe_layer_forward_train(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, y, ws, sw_gu=None,
+                            sw_dn=None, S=0, fs=0, stream=None):
+    T, E = logits.shape
+    d = x.shape[1]
+    _check("moe_layer_forward_train", load().moe_layer_forward_train(
+        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(S), int(fs),
+        _ptr(logits, F32, "logits"), _ptr(x, BF16, "x"), _ptr(slot_of, I32, "slot_of"),
+        _ptr(w_gu, BF16, "w_gu"), _ptr(w_dn, BF16, "w_dn"), _ptr(sw_gu, BF16, "sw_gu"),
+        _ptr(sw_dn, BF16, "sw_dn"), _ptr(y, BF16, "y"), _ptr(ws, None, "ws"), _nbytes(ws),
+        _stream(stream)))
+
+
+def moe_layer_backward(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, dy, dx, d_logits,
+                       dw_gu, dw_dn, ws, sw_gu=None, sw_dn=None, S=0, fs=0, dsw_gu=None,
+                       dsw_dn=None, accumulate=0, d_topk_w=None, stream=None):
+    T, E = logits.shape
+    d = x.shape[1]
+    dw_dtype = dtype_code(dw_gu.dtype if dw_gu is not None else
+                          (dw_dn.dtype if dw_dn is not None else torch.float32))
+    _check("moe_layer_backward", load().moe_layer_backward(
+        int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(S), int(fs),
+        _ptr(logits, F32, "logits"), _ptr(x, BF16, "x"), _ptr(slot_of, I32, "slot_of"),
+        _ptr(w_gu, BF16, "w_gu"), _ptr(w_dn, BF16, "w_dn"), _ptr(sw_gu, BF16, "sw_gu"),
+        _ptr(sw_dn, BF16, "sw_dn"), _ptr(dy, BF16, "dy"), _ptr(dx, BF16, "dx"),
+        _ptr(d_logits, F32, "d_logits"), _ptr(d_topk_w, F32, "d_topk_w"),
+        _ptr(dw_gu, _ACT, "dw_gu"), _ptr(dw_dn, _ACT, "dw_dn"),
+        _ptr(dsw_gu, _ACT, "dsw_gu"), _ptr(dsw_dn, _ACT, "dsw_dn"), int(dw_dtype),
+        int(accumulate), _ptr(ws, None, "ws"), _nbytes(ws), _stream(stream)))
 
 
 def moe_place_greedy(hist, R) -> torch.Tensor:

@@ -2,9 +2,11 @@
 
     python -m expert_warp_top_b200.build [--force] [--ptxas-verbose]
 
-One translation unit (csrc/api.cu includes every kernel header), compiled by
-nvcc with the CUDA runtime linked statically, so the shared object depends on
-no CUDA library at load time (the driver is reached through the runtime).
+Two translation units -- csrc/api.cu (inference entry points) and
+csrc/api_train.cu (training entry points), each including the kernel headers it
+launches -- compiled by nvcc in parallel and linked with the CUDA runtime
+linked statically, so the shared object depends on no CUDA library at load
+time (the driver is reached through the runtime).
 """
 from __future__ import annotations
 
@@ -43,19 +45,44 @@ def needs_build() -> bool:
 def build(force: bool = False, verbose_ptxas: bool = False) -> Path:
     if not force and not needs_build():
         return LIB
-    tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-cudart", "static", "-I", str(ROOT / "include"),
-           str(CSRC / "api.cu"), "-o", str(tmp)]
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = ROOT / "_build"
+    objdir.mkdir(exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+             "-I", str(ROOT / "include")]
     if verbose_ptxas:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError(f"nvcc failed building {LIB.name}")
-    if verbose_ptxas:
-        sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+        flags.insert(0, "-Xptxas=-v")
+    units = sorted(CSRC.glob("*.cu"))
+    tag = os.getpid()
+
+    def compile_unit(src: Path):
+        obj = objdir / f"{src.stem}.{tag}.o"
+        res = subprocess.run([nvcc(), *flags, "-c", str(src), "-o", str(obj)],
+                             capture_output=True, text=True)
+        return src, obj, res
+
+    with ThreadPoolExecutor(max_workers=len(units)) as ex:
+        results = list(ex.map(compile_unit, units))
+    failed = False
+    for src, obj, res in results:
+        if res.returncode != 0 or verbose_ptxas:
+            sys.stderr.write(res.stdout + res.stderr)
+        failed |= res.returncode != 0
+    objs = [obj for _, obj, _ in results]
+    try:
+        if failed:
+            raise RuntimeError(f"nvcc failed building {LIB.name}")
+        tmp = LIB.with_suffix(f".so.tmp{tag}")
+        res = subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", *map(str, objs),
+                              "-o", str(tmp)], capture_output=True, text=True)
+        if res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+            raise RuntimeError(f"nvcc failed linking {LIB.name}")
+        os.replace(tmp, LIB)
+    finally:
+        for obj in objs:
+            if obj.exists():
+                obj.unlink()
     return LIB
 
 

@@ -14,8 +14,7 @@
 #include "../../include/moe_occult.h"
 #include "brim.cuh"
 #include "dispatch.cuh"
-#include "ffn_gemm.cuh"
-#include "ffn_gemm_pair.cuh"
+#include "host.h"
 #include "route.cuh"
 #include "route_brim.cuh"
 
@@ -27,9 +26,13 @@ __device__ unsigned g_moe_err_flag;
 constexpr size_t kNoAllocScratchInts = size_t(1) << 18;
 static __device__ __align__(256) int32_t g_brim_noalloc_scratch[kNoAllocScratchInts];
 
-namespace {
+namespace moe_host {
 
+namespace {
 thread_local char g_msg[512];
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+}  // namespace
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -39,38 +42,7 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
-#define MOE_REQUIRE(cond, code, ...)          \
-  do {                                        \
-    if (!(cond)) return fail(code, __VA_ARGS__); \
-  } while (0)
-
-#define MOE_CUDA(call)                                                              \
-  do {                                                                              \
-    cudaError_t e_ = (call);                                                        \
-    if (e_ != cudaSuccess)                                                          \
-      return fail(MOE_ERR_CUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_),   \
-                  __FILE__, __LINE__);                                              \
-  } while (0)
-
-#define MOE_LAUNCHED(what)                                                          \
-  do {                                                                              \
-    cudaError_t e_ = cudaGetLastError();                                            \
-    if (e_ != cudaSuccess)                                                          \
-      return fail(MOE_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e_)); \
-  } while (0)
-
-constexpr int kMaxDevices = 64;
-
-struct DeviceInfo {
-  bool ready = false;
-  int num_sms = 0;
-  unsigned* err_flag = nullptr;
-  unsigned smem_attr_done = 0;  // bit per GEMM instantiation
-  unsigned pair_attr_done = 0;  // bit per CTA-pair GEMM instantiation
-  int pair_max_clusters[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-};
-DeviceInfo g_dev[kMaxDevices];
-std::mutex g_dev_mu;
+const char* last_message() { return g_msg; }
 
 int device_info(DeviceInfo** out) {
   int dev = 0;
@@ -95,6 +67,82 @@ int device_info(DeviceInfo** out) {
   return MOE_OK;
 }
 
+int ensure_smem(DeviceInfo* di, const void* kern, size_t bytes) {
+  std::lock_guard<std::mutex> lk(di->mu);
+  for (const void* k : di->smem_raised)
+    if (k == kern) return MOE_OK;
+  MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  di->smem_raised.push_back(kern);
+  return MOE_OK;
+}
+
+int g_debug_flags = 0;
+double g_wait_limit_ms = 4000.0;
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encode_fn(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cached) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    MOE_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q));
+    MOE_REQUIRE(q == cudaDriverEntryPointSuccess && p, MOE_ERR_CUDA,
+                "cuTensorMapEncodeTiled is not available from the driver");
+    cached = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = cached;
+  return MOE_OK;
+}
+}  // namespace
+
+int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn;
+  int rc = get_encode_fn(&fn);
+  if (rc) return rc;
+  const int esz = dtype == MOE_BF16 ? 2 : 4;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (cuuint64_t)esz};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype == MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA,
+              "cuTensorMapEncodeTiled failed (%d) for a [%llu x %llu] tensor", (int)r,
+              (unsigned long long)rows, (unsigned long long)cols);
+  return MOE_OK;
+}
+
+int check_common(int T, int E, int k, int R) {
+  MOE_REQUIRE(T >= 0, MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+  MOE_REQUIRE(E >= 1 && E <= moe::kMaxE, MOE_ERR_UNSUPPORTED, "E must be in [1, 256] (got %d)", E);
+  MOE_REQUIRE(k >= 1 && k <= E && k <= moe::kMaxK, MOE_ERR_UNSUPPORTED,
+              "k must be in [1, min(E, 16)] (got k=%d, E=%d)", k, E);
+  MOE_REQUIRE(R >= 1 && R <= E && E % R == 0, MOE_ERR_UNSUPPORTED,
+              "R must divide E (got E=%d, R=%d)", E, R);
+  return MOE_OK;
+}
+
+int check_dtype(int dtype) {
+  MOE_REQUIRE(dtype == MOE_BF16 || dtype == MOE_F32, MOE_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  return MOE_OK;
+}
+
+}  // namespace moe_host
+
+using namespace moe_host;
+
+namespace {
+
 // Device address of g_brim_noalloc_scratch on the current device.  The
 // array's name in host code is only a host-side stand-in, so the address is
 // looked up with cudaGetSymbolAddress, once per device, with that device
@@ -117,225 +165,6 @@ int noalloc_scratch(int32_t** out) {
   return MOE_OK;
 }
 
-// Every kernel is launched with programmatic stream serialization, so the next
-// kernel on the stream can be scheduled while this one finishes; each kernel
-// starts with griddepcontrol.wait (moe::pdl_enter) before it touches memory.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                     Args&&... args) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
-
-// ---- debug knobs (tests only) -------------------------------------------
-int g_debug_flags = 0;
-double g_wait_limit_ms = 4000.0;
-
-uint64_t wait_limit_ns() {
-  return static_cast<uint64_t>(g_wait_limit_ms * 1.0e6);
-}
-
-// ---- tensor maps ---------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-int get_encode_fn(EncodeTiledFn* fn) {
-  static EncodeTiledFn cached = nullptr;
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!cached) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    MOE_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q));
-    MOE_REQUIRE(q == cudaDriverEntryPointSuccess && p, MOE_ERR_CUDA,
-                "cuTensorMapEncodeTiled is not available from the driver");
-    cached = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  *fn = cached;
-  return MOE_OK;
-}
-
-// 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
-int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
-              uint32_t box_cols, uint32_t box_rows) {
-  EncodeTiledFn fn;
-  int rc = get_encode_fn(&fn);
-  if (rc) return rc;
-  const int esz = dtype == MOE_BF16 ? 2 : 4;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * (cuuint64_t)esz};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, dtype == MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                  2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA,
-              "cuTensorMapEncodeTiled failed (%d) for a [%llu x %llu] tensor", (int)r,
-              (unsigned long long)rows, (unsigned long long)cols);
-  return MOE_OK;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int check_common(int T, int E, int k, int R) {
-  MOE_REQUIRE(T >= 0, MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
-  MOE_REQUIRE(E >= 1 && E <= moe::kMaxE, MOE_ERR_UNSUPPORTED, "E must be in [1, 256] (got %d)", E);
-  MOE_REQUIRE(k >= 1 && k <= E && k <= moe::kMaxK, MOE_ERR_UNSUPPORTED,
-              "k must be in [1, min(E, 16)] (got k=%d, E=%d)", k, E);
-  MOE_REQUIRE(R >= 1 && R <= E && E % R == 0, MOE_ERR_UNSUPPORTED,
-              "R must divide E (got E=%d, R=%d)", E, R);
-  return MOE_OK;
-}
-
-int check_dtype(int dtype) {
-  MOE_REQUIRE(dtype == MOE_BF16 || dtype == MOE_F32, MOE_ERR_INVALID_ARG, "unknown dtype %d", dtype);
-  return MOE_OK;
-}
-
-int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
-
-int pick_bn(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
-
-// host-side debug bits (test only): force the single-CTA or the CTA-pair GEMM
-constexpr int kDebugForceSingle = 2;
-constexpr int kDebugForcePair = 4;
-
-// ---- GEMM launch ----------------------------------------------------------
-// A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
-// gathered from it (row p = a[a_row_index[p]]), else they are a's first m_cap.
-template <int BN, int EPI, bool TF32, bool GATHER>
-int launch_gemm(DeviceInfo* di, unsigned attr_bit, const void* a, int a_rows,
-                const int32_t* a_row_index, int m_cap, int K, const void* b, int G, int N,
-                const int32_t* group_off, const float* row_scale, void* out, int ldo,
-                cudaStream_t st) {
-  using Cfg = moe::GemmCfg<BN, TF32>;
-  const int dtype = TF32 ? MOE_F32 : MOE_BF16;
-  CUtensorMap ta, tb;
-  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK,
-                     GATHER ? 1u : (uint32_t)moe::kGemmBM);
-  if (rc) return rc;
-  rc = encode_2d(&tb, b, dtype, (uint64_t)K, (uint64_t)G * N, Cfg::kBK, BN);
-  if (rc) return rc;
-  auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32, GATHER>;
-  if (!(di->smem_attr_done & attr_bit)) {
-    MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)Cfg::kSmemBytes));
-    di->smem_attr_done |= attr_bit;
-  }
-  const long long ub = ((long long)m_cap / moe::kGemmBM + G) * (N / BN);
-  const int grid = (int)(ub < di->num_sms ? (ub < 1 ? 1 : ub) : di->num_sms);
-  moe::GemmArgs args{group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo,
-                     di->err_flag, wait_limit_ns(), g_debug_flags};
-  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, args));
-  MOE_LAUNCHED("ffn_gemm_kernel");
-  return MOE_OK;
-}
-
-template <int EPI, bool TF32, bool GATHER>
-int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int a_rows, const int32_t* a_row_index,
-                   int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
-                   const float* row_scale, void* out, int ldo, cudaStream_t st) {
-  const unsigned base = ((EPI * 2 + (TF32 ? 1 : 0)) * 2 + (GATHER ? 1 : 0)) * 3;
-  if (bn == 256)
-    return launch_gemm<256, EPI, TF32, GATHER>(di, 1u << (base + 0), a, a_rows, a_row_index,
-                                               m_cap, K, b, G, N, group_off, row_scale, out, ldo,
-                                               st);
-  if (bn == 128)
-    return launch_gemm<128, EPI, TF32, GATHER>(di, 1u << (base + 1), a, a_rows, a_row_index,
-                                               m_cap, K, b, G, N, group_off, row_scale, out, ldo,
-                                               st);
-  return launch_gemm<64, EPI, TF32, GATHER>(di, 1u << (base + 2), a, a_rows, a_row_index, m_cap,
-                                            K, b, G, N, group_off, row_scale, out, ldo, st);
-}
-
-// The same GEMM on CTA pairs (cluster of 2, M = 256 tiles).  Needs BN/2 >= 64.
-template <int BN, int EPI, bool TF32>
-int launch_gemm_pair(DeviceInfo* di, int slot, const void* a, int a_rows, int m_cap, int K,
-                     const void* b, int G, int N, const int32_t* group_off,
-                     const float* row_scale, void* out, int ldo, cudaStream_t st) {
-  using Cfg = moe::PairCfg<BN, TF32>;
-  const int dtype = TF32 ? MOE_F32 : MOE_BF16;
-  CUtensorMap ta, tb;
-  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
-  if (rc) return rc;
-  rc = encode_2d(&tb, b, dtype, (uint64_t)K, (uint64_t)G * N, Cfg::kBK, BN / 2);
-  if (rc) return rc;
-  auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32>;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
-  if (!(di->pair_attr_done & (1u << slot))) {
-    MOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)Cfg::kSmemBytes));
-    cfg.gridDim = dim3(2 * (di->num_sms / 2), 1, 1);
-    int clusters = 0;
-    MOE_CUDA(cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg));
-    MOE_REQUIRE(clusters >= 1, MOE_ERR_UNSUPPORTED, "no CTA pair fits on this device");
-    di->pair_max_clusters[slot] = clusters;
-    di->pair_attr_done |= 1u << slot;
-  }
-  const long long ub = ((long long)m_cap / moe::kPairBM + G) * (N / BN);
-  const long long pairs = ub < di->pair_max_clusters[slot] ? (ub < 1 ? 1 : ub)
-                                                            : di->pair_max_clusters[slot];
-  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-  cfg.numAttrs = 2;
-  moe::GemmArgs args{group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo,
-                     di->err_flag, wait_limit_ns(), g_debug_flags};
-  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
-  return MOE_OK;
-}
-
-// GEMM over the groups, on CTA pairs when the groups are tall enough to fill
-// 256-row tiles (and the rows are read in place), else on single CTAs.
-template <int EPI, bool TF32>
-int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_index,
-                     int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
-                     const float* row_scale, void* out, int ldo, cudaStream_t st) {
-#ifndef MOE_PAIR_MIN_ROWS
-#define MOE_PAIR_MIN_ROWS 192
-#endif
-  const bool tall = (long long)m_cap >= (long long)MOE_PAIR_MIN_ROWS * G;
-  bool pair = !a_row_index && N % 128 == 0 && tall;
-  if (g_debug_flags & kDebugForceSingle) pair = false;
-  if ((g_debug_flags & kDebugForcePair) && !a_row_index && N % 128 == 0) pair = true;
-  if (pair) {
-    const int slot = (EPI * 2 + (TF32 ? 1 : 0)) * 2;
-    if (N % 256 == 0)
-      return launch_gemm_pair<256, EPI, TF32>(di, slot, a, a_rows, m_cap, K, b, G, N, group_off,
-                                              row_scale, out, ldo, st);
-    return launch_gemm_pair<128, EPI, TF32>(di, slot + 1, a, a_rows, m_cap, K, b, G, N,
-                                            group_off, row_scale, out, ldo, st);
-  }
-  const int bn = pick_bn(N);
-  if (a_row_index)
-    return launch_gemm_bn<EPI, TF32, true>(di, bn, a, a_rows, a_row_index, m_cap, K, b, G, N,
-                                           group_off, row_scale, out, ldo, st);
-  return launch_gemm_bn<EPI, TF32, false>(di, bn, a, a_rows, nullptr, m_cap, K, b, G, N,
-                                          group_off, row_scale, out, ldo, st);
-}
-
 // How many warps share one token row in the movers: one warp per token when
 // the batch fills the GPU (>= 32 warps per SM), more for small batches.
 int mover_parts(const DeviceInfo* di, int T, int max_parts) {
@@ -347,7 +176,6 @@ int mover_parts(const DeviceInfo* di, int T, int max_parts) {
 
 
 
-size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // The BRIM passes, compiled for a bound KMAX >= k so per-token state stays in
 // registers.
@@ -399,7 +227,7 @@ extern "C" {
 
 int moe_abi_version(void) { return 1; }
 
-const char* moe_last_error(void) { return g_msg; }
+const char* moe_last_error(void) { return last_message(); }
 
 // Test-only knobs: debug flags of the GEMM (1 = skip the first TMA load, so a
 // bounded wait expires) and the device wait limit in milliseconds.

@@ -37,6 +37,19 @@ constexpr int kGemmThreads = 192;
 constexpr int kGemmMaxGroups = 1024;
 constexpr int kEpiSwiGLU = 0;  // out[:, n0/2 + j] = silu(gate) * up   (64-row interleave)
 constexpr int kEpiScale = 1;   // out[:, n0 + j]   = row_scale * acc
+// Training forward of GEMM 1: the pre-activations (gate and up columns, in the
+// GEMM's own interleaved column order) are kept, rounded to bf16, in aux_out
+// [rows, ld_aux], and out receives silu(gate) * up of those rounded values.
+constexpr int kEpiSwiGLUSave = 2;
+// Backward of the SwiGLU and of the gate scaling, fused behind the dgrad GEMM
+// dH' = dO_rows . W_down (the un-gated gradient of h).  With z = the saved
+// pre-activations (aux_in, interleaved like kEpiSwiGLUSave), s = sigmoid(z_g),
+// h = bf16(z_g s z_u) and w = row_scale (1 if null):
+//   aux_out  dZ: dz_g = w dH' z_u s (1 + z_g (1 - s)),  dz_u = w dH' z_g s
+//   out      w h                     (the A^T operand of the down weight gradient)
+//   partial  sum over this tile's columns of dH' h  (the gate gradient, per
+//            row and N block: partial[row * n_part + n0 / BN])
+constexpr int kEpiSwiGLUBwd = 3;
 
 // Debug switch used by the timeout test: the producer skips the first stage it
 // would load, so the MMA issuer's wait can never complete.
@@ -84,16 +97,103 @@ struct GemmArgs {
   unsigned* err;
   uint64_t wait_limit_ns;
   int debug;
+  // kEpiSwiGLUSave / kEpiSwiGLUBwd only
+  const void* aux_in = nullptr;  // saved pre-activations [rows, ld_aux]
+  void* aux_out = nullptr;       // pre-activations (save) or their gradient (bwd)
+  int ld_aux = 0;
+  float* partial = nullptr;      // gate-gradient partials [rows, n_part] (nullable)
+  int n_part = 0;
 };
 
 // Epilogue of one accumulator tile for this thread's TMEM lane (= one tile
 // row): tcgen05.ld 32 columns at a time, fused SwiGLU or row scaling, and a
 // masked store of the row.  Every lane of the warp must call it (tcgen05.ld is
 // warp-collective); `valid` masks the stores.
+__device__ __forceinline__ float round_bf16(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
 template <int BN, int EPI, typename TOut>
 __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t grow, int n0,
-                                              const float* row_scale, TOut* out, int ldo) {
-  if (EPI == kEpiSwiGLU) {
+                                              const GemmArgs& args) {
+  TOut* out = reinterpret_cast<TOut*>(args.out);
+  const int ldo = args.ldo;
+  const float* row_scale = args.row_scale;
+  if constexpr (EPI == kEpiSwiGLUSave) {
+    static_assert(std::is_same<TOut, __nv_bfloat16>::value,
+                  "the training epilogue is bf16 only");
+    TOut* z = reinterpret_cast<TOut*>(args.aux_out);
+#pragma unroll 1
+    for (int p = 0; p < BN / 128; ++p) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t gr[32], ur[32];
+        tc::tmem_ld32(taddr + p * 128 + h * 32, gr);
+        tc::tmem_ld32(taddr + p * 128 + 64 + h * 32, ur);
+        tc::tmem_ld_wait();
+        if (valid) {
+          float gv[32], uv[32], hv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            gv[i] = round_bf16(__uint_as_float(gr[i]));
+            uv[i] = round_bf16(__uint_as_float(ur[i]));
+            hv[i] = gv[i] / (1.0f + __expf(-gv[i])) * uv[i];
+          }
+          TOut* zg = z + grow * args.ld_aux + n0 + p * 128 + h * 32;
+          TOut* dst = out + grow * ldo + (n0 >> 1) + p * 64 + h * 32;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            st_v4(zg + v * 8, Vec16<TOut>::from_f32(gv + v * 8));
+            st_v4(zg + 64 + v * 8, Vec16<TOut>::from_f32(uv + v * 8));
+            st_v4(dst + v * 8, Vec16<TOut>::from_f32(hv + v * 8));
+          }
+        }
+      }
+    }
+  } else if constexpr (EPI == kEpiSwiGLUBwd) {
+    static_assert(std::is_same<TOut, __nv_bfloat16>::value,
+                  "the training epilogue is bf16 only");
+    const TOut* z = reinterpret_cast<const TOut*>(args.aux_in);
+    TOut* dz = reinterpret_cast<TOut*>(args.aux_out);
+    const float w = (valid && row_scale) ? row_scale[grow] : 1.0f;
+    float dgp = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t vr[32];
+      tc::tmem_ld32(taddr + c * 32, vr);
+      tc::tmem_ld_wait();
+      if (valid) {
+        const int i0 = n0 + c * 32;  // column of h (= of W_down's f axis)
+        const size_t zoff = grow * args.ld_aux + (size_t)((i0 >> 6) * 128 + (i0 & 63));
+        float zg[32], zu[32], dg[32], du[32], hg[32];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          Vec16<TOut>::to_f32(ld_v4(z + zoff + v * 8), zg + v * 8);
+          Vec16<TOut>::to_f32(ld_v4(z + zoff + 64 + v * 8), zu + v * 8);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dh = __uint_as_float(vr[i]);
+          const float sg = 1.0f / (1.0f + __expf(-zg[i]));
+          const float silu = zg[i] * sg;
+          const float hv = round_bf16(silu * zu[i]);
+          dgp += dh * hv;
+          const float dhw = w * dh;
+          dg[i] = dhw * zu[i] * sg * (1.0f + zg[i] * (1.0f - sg));
+          du[i] = dhw * silu;
+          hg[i] = w * hv;
+        }
+        TOut* dst = out + grow * ldo + i0;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          st_v4(dz + zoff + v * 8, Vec16<TOut>::from_f32(dg + v * 8));
+          st_v4(dz + zoff + 64 + v * 8, Vec16<TOut>::from_f32(du + v * 8));
+          st_v4(dst + v * 8, Vec16<TOut>::from_f32(hg + v * 8));
+        }
+      }
+    }
+    if (valid && args.partial) args.partial[grow * args.n_part + n0 / BN] = dgp;
+  } else if constexpr (EPI == kEpiSwiGLU) {
     // columns [128p, 128p+64) are gate rows, [128p+64, 128p+128) the matching up rows
 #pragma unroll 1
     for (int p = 0; p < BN / 128; ++p) {
@@ -174,13 +274,18 @@ __device__ __forceinline__ void group_tile_prefix(const int32_t* group_off, int 
   if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_error(err, kErrIndex);
 }
 
-template <int BN, int EPI, bool TF32, bool GATHER>
+// B_MN: B is stored MN-major -- B[g*K + k][n], n contiguous (a weight used
+// transposed, as in the input-gradient GEMMs) -- and is loaded as BN/64 boxes
+// of 64 columns x 64 K rows.
+template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
   using Cfg = GemmCfg<BN, TF32>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
+  static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
+  static_assert(!B_MN || BN % 64 == 0, "MN-major B needs BN a multiple of 64");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -329,8 +434,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               tc::mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
               if (!GATHER)
                 tc::tma_load_2d(tc::smem_u32(sa), &tmap_a, fb, kb * Cfg::kBK, row0, pol_a);
-              tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, kb * Cfg::kBK,
-                              g * args.N + n0, pol_b);
+              if (B_MN) {
+#pragma unroll
+                for (int j = 0; j < BN / 64; ++j)
+                  tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes + j * 8192), &tmap_b, fb,
+                                  n0 + j * 64, g * args.K + kb * Cfg::kBK, pol_b);
+              } else {
+                tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, kb * Cfg::kBK,
+                                g * args.N + n0, pol_b);
+              }
             }
             if (GATHER) {
               __syncwarp();
@@ -359,7 +471,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = tc::idesc_m128<TF32, BN>();
+      constexpr uint32_t idesc = tc::idesc_f32acc<TF32, 128, BN, false, B_MN>();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -377,15 +489,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc::fence_after_sync();
           const uint32_t sa = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
           const uint64_t adesc = tc::desc_sw128_kmajor(sa);
-          const uint64_t bdesc = tc::desc_sw128_kmajor(sa + Cfg::kABytes);
+          const uint64_t bdesc = B_MN ? tc::desc_sw128_mnmajor(sa + Cfg::kABytes, 8192)
+                                      : tc::desc_sw128_kmajor(sa + Cfg::kABytes);
 #pragma unroll
           for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {
-            // +32 bytes along K inside the swizzled row = +2 in the address field
+            // K-major: +32 bytes along K inside the swizzled row = +2 in the
+            // address field; MN-major: +16 K rows = two 1024-byte atoms = +128
             const uint64_t off = static_cast<uint64_t>(kk * 2);
+            const uint64_t boff = B_MN ? static_cast<uint64_t>(kk * 128) : off;
             if (TF32)
-              tc::mma_tf32(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+              tc::mma_tf32(d_tmem, adesc + off, bdesc + boff, idesc, (kb | kk) != 0);
             else
-              tc::mma_f16(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+              tc::mma_f16(d_tmem, adesc + off, bdesc + boff, idesc, (kb | kk) != 0);
           }
           tc::commit(tc::smem_u32(&empty_bar[stage]));  // frees the stage when these MMAs finish
           if (++stage == S) {
@@ -410,7 +525,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r_in_tile = quarter * 32 + (int)lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    TOut* out = reinterpret_cast<TOut*>(args.out);
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int g, row0, rows, n0;
       locate(tile, g, row0, rows, n0);
@@ -425,7 +539,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool valid = r_in_tile < rows;
       const size_t grow = static_cast<size_t>(row0 + r_in_tile);
-      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args.row_scale, out, args.ldo);
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tc::smem_u32(&tempty_bar[acc]));

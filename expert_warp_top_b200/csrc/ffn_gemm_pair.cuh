@@ -41,11 +41,14 @@ struct PairCfg {
                                        sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
 };
 
-template <int BN, int EPI, bool TF32>
+// B_MN: B stored MN-major (B[g*K + k][n], n contiguous); each CTA loads its
+// BN/2 columns as 64-column boxes.
+template <int BN, int EPI, bool TF32, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
+  static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
   using Cfg = PairCfg<BN, TF32>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
@@ -154,8 +157,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (rank == 0) tc::mbar_arrive_expect_tx(fb, 2 * Cfg::kStageBytes);
             tc::tma_load_2d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, kb * Cfg::kBK,
                                  row0 + (int)rank * 128, pol_a);
-            tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
-                                 kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);
+            if (B_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j)
+                tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes + j * 8192), &tmap_b, fb_pair,
+                                     n0 + (int)rank * (BN / 2) + j * 64, g * args.K + kb * Cfg::kBK,
+                                     pol_b);
+            } else {
+              tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
+                                   kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);
+            }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
@@ -175,7 +186,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = tc::idesc_f32acc<TF32, 256, BN>();
+      constexpr uint32_t idesc = tc::idesc_f32acc<TF32, 256, BN, false, B_MN>();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -193,14 +204,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc::fence_after_sync();
           const uint32_t sa = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
           const uint64_t adesc = tc::desc_sw128_kmajor(sa);
-          const uint64_t bdesc = tc::desc_sw128_kmajor(sa + Cfg::kABytes);
+          const uint64_t bdesc = B_MN ? tc::desc_sw128_mnmajor(sa + Cfg::kABytes, 8192)
+                                      : tc::desc_sw128_kmajor(sa + Cfg::kABytes);
 #pragma unroll
           for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {
             const uint64_t off = static_cast<uint64_t>(kk * 2);
+            const uint64_t boff = B_MN ? static_cast<uint64_t>(kk * 128) : off;
             if (TF32)
-              tc::mma_tf32_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+              tc::mma_tf32_pair(d_tmem, adesc + off, bdesc + boff, idesc, (kb | kk) != 0);
             else
-              tc::mma_f16_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+              tc::mma_f16_pair(d_tmem, adesc + off, bdesc + boff, idesc, (kb | kk) != 0);
           }
           // frees this stage in both CTAs once these MMAs have read it
           tc::commit_pair_multicast(tc::smem_u32(&empty_bar[stage]), 0x3);
@@ -225,7 +238,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r_in_half = quarter * 32 + (int)lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    TOut* out = reinterpret_cast<TOut*>(args.out);
     const uint32_t tempty_local = tc::smem_u32(&tempty_bar[0]);
     for (int tile = pair; tile < total_tiles; tile += n_pairs) {
       int g, row0, gend, n0;
@@ -240,8 +252,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              static_cast<uint32_t>(acc * BN);
       const int grow_i = row0 + (int)rank * 128 + r_in_half;
       const bool valid = grow_i < gend;
-      epilogue_rows<BN, EPI, TOut>(taddr, valid, static_cast<size_t>(grow_i), n0, args.row_scale,
-                                   out, args.ldo);
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, static_cast<size_t>(grow_i), n0, args);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) {

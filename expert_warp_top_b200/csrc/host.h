@@ -1,0 +1,288 @@
+// host.h -- host-side helpers shared by the library's translation units:
+// error reporting, per-device state, tensor maps, launch helpers and the
+// launchers of the tcgen05 GEMM kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "../../include/moe_occult.h"
+#include "ffn_gemm.cuh"
+#include "ffn_gemm_pair.cuh"
+#include "wgrad_gemm.cuh"
+
+namespace moe_host {
+
+// Sets this thread's error message (moe_last_error) and returns code.
+int fail(int code, const char* fmt, ...);
+const char* last_message();
+
+#define MOE_REQUIRE(cond, code, ...)                       \
+  do {                                                     \
+    if (!(cond)) return ::moe_host::fail(code, __VA_ARGS__); \
+  } while (0)
+
+#define MOE_CUDA(call)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return ::moe_host::fail(MOE_ERR_CUDA, "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                              __FILE__, __LINE__);                                         \
+  } while (0)
+
+#define MOE_LAUNCHED(what)                                                                 \
+  do {                                                                                     \
+    cudaError_t e_ = cudaGetLastError();                                                   \
+    if (e_ != cudaSuccess)                                                                 \
+      return ::moe_host::fail(MOE_ERR_CUDA, "launch of %s failed: %s", what,               \
+                              cudaGetErrorString(e_));                                     \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned* err_flag = nullptr;  // the device error flag the kernels raise
+  std::mutex mu;
+  std::vector<const void*> smem_raised;                   // kernels with the smem limit raised
+  std::vector<std::pair<const void*, int>> pair_clusters;  // CTA-pair kernels: clusters that fit
+};
+
+// The current device's state (checks that it is an sm_100 part).
+int device_info(DeviceInfo** out);
+
+// Raises kern's dynamic shared-memory limit to `bytes`, once per device.
+int ensure_smem(DeviceInfo* di, const void* kern, size_t bytes);
+
+// Test-only knobs, set by moe_set_debug.
+extern int g_debug_flags;
+extern double g_wait_limit_ms;
+inline uint64_t wait_limit_ns() { return static_cast<uint64_t>(g_wait_limit_ms * 1.0e6); }
+constexpr int kDebugForceSingle = 2;  // GEMMs on single CTAs
+constexpr int kDebugForcePair = 4;    // GEMMs on CTA pairs where the shape allows
+
+// 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
+int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows);
+
+int check_common(int T, int E, int k, int R);
+int check_dtype(int dtype);
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+inline int pick_bn(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Every kernel is launched with programmatic stream serialization, so the next
+// kernel on the stream can be scheduled while this one finishes; each kernel
+// starts with griddepcontrol.wait (moe::pdl_enter) before it touches memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// ---- the grouped GEMM (ffn_gemm.cuh / ffn_gemm_pair.cuh) --------------------
+// Arguments of the training epilogues (kEpiSwiGLUSave, kEpiSwiGLUBwd).
+struct GemmExtra {
+  const void* aux_in = nullptr;
+  void* aux_out = nullptr;
+  int ld_aux = 0;
+  float* partial = nullptr;
+  int n_part = 0;
+};
+
+inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
+                               const int32_t* a_row_index, int a_rows, int G, int N, int K,
+                               int m_cap, const float* row_scale, void* out, int ldo,
+                               const GemmExtra& ex) {
+  moe::GemmArgs a{group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo,
+                  di->err_flag, wait_limit_ns(), g_debug_flags};
+  a.aux_in = ex.aux_in;
+  a.aux_out = ex.aux_out;
+  a.ld_aux = ex.ld_aux;
+  a.partial = ex.partial;
+  a.n_part = ex.n_part;
+  return a;
+}
+
+// B's tensor map: K-major [G*N, K] with box [BN_box rows, 64 cols], or
+// MN-major [G*K, N] with box [64 K rows, 64 cols].
+template <bool B_MN>
+int encode_b(CUtensorMap* tb, const void* b, int dtype, int G, int N, int K, int bk,
+             uint32_t box_rows_kmajor) {
+  if (B_MN) return encode_2d(tb, b, dtype, (uint64_t)N, (uint64_t)G * K, 64, 64);
+  return encode_2d(tb, b, dtype, (uint64_t)K, (uint64_t)G * N, bk, box_rows_kmajor);
+}
+
+// A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
+// gathered from it (row p = a[a_row_index[p]]), else they are a's first m_cap.
+template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN>
+int launch_gemm(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_index, int m_cap,
+                int K, const void* b, int G, int N, const int32_t* group_off,
+                const float* row_scale, void* out, int ldo, const GemmExtra& ex,
+                cudaStream_t st) {
+  using Cfg = moe::GemmCfg<BN, TF32>;
+  const int dtype = TF32 ? MOE_F32 : MOE_BF16;
+  CUtensorMap ta, tb;
+  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK,
+                     GATHER ? 1u : (uint32_t)moe::kGemmBM);
+  if (rc) return rc;
+  if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN))) return rc;
+  auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32, GATHER, B_MN>;
+  if ((rc = ensure_smem(di, reinterpret_cast<const void*>(kern), Cfg::kSmemBytes))) return rc;
+  const long long ub = ((long long)m_cap / moe::kGemmBM + G) * (N / BN);
+  const int grid = (int)(ub < di->num_sms ? (ub < 1 ? 1 : ub) : di->num_sms);
+  const moe::GemmArgs args =
+      gemm_args(di, group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
+  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, args));
+  MOE_LAUNCHED("ffn_gemm_kernel");
+  return MOE_OK;
+}
+
+template <int EPI, bool TF32, bool GATHER, bool B_MN>
+int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int a_rows,
+                   const int32_t* a_row_index, int m_cap, int K, const void* b, int G, int N,
+                   const int32_t* group_off, const float* row_scale, void* out, int ldo,
+                   const GemmExtra& ex, cudaStream_t st) {
+  if (bn == 256)
+    return launch_gemm<256, EPI, TF32, GATHER, B_MN>(di, a, a_rows, a_row_index, m_cap, K, b, G,
+                                                     N, group_off, row_scale, out, ldo, ex, st);
+  if (bn == 128)
+    return launch_gemm<128, EPI, TF32, GATHER, B_MN>(di, a, a_rows, a_row_index, m_cap, K, b, G,
+                                                     N, group_off, row_scale, out, ldo, ex, st);
+  return launch_gemm<64, EPI, TF32, GATHER, B_MN>(di, a, a_rows, a_row_index, m_cap, K, b, G, N,
+                                                  group_off, row_scale, out, ldo, ex, st);
+}
+
+// The same GEMM on CTA pairs (cluster of 2, M = 256 tiles).  Needs BN/2 >= 64.
+template <int BN, int EPI, bool TF32, bool B_MN>
+int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K, const void* b,
+                     int G, int N, const int32_t* group_off, const float* row_scale, void* out,
+                     int ldo, const GemmExtra& ex, cudaStream_t st) {
+  using Cfg = moe::PairCfg<BN, TF32>;
+  const int dtype = TF32 ? MOE_F32 : MOE_BF16;
+  CUtensorMap ta, tb;
+  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
+  if (rc) return rc;
+  if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN / 2))) return rc;
+  auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32, B_MN>;
+  const void* key = reinterpret_cast<const void*>(kern);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
+  if ((rc = ensure_smem(di, key, Cfg::kSmemBytes))) return rc;
+  int max_clusters = 0;
+  {
+    std::lock_guard<std::mutex> lk(di->mu);
+    for (auto& pc : di->pair_clusters)
+      if (pc.first == key) max_clusters = pc.second;
+  }
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(2 * (di->num_sms / 2), 1, 1);
+    MOE_CUDA(cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg));
+    MOE_REQUIRE(max_clusters >= 1, MOE_ERR_UNSUPPORTED, "no CTA pair fits on this device");
+    std::lock_guard<std::mutex> lk(di->mu);
+    di->pair_clusters.emplace_back(key, max_clusters);
+  }
+  const long long ub = ((long long)m_cap / moe::kPairBM + G) * (N / BN);
+  const long long pairs = ub < max_clusters ? (ub < 1 ? 1 : ub) : max_clusters;
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.numAttrs = 2;
+  const moe::GemmArgs args =
+      gemm_args(di, group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
+  return MOE_OK;
+}
+
+// GEMM over the groups, on CTA pairs when the groups are tall enough to fill
+// 256-row tiles (and the rows are read in place), else on single CTAs.
+#ifndef MOE_PAIR_MIN_ROWS
+#define MOE_PAIR_MIN_ROWS 192
+#endif
+template <int EPI, bool TF32, bool B_MN = false>
+int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_index,
+                     int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
+                     const float* row_scale, void* out, int ldo, cudaStream_t st,
+                     const GemmExtra& ex = GemmExtra{}) {
+  const bool tall = (long long)m_cap >= (long long)MOE_PAIR_MIN_ROWS * G;
+  bool pair = !a_row_index && N % 128 == 0 && tall;
+  if (g_debug_flags & kDebugForceSingle) pair = false;
+  if ((g_debug_flags & kDebugForcePair) && !a_row_index && N % 128 == 0) pair = true;
+  if (pair) {
+    if (N % 256 == 0)
+      return launch_gemm_pair<256, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
+                                                    row_scale, out, ldo, ex, st);
+    return launch_gemm_pair<128, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
+                                                  row_scale, out, ldo, ex, st);
+  }
+  const int bn = pick_bn(N);
+  if constexpr (!B_MN) {
+    if (a_row_index)
+      return launch_gemm_bn<EPI, TF32, true, false>(di, bn, a, a_rows, a_row_index, m_cap, K, b,
+                                                    G, N, group_off, row_scale, out, ldo, ex, st);
+  }
+  return launch_gemm_bn<EPI, TF32, false, B_MN>(di, bn, a, a_rows, nullptr, m_cap, K, b, G, N,
+                                                group_off, row_scale, out, ldo, ex, st);
+}
+
+// ---- the weight-gradient GEMM (wgrad_gemm.cuh) -------------------------------
+// out[g] (+)= A_g^T B_g with A [rows, M], B [rows, N] bf16 row-major and the
+// groups' rows given by group_off.  M % 128 == 0, N % 64 == 0.
+template <int BN, typename TOut>
+int launch_wgrad_bn(DeviceInfo* di, const void* a, const void* b, int rows, int M, int N,
+                    const int32_t* group_off, int G, void* out, int accumulate, cudaStream_t st) {
+  using Cfg = moe::WgradCfg<BN>;
+  CUtensorMap ta, tb;
+  int rc = encode_2d(&ta, a, MOE_BF16, (uint64_t)M, (uint64_t)rows, 64, 64);
+  if (rc) return rc;
+  if ((rc = encode_2d(&tb, b, MOE_BF16, (uint64_t)N, (uint64_t)rows, 64, 64))) return rc;
+  auto kern = moe::wgrad_gemm_kernel<BN, TOut>;
+  if ((rc = ensure_smem(di, reinterpret_cast<const void*>(kern), Cfg::kSmemBytes))) return rc;
+  const long long tiles = (long long)G * (M / 128) * (N / BN);
+  const int grid = (int)(tiles < di->num_sms ? (tiles < 1 ? 1 : tiles) : di->num_sms);
+  moe::WgradArgs args{group_off, G, M, N, rows, out, accumulate, di->err_flag, wait_limit_ns(),
+                      g_debug_flags};
+  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, args));
+  MOE_LAUNCHED("wgrad_gemm_kernel");
+  return MOE_OK;
+}
+
+template <typename TOut>
+int launch_wgrad(DeviceInfo* di, const void* a, const void* b, int rows, int M, int N,
+                 const int32_t* group_off, int G, void* out, int accumulate, cudaStream_t st) {
+  const int bn = pick_bn(N);
+  if (bn == 256)
+    return launch_wgrad_bn<256, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);
+  if (bn == 128)
+    return launch_wgrad_bn<128, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);
+  return launch_wgrad_bn<64, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);
+}
+
+}  // namespace moe_host

@@ -128,6 +128,11 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
+// Orders this thread's earlier generic-proxy writes to shared memory before
+// later async-proxy accesses (TMA, tensor-core operand reads) of it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void fence_before_sync() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -293,12 +298,30 @@ __device__ __forceinline__ uint64_t desc_sw128_kmajor(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: D fp32, A/B bf16 (or tf32), both K-major.
-template <bool kTf32, int kM, int kN>
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle
+// layout.  A 1024-byte atom holds 8 K rows of 128 bytes, each row 64 (bf16)
+// MN-consecutive elements; atoms of successive groups of 8 K rows follow
+// every 1024 bytes (stride byte offset), and the next 64-wide MN chunk starts
+// mn_stride bytes later (leading byte offset).
+__device__ __forceinline__ uint64_t desc_sw128_mnmajor(uint32_t saddr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);             // start address
+  d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;   // leading byte offset
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;                   // stride byte offset
+  d |= static_cast<uint64_t>(1u) << 46;                           // descriptor version
+  d |= static_cast<uint64_t>(2u) << 61;                           // swizzle mode: 128 B
+  return d;
+}
+
+// Instruction descriptor: D fp32, A/B bf16 (or tf32); A and B K-major unless
+// kAMn / kBMn make them MN-major (bits 15 and 16).
+template <bool kTf32, int kM, int kN, bool kAMn = false, bool kBMn = false>
 __host__ __device__ constexpr uint32_t idesc_f32acc() {
   return (1u << 4)                              // D format: f32
          | ((kTf32 ? 2u : 1u) << 7)             // A format: bf16 / tf32
          | ((kTf32 ? 2u : 1u) << 10)            // B format: bf16 / tf32
+         | ((kAMn ? 1u : 0u) << 15)             // A major-ness
+         | ((kBMn ? 1u : 0u) << 16)             // B major-ness
          | (static_cast<uint32_t>(kN >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(kM >> 4) << 24);  // M / 16
 }

@@ -1,0 +1,312 @@
+// wgrad_gemm.cuh -- per-expert weight gradients on tcgen05.
+//
+// For every expert group g (rows group_off[g] .. group_off[g+1]-1):
+//   C_g[m, n] = sum over the group's rows p of A[p, m] * B[p, n]
+// with A [rows, M] and B [rows, N] row-major, i.e. C_g = A_g^T B_g.  Both
+// operands are therefore MN-major and the contraction runs over the group's
+// rows, whose count is ragged.  This is the weight gradient of a grouped
+// GEMM: dW_down[g] = dO_g^T (w h)_g and dW_gate/up[g] = dZ_g^T X_g.
+//
+// Kernel shape (one persistent CTA per SM, 192 threads), as the forward GEMM:
+//   warp 0      TMA producer: per stage 64 rows of A (two boxes of 64 columns)
+//               and of B (BN/64 boxes), 128-byte swizzle
+//   warp 1      MMA issuer (lane 0) and tail fixer (whole warp): in a group's
+//               last, partial row block the rows past the group's end belong
+//               to the next group, so the warp zeroes them in shared memory
+//               (a 128-byte row of a swizzled box holds exactly one row)
+//               before the MMAs read the stage
+//   warps 2..5  epilogue: tcgen05.ld of 32 accumulator rows (= 32 values of m)
+//               and a store of BN columns per row (fp32 or bf16, optionally
+//               added to what the output holds)
+// Tiles: group by group, M block, N block fastest.  A group without rows
+// writes zeros (or leaves the output as it is when accumulating).  Every wait
+// is bounded, as in the forward kernel.
+#pragma once
+#include "ffn_gemm.cuh"
+
+namespace moe {
+
+struct WgradArgs {
+  const int32_t* group_off;  // [G+1] device
+  int G;
+  int M, N;                  // output of one group: [M, N]
+  int rows;                  // rows of A and B
+  void* out;                 // [G, M, N]
+  int accumulate;            // 1: out += C, 0: out = C
+  unsigned* err;
+  uint64_t wait_limit_ns;
+  int debug;
+};
+
+template <int BN>
+struct WgradCfg {
+  static constexpr int kBK = 64;                     // rows (the K of this GEMM) per stage
+  static constexpr int kABytes = 128 * 128;          // 128 columns of A x 64 rows
+  static constexpr int kBBytes = BN * 128;           // BN columns of B x 64 rows
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256 +
+                                       sizeof(int32_t) * (2 * kGemmMaxGroups + 2);
+};
+
+template <int BN, typename TOut>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    wgrad_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                      const __grid_constant__ CUtensorMap tmap_b, const WgradArgs args) {
+  static_assert(BN == 64 || BN == 128 || BN == 256, "BN must be 64, 128 or 256");
+  using Cfg = WgradCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  constexpr int kChunks = (Cfg::kABytes + Cfg::kBBytes) / 8192;  // 64-column boxes per stage
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * Cfg::kStageBytes);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + S;
+  uint64_t* tfull_bar = bars + 2 * S;
+  uint64_t* tempty_bar = bars + 2 * S + 2;
+  uint64_t* drain_bar = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_off = reinterpret_cast<int32_t*>(smem + (size_t)S * Cfg::kStageBytes + 256);
+  int32_t* s_end = s_off + kGemmMaxGroups + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  const int G = args.G;
+  const int m_blocks = args.M / 128, n_blocks = args.N / BN;
+  const int tiles_per_group = m_blocks * n_blocks;
+  const int total_tiles = G * tiles_per_group;
+
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmap_a);
+    tc::tma_prefetch_desc(&tmap_b);
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
+      tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(tc::smem_u32(&tfull_bar[a]), 1);
+      tc::mbar_init(tc::smem_u32(&tempty_bar[a]), 4);
+    }
+    tc::mbar_init(tc::smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    tc::mbar_init_fence();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), Cfg::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  pdl_enter();
+  if (warp == 2) {
+    // group bounds; a group that leaves [0, rows] or runs backwards is empty
+    // and raises the index error bit
+    bool bad = false;
+    for (int g = (int)lane; g < G; g += 32) {
+      const int lo = args.group_off[g], hi = args.group_off[g + 1];
+      const bool ok = lo >= 0 && hi >= lo && hi <= args.rows;
+      bad |= !ok;
+      s_off[g] = ok ? lo : 0;
+      s_end[g] = ok ? hi : 0;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_error(args.err, kErrIndex);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const tc::WaitCtl wctl{abort_flag, args.err, args.wait_limit_ns};
+
+  auto locate = [&](int tile, int& g, int& m0, int& n0) {
+    g = tile / tiles_per_group;
+    const int r = tile - g * tiles_per_group;
+    const int mb = r / n_blocks;
+    m0 = mb * 128;
+    n0 = (r - mb * n_blocks) * BN;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = tc::policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_parity = 0;
+      bool skip_next = (args.debug & kDebugSkipFirstLoad) != 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int g, m0, n0;
+        locate(tile, g, m0, n0);
+        const int r0 = s_off[g], r1 = s_end[g];
+        const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl)) {
+            ok = false;
+            break;
+          }
+          if (!skip_next) {
+            const uint32_t fb = tc::smem_u32(&full_bar[stage]);
+            uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
+            const int y = r0 + kb * Cfg::kBK;
+            tc::mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tc::tma_load_2d(tc::smem_u32(sa + j * 8192), &tmap_a, fb, m0 + j * 64, y, pol);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes + j * 8192), &tmap_b, fb,
+                              n0 + j * 64, y, pol);
+            armed |= 1u << stage;
+            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          }
+          skip_next = false;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      for (int s = 0; s < S; ++s)
+        if ((armed >> s) & 1u)
+          tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------- MMA issuer + tail zeroing
+    constexpr uint32_t idesc = tc::idesc_f32acc<false, 128, BN, true, true>();
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int g, m0, n0;
+      locate(tile, g, m0, n0);
+      const int r0 = s_off[g], r1 = s_end[g];
+      const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
+      bool go = true;
+      if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl);
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      tc::fence_after_sync();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&full_bar[stage]), phase, wctl);
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
+        const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
+        if (valid < Cfg::kBK) {
+          // rows valid..63 of every box belong to another group: zero them
+          const int n16 = (Cfg::kBK - valid) * 8;  // 16-byte pieces per box
+          for (int i = (int)lane; i < kChunks * n16; i += 32) {
+            const int c = i / n16, q = i - c * n16;
+            st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
+          }
+          tc::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t sa_u = tc::smem_u32(sa);
+          const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
+          const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
+          const int n_kk = (valid + 15) / 16;
+          for (int kk = 0; kk < n_kk; ++kk) {
+            // +16 rows = two 1024-byte atoms = +128 in the address field
+            const uint64_t off = static_cast<uint64_t>(kk * 128);
+            tc::mma_f16(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+          }
+          tc::commit(tc::smem_u32(&empty_bar[stage]));
+        }
+        __syncwarp();
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) tc::commit(tc::smem_u32(&tfull_bar[acc]));  // also for an empty group
+      __syncwarp();
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) {
+      tc::commit(tc::smem_u32(drain_bar));
+      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    TOut* out = reinterpret_cast<TOut*>(args.out);
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int g, m0, n0;
+      locate(tile, g, m0, n0);
+      const bool has_rows = s_end[g] > s_off[g];
+      bool ok = true;
+      if (lane == 0) ok = tc::wait_bounded(tc::smem_u32(&tfull_bar[acc]), acc_phase, wctl);
+      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+      if (!ok) break;
+      __syncwarp();
+      tc::fence_after_sync();
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const size_t m = (size_t)m0 + quarter * 32 + lane;
+      TOut* dst = out + ((size_t)g * args.M + m) * args.N + n0;
+      if (has_rows || !args.accumulate) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          if (has_rows) {
+            uint32_t vr[32];
+            tc::tmem_ld32(taddr + c * 32, vr);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          TOut* p = dst + c * 32;
+          constexpr int VN = Vec16<TOut>::n;
+          if (args.accumulate) {
+#pragma unroll
+            for (int q = 0; q < 32 / VN; ++q) {
+              float old[VN];
+              Vec16<TOut>::to_f32(ld_v4(p + q * VN), old);
+#pragma unroll
+              for (int i = 0; i < VN; ++i) v[q * VN + i] += old[i];
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 32 / VN; ++q) st_v4(p + q * VN, Vec16<TOut>::from_f32(v + q * VN));
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tc::smem_u32(&tempty_bar[acc]));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -20,6 +20,10 @@ How the experts reach their EPD rows (epd_mode):
   pre-reduce + combine          moe_combine_scatter
   dispatched-row counter        moe_count_dispatched_rows
   co-activation histogram       moe_coact_histogram (accumulating)
+
+Training: forward_train() (moe_layer_forward_train) keeps the layer's state in
+a training workspace and backward() (moe_layer_backward) returns the gradients
+of x, of the router logits and of the packed routed and shared weights.
 """
 from __future__ import annotations
 
@@ -206,3 +210,69 @@ class MoELayer:
                                  sw_dn=getattr(self, "sw_dn", None), S=self.S, fs=self.fs,
                                  prune_m=self.prune_m, stream=stream)
         return h_y
+
+    # -- training: forward that keeps state, and the backward ----------------
+    def _train_ws(self):
+        ws = getattr(self, "_ws_train", None)
+        if ws is None:
+            n = B.moe_layer_train_workspace_size(self.T, self.d, self.f, self.E, self.k, self.R,
+                                                 self.S, self.fs)
+            if n == 0:
+                raise ValueError("this layer shape is not supported for training "
+                                 "(bf16, d a multiple of 128, f of 64)")
+            ws = torch.empty(n, dtype=torch.uint8, device=self.y.device)
+            self._ws_train = ws
+        return ws
+
+    def forward_train(self, logits, x, y=None, stream=None):
+        """The layer (moe_layer_forward_train), keeping what backward() needs."""
+        y = self.y if y is None else y
+        self._train_inputs = (logits, x)
+        B.moe_layer_forward_train(logits, x, self.k, self.R, self.renorm, self.slot_of, self.w_gu,
+                                  self.w_dn, self.f, y, self._train_ws(),
+                                  sw_gu=getattr(self, "sw_gu", None),
+                                  sw_dn=getattr(self, "sw_dn", None), S=self.S, fs=self.fs,
+                                  stream=stream)
+        return y
+
+    def backward(self, dy, dw_dtype=torch.float32, grads=None, accumulate=False, stream=None):
+        """Gradients of the last forward_train for the upstream gradient dy [T, d].
+
+        Returns a dict: dx [T, d], d_logits [T, E] f32, d_topk_w [T, k] f32 (the
+        gate weights' gradient), dw_gu [E, 2f, d] and
+        dw_dn [E, d, f] in the packed slot-order layout of w_gu / w_dn (see
+        unpack_gate_up), and with shared experts dsw_gu / dsw_dn.  `grads`
+        (a dict from an earlier call) is reused, and with accumulate=True the
+        weight gradients are added to it."""
+        logits, x = self._train_inputs
+        dev = self.y.device
+        if grads is None:
+            wd = dict(dtype=dw_dtype, device=dev)
+            grads = dict(dx=torch.empty(self.T, self.d, dtype=self.dtype, device=dev),
+                         d_logits=torch.empty(self.T, self.E, dtype=torch.float32, device=dev),
+                         d_topk_w=torch.empty(self.T, self.k, dtype=torch.float32, device=dev),
+                         dw_gu=torch.empty(self.E, 2 * self.f, self.d, **wd),
+                         dw_dn=torch.empty(self.E, self.d, self.f, **wd))
+            if self.S > 0:
+                F = self.S * self.fs
+                grads["dsw_gu"] = torch.empty(1, 2 * F, self.d, **wd)
+                grads["dsw_dn"] = torch.empty(1, self.d, F, **wd)
+        B.moe_layer_backward(logits, x, self.k, self.R, self.renorm, self.slot_of, self.w_gu,
+                             self.w_dn, self.f, dy, grads["dx"], grads["d_logits"],
+                             grads["dw_gu"], grads["dw_dn"], self._train_ws(),
+                             sw_gu=getattr(self, "sw_gu", None), sw_dn=getattr(self, "sw_dn", None),
+                             S=self.S, fs=self.fs, dsw_gu=grads.get("dsw_gu"),
+                             dsw_dn=grads.get("dsw_dn"), accumulate=int(accumulate),
+                             d_topk_w=grads.get("d_topk_w"), stream=stream)
+        return grads
+
+
+def unpack_gate_up(w_gu: torch.Tensor):
+    """Packed [..., 2F, d] gate/up rows (64-row blocks interleaved, as
+    moe_prepare_weights writes them and the backward returns their gradients)
+    -> (gate [..., F, d], up [..., F, d])."""
+    *lead, two_f, d = w_gu.shape
+    blocks = w_gu.reshape(*lead, two_f // 128, 2, 64, d)
+    gate = blocks[..., 0, :, :].reshape(*lead, two_f // 2, d)
+    up = blocks[..., 1, :, :].reshape(*lead, two_f // 2, d)
+    return gate, up

@@ -379,6 +379,105 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
                            const void* sw_gu, const void* sw_dn, void* h_y,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ===========================================================================
+ * Training: forward that keeps what the backward needs, and the backward.
+ *
+ * The backward is the exact derivative of the layer for fixed expert choices:
+ * the top-k selection passes no gradient, and each gate weight passes its
+ * gradient through the softmax it came from (renorm 0: over all E logits;
+ * renorm 1: over the k selected ones).  Data moves through the same BRIMs as
+ * in the forward ("bidirectional re-index", Occult paper, Figure 4): the
+ * upstream gradient travels ORI -> SFD -> EPD like x did (moe_dispatch_gather)
+ * and the input gradient returns EPD -> SFD -> ORI like y did
+ * (moe_combine_scatter).  Training is bf16 only (MOE_BF16 activations and
+ * weights) and defined for unpruned routing; d must be a multiple of 128.
+ * ========================================================================= */
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_ffn_train -- moe_expert_ffn (SwiGLU) that also returns
+ *   z  [m_cap, 2f] bf16  the gate/up pre-activations A W_gu^T, rounded to bf16,
+ *                        in w_gu's packed column order (64-wide gate and up
+ *                        blocks interleaved)
+ *   h  [m_cap, f]  bf16  silu(z_gate) * z_up of those rounded values
+ *   out [m_cap, d] bf16  row_scale * (h W_down^T)
+ * Rows outside the groups are not written.  No workspace.  Arguments otherwise
+ * as moe_expert_ffn (no row index: a's rows are the groups' rows).
+ * ------------------------------------------------------------------------- */
+int moe_expert_ffn_train(const void* a, int a_rows, const int32_t* group_off, int G, int m_cap,
+                         const void* w_gu, const void* w_dn, int d, int f,
+                         const float* row_scale, void* z, void* h, void* out,
+                         moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_ffn_backward -- gradients of moe_expert_ffn_train for the upstream
+ * gradient dout [a_rows, d] (bf16, the same rows as a):
+ *   dx          [m_cap, d] bf16   d/da                   (rows of the groups)
+ *   d_row_scale [m_cap] f32       d/d row_scale, 0 on rows past the groups
+ *                                 (may be NULL; requires row_scale)
+ *   dw_gu       [G, 2f, d]        d/d w_gu, packed like w_gu   (may be NULL)
+ *   dw_dn       [G, d, f]         d/d w_dn                     (may be NULL)
+ * dw_dtype (MOE_F32 or MOE_BF16) is the type of dw_gu / dw_dn; accumulate = 1
+ * adds to them instead of overwriting (an expert with no rows then leaves
+ * them as they are; with accumulate = 0 it gets zeros).  z is the
+ * moe_expert_ffn_train output.  Kernels: the input-gradient GEMM of the down
+ * projection with the SwiGLU and gate backward fused into its epilogue, the
+ * input-gradient GEMM of gate/up, and two weight-gradient GEMMs (tcgen05).
+ *   ws  at least moe_expert_ffn_backward_workspace_size(m_cap, f) bytes,
+ *       16-byte aligned
+ * ------------------------------------------------------------------------- */
+size_t moe_expert_ffn_backward_workspace_size(int m_cap, int f);
+int moe_expert_ffn_backward(const void* dout, const void* a, int a_rows, const void* z,
+                            const int32_t* group_off, int G, int m_cap, const void* w_gu,
+                            const void* w_dn, int d, int f, const float* row_scale, void* dx,
+                            float* d_row_scale, void* dw_gu, void* dw_dn, int dw_dtype,
+                            int accumulate, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route_backward -- gradient of the router logits.  d_gate_epd [T*k] f32
+ * holds the gradient of each gate weight in EPD order (moe_expert_ffn_backward's
+ * d_row_scale); the row of token t's slot j is found through the BRIMs,
+ * p = BRIM_1[loc(e)][BRIM_0[rank(e)][t]] with e = topk_idx[t][j].  With q the
+ * softmax of the token's logits over the normalisation set of `renorm`,
+ *   d_logits[t][e] = q_e * (dw(e) - sum_j dw_j w_j),   q_e = 0 off the set,
+ * where dw(e) is the gradient of e's gate (0 if e was not selected).
+ *   d_logits [T, E] f32 out;  d_topk_w [T, k] f32 out (may be NULL): dw_j
+ * ------------------------------------------------------------------------- */
+int moe_route_backward(const float* logits, int T, int E, int k, int renorm,
+                       const int32_t* topk_idx, const int32_t* slot_of, int R,
+                       const int32_t* brim0, const int32_t* brim1, const float* d_gate_epd,
+                       float* d_logits, float* d_topk_w, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_layer_forward_train / moe_layer_backward -- the whole layer for
+ * training.  moe_layer_forward_train is moe_layer_forward (no pruning, no
+ * statistics outputs) that keeps in `ws` what moe_layer_backward needs: the
+ * top-k, the BRIMs, the EPD rows and the expert pre-activations.
+ * moe_layer_backward then takes the upstream gradient dy [T, d] and writes
+ *   dx        [T, d] bf16     d/dx (routed experts + shared experts)
+ *   d_logits  [T, E] f32      d/d logits
+ *   d_topk_w  [T, k] f32      d/d the gate weights (may be NULL)
+ *   dw_gu, dw_dn              d/d the routed weights, packed like w_gu / w_dn
+ *                             (slot order), dw_dtype
+ *   dsw_gu, dsw_dn            d/d the shared weights (packed), dw_dtype
+ *                             (NULL when S = 0)
+ * with the same arguments and the same `ws` as the forward call before it
+ * (nothing else may use ws in between).  accumulate as in
+ * moe_expert_ffn_backward.
+ *   ws  at least moe_layer_train_workspace_size(...) bytes, 256-byte aligned
+ * ------------------------------------------------------------------------- */
+size_t moe_layer_train_workspace_size(int T, int d, int f, int E, int k, int R, int S, int fs);
+int moe_layer_forward_train(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                            const float* logits, const void* x, const int32_t* slot_of,
+                            const void* w_gu, const void* w_dn, const void* sw_gu,
+                            const void* sw_dn, void* y, void* ws, size_t ws_bytes,
+                            moe_stream_t stream);
+int moe_layer_backward(int T, int d, int f, int E, int k, int R, int renorm, int S, int fs,
+                       const float* logits, const void* x, const int32_t* slot_of,
+                       const void* w_gu, const void* w_dn, const void* sw_gu, const void* sw_dn,
+                       const void* dy, void* dx, float* d_logits, float* d_topk_w, void* dw_gu,
+                       void* dw_dn, void* dsw_gu, void* dsw_dn, int dw_dtype, int accumulate,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

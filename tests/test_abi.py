@@ -81,6 +81,40 @@ def test_ffn_rejects_bad_shapes():
     assert ffn() == B.MOE_ERR_INVALID_ARG                 # null pointers
 
 
+def test_training_entries_reject_bad_arguments_on_host():
+    lib = moe.load()
+
+    def bwd(G=1, a_rows=16, m_cap=16, d=128, f=128, dw_dtype=B.MOE_F32, acc=0, rs=NULL,
+            drs=NULL):
+        return lib.moe_expert_ffn_backward(NULL, NULL, a_rows, NULL, NULL, G, m_cap, NULL, NULL,
+                                           d, f, rs, NULL, drs, NULL, NULL, dw_dtype, acc, NULL,
+                                           ctypes.c_size_t(0), NULL)
+
+    assert bwd(d=64) == B.MOE_ERR_UNSUPPORTED         # training needs d % 128 == 0
+    assert bwd(f=96) == B.MOE_ERR_UNSUPPORTED
+    assert bwd(G=0) == B.MOE_ERR_UNSUPPORTED
+    assert bwd(a_rows=8) == B.MOE_ERR_INVALID_ARG      # a shorter than m_cap
+    assert bwd(dw_dtype=9) == B.MOE_ERR_INVALID_ARG
+    assert bwd(acc=2) == B.MOE_ERR_INVALID_ARG
+    assert bwd(drs=ctypes.c_void_p(16)) == B.MOE_ERR_INVALID_ARG  # d_row_scale without row_scale
+    assert bwd() == B.MOE_ERR_INVALID_ARG              # null pointers
+    assert lib.moe_expert_ffn_train(NULL, 16, NULL, 1, 16, NULL, NULL, 64, 128, NULL, NULL, NULL,
+                                    NULL, NULL) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_expert_ffn_train(NULL, 16, NULL, 1, 16, NULL, NULL, 128, 128, NULL, NULL, NULL,
+                                    NULL, NULL) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_backward(NULL, 16, 8, 2, 3, NULL, NULL, 4, NULL, NULL, NULL, NULL, NULL,
+                                  NULL) == B.MOE_ERR_INVALID_ARG   # renorm must be 0 or 1
+    assert lib.moe_route_backward(NULL, 16, 8, 2, 0, NULL, NULL, 3, NULL, NULL, NULL, NULL, NULL,
+                                  NULL) == B.MOE_ERR_UNSUPPORTED   # R does not divide E
+    assert lib.moe_route_backward(NULL, 0, 8, 2, 0, NULL, NULL, 4, NULL, NULL, NULL, NULL, NULL,
+                                  NULL) == B.MOE_OK                # empty batch: nothing to do
+    assert moe.moe_layer_train_workspace_size(256, 64, 256, 8, 2, 4) == 0  # d % 128 != 0
+    assert moe.moe_layer_train_workspace_size(256, 128, 256, 8, 2, 3) == 0  # R does not divide E
+    ws = moe.moe_layer_train_workspace_size(256, 128, 256, 8, 2, 4)
+    assert ws > 256 * 2 * (2 * 256 + 256) * 2               # holds z and h of every row
+    assert moe.moe_expert_ffn_backward_workspace_size(1000, 1024) >= 1000 * 3 * 1024 * 2
+
+
 def test_movers_reject_bad_shapes():
     lib = moe.load()
     assert lib.moe_dispatch_gather(NULL, 16, 100, B.MOE_BF16, 2, 4, 2, NULL, NULL, NULL, NULL,
