@@ -17,6 +17,11 @@ to host memory inside the timed region.
 
 `--impl reference` times the CPU oracle (the plain reference implementation
 of the layer) on the host cores on a bounded sample of the same workload.
+
+`--train` measures the training step instead: moe_layer_forward_train then
+moe_layer_backward (gradients of x, of the logits and of every weight, fp32
+weight gradients), with the backward expert GEMMs (moe_expert_ffn_backward)
+timed on their own for the roofline.
 """
 from __future__ import annotations
 
@@ -38,6 +43,8 @@ import torch  # noqa: E402
 from expert_warp_top_b200 import inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (route+BRIM dispatch+grouped GEMM+combine)"
+TRAIN_METRIC = ("MoE-layer training tokens/s (forward + backward: route, BRIM dispatch, grouped "
+                "GEMMs, combine; input, logit and weight gradients)")
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
 # GEMM launches of one layer step, from one ncu capture (profiles/ffn_gemm_pair_olmoe.md),
@@ -208,6 +215,47 @@ def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
                       f"{total_t:.1f} s"}
 
 
+def cpu_baseline_train(cfg, budget_s: float = 12.0, inp=None):
+    """The oracle's training step on sub-batches of the workload: routing, BRIM
+    build, the dense layer and its backward (input, gate and every weight
+    gradient, shared experts included) on the first n tokens as a batch."""
+    import oracle
+    if inp is None:
+        inp = inputs.make_inputs(cfg, device="cpu", weights=True)
+
+    def bits(t):
+        t = t.contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    logits = inp["logits"].numpy()
+    x = bits(inp["x"])
+    wg, wu, wd = bits(inp["wg"]), bits(inp["wu"]), bits(inp["wd"])
+    shared = (bits(inp["sg"]), bits(inp["su"]), bits(inp["sd"])) if cfg.S else None
+    slot_of = np.arange(cfg.E, dtype=np.int32)
+    rng = np.random.default_rng(0)
+    total_n, total_t, n = 0, 0.0, 8
+    while total_t < budget_s and n <= cfg.T:
+        lg = np.ascontiguousarray(logits[:n])
+        xs = np.ascontiguousarray(x[:n])
+        dy = rng.standard_normal((n, cfg.d))
+        t0 = time.perf_counter()
+        idx, w = oracle.route(lg, cfg.k, cfg.renorm)
+        oracle.brim(idx, w, slot_of, cfg.E, cfg.R)
+        oracle.dense_layer(xs, idx, w, wg, wu, wd, shared=shared)
+        g = oracle.dense_layer_backward(xs, idx, w, wg, wu, wd, dy, shared=shared,
+                                        experts=np.arange(cfg.E), shared_grads=cfg.S > 0)
+        oracle.route_backward(lg, idx, g["dw"], cfg.renorm)
+        dt = time.perf_counter() - t0
+        total_t += dt
+        total_n += n
+        n *= 2
+    return {"value": total_n / total_t, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"sub-batches of the first 8, 16, ... tokens, {total_n} tokens in all "
+                      f"(route + BRIM + dense fp64 layer + its backward with every weight "
+                      f"gradient), {total_t:.1f} s"}
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -217,12 +265,13 @@ def run_reference(args, cfg):
     budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
     inp = inputs.make_inputs(cfg, device="cpu", weights=True)
     for i in range(args.warmup + args.steps):
-        res = cpu_baseline(cfg, budget_s=budget, inp=inp)
+        res = (cpu_baseline_train if args.train else cpu_baseline)(cfg, budget_s=budget, inp=inp)
         if i >= args.warmup:
             per_step.append(res)
     value = statistics.median([r["value"] for r in per_step])
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "impl": "reference", "metric": TRAIN_METRIC if args.train else METRIC, "value": value,
+        "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * cfg.T / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -414,6 +463,204 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
 
 
+def run_train(args, cfg):
+    """The training step: moe_layer_forward_train + moe_layer_backward (through
+    MoELayer.forward_train / backward), replayed from one CUDA graph; then the
+    backward expert GEMMs (moe_expert_ffn_backward) alone for the roofline."""
+    import torch.distributed as dist
+    from expert_warp_top_b200 import _binding as B
+    from expert_warp_top_b200.layer import MoELayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    inp = inputs.make_inputs(cfg, device=dev, seed=rank_seed(cfg, rank))
+    kw = dict(wg=inp.pop("wg"), wu=inp.pop("wu"), wd=inp.pop("wd"))
+    if cfg.S:
+        kw.update(sg=inp.pop("sg"), su=inp.pop("su"), sd=inp.pop("sd"))
+    layer = MoELayer(T=cfg.T, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k, R=cfg.R, renorm=cfg.renorm,
+                     dtype=inputs.torch_dtype(cfg), S=cfg.S, fs=cfg.fs, device=dev, **kw)
+    del kw
+    logits, x = inp["logits"], inp["x"]
+    g = torch.Generator(device=dev).manual_seed(rank_seed(cfg, rank) + 77)
+    dy = torch.randn(cfg.T, cfg.d, generator=g, device=dev).to(layer.dtype)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    grads = None
+
+    def step():
+        nonlocal grads
+        layer.forward_train(logits, x)
+        grads = layer.backward(dy, grads=grads)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(args.warmup):
+            step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    if B.moe_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # the backward expert GEMMs alone, on the same EPD rows
+    layer.route_brim(logits)
+    layer.dispatch(x)
+    tk, f, d = cfg.T * cfg.k, cfg.f, cfg.d
+    a = layer.x_epd if layer.x_epd is not None else layer.x_sfd
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    z = torch.empty(tk, 2 * f, **bf)
+    h = torch.empty(tk, f, **bf)
+    o = torch.empty(tk, d, **bf)
+    dy_sfd = torch.empty(layer.cap, d, **bf)
+    dy_epd = torch.empty(tk, d, **bf) if layer.x_epd is not None else None
+    B.moe_dispatch_gather(dy, cfg.k, cfg.R, cfg.L, layer.brim0, layer.brim1, dy_sfd, dy_epd)
+    dout = dy_epd if dy_epd is not None else dy_sfd
+    B.moe_expert_ffn_train(a, layer.epd_off, layer.w_gu, layer.w_dn, f, layer.epd_gate, z, h, o,
+                           m_cap=tk)
+    dxe = torch.empty(tk, d, **bf)
+    dgate = torch.empty(tk, dtype=torch.float32, device=dev)
+    dwg = torch.empty(cfg.E, 2 * f, d, dtype=torch.float32, device=dev)
+    dwd = torch.empty(cfg.E, d, f, dtype=torch.float32, device=dev)
+    bws = torch.empty(B.moe_expert_ffn_backward_workspace_size(tk, f), dtype=torch.uint8,
+                      device=dev)
+
+    def gemm_bwd():
+        B.moe_expert_ffn_backward(dout, a, z, layer.epd_off, layer.w_gu, layer.w_dn, f,
+                                  layer.epd_gate, dxe, dgate, dwg, dwd, bws, m_cap=tk)
+
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            gemm_bwd()
+    torch.cuda.synchronize(dev)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=side):
+        gemm_bwd()
+    torch.cuda.synchronize(dev)
+
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    step_ms, bwd_ms = [], []
+    with ClockSampler(local_rank) as clocks:
+        t_end = time.time() + 5.0
+        while clocks.n_samples() < 2 and time.time() < t_end:
+            for _ in range(5):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            s0.record(stream)
+            graph.replay()
+            s1.record(stream)
+            s1.synchronize()
+            step_ms.append(s0.elapsed_time(s1))
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            s0.record(stream)
+            g2.replay()
+            s1.record(stream)
+            s1.synchronize()
+            bwd_ms.append(s0.elapsed_time(s1))
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        t_end = time.time() + 2.0
+        n0 = clocks.n_samples()
+        while clocks.n_samples() < n0 + 2 and time.time() < t_end:
+            for _ in range(5):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+    if B.moe_get_device_status() != 0:
+        raise RuntimeError("device status after the timed steps")
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
+    ms_per_step = total_ms / args.steps
+    value = whole_job_tokens_per_s(cfg.T, args.steps, world, total_ms)
+
+    # end to end: the step's logits, x and dy from pinned host memory, dx and
+    # d_logits back to pinned host memory, every step (host wall clock)
+    h_logits = logits.cpu().pin_memory()
+    h_x = x.cpu().pin_memory()
+    h_dy = dy.cpu().pin_memory()
+    h_dx = torch.empty(cfg.T, cfg.d, dtype=layer.dtype).pin_memory()
+    h_dl = torch.empty(cfg.T, cfg.E, dtype=torch.float32).pin_memory()
+    d_logits, d_x, d_dy = torch.empty_like(logits), torch.empty_like(x), torch.empty_like(dy)
+
+    def e2e_step():
+        d_logits.copy_(h_logits, non_blocking=True)
+        d_x.copy_(h_x, non_blocking=True)
+        d_dy.copy_(h_dy, non_blocking=True)
+        layer.forward_train(d_logits, d_x)
+        gr = layer.backward(d_dy, grads=grads)
+        h_dx.copy_(gr["dx"], non_blocking=True)
+        h_dl.copy_(gr["d_logits"], non_blocking=True)
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3, dev)
+    e2e = {"value": whole_job_tokens_per_s(cfg.T, args.steps, world, e2e_ms), "unit": UNIT,
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (h_logits, h_x, h_dy)),
+           "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (h_dx, h_dl)),
+           "api": "MoELayer.forward_train + backward (moe_layer_forward_train / "
+                  "moe_layer_backward), pinned host copies in the step, wall clock"}
+
+    pk = peaks()
+    bwd_flops = 2.0 * 6 * d * f * tk          # 2 input-gradient + 2 weight-gradient GEMMs
+    step_flops = 2.0 * 9 * d * f * (tk + cfg.T * cfg.S * cfg.fs / max(f, 1))
+    bwd_s = statistics.mean(bwd_ms) * 1e-3
+    achieved = bwd_flops / bwd_s / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_sust"], "unit": "TFLOP/s",
+            "frac": achieved / pk["bf16_sust"], "peak_source": f"{pk['source']} bf16 sustained",
+            "kernel": "backward expert GEMMs (moe_expert_ffn_backward: 2 input-gradient GEMMs, "
+                      "the first with the SwiGLU/gate backward fused, 2 weight-gradient GEMMs "
+                      "with fp32 output, 1 gate-gradient row sum)",
+            "algorithmic_flops": bwd_flops, "traffic": None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_train(cfg)
+    if rank == 0:
+        n_launch = 14 + (7 if cfg.S else 0)
+        line = {
+            "metric": TRAIN_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} "
+                                   f"k={cfg.k} R={cfg.R} S={cfg.S} (training step)",
+                       "dw_dtype": "fp32", "placement": "contiguous",
+                       "l2": "flushed between steps (256 MiB write outside the per-step events)",
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": roof,
+            "step_flops": step_flops,
+            "step_tflops": step_flops / (ms_per_step * 1e-3) / 1e12,
+            "bwd_gemm_ms": statistics.mean(bwd_ms),
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks.summary(),
+            "gpu_launches": n_launch * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def placement(cfg, how, dev, logits):
     """slot_of for the run.  "histogram": correlated placement from the expert
     co-activation histogram of a separate calibration batch (T = 32768, seed 1),
@@ -483,6 +730,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--placement", default="contiguous", choices=["contiguous", "histogram"])
+    ap.add_argument("--train", action="store_true",
+                    help="time the training step (forward + backward) instead of the forward")
     ap.add_argument("--prune", type=int, default=0,
                     help="routing-score-based collaboration pruning: keep each token's first "
                          "PRUNE ranks (0 = off)")
@@ -491,6 +740,8 @@ def main():
     cfg = inputs.CONFIGS[args.config]
     if args.impl == "reference":
         run_reference(args, cfg)
+    elif args.train:
+        run_train(args, cfg)
     else:
         run_ours(args, cfg)
 

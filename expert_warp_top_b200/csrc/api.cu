@@ -122,6 +122,24 @@ int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint
   return MOE_OK;
 }
 
+int encode_strips(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                  uint32_t box_rows, uint32_t box_strips) {
+  EncodeTiledFn fn;
+  int rc = get_encode_fn(&fn);
+  if (rc) return rc;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_strips};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  MOE_REQUIRE(r == CUDA_SUCCESS, MOE_ERR_CUDA,
+              "cuTensorMapEncodeTiled failed (%d) for a [%llu x %llu] strip tensor", (int)r,
+              (unsigned long long)rows, (unsigned long long)cols);
+  return MOE_OK;
+}
+
 int check_common(int T, int E, int k, int R) {
   MOE_REQUIRE(T >= 0, MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
   MOE_REQUIRE(E >= 1 && E <= moe::kMaxE, MOE_ERR_UNSUPPORTED, "E must be in [1, 256] (got %d)", E);

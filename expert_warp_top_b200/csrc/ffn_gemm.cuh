@@ -275,8 +275,8 @@ __device__ __forceinline__ void group_tile_prefix(const int32_t* group_off, int 
 }
 
 // B_MN: B is stored MN-major -- B[g*K + k][n], n contiguous (a weight used
-// transposed, as in the input-gradient GEMMs) -- and is loaded as BN/64 boxes
-// of 64 columns x 64 K rows.
+// transposed, as in the input-gradient GEMMs) -- and tmap_b sees it as
+// 64-column strips {64, G*K, N/64}: one load brings BN/64 strips of 64 K rows.
 template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -435,10 +435,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               if (!GATHER)
                 tc::tma_load_2d(tc::smem_u32(sa), &tmap_a, fb, kb * Cfg::kBK, row0, pol_a);
               if (B_MN) {
-#pragma unroll
-                for (int j = 0; j < BN / 64; ++j)
-                  tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes + j * 8192), &tmap_b, fb,
-                                  n0 + j * 64, g * args.K + kb * Cfg::kBK, pol_b);
+                // strip map {column in strip, row, strip}: BN/64 strips in one load
+                tc::tma_load_3d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, 0,
+                                g * args.K + kb * Cfg::kBK, n0 / 64, pol_b);
               } else {
                 tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, kb * Cfg::kBK,
                                 g * args.N + n0, pol_b);

@@ -41,8 +41,8 @@ struct PairCfg {
                                        sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
 };
 
-// B_MN: B stored MN-major (B[g*K + k][n], n contiguous); each CTA loads its
-// BN/2 columns as 64-column boxes.
+// B_MN: B stored MN-major (B[g*K + k][n], n contiguous), seen by tmap_b as
+// 64-column strips; each CTA loads its BN/2 columns in one 3-D load.
 template <int BN, int EPI, bool TF32, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -158,11 +158,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc::tma_load_2d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, kb * Cfg::kBK,
                                  row0 + (int)rank * 128, pol_a);
             if (B_MN) {
-#pragma unroll
-              for (int j = 0; j < BN / 128; ++j)
-                tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes + j * 8192), &tmap_b, fb_pair,
-                                     n0 + (int)rank * (BN / 2) + j * 64, g * args.K + kb * Cfg::kBK,
-                                     pol_b);
+              // strip map {column in strip, row, strip}: this CTA's BN/128 strips
+              tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0,
+                                   g * args.K + kb * Cfg::kBK, (n0 + (int)rank * (BN / 2)) / 64,
+                                   pol_b);
             } else {
               tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
                                    kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);

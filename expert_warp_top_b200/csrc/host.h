@@ -9,6 +9,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -72,6 +73,15 @@ constexpr int kDebugForcePair = 4;    // GEMMs on CTA pairs where the shape allo
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
               uint32_t box_cols, uint32_t box_rows);
 
+// The same [rows, cols] tensor seen as 64-column strips: a 3-D map with dims
+// {64, rows, cols / 64} and strides {row pitch, 128 bytes}, box
+// {64, box_rows, box_strips}, 128-byte swizzle.  One load brings box_strips
+// strips of box_rows rows, strip after strip (each box_rows x 128 bytes): the
+// layout of an MN-major operand tile, in one instruction instead of one per
+// strip.  bf16 only; cols % 64 == 0.
+int encode_strips(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                  uint32_t box_rows, uint32_t box_strips);
+
 int check_common(int T, int E, int k, int R);
 int check_dtype(int dtype);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -122,13 +132,13 @@ inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
   return a;
 }
 
-// B's tensor map: K-major [G*N, K] with box [BN_box rows, 64 cols], or
-// MN-major [G*K, N] with box [64 K rows, 64 cols].
+// B's tensor map: K-major [G*N, K] with box [box_n rows, 64 cols], or
+// MN-major [G*K, N] as 64-column strips with box [64 K rows, box_n / 64 strips].
 template <bool B_MN>
 int encode_b(CUtensorMap* tb, const void* b, int dtype, int G, int N, int K, int bk,
-             uint32_t box_rows_kmajor) {
-  if (B_MN) return encode_2d(tb, b, dtype, (uint64_t)N, (uint64_t)G * K, 64, 64);
-  return encode_2d(tb, b, dtype, (uint64_t)K, (uint64_t)G * N, bk, box_rows_kmajor);
+             uint32_t box_n) {
+  if (B_MN) return encode_strips(tb, b, (uint64_t)N, (uint64_t)G * K, 64, box_n / 64);
+  return encode_2d(tb, b, dtype, (uint64_t)K, (uint64_t)G * N, bk, box_n);
 }
 
 // A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
@@ -260,16 +270,23 @@ int launch_wgrad_bn(DeviceInfo* di, const void* a, const void* b, int rows, int 
                     const int32_t* group_off, int G, void* out, int accumulate, cudaStream_t st) {
   using Cfg = moe::WgradCfg<BN>;
   CUtensorMap ta, tb;
-  int rc = encode_2d(&ta, a, MOE_BF16, (uint64_t)M, (uint64_t)rows, 64, 64);
+  int rc = encode_strips(&ta, a, (uint64_t)M, (uint64_t)rows, 64, 2);
   if (rc) return rc;
-  if ((rc = encode_2d(&tb, b, MOE_BF16, (uint64_t)N, (uint64_t)rows, 64, 64))) return rc;
+  if ((rc = encode_strips(&tb, b, (uint64_t)N, (uint64_t)rows, 64, BN / 64))) return rc;
+  // the output [G*M, N]: boxes of 32 rows x 128 bytes for the epilogue's TMA stores
+  constexpr bool kF32 = std::is_same<TOut, float>::value;
+  CUtensorMap to;
+  if ((rc = encode_2d(&to, out, kF32 ? MOE_F32 : MOE_BF16, (uint64_t)N, (uint64_t)G * M,
+                      kF32 ? 32 : 64, 32)))
+    return rc;
   auto kern = moe::wgrad_gemm_kernel<BN, TOut>;
   if ((rc = ensure_smem(di, reinterpret_cast<const void*>(kern), Cfg::kSmemBytes))) return rc;
   const long long tiles = (long long)G * (M / 128) * (N / BN);
   const int grid = (int)(tiles < di->num_sms ? (tiles < 1 ? 1 : tiles) : di->num_sms);
   moe::WgradArgs args{group_off, G, M, N, rows, out, accumulate, di->err_flag, wait_limit_ns(),
                       g_debug_flags};
-  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, args));
+  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, to,
+                    args));
   MOE_LAUNCHED("wgrad_gemm_kernel");
   return MOE_OK;
 }

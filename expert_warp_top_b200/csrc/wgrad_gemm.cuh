@@ -8,16 +8,22 @@
 // GEMM: dW_down[g] = dO_g^T (w h)_g and dW_gate/up[g] = dZ_g^T X_g.
 //
 // Kernel shape (one persistent CTA per SM, 192 threads), as the forward GEMM:
-//   warp 0      TMA producer: per stage 64 rows of A (two boxes of 64 columns)
-//               and of B (BN/64 boxes), 128-byte swizzle
+//   warp 0      TMA producer: per stage 64 rows of A (128 columns) and of B (BN
+//               columns), each one 3-D load of 64-column strips (the tensor
+//               seen as {64, rows, cols/64}), 128-byte swizzle
 //   warp 1      MMA issuer (lane 0) and tail fixer (whole warp): in a group's
 //               last, partial row block the rows past the group's end belong
 //               to the next group, so the warp zeroes them in shared memory
 //               (a 128-byte row of a swizzled box holds exactly one row)
 //               before the MMAs read the stage
-//   warps 2..5  epilogue: tcgen05.ld of 32 accumulator rows (= 32 values of m)
-//               and a store of BN columns per row (fp32 or bf16, optionally
-//               added to what the output holds)
+//   warps 2..5  epilogue: tcgen05.ld of 32 accumulator rows (= 32 values of m),
+//               staged 128 bytes per row (32 fp32 or 64 bf16 columns) into one
+//               of two 128-byte-swizzled shared-memory boxes of this warp
+//               (double-buffered against the store in flight), then written
+//               by one TMA tensor store (or TMA reduce-add when accumulating
+//               fp32): whole 128-byte lines reach L2 instead of 16-byte pieces
+//               of 32 rows.  bf16 accumulation reads and rewrites the rows
+//               with plain loads and stores.
 // Tiles: group by group, M block, N block fastest.  A group without rows
 // writes zeros (or leaves the output as it is when accumulating).  Every wait
 // is bounded, as in the forward kernel.
@@ -46,14 +52,20 @@ struct WgradCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256 +
-                                       sizeof(int32_t) * (2 * kGemmMaxGroups + 2);
+  static constexpr int kStoreBoxBytes = 32 * 128;  // one staging box: 32 rows x 128 bytes
+  static constexpr int kStoreBoxes = 8;             // two per epilogue warp
+  static constexpr size_t kSmemBytes =
+      1024 + (size_t)kStages * kStageBytes + kStoreBoxes * kStoreBoxBytes + 256;
 };
 
+// tmap_a / tmap_b: A and B as 64-column strips (encode_strips), boxes of 64
+// rows x 2 strips (A) and 64 rows x BN/64 strips (B).  tmap_out: the output as
+// a 2-D [G*M, N] tensor of TOut, box of 32 rows x 128 bytes, 128-byte swizzle.
 template <int BN, typename TOut>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     wgrad_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                      const __grid_constant__ CUtensorMap tmap_b, const WgradArgs args) {
+                      const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_out, const WgradArgs args) {
   static_assert(BN == 64 || BN == 128 || BN == 256, "BN must be 64, 128 or 256");
   using Cfg = WgradCfg<BN>;
   constexpr int S = Cfg::kStages;
@@ -63,7 +75,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * Cfg::kStageBytes);
+  uint8_t* store_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 8 x 4 KB, 1024-aligned
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(store_boxes + Cfg::kStoreBoxes * Cfg::kStoreBoxBytes);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + S;
   uint64_t* tfull_bar = bars + 2 * S;
@@ -71,8 +85,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = bars + 2 * S + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_off = reinterpret_cast<int32_t*>(smem + (size_t)S * Cfg::kStageBytes + 256);
-  int32_t* s_end = s_off + kGemmMaxGroups + 1;
 
   const int warp = threadIdx.x >> 5;
   const unsigned lane = lane_id();
@@ -84,6 +96,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tmap_a);
     tc::tma_prefetch_desc(&tmap_b);
+    tc::tma_prefetch_desc(&tmap_out);
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
       tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
@@ -101,18 +114,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tmem_relinquish();
   }
   pdl_enter();
-  if (warp == 2) {
-    // group bounds; a group that leaves [0, rows] or runs backwards is empty
-    // and raises the index error bit
+  if (warp == 2 && blockIdx.x == 0) {
+    // a group that leaves [0, rows] or runs backwards is treated as empty
+    // (see group_rows) and raises the index error bit
     bool bad = false;
     for (int g = (int)lane; g < G; g += 32) {
       const int lo = args.group_off[g], hi = args.group_off[g + 1];
-      const bool ok = lo >= 0 && hi >= lo && hi <= args.rows;
-      bad |= !ok;
-      s_off[g] = ok ? lo : 0;
-      s_end[g] = ok ? hi : 0;
+      bad |= !(lo >= 0 && hi >= lo && hi <= args.rows);
     }
-    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_error(args.err, kErrIndex);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(args.err, kErrIndex);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -127,6 +137,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     m0 = mb * 128;
     n0 = (r - mb * n_blocks) * BN;
   };
+  // rows [r0, r1) of group g (empty if its bounds are invalid)
+  auto group_rows = [&](int g, int& r0, int& r1) {
+    const int lo = __ldg(args.group_off + g), hi = __ldg(args.group_off + g + 1);
+    const bool ok = lo >= 0 && hi >= lo && hi <= args.rows;
+    r0 = ok ? lo : 0;
+    r1 = ok ? hi : 0;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -138,9 +155,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool skip_next = (args.debug & kDebugSkipFirstLoad) != 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        int g, m0, n0;
+        int g, m0, n0, r0, r1;
         locate(tile, g, m0, n0);
-        const int r0 = s_off[g], r1 = s_end[g];
+        group_rows(g, r0, r1);
         const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl)) {
@@ -152,13 +169,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
             const int y = r0 + kb * Cfg::kBK;
             tc::mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-              tc::tma_load_2d(tc::smem_u32(sa + j * 8192), &tmap_a, fb, m0 + j * 64, y, pol);
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tc::tma_load_2d(tc::smem_u32(sa + Cfg::kABytes + j * 8192), &tmap_b, fb,
-                              n0 + j * 64, y, pol);
+            // strip maps: {column in strip, row, strip}; one load per operand
+            tc::tma_load_3d(tc::smem_u32(sa), &tmap_a, fb, 0, y, m0 / 64, pol);
+            tc::tma_load_3d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb, 0, y, n0 / 64, pol);
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
@@ -182,9 +195,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-      int g, m0, n0;
+      int g, m0, n0, r0, r1;
       locate(tile, g, m0, n0);
-      const int r0 = s_off[g], r1 = s_end[g];
+      group_rows(g, r0, r1);
       const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
       bool go = true;
       if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl);
@@ -246,11 +259,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
+    constexpr int VN = Vec16<TOut>::n;             // values per 16-byte piece
+    constexpr int kCols = 8 * VN;                  // columns per 128-byte row of a box
+    // TMA path: plain store, or reduce-add for fp32 accumulation
+    const bool tma_path = std::is_same<TOut, float>::value || !args.accumulate;
+    uint8_t* my_boxes = store_boxes + quarter * 2 * Cfg::kStoreBoxBytes;  // this warp's two
+    int n_stores = 0;
     TOut* out = reinterpret_cast<TOut*>(args.out);
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      int g, m0, n0;
+      int g, m0, n0, r0, r1;
       locate(tile, g, m0, n0);
-      const bool has_rows = s_end[g] > s_off[g];
+      group_rows(g, r0, r1);
+      const bool has_rows = r1 > r0;
       bool ok = true;
       if (lane == 0) ok = tc::wait_bounded(tc::smem_u32(&tfull_bar[acc]), acc_phase, wctl);
       ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -259,35 +279,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc::fence_after_sync();
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const size_t m = (size_t)m0 + quarter * 32 + lane;
-      TOut* dst = out + ((size_t)g * args.M + m) * args.N + n0;
+      const int row0 = g * args.M + m0 + quarter * 32;  // first output row of this warp
       if (has_rows || !args.accumulate) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          if (has_rows) {
-            uint32_t vr[32];
-            tc::tmem_ld32(taddr + c * 32, vr);
-            tc::tmem_ld_wait();
+        for (int c = 0; c < BN / kCols; ++c) {
+          float v[kCols];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]);
-          } else {
+          for (int h = 0; h < kCols / 32; ++h) {
+            if (has_rows) {
+              uint32_t vr[32];
+              tc::tmem_ld32(taddr + c * kCols + h * 32, vr);
+              tc::tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+              for (int i = 0; i < 32; ++i) v[h * 32 + i] = __uint_as_float(vr[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[h * 32 + i] = 0.f;
+            }
           }
-          TOut* p = dst + c * 32;
-          constexpr int VN = Vec16<TOut>::n;
-          if (args.accumulate) {
+          if (tma_path) {
+            // boxes alternate; the store issued two boxes ago (same box) must
+            // have read it before it is rewritten: at most one store pending
+            uint8_t* box = my_boxes + (n_stores & 1) * Cfg::kStoreBoxBytes;
+            const uint32_t box_u = tc::smem_u32(box);
+            if (lane == 0) tc::bulk_wait_read_1();
+            __syncwarp();
+            // row `lane` of the box: 8 pieces of 16 bytes, piece j at slot j ^ (row & 7)
 #pragma unroll
-            for (int q = 0; q < 32 / VN; ++q) {
+            for (int j = 0; j < 8; ++j)
+              st_v4(box + lane * 128 + ((j ^ (lane & 7)) << 4), Vec16<TOut>::from_f32(v + j * VN));
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (args.accumulate) tc::tma_reduce_add_2d(&tmap_out, box_u, n0 + c * kCols, row0);
+              else tc::tma_store_2d(&tmap_out, box_u, n0 + c * kCols, row0);
+              tc::bulk_commit_group();
+            }
+            ++n_stores;
+          } else {
+            // bf16 accumulation: read, add, write this row's columns
+            TOut* p = out + ((size_t)row0 + lane) * args.N + n0 + c * kCols;
+#pragma unroll
+            for (int q = 0; q < kCols / VN; ++q) {
               float old[VN];
               Vec16<TOut>::to_f32(ld_v4(p + q * VN), old);
 #pragma unroll
               for (int i = 0; i < VN; ++i) v[q * VN + i] += old[i];
+              st_v4(p + q * VN, Vec16<TOut>::from_f32(v + q * VN));
             }
           }
-#pragma unroll
-          for (int q = 0; q < 32 / VN; ++q) st_v4(p + q * VN, Vec16<TOut>::from_f32(v + q * VN));
         }
       }
       tc::fence_before_sync();
@@ -298,6 +338,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    // every store issued by this warp has completed before the CTA exits
+    if (lane == 0) tc::bulk_wait_all();
+    __syncwarp();
   }
 
   tc::fence_before_sync();
