@@ -67,6 +67,10 @@ constexpr bool kRasterNFastest = MOE_RASTER_N_FASTEST != 0;
 #endif
 constexpr bool kWeightsEvictLast = MOE_WEIGHTS_EVICT_LAST != 0;
 
+// Shared-memory staging of one epilogue warp: a box of 32 rows x 128 bytes in
+// the 128-byte swizzle, written out by a TMA tensor store.
+constexpr int kEpiBoxBytes = 32 * 128;
+
 template <int BN, bool TF32>
 struct GemmCfg {
   static constexpr int kElemBytes = TF32 ? 4 : 2;
@@ -79,7 +83,8 @@ struct GemmCfg {
   static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
   static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;  // a power of two here
   static constexpr size_t kSmemBytes =
-      1024 /* alignment slack */ + (size_t)kStages * kStageBytes + 256 /* barriers */ +
+      1024 /* alignment slack */ + (size_t)kStages * kStageBytes +
+      4 * kEpiBoxBytes /* epilogue staging */ + 256 /* barriers */ +
       sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
 };
 
@@ -105,20 +110,54 @@ struct GemmArgs {
   int n_part = 0;
 };
 
-// Epilogue of one accumulator tile for this thread's TMEM lane (= one tile
-// row): tcgen05.ld 32 columns at a time, fused SwiGLU or row scaling, and a
-// masked store of the row.  Every lane of the warp must call it (tcgen05.ld is
-// warp-collective); `valid` masks the stores.
 __device__ __forceinline__ float round_bf16(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
 }
 
+// Writes 64 bf16 values of this thread's row at column `col` of `out`.  When
+// the warp's 32 rows are all inside the group (`full`), the rows go through
+// the warp's box and one TMA store (whole 128-byte lines); otherwise each
+// valid row is stored directly, so that no row past the group's end is
+// touched.  Warp-collective.
+__device__ __forceinline__ void store_row64_bf16(const float* v, bool valid, bool full,
+                                                 size_t grow, int wrow0, int col,
+                                                 __nv_bfloat16* out, int ldo, uint8_t* box,
+                                                 const CUtensorMap* tmap_out) {
+  const unsigned lane = lane_id();
+  if (full) {
+    if (lane == 0) tc::bulk_wait_read_all();  // the box's previous store has read it
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      st_v4(box + lane * 128 + ((j ^ (lane & 7)) << 4), Vec16<__nv_bfloat16>::from_f32(v + j * 8));
+    tc::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tc::tma_store_2d(tmap_out, tc::smem_u32(box), col, wrow0);
+      tc::bulk_commit_group();
+    }
+  } else if (valid) {
+    __nv_bfloat16* dst = out + grow * ldo + col;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) st_v4(dst + j * 8, Vec16<__nv_bfloat16>::from_f32(v + j * 8));
+  }
+}
+
+// Epilogue of one accumulator tile for this thread's TMEM lane (= one tile
+// row): tcgen05.ld 32 columns at a time, fused SwiGLU or row scaling, and the
+// row's stores (bf16 SwiGLU / scale: through the warp's staging box and TMA
+// stores, see store_row64_bf16).  Every lane of the warp must call it
+// (tcgen05.ld is warp-collective); `valid` masks the stores.
 template <int BN, int EPI, typename TOut>
 __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t grow, int n0,
-                                              const GemmArgs& args) {
+                                              const GemmArgs& args, uint8_t* box,
+                                              const CUtensorMap* tmap_out) {
   TOut* out = reinterpret_cast<TOut*>(args.out);
   const int ldo = args.ldo;
   const float* row_scale = args.row_scale;
+  constexpr bool kBf16 = std::is_same<TOut, __nv_bfloat16>::value;
+  const bool full = __all_sync(0xffffffffu, valid);
+  const int wrow0 = __shfl_sync(0xffffffffu, (int)grow, 0);  // the warp's rows are consecutive
   if constexpr (EPI == kEpiSwiGLUSave) {
     static_assert(std::is_same<TOut, __nv_bfloat16>::value,
                   "the training epilogue is bf16 only");
@@ -193,8 +232,44 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
       }
     }
     if (valid && args.partial) args.partial[grow * args.n_part + n0 / BN] = dgp;
+  } else if constexpr (EPI == kEpiSwiGLU && kBf16) {
+    // columns [128p, 128p+64) are gate rows, [128p+64, 128p+128) the matching
+    // up rows: 64 h columns per p, one 128-byte row of bf16
+#pragma unroll 1
+    for (int p = 0; p < BN / 128; ++p) {
+      float hv[64];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t gr[32], ur[32];
+        tc::tmem_ld32(taddr + p * 128 + h * 32, gr);
+        tc::tmem_ld32(taddr + p * 128 + 64 + h * 32, ur);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float gv = __uint_as_float(gr[i]);
+          const float uv = __uint_as_float(ur[i]);
+          hv[h * 32 + i] = gv / (1.0f + __expf(-gv)) * uv;
+        }
+      }
+      store_row64_bf16(hv, valid, full, grow, wrow0, (n0 >> 1) + p * 64, out, ldo, box, tmap_out);
+    }
+  } else if constexpr (EPI == kEpiScale && kBf16) {
+    const float scale = (valid && row_scale) ? row_scale[grow] : 1.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 64; ++c) {
+      float v[64];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t vr[32];
+        tc::tmem_ld32(taddr + c * 64 + h * 32, vr);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[h * 32 + i] = __uint_as_float(vr[i]) * scale;
+      }
+      store_row64_bf16(v, valid, full, grow, wrow0, n0 + c * 64, out, ldo, box, tmap_out);
+    }
   } else if constexpr (EPI == kEpiSwiGLU) {
-    // columns [128p, 128p+64) are gate rows, [128p+64, 128p+128) the matching up rows
+    // (fp32 output) columns [128p, 128p+64) gate, [128p+64, 128p+128) up
 #pragma unroll 1
     for (int p = 0; p < BN / 128; ++p) {
 #pragma unroll 1
@@ -280,7 +355,8 @@ __device__ __forceinline__ void group_tile_prefix(const int32_t* group_off, int 
 template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
   using Cfg = GemmCfg<BN, TF32>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
@@ -291,7 +367,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * Cfg::kStageBytes);
+  uint8_t* epi_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 x 4 KB, 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_boxes + 4 * kEpiBoxBytes);
   uint64_t* full_bar = bars;            // [S]   TMA -> MMA
   uint64_t* empty_bar = bars + S;       // [S]   MMA -> TMA
   uint64_t* tfull_bar = bars + 2 * S;   // [2]   MMA -> epilogue
@@ -299,7 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = bars + 2 * S + 4;   // [1] MMA drain at teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_off = reinterpret_cast<int32_t*>(smem + (size_t)S * Cfg::kStageBytes + 256);
+  int32_t* s_off = reinterpret_cast<int32_t*>(epi_boxes + 4 * kEpiBoxBytes + 256);
   int32_t* s_end = s_off + kGemmMaxGroups;
   int32_t* s_prefix = s_end + kGemmMaxGroups;
 
@@ -538,7 +615,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool valid = r_in_tile < rows;
       const size_t grow = static_cast<size_t>(row0 + r_in_tile);
-      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args);
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args, epi_boxes + quarter * kEpiBoxBytes,
+                                   &tmap_out);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tc::smem_u32(&tempty_bar[acc]));
@@ -547,6 +625,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    // this warp's TMA stores have completed before the CTA exits
+    if (lane == 0) tc::bulk_wait_all();
+    __syncwarp();
   }
 
   tc::fence_before_sync();

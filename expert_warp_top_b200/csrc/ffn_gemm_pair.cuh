@@ -37,7 +37,8 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 512 +
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes +
+                                       4 * kEpiBoxBytes + 512 +
                                        sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
 };
 
@@ -46,7 +47,8 @@ struct PairCfg {
 template <int BN, int EPI, bool TF32, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                         const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+                         const __grid_constant__ CUtensorMap tmap_b,
+                         const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
   static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
   using Cfg = PairCfg<BN, TF32>;
@@ -57,7 +59,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)S * Cfg::kStageBytes);
+  uint8_t* epi_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 x 4 KB, 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_boxes + 4 * kEpiBoxBytes);
   uint64_t* full_bar = bars;                 // [S] CTA 0: both CTAs' TMA -> MMA
   uint64_t* empty_bar = bars + S;            // [S] MMA (multicast) -> producers
   uint64_t* tfull_bar = bars + 2 * S;        // [2] MMA (multicast) -> epilogues
@@ -65,7 +68,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = bars + 2 * S + 4;    // [1] MMA drain at teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_off = reinterpret_cast<int32_t*>(smem + (size_t)S * Cfg::kStageBytes + 512);
+  int32_t* s_off = reinterpret_cast<int32_t*>(epi_boxes + 4 * kEpiBoxBytes + 512);
   int32_t* s_end = s_off + kGemmMaxGroups;
   int32_t* s_prefix = s_end + kGemmMaxGroups;
 
@@ -251,7 +254,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              static_cast<uint32_t>(acc * BN);
       const int grow_i = row0 + (int)rank * 128 + r_in_half;
       const bool valid = grow_i < gend;
-      epilogue_rows<BN, EPI, TOut>(taddr, valid, static_cast<size_t>(grow_i), n0, args);
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, static_cast<size_t>(grow_i), n0, args,
+                                   epi_boxes + quarter * kEpiBoxBytes, &tmap_out);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) {
@@ -264,6 +268,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    // this warp's TMA stores have completed before the CTA exits
+    if (lane == 0) tc::bulk_wait_all();
+    __syncwarp();
   }
 
   // Both CTAs meet here only after their own work is done and the MMA issuer

@@ -141,6 +141,13 @@ int encode_b(CUtensorMap* tb, const void* b, int dtype, int G, int N, int K, int
   return encode_2d(tb, b, dtype, (uint64_t)K, (uint64_t)G * N, bk, box_n);
 }
 
+// The GEMM output [m_cap, ldo] for the epilogue's TMA stores: boxes of 32 rows
+// x 128 bytes, 128-byte swizzle.
+inline int encode_out(CUtensorMap* to, const void* out, int dtype, int m_cap, int ldo) {
+  return encode_2d(to, out, dtype, (uint64_t)ldo, (uint64_t)(m_cap > 0 ? m_cap : 1),
+                   dtype == MOE_BF16 ? 64 : 32, 32);
+}
+
 // A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
 // gathered from it (row p = a[a_row_index[p]]), else they are a's first m_cap.
 template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN>
@@ -155,13 +162,16 @@ int launch_gemm(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_
                      GATHER ? 1u : (uint32_t)moe::kGemmBM);
   if (rc) return rc;
   if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN))) return rc;
+  CUtensorMap to;
+  if ((rc = encode_out(&to, out, dtype, m_cap, ldo))) return rc;
   auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32, GATHER, B_MN>;
   if ((rc = ensure_smem(di, reinterpret_cast<const void*>(kern), Cfg::kSmemBytes))) return rc;
   const long long ub = ((long long)m_cap / moe::kGemmBM + G) * (N / BN);
   const int grid = (int)(ub < di->num_sms ? (ub < 1 ? 1 : ub) : di->num_sms);
   const moe::GemmArgs args =
       gemm_args(di, group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
-  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, args));
+  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, to,
+                    args));
   MOE_LAUNCHED("ffn_gemm_kernel");
   return MOE_OK;
 }
@@ -192,6 +202,8 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
   if (rc) return rc;
   if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN / 2))) return rc;
+  CUtensorMap to;
+  if ((rc = encode_out(&to, out, dtype, m_cap, ldo))) return rc;
   auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32, B_MN>;
   const void* key = reinterpret_cast<const void*>(kern);
   cudaLaunchConfig_t cfg = {};
@@ -227,7 +239,7 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   cfg.numAttrs = 2;
   const moe::GemmArgs args =
       gemm_args(di, group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
-  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, to, args));
   return MOE_OK;
 }
 
