@@ -176,9 +176,9 @@ def algorithmic_work(cfg, c_t: int, e_act: int):
 
 
 def launches_per_step(cfg) -> int:
-    # routing + BRIM masks + counter + histogram (one kernel), BRIM scatter 1, dispatch 1,
-    # experts 2 (+2 shared), combine 1
-    return 1 + 1 + 1 + 2 + (2 if cfg.S else 0) + 1
+    # routing + BRIM masks + counter (one kernel), BRIM column scan + histogram 1,
+    # BRIM scatter 1, dispatch 1, experts 2 (+2 shared), combine 1
+    return 1 + 1 + 1 + 1 + 2 + (2 if cfg.S else 0) + 1
 
 
 def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
@@ -637,7 +637,7 @@ def run_train(args, cfg):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_train(cfg)
     if rank == 0:
-        n_launch = 14 + (7 if cfg.S else 0)
+        n_launch = 15 + (7 if cfg.S else 0)
         line = {
             "metric": TRAIN_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

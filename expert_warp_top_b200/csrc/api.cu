@@ -205,14 +205,18 @@ int launch_brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int 
                        cudaStream_t stream) {
   const int n_tiles = (T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
   const int blocks = (n_tiles + 3) / 4;
+  const int ncol = R + E;
+  int32_t* totals = reinterpret_cast<int32_t*>(scratch) + (size_t)ncol * n_tiles;
   MOE_CUDA(launch_k(moe::brim_mask_kernel<KMAX>, blocks, 128, 0, stream, topk_idx, slot_of, T, k, E, R, n_tiles,
                                                           scratch, err));
   MOE_LAUNCHED("brim_mask_kernel");
-  MOE_CUDA(launch_k(moe::brim_scan_kernel, 1, 1024, 0, stream, scratch, n_tiles, E, R, sfd_off, epd_off, c_t));
-  MOE_LAUNCHED("brim_scan_kernel");
-  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KMAX>, blocks, 128, 0, stream, 
+  MOE_CUDA(launch_k(moe::brim_colscan_kernel<KMAX>, ncol, 1024, 0, stream, scratch, n_tiles, ncol,
+                    totals, topk_idx, T, k, E, static_cast<uint32_t*>(nullptr), 0, err));
+  MOE_LAUNCHED("brim_colscan_kernel");
+  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KMAX>, n_tiles, 32 * moe::kScatterWarps, 0, stream,
       topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, reinterpret_cast<const int32_t*>(scratch),
-      brim0, sfd_token, brim1, epd_sfd, epd_gate));
+      static_cast<const int32_t*>(totals), sfd_off, epd_off, c_t, brim0, sfd_token, brim1,
+      epd_sfd, epd_gate));
   MOE_LAUNCHED("brim_scatter_kernel");
   return MOE_OK;
 }
@@ -232,10 +236,19 @@ int brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int k, cons
 #undef MOE_BRIM_K
 }
 
-// Scratch entries (one 32-bit word per column per 32-token tile) of a BRIM build.
+// Scratch entries of a BRIM build: one 32-bit word per column per 32-token
+// tile (the masks, then the tiles' bases), then one total per column.
 size_t brim_scratch_entries(int T, int E, int R) {
   const size_t n_tiles = ((size_t)T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
-  return n_tiles * (size_t)(R + E);
+  return (n_tiles + 1) * (size_t)(R + E);
+}
+
+// Histogram blocks of the column-scan pass: a few thousand tokens each, so
+// that their shared-memory counts merge into few global atomics.
+int hist_blocks(int T, int* tokens_per_block) {
+  const int per = 2048;
+  *tokens_per_block = per;
+  return (T + per - 1) / per;
 }
 
 }  // namespace
@@ -384,7 +397,7 @@ int moe_prune_topk(int32_t* topk_idx, float* topk_w, int T, int k, const int32_t
 // ---------------------------------------------------------------------------
 size_t moe_route_brim_workspace_size(int T, int E, int R) {
   if (T < 0 || E < 1 || R < 1) return 0;
-  return align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)) + 512;
+  return align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)) + 256;
 }
 
 int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const int32_t* slot_of,
@@ -423,21 +436,24 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
               moe_route_brim_workspace_size(T, E, R));
   MOE_REQUIRE(aligned16(ws), MOE_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   uint32_t* masks = static_cast<uint32_t*>(ws);
-  unsigned* ticket = reinterpret_cast<unsigned*>(
-      static_cast<char*>(ws) + align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)));
-  MOE_CUDA(cudaMemsetAsync(ticket, 0, sizeof(unsigned), stream));
   const int n_tiles = (T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
+  const int ncol = R + E;
+  int32_t* totals = reinterpret_cast<int32_t*>(masks) + (size_t)ncol * n_tiles;
+  int hist_tokens = 0;
+  const int n_hist = hist ? hist_blocks(T, &hist_tokens) : 0;
   auto* tot = reinterpret_cast<unsigned long long*>(total);
   auto* rem = reinterpret_cast<unsigned long long*>(remote);
 #define MOE_ROUTE_BRIM(KM)                                                                    \
   MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM>, dim3(n_tiles), dim3(1024), 0, stream,    \
                     logits, T, E, k, renorm, slot_of, R, prune_m, n_tiles, topk_idx, topk_w,    \
-                    masks,                                                                      \
-                    sfd_off, epd_off, c_t, per_rank, tot, rem, hist, ticket, di->err_flag));    \
-  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3((n_tiles + 3) / 4), dim3(128), 0,      \
+                    masks, per_rank, tot, rem, di->err_flag));                                  \
+  MOE_CUDA(launch_k(moe::brim_colscan_kernel<KM>, dim3(ncol + n_hist), dim3(1024), 0, stream, \
+                    masks, n_tiles, ncol, totals, static_cast<const int32_t*>(topk_idx), T, k,  \
+                    E, hist, hist_tokens, di->err_flag));                                       \
+  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3(n_tiles), dim3(32 * moe::kScatterWarps), 0, \
                     stream, topk_idx, topk_w, slot_of, T, k, E, R, n_tiles,                     \
-                    reinterpret_cast<const int32_t*>(masks), brim0, sfd_token, brim1, epd_sfd,  \
-                    epd_gate))
+                    reinterpret_cast<const int32_t*>(masks), static_cast<const int32_t*>(totals), \
+                    sfd_off, epd_off, c_t, brim0, sfd_token, brim1, epd_sfd, epd_gate))
   if (k <= 2) {
     MOE_ROUTE_BRIM(2);
   } else if (k <= 4) {

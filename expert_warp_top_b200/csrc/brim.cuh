@@ -13,11 +13,13 @@
 // 32, one warp per tile and one lane per token.  A "column" is a rank (c < R)
 // or an expert slot (c = R + q).
 //   1. mask    : per tile and column, the 32-bit mask of lanes that hit it
-//   2. scan    : per column, exclusive scan of popcount(mask) over the tiles;
-//                column totals give sfd_off, epd_off and C_T; the masks are
-//                replaced in place by each tile's first global row
-//   3. scatter : each lane rebuilds its tile's masks and finds its row in
-//                column c as base[c][tile] + popcount(mask_c & lanes below it)
+//   2. scan    : one block per column: exclusive scan of popcount(mask) over
+//                the tiles, written in place (each tile's first row within
+//                the column), and the column's total
+//   3. scatter : each warp rebuilds its tile's masks, turns the column totals
+//                into column offsets (sfd_off, epd_off, C_T) and finds each
+//                lane's row in column c as offset[c] + base[c][tile] +
+//                popcount(mask_c & lanes below it)
 // No pass depends on the order in which atomics land.
 #pragma once
 #include "common.cuh"
@@ -209,81 +211,138 @@ __device__ __forceinline__ int warp_exclusive_scan_smem(const int32_t* in, int32
   return carry;
 }
 
-// ---- pass 2 ---------------------------------------------------------------
-// One block of 32 warps.  Each warp scans whole columns: lane i sums a
-// contiguous run of tiles, a warp scan orders the runs, each lane writes its
-// run's bases.  The mask words are replaced by the tile's first global row.
-// Reads go to L2 (ld.cg): the masks may have been written by other blocks of
-// the same grid.
-__device__ __forceinline__ void scan_columns(uint32_t* __restrict__ masks, int n_tiles, int E,
-                                             int R, int32_t* __restrict__ sfd_off,
-                                             int32_t* __restrict__ epd_off,
-                                             int32_t* __restrict__ c_t, int32_t* total,
-                                             int32_t* colbase) {
-  const int ncol = R + E;
-  const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const unsigned lane = lane_id();
-  const int run = (n_tiles + 31) / 32;  // tiles per lane
-  for (int c = warp; c < ncol; c += nwarps) {
-    uint32_t* col = masks + (size_t)c * n_tiles;
-    const int b0 = (int)lane * run;
-    const int b1 = min(b0 + run, n_tiles);
-    int sum = 0;
-#pragma unroll 8
-    for (int b = b0; b < b1; ++b) sum += __popc(__ldcg(col + b));
-    const int inc = warp_inclusive_scan(sum);
-    int base = inc - sum;
-    for (int b = b0; b < b1; ++b) {
-      const int n = __popc(__ldcg(col + b));
-      col[b] = (uint32_t)base;
-      base += n;
-    }
-    if (lane == 31) total[c] = inc;
+// ---- expert co-activation histogram --------------------------------------
+// Integer atomics, so the result does not depend on the order they land in.
+// Small E: a per-block histogram in shared memory flushed once per block.
+constexpr int kHistSmemE = 64;
+
+// Adds tokens [t0, t1) to the histogram, one thread per token.  With
+// E <= kHistSmemE the counts gather in shared memory `sh` first (cleared
+// here) and go to global memory once per nonzero cell.  All threads of the
+// block must call it.  A token with an out-of-range or repeated id raises the
+// index error bit and is skipped; -1 is an empty slot.
+template <int KMAX>
+__device__ __forceinline__ void coact_hist_range(const int32_t* __restrict__ topk_idx, int t0,
+                                                 int t1, int k, int E,
+                                                 uint32_t* __restrict__ hist, unsigned* err,
+                                                 uint32_t* sh) {
+  const bool use_smem = E <= kHistSmemE;
+  if (use_smem) {
+    for (int i = threadIdx.x; i < E * E; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
   }
-  __syncthreads();
-  // where each rank's SFD segment and each slot's EPD group starts
-  if (warp == 0) {
-    const int ct = warp_exclusive_scan_smem(total, colbase, R);
-    for (int r = lane; r < R; r += 32) sfd_off[r] = colbase[r];
-    if (lane == 0) {
-      sfd_off[R] = ct;
-      *c_t = ct;
+  for (int t = t0 + (int)threadIdx.x; t < t1; t += blockDim.x) {
+    int ids[KMAX];
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ids[j] = 0;
+      if (j < k) {
+        ids[j] = __ldg(topk_idx + (size_t)t * k + j);
+        if (ids[j] != -1 && (ids[j] < 0 || ids[j] >= E)) ok = false;
+#pragma unroll
+        for (int i = 0; i < j; ++i) ok &= ids[j] == -1 || ids[i] != ids[j];
+      }
     }
-  } else if (warp == 1) {
-    const int tk = warp_exclusive_scan_smem(total + R, colbase + R, E);
-    for (int q = lane; q < E; q += 32) epd_off[q] = colbase[R + q];
-    if (lane == 0) epd_off[E] = tk;
+    if (!ok) {
+      raise_error(err, kErrIndex);
+      continue;
+    }
+#pragma unroll
+    for (int a = 0; a < KMAX; ++a)
+#pragma unroll
+      for (int b = 0; b < KMAX; ++b)
+        if (a < k && b < k && ids[a] >= 0 && ids[b] >= 0) {
+          const int cell = ids[a] * E + ids[b];
+          if (use_smem) atomicAdd(&sh[cell], 1u);
+          else atomicAdd(&hist[cell], 1u);
+        }
   }
-  __syncthreads();
-  const int n_all = ncol * n_tiles;
-  for (int i = threadIdx.x; i < n_all; i += blockDim.x)
-    masks[i] = (uint32_t)((int32_t)masks[i] + colbase[i / n_tiles]);
+  if (use_smem) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < E * E; i += blockDim.x)
+      if (sh[i]) atomicAdd(&hist[i], sh[i]);
+  }
 }
 
-__global__ void __launch_bounds__(1024) brim_scan_kernel(uint32_t* __restrict__ masks,
-                                                        int n_tiles, int E, int R,
-                                                        int32_t* __restrict__ sfd_off,
-                                                        int32_t* __restrict__ epd_off,
-                                                        int32_t* __restrict__ c_t) {
+// ---- pass 2, parallel ------------------------------------------------------
+// Block c < ncol scans column c on its own: the popcounts of its n_tiles
+// masks, exclusive prefix over the tiles, written back in place (the tile's
+// first row WITHIN the column) and the column total into totals[c].  The
+// scatter (pass 3) adds each column's offset among the columns of its kind.
+// Blocks ncol .. ncol + n_hist - 1, when hist is given, add consecutive token
+// ranges of topk_idx to the co-activation histogram meanwhile.
+template <int KMAX>
+__global__ void __launch_bounds__(1024) brim_colscan_kernel(
+    uint32_t* __restrict__ masks, int n_tiles, int ncol, int32_t* __restrict__ totals,
+    const int32_t* __restrict__ topk_idx, int T, int k, int E, uint32_t* __restrict__ hist,
+    int hist_tokens, unsigned* err) {
   pdl_enter();
-  __shared__ int32_t total[kMaxCols];
-  __shared__ int32_t colbase[kMaxCols];
-  scan_columns(masks, n_tiles, E, R, sfd_off, epd_off, c_t, total, colbase);
+  __shared__ uint32_t sh[kHistSmemE * kHistSmemE];
+  int32_t* warp_sums = reinterpret_cast<int32_t*>(sh);  // the scan needs 32 of them
+  if ((int)blockIdx.x >= ncol) {
+    const int t0 = ((int)blockIdx.x - ncol) * hist_tokens;
+    coact_hist_range<KMAX>(topk_idx, t0, min(T, t0 + hist_tokens), k, E, hist, err, sh);
+    return;
+  }
+  const int c = blockIdx.x;
+  uint32_t* col = masks + (size_t)c * n_tiles;
+  const int per = (n_tiles + blockDim.x - 1) / blockDim.x;  // tiles per thread
+  const int b0 = threadIdx.x * per, b1 = min(b0 + per, n_tiles);
+  int sum = 0;
+  for (int b = b0; b < b1; ++b) sum += __popc(col[b]);
+  // block-wide exclusive scan of the per-thread sums
+  const int warp = threadIdx.x >> 5, lane = (int)lane_id();
+  const int inc = warp_inclusive_scan(sum);
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    const int v = lane < nw ? warp_sums[lane] : 0;
+    const int winc = warp_inclusive_scan(v);
+    if (lane < nw) warp_sums[lane] = winc - v;
+    if (lane == nw - 1) totals[c] = winc;
+  }
+  __syncthreads();
+  int base = warp_sums[warp] + inc - sum;
+  for (int b = b0; b < b1; ++b) {
+    const int n = __popc(col[b]);
+    col[b] = (uint32_t)base;
+    base += n;
+  }
 }
 
 // ---- pass 3 ---------------------------------------------------------------
+// One block of kScatterWarps warps per tile.  Warp 0 rebuilds the tile's
+// masks and the tile's first row in every column; then warp w walks the
+// ranks r = w, w + kScatterWarps, ... and, inside each, the rank's local
+// experts l, so that for one column the lanes that hit it hold consecutive
+// rows: every store of a warp lands on consecutive addresses.
+//   BRIM_0[r][t] = s (or -1), sfd_token[s] = t
+//   BRIM_1[l][s] = p (or -1 for a local expert the token did not pick), for
+//                  all l of each rank the token reaches
+//   epd_sfd[p] = s, epd_gate[p] = the token's gate weight for that expert
+//
+// With `totals` (pass 2), tile_base holds rows within each column; warp 0
+// adds the column offsets -- the exclusive scans of the column totals over
+// the R rank columns and over the E slot columns -- and tile 0 writes
+// sfd_off, epd_off and C_T.
+constexpr int kScatterWarps = 4;
+
 template <int KMAX>
-__global__ void __launch_bounds__(128) brim_scatter_kernel(
+__global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
     const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
     const int32_t* __restrict__ slot_of, int T, int k, int E, int R, int n_tiles,
-    const int32_t* __restrict__ tile_base, int32_t* __restrict__ brim0,
-    int32_t* __restrict__ sfd_token, int32_t* __restrict__ brim1,
+    const int32_t* __restrict__ tile_base, const int32_t* __restrict__ totals,
+    int32_t* __restrict__ sfd_off, int32_t* __restrict__ epd_off, int32_t* __restrict__ c_t,
+    int32_t* __restrict__ brim0, int32_t* __restrict__ sfd_token, int32_t* __restrict__ brim1,
     int32_t* __restrict__ epd_sfd, float* __restrict__ epd_gate) {
   pdl_enter();
-  __shared__ uint32_t sm[4][kMaxCols];
-  const int w = threadIdx.x >> 5;
-  const int tile = blockIdx.x * 4 + w;
-  if (tile >= n_tiles) return;
+  __shared__ uint32_t sm[kMaxCols];
+  __shared__ int32_t sb[kMaxCols];
+  __shared__ int32_t s_tot[kMaxCols], s_off[kMaxCols];
+  const int tile = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
   const int ncol = R + E, L = E / R;
   const size_t cap = (size_t)T * (k < R ? k : R);
   const unsigned lane = lane_id();
@@ -291,43 +350,57 @@ __global__ void __launch_bounds__(128) brim_scatter_kernel(
   TokenRoute<KMAX> tr;
   // the error flag was raised by pass 1 already
   const bool active = t < T && load_token_route<KMAX>(topk_idx, slot_of, t, k, E, L, tr, nullptr);
-  tile_masks<KMAX>(sm[w], ncol, R, active, k, tr);
-  if (t >= T) return;
-  for (int r = 0; r < R; ++r) brim0[(size_t)r * T + t] = -1;
-  if (!active) return;
+  float gate[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    gate[j] = (active && j < k && tr.slot[j] >= 0) ? __ldg(topk_w + (size_t)t * k + j) : 0.f;
+  if (warp == 0) {
+    tile_masks<KMAX>(sm, ncol, R, active, k, tr);
+    // the tile's first global row in every column
+    if (totals) {
+      for (int c = lane; c < ncol; c += 32) s_tot[c] = totals[c];
+      __syncwarp();
+      const int ct = warp_exclusive_scan_smem(s_tot, s_off, R);
+      const int tk = warp_exclusive_scan_smem(s_tot + R, s_off + R, E);
+      __syncwarp();
+      for (int c = lane; c < ncol; c += 32) sb[c] = s_off[c] + tile_base[(size_t)c * n_tiles + tile];
+      if (tile == 0) {
+        for (int r = lane; r < R; r += 32) sfd_off[r] = s_off[r];
+        for (int q = lane; q < E; q += 32) epd_off[q] = s_off[R + q];
+        if (lane == 0) {
+          sfd_off[R] = ct;
+          epd_off[E] = tk;
+          *c_t = ct;
+        }
+      }
+    } else {
+      for (int c = lane; c < ncol; c += 32) sb[c] = tile_base[(size_t)c * n_tiles + tile];
+    }
+  }
+  __syncthreads();
   const uint32_t lt = (1u << lane) - 1u;
-  const int32_t* base = tile_base + tile;  // base[c] at base[c * n_tiles]
-  int s_of[KMAX];
+  for (int r = warp; r < R; r += kScatterWarps) {
+    const uint32_t mr = sm[r];
+    const int s = ((mr >> lane) & 1u) ? sb[r] + __popc(mr & lt) : -1;
+    if (t < T) brim0[(size_t)r * T + t] = s;
+    if (mr == 0u) continue;  // no token of the tile reaches rank r (warp-uniform)
+    if (s >= 0) sfd_token[s] = t;
+    for (int l = 0; l < L; ++l) {
+      const int q = r * L + l;
+      const uint32_t mq = sm[R + q];
+      int p = -1;
+      float g = 0.f;
+      if ((mq >> lane) & 1u) {
+        p = sb[R + q] + __popc(mq & lt);
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    s_of[j] = -1;
-    if (j < k && tr.first[j]) {
-      const int r = tr.rank[j];
-      s_of[j] = __ldg(base + (size_t)r * n_tiles) + __popc(sm[w][r] & lt);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    if (j < k && tr.first[j]) {
-      const int s = s_of[j];
-      brim0[(size_t)tr.rank[j] * T + t] = s;
-      sfd_token[s] = t;
-      // every local expert of this rank starts as "not selected" for row s
-      for (int l = 0; l < L; ++l) brim1[(size_t)l * cap + s] = -1;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    if (j < k && tr.slot[j] >= 0) {
-      const int q = tr.slot[j];
-      int s = -1;
-#pragma unroll
-      for (int i = 0; i <= j; ++i)
-        if (tr.first[i] && tr.rank[i] == tr.rank[j]) s = s_of[i];
-      const int p = __ldg(base + (size_t)(R + q) * n_tiles) + __popc(sm[w][R + q] & lt);
-      brim1[(size_t)(q - tr.rank[j] * L) * cap + s] = p;
-      epd_sfd[p] = s;
-      epd_gate[p] = __ldg(topk_w + (size_t)t * k + j);
+        for (int j = 0; j < KMAX; ++j)
+          if (j < k && tr.slot[j] == q) g = gate[j];
+      }
+      if (s >= 0) brim1[(size_t)l * cap + s] = p;
+      if (p >= 0) {
+        epd_sfd[p] = s;
+        epd_gate[p] = g;
+      }
     }
   }
 }
@@ -380,10 +453,6 @@ __global__ void __launch_bounds__(256) count_dispatched_kernel(
   }
 }
 
-// ---- expert co-activation histogram --------------------------------------
-// Integer atomics, so the result does not depend on the order they land in.
-// Small E: a per-block histogram in shared memory flushed once per block.
-constexpr int kHistSmemE = 64;
 template <int KMAX>
 __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restrict__ topk_idx,
                                                          int T, int k, int E,
@@ -391,44 +460,8 @@ __global__ void __launch_bounds__(256) coact_hist_kernel(const int32_t* __restri
                                                          unsigned* err) {
   pdl_enter();
   __shared__ uint32_t sh[kHistSmemE * kHistSmemE];
-  const bool use_smem = E <= kHistSmemE;
-  if (use_smem) {
-    for (int i = threadIdx.x; i < E * E; i += blockDim.x) sh[i] = 0u;
-    __syncthreads();
-  }
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < T) {
-    int ids[KMAX];
-    bool ok = true;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      ids[j] = 0;
-      if (j < k) {
-        ids[j] = __ldg(topk_idx + (size_t)t * k + j);
-        if (ids[j] != -1 && (ids[j] < 0 || ids[j] >= E)) ok = false;
-#pragma unroll
-        for (int i = 0; i < j; ++i) ok &= ids[j] == -1 || ids[i] != ids[j];
-      }
-    }
-    if (!ok) {
-      raise_error(err, kErrIndex);
-    } else {
-#pragma unroll
-      for (int a = 0; a < KMAX; ++a)
-#pragma unroll
-        for (int b = 0; b < KMAX; ++b)
-          if (a < k && b < k && ids[a] >= 0 && ids[b] >= 0) {
-            const int cell = ids[a] * E + ids[b];
-            if (use_smem) atomicAdd(&sh[cell], 1u);
-            else atomicAdd(&hist[cell], 1u);
-          }
-    }
-  }
-  if (use_smem) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < E * E; i += blockDim.x)
-      if (sh[i]) atomicAdd(&hist[i], sh[i]);
-  }
+  const int t0 = blockIdx.x * blockDim.x;
+  coact_hist_range<KMAX>(topk_idx, t0, min(T, t0 + (int)blockDim.x), k, E, hist, err, sh);
 }
 
 // ---- collaboration pruning, in place ----------------------------------------

@@ -1,14 +1,13 @@
-// route_brim.cuh -- routing, the BRIM passes 1-2, the dispatched-row counter
-// and the co-activation histogram in one kernel.
+// route_brim.cuh -- routing, the BRIM masks and the dispatched-row counter in
+// one kernel (pass 1 of the BRIM build fused with routing).
 //
-// The same computation as moe_route_topk + brim passes 1-2 (brim.cuh) +
-// moe_count_dispatched_rows + moe_coact_histogram, in one launch instead of
-// five: one block of 32 warps per 32-token tile.  Each warp routes one token
-// (route_token_warp, the very code of moe_route_topk); warp 0 then takes the
-// tile lane-per-token, builds its column masks, and adds the tile's
-// contributions to the counter and the histogram.  The last block to finish
-// (a ticket taken after a memory fence) runs the column scan, so pass 3 of the
-// BRIM build can follow directly.
+// The same computation as moe_route_topk + brim_mask_kernel +
+// moe_count_dispatched_rows: one block of 32 warps per 32-token tile.  Each
+// warp routes one token (route_token_warp, the very code of moe_route_topk);
+// warp 0 then takes the tile lane-per-token, prunes (when asked), writes the
+// top-k, builds the tile's column masks and adds the tile's contribution to
+// the counter.  The column scan with the histogram (brim_colscan_kernel) and
+// the scatter (brim_scatter_kernel) follow.
 #pragma once
 #include "brim.cuh"
 #include "route.cuh"
@@ -20,16 +19,13 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     const int32_t* __restrict__ slot_of, int R, int prune_m, int n_tiles,
     int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_w, uint32_t* __restrict__ masks, int32_t* __restrict__ sfd_off,
-    int32_t* __restrict__ epd_off, int32_t* __restrict__ c_t, int32_t* __restrict__ per_rank,
+    float* __restrict__ topk_w, uint32_t* __restrict__ masks, int32_t* __restrict__ per_rank,
     unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
-    uint32_t* __restrict__ hist, unsigned* __restrict__ ticket, unsigned* err) {
+    unsigned* err) {
   pdl_enter();
   __shared__ int s_ids[32][KMAX];
   __shared__ float s_gates[32][KMAX];
   __shared__ uint32_t s_mask[kMaxCols];
-  __shared__ int32_t s_scan_a[kMaxCols], s_scan_b[kMaxCols];
-  __shared__ bool s_last;
   const int warp = threadIdx.x >> 5;
   const unsigned lane = lane_id();
   const int tile = blockIdx.x;
@@ -48,7 +44,7 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
   }
   __syncthreads();
 
-  // 2. warp 0, one lane per token: masks, counter, histogram
+  // 2. warp 0, one lane per token: pruning, top-k out, masks, counter
   if (warp == 0) {
     const int t = tile * kBrimTileTokens + (int)lane;
     int ids[KMAX];
@@ -92,27 +88,6 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
         if (n_remote) atomicAdd(remote, (unsigned long long)n_remote);
       }
     }
-    if (hist && active) {
-#pragma unroll
-      for (int a = 0; a < KMAX; ++a)
-#pragma unroll
-        for (int b = 0; b < KMAX; ++b)
-          if (a < k && b < k && ids[a] >= 0 && ids[b] >= 0)
-            atomicAdd(&hist[ids[a] * E + ids[b]], 1u);
-    }
-  }
-
-  // 3. the last tile to finish scans the columns
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    scan_columns(masks, n_tiles, E, R, sfd_off, epd_off, c_t, s_scan_a, s_scan_b);
-    if (threadIdx.x == 0) *ticket = 0u;
   }
 }
 

@@ -166,7 +166,7 @@ int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
  * workspace to lend, so this entry point takes none.
  * Scratch: a fixed array of 1 MiB (262144 int32) in this library's device
  * memory, reserved on every GPU that loads the library until the process
- * exits.  A call needs ceil(T / 32) * (R + E) entries of it (T <= 116k tokens
+ * exits.  A call needs (ceil(T / 32) + 1) * (R + E) entries of it (T <= 116k tokens
  * at E = 64, R = 8); a larger call returns MOE_ERR_UNSUPPORTED and enqueues
  * nothing.  The passes overwrite
  * every scratch entry they read, so nothing has to be cleared between calls.

@@ -93,7 +93,7 @@ def test_noalloc_brim_build_matches_workspace_version_twice():
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     lib = moe.load()
     null = ctypes.c_void_p(0)
-    # ceil(T/32) * (R + E) > 262144 entries
+    # (ceil(T/32) + 1) * (R + E) > 262144 entries
     T, E, R = 32 * 5000, 64, 8
     rc = lib.moe_brim_build_noalloc(null, null, T, 6, ctypes.c_void_p(8), E, R, null, null,
                                     ctypes.c_void_p(8),
