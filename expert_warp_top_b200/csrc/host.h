@@ -17,6 +17,7 @@
 #include "ffn_gemm.cuh"
 #include "ffn_gemm_pair.cuh"
 #include "wgrad_gemm.cuh"
+#include "wgrad_pair.cuh"
 
 namespace moe_host {
 
@@ -303,9 +304,72 @@ int launch_wgrad_bn(DeviceInfo* di, const void* a, const void* b, int rows, int 
   return MOE_OK;
 }
 
+// The same on CTA pairs: 256 x BN output tiles (M % 256 == 0, N % BN == 0).
+template <int BN, typename TOut>
+int launch_wgrad_pair(DeviceInfo* di, const void* a, const void* b, int rows, int M, int N,
+                      const int32_t* group_off, int G, void* out, int accumulate,
+                      cudaStream_t st) {
+  using Cfg = moe::WgradPairCfg<BN>;
+  CUtensorMap ta, tb, to;
+  int rc = encode_strips(&ta, a, (uint64_t)M, (uint64_t)rows, 64, 2);
+  if (rc) return rc;
+  if ((rc = encode_strips(&tb, b, (uint64_t)N, (uint64_t)rows, 64, BN / 128))) return rc;
+  constexpr bool kF32 = std::is_same<TOut, float>::value;
+  if ((rc = encode_2d(&to, out, kF32 ? MOE_F32 : MOE_BF16, (uint64_t)N, (uint64_t)G * M,
+                      kF32 ? 32 : 64, 32)))
+    return rc;
+  auto kern = moe::wgrad_pair_kernel<BN, TOut>;
+  const void* key = reinterpret_cast<const void*>(kern);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
+  if ((rc = ensure_smem(di, key, Cfg::kSmemBytes))) return rc;
+  int max_clusters = 0;
+  {
+    std::lock_guard<std::mutex> lk(di->mu);
+    for (auto& pc : di->pair_clusters)
+      if (pc.first == key) max_clusters = pc.second;
+  }
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(2 * (di->num_sms / 2), 1, 1);
+    MOE_CUDA(cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg));
+    MOE_REQUIRE(max_clusters >= 1, MOE_ERR_UNSUPPORTED, "no CTA pair fits on this device");
+    std::lock_guard<std::mutex> lk(di->mu);
+    di->pair_clusters.emplace_back(key, max_clusters);
+  }
+  const long long tiles = (long long)G * (M / 256) * (N / BN);
+  const long long pairs = tiles < max_clusters ? (tiles < 1 ? 1 : tiles) : max_clusters;
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.numAttrs = 2;
+  moe::WgradArgs args{group_off, G, M, N, rows, out, accumulate, di->err_flag, wait_limit_ns(),
+                      g_debug_flags};
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, to, args));
+  return MOE_OK;
+}
+
 template <typename TOut>
 int launch_wgrad(DeviceInfo* di, const void* a, const void* b, int rows, int M, int N,
                  const int32_t* group_off, int G, void* out, int accumulate, cudaStream_t st) {
+  // The CTA-pair kernel moves a third less operand traffic per FLOP but
+  // measured slower on the OLMoE-shaped backward (650 vs 515 us): its
+  // per-stage hand-off between the two CTAs adds latency to a loop that is
+  // bound by load latency.  It is kept, tested, behind kDebugForcePair.
+  const bool pair = M % 256 == 0 && N % 128 == 0 && (g_debug_flags & kDebugForcePair);
+  if (pair) {
+    if (N % 256 == 0)
+      return launch_wgrad_pair<256, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);
+    return launch_wgrad_pair<128, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);
+  }
   const int bn = pick_bn(N);
   if (bn == 256)
     return launch_wgrad_bn<256, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);

@@ -32,6 +32,11 @@
 
 namespace moe {
 
+#ifndef MOE_WGRAD_GROUP_BATCH
+#define MOE_WGRAD_GROUP_BATCH 1
+#endif
+constexpr int kWgradGroupBatch = MOE_WGRAD_GROUP_BATCH;
+
 struct WgradArgs {
   const int32_t* group_off;  // [G+1] device
   int G;
@@ -130,9 +135,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const tc::WaitCtl wctl{abort_flag, args.err, args.wait_limit_ns};
 
+  // Tiles go group batch by group batch (kWgradGroupBatch groups each); inside
+  // a batch the groups alternate, so the CTAs running at one time spread over
+  // the batch's groups instead of all reading one group's rows.
   auto locate = [&](int tile, int& g, int& m0, int& n0) {
-    g = tile / tiles_per_group;
-    const int r = tile - g * tiles_per_group;
+    const int batch = tile / (kWgradGroupBatch * tiles_per_group);
+    const int g0 = batch * kWgradGroupBatch;
+    const int gb = min(kWgradGroupBatch, G - g0);
+    const int r0 = tile - g0 * tiles_per_group;
+    g = g0 + r0 % gb;
+    const int r = r0 / gb;
     const int mb = r / n_blocks;
     m0 = mb * 128;
     n0 = (r - mb * n_blocks) * BN;

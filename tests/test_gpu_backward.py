@@ -340,3 +340,51 @@ def test_layer_backward_full_size_sampled(cfg):
                        inp["logits"].numpy()[tokens], idx[tokens], g["dw_abs"],
                        cfg.renorm) <= GRAD_RTOL
     _check_weight_grads(layer, grads, g, experts, cfg)
+
+
+SKIP_FIRST_LOAD = 1
+
+
+@pytest.mark.parametrize("variant", [FORCE_SINGLE, 0], ids=["single", "pair"])
+def test_backward_bounded_wait_expires_and_context_survives(variant):
+    """A stage that is never loaded makes the backward GEMMs' waits expire:
+    MOE_ERR_TIMEOUT comes back through the device flag, and the next call on the
+    same context gives the correct gradients."""
+    sizes, d, f = [300, 0, 212], 256, 256
+    off, x, wg, wu, wd, scale, dout = _ffn_problem(sizes, d, f, seed=21)
+    G, rows = len(sizes), int(sum(sizes))
+    w_gu = torch.empty(G, 2 * f, d, dtype=torch.bfloat16, device=DEV)
+    w_dn = torch.empty(G, d, f, dtype=torch.bfloat16, device=DEV)
+    moe.moe_prepare_weights(wg.to(DEV), wu.to(DEV), wd.to(DEV), None, w_gu, w_dn)
+    z = torch.empty(rows, 2 * f, dtype=torch.bfloat16, device=DEV)
+    h = torch.empty(rows, f, dtype=torch.bfloat16, device=DEV)
+    out = torch.empty(rows, d, dtype=torch.bfloat16, device=DEV)
+    dx = torch.empty_like(out)
+    drs = torch.empty(rows, dtype=torch.float32, device=DEV)
+    dw_gu = torch.empty(G, 2 * f, d, device=DEV)
+    dw_dn = torch.empty(G, d, f, device=DEV)
+    ws = torch.empty(moe.moe_expert_ffn_backward_workspace_size(rows, f), dtype=torch.uint8,
+                     device=DEV)
+    offd, xd, sd, dyd = off.to(DEV), x.to(DEV), scale.to(DEV), dout.to(DEV)
+    moe.moe_expert_ffn_train(xd, offd, w_gu, w_dn, f, sd, z, h, out)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    try:
+        moe.moe_set_debug(SKIP_FIRST_LOAD | variant, 200.0)
+        moe.moe_expert_ffn_backward(dyd, xd, z, offd, w_gu, w_dn, f, sd, dx, drs, dw_gu, dw_dn, ws)
+        status = moe.moe_get_device_status()
+    finally:
+        moe.moe_set_debug(0, 4000.0)
+    assert status == moe.MOE_ERR_TIMEOUT
+    moe.moe_set_debug(variant, 4000.0)
+    try:
+        moe.moe_expert_ffn_backward(dyd, xd, z, offd, w_gu, w_dn, f, sd, dx, drs, dw_gu, dw_dn, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status() == moe.MOE_OK
+    finally:
+        moe.moe_set_debug(0, 4000.0)
+    _, g = _ffn_oracle(off, x, wg, wu, wd, scale, dout)
+    assert rowwise_rel_err(dx.float().cpu().numpy(), g["dx"]) <= GRAD_RTOL
+    dwg, _ = unpack_gate_up(dw_gu.cpu())
+    assert normwise_err(dwg[0].numpy(), g["dwg"][0]) <= GRAD_RTOL
+    assert normwise_err(dw_dn[2].cpu().numpy(), g["dwd"][2]) <= GRAD_RTOL
