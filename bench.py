@@ -175,10 +175,37 @@ def algorithmic_work(cfg, c_t: int, e_act: int):
     return flops_ffn, bytes_
 
 
+def gemm_launches(m_cap: int, G: int, N: int) -> int:
+    """Launches of one grouped GEMM: one (CTA pairs or single CTAs, the
+    library's own choice; the hybrid two-launch tiling is opt-in)."""
+    return 1
+
+
 def launches_per_step(cfg) -> int:
     # routing + BRIM masks + counter (one kernel), BRIM column scan + histogram 1,
-    # BRIM scatter 1, dispatch 1, experts 2 (+2 shared), combine 1
-    return 1 + 1 + 1 + 1 + 2 + (2 if cfg.S else 0) + 1
+    # BRIM scatter 1, dispatch 1, experts (2 GEMMs), shared experts (2 GEMMs), combine 1
+    tk = cfg.T * cfg.k
+    n = 1 + 1 + 1 + 1 + 1
+    n += gemm_launches(tk, cfg.E, 2 * cfg.f) + gemm_launches(tk, cfg.E, cfg.d)
+    if cfg.S:
+        F = cfg.S * cfg.fs
+        n += gemm_launches(cfg.T, 1, 2 * F) + gemm_launches(cfg.T, 1, cfg.d)
+    return n
+
+
+def train_launches_per_step(cfg) -> int:
+    """forward_train (index 3, dispatch, 2 GEMMs, combine) + backward (dispatch of dY,
+    2 input-gradient GEMMs, gate-gradient row sum, 2 weight-gradient GEMMs, combine,
+    routing backward), shared experts included."""
+    tk, f, d = cfg.T * cfg.k, cfg.f, cfg.d
+    g = lambda m, G, N: gemm_launches(m, G, N)  # noqa: E731
+    n = 3 + 1 + g(tk, cfg.E, 2 * f) + g(tk, cfg.E, d) + 1
+    n += 1 + g(tk, cfg.E, f) + g(tk, cfg.E, d) + 1 + 2 + 1 + 1
+    if cfg.S:
+        F = cfg.S * cfg.fs
+        n += 1 + g(cfg.T, 1, 2 * F) + g(cfg.T, 1, d)        # set_two + shared forward
+        n += g(cfg.T, 1, F) + g(cfg.T, 1, d) + 2            # shared backward
+    return n
 
 
 def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
@@ -637,7 +664,7 @@ def run_train(args, cfg):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_train(cfg)
     if rank == 0:
-        n_launch = 15 + (7 if cfg.S else 0)
+        n_launch = train_launches_per_step(cfg)
         line = {
             "metric": TRAIN_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -108,7 +108,29 @@ struct GemmArgs {
   int ld_aux = 0;
   float* partial = nullptr;      // gate-gradient partials [rows, n_part] (nullable)
   int n_part = 0;
+  int tile_mode = 0;             // kTilesAll / kTilesPairNoSmallTail / kTilesSmallTail
 };
+
+// Which rows of each group a launch covers, for mixing CTA-pair and single-CTA
+// tiles: a group of r rows has r / 256 full pair tiles and a tail of r % 256.
+//   kTilesAll              every row, in tiles of the kernel's own height
+//   kTilesPairNoSmallTail  pair tiles (256 rows): the full ones, and the tail
+//                          only when it is longer than 128 rows
+//   kTilesSmallTail        single-CTA tiles (128 rows): only a tail of 1..128
+//                          rows, which then needs half a pair tile's MMA work
+constexpr int kTilesAll = 0;
+constexpr int kTilesPairNoSmallTail = 1;
+constexpr int kTilesSmallTail = 2;
+
+__device__ __forceinline__ int group_m_blocks(int rows, int bm, int mode) {
+  if (mode == kTilesPairNoSmallTail) return rows / 256 + (rows % 256 > 128 ? 1 : 0);
+  if (mode == kTilesSmallTail) return (rows % 256 > 0 && rows % 256 <= 128) ? 1 : 0;
+  return (rows + bm - 1) / bm;
+}
+// First row of a group's first tile in the launch.
+__device__ __forceinline__ int group_first_row(int gstart, int rows, int mode) {
+  return mode == kTilesSmallTail ? gstart + (rows / 256) * 256 : gstart;
+}
 
 __device__ __forceinline__ float round_bf16(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
@@ -316,9 +338,10 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
 // Tile prefix of the groups (one warp): s_off/s_end hold each group's rows
 // (a group whose bounds leave [0, m_cap] or run backwards is treated as empty
 // and raises the index error bit); s_prefix[g] = first tile of group g, where
-// group g has ceil(rows / bm) * n_blocks tiles; s_prefix[G] = all tiles.
+// group g has group_m_blocks(rows, bm, mode) * n_blocks tiles; s_prefix[G] =
+// all tiles.
 __device__ __forceinline__ void group_tile_prefix(const int32_t* group_off, int G, int m_cap,
-                                                  int bm, int n_blocks, int32_t* s_off,
+                                                  int bm, int n_blocks, int mode, int32_t* s_off,
                                                   int32_t* s_end, int32_t* s_prefix,
                                                   unsigned* err) {
   const unsigned lane = lane_id();
@@ -334,7 +357,7 @@ __device__ __forceinline__ void group_tile_prefix(const int32_t* group_off, int 
       s_off[g] = lo;
       s_end[g] = ok ? hi : lo;
       const int rows = ok ? hi - lo : 0;
-      tiles_g = ((rows + bm - 1) / bm) * n_blocks;
+      tiles_g = group_m_blocks(rows, bm, mode) * n_blocks;
     }
     int inc = tiles_g;
 #pragma unroll
@@ -405,37 +428,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tmem_alloc(tc::smem_u32(tmem_slot), Cfg::kTmemCols);
     tc::tmem_relinquish();
   }
-  pdl_enter();  // predecessors' outputs (group offsets, A rows) are visible from here
-  if (warp == 2) {
-    // group offsets and the tile prefix: tiles of group g = m_blocks(g) * n_blocks.
-    // A group whose bounds leave [0, m_cap] or run backwards is treated as
-    // empty and raises the index error bit.
-    int carry = 0;
-    bool bad = false;
-    for (int g0 = 0; g0 < G; g0 += 32) {
-      const int g = g0 + (int)lane;
-      int tiles_g = 0;
-      if (g < G) {
-        const int lo = args.group_off[g], hi = args.group_off[g + 1];
-        const bool ok = lo >= 0 && hi >= lo && hi <= args.m_cap;
-        bad |= !ok;
-        s_off[g] = lo;
-        s_end[g] = ok ? hi : lo;
-        const int rows = ok ? hi - lo : 0;
-        tiles_g = ((rows + kGemmBM - 1) / kGemmBM) * n_blocks;
-      }
-      int inc = tiles_g;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, o);
-        if ((int)lane >= o) inc += y;
-      }
-      if (g < G) s_prefix[g] = carry + inc - tiles_g;
-      carry += __shfl_sync(0xffffffffu, inc, 31);
-    }
-    if (lane == 0) s_prefix[G] = carry;
-    if (__any_sync(0xffffffffu, bad) && lane == 0 && blockIdx.x == 0) raise_error(args.err, kErrIndex);
+  if (args.tile_mode == kTilesSmallTail) {
+    // The small-tail launch follows the pair launch of the same GEMM, whose
+    // CTAs all passed their own wait (the inputs are complete) before this
+    // launch could start; it works alongside the pair launch's last tiles and
+    // waits for that launch only before it exits (end of the kernel).
+    pdl_trigger();
+  } else {
+    pdl_enter();  // predecessors' outputs (group offsets, A rows) are visible from here
   }
+  if (warp == 2)
+    group_tile_prefix(args.group_off, G, args.m_cap, kGemmBM, n_blocks, args.tile_mode, s_off,
+                      s_end, s_prefix, args.err);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -454,7 +458,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     g = lo;
     const int local = tile - s_prefix[g];
     const int gstart = s_off[g], gend = s_end[g];
-    const int m_blocks = (gend - gstart + kGemmBM - 1) / kGemmBM;
+    const int m_blocks = group_m_blocks(gend - gstart, kGemmBM, args.tile_mode);
     int nb, mb;
     if (kRasterNFastest) {
       mb = local / n_blocks;
@@ -463,7 +467,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       nb = local / m_blocks;
       mb = local - nb * m_blocks;
     }
-    row0 = gstart + mb * kGemmBM;
+    row0 = group_first_row(gstart, gend - gstart, args.tile_mode) + mb * kGemmBM;
     rows = min(kGemmBM, gend - row0);
     n0 = nb * BN;
   };
@@ -637,6 +641,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }
+  // the small-tail launch completes only after the pair launch before it, so
+  // that the next kernel's wait covers both
+  if (args.tile_mode == kTilesSmallTail) pdl_wait();
 }
 
 }  // namespace moe

@@ -101,8 +101,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   pdl_enter();  // predecessors' outputs (group offsets, A rows) are visible from here
   if (warp == 2)
-    group_tile_prefix(args.group_off, G, args.m_cap, kPairBM, n_blocks, s_off, s_end, s_prefix,
-                      args.err);
+    group_tile_prefix(args.group_off, G, args.m_cap, kPairBM, n_blocks, args.tile_mode, s_off,
+                      s_end, s_prefix, args.err);
   tc::fence_before_sync();
   __syncwarp();
   tc::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int local = tile - s_prefix[g];
     const int gstart = s_off[g];
     gend = s_end[g];
-    const int m_blocks = (gend - gstart + kPairBM - 1) / kPairBM;
+    const int m_blocks = group_m_blocks(gend - gstart, kPairBM, args.tile_mode);
     int nb, mb;
     if (kRasterNFastest) {
       mb = local / n_blocks;

@@ -68,7 +68,8 @@ extern int g_debug_flags;
 extern double g_wait_limit_ms;
 inline uint64_t wait_limit_ns() { return static_cast<uint64_t>(g_wait_limit_ms * 1.0e6); }
 constexpr int kDebugForceSingle = 2;  // GEMMs on single CTAs
-constexpr int kDebugForcePair = 4;    // GEMMs on CTA pairs where the shape allows
+constexpr int kDebugForcePair = 4;    // GEMMs on CTA pairs only where the shape allows
+constexpr int kDebugForceHybrid = 8;  // pair tiles plus single-CTA small tails
 
 // 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
@@ -117,6 +118,7 @@ struct GemmExtra {
   int ld_aux = 0;
   float* partial = nullptr;
   int n_part = 0;
+  int tile_mode = 0;  // moe::kTilesAll / kTilesPairNoSmallTail / kTilesSmallTail
 };
 
 inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
@@ -130,6 +132,7 @@ inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
   a.ld_aux = ex.ld_aux;
   a.partial = ex.partial;
   a.n_part = ex.n_part;
+  a.tile_mode = ex.tile_mode;
   return a;
 }
 
@@ -245,7 +248,9 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
 }
 
 // GEMM over the groups, on CTA pairs when the groups are tall enough to fill
-// 256-row tiles (and the rows are read in place), else on single CTAs.
+// 256-row tiles (and the rows are read in place), else on single CTAs.  In
+// hybrid mode a group's tail of at most 128 rows goes to a second,
+// single-CTA launch (128-row tiles), which halves that tail's MMA work.
 #ifndef MOE_PAIR_MIN_ROWS
 #define MOE_PAIR_MIN_ROWS 192
 #endif
@@ -255,15 +260,32 @@ int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a
                      const float* row_scale, void* out, int ldo, cudaStream_t st,
                      const GemmExtra& ex = GemmExtra{}) {
   const bool tall = (long long)m_cap >= (long long)MOE_PAIR_MIN_ROWS * G;
-  bool pair = !a_row_index && N % 128 == 0 && tall;
+  const bool pair_ok = !a_row_index && N % 128 == 0;
+  bool pair = pair_ok && tall;
+  // Hybrid tiling (a group's tail of <= 128 rows on single-CTA tiles, in a
+  // second launch) cuts the OLMoE-shaped layer's padded MMA rows from 20% to
+  // 11% but measured no faster (482-485 vs 490 us for both GEMMs): it stays
+  // opt-in, tested, behind kDebugForceHybrid.
+  bool hybrid = false;
   if (g_debug_flags & kDebugForceSingle) pair = false;
-  if ((g_debug_flags & kDebugForcePair) && !a_row_index && N % 128 == 0) pair = true;
+  if ((g_debug_flags & kDebugForcePair) && pair_ok) pair = true;
+  if ((g_debug_flags & kDebugForceHybrid) && pair_ok) {
+    pair = true;
+    hybrid = true;
+  }
   if (pair) {
-    if (N % 256 == 0)
-      return launch_gemm_pair<256, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
-                                                    row_scale, out, ldo, ex, st);
-    return launch_gemm_pair<128, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
-                                                  row_scale, out, ldo, ex, st);
+    GemmExtra exp = ex;
+    exp.tile_mode = hybrid ? moe::kTilesPairNoSmallTail : moe::kTilesAll;
+    int rc = N % 256 == 0
+                 ? launch_gemm_pair<256, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N,
+                                                          group_off, row_scale, out, ldo, exp, st)
+                 : launch_gemm_pair<128, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N,
+                                                          group_off, row_scale, out, ldo, exp, st);
+    if (rc || !hybrid) return rc;
+    GemmExtra ext = ex;
+    ext.tile_mode = moe::kTilesSmallTail;
+    return launch_gemm_bn<EPI, TF32, false, B_MN>(di, pick_bn(N), a, a_rows, nullptr, m_cap, K, b,
+                                                  G, N, group_off, row_scale, out, ldo, ext, st);
   }
   const int bn = pick_bn(N);
   if constexpr (!B_MN) {

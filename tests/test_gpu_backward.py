@@ -32,7 +32,7 @@ from test_gpu_parity import make_layer
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 GRAD_RTOL = 2e-2
-FORCE_SINGLE, FORCE_PAIR = 2, 4
+FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID = 2, 4, 8
 
 
 def normwise_err(a, ref) -> float:
@@ -99,7 +99,8 @@ def _ffn_oracle(off, x, wg, wu, wd, scale, dout):
     return y, g
 
 
-@pytest.mark.parametrize("variant", [0, FORCE_SINGLE, FORCE_PAIR], ids=["auto", "single", "pair"])
+@pytest.mark.parametrize("variant", [0, FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID],
+                         ids=["auto", "single", "pair", "hybrid"])
 @pytest.mark.parametrize("dw_dtype", [torch.float32, torch.bfloat16], ids=["dw_f32", "dw_bf16"])
 def test_expert_ffn_backward_matches_oracle(variant, dw_dtype):
     # an empty group, a one-row group, an exact tile, and ragged multi-tile groups

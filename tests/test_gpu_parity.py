@@ -198,8 +198,9 @@ def test_multi_tile_layers(cfg):
     run_and_check_small(cfg)
 
 
-# test-only switches of the library: force the single-CTA or the CTA-pair GEMM
-FORCE_SINGLE, FORCE_PAIR = 2, 4
+# test-only switches of the library: force the single-CTA GEMM, the CTA-pair
+# GEMM alone, or CTA pairs plus single-CTA tiles for groups' short tails
+FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID = 2, 4, 8
 
 
 @pytest.fixture
@@ -209,7 +210,7 @@ def gemm_variant(request):
     moe.moe_set_debug(0, 4000.0)
 
 
-@pytest.mark.parametrize("gemm_variant", [FORCE_SINGLE, FORCE_PAIR], indirect=True)
+@pytest.mark.parametrize("gemm_variant", [FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID], indirect=True)
 @pytest.mark.parametrize("cfg", [
     # 256-row pair tiles over ragged groups, BN = 256 / 256
     inputs.LayerConfig("pair", T=1500, d=256, f=256, E=8, k=2, R=4, seed=21),
