@@ -49,7 +49,7 @@ TRAIN_METRIC = ("MoE-layer training tokens/s (forward + backward: route, BRIM di
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
 # GEMM launches of one layer step, from one ncu capture (profiles/ffn_gemm_pair_olmoe.md),
 # valid only while the GEMM sources hash to `src`; otherwise reported as null.
-GEMM_TRAFFIC = {"olmoe": {"bytes": 1179.2e6, "src": "99a471e2b083403a"}}
+GEMM_TRAFFIC = {"olmoe": {"bytes": 1179.6e6, "src": "1a819270abe1e6b0"}}
 
 
 def gemm_src_hash() -> str:

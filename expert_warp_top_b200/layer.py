@@ -120,7 +120,7 @@ class MoELayer:
                          self.epd_gate, self.c_t, self.brim_ws, stream)
 
     def route_brim(self, logits, stream=None):
-        """Routing, BRIMs, counter and histogram in two launches (moe_route_brim)."""
+        """Routing, BRIMs, counter and histogram in three launches (moe_route_brim)."""
         B.moe_route_brim(logits, self.k, self.renorm, self.slot_of, self.R, self.topk_idx,
                          self.topk_w, self.brim0, self.sfd_token, self.sfd_off, self.brim1,
                          self.epd_off, self.epd_sfd, self.epd_gate, self.c_t, self.brim_ws,
@@ -163,7 +163,7 @@ class MoELayer:
         """All steps of the layer on `stream`; returns y [T, d] (a view of self.y).
 
         fused_index: routing, BRIMs, counter and histogram through moe_route_brim
-        (two launches); otherwise through the four separate entry points."""
+        (three launches); otherwise through the four separate entry points."""
         if fused_index:
             self.route_brim(logits, stream)
         else:

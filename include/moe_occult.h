@@ -186,12 +186,13 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
 
 /* ---------------------------------------------------------------------------
  * moe_route_brim -- moe_route_topk, moe_brim_build, moe_count_dispatched_rows
- * and moe_coact_histogram in two kernel launches instead of six: one block per
+ * and moe_coact_histogram in three kernel launches instead of six: one block per
  * 32-token tile routes its tokens (warp per token, the code of
- * moe_route_topk), builds the tile's BRIM column masks and adds to the counter
- * and the histogram; the last tile to finish scans the columns; a second kernel
- * scatters BRIM_0 / BRIM_1 and their inverses.  Every output is bit for bit
- * the one the separate entry points produce.
+ * moe_route_topk), builds the tile's BRIM column masks and adds to the counter;
+ * then one block per column scans that column while extra blocks of the same
+ * launch build the histogram; a third kernel scatters BRIM_0 / BRIM_1 and
+ * their inverses.  Every output is bit for bit the one the separate entry
+ * points produce.
  *   prune_m > 0 applies moe_prune_topk with m = prune_m between routing and
  *   the BRIMs (0 = no pruning);
  *   other arguments as in those entry points; per_rank / total / remote are given
