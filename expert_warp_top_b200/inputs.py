@@ -98,6 +98,32 @@ def make_logits(cfg: LayerConfig, device="cpu", seed: int | None = None) -> torc
     return logits.contiguous()
 
 
+def make_layer_pair_logits(cfg: LayerConfig, follow_p: float = 0.8, device="cpu",
+                           seed: int | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Router logits of two consecutive layers, float32 [T, E] each, with
+    planted inter-layer affinity.  A token routes inside a planted group with
+    probability cfg.group_p at both layers (the same tokens); its layer-(l+1)
+    group is next(g) for its layer-l group g with probability follow_p, else a
+    uniform draw, where next is a seeded permutation of the groups.  The
+    layer-(l+1) groups come from their own seeded expert permutation."""
+    assert cfg.groups > 0, "planted groups are needed"
+    seed = cfg.seed if seed is None else seed
+    g = torch.Generator(device=device).manual_seed(seed)
+    G = cfg.groups
+    member1 = group_members(cfg.E, G, seed=0).to(device)
+    member2 = group_members(cfg.E, G, seed=1).to(device)
+    nxt = torch.randperm(G, generator=torch.Generator().manual_seed(2)).to(device)
+    l1 = torch.randn(cfg.T, cfg.E, generator=g, device=device, dtype=torch.float32)
+    l2 = torch.randn(cfg.T, cfg.E, generator=g, device=device, dtype=torch.float32)
+    grouped = torch.rand(cfg.T, generator=g, device=device) < cfg.group_p
+    g1 = torch.randint(0, G, (cfg.T,), generator=g, device=device)
+    follow = torch.rand(cfg.T, generator=g, device=device) < follow_p
+    g2 = torch.where(follow, nxt[g1], torch.randint(0, G, (cfg.T,), generator=g, device=device))
+    l1 = l1 + ((member1[None, :] == g1[:, None]) & grouped[:, None]).float() * cfg.group_boost
+    l2 = l2 + ((member2[None, :] == g2[:, None]) & grouped[:, None]).float() * cfg.group_boost
+    return l1.contiguous(), l2.contiguous()
+
+
 def make_inputs(cfg: LayerConfig, device="cpu", seed: int | None = None,
                 weights: bool = True) -> dict[str, torch.Tensor]:
     """All tensors of one layer invocation.

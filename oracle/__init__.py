@@ -48,6 +48,8 @@ def lib():
         _lib.oracle_gather_rows.restype = None
         _lib.oracle_coact_histogram.restype = None
         _lib.oracle_set_num_threads.restype = None
+        _lib.oracle_interlayer_histogram.restype = None
+        _lib.oracle_predict_home.restype = None
     return _lib
 
 
@@ -338,3 +340,51 @@ def route_backward(logits, idx, dw, renorm: int):
     if rc != 0:
         raise ValueError(f"oracle_route_backward failed ({rc})")
     return dl
+
+
+def interlayer_histogram(idx_a, idx_b, E, hist=None):
+    """uint32 [E,E]: H[a][b] = #tokens with a in idx_a[t] and b in idx_b[t]."""
+    idx_a = np.ascontiguousarray(idx_a, dtype=np.int32)
+    idx_b = np.ascontiguousarray(idx_b, dtype=np.int32)
+    T, k = idx_a.shape
+    acc = hist is not None
+    h = hist if acc else np.empty((E, E), np.uint32)
+    lib().oracle_interlayer_histogram(_p(idx_a), _p(idx_b), T, k, E, _p(h), int(acc))
+    return h
+
+
+def rank_affinity(hist, slot_of_b, R):
+    """uint64 [E,R]: A[a][r] = sum over experts b on rank r of hist[a][b]."""
+    hist = np.ascontiguousarray(hist, dtype=np.uint32)
+    E = hist.shape[0]
+    slot_of_b = np.ascontiguousarray(slot_of_b, dtype=np.int32)
+    A = np.empty((E, R), np.uint64)
+    rc = lib().oracle_rank_affinity(_p(hist), E, _p(slot_of_b), int(R), _p(A))
+    if rc != 0:
+        raise ValueError(f"oracle_rank_affinity failed ({rc})")
+    return A
+
+
+def predict_home(idx_a, A):
+    """int32 [T]: the rank maximising sum_j A[idx_a[t][j]] (ties -> lower rank)."""
+    idx_a = np.ascontiguousarray(idx_a, dtype=np.int32)
+    A = np.ascontiguousarray(A, dtype=np.uint64)
+    T, k = idx_a.shape
+    E, R = A.shape
+    home = np.empty(T, np.int32)
+    lib().oracle_predict_home(_p(idx_a), T, k, E, _p(A), R, _p(home))
+    return home
+
+
+def count_local(idx, slot_of, E, R, home=None):
+    """(assignments on the token's home rank, all assignments)."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    slot_of = np.ascontiguousarray(slot_of, dtype=np.int32)
+    T, k = idx.shape
+    if home is not None:
+        home = np.ascontiguousarray(home, dtype=np.int32)
+    out = np.empty(2, np.int64)
+    rc = lib().oracle_count_local(_p(idx), T, k, _p(slot_of), E, int(R), _p(home), _p(out))
+    if rc != 0:
+        raise ValueError(f"oracle_count_local failed ({rc})")
+    return int(out[0]), int(out[1])

@@ -55,6 +55,8 @@
  *   R12 A weight gradient sums, over every (token, slot) routed to that
  *       expert in ascending token order, the outer products of that row;
  *       shared experts take every token with weight 1.
+ *   R13-R15 Token shuffling across layers: see the section of that name
+ *       below.
  */
 #include <math.h>
 #include <stdint.h>
@@ -855,5 +857,91 @@ int oracle_route_backward(const float* logits, int T, int E, int k, int renorm,
     }
   }
   free(q);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Token shuffling across layers ("Expert Coupling in MoE Pretraining",
+ * Abstract: the experts a token selects at one layer predict those it
+ * selects at the next; token shuffling moves each token to the GPU predicted
+ * to hold its next-layer experts).  Readings R13-R15.
+ *
+ *   R13 The inter-layer statistic is the pair histogram of a calibration
+ *       batch: H[a][b] = #tokens that select expert a at layer l and expert b
+ *       at layer l+1 (empty slots, -1, count nothing).
+ *   R14 The affinity of layer-l expert a to rank r is
+ *       A[a][r] = sum over the layer-(l+1) experts b held by rank r of H[a][b];
+ *       a token's predicted rank is the r maximising sum_j A[idx_l[t][j]][r]
+ *       (ties -> lower r); a token whose scores are all zero keeps its
+ *       contiguous home floor(t * R / T).
+ *   R15 The served-locally share counts token-expert assignments of layer l+1
+ *       whose expert sits on the token's home rank; the shuffle itself is the
+ *       stable reordering of tokens by home rank (a BRIM_0 over one
+ *       "expert" per rank).
+ * ---------------------------------------------------------------------- */
+void oracle_interlayer_histogram(const int32_t* idx_a, const int32_t* idx_b, int T, int k, int E,
+                                 uint32_t* H, int accumulate) {
+  if (!accumulate)
+    for (size_t i = 0; i < (size_t)E * E; ++i) H[i] = 0;
+  for (int t = 0; t < T; ++t)
+    for (int i = 0; i < k; ++i) {
+      int a = idx_a[(size_t)t * k + i];
+      if (a < 0 || a >= E) continue;
+      for (int j = 0; j < k; ++j) {
+        int b = idx_b[(size_t)t * k + j];
+        if (b < 0 || b >= E) continue;
+        H[(size_t)a * E + b] += 1;
+      }
+    }
+}
+
+int oracle_rank_affinity(const uint32_t* H, int E, const int32_t* slot_of_b, int R,
+                         uint64_t* A) {
+  if (R < 1 || E % R != 0) return -1;
+  const int L = E / R;
+  for (int a = 0; a < E; ++a)
+    for (int r = 0; r < R; ++r) {
+      uint64_t s = 0;
+      for (int b = 0; b < E; ++b)
+        if (slot_of_b[b] / L == r) s += H[(size_t)a * E + b];
+      A[(size_t)a * R + r] = s;
+    }
+  return 0;
+}
+
+void oracle_predict_home(const int32_t* idx_a, int T, int k, int E, const uint64_t* A, int R,
+                         int32_t* home) {
+  for (int t = 0; t < T; ++t) {
+    int best = -1;
+    uint64_t best_score = 0;
+    for (int r = 0; r < R; ++r) {
+      uint64_t s = 0;
+      for (int j = 0; j < k; ++j) {
+        int a = idx_a[(size_t)t * k + j];
+        if (a >= 0 && a < E) s += A[(size_t)a * R + r];
+      }
+      if (best < 0 || s > best_score) { best = r; best_score = s; } /* ties keep the lower r */
+    }
+    home[t] = best_score > 0 ? best : (int32_t)(((int64_t)t * R) / T);
+  }
+}
+
+/* out[0] = assignments of layer-l+1 experts held by the token's home rank,
+ * out[1] = all assignments (slots that are not empty).  home == NULL means
+ * the contiguous home floor(t * R / T). */
+int oracle_count_local(const int32_t* idx, int T, int k, const int32_t* slot_of, int E, int R,
+                       const int32_t* home, int64_t* out) {
+  if (R < 1 || E % R != 0) return -1;
+  const int L = E / R;
+  out[0] = out[1] = 0;
+  for (int t = 0; t < T; ++t) {
+    int h = home ? home[t] : (int)(((int64_t)t * R) / T);
+    for (int j = 0; j < k; ++j) {
+      int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) continue;
+      out[1] += 1;
+      if (slot_of[e] / L == h) out[0] += 1;
+    }
+  }
   return 0;
 }
