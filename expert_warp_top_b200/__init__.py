@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     moe_route_brim, moe_route_brim_workspace_size, moe_prune_topk,
     moe_expert_ffn_train, moe_expert_ffn_backward, moe_expert_ffn_backward_workspace_size,
     moe_route_backward, moe_layer_train_workspace_size, moe_layer_forward_train,
-    moe_layer_backward,
+    moe_layer_backward, moe_interlayer_histogram, moe_rank_affinity, moe_predict_home,
+    moe_count_local, moe_token_shuffle_workspace_size, moe_token_shuffle,
 )
 from .layer import MoELayer, unpack_gate_up  # noqa: F401

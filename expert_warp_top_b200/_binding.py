@@ -37,7 +37,8 @@ EXPORTS = (
     "moe_place_greedy", "moe_route_brim_workspace_size", "moe_route_brim", "moe_prune_topk",
     "moe_expert_ffn_train", "moe_expert_ffn_backward_workspace_size", "moe_expert_ffn_backward",
     "moe_route_backward", "moe_layer_train_workspace_size", "moe_layer_forward_train",
-    "moe_layer_backward",
+    "moe_layer_backward", "moe_interlayer_histogram", "moe_rank_affinity", "moe_predict_home",
+    "moe_count_local", "moe_token_shuffle_workspace_size", "moe_token_shuffle",
 )
 
 
@@ -67,6 +68,7 @@ def load():
         lib.moe_route_brim_workspace_size.restype = ctypes.c_size_t
         lib.moe_expert_ffn_backward_workspace_size.restype = ctypes.c_size_t
         lib.moe_layer_train_workspace_size.restype = ctypes.c_size_t
+        lib.moe_token_shuffle_workspace_size.restype = ctypes.c_size_t
         lib.moe_set_debug.argtypes = [ctypes.c_int, ctypes.c_double]
         for name in EXPORTS:
             getattr(lib, name)
@@ -382,6 +384,51 @@ def moe_layer_backward(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, dy, dx, 
         _ptr(dw_gu, _ACT, "dw_gu"), _ptr(dw_dn, _ACT, "dw_dn"),
         _ptr(dsw_gu, _ACT, "dsw_gu"), _ptr(dsw_dn, _ACT, "dsw_dn"), int(dw_dtype),
         int(accumulate), _ptr(ws, None, "ws"), _nbytes(ws), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# token shuffling across layers
+def moe_interlayer_histogram(idx_l, idx_next, E, hist, accumulate=0, stream=None):
+    T, k = idx_l.shape
+    _check("moe_interlayer_histogram", load().moe_interlayer_histogram(
+        _ptr(idx_l, I32, "idx_l"), _ptr(idx_next, I32, "idx_next"), int(T), int(k), int(E),
+        _ptr(hist, (U32, torch.int32), "hist"), int(accumulate), _stream(stream)))
+
+
+def moe_rank_affinity(hist, slot_of_next, R, table, stream=None):
+    E = hist.shape[0]
+    _check("moe_rank_affinity", load().moe_rank_affinity(
+        _ptr(hist, (U32, torch.int32), "hist"), int(E), _ptr(slot_of_next, I32, "slot_of_next"),
+        int(R), _ptr(table, (U32, torch.int32), "table"), _stream(stream)))
+
+
+def moe_predict_home(idx_l, table, home, stream=None):
+    T, k = idx_l.shape
+    E, R = table.shape
+    _check("moe_predict_home", load().moe_predict_home(
+        _ptr(idx_l, I32, "idx_l"), int(T), int(k), int(E), _ptr(table, (U32, torch.int32), "table"),
+        int(R), _ptr(home, I32, "home"), _stream(stream)))
+
+
+def moe_count_local(idx, slot_of, E, R, out, home=None, stream=None):
+    T, k = idx.shape
+    _check("moe_count_local", load().moe_count_local(
+        _ptr(idx, I32, "idx"), int(T), int(k), _ptr(slot_of, I32, "slot_of"), int(E), int(R),
+        _ptr(home, I32, "home"), _ptr(out, I64, "out"), _stream(stream)))
+
+
+def moe_token_shuffle_workspace_size(T: int, R: int) -> int:
+    return int(load().moe_token_shuffle_workspace_size(int(T), int(R)))
+
+
+def moe_token_shuffle(home, R, perm, rank_off, ws, x=None, x_out=None, inv=None, stream=None):
+    T = home.numel()
+    d = x.shape[1] if x is not None else 0
+    dt = dtype_code(x.dtype) if x is not None else MOE_BF16
+    _check("moe_token_shuffle", load().moe_token_shuffle(
+        _ptr(home, I32, "home"), int(T), int(R), _ptr(x, _ACT, "x"), int(d), int(dt),
+        _ptr(x_out, _ACT, "x_out"), _ptr(perm, I32, "perm"), _ptr(rank_off, I32, "rank_off"),
+        _ptr(inv, I32, "inv"), _ptr(ws, None, "ws"), _nbytes(ws), _stream(stream)))
 
 
 def moe_place_greedy(hist, R) -> torch.Tensor:

@@ -17,6 +17,7 @@
 #include "host.h"
 #include "route.cuh"
 #include "route_brim.cuh"
+#include "shuffle.cuh"
 
 // The device error flag the kernels raise (bits moe::kErrIndex, kErrTimeout).
 __device__ unsigned g_moe_err_flag;
@@ -465,6 +466,155 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   }
 #undef MOE_ROUTE_BRIM
   MOE_LAUNCHED("route_brim_tile_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Token shuffling across layers.
+int moe_interlayer_histogram(const int32_t* idx_l, const int32_t* idx_next, int T, int k, int E,
+                             uint32_t* hist, int accumulate, moe_stream_t stream) {
+  int rc = check_common(T, E, k, 1);
+  if (rc) return rc;
+  MOE_REQUIRE(hist, MOE_ERR_INVALID_ARG, "null pointer");
+  if (!accumulate) MOE_CUDA(cudaMemsetAsync(hist, 0, sizeof(uint32_t) * E * E, stream));
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(idx_l && idx_next, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const dim3 grid((T + 255) / 256), block(256);
+#define MOE_IL(KM)                                                                            \
+  MOE_CUDA(launch_k(moe::interlayer_hist_kernel<KM>, grid, block, 0, stream, idx_l, idx_next, T, \
+                    k, E, hist, di->err_flag))
+  if (k <= 2) MOE_IL(2);
+  else if (k <= 4) MOE_IL(4);
+  else if (k <= 8) MOE_IL(8);
+  else MOE_IL(16);
+#undef MOE_IL
+  MOE_LAUNCHED("interlayer_hist_kernel");
+  return MOE_OK;
+}
+
+int moe_rank_affinity(const uint32_t* hist, int E, const int32_t* slot_of_next, int R,
+                      uint32_t* table, moe_stream_t stream) {
+  int rc = check_common(0, E, 1, R);
+  if (rc) return rc;
+  MOE_REQUIRE(hist && slot_of_next && table, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  MOE_CUDA(launch_k(moe::rank_affinity_kernel, dim3((E * R + 255) / 256), dim3(256), 0, stream,
+                    hist, E, slot_of_next, R, table, di->err_flag));
+  MOE_LAUNCHED("rank_affinity_kernel");
+  return MOE_OK;
+}
+
+int moe_predict_home(const int32_t* idx_l, int T, int k, int E, const uint32_t* table, int R,
+                     int32_t* home, moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(idx_l && table && home, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const dim3 grid((unsigned)(((long long)T * 32 + 255) / 256)), block(256);
+#define MOE_PH(KM) \
+  MOE_CUDA(launch_k(moe::predict_home_kernel<KM>, grid, block, 0, stream, idx_l, T, k, E, table, R, home))
+  if (k <= 2) MOE_PH(2);
+  else if (k <= 4) MOE_PH(4);
+  else if (k <= 8) MOE_PH(8);
+  else MOE_PH(16);
+#undef MOE_PH
+  MOE_LAUNCHED("predict_home_kernel");
+  return MOE_OK;
+}
+
+int moe_count_local(const int32_t* idx, int T, int k, const int32_t* slot_of, int E, int R,
+                    const int32_t* home, int64_t* out, moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  MOE_REQUIRE(out, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_CUDA(cudaMemsetAsync(out, 0, 2 * sizeof(int64_t), stream));
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(idx && slot_of, MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const dim3 grid((T + 255) / 256), block(256);
+  auto* o = reinterpret_cast<unsigned long long*>(out);
+#define MOE_CL(KM)                                                                             \
+  MOE_CUDA(launch_k(moe::count_local_kernel<KM>, grid, block, 0, stream, idx, T, k, slot_of, E, R, \
+                    home, o, di->err_flag))
+  if (k <= 2) MOE_CL(2);
+  else if (k <= 4) MOE_CL(4);
+  else if (k <= 8) MOE_CL(8);
+  else MOE_CL(16);
+#undef MOE_CL
+  MOE_LAUNCHED("count_local_kernel");
+  return MOE_OK;
+}
+
+namespace {
+struct ShuffleCarve {
+  uint32_t* scratch; int32_t *brim0, *brim1, *epd_off, *epd_sfd, *c_t; float* epd_gate;
+};
+size_t carve_shuffle(char* base, int T, int R, ShuffleCarve* out) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes ? bytes : 1);
+    return p;
+  };
+  ShuffleCarve c{};
+  c.scratch = reinterpret_cast<uint32_t*>(take(sizeof(int32_t) * brim_scratch_entries(T, R, R)));
+  c.brim0 = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)R * T));
+  c.brim1 = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
+  c.epd_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (R + 1)));
+  c.epd_sfd = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)T));
+  c.epd_gate = reinterpret_cast<float*>(take(sizeof(float) * (size_t)T));
+  c.c_t = reinterpret_cast<int32_t*>(take(sizeof(int32_t)));
+  if (out) *out = c;
+  return off + 256;
+}
+}  // namespace
+
+size_t moe_token_shuffle_workspace_size(int T, int R) {
+  if (T < 0 || R < 1 || R > moe::kMaxE) return 0;
+  return carve_shuffle(nullptr, T, R, nullptr);
+}
+
+int moe_token_shuffle(const int32_t* home, int T, int R, const void* x, int d, int dtype,
+                      void* x_out, int32_t* perm, int32_t* rank_off, int32_t* inv, void* ws,
+                      size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_common(T, R, 1, R);
+  if (rc) return rc;
+  MOE_REQUIRE(perm && rank_off, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(!x || ((rc = check_dtype(dtype)) == 0 && d >= 64 && d % 64 == 0 && x_out),
+              MOE_ERR_INVALID_ARG, "x needs x_out, a known dtype and d a positive multiple of 64");
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(rank_off, 0, sizeof(int32_t) * (R + 1), stream));
+    return MOE_OK;
+  }
+  MOE_REQUIRE(home && ws && aligned16(ws), MOE_ERR_INVALID_ARG, "null or misaligned pointer");
+  MOE_REQUIRE(!x || (aligned16(x) && aligned16(x_out)), MOE_ERR_INVALID_ARG,
+              "rows must be 16-byte aligned");
+  const size_t need = carve_shuffle(nullptr, T, R, nullptr);
+  MOE_REQUIRE(ws_bytes >= need, MOE_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes",
+              ws_bytes, need);
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+  ShuffleCarve c;
+  carve_shuffle(base, T, R, &c);
+  // the home-rank order: BRIM_0 over one "expert" per rank (k = 1, E = R,
+  // identity placement), so the order within a rank is ascending token order
+  if ((rc = brim_passes(home, nullptr, T, 1, nullptr, R, R, c.brim0, perm, rank_off, c.brim1,
+                        c.epd_off, c.epd_sfd, c.epd_gate, c.c_t, c.scratch, di->err_flag, stream)))
+    return rc;
+  if (x || inv) {
+    const int row_bytes = x ? d * esize(dtype) : 0;
+    MOE_CUDA(launch_k(moe::gather_rows_kernel, dim3((unsigned)(((long long)T * 32 + 255) / 256)),
+                      dim3(256), 0, stream, static_cast<const uint8_t*>(x), perm, T, row_bytes,
+                      static_cast<uint8_t*>(x_out), inv, di->err_flag));
+    MOE_LAUNCHED("gather_rows_kernel");
+  }
   return MOE_OK;
 }
 

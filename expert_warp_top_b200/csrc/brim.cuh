@@ -57,7 +57,7 @@ __device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
     tr.rank[j] = -1;
     if (j < k && ids[j] != -1) {
       const int e = ids[j];
-      const int q = (e >= 0 && e < E) ? __ldg(slot_of + e) : -1;
+      const int q = (e >= 0 && e < E) ? (slot_of ? __ldg(slot_of + e) : e) : -1;  // null: identity
       if (q < 0 || q >= E) ok = false;
       tr.slot[j] = q;
       tr.rank[j] = q >= 0 ? q / L : -1;
@@ -353,7 +353,8 @@ __global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
   float gate[KMAX];
 #pragma unroll
   for (int j = 0; j < KMAX; ++j)
-    gate[j] = (active && j < k && tr.slot[j] >= 0) ? __ldg(topk_w + (size_t)t * k + j) : 0.f;
+    gate[j] = (active && j < k && tr.slot[j] >= 0) ? (topk_w ? __ldg(topk_w + (size_t)t * k + j) : 1.f)
+                                                   : 0.f;
   if (warp == 0) {
     tile_masks<KMAX>(sm, ncol, R, active, k, tr);
     // the tile's first global row in every column

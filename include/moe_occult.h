@@ -381,6 +381,59 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* ===========================================================================
+ * Token shuffling across layers ("Expert Coupling in MoE Pretraining",
+ * Abstract): the experts a token selects at one layer predict the experts it
+ * selects at the next, so each token can be moved to the rank predicted to
+ * hold its next-layer experts (in a real system during the reduce-scatter
+ * after attention).  On one GPU the statistics, the prediction, the new token
+ * order and the row movement are computed; the share of next-layer
+ * assignments served on the token's home rank measures the effect.
+ * ========================================================================= */
+
+/* moe_interlayer_histogram -- hist [E, E] uint32 (device):
+ *   hist[a][b] += #tokens t with a in idx_l[t] and b in idx_next[t]
+ * (both [T, k] int32; -1 = empty slot, counts nothing; other ids outside
+ * [0, E) raise MOE_ERR_DEVICE_CHECK).  accumulate = 0 clears hist first.  A
+ * calibration statistic, like the co-activation histogram. */
+int moe_interlayer_histogram(const int32_t* idx_l, const int32_t* idx_next, int T, int k, int E,
+                             uint32_t* hist, int accumulate, moe_stream_t stream);
+
+/* moe_rank_affinity -- table [E, R] uint32 (device):
+ *   table[a][r] = sum of hist[a][b] over the experts b that rank r holds at
+ *                 the next layer (slot_of_next[b] / (E / R) == r).
+ * Sums are 32-bit: the histogram's total must stay below 2^32. */
+int moe_rank_affinity(const uint32_t* hist, int E, const int32_t* slot_of_next, int R,
+                      uint32_t* table, moe_stream_t stream);
+
+/* moe_predict_home -- home [T] int32 (device): the rank r maximising
+ * sum_j table[idx_l[t][j]][r] (ties: the lower r); a token whose scores are all
+ * zero keeps its contiguous home floor(t * R / T).  One warp per token. */
+int moe_predict_home(const int32_t* idx_l, int T, int k, int E, const uint32_t* table, int R,
+                     int32_t* home, moe_stream_t stream);
+
+/* moe_count_local -- out [2] int64 (device): out[0] = assignments in idx [T, k]
+ * whose expert sits on the token's home rank (home [T], or NULL for the
+ * contiguous home floor(t * R / T)); out[1] = all assignments (-1 slots
+ * excluded).  The share out[0] / out[1] is what token shuffling raises. */
+int moe_count_local(const int32_t* idx, int T, int k, const int32_t* slot_of, int E, int R,
+                    const int32_t* home, int64_t* out, moe_stream_t stream);
+
+/* moe_token_shuffle -- the tokens in home-rank order:
+ *   perm [T] int32       perm[i] = the token at position i (ascending token
+ *                        order within each rank's segment)
+ *   rank_off [R+1] int32 where each rank's segment starts; rank_off[R] = T
+ *   inv [T] int32        (may be NULL) inv[t] = the position of token t
+ *   x_out [T, d]         (x may be NULL to skip) x_out[i] = x[perm[i]], rows of
+ *                        dtype, bit for bit
+ * home values must lie in [0, R).  The order is a BRIM_0 over one "expert" per
+ * rank (the BRIM passes with k = 1, E = R); the rows move one warp per row.
+ *   ws  at least moe_token_shuffle_workspace_size(T, R) bytes, 16-byte aligned */
+size_t moe_token_shuffle_workspace_size(int T, int R);
+int moe_token_shuffle(const int32_t* home, int T, int R, const void* x, int d, int dtype,
+                      void* x_out, int32_t* perm, int32_t* rank_off, int32_t* inv, void* ws,
+                      size_t ws_bytes, moe_stream_t stream);
+
+/* ===========================================================================
  * Training: forward that keeps what the backward needs, and the backward.
  *
  * The backward is the exact derivative of the layer for fixed expert choices:
