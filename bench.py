@@ -18,6 +18,12 @@ to host memory inside the timed region.
 `--impl reference` times the CPU oracle (the plain reference implementation
 of the layer) on the host cores on a bounded sample of the same workload.
 
+`--shuffle` measures token shuffling across two layers on the correlated
+prefill workload: per step, the home rank each token is predicted to need at
+the next layer (from its experts at this layer) and the reorder of its rows by
+that rank; the line also reports the share of next-layer assignments served
+on the token's rank before and after.
+
 `--train` measures the training step instead: moe_layer_forward_train then
 moe_layer_backward (gradients of x, of the logits and of every weight, fp32
 weight gradients), with the backward expert GEMMs (moe_expert_ffn_backward)
@@ -43,6 +49,8 @@ import torch  # noqa: E402
 from expert_warp_top_b200 import inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (route+BRIM dispatch+grouped GEMM+combine)"
+SHUFFLE_METRIC = ("token-shuffle tokens/s (predicted home rank from the previous layer's experts "
+                  "+ reorder of the token rows by home rank)")
 TRAIN_METRIC = ("MoE-layer training tokens/s (forward + backward: route, BRIM dispatch, grouped "
                 "GEMMs, combine; input, logit and weight gradients)")
 
@@ -688,6 +696,202 @@ def run_train(args, cfg):
         dist.destroy_process_group()
 
 
+def cpu_baseline_shuffle(cfg, table, idx1, x, budget_s: float = 10.0):
+    """The oracle's shuffle step on growing token prefixes: predicted homes,
+    the home-rank order (BRIM_0 over one "expert" per rank) and the row gather."""
+    import oracle
+    total_n, total_t, n = 0, 0.0, 256
+    while total_t < budget_s and n <= cfg.T:
+        t0 = time.perf_counter()
+        home = oracle.predict_home(np.ascontiguousarray(idx1[:n]), table)
+        b = oracle.brim(home[:, None], np.ones((n, 1)), np.arange(cfg.R, dtype=np.int32), cfg.R,
+                        cfg.R)
+        oracle.gather_rows(np.ascontiguousarray(x[:n]), b["sfd_token"])
+        total_t += time.perf_counter() - t0
+        total_n += n
+        n *= 2
+    return {"value": total_n / total_t, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"token prefixes of 256, 512, ... ({total_n} tokens in all): predicted "
+                      f"homes, home-rank order, row gather; {total_t:.1f} s"}
+
+
+def run_shuffle(args, cfg):
+    import torch.distributed as dist
+    from expert_warp_top_b200 import _binding as B
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    assert cfg.groups > 0, "token shuffling is measured on a workload with planted groups"
+    T, E, k, R = cfg.T, cfg.E, cfg.k, cfg.R
+    i32 = dict(dtype=torch.int32, device=dev)
+
+    def route(logits):
+        idx = torch.empty(logits.shape[0], k, **i32)
+        w = torch.empty(logits.shape[0], k, dtype=torch.float32, device=dev)
+        B.moe_route_topk(logits, k, cfg.renorm, idx, w)
+        return idx
+
+    # calibration batch: layer-(l+1) placement from its co-activation, and the
+    # inter-layer affinity of layer-l experts to layer-(l+1) ranks
+    c1, c2 = (route(l) for l in inputs.make_layer_pair_logits(cfg.with_(seed=1), device=dev))
+    coact = torch.zeros(E, E, **i32)
+    B.moe_coact_histogram(c2, E, coact, 0)
+    slot2 = B.moe_place_greedy(coact.cpu(), R).to(dev)
+    hist = torch.empty(E, E, **i32)
+    B.moe_interlayer_histogram(c1, c2, E, hist, 0)
+    table = torch.empty(E, R, **i32)
+    B.moe_rank_affinity(hist, slot2, R, table)
+    # the evaluation batch (this rank's own)
+    l1, l2 = inputs.make_layer_pair_logits(cfg, device=dev, seed=rank_seed(cfg, rank))
+    idx1, idx2 = route(l1), route(l2)
+    g = torch.Generator(device=dev).manual_seed(rank_seed(cfg, rank) + 5)
+    x = torch.randn(T, cfg.d, generator=g, device=dev).to(inputs.torch_dtype(cfg))
+    home = torch.empty(T, **i32)
+    perm = torch.empty(T, **i32)
+    rank_off = torch.empty(R + 1, **i32)
+    x_out = torch.empty_like(x)
+    ws = torch.empty(B.moe_token_shuffle_workspace_size(T, R), dtype=torch.uint8, device=dev)
+
+    def step():
+        B.moe_predict_home(idx1, table, home)
+        B.moe_token_shuffle(home, R, perm, rank_off, ws, x=x, x_out=x_out)
+
+    stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(args.warmup):
+            step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    if B.moe_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    torch.cuda.synchronize(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    step_ms = []
+    with ClockSampler(local_rank) as clocks:
+        t_end = time.time() + 5.0
+        while clocks.n_samples() < 2 and time.time() < t_end:
+            for _ in range(50):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            s0.record(stream)
+            graph.replay()
+            s1.record(stream)
+            s1.synchronize()
+            step_ms.append(s0.elapsed_time(s1))
+        if world > 1:
+            dist.barrier()
+        t_end = time.time() + 2.0
+        n0 = clocks.n_samples()
+        while clocks.n_samples() < n0 + 2 and time.time() < t_end:
+            for _ in range(50):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+    if B.moe_get_device_status() != 0:
+        raise RuntimeError("device status after the timed steps")
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
+    ms_per_step = total_ms / args.steps
+    value = whole_job_tokens_per_s(T, args.steps, world, total_ms)
+
+    # served on the token's rank at layer l+1: contiguous home vs predicted home
+    cnt = torch.empty(2, dtype=torch.int64, device=dev)
+    B.moe_count_local(idx2, slot2, E, R, cnt)
+    base = cnt.cpu().tolist()
+    B.moe_count_local(idx2, slot2, E, R, cnt, home=home)
+    shuf = cnt.cpu().tolist()
+
+    # end to end: layer-l experts and rows from pinned host memory, the
+    # reordered rows and the order back to pinned host memory
+    h_idx1 = idx1.cpu().pin_memory()
+    h_x = x.cpu().pin_memory()
+    h_out = torch.empty_like(h_x).pin_memory()
+    h_perm = torch.empty(T, dtype=torch.int32).pin_memory()
+    d_idx1, d_x = torch.empty_like(idx1), torch.empty_like(x)
+
+    def e2e_step():
+        d_idx1.copy_(h_idx1, non_blocking=True)
+        d_x.copy_(h_x, non_blocking=True)
+        B.moe_predict_home(d_idx1, table, home)
+        B.moe_token_shuffle(home, R, perm, rank_off, ws, x=d_x, x_out=x_out)
+        h_out.copy_(x_out, non_blocking=True)
+        h_perm.copy_(perm, non_blocking=True)
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3, dev)
+    e2e = {"value": whole_job_tokens_per_s(T, args.steps, world, e2e_ms), "unit": UNIT,
+           "h2d_bytes_per_step": h_idx1.numel() * 4 + h_x.numel() * h_x.element_size(),
+           "d2h_bytes_per_step": h_out.numel() * h_out.element_size() + T * 4,
+           "api": "moe_predict_home + moe_token_shuffle (C ABI), pinned host copies in the "
+                  "step, wall clock"}
+
+    pk = peaks()
+    e = x.element_size()
+    # algorithmic bytes: rows read and written once; top-k ids read twice (prediction
+    # and order), homes written and read, the order and the BRIM_0 written
+    bytes_ = 2.0 * T * cfg.d * e + 4.0 * (T * k + 3 * T + R * T + T)
+    achieved = bytes_ / (ms_per_step * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+            "frac": achieved / pk["hbm"], "peak_source": f"{pk['source']} HBM copy bandwidth",
+            "kernel": "the shuffle step: predict_home + BRIM passes (k = 1, E = R) + row gather",
+            "algorithmic_bytes": bytes_, "traffic": None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        calib_tab = oracle.rank_affinity(hist.cpu().numpy().astype(np.uint32),
+                                         slot2.cpu().numpy(), R)
+        xb = x.cpu().view(torch.int16).numpy().view(np.uint16) if x.dtype == torch.bfloat16 \
+            else x.cpu().numpy()
+        cpu = cpu_baseline_shuffle(cfg, calib_tab, idx1.cpu().numpy(), xb)
+    if rank == 0:
+        line = {
+            "metric": SHUFFLE_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: T={T} d={cfg.d} E={E} k={k} R={R}, two layers "
+                                   f"with planted inter-layer affinity (follow 0.8)",
+                       "calibration": "separate batch (seed 1): layer-(l+1) placement from "
+                                      "its co-activation, inter-layer affinity table",
+                       "l2": "flushed between steps (256 MiB write outside the per-step events)",
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": roof,
+            "served_on_home_rank": {"contiguous_home": base[0] / base[1],
+                                    "predicted_home": shuf[0] / shuf[1],
+                                    "assignments": base[1]},
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks.summary(),
+            "gpu_launches": 5 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def placement(cfg, how, dev, logits):
     """slot_of for the run.  "histogram": correlated placement from the expert
     co-activation histogram of a separate calibration batch (T = 32768, seed 1),
@@ -757,6 +961,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--placement", default="contiguous", choices=["contiguous", "histogram"])
+    ap.add_argument("--shuffle", action="store_true",
+                    help="time token shuffling across two layers (correlated prefill workload)")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (forward + backward) instead of the forward")
     ap.add_argument("--prune", type=int, default=0,
@@ -769,6 +975,8 @@ def main():
         run_reference(args, cfg)
     elif args.train:
         run_train(args, cfg)
+    elif args.shuffle:
+        run_shuffle(args, cfg if args.config != "olmoe" else inputs.CONFIGS["corr_prefill"])
     else:
         run_ours(args, cfg)
 
