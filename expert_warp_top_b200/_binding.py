@@ -39,6 +39,7 @@ EXPORTS = (
     "moe_route_backward", "moe_layer_train_workspace_size", "moe_layer_forward_train",
     "moe_layer_backward", "moe_interlayer_histogram", "moe_rank_affinity", "moe_predict_home",
     "moe_count_local", "moe_token_shuffle_workspace_size", "moe_token_shuffle",
+    "moe_layer_forward_host_async",
 )
 
 
@@ -285,11 +286,14 @@ def moe_layer_forward(logits, x, k, R, renorm, slot_of, w_gu, w_dn, f, y, ws, sw
 
 
 def moe_layer_forward_host(h_logits, h_x, k, R, renorm, slot_of, w_gu, w_dn, f, h_y, ws,
-                           sw_gu=None, sw_dn=None, S=0, fs=0, prune_m=0, stream=None):
-    """The layer on host buffers: H2D copies, every step, D2H copy, then synchronise."""
+                           sw_gu=None, sw_dn=None, S=0, fs=0, prune_m=0, stream=None,
+                           asynchronous=False):
+    """The layer on host buffers: H2D copies, every step, D2H copy, then synchronise
+    (asynchronous=True: moe_layer_forward_host_async, no synchronisation)."""
     T, E = h_logits.shape
     d = h_x.shape[1]
-    _check("moe_layer_forward_host", load().moe_layer_forward_host(
+    name = "moe_layer_forward_host_async" if asynchronous else "moe_layer_forward_host"
+    _check(name, getattr(load(), name)(
         int(T), int(d), int(f), int(E), int(k), int(R), int(renorm), int(prune_m), int(S), int(fs),
         dtype_code(h_x.dtype), _host_ptr(h_logits, F32, "h_logits"), _host_ptr(h_x, _ACT, "h_x"),
         _ptr(slot_of, I32, "slot_of"), _ptr(w_gu, h_x.dtype, "w_gu"),

@@ -1032,11 +1032,12 @@ int moe_layer_forward(int T, int d, int f, int E, int k, int R, int renorm, int 
                      sw_gu, sw_dn, y, c_t, per_rank, total, remote, hist, st, stream);
 }
 
-int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int prune_m,
-                           int S, int fs, int dtype, const float* h_logits, const void* h_x,
-                           const int32_t* slot_of, const void* w_gu, const void* w_dn,
-                           const void* sw_gu, const void* sw_dn, void* h_y, void* ws,
-                           size_t ws_bytes, moe_stream_t stream) {
+namespace {
+int layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int prune_m, int S,
+                       int fs, int dtype, const float* h_logits, const void* h_x,
+                       const int32_t* slot_of, const void* w_gu, const void* w_dn,
+                       const void* sw_gu, const void* sw_dn, void* h_y, void* ws,
+                       size_t ws_bytes, cudaStream_t stream, bool sync) {
   int rc = check_layer_args(T, d, f, E, k, R, renorm, S, fs, dtype);
   if (rc) return rc;
   MOE_REQUIRE(ws && aligned16(ws), MOE_ERR_INVALID_ARG, "workspace missing or misaligned");
@@ -1047,6 +1048,7 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
   if (T == 0) return MOE_OK;
   MOE_REQUIRE(h_logits && h_x && h_y && slot_of && w_gu && w_dn, MOE_ERR_INVALID_ARG,
               "null pointer");
+  MOE_REQUIRE(prune_m >= 0, MOE_ERR_INVALID_ARG, "prune_m must be >= 0 (0 = no pruning)");
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
   LayerState st;
   carve_layer(base, T, d, f, E, k, R, S, fs, dtype, true, &st);
@@ -1054,14 +1056,32 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
   MOE_CUDA(cudaMemcpyAsync(st.logits, h_logits, sizeof(float) * (size_t)T * E,
                            cudaMemcpyHostToDevice, stream));
   MOE_CUDA(cudaMemcpyAsync(st.x, h_x, xb, cudaMemcpyHostToDevice, stream));
-  MOE_REQUIRE(prune_m >= 0, MOE_ERR_INVALID_ARG, "prune_m must be >= 0 (0 = no pruning)");
   rc = layer_steps(T, d, f, E, k, R, renorm, prune_m, S, fs, dtype, st.logits, st.x, slot_of,
-                   w_gu, w_dn,
-                   sw_gu, sw_dn, st.y, nullptr, nullptr, nullptr, nullptr, nullptr, st, stream);
+                   w_gu, w_dn, sw_gu, sw_dn, st.y, nullptr, nullptr, nullptr, nullptr, nullptr,
+                   st, stream);
   if (rc) return rc;
   MOE_CUDA(cudaMemcpyAsync(h_y, st.y, xb, cudaMemcpyDeviceToHost, stream));
-  MOE_CUDA(cudaStreamSynchronize(stream));
+  if (sync) MOE_CUDA(cudaStreamSynchronize(stream));
   return MOE_OK;
+}
+}  // namespace
+
+int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm, int prune_m,
+                           int S, int fs, int dtype, const float* h_logits, const void* h_x,
+                           const int32_t* slot_of, const void* w_gu, const void* w_dn,
+                           const void* sw_gu, const void* sw_dn, void* h_y, void* ws,
+                           size_t ws_bytes, moe_stream_t stream) {
+  return layer_forward_host(T, d, f, E, k, R, renorm, prune_m, S, fs, dtype, h_logits, h_x,
+                            slot_of, w_gu, w_dn, sw_gu, sw_dn, h_y, ws, ws_bytes, stream, true);
+}
+
+int moe_layer_forward_host_async(int T, int d, int f, int E, int k, int R, int renorm,
+                                 int prune_m, int S, int fs, int dtype, const float* h_logits,
+                                 const void* h_x, const int32_t* slot_of, const void* w_gu,
+                                 const void* w_dn, const void* sw_gu, const void* sw_dn,
+                                 void* h_y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return layer_forward_host(T, d, f, E, k, R, renorm, prune_m, S, fs, dtype, h_logits, h_x,
+                            slot_of, w_gu, w_dn, sw_gu, sw_dn, h_y, ws, ws_bytes, stream, false);
 }
 
 }  // extern "C"

@@ -202,14 +202,23 @@ class MoELayer:
                             prune_m=self.prune_m, stream=stream)
         return y
 
-    def forward_host(self, h_logits, h_x, h_y, stream=None):
-        """Host buffers in and out through moe_layer_forward_host (synchronises)."""
+    def forward_host(self, h_logits, h_x, h_y, stream=None, ws=None, asynchronous=False):
+        """Host buffers in and out through moe_layer_forward_host (synchronises), or
+        moe_layer_forward_host_async (asynchronous=True; pass a workspace per batch in
+        flight, from host_workspace())."""
         B.moe_layer_forward_host(h_logits, h_x, self.k, self.R, self.renorm, self.slot_of,
-                                 self.w_gu, self.w_dn, self.f, h_y, self._layer_ws(True),
+                                 self.w_gu, self.w_dn, self.f, h_y,
+                                 self._layer_ws(True) if ws is None else ws,
                                  sw_gu=getattr(self, "sw_gu", None),
                                  sw_dn=getattr(self, "sw_dn", None), S=self.S, fs=self.fs,
-                                 prune_m=self.prune_m, stream=stream)
+                                 prune_m=self.prune_m, stream=stream, asynchronous=asynchronous)
         return h_y
+
+    def host_workspace(self):
+        """A fresh workspace for moe_layer_forward_host(_async)."""
+        n = B.moe_layer_workspace_size(self.T, self.d, self.f, self.E, self.k, self.R, self.S,
+                                       self.fs, B.dtype_code(self.dtype), 1)
+        return torch.empty(max(n, 256), dtype=torch.uint8, device=self.y.device)
 
     # -- training: forward that keeps state, and the backward ----------------
     def _train_ws(self):

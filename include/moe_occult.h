@@ -379,6 +379,17 @@ int moe_layer_forward_host(int T, int d, int f, int E, int k, int R, int renorm,
                            const int32_t* slot_of, const void* w_gu, const void* w_dn,
                            const void* sw_gu, const void* sw_dn, void* h_y,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
+/* moe_layer_forward_host_async -- moe_layer_forward_host without the final
+ * synchronisation: everything (both copies in, the layer, the copy out) is
+ * enqueued on `stream` and the call returns.  The host buffers (pinned) and
+ * the workspace must stay untouched until the stream has passed this work.
+ * With two workspaces on two streams, one batch's copies overlap another
+ * batch's layer. */
+int moe_layer_forward_host_async(int T, int d, int f, int E, int k, int R, int renorm,
+                                 int prune_m, int S, int fs, int dtype, const float* h_logits,
+                                 const void* h_x, const int32_t* slot_of, const void* w_gu,
+                                 const void* w_dn, const void* sw_gu, const void* sw_dn,
+                                 void* h_y, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* ===========================================================================
  * Token shuffling across layers ("Expert Coupling in MoE Pretraining",

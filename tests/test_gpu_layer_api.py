@@ -111,3 +111,32 @@ def test_bounded_wait_expires_and_context_survives(variant):
     y_ref = oracle.dense_layer(to_oracle(inp["x"]), idx, w, to_oracle(inp["wg"]),
                                to_oracle(inp["wu"]), to_oracle(inp["wd"]))
     assert rowwise_rel_err(layer.y.float().cpu().numpy(), y_ref) <= OUT_RTOL
+
+
+def test_layer_forward_host_async_two_batches_in_flight():
+    """moe_layer_forward_host_async on two streams with their own workspaces:
+    two different batches in flight give the same bits as one at a time."""
+    cfg = inputs.LayerConfig("async", T=900, d=256, f=256, E=8, k=2, R=4, S=1, fs=128, seed=41)
+    inp_a = inputs.make_inputs(cfg)
+    inp_b = inputs.make_inputs(cfg, seed=42, weights=False)
+    layer = make_layer(cfg, inp_a)
+    hosts = []
+    for inp in (inp_a, inp_b):
+        hosts.append((inp["logits"].contiguous().pin_memory(), inp["x"].contiguous().pin_memory()))
+    ref = []
+    for h_l, h_x in hosts:
+        h_y = torch.empty_like(h_x).pin_memory()
+        layer.forward_host(h_l, h_x, h_y)
+        ref.append(h_y.clone())
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [layer.host_workspace(), layer.host_workspace()]
+    outs = [torch.empty_like(hosts[0][1]).pin_memory() for _ in range(2)]
+    for rep in range(3):
+        for i, (h_l, h_x) in enumerate(hosts):
+            streams[i].synchronize()
+            layer.forward_host(h_l, h_x, outs[i], stream=streams[i], ws=wss[i], asynchronous=True)
+        for s in streams:
+            s.synchronize()
+        assert moe.moe_get_device_status() == moe.MOE_OK
+        for i in range(2):
+            assert torch.equal(outs[i], ref[i]), (rep, i)
