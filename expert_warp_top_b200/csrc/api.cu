@@ -585,13 +585,14 @@ int moe_token_shuffle(const int32_t* home, int T, int R, const void* x, int d, i
                       size_t ws_bytes, moe_stream_t stream) {
   int rc = check_common(T, R, 1, R);
   if (rc) return rc;
-  MOE_REQUIRE(perm && rank_off, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(rank_off, MOE_ERR_INVALID_ARG, "null pointer");
   MOE_REQUIRE(!x || ((rc = check_dtype(dtype)) == 0 && d >= 64 && d % 64 == 0 && x_out),
               MOE_ERR_INVALID_ARG, "x needs x_out, a known dtype and d a positive multiple of 64");
   if (T == 0) {
     MOE_CUDA(cudaMemsetAsync(rank_off, 0, sizeof(int32_t) * (R + 1), stream));
     return MOE_OK;
   }
+  MOE_REQUIRE(perm, MOE_ERR_INVALID_ARG, "null pointer");
   MOE_REQUIRE(home && ws && aligned16(ws), MOE_ERR_INVALID_ARG, "null or misaligned pointer");
   MOE_REQUIRE(!x || (aligned16(x) && aligned16(x_out)), MOE_ERR_INVALID_ARG,
               "rows must be 16-byte aligned");

@@ -389,3 +389,26 @@ def test_backward_bounded_wait_expires_and_context_survives(variant):
     dwg, _ = unpack_gate_up(dw_gu.cpu())
     assert normwise_err(dwg[0].numpy(), g["dwg"][0]) <= GRAD_RTOL
     assert normwise_err(dw_dn[2].cpu().numpy(), g["dwd"][2]) <= GRAD_RTOL
+
+
+def test_empty_batch_zeroes_weight_gradients():
+    """T = 0: no rows at all; the weight gradients are zero (accumulate = 0) or
+    left as they are (accumulate = 1)."""
+    cfg = inputs.LayerConfig("empty", T=0, d=128, f=128, E=4, k=2, R=2, S=1, fs=128)
+    full = cfg.with_(T=16)
+    inp = inputs.make_inputs(full)
+    layer = make_layer(cfg, inp)
+    logits = torch.empty(0, cfg.E, device=DEV)
+    x = torch.empty(0, cfg.d, dtype=torch.bfloat16, device=DEV)
+    layer.forward_train(logits, x)
+    grads = layer.backward(torch.empty(0, cfg.d, dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    for key in ("dw_gu", "dw_dn", "dsw_gu", "dsw_dn"):
+        assert not grads[key].any(), key
+    for key in ("dw_gu", "dw_dn"):
+        grads[key].fill_(3.0)
+    layer.backward(torch.empty(0, cfg.d, dtype=torch.bfloat16, device=DEV), grads=grads,
+                   accumulate=True)
+    torch.cuda.synchronize()
+    assert bool((grads["dw_gu"] == 3.0).all()) and bool((grads["dw_dn"] == 3.0).all())

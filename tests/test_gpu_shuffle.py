@@ -130,3 +130,18 @@ def test_full_size_pipeline_matches_oracle():
     assert got == oracle.count_local(i2, slot_ref, E, R, home_ref)
     base = oracle.count_local(i2, slot_ref, E, R)
     assert got[0] / got[1] > 2 * base[0] / base[1]   # the shuffle serves far more locally
+
+
+def test_empty_batch():
+    hist = torch.full((8, 8), 5, dtype=torch.int32, device=DEV)
+    e = torch.empty(0, 2, dtype=torch.int32, device=DEV)
+    moe.moe_interlayer_histogram(e, e, 8, hist, 0)
+    out = torch.full((2,), 9, dtype=torch.int64, device=DEV)
+    moe.moe_count_local(e, torch.arange(8, dtype=torch.int32, device=DEV), 8, 4, out)
+    rank_off = torch.full((5,), 9, dtype=torch.int32, device=DEV)
+    perm = torch.empty(0, dtype=torch.int32, device=DEV)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    moe.moe_token_shuffle(torch.empty(0, dtype=torch.int32, device=DEV), 4, perm, rank_off, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    assert not hist.any() and not out.any() and not rank_off.any()
