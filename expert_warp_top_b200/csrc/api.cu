@@ -105,7 +105,7 @@ int get_encode_fn(EncodeTiledFn* fn) {
 
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
               uint32_t box_cols, uint32_t box_rows) {
-  EncodeTiledFn fn;
+  EncodeTiledFn fn = nullptr;
   int rc = get_encode_fn(&fn);
   if (rc) return rc;
   const int esz = dtype == MOE_BF16 ? 2 : 4;
@@ -125,7 +125,7 @@ int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint
 
 int encode_strips(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                   uint32_t box_rows, uint32_t box_strips) {
-  EncodeTiledFn fn;
+  EncodeTiledFn fn = nullptr;
   int rc = get_encode_fn(&fn);
   if (rc) return rc;
   cuuint64_t dims[3] = {64, rows, cols / 64};
