@@ -67,6 +67,14 @@ constexpr bool kRasterNFastest = MOE_RASTER_N_FASTEST != 0;
 #endif
 constexpr bool kWeightsEvictLast = MOE_WEIGHTS_EVICT_LAST != 0;
 
+// The logistic sigmoid of SiLU, 1 / (1 + e^-x), with the fast division
+// (__fdividef: a reciprocal and a multiply).  The IEEE division is a
+// subroutine with a special-case branch, and the epilogues take one per
+// element.  x -> -inf gives 0, x -> +inf gives 1.
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  return __fdividef(1.0f, 1.0f + __expf(-x));
+}
+
 // Shared-memory staging of one epilogue warp: a box of 32 rows x 128 bytes in
 // the 128-byte swizzle, written out by a TMA tensor store.
 constexpr int kEpiBoxBytes = 32 * 128;
@@ -165,6 +173,20 @@ __device__ __forceinline__ void store_row64_bf16(const float* v, bool valid, boo
   }
 }
 
+// kEpiSwiGLUBwd reads, for its row, the saved pre-activations of the tile's BN
+// columns of h: 2 BN contiguous bf16 values (gate and up).  The epilogue warps
+// ask L2 for them one tile ahead, so those loads wait on L2, not on HBM.
+template <int BN, int EPI>
+__device__ __forceinline__ void prefetch_aux_row(const GemmArgs& args, bool valid, size_t grow,
+                                                 int n0) {
+  if constexpr (EPI == kEpiSwiGLUBwd) {
+    if (valid)
+      tc::bulk_prefetch_l2(
+          reinterpret_cast<const __nv_bfloat16*>(args.aux_in) + grow * args.ld_aux + 2 * n0,
+          4 * BN);
+  }
+}
+
 // Epilogue of one accumulator tile for this thread's TMEM lane (= one tile
 // row): tcgen05.ld 32 columns at a time, fused SwiGLU or row scaling, and the
 // row's stores (bf16 SwiGLU / scale: through the warp's staging box and TMA
@@ -198,7 +220,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
           for (int i = 0; i < 32; ++i) {
             gv[i] = round_bf16(__uint_as_float(gr[i]));
             uv[i] = round_bf16(__uint_as_float(ur[i]));
-            hv[i] = gv[i] / (1.0f + __expf(-gv[i])) * uv[i];
+            hv[i] = gv[i] * sigmoid_fast(gv[i]) * uv[i];
           }
           TOut* zg = z + grow * args.ld_aux + n0 + p * 128 + h * 32;
           TOut* dst = out + grow * ldo + (n0 >> 1) + p * 64 + h * 32;
@@ -218,24 +240,48 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
     TOut* dz = reinterpret_cast<TOut*>(args.aux_out);
     const float w = (valid && row_scale) ? row_scale[grow] : 1.0f;
     float dgp = 0.f;
+    // z offset of h column i0 (a multiple of 32): gate and up 64 apart
+    auto z_off = [&](int i0) {
+      return grow * args.ld_aux + (size_t)((i0 >> 6) * 128 + (i0 & 63));
+    };
+    // the saved pre-activations of chunk c + 1 are loaded while chunk c computes
+    uint4 zn[8];
+    if (valid) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        zn[v] = ld_v4(z + z_off(n0) + v * 8);
+        zn[4 + v] = ld_v4(z + z_off(n0) + 64 + v * 8);
+      }
+    }
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       uint32_t vr[32];
       tc::tmem_ld32(taddr + c * 32, vr);
+      uint4 zc[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) zc[v] = zn[v];
+      if (valid && c + 1 < BN / 32) {
+        const size_t zo = z_off(n0 + (c + 1) * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          zn[v] = ld_v4(z + zo + v * 8);
+          zn[4 + v] = ld_v4(z + zo + 64 + v * 8);
+        }
+      }
       tc::tmem_ld_wait();
       if (valid) {
         const int i0 = n0 + c * 32;  // column of h (= of W_down's f axis)
-        const size_t zoff = grow * args.ld_aux + (size_t)((i0 >> 6) * 128 + (i0 & 63));
+        const size_t zoff = z_off(i0);
         float zg[32], zu[32], dg[32], du[32], hg[32];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          Vec16<TOut>::to_f32(ld_v4(z + zoff + v * 8), zg + v * 8);
-          Vec16<TOut>::to_f32(ld_v4(z + zoff + 64 + v * 8), zu + v * 8);
+          Vec16<TOut>::to_f32(zc[v], zg + v * 8);
+          Vec16<TOut>::to_f32(zc[4 + v], zu + v * 8);
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float dh = __uint_as_float(vr[i]);
-          const float sg = 1.0f / (1.0f + __expf(-zg[i]));
+          const float sg = sigmoid_fast(zg[i]);
           const float silu = zg[i] * sg;
           const float hv = round_bf16(silu * zu[i]);
           dgp += dh * hv;
@@ -270,7 +316,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
         for (int i = 0; i < 32; ++i) {
           const float gv = __uint_as_float(gr[i]);
           const float uv = __uint_as_float(ur[i]);
-          hv[h * 32 + i] = gv / (1.0f + __expf(-gv)) * uv;
+          hv[h * 32 + i] = gv * sigmoid_fast(gv) * uv;
         }
       }
       store_row64_bf16(hv, valid, full, grow, wrow0, (n0 >> 1) + p * 64, out, ldo, box, tmap_out);
@@ -306,7 +352,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
           for (int i = 0; i < 32; ++i) {
             const float gv = __uint_as_float(gr[i]);
             const float uv = __uint_as_float(ur[i]);
-            hv[i] = gv / (1.0f + __expf(-gv)) * uv;
+            hv[i] = gv * sigmoid_fast(gv) * uv;
           }
           TOut* dst = out + grow * ldo + (n0 >> 1) + p * 64 + h * 32;
 #pragma unroll
@@ -607,6 +653,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int g, row0, rows, n0;
+      if constexpr (EPI == kEpiSwiGLUBwd) {
+        // this tile's saved rows (first tile only) and the next tile's, into L2
+        for (int t = tile == (int)blockIdx.x ? tile : tile + (int)gridDim.x;
+             t <= tile + (int)gridDim.x && t < total_tiles; t += gridDim.x) {
+          locate(t, g, row0, rows, n0);
+          prefetch_aux_row<BN, EPI>(args, r_in_tile < rows, (size_t)(row0 + r_in_tile), n0);
+        }
+      }
       locate(tile, g, row0, rows, n0);
       // lane 0 waits for the accumulator; the warp then proceeds converged
       bool ok = true;

@@ -243,6 +243,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tempty_local = tc::smem_u32(&tempty_bar[0]);
     for (int tile = pair; tile < total_tiles; tile += n_pairs) {
       int g, row0, gend, n0;
+      if constexpr (EPI == kEpiSwiGLUBwd) {
+        // this tile's saved rows (first tile only) and the next tile's, into L2
+        for (int t = tile == pair ? tile : tile + n_pairs; t <= tile + n_pairs && t < total_tiles;
+             t += n_pairs) {
+          locate(t, g, row0, gend, n0);
+          const int r = row0 + (int)rank * 128 + r_in_half;
+          prefetch_aux_row<BN, EPI>(args, r < gend, (size_t)r, n0);
+        }
+      }
       locate(tile, g, row0, gend, n0);
       bool ok = true;
       if (lane == 0) ok = tc::wait_bounded(tc::smem_u32(&tfull_bar[acc]), acc_phase, wctl);

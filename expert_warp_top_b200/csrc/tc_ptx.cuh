@@ -96,6 +96,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
       : "memory");
 }
 
+// L2 prefetch of a contiguous global range (address and size multiples of 16 bytes).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
 // Tensor store / reduce-add from shared memory (bulk async group of this
 // thread).  Coordinates are never negative here; x * element size is a
 // multiple of 16 bytes.
