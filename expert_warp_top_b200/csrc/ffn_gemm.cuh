@@ -79,7 +79,32 @@ __device__ __forceinline__ float sigmoid_fast(float x) {
 // the 128-byte swizzle, written out by a TMA tensor store.
 constexpr int kEpiBoxBytes = 32 * 128;
 
-template <int BN, bool TF32>
+// Staging boxes per epilogue warp.  The training epilogues write three row
+// pieces per 64 columns of h (gate and up pre-activations or their gradients,
+// and h or w h), so they get three; the others write one.
+#ifndef MOE_STAGE_SAVE_EPI
+#define MOE_STAGE_SAVE_EPI 1
+#endif
+template <int EPI>
+__host__ __device__ constexpr int epi_boxes_per_warp() {
+  return (EPI == kEpiSwiGLUBwd || (EPI == kEpiSwiGLUSave && MOE_STAGE_SAVE_EPI != 0)) ? 3 : 1;
+}
+
+// Shared memory of one GEMM CTA: 1 KB alignment slack, the operand ring, the
+// epilogue boxes of 4 warps, 512 bytes of barriers and the group tables.  The
+// ring takes as many stages (up to 8) as the opt-in limit per CTA on sm_100
+// (227 KB) leaves.
+constexpr int kSmemPerCta = 232448;
+constexpr int kGroupTableBytes = (int)sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
+__host__ __device__ constexpr int ring_stages(int stage_bytes, int boxes_per_warp) {
+  return (kSmemPerCta - 1024 - 512 - kGroupTableBytes - 4 * boxes_per_warp * kEpiBoxBytes) /
+                     stage_bytes > 8
+             ? 8
+             : (kSmemPerCta - 1024 - 512 - kGroupTableBytes - 4 * boxes_per_warp * kEpiBoxBytes) /
+                   stage_bytes;
+}
+
+template <int BN, bool TF32, int EPI>
 struct GemmCfg {
   static constexpr int kElemBytes = TF32 ? 4 : 2;
   static constexpr int kBK = 128 / kElemBytes;       // one 128-byte swizzle row
@@ -88,12 +113,12 @@ struct GemmCfg {
   static constexpr int kABytes = kGemmBM * 128;
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr int kBoxesPerWarp = epi_boxes_per_warp<EPI>();
+  static constexpr int kStages = ring_stages(kStageBytes, kBoxesPerWarp);
   static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;  // a power of two here
-  static constexpr size_t kSmemBytes =
-      1024 /* alignment slack */ + (size_t)kStages * kStageBytes +
-      4 * kEpiBoxBytes /* epilogue staging */ + 256 /* barriers */ +
-      sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes +
+                                       4 * kBoxesPerWarp * kEpiBoxBytes + 512 + kGroupTableBytes;
+  static_assert(kSmemBytes <= (size_t)kSmemPerCta, "GEMM shared memory over the per-CTA limit");
 };
 
 struct GemmArgs {
@@ -195,19 +220,45 @@ __device__ __forceinline__ void prefetch_aux_row(const GemmArgs& args, bool vali
 template <int BN, int EPI, typename TOut>
 __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t grow, int n0,
                                               const GemmArgs& args, uint8_t* box,
-                                              const CUtensorMap* tmap_out) {
+                                              const CUtensorMap* tmap_out,
+                                              const CUtensorMap* tmap_aux) {
   TOut* out = reinterpret_cast<TOut*>(args.out);
   const int ldo = args.ldo;
   const float* row_scale = args.row_scale;
   constexpr bool kBf16 = std::is_same<TOut, __nv_bfloat16>::value;
   const bool full = __all_sync(0xffffffffu, valid);
   const int wrow0 = __shfl_sync(0xffffffffu, (int)grow, 0);  // the warp's rows are consecutive
+  const unsigned lane = lane_id();
+  // The training epilogues stage 64 columns of h at a time in the warp's three
+  // boxes (gate piece, up piece, h piece), as two halves of 32, then write
+  // them with three TMA stores; a warp that straddles a group's end stores
+  // its valid rows directly.  put(b, j, v) writes 16-byte piece j of this
+  // lane's 128-byte row of box b (swizzled).
+  [[maybe_unused]] auto put = [&](int b, int j, const uint4& v) {
+    st_v4(box + b * kEpiBoxBytes + lane * 128 + ((j ^ (lane & 7)) << 4), v);
+  };
+  [[maybe_unused]] auto boxes_free = [&]() {  // the boxes' previous stores have read them
+    if (lane == 0) tc::bulk_wait_read_all();
+    __syncwarp();
+  };
+  [[maybe_unused]] auto store_boxes = [&](int zcol, int hcol) {
+    tc::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tc::tma_store_2d(tmap_aux, tc::smem_u32(box), zcol, wrow0);
+      tc::tma_store_2d(tmap_aux, tc::smem_u32(box + kEpiBoxBytes), zcol + 64, wrow0);
+      tc::tma_store_2d(tmap_out, tc::smem_u32(box + 2 * kEpiBoxBytes), hcol, wrow0);
+      tc::bulk_commit_group();
+    }
+  };
   if constexpr (EPI == kEpiSwiGLUSave) {
     static_assert(std::is_same<TOut, __nv_bfloat16>::value,
                   "the training epilogue is bf16 only");
+    constexpr bool kStaged = epi_boxes_per_warp<EPI>() == 3;
     TOut* z = reinterpret_cast<TOut*>(args.aux_out);
 #pragma unroll 1
     for (int p = 0; p < BN / 128; ++p) {
+      if (kStaged && full) boxes_free();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         uint32_t gr[32], ur[32];
@@ -222,20 +273,31 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
             uv[i] = round_bf16(__uint_as_float(ur[i]));
             hv[i] = gv[i] * sigmoid_fast(gv[i]) * uv[i];
           }
-          TOut* zg = z + grow * args.ld_aux + n0 + p * 128 + h * 32;
-          TOut* dst = out + grow * ldo + (n0 >> 1) + p * 64 + h * 32;
+          if (kStaged && full) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            st_v4(zg + v * 8, Vec16<TOut>::from_f32(gv + v * 8));
-            st_v4(zg + 64 + v * 8, Vec16<TOut>::from_f32(uv + v * 8));
-            st_v4(dst + v * 8, Vec16<TOut>::from_f32(hv + v * 8));
+            for (int v = 0; v < 4; ++v) {
+              put(0, h * 4 + v, Vec16<TOut>::from_f32(gv + v * 8));
+              put(1, h * 4 + v, Vec16<TOut>::from_f32(uv + v * 8));
+              put(2, h * 4 + v, Vec16<TOut>::from_f32(hv + v * 8));
+            }
+          } else {
+            TOut* zg = z + grow * args.ld_aux + n0 + p * 128 + h * 32;
+            TOut* dst = out + grow * ldo + (n0 >> 1) + p * 64 + h * 32;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              st_v4(zg + v * 8, Vec16<TOut>::from_f32(gv + v * 8));
+              st_v4(zg + 64 + v * 8, Vec16<TOut>::from_f32(uv + v * 8));
+              st_v4(dst + v * 8, Vec16<TOut>::from_f32(hv + v * 8));
+            }
           }
         }
       }
+      if (kStaged && full) store_boxes(n0 + p * 128, (n0 >> 1) + p * 64);
     }
   } else if constexpr (EPI == kEpiSwiGLUBwd) {
     static_assert(std::is_same<TOut, __nv_bfloat16>::value,
                   "the training epilogue is bf16 only");
+    static_assert(BN % 64 == 0, "the SwiGLU backward epilogue works in 64-column steps");
     const TOut* z = reinterpret_cast<const TOut*>(args.aux_in);
     TOut* dz = reinterpret_cast<TOut*>(args.aux_out);
     const float w = (valid && row_scale) ? row_scale[grow] : 1.0f;
@@ -269,9 +331,9 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
         }
       }
       tc::tmem_ld_wait();
+      if (full && (c & 1) == 0) boxes_free();
+      const int i0 = n0 + c * 32;  // column of h (= of W_down's f axis)
       if (valid) {
-        const int i0 = n0 + c * 32;  // column of h (= of W_down's f axis)
-        const size_t zoff = z_off(i0);
         float zg[32], zu[32], dg[32], du[32], hg[32];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -290,14 +352,28 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
           du[i] = dhw * silu;
           hg[i] = w * hv;
         }
-        TOut* dst = out + grow * ldo + i0;
+        if (full) {
+          const int jb = (c & 1) * 4;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          st_v4(dz + zoff + v * 8, Vec16<TOut>::from_f32(dg + v * 8));
-          st_v4(dz + zoff + 64 + v * 8, Vec16<TOut>::from_f32(du + v * 8));
-          st_v4(dst + v * 8, Vec16<TOut>::from_f32(hg + v * 8));
+          for (int v = 0; v < 4; ++v) {
+            put(0, jb + v, Vec16<TOut>::from_f32(dg + v * 8));
+            put(1, jb + v, Vec16<TOut>::from_f32(du + v * 8));
+            put(2, jb + v, Vec16<TOut>::from_f32(hg + v * 8));
+          }
+        } else {
+          const size_t zoff = z_off(i0);
+          TOut* dst = out + grow * ldo + i0;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            st_v4(dz + zoff + v * 8, Vec16<TOut>::from_f32(dg + v * 8));
+            st_v4(dz + zoff + 64 + v * 8, Vec16<TOut>::from_f32(du + v * 8));
+            st_v4(dst + v * 8, Vec16<TOut>::from_f32(hg + v * 8));
+          }
         }
       }
+      // after the second half of a 64-column step: gate and up of h columns
+      // [i0 - 32, i0 + 32) sit at z columns 2 (i0 - 32) and 2 (i0 - 32) + 64
+      if (full && (c & 1) == 1) store_boxes(2 * (i0 - 32), i0 - 32);
     }
     if (valid && args.partial) args.partial[grow * args.n_part + n0 / BN] = dgp;
   } else if constexpr (EPI == kEpiSwiGLU && kBf16) {
@@ -425,8 +501,9 @@ template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
-                    const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
-  using Cfg = GemmCfg<BN, TF32>;
+                    const __grid_constant__ CUtensorMap tmap_out,
+                    const __grid_constant__ CUtensorMap tmap_aux, const GemmArgs args) {
+  using Cfg = GemmCfg<BN, TF32, EPI>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
   static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
@@ -436,8 +513,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint8_t* epi_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 x 4 KB, 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_boxes + 4 * kEpiBoxBytes);
+  uint8_t* epi_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 warps' boxes, 1024-aligned
+  constexpr int kWarpBoxBytes = Cfg::kBoxesPerWarp * kEpiBoxBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_boxes + 4 * kWarpBoxBytes);
   uint64_t* full_bar = bars;            // [S]   TMA -> MMA
   uint64_t* empty_bar = bars + S;       // [S]   MMA -> TMA
   uint64_t* tfull_bar = bars + 2 * S;   // [2]   MMA -> epilogue
@@ -445,7 +523,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = bars + 2 * S + 4;   // [1] MMA drain at teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_off = reinterpret_cast<int32_t*>(epi_boxes + 4 * kEpiBoxBytes + 256);
+  int32_t* s_off = reinterpret_cast<int32_t*>(epi_boxes + 4 * kWarpBoxBytes + 512);
   int32_t* s_end = s_off + kGemmMaxGroups;
   int32_t* s_prefix = s_end + kGemmMaxGroups;
 
@@ -673,8 +751,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       const bool valid = r_in_tile < rows;
       const size_t grow = static_cast<size_t>(row0 + r_in_tile);
-      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args, epi_boxes + quarter * kEpiBoxBytes,
-                                   &tmap_out);
+      epilogue_rows<BN, EPI, TOut>(taddr, valid, grow, n0, args, epi_boxes + quarter * kWarpBoxBytes,
+                                   &tmap_out, &tmap_aux);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tc::smem_u32(&tempty_bar[acc]));

@@ -26,7 +26,7 @@ namespace moe {
 
 constexpr int kPairBM = 256;  // rows per pair tile, 128 per CTA
 
-template <int BN, bool TF32>
+template <int BN, bool TF32, int EPI>
 struct PairCfg {
   static constexpr int kElemBytes = TF32 ? 4 : 2;
   static constexpr int kBK = 128 / kElemBytes;
@@ -35,11 +35,12 @@ struct PairCfg {
   static constexpr int kABytes = 128 * 128;          // this CTA's 128 rows of A
   static constexpr int kBBytes = (BN / 2) * 128;     // this CTA's half of B
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
+  static constexpr int kBoxesPerWarp = epi_boxes_per_warp<EPI>();
+  static constexpr int kStages = ring_stages(kStageBytes, kBoxesPerWarp);
   static constexpr int kTmemCols = 2 * BN;
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes +
-                                       4 * kEpiBoxBytes + 512 +
-                                       sizeof(int32_t) * (3 * kGemmMaxGroups + 1);
+                                       4 * kBoxesPerWarp * kEpiBoxBytes + 512 + kGroupTableBytes;
+  static_assert(kSmemBytes <= (size_t)kSmemPerCta, "GEMM shared memory over the per-CTA limit");
 };
 
 // B_MN: B stored MN-major (B[g*K + k][n], n contiguous), seen by tmap_b as
@@ -48,10 +49,11 @@ template <int BN, int EPI, bool TF32, bool B_MN = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b,
-                         const __grid_constant__ CUtensorMap tmap_out, const GemmArgs args) {
+                         const __grid_constant__ CUtensorMap tmap_out,
+                         const __grid_constant__ CUtensorMap tmap_aux, const GemmArgs args) {
   static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
   static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
-  using Cfg = PairCfg<BN, TF32>;
+  using Cfg = PairCfg<BN, TF32, EPI>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
 
@@ -59,8 +61,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint8_t* epi_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 x 4 KB, 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_boxes + 4 * kEpiBoxBytes);
+  uint8_t* epi_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 warps' boxes, 1024-aligned
+  constexpr int kWarpBoxBytes = Cfg::kBoxesPerWarp * kEpiBoxBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_boxes + 4 * kWarpBoxBytes);
   uint64_t* full_bar = bars;                 // [S] CTA 0: both CTAs' TMA -> MMA
   uint64_t* empty_bar = bars + S;            // [S] MMA (multicast) -> producers
   uint64_t* tfull_bar = bars + 2 * S;        // [2] MMA (multicast) -> epilogues
@@ -68,7 +71,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = bars + 2 * S + 4;    // [1] MMA drain at teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_off = reinterpret_cast<int32_t*>(epi_boxes + 4 * kEpiBoxBytes + 512);
+  int32_t* s_off = reinterpret_cast<int32_t*>(epi_boxes + 4 * kWarpBoxBytes + 512);
   int32_t* s_end = s_off + kGemmMaxGroups;
   int32_t* s_prefix = s_end + kGemmMaxGroups;
 
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int grow_i = row0 + (int)rank * 128 + r_in_half;
       const bool valid = grow_i < gend;
       epilogue_rows<BN, EPI, TOut>(taddr, valid, static_cast<size_t>(grow_i), n0, args,
-                                   epi_boxes + quarter * kEpiBoxBytes, &tmap_out);
+                                   epi_boxes + quarter * kWarpBoxBytes, &tmap_out, &tmap_aux);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) {

@@ -152,6 +152,21 @@ inline int encode_out(CUtensorMap* to, const void* out, int dtype, int m_cap, in
                    dtype == MOE_BF16 ? 64 : 32, 32);
 }
 
+// The training epilogues' second output, aux_out [m_cap, ld_aux] (the
+// pre-activations or their gradient), for their TMA stores; the other
+// epilogues never read this map and get a copy of the output's.
+template <int EPI>
+int encode_aux(CUtensorMap* tx, const CUtensorMap& to, const GemmExtra& ex, int dtype, int m_cap) {
+  constexpr bool kTraining = EPI == moe::kEpiSwiGLUSave || EPI == moe::kEpiSwiGLUBwd;
+  MOE_REQUIRE(!kTraining || (ex.aux_out && ex.ld_aux > 0), MOE_ERR_INVALID_ARG,
+              "the training epilogues need their second output");
+  if (!kTraining) {
+    *tx = to;
+    return MOE_OK;
+  }
+  return encode_out(tx, ex.aux_out, dtype, m_cap, ex.ld_aux);
+}
+
 // A is [a_rows, K]; with a_row_index the m_cap rows fed to the GEMM are
 // gathered from it (row p = a[a_row_index[p]]), else they are a's first m_cap.
 template <int BN, int EPI, bool TF32, bool GATHER, bool B_MN>
@@ -159,15 +174,16 @@ int launch_gemm(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_
                 int K, const void* b, int G, int N, const int32_t* group_off,
                 const float* row_scale, void* out, int ldo, const GemmExtra& ex,
                 cudaStream_t st) {
-  using Cfg = moe::GemmCfg<BN, TF32>;
+  using Cfg = moe::GemmCfg<BN, TF32, EPI>;
   const int dtype = TF32 ? MOE_F32 : MOE_BF16;
   CUtensorMap ta, tb;
   int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK,
                      GATHER ? 1u : (uint32_t)moe::kGemmBM);
   if (rc) return rc;
   if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN))) return rc;
-  CUtensorMap to;
+  CUtensorMap to, tx;
   if ((rc = encode_out(&to, out, dtype, m_cap, ldo))) return rc;
+  if ((rc = encode_aux<EPI>(&tx, to, ex, dtype, m_cap))) return rc;
   auto kern = moe::ffn_gemm_kernel<BN, EPI, TF32, GATHER, B_MN>;
   if ((rc = ensure_smem(di, reinterpret_cast<const void*>(kern), Cfg::kSmemBytes))) return rc;
   const long long ub = ((long long)m_cap / moe::kGemmBM + G) * (N / BN);
@@ -175,7 +191,7 @@ int launch_gemm(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_
   const moe::GemmArgs args =
       gemm_args(di, group_off, a_row_index, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
   MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, to,
-                    args));
+                    tx, args));
   MOE_LAUNCHED("ffn_gemm_kernel");
   return MOE_OK;
 }
@@ -200,14 +216,15 @@ template <int BN, int EPI, bool TF32, bool B_MN>
 int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K, const void* b,
                      int G, int N, const int32_t* group_off, const float* row_scale, void* out,
                      int ldo, const GemmExtra& ex, cudaStream_t st) {
-  using Cfg = moe::PairCfg<BN, TF32>;
+  using Cfg = moe::PairCfg<BN, TF32, EPI>;
   const int dtype = TF32 ? MOE_F32 : MOE_BF16;
   CUtensorMap ta, tb;
   int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
   if (rc) return rc;
   if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN / 2))) return rc;
-  CUtensorMap to;
+  CUtensorMap to, tx;
   if ((rc = encode_out(&to, out, dtype, m_cap, ldo))) return rc;
+  if ((rc = encode_aux<EPI>(&tx, to, ex, dtype, m_cap))) return rc;
   auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32, B_MN>;
   const void* key = reinterpret_cast<const void*>(kern);
   cudaLaunchConfig_t cfg = {};
@@ -243,7 +260,7 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   cfg.numAttrs = 2;
   const moe::GemmArgs args =
       gemm_args(di, group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
-  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, to, args));
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, to, tx, args));
   return MOE_OK;
 }
 
