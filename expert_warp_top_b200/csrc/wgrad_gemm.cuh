@@ -13,9 +13,10 @@
 //               seen as {64, rows, cols/64}), 128-byte swizzle
 //   warp 1      MMA issuer (lane 0) and tail fixer (whole warp): in a group's
 //               last, partial row block the rows past the group's end belong
-//               to the next group, so the warp zeroes them in shared memory
-//               (a 128-byte row of a swizzled box holds exactly one row)
-//               before the MMAs read the stage
+//               to the next group, so the MMAs stop at the 16-row block that
+//               holds the group's last row and the warp zeroes that block's
+//               foreign rows in shared memory (a 128-byte row of a swizzled
+//               box holds exactly one row) before the MMAs read the stage
 //   warps 2..5  epilogue: tcgen05.ld of 32 accumulator rows (= 32 values of m),
 //               staged 128 bytes per row (32 fp32 or 64 bf16 columns) into one
 //               of two 128-byte-swizzled shared-memory boxes of this warp
@@ -225,13 +226,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc::fence_after_sync();
         uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
         const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
-        if (valid < Cfg::kBK) {
-          // rows valid..63 of every box belong to another group: zero them
-          const int n16 = (Cfg::kBK - valid) * 8;  // 16-byte pieces per box
-          for (int i = (int)lane; i < kChunks * n16; i += 32) {
-            const int c = i / n16, q = i - c * n16;
-            st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
-          }
+        if (valid % 16 != 0) {
+          // Rows valid.. of every strip belong to another group (or lie past
+          // the tensor).  The MMAs read the stage in 16-row blocks up to the
+          // one holding row valid - 1, so only that block's rows past valid
+          // are zeroed; later rows are never read.
+          const int n16 = (((valid + 15) & ~15) - valid) * 8;  // 16-byte pieces per strip
+          for (int c = 0; c < kChunks; ++c)
+            for (int q = (int)lane; q < n16; q += 32)
+              st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
           tc::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
         }
         __syncwarp();

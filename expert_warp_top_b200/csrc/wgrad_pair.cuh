@@ -202,13 +202,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
         const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
-        if (valid < Cfg::kBK) {
-          // rows valid..63 of this CTA's boxes belong to another group: zero them
-          const int n16 = (Cfg::kBK - valid) * 8;
-          for (int i = (int)lane; i < kChunks * n16; i += 32) {
-            const int c = i / n16, q = i - c * n16;
-            st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
-          }
+        if (valid % 16 != 0) {
+          // rows valid.. of this CTA's strips belong to another group; only
+          // those in the last 16-row block the MMAs read need zeroing
+          const int n16 = (((valid + 15) & ~15) - valid) * 8;
+          for (int c = 0; c < kChunks; ++c)
+            for (int q = (int)lane; q < n16; q += 32)
+              st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
           tc::fence_proxy_async_smem();
         }
         __syncwarp();
