@@ -928,27 +928,36 @@ def placement(cfg, how, dev, logits):
                      "row_reduction_vs_contiguous": 1 - out["histogram"] / out["contiguous"]}
 
 
+# Batches in flight in the end-to-end measurement (one stream, workspace and
+# host output buffer each).  With three, the copies of two batches overlap a
+# third's layer, and the small index and mover kernels of one batch can run
+# beside another's GEMM on the SMs it leaves free.
+E2E_IN_FLIGHT = 3
+
+
 def e2e_host(layer, inp, cfg, args, dev, world):
     """End to end through the host-buffer C entry points: every step copies that
     step's logits and activations from pinned host memory, runs the whole layer
-    and copies y back to pinned host memory (host wall clock).  Two batches are
-    in flight (moe_layer_forward_host_async on two streams with their own
-    workspaces and output buffers), so one batch's copies overlap the other's
-    layer; a stream is synchronised before its buffers are reused and at the
-    end, so every step's y is in host memory inside the timed region.  The
-    fully synchronous moe_layer_forward_host is timed too ("sync")."""
+    and copies y back to pinned host memory (host wall clock).  E2E_IN_FLIGHT
+    batches are in flight (moe_layer_forward_host_async on as many streams,
+    each with its own workspace and output buffer), so batches' copies overlap
+    other batches' layers; a stream is synchronised before its buffers are
+    reused and at the end, so every step's y is in host memory inside the timed
+    region.  The fully synchronous moe_layer_forward_host is timed too
+    ("sync")."""
     import torch.distributed as dist
     h_logits = inp["logits"].cpu().pin_memory()
     h_x = inp["x"].cpu().pin_memory()
-    h_ys = [torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory() for _ in range(2)]
-    wss = [layer.host_workspace() for _ in range(2)]
-    streams = [torch.cuda.Stream(dev) for _ in range(2)]
+    nf = E2E_IN_FLIGHT
+    h_ys = [torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory() for _ in range(nf)]
+    wss = [layer.host_workspace() for _ in range(nf)]
+    streams = [torch.cuda.Stream(dev) for _ in range(nf)]
 
     def pipelined(n):
         for i in range(n):
-            s = streams[i % 2]
-            s.synchronize()  # the batch two steps back: its buffers are free, its y is home
-            layer.forward_host(h_logits, h_x, h_ys[i % 2], stream=s, ws=wss[i % 2],
+            s = streams[i % nf]
+            s.synchronize()  # the batch nf steps back: its buffers are free, its y is home
+            layer.forward_host(h_logits, h_x, h_ys[i % nf], stream=s, ws=wss[i % nf],
                                asynchronous=True)
         for s in streams:
             s.synchronize()
@@ -973,8 +982,8 @@ def e2e_host(layer, inp, cfg, args, dev, world):
     d2h = h_ys[0].numel() * h_ys[0].element_size()
     return {"value": whole_job_tokens_per_s(cfg.T, args.steps, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "api": "moe_layer_forward_host_async (C ABI), two batches in flight on two streams, "
-                   "pinned host buffers, wall clock",
+            "api": f"moe_layer_forward_host_async (C ABI), {nf} batches in flight on {nf} "
+                   "streams, pinned host buffers, wall clock",
             "sync": {"value": whole_job_tokens_per_s(cfg.T, args.steps, world, ms_sync),
                      "api": "moe_layer_forward_host (one batch at a time)"}}
 

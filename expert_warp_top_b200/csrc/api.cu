@@ -244,10 +244,12 @@ size_t brim_scratch_entries(int T, int E, int R) {
   return (n_tiles + 1) * (size_t)(R + E);
 }
 
-// Histogram blocks of the column-scan pass: a few thousand tokens each, so
-// that their shared-memory counts merge into few global atomics.
+// Histogram blocks of the column-scan pass: 512 tokens each.  A block's
+// k^2 shared-memory increments per token are what bound the launch (the
+// column scans are short), so the tokens are spread over several blocks; each
+// block then merges its counts with at most E^2 global atomics.
 int hist_blocks(int T, int* tokens_per_block) {
-  const int per = 2048;
+  const int per = 512;
   *tokens_per_block = per;
   return (T + per - 1) / per;
 }
