@@ -46,7 +46,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_time_and_batches():
     world, port = 2, _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:  # no fork of this threaded process
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
