@@ -399,10 +399,11 @@ int launch_wgrad_pair(DeviceInfo* di, const void* a, const void* b, int rows, in
 template <typename TOut>
 int launch_wgrad(DeviceInfo* di, const void* a, const void* b, int rows, int M, int N,
                  const int32_t* group_off, int G, void* out, int accumulate, cudaStream_t st) {
-  // The CTA-pair kernel moves a third less operand traffic per FLOP but
-  // measured slower on the OLMoE-shaped backward (650 vs 515 us): its
-  // per-stage hand-off between the two CTAs adds latency to a loop that is
-  // bound by load latency.  It is kept, tested, behind kDebugForcePair.
+  // The CTA-pair kernel moves a third less operand traffic per FLOP.  On the
+  // OLMoE-shaped backward it measured level with the single-CTA kernel
+  // (backward expert GEMMs 1.140-1.157 against 1.127-1.128 ms), so the
+  // single-CTA kernel stays the default and the pair is kept, tested, behind
+  // kDebugForcePair.
   const bool pair = M % 256 == 0 && N % 128 == 0 && (g_debug_flags & kDebugForcePair);
   if (pair) {
     if (N % 256 == 0)

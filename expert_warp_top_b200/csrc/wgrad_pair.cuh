@@ -10,17 +10,20 @@
 //
 // Roles, in both CTAs unless noted:
 //   warp 0      TMA producer: this CTA's A strips and B half, into its own
-//               shared memory, completing on its own load barrier
-//   warp 1      waits for its own stage, zeroes the rows past a ragged group's
-//               end in its own boxes, and arrives on CTA 0's ready barrier;
-//               in CTA 0 its lane 0 then waits for both CTAs' arrivals and
-//               issues the pair MMAs, whose commits free the stage in both
-//               CTAs (multicast) and hand the accumulator to both epilogues
+//               shared memory; both CTAs' loads count their bytes on CTA 0's
+//               full barrier, which CTA 0 arms for the pair (no multicast)
+//   warp 1      CTA 0 only: once a stage has landed in both CTAs, zeroes the
+//               foreign rows of a ragged group's last 16-row block in both
+//               CTAs' boxes (the peer's through distributed shared memory),
+//               then its lane 0 issues the pair MMAs, whose commits free the
+//               stage in both CTAs (multicast) and hand the accumulator to
+//               both epilogues
 //   warps 2..5  epilogue of this CTA's 128 accumulator rows, through TMA
 //               stores as in wgrad_gemm.cuh; they arrive on CTA 0's tempty
 //               barrier (remotely from CTA 1)
-// Every wait is bounded; a pair that gives up unwinds, drains its MMAs, meets
-// at a cluster barrier and frees TMEM.
+// No stage needs a per-stage handshake between the CTAs: the full barrier
+// sees both CTAs' bytes.  Every wait is bounded; a pair that gives up unwinds,
+// drains its MMAs, meets at a cluster barrier and frees TMEM.
 #pragma once
 #include "wgrad_gemm.cuh"
 
@@ -35,8 +38,10 @@ struct WgradPairCfg {
   static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kStoreBoxBytes = 32 * 128;
+  static constexpr int kStoreBoxes = 8;             // two per epilogue warp
   static constexpr size_t kSmemBytes =
-      1024 + (size_t)kStages * kStageBytes + 4 * kStoreBoxBytes + 512;
+      1024 + (size_t)kStages * kStageBytes + kStoreBoxes * kStoreBoxBytes + 512;
+  static_assert(kSmemBytes <= 232448, "over the per-CTA shared-memory limit");
 };
 
 // tmap_a: A as 64-column strips, box 64 rows x 2 strips; tmap_b: B as strips,
@@ -56,15 +61,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
-  uint8_t* store_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 4 x 4 KB, 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(store_boxes + 4 * Cfg::kStoreBoxBytes);
-  uint64_t* load_bar = bars;               // [S] this CTA's TMA -> its warp 1
-  uint64_t* ready_bar = bars + S;          // [S] CTA 0: both warps 1 -> MMA issuer
-  uint64_t* empty_bar = bars + 2 * S;      // [S] MMA (multicast) -> producers
-  uint64_t* tfull_bar = bars + 3 * S;      // [2] MMA (multicast) -> epilogues
-  uint64_t* tempty_bar = bars + 3 * S + 2; // [2] CTA 0: 8 epilogue warps -> MMA issuer
-  uint64_t* drain_bar = bars + 3 * S + 4;  // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  uint8_t* store_boxes = smem + (size_t)S * Cfg::kStageBytes;  // 8 x 4 KB, 1024-aligned
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(store_boxes + Cfg::kStoreBoxes * Cfg::kStoreBoxBytes);
+  uint64_t* full_bar = bars;               // [S] CTA 0: both CTAs' TMA -> MMA issuer
+  uint64_t* empty_bar = bars + S;          // [S] MMA (multicast) -> producers
+  uint64_t* tfull_bar = bars + 2 * S;      // [2] MMA (multicast) -> epilogues
+  uint64_t* tempty_bar = bars + 2 * S + 2; // [2] CTA 0: 8 epilogue warps -> MMA issuer
+  uint64_t* drain_bar = bars + 2 * S + 4;  // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -81,8 +86,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tma_prefetch_desc(&tmap_b);
     tc::tma_prefetch_desc(&tmap_out);
     for (int s = 0; s < S; ++s) {
-      tc::mbar_init(tc::smem_u32(&load_bar[s]), 1);
-      tc::mbar_init(tc::smem_u32(&ready_bar[s]), 2);  // one arrival from each CTA
+      tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
       tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -153,13 +157,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           if (!skip_next) {
-            const uint32_t lb = tc::smem_u32(&load_bar[stage]);
+            const uint32_t fb = tc::smem_u32(&full_bar[stage]);
+            const uint32_t fb_pair = tc::mapa_shared(fb, 0);  // the barrier in CTA 0
             uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
             const int y = r0 + kb * Cfg::kBK;
-            tc::mbar_arrive_expect_tx(lb, Cfg::kStageBytes);
-            tc::tma_load_3d(tc::smem_u32(sa), &tmap_a, lb, 0, y, (m0 + (int)rank * 128) / 64, pol);
-            tc::tma_load_3d(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, lb, 0, y,
-                            (n0 + (int)rank * (BN / 2)) / 64, pol);
+            if (rank == 0) tc::mbar_arrive_expect_tx(fb, 2 * Cfg::kStageBytes);
+            tc::tma_load_3d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, 0, y,
+                                 (m0 + (int)rank * 128) / 64, pol);
+            tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0, y,
+                                 (n0 + (int)rank * (BN / 2)) / 64, pol);
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           }
@@ -170,92 +176,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      for (int s = 0; s < S; ++s)
-        if ((armed >> s) & 1u)
-          tc::wait_bounded(tc::smem_u32(&load_bar[s]), (armed_parity >> s) & 1u, wctl, false);
+      // CTA 0 waits for the last arming of every stage (its bytes include CTA 1's)
+      if (rank == 0)
+        for (int s = 0; s < S; ++s)
+          if ((armed >> s) & 1u)
+            tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
     }
   } else if (warp == 1) {
-    // ------------------------------ stage check + tail zeroing; CTA 0: MMA
-    constexpr uint32_t idesc = tc::idesc_f32acc<false, 256, BN, true, true>();
-    const uint32_t ready0 = tc::mapa_shared(tc::smem_u32(&ready_bar[0]), 0);  // in CTA 0
-    int stage = 0;
-    uint32_t phase = 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    bool ok = true;
-    for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
-      int g, m0, n0, r0, r1;
-      locate(tile, g, m0, n0);
-      group_rows(g, r0, r1);
-      const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
-      bool go = true;
-      if (rank == 0 && lane == 0)
-        go = tc::wait_bounded_cluster(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl);
-      if (!__shfl_sync(0xffffffffu, go, 0)) break;
-      tc::fence_after_sync();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int kb = 0; kb < k_blocks; ++kb) {
-        if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&load_bar[stage]), phase, wctl);
-        if (!__shfl_sync(0xffffffffu, go, 0)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
-        const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
-        if (valid % 16 != 0) {
-          // rows valid.. of this CTA's strips belong to another group; only
-          // those in the last 16-row block the MMAs read need zeroing
-          const int n16 = (((valid + 15) & ~15) - valid) * 8;
-          for (int c = 0; c < kChunks; ++c)
-            for (int q = (int)lane; q < n16; q += 32)
-              st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
-          tc::fence_proxy_async_smem();
-        }
-        __syncwarp();
-        if (lane == 0) {
-          const uint32_t rb = ready0 + static_cast<uint32_t>(stage * sizeof(uint64_t));
-          if (rank == 0) tc::mbar_arrive(tc::smem_u32(&ready_bar[stage]));
-          else tc::mbar_arrive_remote(rb);
-        }
-        if (rank == 0 && lane == 0) {
-          go = tc::wait_bounded_cluster(tc::smem_u32(&ready_bar[stage]), phase, wctl);
-          if (go) {
-            tc::fence_after_sync();
-            const uint32_t sa_u = tc::smem_u32(sa);
+    // ------------------------------------ CTA 0: tail zeroing + MMA issuer
+    // (CTA 1's warp 1 has nothing to do after allocating TMEM)
+    if (rank == 0) {
+      constexpr uint32_t idesc = tc::idesc_f32acc<false, 256, BN, true, true>();
+      const uint32_t peer_tiles = tc::mapa_shared(tc::smem_u32(tiles), 1);  // CTA 1's ring
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        int g, m0, n0, r0, r1;
+        locate(tile, g, m0, n0);
+        group_rows(g, r0, r1);
+        const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
+        bool go = true;
+        if (lane == 0)
+          go = tc::wait_bounded_cluster(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl);
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (lane == 0) go = tc::wait_bounded_cluster(tc::smem_u32(&full_bar[stage]), phase, wctl);
+          if (!__shfl_sync(0xffffffffu, go, 0)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t sa_u = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
+          const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
+          if (valid % 16 != 0) {
+            // Rows valid.. of every strip, in both CTAs, belong to another group.
+            // The MMAs read the stage in 16-row blocks up to the one holding row
+            // valid - 1, so only that block's rows past valid are zeroed.  The
+            // full barrier has seen both CTAs' bytes land, so these stores come
+            // after the TMA writes; the proxy fence orders them before the MMAs.
+            const int n16 = (((valid + 15) & ~15) - valid) * 8;  // 16-byte pieces per strip
+            const uint32_t peer = peer_tiles + static_cast<uint32_t>(stage * Cfg::kStageBytes);
+            for (int c = 0; c < kChunks; ++c)
+              for (int q = (int)lane; q < n16; q += 32) {
+                const uint32_t off = static_cast<uint32_t>(c * 8192 + valid * 128 + q * 16);
+                st_v4(tiles + (size_t)stage * Cfg::kStageBytes + off, make_uint4(0u, 0u, 0u, 0u));
+                tc::st_cluster_v4(peer + off, make_uint4(0u, 0u, 0u, 0u));
+              }
+            tc::fence_proxy_async_smem_cluster();
+          }
+          __syncwarp();
+          if (lane == 0) {
             const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
             const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
             const int n_kk = (valid + 15) / 16;
             for (int kk = 0; kk < n_kk; ++kk) {
+              // +16 rows = two 1024-byte atoms = +128 in the address field
               const uint64_t off = static_cast<uint64_t>(kk * 128);
               tc::mma_f16_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
             }
             // frees the stage in both CTAs once these MMAs have read it
             tc::commit_pair_multicast(tc::smem_u32(&empty_bar[stage]), 0x3);
           }
+          __syncwarp();
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
-        if (!__shfl_sync(0xffffffffu, go, 0)) {
-          ok = false;
-          break;
-        }
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
+        if (!ok) break;
+        if (lane == 0)  // also for an empty group
+          tc::commit_pair_multicast(tc::smem_u32(&tfull_bar[acc]), 0x3);
+        __syncwarp();
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
         }
       }
-      if (!ok) break;
-      if (rank == 0 && lane == 0)  // also for an empty group
-        tc::commit_pair_multicast(tc::smem_u32(&tfull_bar[acc]), 0x3);
+      if (lane == 0) {
+        tc::commit_pair_multicast(tc::smem_u32(drain_bar), 0x1);
+        tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
+      }
       __syncwarp();
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
     }
-    if (rank == 0 && lane == 0) {
-      tc::commit_pair_multicast(tc::smem_u32(drain_bar), 0x1);
-      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
@@ -264,8 +271,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int VN = Vec16<TOut>::n;
     constexpr int kCols = 8 * VN;
     const bool tma_path = std::is_same<TOut, float>::value || !args.accumulate;
-    uint8_t* box = store_boxes + quarter * Cfg::kStoreBoxBytes;
-    const uint32_t box_u = tc::smem_u32(box);
+    uint8_t* my_boxes = store_boxes + quarter * 2 * Cfg::kStoreBoxBytes;  // this warp's two
+    int n_stores = 0;
     const uint32_t tempty_local = tc::smem_u32(&tempty_bar[0]);
     TOut* out = reinterpret_cast<TOut*>(args.out);
     for (int tile = pair; tile < total_tiles; tile += n_pairs) {
@@ -300,7 +307,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           if (tma_path) {
-            if (lane == 0) tc::bulk_wait_read_all();
+            // boxes alternate; at most one store (the other box's) may still
+            // be reading when this box is rewritten
+            uint8_t* box = my_boxes + (n_stores & 1) * Cfg::kStoreBoxBytes;
+            const uint32_t box_u = tc::smem_u32(box);
+            if (lane == 0) tc::bulk_wait_read_1();
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -312,6 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               else tc::tma_store_2d(&tmap_out, box_u, n0 + c * kCols, row0);
               tc::bulk_commit_group();
             }
+            ++n_stores;
           } else {
             TOut* p = out + ((size_t)row0 + lane) * args.N + n0 + c * kCols;
 #pragma unroll

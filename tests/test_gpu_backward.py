@@ -346,7 +346,8 @@ def test_layer_backward_full_size_sampled(cfg):
 SKIP_FIRST_LOAD = 1
 
 
-@pytest.mark.parametrize("variant", [FORCE_SINGLE, 0], ids=["single", "pair"])
+@pytest.mark.parametrize("variant", [FORCE_SINGLE, 0, FORCE_PAIR],
+                         ids=["single", "pair", "pair_wgrad"])
 def test_backward_bounded_wait_expires_and_context_survives(variant):
     """A stage that is never loaded makes the backward GEMMs' waits expire:
     MOE_ERR_TIMEOUT comes back through the device flag, and the next call on the
