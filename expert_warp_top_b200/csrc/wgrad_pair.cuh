@@ -28,6 +28,18 @@
 #include "wgrad_gemm.cuh"
 
 namespace moe {
+namespace tc {
+// Proxy fence for generic writes to any CTA's shared memory in the cluster.
+__device__ __forceinline__ void fence_proxy_async_smem_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+// 16-byte store to shared memory of a CTA of this cluster (mapa address).
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, const uint4& v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+}  // namespace tc
 
 template <int BN>
 struct WgradPairCfg {
