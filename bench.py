@@ -57,7 +57,7 @@ TRAIN_METRIC = ("MoE-layer training tokens/s (forward + backward: route, BRIM di
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
 # GEMM launches of one layer step, from one ncu capture (profiles/ffn_gemm_pair_olmoe.md),
 # valid only while the GEMM sources hash to `src`; otherwise reported as null.
-GEMM_TRAFFIC = {"olmoe": {"bytes": 1185.8e6, "src": "6251da83660f68a4"}}
+GEMM_TRAFFIC = {"olmoe": {"bytes": 1185.8e6, "src": "1663b6c94716203e"}}
 
 
 def gemm_src_hash() -> str:

@@ -15,8 +15,11 @@
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma M=128, N=BN, K=16 (8 for
 //               TF32), accumulators double-buffered in TMEM (2 x BN columns)
 //   warps 2..5  epilogue: tcgen05.ld of its 32 TMEM lanes (= 32 tile rows),
-//               fused SwiGLU (GEMM 1) or gate-weight scaling (GEMM 2), masked
-//               row stores (a tile never writes past its group)
+//               fused SwiGLU (GEMM 1) or gate-weight scaling (GEMM 2), or
+//               the training variants below; the warp's 32 rows go through
+//               128-byte-swizzled staging boxes and TMA stores, except in a
+//               warp that straddles its group's end, which stores its valid
+//               rows directly (a tile never writes past its group)
 // Tiles are ordered group by group, N block by N block, M block fastest, and
 // dealt round-robin to the CTAs; the same weight block is then read by
 // neighbouring CTAs at the same time and stays in L2.
