@@ -55,8 +55,8 @@ TRAIN_METRIC = ("MoE-layer training tokens/s (forward + backward: route, BRIM di
                 "GEMMs, combine; input, logit and weight gradients)")
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
-# GEMM launches of one layer step, from one ncu capture (profiles/ffn_gemm_pair_olmoe.md),
-# valid only while the GEMM sources hash to `src`; otherwise reported as null.
+# GEMM launches of one layer step, from one ncu capture of that workload's GEMMs, valid
+# only while the GEMM sources hash to `src`; otherwise reported as null.
 GEMM_TRAFFIC = {"olmoe": {"bytes": 1185.8e6, "src": "1663b6c94716203e"}}
 
 
@@ -74,6 +74,32 @@ def gemm_traffic(cfg):
     return rec["bytes"] if rec and rec["src"] == gemm_src_hash() else None
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+L2_NOTE = "flushed between steps (256 MiB write outside the per-step events)"
+
+
+def config_obj(cfg, args) -> dict:
+    """The workload as both arms print it (one object, the same keys and values)."""
+    mode = "training step" if args.train else "forward"
+    return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} k={cfg.k} "
+                        f"R={cfg.R} S={cfg.S} ({mode})",
+            "T": cfg.T, "d": cfg.d, "f": cfg.f, "E": cfg.E, "k": cfg.k, "R": cfg.R, "S": cfg.S,
+            "fs": cfg.fs, "renorm": cfg.renorm, "activations": cfg.dtype,
+            "placement": args.placement, "prune_m": args.prune, "l2": L2_NOTE,
+            "parallelism": f"{args.gpus} independent replicas"}
+
+
+def host_inputs(cfg, seed=None):
+    """The workload's seeded inputs in host memory.  They are drawn on the GPU
+    when one is present, as the GPU arm draws its own, so that the CPU oracle
+    sees the same values; on a host without a GPU they are drawn there."""
+    if torch.cuda.is_available():
+        dev = torch.device("cuda", torch.cuda.current_device())
+        inp = inputs.make_inputs(cfg, device=dev, seed=seed)
+        out = {k: v.cpu() for k, v in inp.items()}
+        del inp
+        torch.cuda.empty_cache()
+        return out
+    return inputs.make_inputs(cfg, device="cpu", seed=seed)
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -216,12 +242,13 @@ def train_launches_per_step(cfg) -> int:
     return n
 
 
-def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
+def cpu_baseline(cfg, budget_s: float = 12.0, inp=None, slot_of=None):
     """The oracle as it stands, on a bounded sample of the same workload's tokens:
-    routing + BRIM build + the dense layer on the sampled tokens."""
+    routing + BRIM build (under the run's placement) + the dense layer on the
+    sampled tokens."""
     import oracle
     if inp is None:
-        inp = inputs.make_inputs(cfg, device="cpu", weights=True)
+        inp = host_inputs(cfg)
 
     def bits(t):
         t = t.contiguous()
@@ -231,7 +258,8 @@ def cpu_baseline(cfg, budget_s: float = 12.0, inp=None):
     x = bits(inp["x"])
     wg, wu, wd = bits(inp["wg"]), bits(inp["wu"]), bits(inp["wd"])
     shared = (bits(inp["sg"]), bits(inp["su"]), bits(inp["sd"])) if cfg.S else None
-    slot_of = np.arange(cfg.E, dtype=np.int32)
+    slot_of = (np.arange(cfg.E, dtype=np.int32) if slot_of is None
+               else np.ascontiguousarray(np.asarray(slot_of, dtype=np.int32)))
     order = np.random.default_rng(0).permutation(cfg.T).astype(np.int32)
     n, total_t, total_n = 8, 0.0, 0
     while total_t < budget_s and total_n < cfg.T:
@@ -256,7 +284,7 @@ def cpu_baseline_train(cfg, budget_s: float = 12.0, inp=None):
     gradient, shared experts included) on the first n tokens as a batch."""
     import oracle
     if inp is None:
-        inp = inputs.make_inputs(cfg, device="cpu", weights=True)
+        inp = host_inputs(cfg)
 
     def bits(t):
         t = t.contiguous()
@@ -291,6 +319,20 @@ def cpu_baseline_train(cfg, budget_s: float = 12.0, inp=None):
                       f"gradient), {total_t:.1f} s"}
 
 
+def oracle_placement(cfg, how):
+    """slot_of of the run's placement, computed by the oracle: contiguous, or the
+    greedy correlated placement from the co-activation histogram of the same
+    calibration batch the GPU arm uses (T = 32768, seed 1)."""
+    import oracle
+    if how == "contiguous":
+        return np.arange(cfg.E, dtype=np.int32)
+    calib = cfg.with_(T=32768, seed=1)
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
+    logits = inputs.make_logits(calib, device=dev).cpu().numpy()
+    idx, _ = oracle.route(logits, calib.k, 0)
+    return oracle.place_greedy(oracle.coact_histogram(idx, cfg.E), cfg.R)
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -298,9 +340,13 @@ def run_reference(args, cfg):
     import oracle
     per_step = []
     budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
-    inp = inputs.make_inputs(cfg, device="cpu", weights=True)
+    inp = host_inputs(cfg)
+    slot_of = None if args.train else oracle_placement(cfg, args.placement)
     for i in range(args.warmup + args.steps):
-        res = (cpu_baseline_train if args.train else cpu_baseline)(cfg, budget_s=budget, inp=inp)
+        if args.train:
+            res = cpu_baseline_train(cfg, budget_s=budget, inp=inp)
+        else:
+            res = cpu_baseline(cfg, budget_s=budget, inp=inp, slot_of=slot_of)
         if i >= args.warmup:
             per_step.append(res)
     value = statistics.median([r["value"] for r in per_step])
@@ -310,8 +356,7 @@ def run_reference(args, cfg):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * cfg.T / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "f": cfg.f, "E": cfg.E,
-                   "k": cfg.k, "R": cfg.R, "S": cfg.S},
+        "config": config_obj(cfg, args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": per_step[-1]["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -336,6 +381,9 @@ def run_ours(args, cfg):
                                 device_id=dev)
     # each rank: its own independent batch (seed offset by rank), same weights recipe
     inp = inputs.make_inputs(cfg, device=dev, seed=rank_seed(cfg, rank))
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    # the CPU baseline reads these very inputs, copied to host memory
+    host_inp = {k_: v.cpu() for k_, v in inp.items()} if want_cpu else None
     slot_of, placement_info = placement(cfg, args.placement, dev, inp["logits"])
     kw = dict(wg=inp.pop("wg"), wu=inp.pop("wu"), wd=inp.pop("wd"))
     if cfg.S:
@@ -434,16 +482,34 @@ def run_ours(args, cfg):
     status = B.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
+    # The routed-expert GEMMs again, alone in a graph of their own (no event
+    # nodes between them and their neighbours), on the same EPD rows: the
+    # in-step figure above against this one shows what the step's event nodes
+    # and neighbours cost the GEMMs.
+    g_ffn = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ffn, stream=side):
+        part_b()
+    torch.cuda.synchronize(dev)
+    ffn_own_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        s0.record(stream)
+        g_ffn.replay()
+        s1.record(stream)
+        s1.synchronize()
+        ffn_own_ms.append(s0.elapsed_time(s1))
+    del g_ffn
     total_ms = max_over_ranks(float(sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
     value = whole_job_tokens_per_s(cfg.T, args.steps, world, total_ms)
 
     # end to end through the public API: host buffers in and out, copies timed
     e2e = None
-    try:
-        e2e = e2e_host(layer, inp, cfg, args, dev, world)
-    except Exception as exc:  # noqa: BLE001 -- reported, never hidden
-        e2e = {"value": None, "unit": UNIT, "error": str(exc)[:200]}
+    if not args.no_e2e:
+        try:
+            e2e = e2e_host(layer, inp, cfg, args, dev, world)
+        except Exception as exc:  # noqa: BLE001 -- reported, never hidden
+            e2e = {"value": None, "unit": UNIT, "error": str(exc)[:200]}
 
     pk = peaks()
     flops, bytes_ = algorithmic_work(cfg, c_t, e_act)
@@ -470,19 +536,17 @@ def run_ours(args, cfg):
                  "traffic": gemm_traffic(cfg)})
     layer_roof_s = max(flops / (pk["bf16_sust"] * 1e12), bytes_ / (pk["hbm"] * 1e9))
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(cfg)
+    if want_cpu:
+        cpu = cpu_baseline(cfg, inp=host_inp, slot_of=slot_of.cpu().numpy())
+        cpu["inputs"] = "the GPU arm's own inputs, copied to host memory"
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} "
-                                   f"k={cfg.k} R={cfg.R} S={cfg.S}",
-                       "placement": placement_info, "l2": "flushed between steps "
-                       "(256 MiB write outside the per-step events)",
-                       "parallelism": f"{world} independent replicas"},
+            "config": config_obj(cfg, args),
+            "placement": placement_info,
             "roofline": roof,
             "layer_roofline": {"t_roof_ms": layer_roof_s * 1e3, "frac": layer_roof_s * 1e3 /
                                ms_per_step, "flops": flops, "bytes": bytes_},
@@ -491,6 +555,7 @@ def run_ours(args, cfg):
             "clocks": clocks.summary(),
             "gpu_launches": launches_per_step(cfg) * args.steps,
             "ffn_ms": statistics.mean(ffn_ms),
+            "ffn_own_graph_ms": statistics.mean(ffn_own_ms),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -515,6 +580,8 @@ def run_train(args, cfg):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     inp = inputs.make_inputs(cfg, device=dev, seed=rank_seed(cfg, rank))
+    host_inp = ({k_: v.cpu() for k_, v in inp.items()}
+                if rank == 0 and world == 1 and not args.no_cpu_baseline else None)
     kw = dict(wg=inp.pop("wg"), wu=inp.pop("wu"), wd=inp.pop("wd"))
     if cfg.S:
         kw.update(sg=inp.pop("sg"), su=inp.pop("su"), sd=inp.pop("sd"))
@@ -669,8 +736,9 @@ def run_train(args, cfg):
                       "with fp32 output, 1 gate-gradient row sum)",
             "algorithmic_flops": bwd_flops, "traffic": None}
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_train(cfg)
+    if host_inp is not None:
+        cpu = cpu_baseline_train(cfg, inp=host_inp)
+        cpu["inputs"] = "the GPU arm's own inputs, copied to host memory"
     if rank == 0:
         n_launch = train_launches_per_step(cfg)
         line = {
@@ -678,11 +746,8 @@ def run_train(args, cfg):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} "
-                                   f"k={cfg.k} R={cfg.R} S={cfg.S} (training step)",
-                       "dw_dtype": "fp32", "placement": "contiguous",
-                       "l2": "flushed between steps (256 MiB write outside the per-step events)",
-                       "parallelism": f"{world} independent replicas"},
+            "config": config_obj(cfg, args),
+            "dw_dtype": "fp32",
             "roofline": roof,
             "step_flops": step_flops,
             "step_tflops": step_flops / (ms_per_step * 1e-3) / 1e12,
@@ -893,14 +958,13 @@ def run_shuffle(args, cfg):
 
 
 def placement(cfg, how, dev, logits):
-    """slot_of for the run.  "histogram": correlated placement from the expert
-    co-activation histogram of a separate calibration batch (T = 32768, seed 1),
-    routed and counted on the GPU, placed by moe_place_greedy; reports the C_T
-    of the evaluation batch under contiguous and under this placement."""
+    """slot_of for the run ("contiguous", or "histogram": correlated placement
+    from the expert co-activation histogram of a separate calibration batch,
+    T = 32768, seed 1, routed and counted on the GPU and placed by
+    moe_place_greedy), and the C_T of the evaluation batch under both
+    placements (the counter kernel), whichever the run uses."""
     from expert_warp_top_b200 import _binding as B
     ident = torch.arange(cfg.E, dtype=torch.int32)
-    if how == "contiguous":
-        return ident, "contiguous"
     calib = cfg.with_(T=32768, seed=1)
     c_logits = inputs.make_logits(calib, device=dev)
     idx = torch.empty(calib.T, calib.k, dtype=torch.int32, device=dev)
@@ -908,8 +972,7 @@ def placement(cfg, how, dev, logits):
     B.moe_route_topk(c_logits, calib.k, 0, idx, w)
     hist = torch.zeros(cfg.E, cfg.E, dtype=torch.int32, device=dev)
     B.moe_coact_histogram(idx, cfg.E, hist, 0)
-    slot_of = B.moe_place_greedy(hist, cfg.R)
-    # C_T of the evaluation batch under both placements (the counter kernel)
+    slot_hist = B.moe_place_greedy(hist, cfg.R)
     e_idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
     e_w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
     B.moe_route_topk(logits, cfg.k, cfg.renorm, e_idx, e_w)
@@ -917,15 +980,17 @@ def placement(cfg, how, dev, logits):
     tot = torch.empty(1, dtype=torch.int64, device=dev)
     rem = torch.empty(1, dtype=torch.int64, device=dev)
     out = {}
-    for name, s in (("contiguous", ident), ("histogram", slot_of)):
+    for name, s in (("contiguous", ident), ("histogram", slot_hist)):
         B.moe_count_dispatched_rows(e_idx, s.to(dev), cfg.E, cfg.R, per, tot, rem)
         out[name] = int(tot.item())
     tk = cfg.T * cfg.k
-    return slot_of, {"placement": "histogram (calibration batch T=32768, seed 1)",
-                     "c_t_contiguous": out["contiguous"], "c_t_histogram": out["histogram"],
-                     "tk_rows": tk,
-                     "row_reduction_vs_per_expert": 1 - out["histogram"] / tk,
-                     "row_reduction_vs_contiguous": 1 - out["histogram"] / out["contiguous"]}
+    info = {"used": how if how == "contiguous" else
+            "histogram (calibration batch T=32768, seed 1)",
+            "c_t_contiguous": out["contiguous"], "c_t_histogram": out["histogram"],
+            "tk_rows": tk,
+            "histogram_row_reduction_vs_per_expert": 1 - out["histogram"] / tk,
+            "histogram_row_reduction_vs_contiguous": 1 - out["histogram"] / out["contiguous"]}
+    return (ident if how == "contiguous" else slot_hist), info
 
 
 # Batches in flight in the end-to-end measurement (one stream, workspace and
@@ -993,9 +1058,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="olmoe", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--config", default="corr_prefill", choices=sorted(inputs.CONFIGS),
+                    help="workload (default: the correlated-routing prefill layer, T=32768, "
+                         "d=4096, f=2048, E=64, k=6, R=8: the largest one-GPU workload)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) measurement, e.g. under a profiler")
     ap.add_argument("--placement", default="contiguous", choices=["contiguous", "histogram"])
     ap.add_argument("--shuffle", action="store_true",
                     help="time token shuffling across two layers (correlated prefill workload)")
@@ -1012,7 +1081,7 @@ def main():
     elif args.train:
         run_train(args, cfg)
     elif args.shuffle:
-        run_shuffle(args, cfg if args.config != "olmoe" else inputs.CONFIGS["corr_prefill"])
+        run_shuffle(args, cfg)
     else:
         run_ours(args, cfg)
 

@@ -21,6 +21,13 @@
 
 // The device error flag the kernels raise (bits moe::kErrIndex, kErrTimeout).
 __device__ unsigned g_moe_err_flag;
+// moe_get_device_status's reading of the flag, taken and cleared in one step.
+__device__ unsigned g_moe_err_snapshot;
+
+__global__ void take_error_flag_kernel() {
+  moe::pdl_enter();
+  g_moe_err_snapshot = atomicExch(&g_moe_err_flag, 0u);
+}
 
 // Fixed scratch of moe_brim_build_noalloc (1 MiB, held by every GPU that loads
 // this library until the process exits).
@@ -34,6 +41,7 @@ thread_local char g_msg[512];
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 }  // namespace
+std::mutex g_status_mu;
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -276,11 +284,17 @@ int moe_get_device_status(moe_stream_t stream) {
   DeviceInfo* di;
   int rc = device_info(&di);
   if (rc) return rc;
-  MOE_CUDA(cudaStreamSynchronize(stream));
+  // One atomic exchange on the device reads the flag and clears it, ordered
+  // after the stream's earlier work: a bit that a kernel on another stream
+  // raises at any moment is either in this reading or left for the next one.
+  // The host lock keeps two callers from sharing the snapshot word.
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  MOE_CUDA(launch_k(take_error_flag_kernel, 1, 1, 0, stream));
+  MOE_LAUNCHED("take_error_flag_kernel");
   unsigned v = 0;
-  MOE_CUDA(cudaMemcpyFromSymbol(&v, g_moe_err_flag, sizeof v));
-  const unsigned zero = 0;
-  MOE_CUDA(cudaMemcpyToSymbol(g_moe_err_flag, &zero, sizeof zero));
+  MOE_CUDA(cudaMemcpyFromSymbolAsync(&v, g_moe_err_snapshot, sizeof v, 0,
+                                     cudaMemcpyDeviceToHost, stream));
+  MOE_CUDA(cudaStreamSynchronize(stream));
   if (v & moe::kErrTimeout) return fail(MOE_ERR_TIMEOUT, "a bounded device wait expired");
   if (v & moe::kErrIndex) return fail(MOE_ERR_DEVICE_CHECK, "a kernel met an out-of-range index");
   return MOE_OK;
@@ -331,7 +345,6 @@ int moe_brim_build(const int32_t* topk_idx, const float* topk_w, int T, int k,
   return brim_passes(topk_idx, topk_w, T, k, slot_of, E, R, brim0, sfd_token, sfd_off, brim1,
                      epd_off, epd_sfd, epd_gate, c_t, static_cast<uint32_t*>(ws), di->err_flag,
                      stream);
-  return MOE_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -367,7 +380,6 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
   return brim_passes(topk_idx, topk_w, T, k, slot_of, E, R, brim0, sfd_token, sfd_off, brim1,
                      epd_off, epd_sfd, epd_gate, c_t, reinterpret_cast<uint32_t*>(counts),
                      di->err_flag, stream);
-  return MOE_OK;
 }
 
 // ---------------------------------------------------------------------------

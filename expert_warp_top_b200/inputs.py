@@ -4,7 +4,8 @@ This module draws random numbers and nothing else: it holds none of the
 layer's arithmetic (no routing, no softmax, no re-indexing, no FFN).  Both
 the CUDA path and the CPU oracle are fed from it, so the two see the same
 bits.  The shapes and value distributions follow the workloads the layer is
-measured on; the design doc lists the recipe.
+measured on: the configurations in CONFIGS below, with the distributions
+their fields name.
 
 All draws come from one ``torch.Generator`` seeded per call, in a fixed
 order: logits (+ per-expert bias, + planted-group boosts), activations,

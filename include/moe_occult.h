@@ -84,8 +84,11 @@ const char* moe_last_error(void);
  * wide; not for production use. */
 int moe_set_debug(int flags, double wait_limit_ms);
 
-/* Synchronises `stream`, then reads and clears the device error flag that the
- * kernels raise.  Returns MOE_ERR_TIMEOUT if a bounded wait expired,
+/* Reads and clears the device error flag that the kernels raise, in one
+ * atomic exchange enqueued on `stream` after its earlier work, then
+ * synchronises `stream`.  Kernels still running on other streams may raise the
+ * flag at any time; such a bit is never lost, it shows in this reading or in
+ * the next one.  Returns MOE_ERR_TIMEOUT if a bounded wait expired,
  * MOE_ERR_DEVICE_CHECK if an index was out of range, else MOE_OK. */
 int moe_get_device_status(moe_stream_t stream);
 

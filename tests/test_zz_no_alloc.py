@@ -100,3 +100,52 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
                                     null, ctypes.c_void_p(8), null, null, ctypes.c_void_p(8), null)
     assert rc == moe.MOE_ERR_UNSUPPORTED
     assert b"1 MiB" in lib.moe_last_error()
+
+
+def test_noalloc_empty_batch_clears_offsets():
+    """T = 0: no token is sent, so every offset and C_T is zero (the fixed
+    scratch is not touched)."""
+    lib = moe.load()
+    E, R, k = 64, 8, 6
+    i32 = dict(dtype=torch.int32, device=DEV)
+    sfd_off = torch.full((R + 1,), -9, **i32)
+    epd_off = torch.full((E + 1,), -9, **i32)
+    c_t = torch.full((1,), -9, **i32)
+    one = torch.zeros(1, **i32)
+    onef = torch.zeros(1, dtype=torch.float32, device=DEV)
+    slot_of = torch.arange(E, **i32)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = lib.moe_brim_build_noalloc(_p(one), _p(onef), 0, k, _p(slot_of), E, R, _p(one), _p(one),
+                                    _p(sfd_off), _p(one), _p(epd_off), _p(one), _p(onef), _p(c_t),
+                                    stream)
+    assert rc == moe.MOE_OK, lib.moe_last_error()
+    torch.cuda.synchronize()
+    assert int(sfd_off.abs().sum()) == 0 and int(epd_off.abs().sum()) == 0
+    assert int(c_t.item()) == 0
+
+
+def test_noalloc_at_the_exact_limit_and_one_tile_past_it():
+    """The largest batch the fixed scratch holds for E = 64, R = 8:
+    (ceil(T/32) + 1) * (R + E) <= 262144 gives T = 116448 (262080 entries).
+    It must match the workspace version bit for bit; one 32-token tile more
+    (262152 entries) must be refused."""
+    lib = moe.load()
+    E, R, k = 64, 8, 6
+    T = 116448
+    assert (-(-T // 32) + 1) * (R + E) <= 1 << 18 < (-(-(T + 32) // 32) + 1) * (R + E)
+    cfg = inputs.LayerConfig("limit", T=T, d=64, f=64, E=E, k=k, R=R, seed=13)
+    logits = inputs.make_logits(cfg, device=DEV)
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(logits, k, 0, idx, w)
+    slot_of = torch.randperm(E, generator=torch.Generator().manual_seed(13)).to(torch.int32).to(DEV)
+    o = _outputs(T, E, k, R)
+    assert _noalloc_call(lib, idx, w, slot_of, E, R, o) == moe.MOE_OK, lib.moe_last_error()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == moe.MOE_OK
+    _same(o, _reference(idx, w, slot_of, E, R))
+    null = ctypes.c_void_p(0)
+    rc = lib.moe_brim_build_noalloc(null, null, T + 32, k, ctypes.c_void_p(8), E, R, null, null,
+                                    ctypes.c_void_p(8), null, ctypes.c_void_p(8), null, null,
+                                    ctypes.c_void_p(8), null)
+    assert rc == moe.MOE_ERR_UNSUPPORTED
