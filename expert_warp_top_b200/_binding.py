@@ -39,7 +39,7 @@ EXPORTS = (
     "moe_route_backward", "moe_layer_train_workspace_size", "moe_layer_forward_train",
     "moe_layer_backward", "moe_interlayer_histogram", "moe_rank_affinity", "moe_predict_home",
     "moe_count_local", "moe_token_shuffle_workspace_size", "moe_token_shuffle",
-    "moe_layer_forward_host_async",
+    "moe_layer_forward_host_async", "moe_ep_pack_routing", "moe_ep_return_rows", "moe_ep_combine",
 )
 
 
@@ -237,6 +237,32 @@ def moe_combine_scatter(o_epd, T, k, R, L, brim0, brim1, shared_out, y_sfd, y, s
         _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"),
         _ptr(shared_out, o_epd.dtype, "shared_out"), _ptr(y_sfd, o_epd.dtype, "y_sfd"),
         _ptr(y, o_epd.dtype, "y"), _stream(stream)))
+
+
+def moe_ep_pack_routing(topk_idx, topk_w, slot_of, E, R, sfd_token, sfd_off, c_t, idx_send,
+                        w_send, stream=None):
+    T, k = topk_idx.shape
+    _check("moe_ep_pack_routing", load().moe_ep_pack_routing(
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"), T, k,
+        _ptr(slot_of, I32, "slot_of"), int(E), int(R), _ptr(sfd_token, I32, "sfd_token"),
+        _ptr(sfd_off, I32, "sfd_off"), _ptr(c_t, I32, "c_t"), _ptr(idx_send, I32, "idx_send"),
+        _ptr(w_send, F32, "w_send"), _stream(stream)))
+
+
+def moe_ep_return_rows(o_epd, T, k, R, L, brim0, brim1, y_ret, stream=None):
+    d = o_epd.shape[1]
+    _check("moe_ep_return_rows", load().moe_ep_return_rows(
+        _ptr(o_epd, _ACT, "o_epd"), int(T), d, dtype_code(o_epd.dtype), int(k), int(R), int(L),
+        _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"), _ptr(y_ret, o_epd.dtype, "y_ret"),
+        _stream(stream)))
+
+
+def moe_ep_combine(y_ret, T, k, R, brim0, shared_out, y, stream=None):
+    d = y_ret.shape[1]
+    _check("moe_ep_combine", load().moe_ep_combine(
+        _ptr(y_ret, _ACT, "y_ret"), int(T), d, dtype_code(y_ret.dtype), int(k), int(R),
+        _ptr(brim0, I32, "brim0"), _ptr(shared_out, y_ret.dtype, "shared_out"),
+        _ptr(y, y_ret.dtype, "y"), _stream(stream)))
 
 
 def moe_count_dispatched_rows(topk_idx, slot_of, E, R, per_rank, total, remote, stream=None):

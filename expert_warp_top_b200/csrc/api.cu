@@ -14,6 +14,7 @@
 #include "../../include/moe_occult.h"
 #include "brim.cuh"
 #include "dispatch.cuh"
+#include "ep.cuh"
 #include "host.h"
 #include "route.cuh"
 #include "route_brim.cuh"
@@ -700,6 +701,98 @@ int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R
 #undef MOE_COMBINE
   MOE_LAUNCHED("combine_kernel");
   return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Real expert parallelism: the device steps around the all-to-all exchanges.
+int moe_ep_pack_routing(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                        const int32_t* slot_of, int E, int R, const int32_t* sfd_token,
+                        const int32_t* sfd_off, const int32_t* c_t, int32_t* idx_send,
+                        float* w_send, moe_stream_t stream) {
+  int rc = check_common(T, E, k, R);
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(topk_idx && topk_w && slot_of && sfd_token && sfd_off && c_t && idx_send && w_send,
+              MOE_ERR_INVALID_ARG, "null pointer");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  const long long cap = (long long)T * (k < R ? k : R);
+  long long blocks = (cap + 255) / 256;
+  if (blocks > 8LL * di->num_sms) blocks = 8LL * di->num_sms;
+  MOE_CUDA(launch_k(moe::ep_pack_routing_kernel, (int)blocks, 256, 0, stream, topk_idx, topk_w,
+                    T, k, slot_of, E, R, E / R, sfd_token, sfd_off, c_t, cap, idx_send, w_send,
+                    di->err_flag));
+  MOE_LAUNCHED("ep_pack_routing_kernel");
+  return MOE_OK;
+}
+
+namespace {
+// The combine kernel for the EP entry points: y_sfd only (y == NULL), or the
+// returned rows summed into y (brim1 == NULL, L == 1, rows = the SFD rows).
+int launch_combine(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                   size_t cap, int tk, const int32_t* brim0, const int32_t* brim1,
+                   const void* shared_out, void* y_sfd, void* y, cudaStream_t stream) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  const int P = mover_parts(di, T, (d * esize(dtype) + 511) / 512);
+  const long long warps = (long long)T * P;
+  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
+#define MOE_COMBINE(TA, KM)                                                                    \
+  MOE_CUDA(launch_k(moe::combine_kernel<TA, KM>, blocks, moe::kMoverWarps * 32, 0, stream,     \
+      static_cast<const TA*>(o_epd), T, d, P, R, L, cap, tk, brim0, brim1,                     \
+      static_cast<const TA*>(shared_out), static_cast<TA*>(y_sfd), static_cast<TA*>(y),        \
+      di->err_flag))
+  if (dtype == MOE_BF16) {
+    using B = __nv_bfloat16;
+    if (k <= 2) MOE_COMBINE(B, 2);
+    else if (k <= 4) MOE_COMBINE(B, 4);
+    else if (k <= 8) MOE_COMBINE(B, 8);
+    else MOE_COMBINE(B, 16);
+  } else {
+    if (k <= 2) MOE_COMBINE(float, 2);
+    else if (k <= 4) MOE_COMBINE(float, 4);
+    else if (k <= 8) MOE_COMBINE(float, 8);
+    else MOE_COMBINE(float, 16);
+  }
+#undef MOE_COMBINE
+  MOE_LAUNCHED("combine_kernel");
+  return MOE_OK;
+}
+}  // namespace
+
+int moe_ep_return_rows(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                       const int32_t* brim0, const int32_t* brim1, void* y_ret,
+                       moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= moe::kMaxK && R >= 1 && L >= 1 && R * L <= moe::kMaxE,
+              MOE_ERR_UNSUPPORTED, "bad shape (T=%d k=%d R=%d L=%d)", T, k, R, L);
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(o_epd && brim0 && brim1 && y_ret, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(o_epd) && aligned16(y_ret), MOE_ERR_INVALID_ARG,
+              "row buffers must be 16-byte aligned");
+  const size_t cap = (size_t)T * (k < R ? k : R);
+  return launch_combine(o_epd, T, d, dtype, k, R, L, cap, T * k, brim0, brim1, nullptr, y_ret,
+                        nullptr, stream);
+}
+
+int moe_ep_combine(const void* y_ret, int T, int d, int dtype, int k, int R,
+                   const int32_t* brim0, const void* shared_out, void* y, moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= moe::kMaxK && R >= 1 && R <= moe::kMaxE,
+              MOE_ERR_UNSUPPORTED, "bad shape (T=%d k=%d R=%d)", T, k, R);
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(y_ret && brim0 && y, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(y_ret) && aligned16(y) && aligned16(shared_out), MOE_ERR_INVALID_ARG,
+              "row buffers must be 16-byte aligned");
+  const int kr = k < R ? k : R;  // at most this many ranks per token
+  const size_t cap = (size_t)T * kr;
+  return launch_combine(y_ret, T, d, dtype, kr, R, 1, cap, (int)cap, brim0, nullptr, shared_out,
+                        nullptr, y, stream);
 }
 
 // ---------------------------------------------------------------------------

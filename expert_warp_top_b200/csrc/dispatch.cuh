@@ -36,7 +36,9 @@ struct WarpDst {
 
 // Reads token t's BRIM_0 column and, for every (rank, local expert) slot, its
 // BRIM_1 entry; ballots keep ascending order.  Out-of-range entries raise the
-// error flag and are dropped.
+// error flag and are dropped.  A null brim1 stands for one "expert" per rank
+// whose row is the SFD row itself (p = s; L must be 1): the rows a source rank
+// gets back from its destinations under real expert parallelism.
 __device__ __forceinline__ void collect_dst(const int32_t* __restrict__ brim0,
                                             const int32_t* __restrict__ brim1, int t, int T,
                                             int R, int L, size_t cap, int tk, WarpDst& w,
@@ -67,7 +69,7 @@ __device__ __forceinline__ void collect_dst(const int32_t* __restrict__ brim0,
     if (q < E) {
       const int r = q / L, l = q - r * L;
       s = __ldg(brim0 + (size_t)r * T + t);
-      if (s >= 0 && s < (int)cap) p = __ldg(brim1 + (size_t)l * cap + s);
+      if (s >= 0 && s < (int)cap) p = brim1 ? __ldg(brim1 + (size_t)l * cap + s) : s;
       if (p >= tk) {
         bad = true;
         p = -1;
@@ -140,7 +142,9 @@ __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
 
 // y_sfd[s] = sum_l o_epd[BRIM_1[l][s]] (fp32, rounded to TA); y[t] = sum_r y_sfd[..]
 // (+ shared[t]).  y sums the rounded payload rows, exactly as if it had read
-// them back.  One warp per token (or 1/P of its row); the k expert rows of the
+// them back.  A null y leaves only the return rows y_sfd (the destination
+// side of real expert parallelism); a null brim1 sums rows already reduced
+// per rank (see collect_dst).  One warp per token (or 1/P of its row); the k expert rows of the
 // next 512-byte slice are loaded while the current slice is summed, so up to
 // 2k loads are in flight per warp.  KMAX >= k bounds the register arrays.
 template <typename TA, int KMAX>
@@ -207,13 +211,15 @@ __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
           }
         }
       }
-      if (shared_out) {
-        float f[VN];
-        Vec16<TA>::to_f32(ld_nc_v4(shared_out + (size_t)t * d + c), f);
+      if (y) {
+        if (shared_out) {
+          float f[VN];
+          Vec16<TA>::to_f32(ld_nc_v4(shared_out + (size_t)t * d + c), f);
 #pragma unroll
-        for (int e = 0; e < VN; ++e) ya[e] += f[e];
+          for (int e = 0; e < VN; ++e) ya[e] += f[e];
+        }
+        st_v4(y + (size_t)t * d + c, Vec16<TA>::from_f32(ya));
       }
-      st_v4(y + (size_t)t * d + c, Vec16<TA>::from_f32(ya));
     }
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) cur[j] = nxt[j];

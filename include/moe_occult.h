@@ -301,6 +301,64 @@ int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R
                         moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Real expert parallelism (one process per GPU, R = the number of ranks).
+ * Rank r holds the experts at slots r*L .. r*L+L-1 and the tokens of its own
+ * batch.  The Occult paper's all-to-all (Abstract; Figure 2) then carries
+ * the SFD segments to their ranks and the return rows back, and the count of
+ * rows sent is the budget C_T.  The exchanges themselves are collectives of
+ * the caller's process group; these are the device steps around them.
+ *
+ * Source rank, before the exchange: moe_route_brim (or route + brim build) on
+ * its own T tokens gives BRIM_0, sfd_token, sfd_off (row counts per
+ * destination: sfd_off[q+1] - sfd_off[q]) and C_T; moe_dispatch_gather with
+ * x_epd = NULL writes the SFD rows; moe_ep_pack_routing writes, for each SFD
+ * row, the token's top-k list restricted to the destination's experts.
+ * Destination rank, after receiving n rows (source-major, then ascending
+ * token: exactly its SFD segment of the single-GPU layer over the
+ * concatenated batches): moe_brim_build over the n received rows with their
+ * restricted lists gives its local BRIM_1 and EPD groups; moe_dispatch_gather
+ * with x_sfd = NULL writes the EPD rows; moe_expert_ffn runs its L groups
+ * (group_off = epd_off + r*L, G = L, its own packed weights);
+ * moe_ep_return_rows sums each row's expert outputs into one return row.
+ * Source rank, after the return exchange: moe_ep_combine sums every token's
+ * returned rows in ORI order (+ the shared experts).
+ * ------------------------------------------------------------------------- */
+
+/* moe_ep_pack_routing -- for every SFD row s < C_T, with t = sfd_token[s] and
+ * q the destination whose segment [sfd_off[q], sfd_off[q+1]) holds s:
+ *   idx_send[s][j] = topk_idx[t][j] if that expert lives on rank q, else -1
+ *   w_send[s][j]   = topk_w[t][j]   for the same entries, else 0
+ *   topk_idx, topk_w [T, k]; slot_of [E]; sfd_token [cap]; sfd_off [R+1];
+ *   c_t [1] (device); idx_send [cap, k] int32, w_send [cap, k] float32 out
+ *   (rows >= C_T are not written).  Invalid ids raise the device error flag.
+ * ------------------------------------------------------------------------- */
+int moe_ep_pack_routing(const int32_t* topk_idx, const float* topk_w, int T, int k,
+                        const int32_t* slot_of, int E, int R, const int32_t* sfd_token,
+                        const int32_t* sfd_off, const int32_t* c_t, int32_t* idx_send,
+                        float* w_send, moe_stream_t stream);
+
+/* moe_ep_return_rows -- the destination's intra-collaboration pre-reduce
+ * (Occult paper, Abstract): for every received row s (here the T "tokens"
+ * of the local BRIM build are the received rows),
+ *   y_ret[s] = sum over l ascending with BRIM_1[l][s] >= 0 of o_epd[BRIM_1[l][s]]
+ * in fp32, rounded to dtype.  Arguments as moe_combine_scatter (brim0, brim1
+ * of the local build); y_ret [T*min(k,R), d].  Nothing is written in ORI order.
+ * ------------------------------------------------------------------------- */
+int moe_ep_return_rows(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                       const int32_t* brim0, const int32_t* brim1, void* y_ret,
+                       moe_stream_t stream);
+
+/* moe_ep_combine -- the source's combine of the returned rows: y_ret holds
+ * one row per SFD row of the source's build (the return exchange delivers
+ * them in the order the SFD rows were sent), and
+ *   y[t] = sum over q ascending with BRIM_0[q][t] >= 0 of y_ret[BRIM_0[q][t]]
+ *          (+ shared_out[t] when not NULL), fp32 sums rounded to dtype.
+ *   y_ret [T*min(k,R), d]; brim0 [R, T]; shared_out [T, d] or NULL; y [T, d].
+ * ------------------------------------------------------------------------- */
+int moe_ep_combine(const void* y_ret, int T, int d, int dtype, int k, int R,
+                   const int32_t* brim0, const void* shared_out, void* y, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_count_dispatched_rows -- rows a once-per-rank dispatcher sends under a
  * placement ("Expert Coupling in MoE Pretraining", Abstract), without
  * building BRIMs:
