@@ -557,6 +557,10 @@ def run_ours(args, cfg):
             "ffn_ms": statistics.mean(ffn_ms),
             "ffn_own_graph_ms": statistics.mean(ffn_own_ms),
         }
+        # the GEMMs' time in SM clock cycles at the median sampled clock: the
+        # figure to compare across runs and with ncu at different clocks
+        mhz = line["clocks"].get("sm_mhz")
+        line["ffn_mcycles"] = line["ffn_ms"] * mhz * 1e-3 if mhz else None
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -1073,9 +1077,17 @@ def main():
     ap.add_argument("--prune", type=int, default=0,
                     help="routing-score-based collaboration pruning: keep each token's first "
                          "PRUNE ranks (0 = off)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's T (for profiling a smaller case of the same "
+                         "kernels; the line's config names the override)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the workload's E (R must divide it)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     cfg = inputs.CONFIGS[args.config]
+    if args.tokens or args.experts:
+        cfg = cfg.with_(name=f"{cfg.name}[T={args.tokens or cfg.T},E={args.experts or cfg.E}]",
+                        T=args.tokens or cfg.T, E=args.experts or cfg.E)
     if args.impl == "reference":
         run_reference(args, cfg)
     elif args.train:

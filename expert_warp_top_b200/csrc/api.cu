@@ -265,6 +265,105 @@ int hist_blocks(int T, int* tokens_per_block) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+namespace moe_host {
+namespace {
+// Shared memory the bulk combine takes per block, for its piece size.
+size_t combine_bulk_smem(int kmax, int piece_bytes) {
+  return (size_t)moe::kBulkWarps * (3 * kmax + 1) * piece_bytes;
+}
+
+template <typename TA, int KM>
+int launch_combine_bulk(DeviceInfo* di, const void* o_epd, int T, int d, int R, int L,
+                        size_t cap, int tk, const int32_t* brim0, const int32_t* brim1,
+                        const void* shared_out, void* y_sfd, void* y, cudaStream_t stream) {
+  // piece: as large as two blocks per SM allow (~110 KB each), 512 B .. 8 KB;
+  // shorter for batches too small to give every SM 16 units of work
+  const int row_bytes = d * (int)sizeof(TA);
+  int piece = (110 * 1024) / (moe::kBulkWarps * (3 * KM + 1));
+  piece = piece / 512 * 512;
+  if (piece < 512) piece = 512;
+  if (piece > moe::kBulkPiece) piece = moe::kBulkPiece;
+  if (piece > row_bytes) piece = row_bytes;
+  const long long want = (long long)di->num_sms * 16;
+  while ((long long)T * ((row_bytes + piece - 1) / piece) < want && piece >= 1024) piece /= 2;
+  piece = piece / 128 * 128;
+  const int n_pieces = (row_bytes + piece - 1) / piece;
+  const size_t smem = combine_bulk_smem(KM, piece);
+  // the kernel's limit is raised once per device, to the most any piece size
+  // above can ask for (110 KB)
+  constexpr size_t kMaxSmem = 110 * 1024;
+  MOE_REQUIRE(smem <= kMaxSmem, MOE_ERR_UNSUPPORTED, "combine staging too large");
+  auto kern = moe::combine_bulk_kernel<TA, KM>;
+  int rc = ensure_smem(di, reinterpret_cast<const void*>(kern), kMaxSmem);
+  if (rc) return rc;
+  const long long units = (long long)T * n_pieces;
+  long long blocks = (units + moe::kBulkWarps - 1) / moe::kBulkWarps;
+  if (blocks > 2LL * di->num_sms) blocks = 2LL * di->num_sms;
+  MOE_CUDA(launch_k(kern, (int)blocks, moe::kBulkWarps * 32, smem, stream,
+                    static_cast<const TA*>(o_epd), T, d, piece / (int)sizeof(TA), n_pieces, R, L,
+                    cap, tk, brim0, brim1, static_cast<const TA*>(shared_out),
+                    static_cast<TA*>(y_sfd), static_cast<TA*>(y), di->err_flag,
+                    wait_limit_ns()));
+  MOE_LAUNCHED("combine_bulk_kernel");
+  return MOE_OK;
+}
+
+// The combine kernel (register path, or the copy engine's under
+// kDebugBulkMovers) for every combine entry point: the whole return path,
+// y_sfd only (y == NULL), or the returned rows summed into y (brim1 == NULL,
+// L == 1, rows = the SFD rows).
+int launch_combine(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                   size_t cap, int tk, const int32_t* brim0, const int32_t* brim1,
+                   const void* shared_out, void* y_sfd, void* y, cudaStream_t stream) {
+  DeviceInfo* di;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  if (g_debug_flags & kDebugBulkMovers) {
+#define MOE_CB(TA, KM)                                                                         \
+  return launch_combine_bulk<TA, KM>(di, o_epd, T, d, R, L, cap, tk, brim0, brim1, shared_out, \
+                                     y_sfd, y, stream)
+    if (dtype == MOE_BF16) {
+      using B = __nv_bfloat16;
+      if (k <= 2) MOE_CB(B, 2);
+      if (k <= 4) MOE_CB(B, 4);
+      if (k <= 8) MOE_CB(B, 8);
+      MOE_CB(B, 16);
+    } else {
+      if (k <= 2) MOE_CB(float, 2);
+      if (k <= 4) MOE_CB(float, 4);
+      if (k <= 8) MOE_CB(float, 8);
+      MOE_CB(float, 16);
+    }
+#undef MOE_CB
+  }
+  const int P = mover_parts(di, T, (d * esize(dtype) + 511) / 512);
+  const long long warps = (long long)T * P;
+  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
+#define MOE_COMBINE(TA, KM)                                                                    \
+  MOE_CUDA(launch_k(moe::combine_kernel<TA, KM>, blocks, moe::kMoverWarps * 32, 0, stream,     \
+      static_cast<const TA*>(o_epd), T, d, P, R, L, cap, tk, brim0, brim1,                     \
+      static_cast<const TA*>(shared_out), static_cast<TA*>(y_sfd), static_cast<TA*>(y),        \
+      di->err_flag))
+  if (dtype == MOE_BF16) {
+    using B = __nv_bfloat16;
+    if (k <= 2) MOE_COMBINE(B, 2);
+    else if (k <= 4) MOE_COMBINE(B, 4);
+    else if (k <= 8) MOE_COMBINE(B, 8);
+    else MOE_COMBINE(B, 16);
+  } else {
+    if (k <= 2) MOE_COMBINE(float, 2);
+    else if (k <= 4) MOE_COMBINE(float, 4);
+    else if (k <= 8) MOE_COMBINE(float, 8);
+    else MOE_COMBINE(float, 16);
+  }
+#undef MOE_COMBINE
+  MOE_LAUNCHED("combine_kernel");
+  return MOE_OK;
+}
+}  // namespace
+}  // namespace moe_host
+
 // ===========================================================================
 extern "C" {
 
@@ -650,8 +749,31 @@ int moe_dispatch_gather(const void* x, int T, int d, int dtype, int k, int R, in
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
   const size_t cap = (size_t)T * (k < R ? k : R);
-  constexpr int CH = 4;  // 512-byte chunks in flight per warp
   const int row_bytes = d * esize(dtype);
+  if (g_debug_flags & kDebugBulkMovers) {
+    // copy-engine dispatch: whole rows (up to 8 KB) per unit when the batch
+    // fills the GPU, shorter pieces (>= 512 bytes) when it does not
+    const long long want = (long long)di->num_sms * 16;
+    int n_pieces = (row_bytes + moe::kBulkPiece - 1) / moe::kBulkPiece;
+    while ((long long)T * n_pieces < want && row_bytes / (2 * n_pieces) >= 512) n_pieces *= 2;
+    int piece = (row_bytes + n_pieces - 1) / n_pieces;
+    piece = (piece + 127) & ~127;
+    if (piece > moe::kBulkPiece) piece = moe::kBulkPiece;
+    n_pieces = (row_bytes + piece - 1) / piece;
+    const long long units = (long long)T * n_pieces;
+    long long blocks = (units + moe::kBulkWarps - 1) / moe::kBulkWarps;
+    if (blocks > 2LL * di->num_sms) blocks = 2LL * di->num_sms;
+    if ((rc = ensure_smem(di, reinterpret_cast<const void*>(moe::dispatch_bulk_kernel),
+                          moe::kBulkSmem)))
+      return rc;
+    MOE_CUDA(launch_k(moe::dispatch_bulk_kernel, (int)blocks, moe::kBulkWarps * 32,
+                      moe::kBulkSmem, stream, static_cast<const uint8_t*>(x), T, row_bytes, piece,
+                      n_pieces, R, L, cap, T * k, brim0, brim1, static_cast<uint8_t*>(x_sfd),
+                      static_cast<uint8_t*>(x_epd), di->err_flag, wait_limit_ns()));
+    MOE_LAUNCHED("dispatch_bulk_kernel");
+    return MOE_OK;
+  }
+  constexpr int CH = 4;  // 512-byte chunks in flight per warp
   const int P = mover_parts(di, T, (row_bytes + CH * 512 - 1) / (CH * 512));
   const long long warps = (long long)T * P;
   const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
@@ -678,29 +800,8 @@ int moe_combine_scatter(const void* o_epd, int T, int d, int dtype, int k, int R
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
   const size_t cap = (size_t)T * (k < R ? k : R);
-  const int P = mover_parts(di, T, (d * esize(dtype) + 511) / 512);
-  const long long warps = (long long)T * P;
-  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
-#define MOE_COMBINE(TA, KM)                                                                    \
-  MOE_CUDA(launch_k(moe::combine_kernel<TA, KM>, blocks, moe::kMoverWarps * 32, 0, stream,                    \
-      static_cast<const TA*>(o_epd), T, d, P, R, L, cap, T * k, brim0, brim1,                  \
-      static_cast<const TA*>(shared_out), static_cast<TA*>(y_sfd), static_cast<TA*>(y),        \
-      di->err_flag))
-  if (dtype == MOE_BF16) {
-    using B = __nv_bfloat16;
-    if (k <= 2) MOE_COMBINE(B, 2);
-    else if (k <= 4) MOE_COMBINE(B, 4);
-    else if (k <= 8) MOE_COMBINE(B, 8);
-    else MOE_COMBINE(B, 16);
-  } else {
-    if (k <= 2) MOE_COMBINE(float, 2);
-    else if (k <= 4) MOE_COMBINE(float, 4);
-    else if (k <= 8) MOE_COMBINE(float, 8);
-    else MOE_COMBINE(float, 16);
-  }
-#undef MOE_COMBINE
-  MOE_LAUNCHED("combine_kernel");
-  return MOE_OK;
+  return launch_combine(o_epd, T, d, dtype, k, R, L, cap, T * k, brim0, brim1, shared_out, y_sfd,
+                        y, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -726,40 +827,6 @@ int moe_ep_pack_routing(const int32_t* topk_idx, const float* topk_w, int T, int
   return MOE_OK;
 }
 
-namespace {
-// The combine kernel for the EP entry points: y_sfd only (y == NULL), or the
-// returned rows summed into y (brim1 == NULL, L == 1, rows = the SFD rows).
-int launch_combine(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
-                   size_t cap, int tk, const int32_t* brim0, const int32_t* brim1,
-                   const void* shared_out, void* y_sfd, void* y, cudaStream_t stream) {
-  DeviceInfo* di;
-  int rc = device_info(&di);
-  if (rc) return rc;
-  const int P = mover_parts(di, T, (d * esize(dtype) + 511) / 512);
-  const long long warps = (long long)T * P;
-  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
-#define MOE_COMBINE(TA, KM)                                                                    \
-  MOE_CUDA(launch_k(moe::combine_kernel<TA, KM>, blocks, moe::kMoverWarps * 32, 0, stream,     \
-      static_cast<const TA*>(o_epd), T, d, P, R, L, cap, tk, brim0, brim1,                     \
-      static_cast<const TA*>(shared_out), static_cast<TA*>(y_sfd), static_cast<TA*>(y),        \
-      di->err_flag))
-  if (dtype == MOE_BF16) {
-    using B = __nv_bfloat16;
-    if (k <= 2) MOE_COMBINE(B, 2);
-    else if (k <= 4) MOE_COMBINE(B, 4);
-    else if (k <= 8) MOE_COMBINE(B, 8);
-    else MOE_COMBINE(B, 16);
-  } else {
-    if (k <= 2) MOE_COMBINE(float, 2);
-    else if (k <= 4) MOE_COMBINE(float, 4);
-    else if (k <= 8) MOE_COMBINE(float, 8);
-    else MOE_COMBINE(float, 16);
-  }
-#undef MOE_COMBINE
-  MOE_LAUNCHED("combine_kernel");
-  return MOE_OK;
-}
-}  // namespace
 
 int moe_ep_return_rows(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
                        const int32_t* brim0, const int32_t* brim1, void* y_ret,

@@ -16,6 +16,7 @@
 // then moves its slice.
 #pragma once
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 
@@ -140,6 +141,102 @@ __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
   }
 }
 
+// The same dispatch through the copy engine (TMA bulk copies, no multicast):
+// a warp's lane 0 loads a piece of a token row (at most kBulkPiece bytes) into
+// one of the warp's kBulkBufs shared-memory buffers with one cp.async.bulk,
+// then stores it to every destination row with one cp.async.bulk each.  The
+// loads of the warp's next pieces are in flight while the current piece is
+// stored.  A unit of work is (token, piece): pieces are whole rows when the
+// batch fills the GPU, shorter for small batches.  Every mbarrier wait is
+// bounded: on expiry the timeout bit is raised, the warp stops issuing, waits
+// (bounded) for its loads in flight and lets its stores drain before exit.
+constexpr int kBulkWarps = 4;       // warps per block
+constexpr int kBulkBufs = 3;        // row buffers per warp
+constexpr int kBulkPiece = 8192;    // bytes per buffer
+constexpr size_t kBulkSmem = (size_t)kBulkWarps * kBulkBufs * kBulkPiece;
+
+__global__ void __launch_bounds__(kBulkWarps * 32) dispatch_bulk_kernel(
+    const uint8_t* __restrict__ x, int T, int row_bytes, int piece, int n_pieces, int R, int L,
+    size_t cap, int tk, const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
+    uint8_t* __restrict__ x_sfd, uint8_t* __restrict__ x_epd, unsigned* err,
+    uint64_t wait_limit_ns) {
+  extern __shared__ __align__(128) uint8_t bulk_smem[];
+  __shared__ __align__(8) uint64_t bars[kBulkWarps][kBulkBufs];
+  __shared__ WarpDst sdst[kBulkWarps];
+  __shared__ int abort_flag;
+  const int wib = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0)
+    for (int b = 0; b < kBulkBufs; ++b) tc::mbar_init(tc::smem_u32(&bars[wib][b]), 1);
+  tc::mbar_init_fence();
+  __syncthreads();
+  pdl_enter();
+  const tc::WaitCtl wctl{&abort_flag, err, wait_limit_ns};
+  uint8_t* bufs = bulk_smem + (size_t)wib * kBulkBufs * kBulkPiece;
+  const long long n_units = (long long)T * n_pieces;
+  const long long stride = (long long)gridDim.x * kBulkWarps;
+  const long long first = (long long)blockIdx.x * kBulkWarps + wib;
+  const long long mine = first < n_units ? (n_units - first + stride - 1) / stride : 0;
+  auto unit_of = [&](long long i, int& t, int& off, int& bytes) {
+    const long long u = first + i * stride;
+    t = (int)(u / n_pieces);
+    off = (int)(u - (long long)t * n_pieces) * piece;
+    bytes = min(piece, row_bytes - off);
+  };
+  auto issue_load = [&](long long i) {  // lane 0
+    int t, off, bytes;
+    unit_of(i, t, off, bytes);
+    const int b = (int)(i % kBulkBufs);
+    const uint32_t bar = tc::smem_u32(&bars[wib][b]);
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)bytes);
+    tc::bulk_load(tc::smem_u32(bufs + (size_t)b * kBulkPiece), x + (size_t)t * row_bytes + off,
+                  (uint32_t)bytes, bar);
+  };
+  long long issued = 0;  // loads issued (lane 0)
+  if (lane == 0)
+    for (; issued < mine && issued < kBulkBufs - 1; ++issued) issue_load(issued);
+  bool ok = true;
+  for (long long i = 0; i < mine; ++i) {
+    int t, off, bytes;
+    unit_of(i, t, off, bytes);
+    WarpDst& w = sdst[wib];
+    collect_dst(brim0, brim1, t, T, R, L, cap, tk, w, err);
+    if (lane == 0) {
+      // the buffer of load i + kBulkBufs - 1 was last read by the stores of unit i - 1
+      if (issued < mine) {
+        tc::bulk_wait_read_all();
+        issue_load(issued++);
+      }
+      const int b = (int)(i % kBulkBufs);
+      ok = tc::wait_bounded(tc::smem_u32(&bars[wib][b]), (uint32_t)((i / kBulkBufs) & 1), wctl);
+      if (ok) {
+        const uint32_t src = tc::smem_u32(bufs + (size_t)b * kBulkPiece);
+        if (x_sfd)
+          for (int j = 0; j < w.n_sfd; ++j)
+            tc::bulk_store(x_sfd + (size_t)w.sfd[j] * row_bytes + off, src, (uint32_t)bytes);
+        if (x_epd)
+          for (int j = 0; j < w.n_p; ++j)
+            tc::bulk_store(x_epd + (size_t)w.p[j] * row_bytes + off, src, (uint32_t)bytes);
+        tc::bulk_commit_group();
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+    __syncwarp();  // the destination list may be rewritten
+    if (!ok) {
+      // leave no load in flight into this warp's buffers: wait (bounded) for
+      // every load issued and not yet consumed
+      if (lane == 0)
+        for (long long j = i; j < issued; ++j)
+          tc::wait_bounded(tc::smem_u32(&bars[wib][j % kBulkBufs]),
+                           (uint32_t)((j / kBulkBufs) & 1), wctl, false);
+      break;
+    }
+  }
+  if (lane == 0) tc::bulk_wait_all();  // stores complete before the warp's buffers go away
+  __syncwarp();
+}
+
 // y_sfd[s] = sum_l o_epd[BRIM_1[l][s]] (fp32, rounded to TA); y[t] = sum_r y_sfd[..]
 // (+ shared[t]).  y sums the rounded payload rows, exactly as if it had read
 // them back.  A null y leaves only the return rows y_sfd (the destination
@@ -224,6 +321,152 @@ __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) cur[j] = nxt[j];
   }
+}
+
+// The combine through the copy engine.  A unit is (token, piece of its row);
+// per unit, lane 0 loads the piece of each of the token's expert rows into the
+// warp's input stage with one cp.async.bulk each (the next unit's loads are in
+// flight while this one is summed), every lane sums its 16-byte columns in
+// fp32 per rank, and the return pieces and the output piece are written to
+// the warp's output stage and stored with one cp.async.bulk each.  Per warp:
+// two input stages of KMAX x piece bytes and one output stage of
+// (KMAX + 1) x piece bytes, carved from dynamic shared memory.
+template <typename TA, int KMAX>
+__global__ void __launch_bounds__(kBulkWarps * 32) combine_bulk_kernel(
+    const TA* __restrict__ o_epd, int T, int d, int piece_elems, int n_pieces, int R, int L,
+    size_t cap, int tk, const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
+    const TA* __restrict__ shared_out, TA* __restrict__ y_sfd, TA* __restrict__ y,
+    unsigned* err, uint64_t wait_limit_ns) {
+  constexpr int VN = Vec16<TA>::n;
+  extern __shared__ __align__(128) uint8_t bulk_smem[];
+  __shared__ __align__(8) uint64_t bars[kBulkWarps][2];
+  __shared__ WarpDst sdst[kBulkWarps][2];
+  __shared__ int abort_flag;
+  const int wib = threadIdx.x >> 5;
+  const unsigned lane = lane_id();
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0)
+    for (int b = 0; b < 2; ++b) tc::mbar_init(tc::smem_u32(&bars[wib][b]), 1);
+  tc::mbar_init_fence();
+  __syncthreads();
+  pdl_enter();
+  const tc::WaitCtl wctl{&abort_flag, err, wait_limit_ns};
+  const int piece_bytes = piece_elems * (int)sizeof(TA);
+  const size_t warp_bytes = (size_t)(3 * KMAX + 1) * piece_bytes;
+  uint8_t* in_stage = bulk_smem + (size_t)wib * warp_bytes;  // [2][KMAX][piece]
+  uint8_t* out_stage = in_stage + (size_t)2 * KMAX * piece_bytes;  // [KMAX + 1][piece]
+  const long long n_units = (long long)T * n_pieces;
+  const long long stride = (long long)gridDim.x * kBulkWarps;
+  const long long first = (long long)blockIdx.x * kBulkWarps + wib;
+  const long long mine = first < n_units ? (n_units - first + stride - 1) / stride : 0;
+  auto unit_of = [&](long long i, int& t, int& c0, int& n) {
+    const long long u = first + i * stride;
+    t = (int)(u / n_pieces);
+    c0 = (int)(u - (long long)t * n_pieces) * piece_elems;
+    n = min(piece_elems, d - c0);
+  };
+  // lane 0: the expert pieces of unit i into input stage i % 2
+  auto issue_loads = [&](long long i) {
+    int t, c0, n;
+    unit_of(i, t, c0, n);
+    const WarpDst& w = sdst[wib][i & 1];
+    const int n_p = min(w.n_p, KMAX);
+    const uint32_t bar = tc::smem_u32(&bars[wib][i & 1]);
+    const uint32_t bytes = (uint32_t)(n * (int)sizeof(TA));
+    tc::mbar_arrive_expect_tx(bar, bytes * (uint32_t)n_p);
+    uint8_t* st = in_stage + (size_t)(i & 1) * KMAX * piece_bytes;
+    for (int j = 0; j < n_p; ++j)
+      tc::bulk_load(tc::smem_u32(st + (size_t)j * piece_bytes), o_epd + (size_t)w.p[j] * d + c0,
+                    bytes, bar);
+  };
+  if (mine > 0) {
+    int t, c0, n;
+    unit_of(0, t, c0, n);
+    collect_dst(brim0, brim1, t, T, R, L, cap, tk, sdst[wib][0], err);
+    if (lane == 0) issue_loads(0);
+  }
+  bool ok = true;
+  long long i = 0;
+  for (; i < mine; ++i) {
+    int t, c0, n;
+    unit_of(i, t, c0, n);
+    if (i + 1 < mine) {  // the next unit's destinations and loads (its stage was freed below)
+      int t1, c1, n1;
+      unit_of(i + 1, t1, c1, n1);
+      collect_dst(brim0, brim1, t1, T, R, L, cap, tk, sdst[wib][(i + 1) & 1], err);
+      if (lane == 0) issue_loads(i + 1);
+    }
+    ok = tc::wait_bounded(tc::smem_u32(&bars[wib][i & 1]), (uint32_t)((i >> 1) & 1), wctl);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    const WarpDst& w = sdst[wib][i & 1];
+    const int n_p = min(w.n_p, KMAX);
+    const uint8_t* st = in_stage + (size_t)(i & 1) * KMAX * piece_bytes;
+    if (lane == 0) tc::bulk_wait_read_all();  // the output stage's last stores have read it
+    __syncwarp();
+    int n_ret = 0;  // return pieces written to the output stage
+    int ret_row[KMAX];
+    for (int c = (int)lane * VN; c < n; c += 32 * VN) {
+      float acc[VN], ya[VN];
+#pragma unroll
+      for (int e = 0; e < VN; ++e) ya[e] = acc[e] = 0.f;
+      int nr = 0;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < n_p) {
+          float f[VN];
+          Vec16<TA>::to_f32(ld_v4(st + (size_t)j * piece_bytes + c * sizeof(TA)), f);
+#pragma unroll
+          for (int e = 0; e < VN; ++e) acc[e] += f[e];
+          if (j + 1 == n_p || w.p_sfd[j + 1 < KMAX ? j + 1 : j] != w.p_sfd[j]) {
+            const uint4 packed = Vec16<TA>::from_f32(acc);
+            st_v4(out_stage + (size_t)nr * piece_bytes + c * sizeof(TA), packed);
+            ret_row[nr] = w.p_sfd[j];
+            ++nr;
+            float r[VN];
+            Vec16<TA>::to_f32(packed, r);
+#pragma unroll
+            for (int e = 0; e < VN; ++e) {
+              ya[e] += r[e];
+              acc[e] = 0.f;
+            }
+          }
+        }
+      }
+      n_ret = nr;
+      if (y) {
+        if (shared_out) {
+          float f[VN];
+          Vec16<TA>::to_f32(ld_nc_v4(shared_out + (size_t)t * d + c0 + c), f);
+#pragma unroll
+          for (int e = 0; e < VN; ++e) ya[e] += f[e];
+        }
+        st_v4(out_stage + (size_t)KMAX * piece_bytes + c * sizeof(TA), Vec16<TA>::from_f32(ya));
+      }
+    }
+    tc::fence_proxy_async_smem();  // this lane's stage writes, before the copy engine reads them
+    __syncwarp();
+    if (lane == 0) {
+      // lane 0 always handles column 0 (n >= VN), so its n_ret and ret_row are the warp's
+      const uint32_t bytes = (uint32_t)(n * (int)sizeof(TA));
+      const uint32_t ob = tc::smem_u32(out_stage);
+      if (y_sfd)
+        for (int r = 0; r < n_ret; ++r)
+          tc::bulk_store(y_sfd + (size_t)ret_row[r] * d + c0, ob + (uint32_t)(r * piece_bytes),
+                         bytes);
+      if (y)
+        tc::bulk_store(y + (size_t)t * d + c0, ob + (uint32_t)(KMAX * piece_bytes), bytes);
+      tc::bulk_commit_group();
+    }
+    __syncwarp();
+  }
+  if (!ok && lane == 0) {
+    // leave no load in flight: units i and i + 1 had their loads issued (bounded waits)
+    for (long long j = i; j <= i + 1 && j < mine; ++j)
+      tc::wait_bounded(tc::smem_u32(&bars[wib][j & 1]), (uint32_t)((j >> 1) & 1), wctl, false);
+  }
+  if (lane == 0) tc::bulk_wait_all();
+  __syncwarp();
 }
 
 // Identity expert: out[p] = row_scale[p] * a[p] for the rows of all groups.

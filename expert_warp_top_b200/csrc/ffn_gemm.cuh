@@ -58,17 +58,6 @@ constexpr int kEpiSwiGLUBwd = 3;
 // would load, so the MMA issuer's wait can never complete.
 constexpr int kDebugSkipFirstLoad = 1;
 
-// Tile order inside a group: M blocks fastest (default; concurrently running
-// CTAs share one weight block in L2) or N blocks fastest (they share A rows).
-#ifndef MOE_RASTER_N_FASTEST
-#define MOE_RASTER_N_FASTEST 0
-#endif
-constexpr bool kRasterNFastest = MOE_RASTER_N_FASTEST != 0;
-// L2 policy of the weight tiles: keep them (evict_last, default) or not.
-#ifndef MOE_WEIGHTS_EVICT_LAST
-#define MOE_WEIGHTS_EVICT_LAST 1
-#endif
-constexpr bool kWeightsEvictLast = MOE_WEIGHTS_EVICT_LAST != 0;
 
 // The logistic sigmoid of SiLU, 1 / (1 + e^-x), with the fast division
 // (__fdividef: a reciprocal and a multiply).  The IEEE division is a
@@ -145,6 +134,12 @@ struct GemmArgs {
   float* partial = nullptr;      // gate-gradient partials [rows, n_part] (nullable)
   int n_part = 0;
   int tile_mode = 0;             // kTilesAll / kTilesPairNoSmallTail / kTilesSmallTail
+  // L2 policies (0 evict_normal, 1 evict_last, 2 evict_first): of the A-row
+  // loads, the weight loads and the epilogue's tensor stores of `out`
+  int l2_a = 0, l2_b = 1, l2_out = 0;
+  // tile order inside a group: 0 M blocks fastest (concurrently running CTAs
+  // share one weight block in L2), 1 N blocks fastest (they share A rows)
+  int raster = 0;
 };
 
 // Which rows of each group a launch covers, for mixing CTA-pair and single-CTA
@@ -180,7 +175,7 @@ __device__ __forceinline__ float round_bf16(float v) {
 __device__ __forceinline__ void store_row64_bf16(const float* v, bool valid, bool full,
                                                  size_t grow, int wrow0, int col,
                                                  __nv_bfloat16* out, int ldo, uint8_t* box,
-                                                 const CUtensorMap* tmap_out) {
+                                                 const CUtensorMap* tmap_out, int l2_out) {
   const unsigned lane = lane_id();
   if (full) {
     if (lane == 0) tc::bulk_wait_read_all();  // the box's previous store has read it
@@ -191,7 +186,9 @@ __device__ __forceinline__ void store_row64_bf16(const float* v, bool valid, boo
     tc::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tc::tma_store_2d(tmap_out, tc::smem_u32(box), col, wrow0);
+      if (l2_out) tc::tma_store_2d_hint(tmap_out, tc::smem_u32(box), col, wrow0,
+                                        tc::policy_from_code(l2_out));
+      else tc::tma_store_2d(tmap_out, tc::smem_u32(box), col, wrow0);
       tc::bulk_commit_group();
     }
   } else if (valid) {
@@ -398,7 +395,8 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
           hv[h * 32 + i] = gv * sigmoid_fast(gv) * uv;
         }
       }
-      store_row64_bf16(hv, valid, full, grow, wrow0, (n0 >> 1) + p * 64, out, ldo, box, tmap_out);
+      store_row64_bf16(hv, valid, full, grow, wrow0, (n0 >> 1) + p * 64, out, ldo, box, tmap_out,
+                       args.l2_out);
     }
   } else if constexpr (EPI == kEpiScale && kBf16) {
     const float scale = (valid && row_scale) ? row_scale[grow] : 1.0f;
@@ -413,7 +411,8 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, bool valid, size_t
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[h * 32 + i] = __uint_as_float(vr[i]) * scale;
       }
-      store_row64_bf16(v, valid, full, grow, wrow0, n0 + c * 64, out, ldo, box, tmap_out);
+      store_row64_bf16(v, valid, full, grow, wrow0, n0 + c * 64, out, ldo, box, tmap_out,
+                       args.l2_out);
     }
   } else if constexpr (EPI == kEpiSwiGLU) {
     // (fp32 output) columns [128p, 128p+64) gate, [128p+64, 128p+128) up
@@ -587,7 +586,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int gstart = s_off[g], gend = s_end[g];
     const int m_blocks = group_m_blocks(gend - gstart, kGemmBM, args.tile_mode);
     int nb, mb;
-    if (kRasterNFastest) {
+    if (args.raster) {
       mb = local / n_blocks;
       nb = local - mb * n_blocks;
     } else {
@@ -604,8 +603,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // The whole warp runs the loop: lane 0 waits, arms the stage and loads B;
     // in GATHER mode every lane then gathers 4 of the tile's 128 A rows.
     if (GATHER || lane == 0) {
-      const uint64_t pol_a = tc::policy_evict_normal();
-      const uint64_t pol_b = kWeightsEvictLast ? tc::policy_evict_last() : tc::policy_evict_normal();
+      const uint64_t pol_a = tc::policy_from_code(args.l2_a);
+      const uint64_t pol_b = tc::policy_from_code(args.l2_b);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per stage: armed at least once, parity of the last arming

@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gend = s_end[g];
     const int m_blocks = group_m_blocks(gend - gstart, kPairBM, args.tile_mode);
     int nb, mb;
-    if (kRasterNFastest) {
+    if (args.raster) {
       mb = local / n_blocks;
       nb = local - mb * n_blocks;
     } else {
@@ -141,8 +141,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_a = tc::policy_evict_normal();
-      const uint64_t pol_b = kWeightsEvictLast ? tc::policy_evict_last() : tc::policy_evict_normal();
+      const uint64_t pol_a = tc::policy_from_code(args.l2_a);
+      const uint64_t pol_b = tc::policy_from_code(args.l2_b);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;

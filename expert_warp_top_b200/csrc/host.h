@@ -70,6 +70,12 @@ inline uint64_t wait_limit_ns() { return static_cast<uint64_t>(g_wait_limit_ms *
 constexpr int kDebugForceSingle = 2;  // GEMMs on single CTAs
 constexpr int kDebugForcePair = 4;    // GEMMs on CTA pairs only where the shape allows
 constexpr int kDebugForceHybrid = 8;  // pair tiles plus single-CTA small tails
+constexpr int kDebugBulkMovers = 16;  // dispatch and combine through TMA bulk copies
+// Tuning knobs of the expert GEMMs: with kDebugGemmPolicy set, bits 8..9, 10..11
+// and 12..13 of the flags give the L2 policy of the A loads, the weight loads and
+// the output stores (0 evict_normal, 1 evict_last, 2 evict_first; output 0 = no
+// hint), and bit 14 the N-fastest tile order.
+constexpr int kDebugGemmPolicy = 32;
 
 // 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
@@ -133,6 +139,12 @@ inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
   a.partial = ex.partial;
   a.n_part = ex.n_part;
   a.tile_mode = ex.tile_mode;
+  if (g_debug_flags & kDebugGemmPolicy) {
+    a.l2_a = (g_debug_flags >> 8) & 3;
+    a.l2_b = (g_debug_flags >> 10) & 3;
+    a.l2_out = (g_debug_flags >> 12) & 3;
+    a.raster = (g_debug_flags >> 14) & 1;
+  }
   return a;
 }
 
