@@ -140,6 +140,11 @@ struct GemmArgs {
   // tile order inside a group: 0 M blocks fastest (concurrently running CTAs
   // share one weight block in L2), 1 N blocks fastest (they share A rows)
   int raster = 0;
+  // L2 prefetch of the next tile's first-use operand panels (CTA-pair kernel,
+  // K-major operands): the base addresses of A [m_cap, K] and B [G*N, K]
+  const void* a_ptr = nullptr;
+  const void* b_ptr = nullptr;
+  int l2_prefetch = 0;
 };
 
 // Which rows of each group a launch covers, for mixing CTA-pair and single-CTA

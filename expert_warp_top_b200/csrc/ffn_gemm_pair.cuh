@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int total_tiles = s_prefix[G];
   const tc::WaitCtl wctl{abort_flag, args.err, args.wait_limit_ns};
 
+  int last_mb = 0, last_nb = 0;  // the M and N block of the tile last located
   auto locate = [&](int tile, int& g, int& row0, int& gend, int& n0) {
     int lo = 0, hi = G;
     while (hi - lo > 1) {
@@ -136,6 +137,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     row0 = gstart + mb * kPairBM;
     n0 = nb * BN;
+    last_mb = mb;
+    last_nb = nb;
   };
 
   if (warp == 0) {
@@ -150,6 +153,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
         int g, row0, gend, n0;
+        if (!B_MN && args.l2_prefetch && tile + n_pairs < total_tiles) {
+          // This pair's next tile, one tile's time ahead: the first tile of its
+          // M block (N block 0) brings this CTA's A rows, and the first tile of
+          // its N block (M block 0) this CTA's half of the weight panel, into L2
+          // (both contiguous: all K columns of consecutive rows).
+          locate(tile + n_pairs, g, row0, gend, n0);
+          const size_t kbytes = (size_t)args.K * Cfg::kElemBytes;
+          const int r0 = row0 + (int)rank * 128;
+          if (last_nb == 0 && r0 < gend)
+            tc::bulk_prefetch_l2(static_cast<const uint8_t*>(args.a_ptr) + (size_t)r0 * kbytes,
+                                 (uint32_t)(min(128, gend - r0) * kbytes));
+          if (last_mb == 0)
+            tc::bulk_prefetch_l2(static_cast<const uint8_t*>(args.b_ptr) +
+                                     ((size_t)g * args.N + n0 + (int)rank * (BN / 2)) * kbytes,
+                                 (uint32_t)((BN / 2) * kbytes));
+        }
         locate(tile, g, row0, gend, n0);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!tc::wait_bounded(tc::smem_u32(&empty_bar[stage]), phase ^ 1u, wctl)) {

@@ -74,7 +74,8 @@ constexpr int kDebugBulkMovers = 16;  // dispatch and combine through TMA bulk c
 // Tuning knobs of the expert GEMMs: with kDebugGemmPolicy set, bits 8..9, 10..11
 // and 12..13 of the flags give the L2 policy of the A loads, the weight loads and
 // the output stores (0 evict_normal, 1 evict_last, 2 evict_first; output 0 = no
-// hint), and bit 14 the N-fastest tile order.
+// hint), bit 14 the N-fastest tile order and bit 15 the L2 prefetch of the next
+// tile's first-use panels.
 constexpr int kDebugGemmPolicy = 32;
 
 // 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
@@ -144,6 +145,7 @@ inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
     a.l2_b = (g_debug_flags >> 10) & 3;
     a.l2_out = (g_debug_flags >> 12) & 3;
     a.raster = (g_debug_flags >> 14) & 1;
+    a.l2_prefetch = (g_debug_flags >> 15) & 1;
   }
   return a;
 }
@@ -270,8 +272,10 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   const long long pairs = ub < max_clusters ? (ub < 1 ? 1 : ub) : max_clusters;
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
   cfg.numAttrs = 2;
-  const moe::GemmArgs args =
+  moe::GemmArgs args =
       gemm_args(di, group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo, ex);
+  args.a_ptr = a;
+  args.b_ptr = b;
   MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, to, tx, args));
   return MOE_OK;
 }
