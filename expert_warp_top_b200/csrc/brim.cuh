@@ -313,9 +313,8 @@ __global__ void __launch_bounds__(1024) brim_colscan_kernel(
 }
 
 // ---- pass 3 ---------------------------------------------------------------
-// One block of kScatterWarps warps per tile.  The warps rebuild the tile's
-// masks (by ballot, sharing the columns) and warp 0 the tile's first row in
-// every column; then warp w walks the
+// One block of kScatterWarps warps per tile.  Warp 0 rebuilds the tile's
+// masks and the tile's first row in every column; then warp w walks the
 // ranks r = w, w + kScatterWarps, ... and, inside each, the rank's local
 // experts l, so that for one column the lanes that hit it hold consecutive
 // rows: every store of a warp lands on consecutive addresses.
@@ -356,18 +355,8 @@ __global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
   for (int j = 0; j < KMAX; ++j)
     gate[j] = (active && j < k && tr.slot[j] >= 0) ? (topk_w ? __ldg(topk_w + (size_t)t * k + j) : 1.f)
                                                    : 0.f;
-  // the tile's column masks, by ballot, the warps sharing the columns
-  for (int c = warp; c < ncol; c += kScatterWarps) {
-    bool hit = false;
-    if (active) {
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k && tr.slot[j] >= 0) hit |= c < R ? tr.rank[j] == c : tr.slot[j] == c - R;
-    }
-    const uint32_t m = __ballot_sync(0xffffffffu, hit);
-    if (lane == 0) sm[c] = m;
-  }
   if (warp == 0) {
+    tile_masks<KMAX>(sm, ncol, R, active, k, tr);
     // the tile's first global row in every column
     if (totals) {
       for (int c = lane; c < ncol; c += 32) s_tot[c] = totals[c];

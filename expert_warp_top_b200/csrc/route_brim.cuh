@@ -2,11 +2,11 @@
 // one kernel (pass 1 of the BRIM build fused with routing).
 //
 // The same computation as moe_route_topk + brim_mask_kernel +
-// moe_count_dispatched_rows: one block of kRouteTileWarps warps per 32-token
-// tile.  The warps route the tile's tokens (route_token_warp, the very code of
-// moe_route_topk), then every warp takes the tile lane-per-token and builds a
-// share of its column masks by ballot; warp 0 writes the top-k (pruned, when
-// asked) and adds the tile's contribution to the counter.  The column scan with the histogram (brim_colscan_kernel) and
+// moe_count_dispatched_rows: one block of 32 warps per 32-token tile.  Each
+// warp routes one token (route_token_warp, the very code of moe_route_topk);
+// warp 0 then takes the tile lane-per-token, prunes (when asked), writes the
+// top-k, builds the tile's column masks and adds the tile's contribution to
+// the counter.  The column scan with the histogram (brim_colscan_kernel) and
 // the scatter (brim_scatter_kernel) follow.
 #pragma once
 #include "brim.cuh"
@@ -14,10 +14,8 @@
 
 namespace moe {
 
-constexpr int kRouteTileWarps = 32;  // warps per 32-token tile: one token each
-
 template <int KMAX>
-__global__ void __launch_bounds__(32 * kRouteTileWarps) route_brim_tile_kernel(
+__global__ void __launch_bounds__(1024) route_brim_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     const int32_t* __restrict__ slot_of, int R, int prune_m, int n_tiles,
     int32_t* __restrict__ topk_idx,
@@ -27,53 +25,36 @@ __global__ void __launch_bounds__(32 * kRouteTileWarps) route_brim_tile_kernel(
   pdl_enter();
   __shared__ int s_ids[32][KMAX];
   __shared__ float s_gates[32][KMAX];
+  __shared__ uint32_t s_mask[kMaxCols];
   const int warp = threadIdx.x >> 5;
   const unsigned lane = lane_id();
   const int tile = blockIdx.x;
   const int L = E / R, ncol = R + E;
 
-  // 1. warp w routes tokens w, w + kRouteTileWarps, ... of the tile
-  for (int i = warp; i < kBrimTileTokens; i += kRouteTileWarps) {
-    const int t = tile * kBrimTileTokens + i;
+  // 1. each warp routes one token of the tile
+  {
+    const int t = tile * kBrimTileTokens + warp;
     int id = -1;
     float gate = 0.f;
     if (t < T) route_token_warp(logits + (size_t)t * E, E, k, renorm, &id, &gate);
     if ((int)lane < KMAX) {
-      s_ids[i][lane] = (t < T && (int)lane < k) ? id : -1;
-      s_gates[i][lane] = (t < T && (int)lane < k) ? gate : 0.f;
+      s_ids[warp][lane] = (t < T && (int)lane < k) ? id : -1;
+      s_gates[warp][lane] = (t < T && (int)lane < k) ? gate : 0.f;
     }
   }
   __syncthreads();
 
-  // 2. every warp takes the tile lane-per-token (each builds the same routes);
-  //    warp w then makes the column masks c = w, w + kRouteTileWarps, ... by
-  //    ballot, and warp 0 writes the top-k and adds the tile to the counter
-  const int t = tile * kBrimTileTokens + (int)lane;
-  int ids[KMAX];
-  float gates[KMAX];
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    ids[j] = s_ids[lane][j];
-    gates[j] = s_gates[lane][j];
-  }
-  if (prune_m > 0 && t < T) prune_token<KMAX>(ids, gates, slot_of, k, E, L, prune_m);
-  TokenRoute<KMAX> tr;
-  const bool active =
-      t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, warp == 0 ? err : nullptr);
-  for (int c = warp; c < ncol; c += kRouteTileWarps) {
-    bool hit = false;
-    if (active) {
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k && tr.slot[j] >= 0) hit |= c < R ? tr.rank[j] == c : tr.slot[j] == c - R;
-    }
-    const uint32_t m = __ballot_sync(0xffffffffu, hit);
-    if (lane == 0) {
-      masks[(size_t)c * n_tiles + tile] = m;
-      if (per_rank && c < R && m) atomicAdd(&per_rank[c], __popc(m));  // tokens per rank
-    }
-  }
+  // 2. warp 0, one lane per token: pruning, top-k out, masks, counter
   if (warp == 0) {
+    const int t = tile * kBrimTileTokens + (int)lane;
+    int ids[KMAX];
+    float gates[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ids[j] = s_ids[lane][j];
+      gates[j] = s_gates[lane][j];
+    }
+    if (prune_m > 0 && t < T) prune_token<KMAX>(ids, gates, slot_of, k, E, L, prune_m);
     if (t < T)
 #pragma unroll
       for (int j = 0; j < KMAX; ++j)
@@ -81,9 +62,17 @@ __global__ void __launch_bounds__(32 * kRouteTileWarps) route_brim_tile_kernel(
           topk_idx[(size_t)t * k + j] = ids[j];
           topk_w[(size_t)t * k + j] = gates[j];
         }
+    TokenRoute<KMAX> tr;
+    const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
+    tile_masks<KMAX>(s_mask, ncol, R, active, k, tr);
+    for (int c = lane; c < ncol; c += 32) masks[(size_t)c * n_tiles + tile] = s_mask[c];
     if (per_rank) {
-      // rows sent, and the remote ones: ranks other than the token's source
-      // rank floor(t * R / T)
+      // tokens per rank: popcount of the rank columns; remote: ranks other than
+      // the token's source rank floor(t * R / T)
+      for (int r = lane; r < R; r += 32) {
+        const int n = __popc(s_mask[r]);
+        if (n) atomicAdd(&per_rank[r], n);
+      }
       const int src = (int)(((long long)t * R) / (T > 0 ? T : 1));
       unsigned n_rank = 0, n_remote = 0;
 #pragma unroll
