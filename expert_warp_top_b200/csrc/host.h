@@ -16,6 +16,7 @@
 #include "../../include/moe_occult.h"
 #include "ffn_gemm.cuh"
 #include "ffn_gemm_pair.cuh"
+#include "ffn_gemm_swap.cuh"
 #include "wgrad_gemm.cuh"
 #include "wgrad_pair.cuh"
 
@@ -77,6 +78,8 @@ constexpr int kDebugBulkMovers = 16;  // dispatch and combine through TMA bulk c
 // hint), bit 14 the N-fastest tile order and bit 15 the L2 prefetch of the next
 // tile's first-use panels.
 constexpr int kDebugGemmPolicy = 32;
+constexpr int kDebugForceSwap = 64;   // inference GEMMs on the swapped-operand kernel
+constexpr int kDebugNoSwap = 128;     // never on the swapped-operand kernel
 
 // 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
@@ -280,6 +283,72 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   return MOE_OK;
 }
 
+// The same GEMM with the operands swapped (ffn_gemm_swap.cuh): CTA pairs on
+// 256 weight rows x up to 256 of a group's rows.  bf16, K-major weights, the
+// two inference epilogues; N % 256 == 0, G <= kSwapMaxGroups.
+template <int EPI>
+int launch_gemm_swap(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K, const void* b,
+                     int G, int N, const int32_t* group_off, const float* row_scale, void* out,
+                     int ldo, cudaStream_t st) {
+  using Cfg = moe::SwapCfg;
+  moe::SwapMaps rows;
+  int rc;
+  for (int i = 0; i < moe::kSwapMaps; ++i)
+    if ((rc = encode_2d(&rows.rows[i], a, MOE_BF16, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK,
+                        8u << i)))
+      return rc;
+  CUtensorMap tw, to;
+  if ((rc = encode_2d(&tw, b, MOE_BF16, (uint64_t)K, (uint64_t)G * N, Cfg::kBK, 128))) return rc;
+  if ((rc = encode_out(&to, out, MOE_BF16, m_cap, ldo))) return rc;
+  auto kern = moe::ffn_gemm_swap_kernel<EPI>;
+  const void* key = reinterpret_cast<const void*>(kern);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;  // the occupancy query below sees the cluster shape only
+  if ((rc = ensure_smem(di, key, Cfg::kSmemBytes))) return rc;
+  int max_clusters = 0;
+  {
+    std::lock_guard<std::mutex> lk(di->mu);
+    for (auto& pc : di->pair_clusters)
+      if (pc.first == key) max_clusters = pc.second;
+  }
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(2 * (di->num_sms / 2), 1, 1);
+    MOE_CUDA(cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg));
+    MOE_REQUIRE(max_clusters >= 1, MOE_ERR_UNSUPPORTED, "no CTA pair fits on this device");
+    std::lock_guard<std::mutex> lk(di->mu);
+    di->pair_clusters.emplace_back(key, max_clusters);
+  }
+  const long long ub = ((long long)m_cap / moe::kSwapMaxRows + G) * (N / moe::kSwapBM);
+  const long long pairs = ub < max_clusters ? (ub < 1 ? 1 : ub) : max_clusters;
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.numAttrs = 2;
+  const moe::GemmArgs args =
+      gemm_args(di, group_off, nullptr, a_rows, G, N, K, m_cap, row_scale, out, ldo, GemmExtra{});
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, kern, rows, tw, to, args));
+  return MOE_OK;
+}
+
+// Groups this short (rows on average) go to the swapped-operand kernel.  It
+// measured slower than the row-major pair kernel on every workload (the
+// OLMoE-shaped layer's GEMMs 0.43 against 0.41 ms, DSV2-Lite-shaped 1.52 against
+// 1.43 ms): its tail tiles still stream the full weight tile into each SM, and
+// its epilogue turns the accumulators around through shared memory.  So it
+// runs only when asked for (kDebugForceSwap), tested.
+#ifndef MOE_SWAP_MAX_AVG_ROWS
+#define MOE_SWAP_MAX_AVG_ROWS 0
+#endif
+
 // GEMM over the groups, on CTA pairs when the groups are tall enough to fill
 // 256-row tiles (and the rows are read in place), else on single CTAs.  In
 // hybrid mode a group's tail of at most 128 rows goes to a second,
@@ -294,6 +363,14 @@ int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a
                      const GemmExtra& ex = GemmExtra{}) {
   const bool tall = (long long)m_cap >= (long long)MOE_PAIR_MIN_ROWS * G;
   const bool pair_ok = !a_row_index && N % 128 == 0;
+  if constexpr (!TF32 && !B_MN && (EPI == moe::kEpiSwiGLU || EPI == moe::kEpiScale)) {
+    const bool swap_ok = !a_row_index && N % moe::kSwapBM == 0 && G <= moe::kSwapMaxGroups &&
+                         K % 64 == 0 && !(g_debug_flags & kDebugNoSwap);
+    const bool short_groups = (long long)m_cap < (long long)MOE_SWAP_MAX_AVG_ROWS * G;
+    if (swap_ok && ((g_debug_flags & kDebugForceSwap) || short_groups))
+      return launch_gemm_swap<EPI>(di, a, a_rows, m_cap, K, b, G, N, group_off, row_scale, out,
+                                   ldo, st);
+  }
   bool pair = pair_ok && tall;
   // Hybrid tiling (a group's tail of <= 128 rows on single-CTA tiles, in a
   // second launch) cuts the OLMoE-shaped layer's padded MMA rows from 20% to
