@@ -37,7 +37,12 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBoxesPerWarp = epi_boxes_per_warp<EPI>();
   static constexpr int kStages = ring_stages(kStageBytes, kBoxesPerWarp);
-  static constexpr int kTmemCols = 2 * BN;
+  // BN = 512 fills TMEM's 512 columns with one accumulator (no double buffer)
+  static constexpr int kAccBufs = 2 * BN <= 512 ? 2 : 1;
+  static constexpr int kTmemCols = kAccBufs * BN;
+  // the MMA's N (at most 256) and the MMAs per K step that cover BN
+  static constexpr int kMmaN = BN > 256 ? 256 : BN;
+  static constexpr int kNSub = BN / kMmaN;
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes +
                                        4 * kBoxesPerWarp * kEpiBoxBytes + 512 + kGroupTableBytes;
   static_assert(kSmemBytes <= (size_t)kSmemPerCta, "GEMM shared memory over the per-CTA limit");
@@ -51,7 +56,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_out,
                          const __grid_constant__ CUtensorMap tmap_aux, const GemmArgs args) {
-  static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
+  static_assert(BN == 128 || BN == 256 || BN == 512, "pair tiles use BN = 128, 256 or 512");
+  static_assert(BN <= 256 || (!B_MN && EPI != kEpiSwiGLUSave && EPI != kEpiSwiGLUBwd),
+                "512-wide pair tiles: K-major weights, the inference epilogues");
   static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
   using Cfg = PairCfg<BN, TF32, EPI>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
@@ -187,6 +194,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0,
                                    g * args.K + kb * Cfg::kBK, (n0 + (int)rank * (BN / 2)) / 64,
                                    pol_b);
+            } else if (BN > 256) {
+              // two 256-column halves; CTA r loads rows [h*256 + r*128, +128) of the
+              // panel, so that MMA h covers panel columns [h*256, h*256 + 256)
+#pragma unroll
+              for (int h = 0; h < Cfg::kNSub; ++h)
+                tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes + h * 128 * 128), &tmap_b,
+                                     fb_pair, kb * Cfg::kBK,
+                                     g * args.N + n0 + h * 256 + (int)rank * 128, pol_b);
             } else {
               tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
                                    kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);
@@ -210,7 +225,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc = tc::idesc_f32acc<TF32, 256, BN, false, B_MN>();
+      constexpr uint32_t idesc = tc::idesc_f32acc<TF32, 256, Cfg::kMmaN, false, B_MN>();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -234,10 +249,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {
             const uint64_t off = static_cast<uint64_t>(kk * 2);
             const uint64_t boff = B_MN ? static_cast<uint64_t>(kk * 128) : off;
-            if (TF32)
-              tc::mma_tf32_pair(d_tmem, adesc + off, bdesc + boff, idesc, (kb | kk) != 0);
-            else
-              tc::mma_f16_pair(d_tmem, adesc + off, bdesc + boff, idesc, (kb | kk) != 0);
+#pragma unroll
+            for (int h = 0; h < Cfg::kNSub; ++h) {
+              // the h-th 256-column half: 16 KB further in shared memory, 256 TMEM columns on
+              const uint64_t hoff = static_cast<uint64_t>(h * ((128 * 128) >> 4));
+              const uint32_t dh = d_tmem + static_cast<uint32_t>(h * Cfg::kMmaN);
+              if (TF32)
+                tc::mma_tf32_pair(dh, adesc + off, bdesc + boff + hoff, idesc, (kb | kk) != 0);
+              else
+                tc::mma_f16_pair(dh, adesc + off, bdesc + boff + hoff, idesc, (kb | kk) != 0);
+            }
           }
           // frees this stage in both CTAs once these MMAs have read it
           tc::commit_pair_multicast(tc::smem_u32(&empty_bar[stage]), 0x3);
@@ -248,7 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         tc::commit_pair_multicast(tc::smem_u32(&tfull_bar[acc]), 0x3);
-        if (++acc == 2) {
+        if (++acc == Cfg::kAccBufs) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -294,7 +315,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (rank == 0) tc::mbar_arrive(bar);
         else tc::mbar_arrive_remote(tc::mapa_shared(bar, 0));
       }
-      if (++acc == 2) {
+      if (++acc == Cfg::kAccBufs) {
         acc = 0;
         acc_phase ^= 1u;
       }

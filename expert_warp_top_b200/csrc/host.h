@@ -80,6 +80,8 @@ constexpr int kDebugBulkMovers = 16;  // dispatch and combine through TMA bulk c
 constexpr int kDebugGemmPolicy = 32;
 constexpr int kDebugForceSwap = 64;   // inference GEMMs on the swapped-operand kernel
 constexpr int kDebugNoSwap = 128;     // never on the swapped-operand kernel
+constexpr int kDebugWideTiles = 256;  // inference GEMMs on 256 x 512 pair tiles where N allows
+constexpr int kDebugNoWideTiles = 512;
 
 // 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
@@ -238,7 +240,9 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   CUtensorMap ta, tb;
   int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
   if (rc) return rc;
-  if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN / 2))) return rc;
+  // each CTA loads its BN/2 weight rows in one box, or (BN = 512) in two of 128
+  if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN > 256 ? 128 : BN / 2)))
+    return rc;
   CUtensorMap to, tx;
   if ((rc = encode_out(&to, out, dtype, m_cap, ldo))) return rc;
   if ((rc = encode_aux<EPI>(&tx, to, ex, dtype, m_cap))) return rc;
@@ -349,6 +353,19 @@ int launch_gemm_swap(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
 #define MOE_SWAP_MAX_AVG_ROWS 0
 #endif
 
+// Groups at least this tall (rows on average) take the 256 x 512 pair tiles
+// when N allows (0: only when asked for, kDebugWideTiles).  Measured against the
+// 256 x 256 tiles on one B200 (GEMM-only replays, three rounds): level on the
+// correlated prefill layer (8.12-8.14 against 8.07-8.22 ms) and the
+// Mixtral-shaped one (4.76 against 4.79 ms), slower on the DSV2-Lite-shaped
+// (1.52 against 1.45 ms) and OLMoE-shaped (0.463 against 0.414 ms) layers.  They
+// ran ~100 MHz higher under the same power cap: fewer bytes into each SM per
+// FLOP, but the accumulator is not double-buffered, so every tile's epilogue
+// stalls the tensor pipe.
+#ifndef MOE_WIDE_MIN_AVG_ROWS
+#define MOE_WIDE_MIN_AVG_ROWS 0
+#endif
+
 // GEMM over the groups, on CTA pairs when the groups are tall enough to fill
 // 256-row tiles (and the rows are read in place), else on single CTAs.  In
 // hybrid mode a group's tail of at most 128 rows goes to a second,
@@ -382,6 +399,16 @@ int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a
   if ((g_debug_flags & kDebugForceHybrid) && pair_ok) {
     pair = true;
     hybrid = true;
+  }
+  if constexpr (!TF32 && !B_MN && (EPI == moe::kEpiSwiGLU || EPI == moe::kEpiScale)) {
+    // 256 x 512 pair tiles, one accumulator: half the row-operand bytes into each
+    // SM per FLOP of the 256 x 256 tiles, for tall groups
+    const bool wide_tall = MOE_WIDE_MIN_AVG_ROWS > 0 &&
+                           (long long)m_cap >= (long long)MOE_WIDE_MIN_AVG_ROWS * G;
+    if (pair && !hybrid && N % 512 == 0 && !(g_debug_flags & kDebugNoWideTiles) &&
+        ((g_debug_flags & kDebugWideTiles) || wide_tall))
+      return launch_gemm_pair<512, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
+                                                    row_scale, out, ldo, ex, st);
   }
   if (pair) {
     GemmExtra exp = ex;
