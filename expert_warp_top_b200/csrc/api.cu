@@ -559,7 +559,7 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   auto* tot = reinterpret_cast<unsigned long long*>(total);
   auto* rem = reinterpret_cast<unsigned long long*>(remote);
 #define MOE_ROUTE_BRIM(KM)                                                                    \
-  MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM>, dim3(n_tiles), dim3(1024), 0, stream,    \
+  MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM>, dim3(n_tiles), dim3(moe::kRouteTileThreads), 0, stream,    \
                     logits, T, E, k, renorm, slot_of, R, prune_m, n_tiles, topk_idx, topk_w,    \
                     masks, per_rank, tot, rem, di->err_flag));                                  \
   MOE_CUDA(launch_k(moe::brim_colscan_kernel<KM>, dim3(ncol + n_hist), dim3(1024), 0, stream, \

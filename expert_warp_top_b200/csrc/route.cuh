@@ -25,25 +25,34 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Routes one token with the whole warp.  On return lane j < k holds the j-th
-// selected expert id in *sel_id and its gate weight in *gate (other lanes:
-// unspecified).  All lanes must call it.
-__device__ __forceinline__ void route_token_warp(const float* __restrict__ row, int E, int k,
-                                                 int renorm, int* sel_id_out, float* gate_out) {
+// This lane's logits of one token: lane i holds logits i, i + 32, ... (the
+// slots past E hold -inf and are never selected).
+__device__ __forceinline__ void load_token_logits(const float* __restrict__ row, int E,
+                                                  float (&v)[kRouteMaxPerLane]) {
   const unsigned lane = lane_id();
-  float v[kRouteMaxPerLane];
+  const int per_lane = (E + 31) >> 5;
+#pragma unroll
+  for (int i = 0; i < kRouteMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = (i < per_lane && e < E) ? __ldg(row + e) : -INFINITY;
+  }
+}
+
+// Routes one token with the whole warp, from its logits as load_token_logits
+// leaves them.  On return lane j < k holds the j-th selected expert id in
+// *sel_id and its gate weight in *gate (other lanes: unspecified).  All lanes
+// must call it.
+__device__ __forceinline__ void route_token_warp_v(const float (&v)[kRouteMaxPerLane], int E,
+                                                   int k, int renorm, int* sel_id_out,
+                                                   float* gate_out) {
+  const unsigned lane = lane_id();
   uint32_t key[kRouteMaxPerLane];
   const int per_lane = (E + 31) >> 5;
 #pragma unroll
   for (int i = 0; i < kRouteMaxPerLane; ++i) {
     const int e = lane + 32 * i;
-    if (i < per_lane && e < E) {
-      v[i] = __ldg(row + e);
-      key[i] = float_order_key(v[i]);
-    } else {
-      v[i] = -INFINITY;
-      key[i] = 0u;  // below every real key; never selected (valid[] is false)
-    }
+    // below every real key; never selected (valid[] is false)
+    key[i] = (i < per_lane && e < E) ? float_order_key(v[i]) : 0u;
   }
   unsigned valid = 0;  // bit i: slot i of this lane is a live candidate
 #pragma unroll
@@ -99,6 +108,13 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ row, 
   }
   *sel_id_out = sel_id;
   *gate_out = expf(sel_logit - m) / denom;
+}
+
+__device__ __forceinline__ void route_token_warp(const float* __restrict__ row, int E, int k,
+                                                 int renorm, int* sel_id_out, float* gate_out) {
+  float v[kRouteMaxPerLane];
+  load_token_logits(row, E, v);
+  route_token_warp_v(v, E, k, renorm, sel_id_out, gate_out);
 }
 
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,

@@ -2,8 +2,8 @@
 // one kernel (pass 1 of the BRIM build fused with routing).
 //
 // The same computation as moe_route_topk + brim_mask_kernel +
-// moe_count_dispatched_rows: one block of 32 warps per 32-token tile.  Each
-// warp routes one token (route_token_warp, the very code of moe_route_topk);
+// moe_count_dispatched_rows: one block of 16 warps per 32-token tile.  Each
+// warp routes two tokens (route_token_warp_v, the very code of moe_route_topk);
 // warp 0 then takes the tile lane-per-token, prunes (when asked), writes the
 // top-k, builds the tile's column masks and adds the tile's contribution to
 // the counter.  The column scan with the histogram (brim_colscan_kernel) and
@@ -14,8 +14,14 @@
 
 namespace moe {
 
+// Tokens each warp routes (its logits loaded together up front): the block is
+// 32 / kRouteTokensPerWarp warps, so two blocks fit on an SM and one block's
+// tile work overlaps another's routing.
+constexpr int kRouteTokensPerWarp = 2;
+constexpr int kRouteTileThreads = 32 * (kBrimTileTokens / kRouteTokensPerWarp);
+
 template <int KMAX>
-__global__ void __launch_bounds__(1024) route_brim_tile_kernel(
+__global__ void __launch_bounds__(kRouteTileThreads, 2) route_brim_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     const int32_t* __restrict__ slot_of, int R, int prune_m, int n_tiles,
     int32_t* __restrict__ topk_idx,
@@ -31,15 +37,26 @@ __global__ void __launch_bounds__(1024) route_brim_tile_kernel(
   const int tile = blockIdx.x;
   const int L = E / R, ncol = R + E;
 
-  // 1. each warp routes one token of the tile
+  // 1. warp w routes tokens w, w + 16 of the tile (both rows' logits loaded first)
   {
-    const int t = tile * kBrimTileTokens + warp;
-    int id = -1;
-    float gate = 0.f;
-    if (t < T) route_token_warp(logits + (size_t)t * E, E, k, renorm, &id, &gate);
-    if ((int)lane < KMAX) {
-      s_ids[warp][lane] = (t < T && (int)lane < k) ? id : -1;
-      s_gates[warp][lane] = (t < T && (int)lane < k) ? gate : 0.f;
+    constexpr int kWarps = kRouteTileThreads / 32;
+    float v[kRouteTokensPerWarp][kRouteMaxPerLane];
+#pragma unroll
+    for (int u = 0; u < kRouteTokensPerWarp; ++u) {
+      const int t = tile * kBrimTileTokens + warp + u * kWarps;
+      if (t < T) load_token_logits(logits + (size_t)t * E, E, v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kRouteTokensPerWarp; ++u) {
+      const int i = warp + u * kWarps;
+      const int t = tile * kBrimTileTokens + i;
+      int id = -1;
+      float gate = 0.f;
+      if (t < T) route_token_warp_v(v[u], E, k, renorm, &id, &gate);
+      if ((int)lane < KMAX) {
+        s_ids[i][lane] = (t < T && (int)lane < k) ? id : -1;
+        s_gates[i][lane] = (t < T && (int)lane < k) ? gate : 0.f;
+      }
     }
   }
   __syncthreads();
