@@ -962,6 +962,113 @@ def run_shuffle(args, cfg):
         dist.destroy_process_group()
 
 
+EP_METRIC = ("expert-parallel MoE-layer tokens/s (route + BRIM + SFD rows out by all-to-all-v "
+             "+ destination BRIM/EPD + grouped GEMMs + pre-reduce + return rows by "
+             "all-to-all-v + combine)")
+
+
+def run_ep(args, cfg):
+    """Real expert parallelism (expert_warp_top_b200/ep.py).  Under torchrun each
+    of the N ranks is an EP rank (R = N) with T / N of the workload's tokens and
+    the experts at its slots, exchanging over NCCL; with one process, the
+    workload's R ranks run on the one GPU and exchange through loopback copies
+    (every rank's kernels and copies on that GPU, one after another)."""
+    import datetime
+    import torch.distributed as dist
+    from expert_warp_top_b200 import _binding as B
+    from expert_warp_top_b200.ep import DistExchange, EPRank, LoopbackExchange, ep_forward
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    R = world if world > 1 else cfg.R
+    cfg = cfg.with_(R=R)
+    if cfg.E % R or cfg.T % R:
+        raise SystemExit(f"--ep needs R = {R} to divide E = {cfg.E} and T = {cfg.T}")
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        ex = DistExchange()
+        mine = [rank]
+    else:
+        ex = LoopbackExchange(R)
+        mine = list(range(R))
+    L, Tr = cfg.E // R, cfg.T // R
+    inp = inputs.make_inputs(cfg, device=dev)  # the same seeded batch and weights on every rank
+    slot_of, placement_info = placement(cfg, args.placement, dev, inp["logits"])
+    at = torch.empty(cfg.E, dtype=torch.long)
+    at[slot_of.long()] = torch.arange(cfg.E)
+    ranks, lgs, xs = [], [], []
+    for r in mine:
+        e = at[r * L:(r + 1) * L].to(dev)
+        kw = {}
+        if cfg.S:
+            kw = dict(S=cfg.S, fs=cfg.fs, sg=inp["sg"], su=inp["su"], sd=inp["sd"])
+        ranks.append(EPRank(rank=r, R=R, T=Tr, d=cfg.d, f=cfg.f, E=cfg.E, k=cfg.k,
+                            renorm=cfg.renorm, dtype=inputs.torch_dtype(cfg), slot_of=slot_of,
+                            wg=inp["wg"][e], wu=inp["wu"][e], wd=inp["wd"][e], device=dev, **kw))
+        lgs.append(inp["logits"][r * Tr:(r + 1) * Tr].contiguous())
+        xs.append(inp["x"][r * Tr:(r + 1) * Tr].contiguous())
+    for key in ("wg", "wu", "wd"):
+        inp.pop(key)
+    stream = torch.cuda.current_stream(dev)
+    names = ("start", "sent", "exchanged", "computed", "returned", "end")
+    ev = {n: torch.cuda.Event(enable_timing=True) for n in names}
+    marks = lambda n: ev[n].record(stream)  # noqa: E731
+    for _ in range(args.warmup):
+        ep_forward(ranks, ex, lgs, xs)
+    torch.cuda.synchronize(dev)
+    if B.moe_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    step_ms, phase_ms = [], {n: [] for n in names[1:]}
+    with ClockSampler(local_rank) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev["start"].record(stream)
+            ep_forward(ranks, ex, lgs, xs, marks=marks)
+            ev["end"].record(stream)
+            ev["end"].synchronize()
+            step_ms.append(ev["start"].elapsed_time(ev["end"]))
+            prev = "start"
+            for n in names[1:]:
+                phase_ms[n].append(ev[prev].elapsed_time(ev[n]))
+                prev = n
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    if B.moe_get_device_status() != 0:
+        raise RuntimeError("device status after the timed steps")
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
+    counts = ep_forward.counts
+    c_t = sum(sum(row) for row in counts)
+    e = 2 if cfg.dtype == "bf16" else 4
+    wire = sum(counts[s][q] for s in range(R) for q in range(R) if s != q)
+    if rank == 0:
+        line = {
+            "metric": EP_METRIC, "value": cfg.T * args.steps / (total_ms * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": dict(config_obj(cfg, args), parallelism=(
+                f"expert parallel over {world} GPUs (NCCL)" if world > 1 else
+                f"{R} expert-parallel ranks on one GPU, loopback exchange")),
+            "placement": placement_info,
+            "ep": {"ranks": R, "c_t": c_t, "rows_between_ranks": wire,
+                   "payload_bytes_each_way": wire * cfg.d * e,
+                   "phase_ms": {n: statistics.mean(v) for n, v in phase_ms.items()}},
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    del ranks
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def placement(cfg, how, dev, logits):
     """slot_of for the run ("contiguous", or "histogram": correlated placement
     from the expert co-activation histogram of a separate calibration batch,
@@ -1073,6 +1180,9 @@ def main():
     ap.add_argument("--placement", default="contiguous", choices=["contiguous", "histogram"])
     ap.add_argument("--shuffle", action="store_true",
                     help="time token shuffling across two layers (correlated prefill workload)")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the real expert-parallel layer: R = N ranks over NCCL under "
+                         "torchrun, or the workload's R ranks on one GPU (loopback)")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (forward + backward) instead of the forward")
     ap.add_argument("--prune", type=int, default=0,
@@ -1095,6 +1205,8 @@ def main():
         run_train(args, cfg)
     elif args.shuffle:
         run_shuffle(args, cfg)
+    elif args.ep:
+        run_ep(args, cfg)
     else:
         run_ours(args, cfg)
 

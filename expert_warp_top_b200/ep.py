@@ -108,15 +108,21 @@ def pair_counts(offs, R):
     return [[offs[s][q + 1] - offs[s][q] for q in range(R)] for s in range(R)]
 
 
-def ep_forward(ranks, exchange, logits, xs):
+def ep_forward(ranks, exchange, logits, xs, marks=None):
     """One forward of the expert-parallel layer over the ranks this process
     holds (ranks[i] is rank exchange.ranks[i]; logits[i], xs[i] its batch).
     Returns each rank's output y [T_r, d] (a view of its buffer) and keeps
-    every intermediate in the rank objects."""
+    every intermediate in the rank objects.  `marks`, if given, is called with
+    a phase name ("sent", "exchanged", "computed", "returned") as each phase
+    ends (e.g. to record CUDA events), and the pair counts of the forward are
+    kept in `ep_forward.counts`."""
     R = exchange.R
+    mark = marks or (lambda name: None)
     for r, lg, x in zip(ranks, logits, xs):
         r.send_phase(lg, x)
+    mark("sent")
     counts = pair_counts(exchange.gather_offsets([r.sfd_off for r in ranks]), R)
+    ep_forward.counts = counts
     send_splits = [counts[q] for q in exchange.ranks]
     recv_splits = [[counts[s][q] for s in range(R)] for q in exchange.ranks]
     for r, rs in zip(ranks, recv_splits):
@@ -125,9 +131,12 @@ def ep_forward(ranks, exchange, logits, xs):
     exchange.rows([r.idx_send for r in ranks], send_splits, [r.idx_recv for r in ranks],
                   recv_splits)
     exchange.rows([r.w_send for r in ranks], send_splits, [r.w_recv for r in ranks], recv_splits)
+    mark("exchanged")
     for r, rs in zip(ranks, recv_splits):
         r.recv_phase(sum(rs))
+    mark("computed")
     exchange.rows([r.y_recv for r in ranks], recv_splits, [r.y_ret for r in ranks], send_splits)
+    mark("returned")
     for r in ranks:
         r.combine_phase()
     return [r.y for r in ranks]

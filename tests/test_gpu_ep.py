@@ -151,3 +151,26 @@ def test_ep_nccl_one_rank():
         assert rowwise_rel_err(y.float().cpu().numpy(), y_ref) <= OUT_RTOL
     finally:
         dist.destroy_process_group()
+
+
+def test_bench_ep_mode_line():
+    """`bench.py --ep` on the tiny workload (4 loopback ranks on the one GPU):
+    one JSON line whose C_T is the counter's, whose rows between ranks are the
+    off-diagonal pair counts, and whose phases add up to the step."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--ep", "--config", "tiny",
+                        "--steps", "3", "--warmup", "3"], capture_output=True, text=True,
+                       timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    cfg = inputs.CONFIGS["tiny"]
+    ep = line["ep"]
+    assert ep["ranks"] == cfg.R and line["config"]["R"] == cfg.R
+    assert ep["c_t"] == line["placement"]["c_t_contiguous"]
+    assert 0 <= ep["rows_between_ranks"] <= ep["c_t"]
+    assert ep["payload_bytes_each_way"] == ep["rows_between_ranks"] * cfg.d * 2
+    assert abs(sum(ep["phase_ms"].values()) - line["ms_per_step"]) <= 0.05 * line["ms_per_step"]
+    assert line["value"] > 0 and line["unit"] == "tokens/s"
