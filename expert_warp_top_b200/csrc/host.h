@@ -457,7 +457,7 @@ int launch_wgrad_bn(DeviceInfo* di, const void* a, const void* b, int rows, int 
   const int grid = (int)(tiles < di->num_sms ? (tiles < 1 ? 1 : tiles) : di->num_sms);
   moe::WgradArgs args{group_off, G, M, N, rows, out, accumulate, di->err_flag, wait_limit_ns(),
                       g_debug_flags};
-  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kGemmThreads), Cfg::kSmemBytes, st, ta, tb, to,
+  MOE_CUDA(launch_k(kern, dim3(grid), dim3(moe::kWgradThreads), Cfg::kSmemBytes, st, ta, tb, to,
                     args));
   MOE_LAUNCHED("wgrad_gemm_kernel");
   return MOE_OK;
@@ -487,7 +487,7 @@ int launch_wgrad_pair(DeviceInfo* di, const void* a, const void* b, int rows, in
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(moe::kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(moe::kWgradThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -519,12 +519,13 @@ int launch_wgrad_pair(DeviceInfo* di, const void* a, const void* b, int rows, in
 template <typename TOut>
 int launch_wgrad(DeviceInfo* di, const void* a, const void* b, int rows, int M, int N,
                  const int32_t* group_off, int G, void* out, int accumulate, cudaStream_t st) {
-  // The CTA-pair kernel moves a third less operand traffic per FLOP.  On the
-  // OLMoE-shaped backward it measured level with the single-CTA kernel
-  // (backward expert GEMMs 1.140-1.157 against 1.127-1.128 ms), so the
-  // single-CTA kernel stays the default and the pair is kept, tested, behind
-  // kDebugForcePair.
-  const bool pair = M % 256 == 0 && N % 128 == 0 && (g_debug_flags & kDebugForcePair);
+  // The CTA-pair kernel moves a third less operand traffic per FLOP into each
+  // SM, so its six stages cover more of the load latency than the single-CTA
+  // kernel's four.  Alone on one B200 (fp32 out, ragged groups) it measured
+  // 1175 against 1250 us on the DSV2-Lite-shaped gate/up gradient and 219
+  // against 225 us on the OLMoE-shaped down gradient, so it is the default
+  // where the shape allows; kDebugForceSingle keeps the single-CTA kernel.
+  const bool pair = M % 256 == 0 && N % 128 == 0 && !(g_debug_flags & kDebugForceSingle);
   if (pair) {
     if (N % 256 == 0)
       return launch_wgrad_pair<256, TOut>(di, a, b, rows, M, N, group_off, G, out, accumulate, st);

@@ -7,16 +7,22 @@
 // rows, whose count is ragged.  This is the weight gradient of a grouped
 // GEMM: dW_down[g] = dO_g^T (w h)_g and dW_gate/up[g] = dZ_g^T X_g.
 //
-// Kernel shape (one persistent CTA per SM, 192 threads), as the forward GEMM:
+// Kernel shape (one persistent CTA per SM, 224 threads):
 //   warp 0      TMA producer: per stage 64 rows of A (128 columns) and of B (BN
 //               columns), each one 3-D load of 64-column strips (the tensor
 //               seen as {64, rows, cols/64}), 128-byte swizzle
-//   warp 1      MMA issuer (lane 0) and tail fixer (whole warp): in a group's
-//               last, partial row block the rows past the group's end belong
-//               to the next group, so the MMAs stop at the 16-row block that
-//               holds the group's last row and the warp zeroes that block's
-//               foreign rows in shared memory (a 128-byte row of a swizzled
-//               box holds exactly one row) before the MMAs read the stage
+//   warp 1      MMA issuer, lane 0 alone: four MMAs per stage, unrolled, with
+//               no warp-wide step between stages (a per-stage shuffle and two
+//               warp syncs held the MMA rate to two thirds of the lane-0 loop)
+//   warp 6      tail fixer: in a group's last, partial row block the rows past
+//               the group's end belong to the next group, so the MMAs stop at
+//               the 16-row block that holds the group's last row, and this
+//               warp zeroes that block's foreign rows in shared memory (a
+//               128-byte row of a swizzled box holds exactly one row) and then
+//               signals the stage's fixed barrier, which the issuer waits for
+//               on those stages only; the zeroing overlaps earlier MMAs.  It
+//               waits for every fill and takes part in releasing every stage,
+//               so its phase tracking stays exact
 //   warps 2..5  epilogue: tcgen05.ld of 32 accumulator rows (= 32 values of m),
 //               staged 128 bytes per row (32 fp32 or 64 bf16 columns) into one
 //               of two 128-byte-swizzled shared-memory boxes of this warp
@@ -50,6 +56,8 @@ struct WgradArgs {
   int debug;
 };
 
+constexpr int kWgradThreads = 224;  // 7 warps: producer, issuer, 4 epilogue, tail fixer
+
 template <int BN>
 struct WgradCfg {
   static constexpr int kBK = 64;                     // rows (the K of this GEMM) per stage
@@ -61,14 +69,14 @@ struct WgradCfg {
   static constexpr int kStoreBoxBytes = 32 * 128;  // one staging box: 32 rows x 128 bytes
   static constexpr int kStoreBoxes = 8;             // two per epilogue warp
   static constexpr size_t kSmemBytes =
-      1024 + (size_t)kStages * kStageBytes + kStoreBoxes * kStoreBoxBytes + 256;
+      1024 + (size_t)kStages * kStageBytes + kStoreBoxes * kStoreBoxBytes + 512;
 };
 
 // tmap_a / tmap_b: A and B as 64-column strips (encode_strips), boxes of 64
 // rows x 2 strips (A) and 64 rows x BN/64 strips (B).  tmap_out: the output as
 // a 2-D [G*M, N] tensor of TOut, box of 32 rows x 128 bytes, 128-byte swizzle.
 template <int BN, typename TOut>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kWgradThreads, 1)
     wgrad_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_out, const WgradArgs args) {
@@ -89,7 +97,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull_bar = bars + 2 * S;
   uint64_t* tempty_bar = bars + 2 * S + 2;
   uint64_t* drain_bar = bars + 2 * S + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  uint64_t* fixed_bar = bars + 2 * S + 5;  // [S]: a tail stage's foreign rows are zeroed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -105,7 +114,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tma_prefetch_desc(&tmap_out);
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
-      tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
+      tc::mbar_init(tc::smem_u32(&empty_bar[s]), 2);  // the MMAs' commit and the tail fixer
+      tc::mbar_init(tc::smem_u32(&fixed_bar[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(tc::smem_u32(&tfull_bar[a]), 1);
@@ -200,75 +210,109 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
     }
   } else if (warp == 1) {
-    // ------------------------------------------- MMA issuer + tail zeroing
-    constexpr uint32_t idesc = tc::idesc_f32acc<false, 128, BN, true, true>();
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_f32acc<false, 128, BN, true, true>();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fixed_parity = 0;  // per stage: the next completion of its fixed barrier
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int g, m0, n0, r0, r1;
+        locate(tile, g, m0, n0);
+        group_rows(g, r0, r1);
+        const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
+        if (!tc::wait_bounded(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl)) break;
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
+          bool got = tc::wait_bounded(tc::smem_u32(&full_bar[stage]), phase, wctl);
+          if (got && valid % 16 != 0) {
+            got = tc::wait_bounded(tc::smem_u32(&fixed_bar[stage]), (fixed_parity >> stage) & 1u,
+                                   wctl);
+            fixed_parity ^= 1u << stage;
+          }
+          if (!got) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t sa_u = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
+          const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
+          const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
+          // Unrolled with a guard per MMA: a loop bounded at run time cost a
+          // fifth of the MMA rate.
+          const int n_kk = (valid + 15) / 16;
+#pragma unroll
+          for (int kk = 0; kk < Cfg::kBK / 16; ++kk) {
+            // +16 rows = two 1024-byte atoms = +128 in the address field
+            const uint64_t off = static_cast<uint64_t>(kk * 128);
+            if (kk < n_kk) tc::mma_f16(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+          }
+          tc::commit(tc::smem_u32(&empty_bar[stage]));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::commit(tc::smem_u32(&tfull_bar[acc]));  // also for an empty group
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc::commit(tc::smem_u32(drain_bar));
+      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ tail fixer
+    // The same stage sequence as the producer and the issuer.  It waits for
+    // every fill in order and releases every stage (the empty barrier counts
+    // its arrival beside the MMAs' commit), so it can neither run a fill ahead
+    // of the loads nor be lapped by them; only stages holding a group's
+    // partial last row block are written.
     int stage = 0;
     uint32_t phase = 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       int g, m0, n0, r0, r1;
       locate(tile, g, m0, n0);
       group_rows(g, r0, r1);
       const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
-      bool go = true;
-      if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl);
-      if (!__shfl_sync(0xffffffffu, go, 0)) break;
-      tc::fence_after_sync();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (lane == 0) go = tc::wait_bounded(tc::smem_u32(&full_bar[stage]), phase, wctl);
-        if (!__shfl_sync(0xffffffffu, go, 0)) {
+        bool got = true;
+        if (lane == 0) got = tc::wait_bounded(tc::smem_u32(&full_bar[stage]), phase, wctl);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
           ok = false;
           break;
         }
-        tc::fence_after_sync();
-        uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
         const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
         if (valid % 16 != 0) {
           // Rows valid.. of every strip belong to another group (or lie past
           // the tensor).  The MMAs read the stage in 16-row blocks up to the
           // one holding row valid - 1, so only that block's rows past valid
           // are zeroed; later rows are never read.
+          uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
           const int n16 = (((valid + 15) & ~15) - valid) * 8;  // 16-byte pieces per strip
           for (int c = 0; c < kChunks; ++c)
             for (int q = (int)lane; q < n16; q += 32)
               st_v4(sa + c * 8192 + valid * 128 + q * 16, make_uint4(0u, 0u, 0u, 0u));
           tc::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(tc::smem_u32(&fixed_bar[stage]));
         }
-        __syncwarp();
-        if (lane == 0) {
-          const uint32_t sa_u = tc::smem_u32(sa);
-          const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
-          const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
-          const int n_kk = (valid + 15) / 16;
-          for (int kk = 0; kk < n_kk; ++kk) {
-            // +16 rows = two 1024-byte atoms = +128 in the address field
-            const uint64_t off = static_cast<uint64_t>(kk * 128);
-            tc::mma_f16(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
-          }
-          tc::commit(tc::smem_u32(&empty_bar[stage]));
-        }
-        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(tc::smem_u32(&empty_bar[stage]));
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      if (!ok) break;
-      if (lane == 0) tc::commit(tc::smem_u32(&tfull_bar[acc]));  // also for an empty group
-      __syncwarp();
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
     }
-    if (lane == 0) {
-      tc::commit(tc::smem_u32(drain_bar));
-      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;

@@ -12,12 +12,16 @@
 //   warp 0      TMA producer: this CTA's A strips and B half, into its own
 //               shared memory; both CTAs' loads count their bytes on CTA 0's
 //               full barrier, which CTA 0 arms for the pair (no multicast)
-//   warp 1      CTA 0 only: once a stage has landed in both CTAs, zeroes the
-//               foreign rows of a ragged group's last 16-row block in both
-//               CTAs' boxes (the peer's through distributed shared memory),
-//               then its lane 0 issues the pair MMAs, whose commits free the
-//               stage in both CTAs (multicast) and hand the accumulator to
-//               both epilogues
+//   warp 1      CTA 0 only, lane 0 alone: issues the pair MMAs, whose commits
+//               free the stage in both CTAs (multicast) and hand the
+//               accumulator to both epilogues
+//   warp 6      CTA 0 only, tail fixer: once a stage holding a ragged group's
+//               last 16-row block has landed in both CTAs, zeroes that block's
+//               foreign rows in both CTAs' boxes (the peer's through
+//               distributed shared memory) and signals the stage's fixed
+//               barrier, which the issuer waits for on those stages only.  It
+//               waits for every fill and its arrival is counted by CTA 0's
+//               empty barrier, so its phase tracking stays exact.
 //   warps 2..5  epilogue of this CTA's 128 accumulator rows, through TMA
 //               stores as in wgrad_gemm.cuh; they arrive on CTA 0's tempty
 //               barrier (remotely from CTA 1)
@@ -60,7 +64,7 @@ struct WgradPairCfg {
 // box 64 rows x BN/128 strips; tmap_out: the output [G*M, N], box 32 rows x
 // 128 bytes.  M % 256 == 0, N % BN == 0.
 template <int BN, typename TOut>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kWgradThreads, 1)
     wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_out, const WgradArgs args) {
@@ -81,7 +85,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull_bar = bars + 2 * S;      // [2] MMA (multicast) -> epilogues
   uint64_t* tempty_bar = bars + 2 * S + 2; // [2] CTA 0: 8 epilogue warps -> MMA issuer
   uint64_t* drain_bar = bars + 2 * S + 4;  // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  uint64_t* fixed_bar = bars + 2 * S + 5;  // [S] CTA 0: tail fixer -> MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -99,7 +104,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tma_prefetch_desc(&tmap_out);
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(tc::smem_u32(&full_bar[s]), 1);
-      tc::mbar_init(tc::smem_u32(&empty_bar[s]), 1);
+      // CTA 0's stage is released by the MMAs' commit and by the tail fixer
+      tc::mbar_init(tc::smem_u32(&empty_bar[s]), rank == 0 ? 2 : 1);
+      tc::mbar_init(tc::smem_u32(&fixed_bar[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(tc::smem_u32(&tfull_bar[a]), 1);
@@ -195,13 +202,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc::wait_bounded(tc::smem_u32(&full_bar[s]), (armed_parity >> s) & 1u, wctl, false);
     }
   } else if (warp == 1) {
-    // ------------------------------------ CTA 0: tail zeroing + MMA issuer
+    // ------------------------------------------------------ CTA 0: MMA issuer
     // (CTA 1's warp 1 has nothing to do after allocating TMEM)
-    if (rank == 0) {
+    if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc = tc::idesc_f32acc<false, 256, BN, true, true>();
-      const uint32_t peer_tiles = tc::mapa_shared(tc::smem_u32(tiles), 1);  // CTA 1's ring
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t fixed_parity = 0;  // per stage: the next completion of its fixed barrier
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -210,27 +217,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         locate(tile, g, m0, n0);
         group_rows(g, r0, r1);
         const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
-        bool go = true;
-        if (lane == 0)
-          go = tc::wait_bounded_cluster(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl);
-        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        if (!tc::wait_bounded_cluster(tc::smem_u32(&tempty_bar[acc]), acc_phase ^ 1u, wctl)) break;
         tc::fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < k_blocks; ++kb) {
-          if (lane == 0) go = tc::wait_bounded_cluster(tc::smem_u32(&full_bar[stage]), phase, wctl);
-          if (!__shfl_sync(0xffffffffu, go, 0)) {
+          const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
+          bool got = tc::wait_bounded_cluster(tc::smem_u32(&full_bar[stage]), phase, wctl);
+          if (got && valid % 16 != 0) {
+            got = tc::wait_bounded_cluster(tc::smem_u32(&fixed_bar[stage]),
+                                           (fixed_parity >> stage) & 1u, wctl);
+            fixed_parity ^= 1u << stage;
+          }
+          if (!got) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
           const uint32_t sa_u = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
+          const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
+          const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
+          // unrolled with a guard per MMA, as in the single-CTA kernel
+          const int n_kk = (valid + 15) / 16;
+#pragma unroll
+          for (int kk = 0; kk < Cfg::kBK / 16; ++kk) {
+            // +16 rows = two 1024-byte atoms = +128 in the address field
+            const uint64_t off = static_cast<uint64_t>(kk * 128);
+            if (kk < n_kk) tc::mma_f16_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
+          }
+          // frees the stage in both CTAs once these MMAs have read it
+          tc::commit_pair_multicast(tc::smem_u32(&empty_bar[stage]), 0x3);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::commit_pair_multicast(tc::smem_u32(&tfull_bar[acc]), 0x3);  // also for an empty group
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc::commit_pair_multicast(tc::smem_u32(drain_bar), 0x1);
+      tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------ CTA 0: tail fixer
+    if (rank == 0) {
+      const uint32_t peer_tiles = tc::mapa_shared(tc::smem_u32(tiles), 1);  // CTA 1's ring
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        int g, m0, n0, r0, r1;
+        locate(tile, g, m0, n0);
+        group_rows(g, r0, r1);
+        const int k_blocks = (r1 - r0 + Cfg::kBK - 1) / Cfg::kBK;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          bool got = true;
+          if (lane == 0) got = tc::wait_bounded_cluster(tc::smem_u32(&full_bar[stage]), phase, wctl);
+          if (!__shfl_sync(0xffffffffu, got, 0)) {
+            ok = false;
+            break;
+          }
           const int valid = min(Cfg::kBK, r1 - (r0 + kb * Cfg::kBK));
           if (valid % 16 != 0) {
-            // Rows valid.. of every strip, in both CTAs, belong to another group.
-            // The MMAs read the stage in 16-row blocks up to the one holding row
-            // valid - 1, so only that block's rows past valid are zeroed.  The
-            // full barrier has seen both CTAs' bytes land, so these stores come
-            // after the TMA writes; the proxy fence orders them before the MMAs.
+            // Rows valid.. of every strip, in both CTAs, belong to another
+            // group.  The MMAs read the stage in 16-row blocks up to the one
+            // holding row valid - 1, so only that block's rows past valid are
+            // zeroed.  The full barrier has seen both CTAs' bytes land, so
+            // these stores come after the TMA writes; the proxy fence and the
+            // cluster-scope arrive order them before the MMAs.
             const int n16 = (((valid + 15) & ~15) - valid) * 8;  // 16-byte pieces per strip
             const uint32_t peer = peer_tiles + static_cast<uint32_t>(stage * Cfg::kStageBytes);
             for (int c = 0; c < kChunks; ++c)
@@ -240,40 +298,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc::st_cluster_v4(peer + off, make_uint4(0u, 0u, 0u, 0u));
               }
             tc::fence_proxy_async_smem_cluster();
+            __syncwarp();
+            if (lane == 0)
+              tc::mbar_arrive_remote(tc::mapa_shared(tc::smem_u32(&fixed_bar[stage]), 0));
           }
-          __syncwarp();
-          if (lane == 0) {
-            const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
-            const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
-            const int n_kk = (valid + 15) / 16;
-            for (int kk = 0; kk < n_kk; ++kk) {
-              // +16 rows = two 1024-byte atoms = +128 in the address field
-              const uint64_t off = static_cast<uint64_t>(kk * 128);
-              tc::mma_f16_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | kk) != 0);
-            }
-            // frees the stage in both CTAs once these MMAs have read it
-            tc::commit_pair_multicast(tc::smem_u32(&empty_bar[stage]), 0x3);
-          }
-          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(tc::smem_u32(&empty_bar[stage]));
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (!ok) break;
-        if (lane == 0)  // also for an empty group
-          tc::commit_pair_multicast(tc::smem_u32(&tfull_bar[acc]), 0x3);
-        __syncwarp();
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
       }
-      if (lane == 0) {
-        tc::commit_pair_multicast(tc::smem_u32(drain_bar), 0x1);
-        tc::wait_bounded(tc::smem_u32(drain_bar), 0u, wctl, false);
-      }
-      __syncwarp();
     }
   } else {
     // ------------------------------------------------------------ epilogue
