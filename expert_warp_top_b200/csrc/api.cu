@@ -410,8 +410,25 @@ int moe_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t
   MOE_REQUIRE(logits && topk_idx && topk_w, MOE_ERR_INVALID_ARG, "null pointer");
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
-  const int blocks = (T + 7) / 8;
-  MOE_CUDA(launch_k(moe::route_topk_kernel, blocks, 256, 0, stream, logits, T, E, k, renorm, topk_idx, topk_w));
+  // G lanes per token (the result does not depend on G)
+  const int G = moe::route_lanes_per_token(T, di->num_sms);
+  const int blocks = (int)(((long long)T * G + 255) / 256);
+#define MOE_ROUTE_TOPK(KM, GG)                                                                \
+  MOE_CUDA(launch_k(moe::route_topk_kernel<KM, GG>, blocks, 256, 0, stream, logits, T, E, k,  \
+                    renorm, topk_idx, topk_w))
+#define MOE_ROUTE_TOPK_G(KM)                                                                   \
+  do {                                                                                        \
+    if (G == 8) MOE_ROUTE_TOPK(KM, 8);                                                        \
+    else if (G == 4) MOE_ROUTE_TOPK(KM, 4);                                                   \
+    else if (G == 2) MOE_ROUTE_TOPK(KM, 2);                                                   \
+    else MOE_ROUTE_TOPK(KM, 1);                                                               \
+  } while (0)
+  if (k <= 2) MOE_ROUTE_TOPK_G(2);
+  else if (k <= 4) MOE_ROUTE_TOPK_G(4);
+  else if (k <= 8) MOE_ROUTE_TOPK_G(8);
+  else MOE_ROUTE_TOPK_G(16);
+#undef MOE_ROUTE_TOPK_G
+#undef MOE_ROUTE_TOPK
   MOE_LAUNCHED("route_topk_kernel");
   return MOE_OK;
 }
@@ -558,10 +575,22 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   const int n_hist = hist ? hist_blocks(T, &hist_tokens) : 0;
   auto* tot = reinterpret_cast<unsigned long long*>(total);
   auto* rem = reinterpret_cast<unsigned long long*>(remote);
+  const int G = moe::route_lanes_per_token(T, di->num_sms);
+#define MOE_ROUTE_TILE(KM, GG)                                                                \
+  MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM, GG>,                                     \
+                    dim3((n_tiles + moe::RouteTile<GG>::kTiles - 1) / moe::RouteTile<GG>::kTiles), \
+                    dim3(moe::RouteTile<GG>::kThreads), 0, stream, logits, T, E, k, renorm,    \
+                    slot_of, R, prune_m, n_tiles, topk_idx, topk_w, masks, per_rank, tot, rem,  \
+                    di->err_flag))
+#define MOE_ROUTE_TILE_G(KM)                                                                   \
+  do {                                                                                        \
+    if (G == 8) MOE_ROUTE_TILE(KM, 8);                                                        \
+    else if (G == 4) MOE_ROUTE_TILE(KM, 4);                                                   \
+    else if (G == 2) MOE_ROUTE_TILE(KM, 2);                                                   \
+    else MOE_ROUTE_TILE(KM, 1);                                                               \
+  } while (0)
 #define MOE_ROUTE_BRIM(KM)                                                                    \
-  MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM>, dim3(n_tiles), dim3(moe::kRouteTileThreads), 0, stream,    \
-                    logits, T, E, k, renorm, slot_of, R, prune_m, n_tiles, topk_idx, topk_w,    \
-                    masks, per_rank, tot, rem, di->err_flag));                                  \
+  MOE_ROUTE_TILE_G(KM);                                                                       \
   MOE_CUDA(launch_k(moe::brim_colscan_kernel<KM>, dim3(ncol + n_hist), dim3(1024), 0, stream, \
                     masks, n_tiles, ncol, totals, static_cast<const int32_t*>(topk_idx), T, k,  \
                     E, hist, hist_tokens, di->err_flag));                                       \
@@ -579,6 +608,8 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
     MOE_ROUTE_BRIM(16);
   }
 #undef MOE_ROUTE_BRIM
+#undef MOE_ROUTE_TILE_G
+#undef MOE_ROUTE_TILE
   MOE_LAUNCHED("route_brim_tile_kernel");
   return MOE_OK;
 }

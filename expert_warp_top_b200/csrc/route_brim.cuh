@@ -2,26 +2,76 @@
 // one kernel (pass 1 of the BRIM build fused with routing).
 //
 // The same computation as moe_route_topk + brim_mask_kernel +
-// moe_count_dispatched_rows: one block of 16 warps per 32-token tile.  Each
-// warp routes two tokens (route_token_warp_v, the very code of moe_route_topk);
-// warp 0 then takes the tile lane-per-token, prunes (when asked), writes the
-// top-k, builds the tile's column masks and adds the tile's contribution to
-// the counter.  The column scan with the histogram (brim_colscan_kernel) and
-// the scatter (brim_scatter_kernel) follow.
+// moe_count_dispatched_rows.  Tokens are routed by groups of G lanes
+// (route_token_group, the very code of moe_route_topk; G from the batch size,
+// the result does not depend on it).  Then one warp per 32-token tile, one
+// lane per token, prunes (when asked), writes the top-k, builds the tile's
+// column masks and adds the tile's contribution to the counter.  With G = 1
+// a lane keeps its own token throughout; with G > 1 the routes pass through
+// shared memory.  The column scan with the histogram (brim_colscan_kernel)
+// and the scatter (brim_scatter_kernel) follow.
 #pragma once
 #include "brim.cuh"
 #include "route.cuh"
 
 namespace moe {
 
-// Tokens each warp routes (its logits loaded together up front): the block is
-// 32 / kRouteTokensPerWarp warps, so two blocks fit on an SM and one block's
-// tile work overlaps another's routing.
-constexpr int kRouteTokensPerWarp = 2;
-constexpr int kRouteTileThreads = 32 * (kBrimTileTokens / kRouteTokensPerWarp);
+// threads per block and 32-token tiles per block for G lanes per token
+template <int G>
+struct RouteTile {
+  static constexpr int kThreads = G <= 4 ? 128 : 32 * G;
+  static constexpr int kTiles = kThreads / (32 * G);
+};
 
 template <int KMAX>
-__global__ void __launch_bounds__(kRouteTileThreads, 2) route_brim_tile_kernel(
+__device__ __forceinline__ void route_tile_masks(
+    int t, int tile, int T, int E, int k, int R, int prune_m, int n_tiles,
+    const int32_t* __restrict__ slot_of, int (&ids)[KMAX], float (&gates)[KMAX],
+    uint32_t* s_mask, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+    uint32_t* __restrict__ masks, int32_t* __restrict__ per_rank,
+    unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
+    unsigned* err) {
+  const unsigned lane = lane_id();
+  const int L = E / R, ncol = R + E;
+  if (t < T) {
+    if (prune_m > 0) prune_token<KMAX>(ids, gates, slot_of, k, E, L, prune_m);
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k) {
+        topk_idx[(size_t)t * k + j] = ids[j];
+        topk_w[(size_t)t * k + j] = gates[j];
+      }
+  }
+  TokenRoute<KMAX> tr;
+  const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
+  tile_masks<KMAX>(s_mask, ncol, R, active, k, tr);
+  for (int c = lane; c < ncol; c += 32) masks[(size_t)c * n_tiles + tile] = s_mask[c];
+  if (per_rank) {
+    // tokens per rank: popcount of the rank columns; remote: ranks other than
+    // the token's source rank floor(t * R / T)
+    for (int r = lane; r < R; r += 32) {
+      const int n = __popc(s_mask[r]);
+      if (n) atomicAdd(&per_rank[r], n);
+    }
+    const int src = (int)(((long long)t * R) / (T > 0 ? T : 1));
+    unsigned n_rank = 0, n_remote = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (active && j < k && tr.first[j]) {
+        ++n_rank;
+        n_remote += tr.rank[j] != src;
+      }
+    n_rank = __reduce_add_sync(0xffffffffu, n_rank);
+    n_remote = __reduce_add_sync(0xffffffffu, n_remote);
+    if (lane == 0) {
+      if (n_rank) atomicAdd(total, (unsigned long long)n_rank);
+      if (n_remote) atomicAdd(remote, (unsigned long long)n_remote);
+    }
+  }
+}
+
+template <int KMAX, int G>
+__global__ void __launch_bounds__(RouteTile<G>::kThreads) route_brim_tile_kernel(
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     const int32_t* __restrict__ slot_of, int R, int prune_m, int n_tiles,
     int32_t* __restrict__ topk_idx,
@@ -29,81 +79,48 @@ __global__ void __launch_bounds__(kRouteTileThreads, 2) route_brim_tile_kernel(
     unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
     unsigned* err) {
   pdl_enter();
-  __shared__ int s_ids[32][KMAX];
-  __shared__ float s_gates[32][KMAX];
-  __shared__ uint32_t s_mask[kMaxCols];
-  const int warp = threadIdx.x >> 5;
+  constexpr int kTiles = RouteTile<G>::kTiles;
+  __shared__ uint32_t s_mask[kTiles][kMaxCols];
+  const int w = threadIdx.x >> 5;
   const unsigned lane = lane_id();
-  const int tile = blockIdx.x;
-  const int L = E / R, ncol = R + E;
-
-  // 1. warp w routes tokens w, w + 16 of the tile (both rows' logits loaded first)
-  {
-    constexpr int kWarps = kRouteTileThreads / 32;
-    float v[kRouteTokensPerWarp][kRouteMaxPerLane];
-#pragma unroll
-    for (int u = 0; u < kRouteTokensPerWarp; ++u) {
-      const int t = tile * kBrimTileTokens + warp + u * kWarps;
-      if (t < T) load_token_logits(logits + (size_t)t * E, E, v[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kRouteTokensPerWarp; ++u) {
-      const int i = warp + u * kWarps;
-      const int t = tile * kBrimTileTokens + i;
-      int id = -1;
-      float gate = 0.f;
-      if (t < T) route_token_warp_v(v[u], E, k, renorm, &id, &gate);
-      if ((int)lane < KMAX) {
-        s_ids[i][lane] = (t < T && (int)lane < k) ? id : -1;
-        s_gates[i][lane] = (t < T && (int)lane < k) ? gate : 0.f;
-      }
-    }
-  }
-  __syncthreads();
-
-  // 2. warp 0, one lane per token: pruning, top-k out, masks, counter
-  if (warp == 0) {
+  int ids[KMAX];
+  float gates[KMAX];
+  if constexpr (G == 1) {
+    // a lane per token from routing to masks
+    const int tile = blockIdx.x * kTiles + w;
+    if (tile >= n_tiles) return;
     const int t = tile * kBrimTileTokens + (int)lane;
-    int ids[KMAX];
-    float gates[KMAX];
+    route_token_group<KMAX, 1>(logits + (size_t)(t < T ? t : 0) * E, t < T, E, k, renorm, ids,
+                               gates);
+    route_tile_masks<KMAX>(t, tile, T, E, k, R, prune_m, n_tiles, slot_of, ids, gates, s_mask[w],
+                           topk_idx, topk_w, masks, per_rank, total, remote, err);
+  } else {
+    __shared__ int s_ids[kTiles * kBrimTileTokens][KMAX];
+    __shared__ float s_gates[kTiles * kBrimTileTokens][KMAX];
+    const int tok = threadIdx.x / G;  // this group's token within the block
+    const int t0 = blockIdx.x * kTiles * kBrimTileTokens;
+    const int t = t0 + tok;
+    route_token_group<KMAX, G>(logits + (size_t)(t < T ? t : 0) * E, t < T, E, k, renorm, ids,
+                               gates);
+    if ((threadIdx.x & (G - 1)) == 0) {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      ids[j] = s_ids[lane][j];
-      gates[j] = s_gates[lane][j];
+      for (int j = 0; j < KMAX; ++j) {
+        s_ids[tok][j] = ids[j];
+        s_gates[tok][j] = gates[j];
+      }
     }
-    if (prune_m > 0 && t < T) prune_token<KMAX>(ids, gates, slot_of, k, E, L, prune_m);
-    if (t < T)
+    __syncthreads();
+    const int tile = blockIdx.x * kTiles + w;
+    if (w < kTiles && tile < n_tiles) {
+      const int lt = w * kBrimTileTokens + (int)lane;
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k) {
-          topk_idx[(size_t)t * k + j] = ids[j];
-          topk_w[(size_t)t * k + j] = gates[j];
-        }
-    TokenRoute<KMAX> tr;
-    const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
-    tile_masks<KMAX>(s_mask, ncol, R, active, k, tr);
-    for (int c = lane; c < ncol; c += 32) masks[(size_t)c * n_tiles + tile] = s_mask[c];
-    if (per_rank) {
-      // tokens per rank: popcount of the rank columns; remote: ranks other than
-      // the token's source rank floor(t * R / T)
-      for (int r = lane; r < R; r += 32) {
-        const int n = __popc(s_mask[r]);
-        if (n) atomicAdd(&per_rank[r], n);
+      for (int j = 0; j < KMAX; ++j) {
+        ids[j] = s_ids[lt][j];
+        gates[j] = s_gates[lt][j];
       }
-      const int src = (int)(((long long)t * R) / (T > 0 ? T : 1));
-      unsigned n_rank = 0, n_remote = 0;
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (active && j < k && tr.first[j]) {
-          ++n_rank;
-          n_remote += tr.rank[j] != src;
-        }
-      n_rank = __reduce_add_sync(0xffffffffu, n_rank);
-      n_remote = __reduce_add_sync(0xffffffffu, n_remote);
-      if (lane == 0) {
-        if (n_rank) atomicAdd(total, (unsigned long long)n_rank);
-        if (n_remote) atomicAdd(remote, (unsigned long long)n_remote);
-      }
+      route_tile_masks<KMAX>(tile * kBrimTileTokens + (int)lane, tile, T, E, k, R, prune_m,
+                             n_tiles, slot_of, ids, gates, s_mask[w], topk_idx, topk_w, masks,
+                             per_rank, total, remote, err);
     }
   }
 }
