@@ -976,7 +976,8 @@ def run_ep(args, cfg):
     import datetime
     import torch.distributed as dist
     from expert_warp_top_b200 import _binding as B
-    from expert_warp_top_b200.ep import DistExchange, EPRank, LoopbackExchange, ep_forward
+    from expert_warp_top_b200.ep import (DistExchange, EPRank, LoopbackExchange, PeerExchange,
+                                         ep_forward)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -987,11 +988,13 @@ def run_ep(args, cfg):
     if cfg.E % R or cfg.T % R:
         raise SystemExit(f"--ep needs R = {R} to divide E = {cfg.E} and T = {cfg.T}")
     if world > 1:
+        if args.exchange == "peer":
+            raise SystemExit("--exchange peer holds all ranks in one process (N = 1)")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         ex = DistExchange()
         mine = [rank]
     else:
-        ex = LoopbackExchange(R)
+        ex = PeerExchange(R) if args.exchange == "peer" else LoopbackExchange(R)
         mine = list(range(R))
     L, Tr = cfg.E // R, cfg.T // R
     inp = inputs.make_inputs(cfg, device=dev)  # the same seeded batch and weights on every rank
@@ -1055,7 +1058,9 @@ def run_ep(args, cfg):
             "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": dict(config_obj(cfg, args), parallelism=(
                 f"expert parallel over {world} GPUs (NCCL)" if world > 1 else
-                f"{R} expert-parallel ranks on one GPU, loopback exchange")),
+                f"{R} expert-parallel ranks on one GPU, " + (
+                    "rows written straight into the receiving ranks' buffers (peer movers)"
+                    if args.exchange == "peer" else "loopback copies for the all-to-all"))),
             "placement": placement_info,
             "ep": {"ranks": R, "c_t": c_t, "rows_between_ranks": wire,
                    "payload_bytes_each_way": wire * cfg.d * e,
@@ -1183,6 +1188,9 @@ def main():
     ap.add_argument("--ep", action="store_true",
                     help="time the real expert-parallel layer: R = N ranks over NCCL under "
                          "torchrun, or the workload's R ranks on one GPU (loopback)")
+    ap.add_argument("--exchange", choices=["collective", "peer"], default="collective",
+                    help="--ep with one process: loopback copies standing for the all-to-all, "
+                         "or the peer movers that write into the receiving ranks' buffers")
     ap.add_argument("--train", action="store_true",
                     help="time the training step (forward + backward) instead of the forward")
     ap.add_argument("--prune", type=int, default=0,

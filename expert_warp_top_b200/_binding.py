@@ -40,6 +40,7 @@ EXPORTS = (
     "moe_layer_backward", "moe_interlayer_histogram", "moe_rank_affinity", "moe_predict_home",
     "moe_count_local", "moe_token_shuffle_workspace_size", "moe_token_shuffle",
     "moe_layer_forward_host_async", "moe_ep_pack_routing", "moe_ep_return_rows", "moe_ep_combine",
+    "moe_ep_send_peer", "moe_ep_return_peer",
 )
 
 
@@ -263,6 +264,57 @@ def moe_ep_combine(y_ret, T, k, R, brim0, shared_out, y, stream=None):
         _ptr(y_ret, _ACT, "y_ret"), int(T), d, dtype_code(y_ret.dtype), int(k), int(R),
         _ptr(brim0, I32, "brim0"), _ptr(shared_out, y_ret.dtype, "shared_out"),
         _ptr(y, y_ret.dtype, "y"), _stream(stream)))
+
+
+MOE_EP_MAX_PEERS = 64
+
+
+class EpPeers(ctypes.Structure):
+    """moe_ep_peers: the buffers of the ranks a mover writes into, by device address."""
+    _fields_ = [("rows", ctypes.c_void_p * MOE_EP_MAX_PEERS),
+                ("idx", ctypes.c_void_p * MOE_EP_MAX_PEERS),
+                ("w", ctypes.c_void_p * MOE_EP_MAX_PEERS),
+                ("row0", ctypes.c_int64 * MOE_EP_MAX_PEERS),
+                ("seg", ctypes.c_int32 * (MOE_EP_MAX_PEERS + 1))]
+
+
+def ep_peers(rows, row0, idx=None, w=None, seg=None) -> EpPeers:
+    """The table for R ranks: rows[q], idx[q], w[q] device addresses (int), row0[q]
+    and seg[0..R] ints (see moe_ep_peers in the header)."""
+    R = len(rows)
+    if R > MOE_EP_MAX_PEERS or len(row0) != R:
+        raise ValueError("one row buffer and one row0 per rank, at most MOE_EP_MAX_PEERS")
+    p = EpPeers()
+    for q in range(R):
+        p.rows[q] = int(rows[q])
+        p.row0[q] = int(row0[q])
+        if idx is not None:
+            p.idx[q] = int(idx[q])
+            p.w[q] = int(w[q])
+    if seg is not None:
+        for q in range(R + 1):
+            p.seg[q] = int(seg[q])
+    return p
+
+
+def moe_ep_send_peer(x, topk_idx, topk_w, slot_of, R, L, brim0, brim1, sfd_token, sfd_off, c_t,
+                     peers: EpPeers, stream=None):
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _check("moe_ep_send_peer", load().moe_ep_send_peer(
+        _ptr(x, _ACT, "x"), T, d, dtype_code(x.dtype), int(k), int(R), int(L),
+        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"), _ptr(slot_of, I32, "slot_of"),
+        _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"), _ptr(sfd_token, I32, "sfd_token"),
+        _ptr(sfd_off, I32, "sfd_off"), _ptr(c_t, I32, "c_t"), ctypes.byref(peers),
+        _stream(stream)))
+
+
+def moe_ep_return_peer(o_epd, T, k, R, L, brim0, brim1, peers: EpPeers, stream=None):
+    d = o_epd.shape[1]
+    _check("moe_ep_return_peer", load().moe_ep_return_peer(
+        _ptr(o_epd, _ACT, "o_epd"), int(T), d, dtype_code(o_epd.dtype), int(k), int(R), int(L),
+        _ptr(brim0, I32, "brim0"), _ptr(brim1, I32, "brim1"), ctypes.byref(peers),
+        _stream(stream)))
 
 
 def moe_count_dispatched_rows(topk_idx, slot_of, E, R, per_rank, total, remote, stream=None):

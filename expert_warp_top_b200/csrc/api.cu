@@ -894,6 +894,111 @@ int moe_ep_combine(const void* y_ret, int T, int d, int dtype, int k, int R,
 }
 
 // ---------------------------------------------------------------------------
+// The exchange over peer memory.  The host struct is copied, as it is, into
+// the kernels' parameter of the same layout.
+static_assert(sizeof(moe_ep_peers) == sizeof(moe::EpPeers) &&
+                  offsetof(moe_ep_peers, row0) == offsetof(moe::EpPeers, row0) &&
+                  offsetof(moe_ep_peers, seg) == offsetof(moe::EpPeers, seg) &&
+                  MOE_EP_MAX_PEERS == moe::kMaxEpPeers,
+              "moe_ep_peers and the device table must match");
+
+static int check_peers(const moe_ep_peers* peers, int R, size_t row_bytes, bool lists) {
+  MOE_REQUIRE(peers, MOE_ERR_INVALID_ARG, "null peer table");
+  MOE_REQUIRE(R <= MOE_EP_MAX_PEERS, MOE_ERR_UNSUPPORTED, "R = %d peers, at most %d", R,
+              MOE_EP_MAX_PEERS);
+  for (int q = 0; q < R; ++q) {
+    MOE_REQUIRE(peers->rows[q] && aligned16(peers->rows[q]) && peers->row0[q] >= -(1LL << 40),
+                MOE_ERR_INVALID_ARG, "peer %d: row buffer missing or not 16-byte aligned", q);
+    MOE_REQUIRE(!lists || (peers->idx[q] && peers->w[q]), MOE_ERR_INVALID_ARG,
+                "peer %d: routing-list buffers missing", q);
+  }
+  (void)row_bytes;
+  return MOE_OK;
+}
+
+int moe_ep_send_peer(const void* x, int T, int d, int dtype, int k, int R, int L,
+                     const int32_t* topk_idx, const float* topk_w, const int32_t* slot_of,
+                     const int32_t* brim0, const int32_t* brim1, const int32_t* sfd_token,
+                     const int32_t* sfd_off, const int32_t* c_t, const moe_ep_peers* peers,
+                     moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= moe::kMaxK && R >= 1 && L >= 1 && R * L <= moe::kMaxE,
+              MOE_ERR_UNSUPPORTED, "bad shape (T=%d k=%d R=%d L=%d)", T, k, R, L);
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(x && topk_idx && topk_w && slot_of && brim0 && brim1 && sfd_token && sfd_off && c_t,
+              MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(x), MOE_ERR_INVALID_ARG, "row buffers must be 16-byte aligned");
+  const int row_bytes = d * esize(dtype);
+  if ((rc = check_peers(peers, R, (size_t)row_bytes, true))) return rc;
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  moe::EpPeers pe;
+  std::memcpy(&pe, peers, sizeof pe);
+  const size_t cap = (size_t)T * (k < R ? k : R);
+  constexpr int CH = 4;  // 512-byte chunks in flight per warp
+  const int P = mover_parts(di, T, (row_bytes + CH * 512 - 1) / (CH * 512));
+  const long long warps = (long long)T * P;
+  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
+  MOE_CUDA(launch_k(moe::dispatch_peer_kernel<CH>, blocks, moe::kMoverWarps * 32, 0, stream,
+                    static_cast<const uint8_t*>(x), T, row_bytes, P, R, L, cap, T * k, brim0,
+                    brim1, static_cast<uint8_t*>(nullptr), di->err_flag, pe));
+  MOE_LAUNCHED("dispatch_peer_kernel");
+  long long pblocks = ((long long)cap + 255) / 256;
+  if (pblocks > 8LL * di->num_sms) pblocks = 8LL * di->num_sms;
+  MOE_CUDA(launch_k(moe::ep_pack_routing_peer_kernel, (int)pblocks, 256, 0, stream, topk_idx,
+                    topk_w, T, k, slot_of, R * L, R, L, sfd_token, sfd_off, c_t,
+                    (long long)cap, di->err_flag, pe));
+  MOE_LAUNCHED("ep_pack_routing_peer_kernel");
+  return MOE_OK;
+}
+
+int moe_ep_return_peer(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                       const int32_t* brim0, const int32_t* brim1, const moe_ep_peers* peers,
+                       moe_stream_t stream) {
+  int rc = check_dtype(dtype);
+  if (rc) return rc;
+  MOE_REQUIRE(T >= 0 && k >= 1 && k <= moe::kMaxK && R >= 1 && L >= 1 && R * L <= moe::kMaxE,
+              MOE_ERR_UNSUPPORTED, "bad shape (T=%d k=%d R=%d L=%d)", T, k, R, L);
+  MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 64");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(o_epd && brim0 && brim1, MOE_ERR_INVALID_ARG, "null pointer");
+  MOE_REQUIRE(aligned16(o_epd), MOE_ERR_INVALID_ARG, "row buffers must be 16-byte aligned");
+  if ((rc = check_peers(peers, R, (size_t)d * esize(dtype), false))) return rc;
+  for (int q = 0; q < R; ++q)
+    MOE_REQUIRE(peers->seg[q] <= peers->seg[q + 1], MOE_ERR_INVALID_ARG,
+                "peer segments must not run backwards");
+  DeviceInfo* di;
+  if ((rc = device_info(&di))) return rc;
+  moe::EpPeers pe;
+  std::memcpy(&pe, peers, sizeof pe);
+  const size_t cap = (size_t)T * (k < R ? k : R);
+  const int P = mover_parts(di, T, (d * esize(dtype) + 511) / 512);
+  const long long warps = (long long)T * P;
+  const int blocks = (int)((warps + moe::kMoverWarps - 1) / moe::kMoverWarps);
+#define MOE_RET(TA, KM)                                                                        \
+  MOE_CUDA(launch_k(moe::combine_peer_kernel<TA, KM>, blocks, moe::kMoverWarps * 32, 0, stream, \
+                    static_cast<const TA*>(o_epd), T, d, P, R, L, cap, T * k, brim0, brim1,    \
+                    di->err_flag, pe))
+  if (dtype == MOE_BF16) {
+    using B = __nv_bfloat16;
+    if (k <= 2) MOE_RET(B, 2);
+    else if (k <= 4) MOE_RET(B, 4);
+    else if (k <= 8) MOE_RET(B, 8);
+    else MOE_RET(B, 16);
+  } else {
+    if (k <= 2) MOE_RET(float, 2);
+    else if (k <= 4) MOE_RET(float, 4);
+    else if (k <= 8) MOE_RET(float, 8);
+    else MOE_RET(float, 16);
+  }
+#undef MOE_RET
+  MOE_LAUNCHED("combine_peer_kernel");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
 int moe_prepare_weights(const void* wg, const void* wu, const void* wd, int E, int d, int f,
                         int dtype, const int32_t* slot_of, void* w_gu, void* w_dn,
                         moe_stream_t stream) {

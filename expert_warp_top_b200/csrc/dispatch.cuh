@@ -23,14 +23,43 @@ namespace moe {
 constexpr int kMoverWarps = 8;     // warps per block
 constexpr int kMaxDst = 16;        // >= k (and >= min(k, R))
 
+// Destination buffers of the other ranks, for the movers that write their rows
+// straight into the ranks that receive them (real expert parallelism over
+// peer memory).  For rank q: rows[q] its row buffer, idx[q] / w[q] its
+// routing-list buffers (k entries per row), and this rank's row i lands at
+// row row0[q] + i there.  seg[0..R] splits this rank's own rows by owner when
+// the owner is found from the row (the return rows: row i belongs to source q
+// when seg[q] <= i < seg[q + 1]).  Passed by value as a kernel parameter.
+constexpr int kMaxEpPeers = 64;
+struct EpPeers {
+  uint8_t* rows[kMaxEpPeers];
+  int32_t* idx[kMaxEpPeers];
+  float* w[kMaxEpPeers];
+  long long row0[kMaxEpPeers];
+  int seg[kMaxEpPeers + 1];
+};
+
+// The owner q of row i: the largest q < R with seg[q] <= i.
+__device__ __forceinline__ int ep_peer_owner(const EpPeers& peers, int R, long long i) {
+  int lo = 0, hi = R;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (peers.seg[mid] <= i) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
 // Destinations of one token, per warp, in shared memory:
-//   sfd[i]   SFD rows of the ranks the token is sent to (ascending rank)
+//   sfd[i]   SFD rows of the ranks the token is sent to (ascending rank), and
+//   sfd_r[i] the rank of each
 //   p[j]     EPD rows of its experts, ascending (rank, local expert), and
 //   p_sfd[j] the SFD row each of them hangs off
 struct WarpDst {
   int n_sfd;
   int n_p;
   int sfd[kMaxDst];
+  int sfd_r[kMaxDst];
   int p[kMaxDst];
   int p_sfd[kMaxDst];
 };
@@ -57,7 +86,10 @@ __device__ __forceinline__ void collect_dst(const int32_t* __restrict__ brim0,
     }
     const unsigned hit = __ballot_sync(0xffffffffu, s >= 0);
     const int pos = n + __popc(hit & lt);
-    if (s >= 0 && pos < kMaxDst) w.sfd[pos] = s;
+    if (s >= 0 && pos < kMaxDst) {
+      w.sfd[pos] = s;
+      w.sfd_r[pos] = r;
+    }
     n += __popc(hit);
   }
   if (n > kMaxDst) bad = true;
@@ -96,11 +128,14 @@ __device__ __forceinline__ void collect_dst(const int32_t* __restrict__ brim0,
 // x_sfd[s] = x[t] and x_epd[p] = x[t] for every destination of token t.
 // One warp per token (P > 1: per 1/P of its row, for small batches); the row
 // is read CH x 512 bytes at a time, all CH loads in flight before the stores.
-template <int CH>
-__global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
+// PEER: the SFD row s of rank r goes to peers.rows[r] row peers.row0[r] + s
+// instead (the receiving rank's buffer), and x_sfd is unused.
+template <int CH, bool PEER>
+__device__ __forceinline__ void dispatch_body(
     const uint8_t* __restrict__ x, int T, int row_bytes, int P, int R, int L, size_t cap, int tk,
     const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
-    uint8_t* __restrict__ x_sfd, uint8_t* __restrict__ x_epd, unsigned* err) {
+    uint8_t* __restrict__ x_sfd, uint8_t* __restrict__ x_epd, unsigned* err,
+    const EpPeers* peers) {
   pdl_enter();
   __shared__ WarpDst sdst[kMoverWarps];
   const int wib = threadIdx.x >> 5;
@@ -114,7 +149,7 @@ __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
   const int span = (row_bytes + P - 1) / P;
   const int lo = part * span, hi = min(row_bytes, lo + span);
   const uint8_t* src = x + (size_t)t * row_bytes;
-  const int n_sfd = x_sfd ? w.n_sfd : 0, n_p = x_epd ? w.n_p : 0;
+  const int n_sfd = (x_sfd || PEER) ? w.n_sfd : 0, n_p = x_epd ? w.n_p : 0;
   for (int off0 = lo; off0 < hi; off0 += CH * 512) {
     uint4 v[CH];
 #pragma unroll
@@ -123,7 +158,13 @@ __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
       if (off < hi) v[u] = ld_nc_v4(src + off);
     }
     for (int i = 0; i < n_sfd; ++i) {
-      uint8_t* dst = x_sfd + (size_t)w.sfd[i] * row_bytes;
+      uint8_t* dst;
+      if constexpr (PEER) {
+        const int r = w.sfd_r[i];
+        dst = peers->rows[r] + (size_t)(peers->row0[r] + w.sfd[i]) * row_bytes;
+      } else {
+        dst = x_sfd + (size_t)w.sfd[i] * row_bytes;
+      }
 #pragma unroll
       for (int u = 0; u < CH; ++u) {
         const int off = off0 + u * 512 + (int)lane * 16;
@@ -139,6 +180,23 @@ __global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
       }
     }
   }
+}
+
+template <int CH>
+__global__ void __launch_bounds__(kMoverWarps * 32) dispatch_kernel(
+    const uint8_t* __restrict__ x, int T, int row_bytes, int P, int R, int L, size_t cap, int tk,
+    const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
+    uint8_t* __restrict__ x_sfd, uint8_t* __restrict__ x_epd, unsigned* err) {
+  dispatch_body<CH, false>(x, T, row_bytes, P, R, L, cap, tk, brim0, brim1, x_sfd, x_epd, err,
+                           nullptr);
+}
+template <int CH>
+__global__ void __launch_bounds__(kMoverWarps * 32) dispatch_peer_kernel(
+    const uint8_t* __restrict__ x, int T, int row_bytes, int P, int R, int L, size_t cap, int tk,
+    const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1, uint8_t* __restrict__ x_epd,
+    unsigned* err, const __grid_constant__ EpPeers peers) {
+  dispatch_body<CH, true>(x, T, row_bytes, P, R, L, cap, tk, brim0, brim1, nullptr, x_epd, err,
+                          &peers);
 }
 
 // The same dispatch through the copy engine (TMA bulk copies, no multicast):
@@ -244,12 +302,14 @@ __global__ void __launch_bounds__(kBulkWarps * 32) dispatch_bulk_kernel(
 // per rank (see collect_dst).  One warp per token (or 1/P of its row); the k expert rows of the
 // next 512-byte slice are loaded while the current slice is summed, so up to
 // 2k loads are in flight per warp.  KMAX >= k bounds the register arrays.
-template <typename TA, int KMAX>
-__global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
+// PEER: the return row of SFD row s goes to its owner q (peers.seg) at row
+// peers.row0[q] + s of peers.rows[q] (the source rank's buffer); y_sfd unused.
+template <typename TA, int KMAX, bool PEER>
+__device__ __forceinline__ void combine_body(
     const TA* __restrict__ o_epd, int T, int d, int P, int R, int L, size_t cap, int tk,
     const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
     const TA* __restrict__ shared_out, TA* __restrict__ y_sfd, TA* __restrict__ y,
-    unsigned* err) {
+    unsigned* err, const EpPeers* peers) {
   pdl_enter();
   constexpr int VN = Vec16<TA>::n;  // elements per 16 bytes
   constexpr int SL = 32 * VN;       // elements per 512-byte slice
@@ -267,10 +327,20 @@ __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
   const int s_lo = part * per, s_hi = min(n_slices, s_lo + per);
   const int n_p = min(w.n_p, KMAX);
   int prow[KMAX], psfd[KMAX];
+  TA* ydst[KMAX];  // where the return row of psfd[j] goes (null: nowhere)
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     prow[j] = j < n_p ? w.p[j] : 0;
     psfd[j] = j < n_p ? w.p_sfd[j] : -1;
+    ydst[j] = nullptr;
+    if (j < n_p) {
+      if constexpr (PEER) {
+        const int q = ep_peer_owner(*peers, R, psfd[j]);
+        ydst[j] = reinterpret_cast<TA*>(peers->rows[q]) + (size_t)(peers->row0[q] + psfd[j]) * d;
+      } else if (y_sfd) {
+        ydst[j] = y_sfd + (size_t)psfd[j] * d;
+      }
+    }
   }
   uint4 cur[KMAX], nxt[KMAX];
   auto load_slice = [&](int sl, uint4 (&v)[KMAX]) {
@@ -297,7 +367,7 @@ __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
           // the last expert of this rank: emit the rank's return row
           if (j + 1 == n_p || psfd[j + 1 < KMAX ? j + 1 : j] != psfd[j]) {
             const uint4 packed = Vec16<TA>::from_f32(acc);
-            if (y_sfd) st_v4(y_sfd + (size_t)psfd[j] * d + c, packed);
+            if (ydst[j]) st_v4(ydst[j] + c, packed);
             float rounded[VN];
             Vec16<TA>::to_f32(packed, rounded);
 #pragma unroll
@@ -321,6 +391,25 @@ __global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) cur[j] = nxt[j];
   }
+}
+
+template <typename TA, int KMAX>
+__global__ void __launch_bounds__(kMoverWarps * 32) combine_kernel(
+    const TA* __restrict__ o_epd, int T, int d, int P, int R, int L, size_t cap, int tk,
+    const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1,
+    const TA* __restrict__ shared_out, TA* __restrict__ y_sfd, TA* __restrict__ y,
+    unsigned* err) {
+  combine_body<TA, KMAX, false>(o_epd, T, d, P, R, L, cap, tk, brim0, brim1, shared_out, y_sfd,
+                                y, err, nullptr);
+}
+// Return rows only, each written into its source rank's buffer.
+template <typename TA, int KMAX>
+__global__ void __launch_bounds__(kMoverWarps * 32) combine_peer_kernel(
+    const TA* __restrict__ o_epd, int T, int d, int P, int R, int L, size_t cap, int tk,
+    const int32_t* __restrict__ brim0, const int32_t* __restrict__ brim1, unsigned* err,
+    const __grid_constant__ EpPeers peers) {
+  combine_body<TA, KMAX, true>(o_epd, T, d, P, R, L, cap, tk, brim0, brim1, nullptr, nullptr,
+                               nullptr, err, &peers);
 }
 
 // The combine through the copy engine.  A unit is (token, piece of its row);

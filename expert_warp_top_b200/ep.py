@@ -39,7 +39,12 @@ The exchanges go through an exchange object: DistExchange uses a
 torch.distributed process group (NCCL between GPUs, gloo on the host);
 LoopbackExchange moves the segments between R ranks held by one process (all
 on one GPU), so the whole data plane of R ranks can run and be checked on a
-single GPU.  ep_forward() drives the six steps over the ranks a process
+single GPU.  PeerExchange takes no collective for the rows: steps 1 and 3
+become one mover that writes each SFD row and its routing list straight into
+the receiving rank's buffer (moe_ep_send_peer), and steps 4 and 5 one mover
+that writes each pre-reduced return row straight into its source's buffer
+(moe_ep_return_peer); only the row counts (step 2) are exchanged on the host.
+It holds the R ranks in one process and addresses their buffers directly.  ep_forward() drives the six steps over the ranks a process
 holds: one with DistExchange, all R with LoopbackExchange.  The rank objects
 are EPRank (the CUDA kernels) or anything with the same steps and buffers.
 """
@@ -103,6 +108,41 @@ class LoopbackExchange:
                 at += n
 
 
+class PeerExchange(LoopbackExchange):
+    """The exchange over peer memory for R ranks held by one process: the
+    movers write into the other ranks' buffers through a table of their
+    device addresses (moe_ep_peers).  The ranks' kernels run on one stream
+    in rank order, which orders every send before every read of it."""
+
+    peer = True
+
+    def barrier(self):
+        pass
+
+    @staticmethod
+    def send_peers(ranks, counts, offs, src):
+        """The table for source `src`: its rows for rank q start at row
+        sum(counts[s][q] for s < src) of q's receive buffers, and its SFD
+        segment for q starts at offs[src][q]."""
+        R = len(ranks)
+        row0 = [sum(counts[s][q] for s in range(src)) - offs[src][q] for q in range(R)]
+        return B.ep_peers([r.x_recv.data_ptr() for r in ranks], row0,
+                          idx=[r.idx_recv.data_ptr() for r in ranks],
+                          w=[r.w_recv.data_ptr() for r in ranks])
+
+    @staticmethod
+    def return_peers(ranks, counts, offs, dst):
+        """The table for destination `dst`: its received rows from source q
+        are rows seg[q] .. seg[q+1]-1 (source-major), and q wants row i of
+        them at its SFD row offs[q][dst] + (i - seg[q])."""
+        R = len(ranks)
+        seg = [0]
+        for q in range(R):
+            seg.append(seg[-1] + counts[q][dst])
+        row0 = [offs[q][dst] - seg[q] for q in range(R)]
+        return B.ep_peers([r.y_ret.data_ptr() for r in ranks], row0, seg=seg)
+
+
 def pair_counts(offs, R):
     """rows[s][q]: rows rank s sends to rank q, from every rank's sfd_off."""
     return [[offs[s][q + 1] - offs[s][q] for q in range(R)] for s in range(R)]
@@ -118,6 +158,8 @@ def ep_forward(ranks, exchange, logits, xs, marks=None):
     kept in `ep_forward.counts`."""
     R = exchange.R
     mark = marks or (lambda name: None)
+    if getattr(exchange, "peer", False):
+        return _ep_forward_peer(ranks, exchange, logits, xs, mark)
     for r, lg, x in zip(ranks, logits, xs):
         r.send_phase(lg, x)
     mark("sent")
@@ -136,6 +178,37 @@ def ep_forward(ranks, exchange, logits, xs, marks=None):
         r.recv_phase(sum(rs))
     mark("computed")
     exchange.rows([r.y_recv for r in ranks], recv_splits, [r.y_ret for r in ranks], send_splits)
+    mark("returned")
+    for r in ranks:
+        r.combine_phase()
+    return [r.y for r in ranks]
+
+
+def _ep_forward_peer(ranks, exchange, logits, xs, mark):
+    """ep_forward over peer memory: the routing and BRIMs of every source,
+    the row counts, then each source's send straight into the receivers'
+    buffers, each destination's experts and its return rows straight into
+    the sources' buffers, and the combine."""
+    R = exchange.R
+    for r, lg, x in zip(ranks, logits, xs):
+        r.route_phase(lg, x)
+    offs = exchange.gather_offsets([r.sfd_off for r in ranks])
+    counts = pair_counts(offs, R)
+    ep_forward.counts = counts
+    for q, r in enumerate(ranks):
+        r.reserve_received(sum(counts[s][q] for s in range(R)))
+    exchange.barrier()  # every receive buffer is free
+    for q, (r, x) in enumerate(zip(ranks, xs)):
+        r.send_peer(x, exchange.send_peers(ranks, counts, offs, q))
+    mark("sent")
+    exchange.barrier()  # every row has landed
+    mark("exchanged")
+    for q, r in enumerate(ranks):
+        r.compute_phase(sum(counts[s][q] for s in range(R)))
+    mark("computed")
+    for q, r in enumerate(ranks):
+        r.return_peer(exchange.return_peers(ranks, counts, offs, q))
+    exchange.barrier()  # every return row has landed
     mark("returned")
     for r in ranks:
         r.combine_phase()
@@ -237,7 +310,9 @@ class EPRank:
                 dtype=torch.uint8, device=dev)
 
     # -- source side -------------------------------------------------------
-    def send_phase(self, logits, x, stream=None):
+    def route_phase(self, logits, x, stream=None):
+        """Routing and the BRIM build over this rank's tokens, and its shared
+        experts."""
         T, k, R = self.T, self.k, self.R
         if T == 0:
             B.moe_brim_build(self.topk_idx[:0], self.topk_w[:0], self.slot_of, self.E, R,
@@ -247,13 +322,30 @@ class EPRank:
         B.moe_route_brim(logits, k, self.renorm, self.slot_of, R, self.topk_idx, self.topk_w,
                          self.brim0, self.sfd_token, self.sfd_off, self.brim1, self.epd_off,
                          self.epd_sfd, self.epd_gate, self.c_t, self.ws, stream=stream)
-        B.moe_dispatch_gather(x, k, R, self.L, self.brim0, self.brim1, self.x_sfd, None, stream)
-        B.moe_ep_pack_routing(self.topk_idx, self.topk_w, self.slot_of, self.E, R,
-                              self.sfd_token, self.sfd_off, self.c_t, self.idx_send, self.w_send,
-                              stream)
         if self.S > 0:
             B.moe_expert_ffn(x, self.shared_off, self.sw_gu, self.sw_dn, self.S * self.fs, None,
                              B.MOE_FFN_SWIGLU, self.shared_out, self.shared_ws, stream)
+
+    def send_phase(self, logits, x, stream=None):
+        """route_phase, then the SFD rows and their routing lists in this
+        rank's send buffers (for a collective)."""
+        self.route_phase(logits, x, stream)
+        if self.T == 0:
+            return
+        B.moe_dispatch_gather(x, self.k, self.R, self.L, self.brim0, self.brim1, self.x_sfd, None,
+                              stream)
+        B.moe_ep_pack_routing(self.topk_idx, self.topk_w, self.slot_of, self.E, self.R,
+                              self.sfd_token, self.sfd_off, self.c_t, self.idx_send, self.w_send,
+                              stream)
+
+    def send_peer(self, x, peers, stream=None):
+        """The SFD rows and their routing lists written straight into the
+        receiving ranks' buffers (moe_ep_send_peer)."""
+        if self.T == 0:
+            return
+        B.moe_ep_send_peer(x, self.topk_idx, self.topk_w, self.slot_of, self.R, self.L,
+                           self.brim0, self.brim1, self.sfd_token, self.sfd_off, self.c_t, peers,
+                           stream)
 
     # -- destination side ----------------------------------------------------
     def reserve_received(self, n):
@@ -273,6 +365,28 @@ class EPRank:
                     epd_gate=self._l_epd_gate[:max(n * k, 1)], c_t=self._l_c_t)
 
     def recv_phase(self, n, stream=None):
+        """compute_phase, then one pre-reduced return row per received row in
+        this rank's return buffer (for a collective)."""
+        self.compute_phase(n, stream)
+        if n == 0:
+            return
+        s = self.local_state(n)
+        B.moe_ep_return_rows(self.o_epd, n, self.k, self.R, self.L, s["brim0"], s["brim1"],
+                             self.y_recv, stream)
+
+    def return_peer(self, peers, stream=None):
+        """The pre-reduced return rows written straight into their sources'
+        buffers (moe_ep_return_peer)."""
+        n = self.n_recv
+        if n == 0:
+            return
+        s = self.local_state(n)
+        B.moe_ep_return_peer(self.o_epd, n, self.k, self.R, self.L, s["brim0"], s["brim1"], peers,
+                             stream)
+
+    def compute_phase(self, n, stream=None):
+        """The local BRIM build over the n received rows, their EPD rows and
+        the grouped GEMMs of this rank's experts."""
         self.n_recv = n
         s = self.local_state(n)
         B.moe_brim_build(self.idx_recv[:n], self.w_recv[:n], self.slot_of, self.E, self.R,
@@ -286,8 +400,6 @@ class EPRank:
         B.moe_expert_ffn(self.x_epd, s["epd_off"][lo:lo + self.L + 1], self.w_gu, self.w_dn,
                          self.f, s["epd_gate"], B.MOE_FFN_SWIGLU, self.o_epd, self.ffn_ws, stream,
                          m_cap=n * self.k)
-        B.moe_ep_return_rows(self.o_epd, n, self.k, self.R, self.L, s["brim0"], s["brim1"],
-                             self.y_recv, stream)
 
     # -- source side, after the return exchange ------------------------------
     def combine_phase(self, stream=None):

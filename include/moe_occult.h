@@ -359,6 +359,62 @@ int moe_ep_combine(const void* y_ret, int T, int d, int dtype, int k, int R,
                    const int32_t* brim0, const void* shared_out, void* y, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The same exchange without a collective: the movers write every row straight
+ * into the buffer of the rank that receives it (peer memory: on a multi-GPU
+ * node, the other processes' buffers mapped into this one, reached over
+ * NVLink; within one process, plain device buffers).  The caller owns the
+ * ordering between ranks: before a send every destination's receive buffers
+ * must be free, and a rank may read what it received only once every sender's
+ * kernel has completed (a stream synchronisation on each rank and a host
+ * barrier between them, or one stream for ranks in one process).
+ *
+ * moe_ep_peers -- one entry per rank q < R (MOE_EP_MAX_PEERS at most):
+ *   rows[q]  the rank's row buffer (dtype rows of d elements)
+ *   idx[q]   its routing-list buffer (k int32 per row), or NULL
+ *   w[q]     its gate buffer (k float32 per row), or NULL
+ *   row0[q]  this rank's row i for q lands at row row0[q] + i there
+ *   seg[0..R] (moe_ep_return_peer) the owners of this rank's own rows: row i
+ *            belongs to rank q when seg[q] <= i < seg[q+1]
+ * Passed by value to the kernels (the struct is read on the host only).
+ * ------------------------------------------------------------------------- */
+#define MOE_EP_MAX_PEERS 64
+typedef struct moe_ep_peers {
+  void* rows[MOE_EP_MAX_PEERS];
+  int32_t* idx[MOE_EP_MAX_PEERS];
+  float* w[MOE_EP_MAX_PEERS];
+  int64_t row0[MOE_EP_MAX_PEERS];
+  int32_t seg[MOE_EP_MAX_PEERS + 1];
+} moe_ep_peers;
+
+/* moe_ep_send_peer -- the source's send: moe_dispatch_gather (SFD rows) and
+ * moe_ep_pack_routing fused with the transfer.  Every SFD row s of this rank's
+ * build, for destination q (its segment of sfd_off), is written to row
+ * peers->row0[q] + s of peers->rows[q], and its restricted routing list to the
+ * same row of peers->idx[q] and peers->w[q].  With row0[q] = (the first row of
+ * this source's segment in q's receive buffer) - sfd_off[q], each destination
+ * gets exactly the rows the all-to-all would deliver.  x [T, d]; topk_idx,
+ * topk_w [T, k]; slot_of [E]; brim0 [R, T], brim1 [L, cap], sfd_token, sfd_off,
+ * c_t of this rank's build (device).  Bad indices raise the device error flag.
+ * ------------------------------------------------------------------------- */
+int moe_ep_send_peer(const void* x, int T, int d, int dtype, int k, int R, int L,
+                     const int32_t* topk_idx, const float* topk_w, const int32_t* slot_of,
+                     const int32_t* brim0, const int32_t* brim1, const int32_t* sfd_token,
+                     const int32_t* sfd_off, const int32_t* c_t, const moe_ep_peers* peers,
+                     moe_stream_t stream);
+
+/* moe_ep_return_peer -- the destination's pre-reduce (moe_ep_return_rows)
+ * fused with the return transfer: the return row of received row s, whose
+ * source q is found by peers->seg, is written to row peers->row0[q] + s of
+ * peers->rows[q].  With seg = the first received row of each source and
+ * row0[q] = (q's sfd_off[this rank]) - seg[q], every source gets its rows at
+ * its own SFD positions, ready for moe_ep_combine.  Other arguments as
+ * moe_ep_return_rows (T = the received rows; brim0, brim1 of the local build).
+ * ------------------------------------------------------------------------- */
+int moe_ep_return_peer(const void* o_epd, int T, int d, int dtype, int k, int R, int L,
+                       const int32_t* brim0, const int32_t* brim1, const moe_ep_peers* peers,
+                       moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * moe_count_dispatched_rows -- rows a once-per-rank dispatcher sends under a
  * placement ("Expert Coupling in MoE Pretraining", Abstract), without
  * building BRIMs:

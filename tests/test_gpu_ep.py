@@ -13,7 +13,9 @@ returned rows (moe_ep_combine).  Checked:
     restricted to that rank's experts;
   - every token's output matches the oracle within the per-row tolerance,
     and the one-GPU layer's output;
-  - NCCL with one rank (DistExchange over a real process group).
+  - NCCL with one rank (DistExchange over a real process group);
+  - the exchange over peer memory (PeerExchange: the movers write straight
+    into the receiving ranks' buffers), bit for bit against the loopback.
 """
 import os
 import socket
@@ -25,7 +27,8 @@ import torch
 import oracle
 import expert_warp_top_b200 as moe
 from expert_warp_top_b200 import inputs
-from expert_warp_top_b200.ep import DistExchange, EPRank, LoopbackExchange, ep_forward
+from expert_warp_top_b200.ep import (DistExchange, EPRank, LoopbackExchange, PeerExchange,
+                                     ep_forward)
 from expert_warp_top_b200.layer import MoELayer
 from helpers import OUT_RTOL, expert_at_slot, rowwise_rel_err, to_oracle
 
@@ -50,7 +53,7 @@ def _ranks(cfg, Ts, slot_of, inp):
     return ranks
 
 
-def _check(cfg, Ts, seed=0, starve=False, placement="random"):
+def _check(cfg, Ts, seed=0, starve=False, placement="random", exchange=LoopbackExchange):
     assert sum(Ts) == cfg.T
     R, L = cfg.R, cfg.E // cfg.R
     inp = inputs.make_inputs(cfg, seed=seed)
@@ -74,7 +77,7 @@ def _check(cfg, Ts, seed=0, starve=False, placement="random"):
     # the R ranks, exchanging through loopback copies
     ranks = _ranks(cfg, Ts, slot_of, inp)
     bounds = np.cumsum([0] + list(Ts))
-    ys = ep_forward(ranks, LoopbackExchange(R),
+    ys = ep_forward(ranks, exchange(R),
                     [logits_d[bounds[r]:bounds[r + 1]].contiguous() for r in range(R)],
                     [x_d[bounds[r]:bounds[r + 1]].contiguous() for r in range(R)])
     torch.cuda.synchronize()
@@ -174,3 +177,39 @@ def test_bench_ep_mode_line():
     assert ep["payload_bytes_each_way"] == ep["rows_between_ranks"] * cfg.d * 2
     assert abs(sum(ep["phase_ms"].values()) - line["ms_per_step"]) <= 0.05 * line["ms_per_step"]
     assert line["value"] > 0 and line["unit"] == "tokens/s"
+
+
+@pytest.mark.parametrize("case", ["tiny", "uneven_starved", "shared", "olmoe"])
+def test_ep_peer_exchange(case):
+    """The same checks with the rows moved by moe_ep_send_peer / moe_ep_return_peer."""
+    if case == "tiny":
+        cfg = inputs.CONFIGS["tiny"]
+        _check(cfg, [cfg.T // cfg.R] * cfg.R, exchange=PeerExchange)
+    elif case == "uneven_starved":
+        cfg = inputs.LayerConfig("ep_uneven", T=700, d=128, f=128, E=16, k=4, R=4, seed=3)
+        _check(cfg, [300, 0, 250, 150], seed=3, starve=True, exchange=PeerExchange)
+    elif case == "shared":
+        cfg = inputs.LayerConfig("ep_shared", T=512, d=256, f=128, E=8, k=2, R=4, S=1, fs=128,
+                                 seed=4)
+        _check(cfg, [128] * 4, seed=4, exchange=PeerExchange)
+    else:
+        cfg = inputs.CONFIGS["olmoe"]
+        _check(cfg, [512] * 8, placement="contiguous", exchange=PeerExchange)
+
+
+def test_ep_peer_exchange_equals_loopback_bit_for_bit():
+    """Every received row, routing list and gate, and every output, equal to
+    the loopback exchange's (random placement, uneven batches)."""
+    cfg = inputs.LayerConfig("ep_bits", T=1536, d=256, f=256, E=32, k=6, R=8, seed=9)
+    Ts = [300, 100, 0, 256, 180, 300, 200, 200]
+    ranks_l, _ = _check(cfg, Ts, seed=9)
+    ranks_p, _ = _check(cfg, Ts, seed=9, exchange=PeerExchange)
+    for a, b in zip(ranks_l, ranks_p):
+        n = a.n_recv
+        assert b.n_recv == n
+        assert torch.equal(a.x_recv[:n], b.x_recv[:n])
+        assert torch.equal(a.idx_recv[:n], b.idx_recv[:n])
+        assert torch.equal(a.w_recv[:n], b.w_recv[:n])
+        c_t = int(a.c_t.item())
+        assert torch.equal(a.y_ret[:c_t], b.y_ret[:c_t])
+        assert torch.equal(a.y[:a.T], b.y[:b.T])
