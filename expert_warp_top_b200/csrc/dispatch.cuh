@@ -327,18 +327,21 @@ __device__ __forceinline__ void combine_body(
   const int s_lo = part * per, s_hi = min(n_slices, s_lo + per);
   const int n_p = min(w.n_p, KMAX);
   int prow[KMAX], psfd[KMAX];
-  TA* ydst[KMAX];  // where the return row of psfd[j] goes (null: nowhere)
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     prow[j] = j < n_p ? w.p[j] : 0;
     psfd[j] = j < n_p ? w.p_sfd[j] : -1;
-    ydst[j] = nullptr;
-    if (j < n_p) {
-      if constexpr (PEER) {
+  }
+  // PEER: where the return row of psfd[j] goes (an array the plain kernel
+  // does not carry: its registers would halve that kernel's occupancy)
+  TA* ydst[PEER ? KMAX : 1];
+  if constexpr (PEER) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ydst[j] = nullptr;
+      if (j < n_p) {
         const int q = ep_peer_owner(*peers, R, psfd[j]);
         ydst[j] = reinterpret_cast<TA*>(peers->rows[q]) + (size_t)(peers->row0[q] + psfd[j]) * d;
-      } else if (y_sfd) {
-        ydst[j] = y_sfd + (size_t)psfd[j] * d;
       }
     }
   }
@@ -367,7 +370,11 @@ __device__ __forceinline__ void combine_body(
           // the last expert of this rank: emit the rank's return row
           if (j + 1 == n_p || psfd[j + 1 < KMAX ? j + 1 : j] != psfd[j]) {
             const uint4 packed = Vec16<TA>::from_f32(acc);
-            if (ydst[j]) st_v4(ydst[j] + c, packed);
+            if constexpr (PEER) {
+              st_v4(ydst[j] + c, packed);
+            } else {
+              if (y_sfd) st_v4(y_sfd + (size_t)psfd[j] * d + c, packed);
+            }
             float rounded[VN];
             Vec16<TA>::to_f32(packed, rounded);
 #pragma unroll
