@@ -470,9 +470,9 @@ int launch_wgrad_pair(DeviceInfo* di, const void* a, const void* b, int rows, in
                       cudaStream_t st) {
   using Cfg = moe::WgradPairCfg<BN>;
   CUtensorMap ta, tb, to;
-  int rc = encode_strips(&ta, a, (uint64_t)M, (uint64_t)rows, 64, 2);
+  int rc = encode_strips(&ta, a, (uint64_t)M, (uint64_t)rows, Cfg::kBK, 2);
   if (rc) return rc;
-  if ((rc = encode_strips(&tb, b, (uint64_t)N, (uint64_t)rows, 64, BN / 128))) return rc;
+  if ((rc = encode_strips(&tb, b, (uint64_t)N, (uint64_t)rows, Cfg::kBK, BN / 128))) return rc;
   constexpr bool kF32 = std::is_same<TOut, float>::value;
   if ((rc = encode_2d(&to, out, kF32 ? MOE_F32 : MOE_BF16, (uint64_t)N, (uint64_t)G * M,
                       kF32 ? 32 : 64, 32)))

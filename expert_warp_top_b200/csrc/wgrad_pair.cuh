@@ -45,11 +45,15 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, const uint4
 }
 }  // namespace tc
 
+#ifndef MOE_WGRAD_PAIR_BK
+#define MOE_WGRAD_PAIR_BK 64
+#endif
 template <int BN>
 struct WgradPairCfg {
-  static constexpr int kBK = 64;                    // contracted rows per stage
-  static constexpr int kABytes = 128 * 128;         // this CTA's 128 columns of A x 64 rows
-  static constexpr int kBBytes = (BN / 2) * 128;    // this CTA's BN/2 columns of B x 64 rows
+  static constexpr int kBK = MOE_WGRAD_PAIR_BK;     // contracted rows per stage
+  static constexpr int kStripBytes = kBK * 128;     // one 64-column strip of kBK rows
+  static constexpr int kABytes = 2 * kStripBytes;   // this CTA's 128 columns of A
+  static constexpr int kBBytes = (BN / 128) * kStripBytes;  // this CTA's BN/2 columns of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
   static constexpr int kTmemCols = 2 * BN;
@@ -71,7 +75,7 @@ __global__ void __launch_bounds__(kWgradThreads, 1)
   static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
   using Cfg = WgradPairCfg<BN>;
   constexpr int S = Cfg::kStages;
-  constexpr int kChunks = Cfg::kStageBytes / 8192;  // 64-column boxes per stage
+  constexpr int kChunks = Cfg::kStageBytes / Cfg::kStripBytes;  // 64-column strips per stage
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -234,8 +238,8 @@ __global__ void __launch_bounds__(kWgradThreads, 1)
           }
           tc::fence_after_sync();
           const uint32_t sa_u = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
-          const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, 8192);
-          const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, 8192);
+          const uint64_t adesc = tc::desc_sw128_mnmajor(sa_u, Cfg::kStripBytes);
+          const uint64_t bdesc = tc::desc_sw128_mnmajor(sa_u + Cfg::kABytes, Cfg::kStripBytes);
           // unrolled with a guard per MMA, as in the single-CTA kernel
           const int n_kk = (valid + 15) / 16;
 #pragma unroll
@@ -293,7 +297,8 @@ __global__ void __launch_bounds__(kWgradThreads, 1)
             const uint32_t peer = peer_tiles + static_cast<uint32_t>(stage * Cfg::kStageBytes);
             for (int c = 0; c < kChunks; ++c)
               for (int q = (int)lane; q < n16; q += 32) {
-                const uint32_t off = static_cast<uint32_t>(c * 8192 + valid * 128 + q * 16);
+                const uint32_t off =
+                    static_cast<uint32_t>(c * Cfg::kStripBytes + valid * 128 + q * 16);
                 st_v4(tiles + (size_t)stage * Cfg::kStageBytes + off, make_uint4(0u, 0u, 0u, 0u));
                 tc::st_cluster_v4(peer + off, make_uint4(0u, 0u, 0u, 0u));
               }
