@@ -26,14 +26,20 @@ namespace moe {
 
 constexpr int kPairBM = 256;  // rows per pair tile, 128 per CTA
 
-template <int BN, bool TF32, int EPI>
+// KCH: 128-byte K chunks per stage.  With 2, one 3-D load (the operand seen as
+// 64-element strips {64, rows, K/64}) brings two consecutive K-major chunks of
+// a tile, laid out one after the other as two 128-byte-swizzled tiles: half
+// the TMA operations and barrier round trips per K of one chunk per stage.
+template <int BN, bool TF32, int EPI, int KCH = 1>
 struct PairCfg {
   static constexpr int kElemBytes = TF32 ? 4 : 2;
-  static constexpr int kBK = 128 / kElemBytes;
+  static constexpr int kBK = KCH * 128 / kElemBytes;
   static constexpr int kMmaK = 32 / kElemBytes;
   static constexpr int kMmaPerStage = kBK / kMmaK;
-  static constexpr int kABytes = 128 * 128;          // this CTA's 128 rows of A
-  static constexpr int kBBytes = (BN / 2) * 128;     // this CTA's half of B
+  static constexpr int kAChunk = 128 * 128;          // this CTA's 128 rows x 128 bytes
+  static constexpr int kBChunk = (BN / 2) * 128;     // its half of B x 128 bytes
+  static constexpr int kABytes = KCH * kAChunk;      // this CTA's 128 rows of A
+  static constexpr int kBBytes = KCH * kBChunk;      // this CTA's half of B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBoxesPerWarp = epi_boxes_per_warp<EPI>();
   static constexpr int kStages = ring_stages(kStageBytes, kBoxesPerWarp);
@@ -50,7 +56,7 @@ struct PairCfg {
 
 // B_MN: B stored MN-major (B[g*K + k][n], n contiguous), seen by tmap_b as
 // 64-column strips; each CTA loads its BN/2 columns in one 3-D load.
-template <int BN, int EPI, bool TF32, bool B_MN = false>
+template <int BN, int EPI, bool TF32, bool B_MN = false, int KCH = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     ffn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b,
@@ -60,7 +66,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(BN <= 256 || (!B_MN && EPI != kEpiSwiGLUSave && EPI != kEpiSwiGLUBwd),
                 "512-wide pair tiles: K-major weights, the inference epilogues");
   static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
-  using Cfg = PairCfg<BN, TF32, EPI>;
+  static_assert(KCH == 1 || (KCH == 2 && !TF32 && !B_MN && BN <= 256),
+                "two K chunks per stage: bf16, K-major B, BN <= 256");
+  using Cfg = PairCfg<BN, TF32, EPI, KCH>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
 
@@ -187,6 +195,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t fb_pair = tc::mapa_shared(fb, 0);  // the barrier in CTA 0
             uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
             if (rank == 0) tc::mbar_arrive_expect_tx(fb, 2 * Cfg::kStageBytes);
+            if (KCH == 2) {
+              // strip maps {element in chunk, row, chunk}: chunks 2kb, 2kb + 1
+              tc::tma_load_3d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, 0, row0 + (int)rank * 128,
+                                   2 * kb, pol_a);
+              tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0,
+                                   g * args.N + n0 + (int)rank * (BN / 2), 2 * kb, pol_b);
+            } else {
             tc::tma_load_2d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, kb * Cfg::kBK,
                                  row0 + (int)rank * 128, pol_a);
             if (B_MN) {
@@ -205,6 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
               tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
                                    kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);
+            }
             }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -247,8 +263,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                       : tc::desc_sw128_kmajor(sa + Cfg::kABytes);
 #pragma unroll
           for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(kk * 2);
-            const uint64_t boff = B_MN ? static_cast<uint64_t>(kk * 128) : off;
+            // +32 bytes per MMA along K inside a chunk's 128-byte rows (+2 in the
+            // address field); the next chunk starts a whole chunk tile later
+            constexpr int kPerChunk = 128 / 32;
+            const int ch = kk / kPerChunk, ki = kk % kPerChunk;
+            const uint64_t off = static_cast<uint64_t>(ch * (Cfg::kAChunk >> 4) + ki * 2);
+            const uint64_t boff = B_MN ? static_cast<uint64_t>(kk * 128)
+                                       : static_cast<uint64_t>(ch * (Cfg::kBChunk >> 4) + ki * 2);
 #pragma unroll
             for (int h = 0; h < Cfg::kNSub; ++h) {
               // the h-th 256-column half: 16 KB further in shared memory, 256 TMEM columns on

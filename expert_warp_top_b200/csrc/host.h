@@ -82,6 +82,7 @@ constexpr int kDebugForceSwap = 64;   // inference GEMMs on the swapped-operand 
 constexpr int kDebugNoSwap = 128;     // never on the swapped-operand kernel
 constexpr int kDebugWideTiles = 256;  // inference GEMMs on 256 x 512 pair tiles where N allows
 constexpr int kDebugNoWideTiles = 512;
+constexpr int kDebugKch1 = 65536;  // pair GEMMs with one K chunk per stage only
 
 // 2-D row-major [rows, cols] tensor, box [box_rows, box_cols], 128-byte swizzle.
 int encode_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows,
@@ -231,22 +232,29 @@ int launch_gemm_bn(DeviceInfo* di, int bn, const void* a, int a_rows,
 }
 
 // The same GEMM on CTA pairs (cluster of 2, M = 256 tiles).  Needs BN/2 >= 64.
-template <int BN, int EPI, bool TF32, bool B_MN>
+// KCH = 2: two 128-byte K chunks per stage through 3-D strip maps (K % 128 == 0).
+template <int BN, int EPI, bool TF32, bool B_MN, int KCH = 1>
 int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K, const void* b,
                      int G, int N, const int32_t* group_off, const float* row_scale, void* out,
                      int ldo, const GemmExtra& ex, cudaStream_t st) {
-  using Cfg = moe::PairCfg<BN, TF32, EPI>;
+  using Cfg = moe::PairCfg<BN, TF32, EPI, KCH>;
   const int dtype = TF32 ? MOE_F32 : MOE_BF16;
   CUtensorMap ta, tb;
-  int rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128);
-  if (rc) return rc;
-  // each CTA loads its BN/2 weight rows in one box, or (BN = 512) in two of 128
-  if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN > 256 ? 128 : BN / 2)))
-    return rc;
+  int rc;
+  if (KCH == 2) {
+    // {element in chunk, row, chunk}: boxes of 128 rows (A) or BN/2 rows (B) x 2 chunks
+    if ((rc = encode_strips(&ta, a, (uint64_t)K, (uint64_t)a_rows, 128, 2))) return rc;
+    if ((rc = encode_strips(&tb, b, (uint64_t)K, (uint64_t)G * N, BN / 2, 2))) return rc;
+  } else {
+    if ((rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128))) return rc;
+    // each CTA loads its BN/2 weight rows in one box, or (BN = 512) in two of 128
+    if ((rc = encode_b<B_MN>(&tb, b, dtype, G, N, K, Cfg::kBK, BN > 256 ? 128 : BN / 2)))
+      return rc;
+  }
   CUtensorMap to, tx;
   if ((rc = encode_out(&to, out, dtype, m_cap, ldo))) return rc;
   if ((rc = encode_aux<EPI>(&tx, to, ex, dtype, m_cap))) return rc;
-  auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32, B_MN>;
+  auto kern = moe::ffn_gemm_pair_kernel<BN, EPI, TF32, B_MN, KCH>;
   const void* key = reinterpret_cast<const void*>(kern);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
@@ -373,6 +381,9 @@ int launch_gemm_swap(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
 #ifndef MOE_PAIR_MIN_ROWS
 #define MOE_PAIR_MIN_ROWS 192
 #endif
+#ifndef MOE_PAIR_KCH2
+#define MOE_PAIR_KCH2 1
+#endif
 template <int EPI, bool TF32, bool B_MN = false>
 int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a_row_index,
                      int m_cap, int K, const void* b, int G, int N, const int32_t* group_off,
@@ -409,6 +420,20 @@ int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a
         ((g_debug_flags & kDebugWideTiles) || wide_tall))
       return launch_gemm_pair<512, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
                                                     row_scale, out, ldo, ex, st);
+  }
+  if constexpr (!TF32 && !B_MN) {
+    // two K chunks per stage (3-D strip loads) where K allows
+    if (pair && !hybrid && MOE_PAIR_KCH2 && K % 128 == 0 && !(g_debug_flags & kDebugKch1)) {
+      GemmExtra exp = ex;
+      exp.tile_mode = moe::kTilesAll;
+      return N % 256 == 0
+                 ? launch_gemm_pair<256, EPI, TF32, B_MN, 2>(di, a, a_rows, m_cap, K, b, G, N,
+                                                             group_off, row_scale, out, ldo, exp,
+                                                             st)
+                 : launch_gemm_pair<128, EPI, TF32, B_MN, 2>(di, a, a_rows, m_cap, K, b, G, N,
+                                                             group_off, row_scale, out, ldo, exp,
+                                                             st);
+    }
   }
   if (pair) {
     GemmExtra exp = ex;
