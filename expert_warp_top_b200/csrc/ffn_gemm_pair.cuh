@@ -66,8 +66,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   static_assert(BN <= 256 || (!B_MN && EPI != kEpiSwiGLUSave && EPI != kEpiSwiGLUBwd),
                 "512-wide pair tiles: K-major weights, the inference epilogues");
   static_assert(!(B_MN && TF32), "MN-major B is bf16 only");
-  static_assert(KCH == 1 || (KCH == 2 && !TF32 && !B_MN && BN <= 256),
-                "two K chunks per stage: bf16, K-major B, BN <= 256");
+  static_assert(KCH == 1 || (KCH == 2 && !TF32 && BN <= 256),
+                "two K chunks per stage: bf16, BN <= 256");
   using Cfg = PairCfg<BN, TF32, EPI, KCH>;
   using TOut = typename std::conditional<TF32, float, __nv_bfloat16>::type;
   constexpr int S = Cfg::kStages;
@@ -196,19 +196,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint8_t* sa = tiles + (size_t)stage * Cfg::kStageBytes;
             if (rank == 0) tc::mbar_arrive_expect_tx(fb, 2 * Cfg::kStageBytes);
             if (KCH == 2) {
-              // strip maps {element in chunk, row, chunk}: chunks 2kb, 2kb + 1
+              // strip map {element in chunk, row, chunk}: chunks 2kb, 2kb + 1
               tc::tma_load_3d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, 0, row0 + (int)rank * 128,
                                    2 * kb, pol_a);
-              tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0,
-                                   g * args.N + n0 + (int)rank * (BN / 2), 2 * kb, pol_b);
             } else {
-            tc::tma_load_2d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, kb * Cfg::kBK,
-                                 row0 + (int)rank * 128, pol_a);
+              tc::tma_load_2d_pair(tc::smem_u32(sa), &tmap_a, fb_pair, kb * Cfg::kBK,
+                                   row0 + (int)rank * 128, pol_a);
+            }
             if (B_MN) {
               // strip map {column in strip, row, strip}: this CTA's BN/128 strips
               tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0,
                                    g * args.K + kb * Cfg::kBK, (n0 + (int)rank * (BN / 2)) / 64,
                                    pol_b);
+            } else if (KCH == 2) {
+              tc::tma_load_3d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair, 0,
+                                   g * args.N + n0 + (int)rank * (BN / 2), 2 * kb, pol_b);
             } else if (BN > 256) {
               // two 256-column halves; CTA r loads rows [h*256 + r*128, +128) of the
               // panel, so that MMA h covers panel columns [h*256, h*256 + 256)
@@ -220,7 +222,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
               tc::tma_load_2d_pair(tc::smem_u32(sa + Cfg::kABytes), &tmap_b, fb_pair,
                                    kb * Cfg::kBK, g * args.N + n0 + (int)rank * (BN / 2), pol_b);
-            }
             }
             armed |= 1u << stage;
             armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -259,7 +260,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc::fence_after_sync();
           const uint32_t sa = tc::smem_u32(tiles + (size_t)stage * Cfg::kStageBytes);
           const uint64_t adesc = tc::desc_sw128_kmajor(sa);
-          const uint64_t bdesc = B_MN ? tc::desc_sw128_mnmajor(sa + Cfg::kABytes, 8192)
+          // MN-major B: strips of kBK rows x 128 bytes, one after the other
+          const uint64_t bdesc = B_MN ? tc::desc_sw128_mnmajor(sa + Cfg::kABytes, Cfg::kBK * 128)
                                       : tc::desc_sw128_kmajor(sa + Cfg::kABytes);
 #pragma unroll
           for (int kk = 0; kk < Cfg::kMmaPerStage; ++kk) {

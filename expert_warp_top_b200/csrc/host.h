@@ -161,7 +161,7 @@ inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
 template <bool B_MN>
 int encode_b(CUtensorMap* tb, const void* b, int dtype, int G, int N, int K, int bk,
              uint32_t box_n) {
-  if (B_MN) return encode_strips(tb, b, (uint64_t)N, (uint64_t)G * K, 64, box_n / 64);
+  if (B_MN) return encode_strips(tb, b, (uint64_t)N, (uint64_t)G * K, bk, box_n / 64);
   return encode_2d(tb, b, dtype, (uint64_t)K, (uint64_t)G * N, bk, box_n);
 }
 
@@ -244,7 +244,11 @@ int launch_gemm_pair(DeviceInfo* di, const void* a, int a_rows, int m_cap, int K
   if (KCH == 2) {
     // {element in chunk, row, chunk}: boxes of 128 rows (A) or BN/2 rows (B) x 2 chunks
     if ((rc = encode_strips(&ta, a, (uint64_t)K, (uint64_t)a_rows, 128, 2))) return rc;
-    if ((rc = encode_strips(&tb, b, (uint64_t)K, (uint64_t)G * N, BN / 2, 2))) return rc;
+    if (B_MN) {
+      if ((rc = encode_b<true>(&tb, b, dtype, G, N, K, Cfg::kBK, BN / 2))) return rc;
+    } else if ((rc = encode_strips(&tb, b, (uint64_t)K, (uint64_t)G * N, BN / 2, 2))) {
+      return rc;
+    }
   } else {
     if ((rc = encode_2d(&ta, a, dtype, (uint64_t)K, (uint64_t)a_rows, Cfg::kBK, 128))) return rc;
     // each CTA loads its BN/2 weight rows in one box, or (BN = 512) in two of 128
@@ -421,8 +425,10 @@ int launch_gemm_auto(DeviceInfo* di, const void* a, int a_rows, const int32_t* a
       return launch_gemm_pair<512, EPI, TF32, B_MN>(di, a, a_rows, m_cap, K, b, G, N, group_off,
                                                     row_scale, out, ldo, ex, st);
   }
-  if constexpr (!TF32 && !B_MN) {
-    // two K chunks per stage (3-D strip loads) where K allows
+  // two K chunks per stage (3-D strip loads) where K allows and the ring keeps
+  // three stages: the epilogues with three staging boxes per warp would be left
+  // with two, which measured slower than five single-chunk stages
+  if constexpr (!TF32 && moe::PairCfg<256, TF32, EPI, 2>::kStages >= 3) {
     if (pair && !hybrid && MOE_PAIR_KCH2 && K % 128 == 0 && !(g_debug_flags & kDebugKch1)) {
       GemmExtra exp = ex;
       exp.tile_mode = moe::kTilesAll;
