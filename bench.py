@@ -57,8 +57,8 @@ TRAIN_METRIC = ("MoE-layer training tokens/s (forward + backward: route, BRIM di
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the two routed-expert
 # GEMM launches of one layer step, from one ncu capture of that workload's GEMMs, valid
 # only while the GEMM sources hash to `src`; otherwise reported as null.
-GEMM_TRAFFIC = {"corr_prefill": {"bytes": (5176.7 + 798.1 + 1963.5 + 1581.0) * 1e6,
-                                 "src": "c18b44d414d15e56"}}
+GEMM_TRAFFIC = {"corr_prefill": {"bytes": (8113.1 + 798.7 + 1942.2 + 1579.3) * 1e6,
+                                 "src": "16ac570cf420e614"}}
 
 
 def gemm_src_hash() -> str:

@@ -72,11 +72,11 @@ constexpr int kDebugForceSingle = 2;  // GEMMs on single CTAs
 constexpr int kDebugForcePair = 4;    // GEMMs on CTA pairs only where the shape allows
 constexpr int kDebugForceHybrid = 8;  // pair tiles plus single-CTA small tails
 constexpr int kDebugBulkMovers = 16;  // dispatch and combine through TMA bulk copies
-// Tuning knobs of the expert GEMMs: with kDebugGemmPolicy set, bits 8..9, 10..11
-// and 12..13 of the flags give the L2 policy of the A loads, the weight loads and
+// Tuning knobs of the expert GEMMs: with kDebugGemmPolicy set, bits 20..21, 22..23
+// and 24..25 of the flags give the L2 policy of the A loads, the weight loads and
 // the output stores (0 evict_normal, 1 evict_last, 2 evict_first; output 0 = no
-// hint), bit 14 the N-fastest tile order and bit 15 the L2 prefetch of the next
-// tile's first-use panels.
+// hint), bit 26 the N-fastest tile order and bit 27 the L2 prefetch of the next
+// tile's first-use panels.  (They sit above every switch below.)
 constexpr int kDebugGemmPolicy = 32;
 constexpr int kDebugForceSwap = 64;   // inference GEMMs on the swapped-operand kernel
 constexpr int kDebugNoSwap = 128;     // never on the swapped-operand kernel
@@ -147,11 +147,11 @@ inline moe::GemmArgs gemm_args(const DeviceInfo* di, const int32_t* group_off,
   a.n_part = ex.n_part;
   a.tile_mode = ex.tile_mode;
   if (g_debug_flags & kDebugGemmPolicy) {
-    a.l2_a = (g_debug_flags >> 8) & 3;
-    a.l2_b = (g_debug_flags >> 10) & 3;
-    a.l2_out = (g_debug_flags >> 12) & 3;
-    a.raster = (g_debug_flags >> 14) & 1;
-    a.l2_prefetch = (g_debug_flags >> 15) & 1;
+    a.l2_a = (g_debug_flags >> 20) & 3;
+    a.l2_b = (g_debug_flags >> 22) & 3;
+    a.l2_out = (g_debug_flags >> 24) & 3;
+    a.raster = (g_debug_flags >> 26) & 1;
+    a.l2_prefetch = (g_debug_flags >> 27) & 1;
   }
   return a;
 }

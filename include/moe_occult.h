@@ -79,9 +79,15 @@ const char* moe_last_error(void);
 
 /* Test-only knobs.  flags bit 0: the expert GEMM's producer skips its first
  * TMA load, so a bounded wait is certain to expire (exercises the timeout
- * path without faulting or hanging the GPU).  wait_limit_ms: how long a
- * device-side wait may last before it gives up (default 4000 ms).  Process
- * wide; not for production use. */
+ * path without faulting or hanging the GPU).  The other bits choose among the
+ * library's equivalent kernel variants, for tests and measurements:
+ *   2 single-CTA GEMMs, 4 CTA-pair GEMMs where the shape allows, 8 pair tiles
+ *   with single-CTA tails, 16 the movers through TMA bulk copies, 32 the GEMM
+ *   L2 policies and tile order of bits 20..27, 64 / 128 force / forbid the
+ *   swapped-operand GEMM, 256 / 512 force / forbid 256 x 512 pair tiles,
+ *   65536 pair GEMMs with one K chunk per stage only.
+ * wait_limit_ms: how long a device-side wait may last before it gives up
+ * (default 4000 ms).  Process wide; not for production use. */
 int moe_set_debug(int flags, double wait_limit_ms);
 
 /* Reads and clears the device error flag that the kernels raise, in one
