@@ -45,12 +45,12 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, const uint4
 }
 }  // namespace tc
 
-#ifndef MOE_WGRAD_PAIR_BK
-#define MOE_WGRAD_PAIR_BK 64
-#endif
-template <int BN>
+// BK: contracted rows per stage.  128 halves the TMA operations per row but
+// loads up to 127 rows past a group's end; the host takes it for long groups.
+template <int BN, int BK = 64>
 struct WgradPairCfg {
-  static constexpr int kBK = MOE_WGRAD_PAIR_BK;     // contracted rows per stage
+  static_assert(BK == 64 || BK == 128, "stages of 64 or 128 contracted rows");
+  static constexpr int kBK = BK;                    // contracted rows per stage
   static constexpr int kStripBytes = kBK * 128;     // one 64-column strip of kBK rows
   static constexpr int kABytes = 2 * kStripBytes;   // this CTA's 128 columns of A
   static constexpr int kBBytes = (BN / 128) * kStripBytes;  // this CTA's BN/2 columns of B
@@ -64,16 +64,16 @@ struct WgradPairCfg {
   static_assert(kSmemBytes <= 232448, "over the per-CTA shared-memory limit");
 };
 
-// tmap_a: A as 64-column strips, box 64 rows x 2 strips; tmap_b: B as strips,
-// box 64 rows x BN/128 strips; tmap_out: the output [G*M, N], box 32 rows x
+// tmap_a: A as 64-column strips, box BK rows x 2 strips; tmap_b: B as strips,
+// box BK rows x BN/128 strips; tmap_out: the output [G*M, N], box 32 rows x
 // 128 bytes.  M % 256 == 0, N % BN == 0.
-template <int BN, typename TOut>
+template <int BN, typename TOut, int BK = 64>
 __global__ void __launch_bounds__(kWgradThreads, 1)
     wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_out, const WgradArgs args) {
   static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
-  using Cfg = WgradPairCfg<BN>;
+  using Cfg = WgradPairCfg<BN, BK>;
   constexpr int S = Cfg::kStages;
   constexpr int kChunks = Cfg::kStageBytes / Cfg::kStripBytes;  // 64-column strips per stage
 

@@ -85,7 +85,8 @@ const char* moe_last_error(void);
  *   with single-CTA tails, 16 the movers through TMA bulk copies, 32 the GEMM
  *   L2 policies and tile order of bits 20..27, 64 / 128 force / forbid the
  *   swapped-operand GEMM, 256 / 512 force / forbid 256 x 512 pair tiles,
- *   65536 pair GEMMs with one K chunk per stage only.
+ *   65536 pair GEMMs with one K chunk per stage only, 131072 weight-gradient
+ *   pairs on 64-row stages only.
  * wait_limit_ms: how long a device-side wait may last before it gives up
  * (default 4000 ms).  Process wide; not for production use. */
 int moe_set_debug(int flags, double wait_limit_ms);

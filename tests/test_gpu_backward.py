@@ -99,12 +99,18 @@ def _ffn_oracle(off, x, wg, wu, wd, scale, dout):
     return y, g
 
 
+SHORT_SIZES = [0, 1, 64, 200, 413]  # an empty group, a one-row group, an exact tile, ragged
+# groups averaging more than 1024 rows (the weight gradient's 128-row stages),
+# with last blocks of 76, 1, 64 and 92 rows and an empty group
+LONG_SIZES = [1100, 0, 2049, 1600, 1500]
+
+
 @pytest.mark.parametrize("variant", [0, FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID],
                          ids=["auto", "single", "pair", "hybrid"])
 @pytest.mark.parametrize("dw_dtype", [torch.float32, torch.bfloat16], ids=["dw_f32", "dw_bf16"])
-def test_expert_ffn_backward_matches_oracle(variant, dw_dtype):
-    # an empty group, a one-row group, an exact tile, and ragged multi-tile groups
-    sizes, d, f = [0, 1, 64, 200, 413], 256, 256
+@pytest.mark.parametrize("sizes", [SHORT_SIZES, LONG_SIZES], ids=["short", "long"])
+def test_expert_ffn_backward_matches_oracle(variant, dw_dtype, sizes):
+    d, f = 256, 256
     off, x, wg, wu, wd, scale, dout = _ffn_problem(sizes, d, f, seed=11)
     G, rows = len(sizes), int(sum(sizes))
     w_gu = torch.empty(G, 2 * f, d, dtype=torch.bfloat16, device=DEV)
