@@ -199,8 +199,10 @@ def test_multi_tile_layers(cfg):
 
 
 # test-only switches of the library: force the single-CTA GEMM, the CTA-pair
-# GEMM alone, or CTA pairs plus single-CTA tiles for groups' short tails
+# GEMM alone, or CTA pairs plus single-CTA tiles for groups' short tails; and
+# the CTA-pair GEMM with one K chunk per stage (2-D loads) where two would run
 FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID = 2, 4, 8
+FORCE_PAIR_ONE_CHUNK = 4 | 65536
 
 
 @pytest.fixture
@@ -210,7 +212,8 @@ def gemm_variant(request):
     moe.moe_set_debug(0, 4000.0)
 
 
-@pytest.mark.parametrize("gemm_variant", [FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID], indirect=True)
+@pytest.mark.parametrize("gemm_variant", [FORCE_SINGLE, FORCE_PAIR, FORCE_HYBRID,
+                                          FORCE_PAIR_ONE_CHUNK], indirect=True)
 @pytest.mark.parametrize("cfg", [
     # 256-row pair tiles over ragged groups, BN = 256 / 256
     inputs.LayerConfig("pair", T=1500, d=256, f=256, E=8, k=2, R=4, seed=21),
