@@ -220,13 +220,15 @@ int launch_brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int 
   MOE_CUDA(launch_k(moe::brim_mask_kernel<KMAX>, blocks, 128, 0, stream, topk_idx, slot_of, T, k, E, R, n_tiles,
                                                           scratch, err));
   MOE_LAUNCHED("brim_mask_kernel");
-  MOE_CUDA(launch_k(moe::brim_colscan_kernel<KMAX>, ncol, 1024, 0, stream, scratch, n_tiles, ncol,
-                    totals, topk_idx, T, k, E, static_cast<uint32_t*>(nullptr), 0, err));
+  // the column scan writes the tiles' bases over the masks
+  MOE_CUDA(launch_k(moe::brim_colscan_kernel, ncol, 1024, 0, stream,
+                    static_cast<const uint32_t*>(scratch), scratch, n_tiles, ncol, totals, T, R,
+                    static_cast<int32_t*>(nullptr)));
   MOE_LAUNCHED("brim_colscan_kernel");
   MOE_CUDA(launch_k(moe::brim_scatter_kernel<KMAX>, n_tiles, 32 * moe::kScatterWarps, 0, stream,
       topk_idx, topk_w, slot_of, T, k, E, R, n_tiles, reinterpret_cast<const int32_t*>(scratch),
       static_cast<const int32_t*>(totals), sfd_off, epd_off, c_t, brim0, sfd_token, brim1,
-      epd_sfd, epd_gate));
+      epd_sfd, epd_gate, moe::BrimExtras{}));
   MOE_LAUNCHED("brim_scatter_kernel");
   return MOE_OK;
 }
@@ -247,20 +249,11 @@ int brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int k, cons
 }
 
 // Scratch entries of a BRIM build: one 32-bit word per column per 32-token
-// tile (the masks, then the tiles' bases), then one total per column.
+// tile (the masks, which the column scan overwrites with the tiles' bases),
+// then one total per column.
 size_t brim_scratch_entries(int T, int E, int R) {
   const size_t n_tiles = ((size_t)T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
   return (n_tiles + 1) * (size_t)(R + E);
-}
-
-// Histogram blocks of the column-scan pass: 512 tokens each.  A block's
-// k^2 shared-memory increments per token are what bound the launch (the
-// column scans are short), so the tokens are spread over several blocks; each
-// block then merges its counts with at most E^2 global atomics.
-int hist_blocks(int T, int* tokens_per_block) {
-  const int per = 512;
-  *tokens_per_block = per;
-  return (T + per - 1) / per;
 }
 
 }  // namespace
@@ -527,9 +520,17 @@ int moe_prune_topk(int32_t* topk_idx, float* topk_w, int T, int k, const int32_t
 }
 
 // ---------------------------------------------------------------------------
+// Scratch of the fused index path: the masks, the tiles' bases (kept apart so
+// that the histogram can read the masks after the column scan), the column
+// totals and the rank columns' own-rank hits.
+size_t route_brim_scratch_entries(int T, int E, int R) {
+  const size_t n_tiles = ((size_t)T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
+  return (2 * n_tiles + 1) * (size_t)(R + E) + (size_t)R;
+}
+
 size_t moe_route_brim_workspace_size(int T, int E, int R) {
   if (T < 0 || E < 1 || R < 1) return 0;
-  return align256(sizeof(int32_t) * brim_scratch_entries(T, E, R)) + 256;
+  return align256(sizeof(int32_t) * route_brim_scratch_entries(T, E, R)) + 256;
 }
 
 int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const int32_t* slot_of,
@@ -547,14 +548,14 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
               MOE_ERR_INVALID_ARG, "per_rank, total and remote are given together or not at all");
   DeviceInfo* di;
   if ((rc = device_info(&di))) return rc;
-  if (per_rank) {
-    MOE_CUDA(cudaMemsetAsync(per_rank, 0, sizeof(int32_t) * R, stream));
-    MOE_CUDA(cudaMemsetAsync(total, 0, sizeof(int64_t), stream));
-    MOE_CUDA(cudaMemsetAsync(remote, 0, sizeof(int64_t), stream));
-  }
   if (hist && !hist_accumulate)
     MOE_CUDA(cudaMemsetAsync(hist, 0, sizeof(uint32_t) * E * E, stream));
   if (T == 0) {
+    if (per_rank) {
+      MOE_CUDA(cudaMemsetAsync(per_rank, 0, sizeof(int32_t) * R, stream));
+      MOE_CUDA(cudaMemsetAsync(total, 0, sizeof(int64_t), stream));
+      MOE_CUDA(cudaMemsetAsync(remote, 0, sizeof(int64_t), stream));
+    }
     MOE_CUDA(cudaMemsetAsync(sfd_off, 0, sizeof(int32_t) * (R + 1), stream));
     MOE_CUDA(cudaMemsetAsync(epd_off, 0, sizeof(int32_t) * (E + 1), stream));
     MOE_CUDA(cudaMemsetAsync(c_t, 0, sizeof(int32_t), stream));
@@ -570,18 +571,28 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   uint32_t* masks = static_cast<uint32_t*>(ws);
   const int n_tiles = (T + moe::kBrimTileTokens - 1) / moe::kBrimTileTokens;
   const int ncol = R + E;
-  int32_t* totals = reinterpret_cast<int32_t*>(masks) + (size_t)ncol * n_tiles;
-  int hist_tokens = 0;
-  const int n_hist = hist ? hist_blocks(T, &hist_tokens) : 0;
-  auto* tot = reinterpret_cast<unsigned long long*>(total);
-  auto* rem = reinterpret_cast<unsigned long long*>(remote);
+  uint32_t* bases = masks + (size_t)ncol * n_tiles;
+  int32_t* totals = reinterpret_cast<int32_t*>(bases + (size_t)ncol * n_tiles);
+  int32_t* own = totals + ncol;
+  moe::BrimExtras extras{};
+  if (per_rank) {
+    extras.per_rank = per_rank;
+    extras.total = reinterpret_cast<unsigned long long*>(total);
+    extras.remote = reinterpret_cast<unsigned long long*>(remote);
+    extras.own = own;
+  }
+  if (hist) {
+    extras.hist = hist;
+    extras.masks = masks;
+    const int ct = moe::hist_chunk_tiles(E);
+    extras.n_hist = (n_tiles + ct - 1) / ct;
+  }
   const int G = moe::route_lanes_per_token(T, di->num_sms);
 #define MOE_ROUTE_TILE(KM, GG)                                                                \
   MOE_CUDA(launch_k(moe::route_brim_tile_kernel<KM, GG>,                                     \
                     dim3((n_tiles + moe::RouteTile<GG>::kTiles - 1) / moe::RouteTile<GG>::kTiles), \
                     dim3(moe::RouteTile<GG>::kThreads), 0, stream, logits, T, E, k, renorm,    \
-                    slot_of, R, prune_m, n_tiles, topk_idx, topk_w, masks, per_rank, tot, rem,  \
-                    di->err_flag))
+                    slot_of, R, prune_m, n_tiles, topk_idx, topk_w, masks, di->err_flag))
 #define MOE_ROUTE_TILE_G(KM)                                                                   \
   do {                                                                                        \
     if (G == 8) MOE_ROUTE_TILE(KM, 8);                                                        \
@@ -591,13 +602,14 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   } while (0)
 #define MOE_ROUTE_BRIM(KM)                                                                    \
   MOE_ROUTE_TILE_G(KM);                                                                       \
-  MOE_CUDA(launch_k(moe::brim_colscan_kernel<KM>, dim3(ncol + n_hist), dim3(1024), 0, stream, \
-                    masks, n_tiles, ncol, totals, static_cast<const int32_t*>(topk_idx), T, k,  \
-                    E, hist, hist_tokens, di->err_flag));                                       \
-  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3(n_tiles), dim3(32 * moe::kScatterWarps), 0, \
-                    stream, topk_idx, topk_w, slot_of, T, k, E, R, n_tiles,                     \
-                    reinterpret_cast<const int32_t*>(masks), static_cast<const int32_t*>(totals), \
-                    sfd_off, epd_off, c_t, brim0, sfd_token, brim1, epd_sfd, epd_gate))
+  MOE_CUDA(launch_k(moe::brim_colscan_kernel, dim3(ncol), dim3(1024), 0, stream,              \
+                    static_cast<const uint32_t*>(masks), bases, n_tiles, ncol, totals, T, R,    \
+                    per_rank ? own : static_cast<int32_t*>(nullptr)));                          \
+  MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3(extras.n_hist + n_tiles),              \
+                    dim3(32 * moe::kScatterWarps), 0, stream, static_cast<const int32_t*>(topk_idx), \
+                    static_cast<const float*>(topk_w), slot_of, T, k, E, R, n_tiles,            \
+                    reinterpret_cast<const int32_t*>(bases), static_cast<const int32_t*>(totals), \
+                    sfd_off, epd_off, c_t, brim0, sfd_token, brim1, epd_sfd, epd_gate, extras))
   if (k <= 2) {
     MOE_ROUTE_BRIM(2);
   } else if (k <= 4) {

@@ -266,36 +266,55 @@ __device__ __forceinline__ void coact_hist_range(const int32_t* __restrict__ top
 }
 
 // ---- pass 2, parallel ------------------------------------------------------
-// Block c < ncol scans column c on its own: the popcounts of its n_tiles
-// masks, exclusive prefix over the tiles, written back in place (the tile's
-// first row WITHIN the column) and the column total into totals[c].  The
-// scatter (pass 3) adds each column's offset among the columns of its kind.
-// Blocks ncol .. ncol + n_hist - 1, when hist is given, add consecutive token
-// ranges of topk_idx to the co-activation histogram meanwhile.
-template <int KMAX>
+// Block c scans column c on its own: the popcounts of its n_tiles masks,
+// exclusive prefix over the tiles, written to bases[c * n_tiles + tile] (the
+// tile's first row WITHIN the column; bases may be the masks themselves) and
+// the column total into totals[c].  The scatter (pass 3) adds each column's
+// offset among the columns of its kind.  With `own`, each rank column r < R
+// also counts its own-rank hits: the tokens t of rank r's own slice of the
+// batch, floor(t * R / T) = r, that are sent to rank r.
+__device__ __forceinline__ uint32_t lanes_in_range(int tile, long long lo, long long hi) {
+  const long long base = (long long)tile * kBrimTileTokens;
+  const long long s = lo > base ? lo - base : 0;
+  const long long e = hi - base < 32 ? hi - base : 32;
+  if (e <= s) return 0u;
+  const uint32_t below_e = e == 32 ? 0xffffffffu : ((1u << e) - 1u);
+  return below_e & ~((1u << s) - 1u);
+}
+
 __global__ void __launch_bounds__(1024) brim_colscan_kernel(
-    uint32_t* __restrict__ masks, int n_tiles, int ncol, int32_t* __restrict__ totals,
-    const int32_t* __restrict__ topk_idx, int T, int k, int E, uint32_t* __restrict__ hist,
-    int hist_tokens, unsigned* err) {
+    const uint32_t* masks, uint32_t* bases, int n_tiles, int ncol, int32_t* __restrict__ totals,
+    int T, int R, int32_t* __restrict__ own) {
   pdl_enter();
-  __shared__ uint32_t sh[kHistSmemE * kHistSmemE];
-  int32_t* warp_sums = reinterpret_cast<int32_t*>(sh);  // the scan needs 32 of them
-  if ((int)blockIdx.x >= ncol) {
-    const int t0 = ((int)blockIdx.x - ncol) * hist_tokens;
-    coact_hist_range<KMAX>(topk_idx, t0, min(T, t0 + hist_tokens), k, E, hist, err, sh);
-    return;
-  }
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t s_own;
   const int c = blockIdx.x;
-  uint32_t* col = masks + (size_t)c * n_tiles;
+  const uint32_t* col = masks + (size_t)c * n_tiles;
+  uint32_t* out = bases + (size_t)c * n_tiles;
   const int per = (n_tiles + blockDim.x - 1) / blockDim.x;  // tiles per thread
   const int b0 = threadIdx.x * per, b1 = min(b0 + per, n_tiles);
-  int sum = 0;
-  for (int b = b0; b < b1; ++b) sum += __popc(col[b]);
+  const bool count_own = own != nullptr && c < R;
+  long long lo = 0, hi = 0;  // rank c's own tokens: [lo, hi)
+  if (count_own) {
+    lo = ((long long)c * T + R - 1) / R;
+    hi = ((long long)(c + 1) * T + R - 1) / R;
+  }
+  int sum = 0, mine = 0;
+  for (int b = b0; b < b1; ++b) {
+    const uint32_t m = col[b];
+    sum += __popc(m);
+    if (count_own) mine += __popc(m & lanes_in_range(b, lo, hi));
+  }
   // block-wide exclusive scan of the per-thread sums
   const int warp = threadIdx.x >> 5, lane = (int)lane_id();
   const int inc = warp_inclusive_scan(sum);
   if (lane == 31) warp_sums[warp] = inc;
+  if (threadIdx.x == 0) s_own = 0;
   __syncthreads();
+  if (count_own) {
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    if (lane == 0 && mine) atomicAdd(&s_own, mine);
+  }
   if (warp == 0) {
     const int nw = blockDim.x >> 5;
     const int v = lane < nw ? warp_sums[lane] : 0;
@@ -304,11 +323,56 @@ __global__ void __launch_bounds__(1024) brim_colscan_kernel(
     if (lane == nw - 1) totals[c] = winc;
   }
   __syncthreads();
+  if (count_own && threadIdx.x == 0) own[c] = s_own;
   int base = warp_sums[warp] + inc - sum;
   for (int b = b0; b < b1; ++b) {
     const int n = __popc(col[b]);
-    col[b] = (uint32_t)base;
+    out[b] = (uint32_t)base;
     base += n;
+  }
+}
+
+// ---- co-activation histogram from the slot masks -----------------------------
+// hist[a][b] += the number of tokens routed to both experts a and b: the sum
+// over the tiles of popcount(mask(a) & mask(b)), mask(e) being the column of
+// e's slot.  The masks hold exactly the tokens with a valid route, without
+// their empty (pruned) slots, so this is the count coact_hist_range makes
+// from the ids.  One block per chunk of hist_chunk_tiles(E) tiles: it stages
+// the chunk's E columns in shared memory, tile-major and by expert id, sums
+// every cell over the chunk and adds the nonzero sums to hist, one atomic
+// per cell per chunk.
+__host__ __device__ constexpr int hist_chunk_tiles(int E) { return E <= 128 ? 16 : 8; }
+constexpr int kHistStageWords = 16 * 128;  // chunk tiles x E, for every E <= kMaxE
+
+__device__ __forceinline__ void coact_hist_chunk_from_masks(
+    const uint32_t* __restrict__ masks, int n_tiles, int R, int E,
+    const int32_t* __restrict__ slot_of, int chunk, uint32_t* __restrict__ hist,
+    uint32_t* stage) {
+  const int ct = hist_chunk_tiles(E);
+  const int tile0 = chunk * ct;
+  for (int i = threadIdx.x; i < E * ct; i += blockDim.x) {
+    const int e = i / ct, t = i % ct;
+    const int q = slot_of ? __ldg(slot_of + e) : e;
+    stage[t * E + e] = tile0 + t < n_tiles ? masks[(size_t)(R + q) * n_tiles + tile0 + t] : 0u;
+  }
+  __syncthreads();
+  // tpr threads per row a: row a's chunk in registers, the b columns read
+  // from shared memory (a warp reads at most tpr distinct words per load)
+  const int nt = blockDim.x;
+  const int tpr = nt >= E ? nt / E : 1;
+  const int rows = nt / tpr;
+  const int sub = threadIdx.x % tpr;
+  for (int a = threadIdx.x / tpr; a < E; a += rows) {
+    uint32_t ra[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) ra[t] = t < ct ? stage[t * E + a] : 0u;
+    for (int b = sub; b < E; b += tpr) {
+      int n = 0;
+#pragma unroll
+      for (int t = 0; t < 16; ++t)
+        if (t < ct) n += __popc(ra[t] & stage[t * E + b]);
+      if (n) atomicAdd(&hist[(size_t)a * E + b], (uint32_t)n);
+    }
   }
 }
 
@@ -323,11 +387,31 @@ __global__ void __launch_bounds__(1024) brim_colscan_kernel(
 //                  all l of each rank the token reaches
 //   epd_sfd[p] = s, epd_gate[p] = the token's gate weight for that expert
 //
-// With `totals` (pass 2), tile_base holds rows within each column; warp 0
+// tile_base holds each tile's first row within each column (pass 2); warp 0
 // adds the column offsets -- the exclusive scans of the column totals over
 // the R rank columns and over the E slot columns -- and tile 0 writes
-// sfd_off, epd_off and C_T.
+// sfd_off, epd_off and C_T.  Every global load a block needs before its
+// stores is issued first, so a block waits on two load round trips: the
+// ids, gates, totals and bases, then slot_of.
+//
+// BrimExtras adds, in the fused index path, the dispatched-row counter and
+// the co-activation histogram to the same launch:
+//   * tile 0 writes per_rank (the rank columns' totals), total (C_T) and
+//     remote (C_T less the own-rank hits that pass 2 counted);
+//   * blocks 0 .. n_hist - 1 come before the tiles and each add one chunk of
+//     tiles to the histogram from the slot masks, which must then still be
+//     intact (pass 2 writing its bases elsewhere).
 constexpr int kScatterWarps = 4;
+
+struct BrimExtras {
+  int32_t* per_rank;             // [R], or null: no counter
+  unsigned long long* total;     // rows sent, C_T
+  unsigned long long* remote;    // rows sent to a rank other than the token's source
+  const int32_t* own;            // [R] own-rank hits (pass 2)
+  uint32_t* hist;                // [E, E], accumulated; or null
+  const uint32_t* masks;         // the slot masks (pass 1), for the histogram rows
+  int n_hist;                    // tile chunks (hist_chunk_tiles) when hist is given, else 0
+};
 
 template <int KMAX>
 __global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
@@ -336,46 +420,72 @@ __global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
     const int32_t* __restrict__ tile_base, const int32_t* __restrict__ totals,
     int32_t* __restrict__ sfd_off, int32_t* __restrict__ epd_off, int32_t* __restrict__ c_t,
     int32_t* __restrict__ brim0, int32_t* __restrict__ sfd_token, int32_t* __restrict__ brim1,
-    int32_t* __restrict__ epd_sfd, float* __restrict__ epd_gate) {
+    int32_t* __restrict__ epd_sfd, float* __restrict__ epd_gate, BrimExtras x) {
   pdl_enter();
-  __shared__ uint32_t sm[kMaxCols];
-  __shared__ int32_t sb[kMaxCols];
-  __shared__ int32_t s_tot[kMaxCols], s_off[kMaxCols];
-  const int tile = blockIdx.x;
+  // the histogram's staging and the tile's arrays share one buffer
+  static_assert(kHistStageWords <= 4 * kMaxCols, "staging fits the scatter's arrays");
+  __shared__ uint32_t s_buf[4 * kMaxCols];
+  if ((int)blockIdx.x < x.n_hist) {
+    coact_hist_chunk_from_masks(x.masks, n_tiles, R, E, slot_of, (int)blockIdx.x, x.hist, s_buf);
+    return;
+  }
+  uint32_t* sm = s_buf;
+  int32_t* sb = reinterpret_cast<int32_t*>(s_buf + kMaxCols);
+  int32_t* s_tot = reinterpret_cast<int32_t*>(s_buf + 2 * kMaxCols);
+  int32_t* s_off = reinterpret_cast<int32_t*>(s_buf + 3 * kMaxCols);
+  const int tile = (int)blockIdx.x - x.n_hist;
   const int warp = threadIdx.x >> 5;
   const int ncol = R + E, L = E / R;
   const size_t cap = (size_t)T * (k < R ? k : R);
   const unsigned lane = lane_id();
   const int t = tile * kBrimTileTokens + (int)lane;
+  int ids[KMAX];
+  float gw[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const bool in = t < T && j < k;
+    ids[j] = in ? __ldg(topk_idx + (size_t)t * k + j) : -1;
+    gw[j] = in && topk_w ? __ldg(topk_w + (size_t)t * k + j) : 1.f;
+  }
+  if (warp == 0) {
+    for (int c = lane; c < ncol; c += 32) {
+      s_tot[c] = totals[c];
+      sb[c] = tile_base[(size_t)c * n_tiles + tile];
+    }
+  }
   TokenRoute<KMAX> tr;
   // the error flag was raised by pass 1 already
-  const bool active = t < T && load_token_route<KMAX>(topk_idx, slot_of, t, k, E, L, tr, nullptr);
+  const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, nullptr);
   float gate[KMAX];
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j)
-    gate[j] = (active && j < k && tr.slot[j] >= 0) ? (topk_w ? __ldg(topk_w + (size_t)t * k + j) : 1.f)
-                                                   : 0.f;
+  for (int j = 0; j < KMAX; ++j) gate[j] = (active && j < k && tr.slot[j] >= 0) ? gw[j] : 0.f;
   if (warp == 0) {
     tile_masks<KMAX>(sm, ncol, R, active, k, tr);
     // the tile's first global row in every column
-    if (totals) {
-      for (int c = lane; c < ncol; c += 32) s_tot[c] = totals[c];
-      __syncwarp();
-      const int ct = warp_exclusive_scan_smem(s_tot, s_off, R);
-      const int tk = warp_exclusive_scan_smem(s_tot + R, s_off + R, E);
-      __syncwarp();
-      for (int c = lane; c < ncol; c += 32) sb[c] = s_off[c] + tile_base[(size_t)c * n_tiles + tile];
-      if (tile == 0) {
-        for (int r = lane; r < R; r += 32) sfd_off[r] = s_off[r];
-        for (int q = lane; q < E; q += 32) epd_off[q] = s_off[R + q];
+    const int ct = warp_exclusive_scan_smem(s_tot, s_off, R);
+    const int tk = warp_exclusive_scan_smem(s_tot + R, s_off + R, E);
+    __syncwarp();
+    for (int c = lane; c < ncol; c += 32) sb[c] += s_off[c];
+    if (tile == 0) {
+      for (int r = lane; r < R; r += 32) sfd_off[r] = s_off[r];
+      for (int q = lane; q < E; q += 32) epd_off[q] = s_off[R + q];
+      if (lane == 0) {
+        sfd_off[R] = ct;
+        epd_off[E] = tk;
+        *c_t = ct;
+      }
+      if (x.per_rank) {
+        int o = 0;
+        for (int r = lane; r < R; r += 32) {
+          x.per_rank[r] = s_tot[r];
+          o += x.own[r];
+        }
+        o = __reduce_add_sync(0xffffffffu, o);
         if (lane == 0) {
-          sfd_off[R] = ct;
-          epd_off[E] = tk;
-          *c_t = ct;
+          *x.total = (unsigned long long)ct;
+          *x.remote = (unsigned long long)(ct - o);
         }
       }
-    } else {
-      for (int c = lane; c < ncol; c += 32) sb[c] = tile_base[(size_t)c * n_tiles + tile];
     }
   }
   __syncthreads();

@@ -1,15 +1,15 @@
-// route_brim.cuh -- routing, the BRIM masks and the dispatched-row counter in
-// one kernel (pass 1 of the BRIM build fused with routing).
+// route_brim.cuh -- routing and the BRIM masks in one kernel (pass 1 of the
+// BRIM build fused with routing).
 //
-// The same computation as moe_route_topk + brim_mask_kernel +
-// moe_count_dispatched_rows.  Tokens are routed by groups of G lanes
-// (route_token_group, the very code of moe_route_topk; G from the batch size,
-// the result does not depend on it).  Then one warp per 32-token tile, one
-// lane per token, prunes (when asked), writes the top-k, builds the tile's
-// column masks and adds the tile's contribution to the counter.  With G = 1
-// a lane keeps its own token throughout; with G > 1 the routes pass through
-// shared memory.  The column scan with the histogram (brim_colscan_kernel)
-// and the scatter (brim_scatter_kernel) follow.
+// The same computation as moe_route_topk + brim_mask_kernel.  Tokens are
+// routed by groups of G lanes (route_token_group, the very code of
+// moe_route_topk; G from the batch size, the result does not depend on it).
+// Then one warp per 32-token tile, one lane per token, prunes (when asked),
+// writes the top-k and builds the tile's column masks.  With G = 1 a lane
+// keeps its own token throughout; with G > 1 the routes pass through shared
+// memory.  The column scan (brim_colscan_kernel) and the scatter
+// (brim_scatter_kernel) follow; the dispatched-row counter and the
+// co-activation histogram come out of those two from the masks.
 #pragma once
 #include "brim.cuh"
 #include "route.cuh"
@@ -28,9 +28,7 @@ __device__ __forceinline__ void route_tile_masks(
     int t, int tile, int T, int E, int k, int R, int prune_m, int n_tiles,
     const int32_t* __restrict__ slot_of, int (&ids)[KMAX], float (&gates)[KMAX],
     uint32_t* s_mask, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-    uint32_t* __restrict__ masks, int32_t* __restrict__ per_rank,
-    unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
-    unsigned* err) {
+    uint32_t* __restrict__ masks, unsigned* err) {
   const unsigned lane = lane_id();
   const int L = E / R, ncol = R + E;
   if (t < T) {
@@ -46,28 +44,6 @@ __device__ __forceinline__ void route_tile_masks(
   const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, err);
   tile_masks<KMAX>(s_mask, ncol, R, active, k, tr);
   for (int c = lane; c < ncol; c += 32) masks[(size_t)c * n_tiles + tile] = s_mask[c];
-  if (per_rank) {
-    // tokens per rank: popcount of the rank columns; remote: ranks other than
-    // the token's source rank floor(t * R / T)
-    for (int r = lane; r < R; r += 32) {
-      const int n = __popc(s_mask[r]);
-      if (n) atomicAdd(&per_rank[r], n);
-    }
-    const int src = (int)(((long long)t * R) / (T > 0 ? T : 1));
-    unsigned n_rank = 0, n_remote = 0;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-      if (active && j < k && tr.first[j]) {
-        ++n_rank;
-        n_remote += tr.rank[j] != src;
-      }
-    n_rank = __reduce_add_sync(0xffffffffu, n_rank);
-    n_remote = __reduce_add_sync(0xffffffffu, n_remote);
-    if (lane == 0) {
-      if (n_rank) atomicAdd(total, (unsigned long long)n_rank);
-      if (n_remote) atomicAdd(remote, (unsigned long long)n_remote);
-    }
-  }
 }
 
 template <int KMAX, int G>
@@ -75,9 +51,7 @@ __global__ void __launch_bounds__(RouteTile<G>::kThreads) route_brim_tile_kernel
     const float* __restrict__ logits, int T, int E, int k, int renorm,
     const int32_t* __restrict__ slot_of, int R, int prune_m, int n_tiles,
     int32_t* __restrict__ topk_idx,
-    float* __restrict__ topk_w, uint32_t* __restrict__ masks, int32_t* __restrict__ per_rank,
-    unsigned long long* __restrict__ total, unsigned long long* __restrict__ remote,
-    unsigned* err) {
+    float* __restrict__ topk_w, uint32_t* __restrict__ masks, unsigned* err) {
   pdl_enter();
   constexpr int kTiles = RouteTile<G>::kTiles;
   __shared__ uint32_t s_mask[kTiles][kMaxCols];
@@ -93,7 +67,7 @@ __global__ void __launch_bounds__(RouteTile<G>::kThreads) route_brim_tile_kernel
     route_token_group<KMAX, 1>(logits + (size_t)(t < T ? t : 0) * E, t < T, E, k, renorm, ids,
                                gates);
     route_tile_masks<KMAX>(t, tile, T, E, k, R, prune_m, n_tiles, slot_of, ids, gates, s_mask[w],
-                           topk_idx, topk_w, masks, per_rank, total, remote, err);
+                           topk_idx, topk_w, masks, err);
   } else {
     __shared__ int s_ids[kTiles * kBrimTileTokens][KMAX];
     __shared__ float s_gates[kTiles * kBrimTileTokens][KMAX];
@@ -120,7 +94,7 @@ __global__ void __launch_bounds__(RouteTile<G>::kThreads) route_brim_tile_kernel
       }
       route_tile_masks<KMAX>(tile * kBrimTileTokens + (int)lane, tile, T, E, k, R, prune_m,
                              n_tiles, slot_of, ids, gates, s_mask[w], topk_idx, topk_w, masks,
-                             per_rank, total, remote, err);
+                             err);
     }
   }
 }

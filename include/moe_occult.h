@@ -196,13 +196,15 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
 
 /* ---------------------------------------------------------------------------
  * moe_route_brim -- moe_route_topk, moe_brim_build, moe_count_dispatched_rows
- * and moe_coact_histogram in three kernel launches instead of six: one block per
- * 32-token tile routes its tokens (warp per token, the code of
- * moe_route_topk), builds the tile's BRIM column masks and adds to the counter;
- * then one block per column scans that column while extra blocks of the same
- * launch build the histogram; a third kernel scatters BRIM_0 / BRIM_1 and
- * their inverses.  Every output is bit for bit the one the separate entry
- * points produce.
+ * and moe_coact_histogram in three kernel launches instead of six, with no
+ * memset: one block per 32-token tile routes its tokens (the code of
+ * moe_route_topk) and builds the tile's BRIM column masks; then one block per
+ * column scans that column, the rank columns also counting the tokens their
+ * own rank receives; a third kernel scatters BRIM_0 / BRIM_1 and their
+ * inverses, writes the counter from the column totals, and has more blocks
+ * that add the histogram from the masks, 256 or 512 tokens each (tokens on
+ * both experts: the popcount of the AND of their columns).  Every output is bit for bit the one
+ * the separate entry points produce.
  *   prune_m > 0 applies moe_prune_topk with m = prune_m between routing and
  *   the BRIMs (0 = no pruning);
  *   other arguments as in those entry points; per_rank / total / remote are given
