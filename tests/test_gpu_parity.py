@@ -151,6 +151,34 @@ def test_fused_index_equals_separate():
     assert torch.equal(ya, yb)
 
 
+@pytest.mark.parametrize("E", [64, 8, 160, 6])
+@pytest.mark.parametrize("renorm", [0, 1])
+def test_routing_does_not_depend_on_batch_size(E, renorm):
+    """The lanes per token (G = 1, 2, 4 or 8) follow the batch size; the routes and gates
+    of a token do not: the same rows routed inside batches of 40000, 30000, 15000 and 300
+    tokens (G = 1, 2, 4, 8 on a 148-SM part) come out bit for bit equal, and match the
+    oracle."""
+    k = min(6, E)
+    g = torch.Generator().manual_seed(11 + E)
+    big = torch.randn(40000, E, generator=g, dtype=torch.float32) * 2.0
+    ref_idx = ref_w = None
+    for T in (40000, 30000, 15000, 300):
+        logits = big[:T].contiguous().to(DEV)
+        idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+        w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+        moe.moe_route_topk(logits, k, renorm, idx, w)
+        torch.cuda.synchronize()
+        if ref_idx is None:
+            ref_idx, ref_w = idx[:300].cpu(), w[:300].cpu()
+        else:
+            assert torch.equal(idx[:300].cpu(), ref_idx), T
+            assert torch.equal(w[:300].cpu(), ref_w), T
+    idx_o, w_o = oracle_route(big[:300], k, renorm)
+    assert np.array_equal(ref_idx.numpy(), idx_o)
+    np.testing.assert_allclose(ref_w.numpy().astype(np.float64), w_o, rtol=softmax_rtol(E),
+                               atol=1e-30)
+
+
 @pytest.mark.parametrize("epd_mode", ["stored", "gather"])
 def test_tiny_layer_permuted_placement(epd_mode):
     cfg = inputs.CONFIGS["tiny"]
