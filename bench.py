@@ -413,8 +413,9 @@ def run_ours(args, cfg):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     # The step is replayed from one CUDA graph, so host launch overhead does not
-    # enter the timing.  Two external event-record nodes inside the graph time
-    # the routed-expert GEMMs on their own within every timed step.
+    # enter the timing.  External event-record nodes inside the graph time the
+    # index path (routing, BRIMs, counter, histogram) and the routed-expert
+    # GEMMs on their own within every timed step.
     def part_a():
         layer.route_brim(logits)  # routing, BRIMs, counter, histogram
         layer.dispatch(x)
@@ -436,11 +437,16 @@ def run_ours(args, cfg):
     status = B.moe_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
+    i0 = torch.cuda.Event(enable_timing=True, external=True)
+    i1 = torch.cuda.Event(enable_timing=True, external=True)
     f0 = torch.cuda.Event(enable_timing=True, external=True)
     f1 = torch.cuda.Event(enable_timing=True, external=True)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=side):
-        part_a()
+        i0.record(side)
+        layer.route_brim(logits)
+        i1.record(side)
+        layer.dispatch(x)
         f0.record(side)
         part_b()
         f1.record(side)
@@ -451,7 +457,7 @@ def run_ours(args, cfg):
 
     s0 = torch.cuda.Event(enable_timing=True)
     s1 = torch.cuda.Event(enable_timing=True)
-    step_ms, ffn_ms = [], []
+    step_ms, ffn_ms, index_ms = [], [], []
     with ClockSampler(local_rank) as clocks:
         # keep the GPU busy until the sampler reports, so its samples see the load
         t_end = time.time() + 5.0
@@ -470,6 +476,7 @@ def run_ours(args, cfg):
             s1.synchronize()
             step_ms.append(s0.elapsed_time(s1))
             ffn_ms.append(f0.elapsed_time(f1))
+            index_ms.append(i0.elapsed_time(i1))
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
@@ -557,6 +564,7 @@ def run_ours(args, cfg):
             "gpu_launches": launches_per_step(cfg) * args.steps,
             "ffn_ms": statistics.mean(ffn_ms),
             "ffn_own_graph_ms": statistics.mean(ffn_own_ms),
+            "index_ms": statistics.mean(index_ms),
         }
         # the GEMMs' time in SM clock cycles at the median sampled clock: the
         # figure to compare across runs and with ncu at different clocks

@@ -341,8 +341,11 @@ __global__ void __launch_bounds__(1024) brim_colscan_kernel(
 // the chunk's E columns in shared memory, tile-major and by expert id, sums
 // every cell over the chunk and adds the nonzero sums to hist, one atomic
 // per cell per chunk.
-__host__ __device__ constexpr int hist_chunk_tiles(int E) { return E <= 128 ? 16 : 8; }
-constexpr int kHistStageWords = 16 * 128;  // chunk tiles x E, for every E <= kMaxE
+constexpr int kHistMaxChunk = 8;
+__host__ __device__ constexpr int hist_chunk_tiles(int E) {
+  return E <= 128 ? kHistMaxChunk : kHistMaxChunk / 2;
+}
+constexpr int kHistStageWords = kHistMaxChunk * 128;  // chunk tiles x E, for every E <= kMaxE
 
 __device__ __forceinline__ void coact_hist_chunk_from_masks(
     const uint32_t* __restrict__ masks, int n_tiles, int R, int E,
@@ -363,13 +366,13 @@ __device__ __forceinline__ void coact_hist_chunk_from_masks(
   const int rows = nt / tpr;
   const int sub = threadIdx.x % tpr;
   for (int a = threadIdx.x / tpr; a < E; a += rows) {
-    uint32_t ra[16];
+    uint32_t ra[kHistMaxChunk];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) ra[t] = t < ct ? stage[t * E + a] : 0u;
+    for (int t = 0; t < kHistMaxChunk; ++t) ra[t] = t < ct ? stage[t * E + a] : 0u;
     for (int b = sub; b < E; b += tpr) {
       int n = 0;
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
+      for (int t = 0; t < kHistMaxChunk; ++t)
         if (t < ct) n += __popc(ra[t] & stage[t * E + b]);
       if (n) atomicAdd(&hist[(size_t)a * E + b], (uint32_t)n);
     }

@@ -202,7 +202,7 @@ int moe_brim_build_noalloc(const int32_t* topk_idx, const float* topk_w, int T, 
  * column scans that column, the rank columns also counting the tokens their
  * own rank receives; a third kernel scatters BRIM_0 / BRIM_1 and their
  * inverses, writes the counter from the column totals, and has more blocks
- * that add the histogram from the masks, 256 or 512 tokens each (tokens on
+ * that add the histogram from the masks, 128 or 256 tokens each (tokens on
  * both experts: the popcount of the AND of their columns).  Every output is bit for bit the one
  * the separate entry points produce.
  *   prune_m > 0 applies moe_prune_topk with m = prune_m between routing and
