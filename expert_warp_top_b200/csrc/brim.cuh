@@ -41,7 +41,8 @@ struct TokenRoute {
   bool first[KMAX];
 };
 
-// Builds a token's route from its k expert ids.  An id of -1 is an empty slot
+// Builds a token's route from its k expert ids (slot_of in global or shared
+// memory; null: the identity placement).  An id of -1 is an empty slot
 // (a pruned assignment): it is sent nowhere and is not an error.  Returns
 // false (and raises the error flag) when an id is otherwise out of range or
 // repeated; such a token is sent nowhere.
@@ -57,7 +58,7 @@ __device__ __forceinline__ bool make_token_route(const int (&ids)[KMAX],
     tr.rank[j] = -1;
     if (j < k && ids[j] != -1) {
       const int e = ids[j];
-      const int q = (e >= 0 && e < E) ? (slot_of ? __ldg(slot_of + e) : e) : -1;  // null: identity
+      const int q = (e >= 0 && e < E) ? (slot_of ? slot_of[e] : e) : -1;  // null: identity
       if (q < 0 || q >= E) ok = false;
       tr.slot[j] = q;
       tr.rank[j] = q >= 0 ? q / L : -1;
@@ -91,7 +92,7 @@ __device__ __forceinline__ void prune_token(int (&ids)[KMAX], float (&gates)[KMA
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     const int e = ids[j];
-    rank[j] = (j < k && e >= 0 && e < E) ? __ldg(slot_of + e) / L : -1;
+    rank[j] = (j < k && e >= 0 && e < E) ? slot_of[e] / L : -1;
   }
   int n_kept_ranks = 0;
 #pragma unroll
@@ -394,8 +395,8 @@ __device__ __forceinline__ void coact_hist_chunk_from_masks(
 // adds the column offsets -- the exclusive scans of the column totals over
 // the R rank columns and over the E slot columns -- and tile 0 writes
 // sfd_off, epd_off and C_T.  Every global load a block needs before its
-// stores is issued first, so a block waits on two load round trips: the
-// ids, gates, totals and bases, then slot_of.
+// stores is issued first, slot_of staged in shared memory among them, so a
+// block waits on one load round trip before it computes.
 //
 // BrimExtras adds, in the fused index path, the dispatched-row counter and
 // the co-activation histogram to the same launch:
@@ -442,6 +443,7 @@ __global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
   const size_t cap = (size_t)T * (k < R ? k : R);
   const unsigned lane = lane_id();
   const int t = tile * kBrimTileTokens + (int)lane;
+  __shared__ int32_t s_slot[kMaxE];
   int ids[KMAX];
   float gw[KMAX];
 #pragma unroll
@@ -451,14 +453,32 @@ __global__ void __launch_bounds__(32 * kScatterWarps) brim_scatter_kernel(
     gw[j] = in && topk_w ? __ldg(topk_w + (size_t)t * k + j) : 1.f;
   }
   if (warp == 0) {
-    for (int c = lane; c < ncol; c += 32) {
+    // the first 128 columns' loads all issue before any of them is stored
+    int32_t tot[4], base[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      tot[i] = c < ncol ? totals[c] : 0;
+      base[i] = c < ncol ? tile_base[(size_t)c * n_tiles + tile] : 0;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      if (c < ncol) {
+        s_tot[c] = tot[i];
+        sb[c] = base[i];
+      }
+    }
+    for (int c = lane + 128; c < ncol; c += 32) {
       s_tot[c] = totals[c];
       sb[c] = tile_base[(size_t)c * n_tiles + tile];
     }
   }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_slot[e] = slot_of ? __ldg(slot_of + e) : e;
+  __syncthreads();  // s_slot
   TokenRoute<KMAX> tr;
   // the error flag was raised by pass 1 already
-  const bool active = t < T && make_token_route<KMAX>(ids, slot_of, k, E, L, tr, nullptr);
+  const bool active = t < T && make_token_route<KMAX>(ids, s_slot, k, E, L, tr, nullptr);
   float gate[KMAX];
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) gate[j] = (active && j < k && tr.slot[j] >= 0) ? gw[j] : 0.f;

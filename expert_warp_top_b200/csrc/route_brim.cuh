@@ -55,6 +55,12 @@ __global__ void __launch_bounds__(RouteTile<G>::kThreads) route_brim_tile_kernel
   pdl_enter();
   constexpr int kTiles = RouteTile<G>::kTiles;
   __shared__ uint32_t s_mask[kTiles][kMaxCols];
+  // With G > 1, slot_of is staged in shared memory while the tokens are
+  // routed (the block's barrier follows the routing); with G = 1 the warps
+  // never meet, so they read it from global memory.
+  __shared__ int32_t s_slot[G > 1 ? kMaxE : 1];
+  if constexpr (G > 1)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_slot[e] = __ldg(slot_of + e);
   const int w = threadIdx.x >> 5;
   const unsigned lane = lane_id();
   int ids[KMAX];
@@ -93,7 +99,7 @@ __global__ void __launch_bounds__(RouteTile<G>::kThreads) route_brim_tile_kernel
         gates[j] = s_gates[lt][j];
       }
       route_tile_masks<KMAX>(tile * kBrimTileTokens + (int)lane, tile, T, E, k, R, prune_m,
-                             n_tiles, slot_of, ids, gates, s_mask[w], topk_idx, topk_w, masks,
+                             n_tiles, s_slot, ids, gates, s_mask[w], topk_idx, topk_w, masks,
                              err);
     }
   }
