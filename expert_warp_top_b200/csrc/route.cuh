@@ -27,26 +27,27 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Offers expert e with logit x to a thread's best-KMAX list: ranks top[]
-// ascending, their logits val[].  top[0] is the entry threshold.  The k best
-// are top[KMAX - 1], top[KMAX - 2], ... (k <= KMAX), so every index is a
-// compile-time constant and the list stays in registers.
+// The float a key came from (-0.0 comes back as +0.0).
+__device__ __forceinline__ float float_from_order_key(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// Offers expert e with logit x to a thread's best-KMAX list of ranks top[],
+// ascending; a rank holds the logit's key, so the list needs no logits beside
+// it.  top[0] is the entry threshold.  The k best are top[KMAX - 1],
+// top[KMAX - 2], ... (k <= KMAX), so every index is a compile-time constant and
+// the list stays in registers.
 template <int KMAX>
-__device__ __forceinline__ void route_offer(uint64_t (&top)[KMAX], float (&val)[KMAX], int e,
-                                            float x) {
+__device__ __forceinline__ void route_offer(uint64_t (&top)[KMAX], int e, float x) {
   const uint64_t c = (static_cast<uint64_t>(float_order_key(x)) << 32) | static_cast<uint32_t>(~e);
   if (c > top[0]) {
     top[0] = c;
-    val[0] = x;
 #pragma unroll
     for (int j = 0; j + 1 < KMAX; ++j) {
       const bool sw = top[j] > top[j + 1];
       const uint64_t lo = sw ? top[j + 1] : top[j], hi = sw ? top[j] : top[j + 1];
-      const float vlo = sw ? val[j + 1] : val[j], vhi = sw ? val[j] : val[j + 1];
       top[j] = lo;
       top[j + 1] = hi;
-      val[j] = vlo;
-      val[j + 1] = vhi;
     }
   }
 }
@@ -71,68 +72,54 @@ __device__ __forceinline__ void route_token_group(const float* __restrict__ row,
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "G must be 1, 2, 4 or 8");
   const int sub = static_cast<int>(lane_id()) & (G - 1);
   uint64_t top[KMAX];  // this lane's best ranks, ascending; 0 = empty
-  float val[KMAX];
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    top[j] = 0ull;
-    val[j] = 0.f;
-  }
+  for (int j = 0; j < KMAX; ++j) top[j] = 0ull;
   const bool vec = (E & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 15) == 0;
   if (valid) {
     if (vec) {
       const float4* r4 = reinterpret_cast<const float4*>(row);
       for (int q = sub; q < (E >> 2); q += G) {
         const float4 x = __ldg(r4 + q);
-        route_offer<KMAX>(top, val, 4 * q, x.x);
-        route_offer<KMAX>(top, val, 4 * q + 1, x.y);
-        route_offer<KMAX>(top, val, 4 * q + 2, x.z);
-        route_offer<KMAX>(top, val, 4 * q + 3, x.w);
+        route_offer<KMAX>(top, 4 * q, x.x);
+        route_offer<KMAX>(top, 4 * q + 1, x.y);
+        route_offer<KMAX>(top, 4 * q + 2, x.z);
+        route_offer<KMAX>(top, 4 * q + 3, x.w);
       }
     } else {
-      for (int e = sub; e < E; e += G) route_offer<KMAX>(top, val, e, __ldg(row + e));
+      for (int e = sub; e < E; e += G) route_offer<KMAX>(top, e, __ldg(row + e));
     }
   }
   uint64_t sel[KMAX];
-  float selv[KMAX];
   if constexpr (G == 1) {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      sel[j] = top[KMAX - 1 - j];
-      selv[j] = val[KMAX - 1 - j];
-    }
+    for (int j = 0; j < KMAX; ++j) sel[j] = top[KMAX - 1 - j];
   } else {
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       sel[j] = 0ull;
-      selv[j] = 0.f;
       if (j < k) {  // k is the same on every lane: the shuffles stay converged
         uint64_t best = top[KMAX - 1];
-        float bv = val[KMAX - 1];
 #pragma unroll
         for (int off = G / 2; off >= 1; off >>= 1) {
           const uint32_t olo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(best), off);
           const uint32_t ohi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(best >> 32), off);
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
           const uint64_t o = (static_cast<uint64_t>(ohi) << 32) | olo;
-          if (o > best) {
-            best = o;
-            bv = ov;
-          }
+          if (o > best) best = o;
         }
         sel[j] = best;
-        selv[j] = bv;
         if (best != 0ull && top[KMAX - 1] == best) {  // this lane held it: pop the head
 #pragma unroll
-          for (int i = KMAX - 1; i > 0; --i) {
-            top[i] = top[i - 1];
-            val[i] = val[i - 1];
-          }
+          for (int i = KMAX - 1; i > 0; --i) top[i] = top[i - 1];
           top[0] = 0ull;
-          val[0] = 0.f;
         }
       }
     }
   }
+  // the selected logits, from their keys
+  float selv[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    selv[j] = float_from_order_key(static_cast<uint32_t>(sel[j] >> 32));
   // softmax: m = the largest logit (the first selected one)
   const float m = selv[0];
   float denom = 0.f;
