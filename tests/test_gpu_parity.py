@@ -258,7 +258,10 @@ def test_gemm_variants(cfg, gemm_variant):
 
 
 @pytest.mark.parametrize("T,E,k,R", [(1, 8, 2, 4), (2, 64, 6, 8), (257, 8, 2, 1),
-                                     (300, 8, 2, 8), (100, 256, 16, 8), (513, 64, 8, 64)])
+                                     (300, 8, 2, 8), (100, 256, 16, 8), (513, 64, 8, 64),
+                                     # several histogram chunks with E > 128 (4-tile chunks), and
+                                     # an E that is no power of two
+                                     (2000, 256, 16, 8), (1500, 160, 6, 8)])
 def test_edge_shapes(T, E, k, R):
     cfg = inputs.LayerConfig("edge", T=T, d=128, f=128, E=E, k=k, R=R, seed=T)
     run_and_check_small(cfg)
