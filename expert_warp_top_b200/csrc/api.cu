@@ -224,7 +224,7 @@ int launch_brim_passes(const int32_t* topk_idx, const float* topk_w, int T, int 
                                                           scratch, err));
   MOE_LAUNCHED("brim_mask_kernel");
   // the column scan writes the tiles' bases over the masks
-  MOE_CUDA(launch_k(moe::brim_colscan_kernel, ncol, 1024, 0, stream,
+  MOE_CUDA(launch_k(moe::brim_colscan_kernel, ncol, moe::kColscanThreads, 0, stream,
                     static_cast<const uint32_t*>(scratch), scratch, n_tiles, ncol, totals, T, R,
                     static_cast<int32_t*>(nullptr)));
   MOE_LAUNCHED("brim_colscan_kernel");
@@ -605,9 +605,9 @@ int moe_route_brim(const float* logits, int T, int E, int k, int renorm, const i
   } while (0)
 #define MOE_ROUTE_BRIM(KM)                                                                    \
   MOE_ROUTE_TILE_G(KM);                                                                       \
-  MOE_CUDA(launch_k(moe::brim_colscan_kernel, dim3(ncol), dim3(1024), 0, stream,              \
-                    static_cast<const uint32_t*>(masks), bases, n_tiles, ncol, totals, T, R,    \
-                    per_rank ? own : static_cast<int32_t*>(nullptr)));                          \
+  MOE_CUDA(launch_k(moe::brim_colscan_kernel, dim3(ncol), dim3(moe::kColscanThreads), 0,      \
+                    stream, static_cast<const uint32_t*>(masks), bases, n_tiles, ncol, totals,  \
+                    T, R, per_rank ? own : static_cast<int32_t*>(nullptr)));                    \
   MOE_CUDA(launch_k(moe::brim_scatter_kernel<KM>, dim3(extras.n_hist + n_tiles),              \
                     dim3(32 * moe::kScatterWarps), 0, stream, static_cast<const int32_t*>(topk_idx), \
                     static_cast<const float*>(topk_w), slot_of, T, k, E, R, n_tiles,            \
