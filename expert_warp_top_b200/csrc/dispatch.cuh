@@ -20,7 +20,7 @@
 
 namespace moe {
 
-constexpr int kMoverWarps = 8;     // warps per block
+constexpr int kMoverWarps = 4;     // warps per block
 constexpr int kMaxDst = 16;        // >= k (and >= min(k, R))
 
 // Destination buffers of the other ranks, for the movers that write their rows
