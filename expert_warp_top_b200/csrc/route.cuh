@@ -75,7 +75,35 @@ __device__ __forceinline__ void route_token_group(const float* __restrict__ row,
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) top[j] = 0ull;
   const bool vec = (E & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 15) == 0;
-  if (valid) {
+  // With KMAX = 8 and E = 8 G, a lane holds exactly eight logits: it sorts their
+  // ranks with a 19-comparator network (Batcher's odd-even merge sort) instead
+  // of eight insertions.  The list comes out the same, as the ranks are unique.
+  bool sorted8 = false;
+  if constexpr (KMAX == 8) {
+    if (valid && vec && (E >> 2) == 2 * G) {
+      const float4* r4 = reinterpret_cast<const float4*>(row);
+      const float4 x0 = __ldg(r4 + sub), x1 = __ldg(r4 + sub + G);
+      const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = 4 * (i < 4 ? sub : sub + G) + (i & 3);
+        top[i] = (static_cast<uint64_t>(float_order_key(xs[i])) << 32) |
+                 static_cast<uint32_t>(~e);
+      }
+      constexpr int kNet[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6},
+                                   {5, 7}, {1, 2}, {5, 6}, {0, 4}, {1, 5}, {2, 6}, {3, 7},
+                                   {2, 4}, {3, 5}, {1, 2}, {3, 4}, {5, 6}};
+#pragma unroll
+      for (int c = 0; c < 19; ++c) {
+        const uint64_t lo = top[kNet[c][0]], hi = top[kNet[c][1]];
+        const bool sw = lo > hi;
+        top[kNet[c][0]] = sw ? hi : lo;
+        top[kNet[c][1]] = sw ? lo : hi;
+      }
+      sorted8 = true;
+    }
+  }
+  if (valid && !sorted8) {
     if (vec) {
       const float4* r4 = reinterpret_cast<const float4*>(row);
       for (int q = sub; q < (E >> 2); q += G) {
